@@ -1,0 +1,266 @@
+"""fp64 CPU oracle for the routed mixture-of-experts expert FFN.
+
+TEST INFRASTRUCTURE ONLY. Nothing on the product path may import, call or run
+this package: only ``tests/``, ``__graft_entry__.smoke()`` and the CPU-baseline
+leg of ``bench.py`` use it. It shares no code with the CUDA library; both take
+their inputs from the ``synth`` generator alone.
+
+It is the plain definition of what the path computes, in float64, with no
+blocking, fusion or reordering beyond what the definition states. Sources:
+
+* "mini-AGI PR #3" (gt50/mini-AGI, files diff), ``minagi/pool.py``, the
+  ``requested(scores)`` router hunk: full softmax ``probs`` of the router
+  logits, the top-k ``idx``/``w``, ``w`` renormalised after the telemetry has
+  read its pre-normalisation mass; then the flatten / ``argsort`` by expert /
+  ``bincount`` hunk, and the capacity-drop hunk (``keep`` mask over the sorted
+  pairs, ``counts.clamp(max=limit)``).
+* the same pages' ``configs/strix_halo_large.yaml`` ``capacity_factor`` comment:
+  the most of a batch one expert may take, as a multiple of its fair share; the
+  rest is dropped; 0 removes the cap.
+* "mini-AGI PR #4" ``minagi/pool.py`` ``experts()``/``run()``: per expert,
+  ``silu(x W1) * (x W3)`` then ``W2``, gathered back in pair order.
+* "Strata PR #4366" (DS4_FAT_ROWS), "Approach": the SwiGLU is clamped.
+* "TensorFold PR #1607", "What this changes": served plans with "256 + shared"
+  experts (an always-on shared expert).
+
+Readings taken where the pages are silent (each one is listed in the design doc):
+top-k ties go to the lower expert index; the capacity is
+``ceil(cf * T * k / E)`` with cf widened from float32; overflow is dropped in
+token order and the kept weights are NOT renormalised; the clamp bounds both
+the gate and the up pre-activation to [-L, L]; the shared expert is un-gated
+(weight 1) and holds every token.
+
+Pins: every function here is checked in ``tests/test_oracle_pins.py`` against
+closed forms, brute force on tiny inputs, invariants and special cases.
+"""
+from __future__ import annotations
+
+import math
+
+import numpy as np
+
+__all__ = [
+    "route", "capacity", "permute", "silu", "swiglu_clamped", "expert_ffn",
+    "dequant_q4g32", "combine", "forward", "token_outputs",
+]
+
+
+# --------------------------------------------------------------------------- route
+
+def route(logits: np.ndarray, k: int):
+    """Top-k experts per token and their weights.
+
+    mini-AGI PR #3, ``requested()``: ``probs = softmax(logits)``, ``idx, w`` =
+    top-k of ``probs``, then ``w / w.sum(-1)``. Renormalising the top-k of a
+    full softmax equals a softmax over the k selected logits, which is what is
+    computed here (in float64).
+
+    The ranking compares the given float32 logits exactly; ties go to the lower
+    expert index (stable sort of the negated values). NaN logits are outside
+    the contract.
+
+    Returns idx int32 [T, k] (descending logit order) and w float64 [T, k].
+    """
+    lg = np.asarray(logits, dtype=np.float32)
+    T, E = lg.shape
+    if not 1 <= k <= E:
+        raise ValueError("need 1 <= k <= E")
+    order = np.argsort(-lg, axis=1, kind="stable")[:, :k]
+    sel = np.take_along_axis(lg, order, axis=1).astype(np.float64)
+    m = sel[:, :1]
+    ex = np.exp(sel - m)
+    w = ex / ex.sum(axis=1, keepdims=True)
+    return order.astype(np.int32), w
+
+
+# --------------------------------------------------------------------------- capacity
+
+def capacity(T: int, k: int, E: int, capacity_factor: float):
+    """Rows one expert may take, or None for no cap.
+
+    mini-AGI ``capacity_factor``: a multiple of an expert's fair share T*k/E;
+    0 removes the cap. The rounding up (ceil) is the stated workload's. The
+    factor is read as float32 (the boundary passes it so) and widened.
+    """
+    cf = float(np.float32(capacity_factor))
+    if cf <= 0.0:
+        return None
+    return int(math.ceil(cf * T * k / E))
+
+
+# --------------------------------------------------------------------------- permute
+
+def permute(idx: np.ndarray, E: int, cap=None, shared_T: int = 0):
+    """Group the (token, expert) pairs by expert, in token order, and drop overflow.
+
+    mini-AGI PR #3, ``requested()``: ``flat_e``/``tok`` flattened, ``order =
+    argsort(flat_e)``, ``counts = bincount(e_sorted)``; with a capacity,
+    ``keep`` = the pairs whose slot is below the limit, the rest counted as
+    dropped and filtered out, ``counts.clamp(max=limit)``.
+
+    Pair p = t*k + j. Within an expert, rows are in ascending p, which is
+    ascending token (a token's k experts are distinct). A pair of rank >= cap
+    in its expert is dropped: ``pair_row[p] = -1``.
+
+    With ``shared_T > 0`` an always-on shared expert is appended as expert
+    index E holding every token 0..T-1 in order (``sorted_pair = -1``).
+
+    Returns a dict of int32/int64 arrays: counts, kept, offsets, sorted_token,
+    sorted_pair, pair_row.
+    """
+    idx = np.asarray(idx)
+    T, k = idx.shape
+    flat_e = idx.reshape(-1).astype(np.int64)
+    counts = np.bincount(flat_e, minlength=E).astype(np.int64)
+    order = np.argsort(flat_e, kind="stable")  # pairs grouped by expert, ascending p
+    e_sorted = flat_e[order]
+    first = np.concatenate([[0], np.cumsum(counts)[:-1]])
+    rank = np.arange(order.size) - first[e_sorted]
+    keep = np.ones(order.size, bool) if cap is None else rank < cap
+    kept = counts if cap is None else np.minimum(counts, cap)
+    sorted_pair = order[keep]
+    sorted_token = sorted_pair // k
+    if shared_T:
+        counts = np.concatenate([counts, [shared_T]])
+        kept = np.concatenate([kept, [shared_T]])
+        sorted_token = np.concatenate([sorted_token, np.arange(shared_T)])
+        sorted_pair = np.concatenate([sorted_pair, np.full(shared_T, -1)])
+    offsets = np.concatenate([[0], np.cumsum(kept)])
+    pair_row = np.full(T * k, -1, np.int64)
+    n_routed = int(keep.sum())
+    pair_row[sorted_pair[:n_routed]] = np.arange(n_routed)
+    return {
+        "counts": counts.astype(np.int32), "kept": kept.astype(np.int32),
+        "offsets": offsets.astype(np.int32), "sorted_token": sorted_token.astype(np.int32),
+        "sorted_pair": sorted_pair.astype(np.int32), "pair_row": pair_row.astype(np.int32),
+    }
+
+
+# --------------------------------------------------------------------------- FFN
+
+def silu(z):
+    """silu(z) = z * sigmoid(z) = z / (1 + exp(-z)), float64."""
+    z = np.asarray(z, dtype=np.float64)
+    return z / (1.0 + np.exp(-z))
+
+
+def swiglu_clamped(g, u, limit: float):
+    """Clamped SwiGLU: silu(clamp(g, -L, L)) * clamp(u, -L, L).
+
+    Strata PR #4366, "Approach": the fat-rows route applies a clamped SwiGLU.
+    The bound L (7.0 for the stated workloads) applies to both the gate and
+    the up pre-activation. ``limit <= 0`` means no clamp.
+    """
+    g = np.asarray(g, dtype=np.float64)
+    u = np.asarray(u, dtype=np.float64)
+    if limit > 0:
+        g = np.clip(g, -limit, limit)
+        u = np.clip(u, -limit, limit)
+    return silu(g) * u
+
+
+def expert_ffn(x_rows, w_gate, w_up, w_down, limit: float):
+    """One expert on its rows: y = swiglu(x Wg, x Wu) Wd, all float64.
+
+    mini-AGI PR #4, ``experts()``: ``h = silu(x W1) * (x W3)``, ``y = h W2``
+    (W_gate, W_up are [d, f]; W_down is [f, d]). No intermediate rounding.
+    """
+    x_rows = np.asarray(x_rows, dtype=np.float64)
+    g = x_rows @ np.asarray(w_gate, dtype=np.float64)
+    u = x_rows @ np.asarray(w_up, dtype=np.float64)
+    h = swiglu_clamped(g, u, limit)
+    return h @ np.asarray(w_down, dtype=np.float64)
+
+
+def dequant_q4g32(packed: np.ndarray, scales: np.ndarray) -> np.ndarray:
+    """Q4G32 (self-defined) → float64 [K, N]: w[k, n] = q * s exactly.
+
+    packed uint8 [N, K/2]: byte j of row n holds k=2j (low nibble) and k=2j+1
+    (high nibble), each nibble u = q + 8. scales fp16 [N, K/32]: one scale per
+    group of 32 consecutive k.
+    """
+    packed = np.asarray(packed, dtype=np.uint8)
+    N, K2 = packed.shape
+    K = 2 * K2
+    q = np.empty((N, K), np.float64)
+    q[:, 0::2] = (packed & 0x0F).astype(np.float64) - 8.0
+    q[:, 1::2] = (packed >> 4).astype(np.float64) - 8.0
+    s = np.repeat(np.asarray(scales, dtype=np.float16).astype(np.float64), 32, axis=1)
+    return (q * s).T.copy()
+
+
+# --------------------------------------------------------------------------- combine
+
+def combine(y_rows, pair_row, w, T: int, k: int, shared_rows=None, shared_base: int = 0):
+    """Gate-weighted sum back to token order.
+
+    mini-AGI PR #4, ``run()``: expert outputs are read back in pair order
+    (``y[e_sorted, slot]``) and each token's k outputs are weighted by ``w`` and
+    summed. A dropped pair (``pair_row = -1``) adds nothing; the remaining
+    weights are not renormalised. With a shared expert its row
+    ``shared_base + t`` is added with weight 1.
+    """
+    d = y_rows.shape[1]
+    out = np.zeros((T, d), np.float64)
+    pr = np.asarray(pair_row).reshape(T, k)
+    w = np.asarray(w, dtype=np.float64).reshape(T, k)
+    for j in range(k):
+        r = pr[:, j]
+        ok = r >= 0
+        out[ok] += w[ok, j:j + 1] * y_rows[r[ok]]
+    if shared_rows:
+        out += y_rows[shared_base:shared_base + T]
+    return out
+
+
+# --------------------------------------------------------------------------- forward
+
+def forward(x, logits, k: int, experts, limit: float, capacity_factor: float = 0.0,
+            shared=None):
+    """The whole layer: route → permute → per-expert FFN → combine, float64.
+
+    x: [T, d] (any float dtype; widened exactly). logits: [T, E] float32.
+    experts: callable e -> (W_gate [d,f], W_up [d,f], W_down [f,d]).
+    shared: None or (W_gate, W_up, W_down) of the always-on shared expert.
+    Returns (out [T, d] float64, dict of intermediates).
+    """
+    x = np.asarray(x, dtype=np.float64)
+    T = x.shape[0]
+    E = np.asarray(logits).shape[1]
+    idx, w = route(logits, k)
+    cap = capacity(T, k, E, capacity_factor)
+    perm = permute(idx, E, cap, shared_T=T if shared is not None else 0)
+    off, tok = perm["offsets"], perm["sorted_token"]
+    y = np.zeros((int(off[-1]), x.shape[1]), np.float64)
+    for e in range(E):
+        a, b = int(off[e]), int(off[e + 1])
+        if b > a:
+            y[a:b] = expert_ffn(x[tok[a:b]], *experts(e), limit)
+    if shared is not None:
+        a, b = int(off[E]), int(off[E + 1])
+        y[a:b] = expert_ffn(x[tok[a:b]], *shared, limit)
+    out = combine(y, perm["pair_row"], w, T, k,
+                  shared_rows=shared is not None, shared_base=int(off[E]))
+    return out, {"idx": idx, "w": w, "cap": cap, "y": y, **perm}
+
+
+def token_outputs(tokens, x, idx, w, pair_row, experts, limit: float, shared=None):
+    """Outputs of selected tokens, each from its own definition.
+
+    out[t] = sum over kept j of w[t, j] * FFN_{idx[t, j]}(x[t])  (+ shared(x[t])).
+    Used to check full-size runs on sampled tokens without running the layer.
+    """
+    x = np.asarray(x)
+    T, k = idx.shape
+    pr = np.asarray(pair_row).reshape(T, k)
+    res = []
+    for t in tokens:
+        xt = np.asarray(x[t:t + 1], dtype=np.float64)
+        acc = np.zeros((1, x.shape[1]), np.float64)
+        for j in range(k):
+            if pr[t, j] >= 0:
+                acc += float(w[t, j]) * expert_ffn(xt, *experts(int(idx[t, j])), limit)
+        if shared is not None:
+            acc += expert_ffn(xt, *shared, limit)
+        res.append(acc[0])
+    return np.stack(res) if res else np.zeros((0, x.shape[1]))

@@ -1,0 +1,331 @@
+"""Pins for the fp64 oracle: closed forms, brute force, invariants, golden cases.
+
+Each check ties the oracle to something other than its own code: hand-worked
+golden fixtures (tests/golden/, each citing its source), brute force over all
+k-subsets, pure-Python loop versions of the definitions, closed forms and
+symmetry properties. A plausible mistake (dropped term, wrong sign, transposed
+operand, wrong tie-break, renormalising after a drop) fails at least one.
+"""
+import itertools
+import math
+import os
+
+import numpy as np
+import pytest
+
+import oracle
+import synth
+
+GOLD = os.path.join(os.path.dirname(__file__), "golden")
+
+
+def _lines(name):
+    with open(os.path.join(GOLD, name)) as fh:
+        return [ln.strip() for ln in fh if ln.strip() and not ln.startswith("#")]
+
+
+# --------------------------------------------------------------------------- route
+
+def test_route_golden_cases():
+    for ln in _lines("route_cases.txt"):
+        k, lg, ix, w = [p.split() for p in ln.split("|")]
+        k = int(k[0])
+        logits = np.array([[float(v) for v in lg]], np.float32)
+        idx, ww = oracle.route(logits, k)
+        assert idx[0].tolist() == [int(v) for v in ix], ln
+        np.testing.assert_allclose(ww[0], [float(v) for v in w], rtol=0, atol=1e-12)
+
+
+def test_route_brute_force_topk():
+    """Over all k-subsets, the top-k set is the one with the largest logit sum."""
+    rng = np.random.default_rng(11)
+    for E in (2, 3, 5, 8):
+        for k in range(1, E + 1):
+            lg = rng.standard_normal((20, E)).astype(np.float32)
+            idx, w = oracle.route(lg, k)
+            for t in range(lg.shape[0]):
+                best = max(itertools.combinations(range(E), k),
+                           key=lambda s: sum(float(lg[t, e]) for e in s))
+                want = sorted(best, key=lambda e: -float(lg[t, e]))
+                assert idx[t].tolist() == want
+                # softmax over the selected, by its definition with Python floats
+                ex = [math.exp(float(lg[t, e]) - float(lg[t, want[0]])) for e in want]
+                np.testing.assert_allclose(w[t], [v / sum(ex) for v in ex], rtol=1e-13)
+
+
+def test_route_equals_renormalised_full_softmax():
+    """The pages' procedure: full softmax, take top-k, divide by their sum."""
+    from scipy.special import softmax
+    lg = np.random.default_rng(5).standard_normal((50, 16)).astype(np.float32) * 3
+    idx, w = oracle.route(lg, 4)
+    probs = softmax(lg.astype(np.float64), axis=1)
+    sel = np.take_along_axis(probs, idx.astype(np.int64), axis=1)
+    np.testing.assert_allclose(w, sel / sel.sum(1, keepdims=True), rtol=1e-12)
+    # shift invariance of the weights, and they sum to one
+    idx2, w2 = oracle.route(lg + np.float32(0.0), 4)
+    np.testing.assert_allclose(w.sum(1), 1.0, rtol=1e-14)
+    assert (idx2 == idx).all()
+
+
+def test_route_k1_and_k2_closed_forms():
+    lg = np.random.default_rng(3).standard_normal((30, 6)).astype(np.float32)
+    _, w1 = oracle.route(lg, 1)
+    assert (w1 == 1.0).all()
+    idx, w2 = oracle.route(lg, 2)
+    a = lg[np.arange(30), idx[:, 0]].astype(np.float64)
+    b = lg[np.arange(30), idx[:, 1]].astype(np.float64)
+    np.testing.assert_allclose(w2[:, 0], 1.0 / (1.0 + np.exp(b - a)), rtol=1e-14)
+    assert (a >= b).all()
+
+
+# --------------------------------------------------------------------------- capacity
+
+def test_capacity_golden():
+    for ln in _lines("capacity_cases.txt"):
+        T, k, E, cf, want = ln.split()
+        got = oracle.capacity(int(T), int(k), int(E), float(cf))
+        assert got == (None if want == "none" else int(want)), ln
+
+
+# --------------------------------------------------------------------------- permute
+
+def _permute_loop(idx, E, cap):
+    """Plain per-expert loop: walk the tokens in order, each expert takes rows until full."""
+    T, k = idx.shape
+    rows = {e: [] for e in range(E)}
+    counts = [0] * E
+    for t in range(T):
+        for j in range(k):
+            e = int(idx[t, j])
+            counts[e] += 1
+            if cap is None or len(rows[e]) < cap:
+                rows[e].append((t, t * k + j))
+    pair_row = [-1] * (T * k)
+    sorted_token, offsets = [], [0]
+    for e in range(E):
+        for (t, p) in rows[e]:
+            pair_row[p] = len(sorted_token)
+            sorted_token.append(t)
+        offsets.append(len(sorted_token))
+    return counts, offsets, sorted_token, pair_row
+
+
+def test_permute_golden_drop_order():
+    g = {}
+    for ln in _lines("drop_order.txt"):
+        key, *vals = ln.split()
+        g[key] = [int(v) for v in vals]
+    idx = np.array(g["idx"], np.int32)[:, None]
+    p = oracle.permute(idx, g["E"][0], g["cap"][0])
+    for key in ("counts", "kept", "offsets", "sorted_token", "pair_row"):
+        assert p[key].tolist() == g[key], key
+
+
+@pytest.mark.parametrize("cap", [None, 1, 3, 7])
+def test_permute_matches_loop(cap):
+    rng = np.random.default_rng(7)
+    for E, k, T in ((4, 2, 9), (8, 3, 40), (5, 5, 12), (16, 1, 50)):
+        lg = rng.standard_normal((T, E)).astype(np.float32)
+        idx, _ = oracle.route(lg, k)
+        p = oracle.permute(idx, E, cap)
+        counts, offsets, st, pr = _permute_loop(idx, E, cap)
+        assert p["counts"].tolist() == counts
+        assert p["offsets"].tolist() == offsets
+        assert p["sorted_token"].tolist() == st
+        assert p["pair_row"].tolist() == pr
+
+
+def test_permute_invariants_capped_workload():
+    cfg = synth.CONFIGS["capped"]
+    idx, _ = oracle.route(synth.logits(cfg), cfg.k)
+    cap = oracle.capacity(cfg.T, cfg.k, cfg.E, cfg.capacity_factor)
+    assert cap == 192
+    p = oracle.permute(idx, cfg.E, cap)
+    assert p["counts"].sum() == cfg.T * cfg.k
+    assert (p["kept"] <= cap).all()
+    P = int(p["offsets"][-1])
+    assert p["kept"].sum() == P and (np.diff(p["offsets"]) >= 0).all()
+    dropped = cfg.T * cfg.k - P
+    assert dropped > 0.5 * cfg.T * cfg.k  # the +4 bias crowds 8 experts: most pairs drop
+    # every kept pair once, pair_row the inverse of sorted_pair
+    sp = p["sorted_pair"]
+    assert len(set(sp.tolist())) == P
+    assert (p["pair_row"][sp] == np.arange(P)).all()
+    assert ((p["pair_row"] >= 0).sum()) == P
+    # tokens ascend inside each expert
+    st = p["sorted_token"]
+    for e in range(cfg.E):
+        seg = st[p["offsets"][e]:p["offsets"][e + 1]]
+        assert (np.diff(seg) > 0).all()
+
+
+def test_permute_shared_expert_rows():
+    idx = np.array([[0, 1], [1, 2], [0, 2]], np.int32)
+    p = oracle.permute(idx, 3, None, shared_T=3)
+    assert p["offsets"].tolist() == [0, 2, 4, 6, 9]
+    assert p["sorted_token"][6:].tolist() == [0, 1, 2]
+    assert p["sorted_pair"][6:].tolist() == [-1, -1, -1]
+    assert p["kept"].tolist() == [2, 2, 2, 3]
+
+
+# --------------------------------------------------------------------------- FFN
+
+def test_swiglu_golden_points():
+    for ln in _lines("swiglu_points.txt"):
+        g, u, L, want = (float(v) for v in ln.split())
+        got = float(oracle.swiglu_clamped(np.array([g]), np.array([u]), L)[0])
+        assert got == pytest.approx(want, rel=1e-14, abs=1e-15), ln
+
+
+def _ffn_loops(x, wg, wu, wd, L):
+    """SwiGLU FFN with explicit Python loops (no matrix library)."""
+    d, f = len(wg), len(wg[0])
+    out = []
+    for row in x:
+        h = []
+        for n in range(f):
+            g = sum(row[i] * wg[i][n] for i in range(d))
+            u = sum(row[i] * wu[i][n] for i in range(d))
+            if L > 0:
+                g, u = min(max(g, -L), L), min(max(u, -L), L)
+            h.append(g / (1.0 + math.exp(-g)) * u)
+        out.append([sum(h[n] * wd[n][i] for n in range(f)) for i in range(d)])
+    return np.array(out)
+
+
+@pytest.mark.parametrize("scale,L,d,f", [(1.0, 7.0, 5, 7), (20.0, 7.0, 5, 7), (20.0, 0.0, 5, 7),
+                                         (1.0, 7.0, 6, 6)])
+def test_expert_ffn_matches_loops(scale, L, d, f):
+    rng = np.random.default_rng(2)
+    # non-square and square shapes: a transposed operand fails either way
+    x = rng.standard_normal((4, d))
+    wg, wu = rng.standard_normal((d, f)) * scale, rng.standard_normal((d, f)) * scale
+    wd = rng.standard_normal((f, d))
+    got = oracle.expert_ffn(x, wg, wu, wd, L)
+    want = _ffn_loops(x.tolist(), wg.tolist(), wu.tolist(), wd.tolist(), L)
+    np.testing.assert_allclose(got, want, rtol=1e-12, atol=1e-12)
+    if scale == 20.0 and L > 0:
+        unclamped = _ffn_loops(x.tolist(), wg.tolist(), wu.tolist(), wd.tolist(), 0.0)
+        assert np.abs(unclamped - want).max() > 1.0  # the clamp fires in this case
+
+
+def test_e1_top1_is_dense_ffn():
+    """E=1, k=1: routing weight 1, every token kept → the layer is one dense FFN."""
+    cfg = synth.LayerConfig("e1", T=12, d=16, f=24, E=1, k=1)
+    x = synth.bf16_bits_to_f32(synth.x_bits(cfg)).astype(np.float64)
+    W = [synth.bf16_bits_to_f32(synth.expert_weight_bits(cfg, 0, w)) for w in ("gate", "up", "down")]
+    out, inter = oracle.forward(x, synth.logits(cfg), 1, lambda e: W, 7.0)
+    assert (inter["w"] == 1.0).all()
+    dense = _ffn_loops(x.tolist(), *(w.astype(np.float64).tolist() for w in W), 7.0)
+    np.testing.assert_allclose(out, dense, rtol=1e-12, atol=1e-14)
+
+
+# --------------------------------------------------------------------------- whole layer
+
+def _layer_loops(x, lg, k, Ws, L, cap, shared=None):
+    """The layer straight from its definition: per token, sum of weighted expert
+    outputs, with the capacity drop decided by a running per-expert count."""
+    T, E = lg.shape
+    taken = [0] * E
+    out = np.zeros_like(x)
+    for t in range(T):
+        order = sorted(range(E), key=lambda e: (-float(lg[t, e]), e))[:k]
+        ex = [math.exp(float(lg[t, e]) - float(lg[t, order[0]])) for e in order]
+        for e, v in zip(order, ex):
+            taken[e] += 1
+            if cap is not None and taken[e] > cap:
+                continue  # dropped: contributes nothing, the others are not renormalised
+            y = _ffn_loops([x[t].tolist()], *(w.tolist() for w in Ws[e]), L)[0]
+            out[t] += v / sum(ex) * y
+        if shared is not None:
+            out[t] += _ffn_loops([x[t].tolist()], *(w.tolist() for w in shared), L)[0]
+    return out
+
+
+@pytest.mark.parametrize("cf,shared", [(0.0, False), (1.0, False), (0.5, True)])
+def test_forward_matches_per_token_loops(cf, shared):
+    rng = np.random.default_rng(9)
+    T, d, f, E, k = 9, 4, 6, 3, 2
+    x = rng.standard_normal((T, d))
+    lg = rng.standard_normal((T, E)).astype(np.float32)
+    Ws = [tuple(rng.standard_normal(s) * 0.7 for s in ((d, f), (d, f), (f, d))) for _ in range(E)]
+    sh = tuple(rng.standard_normal(s) * 0.7 for s in ((d, f), (d, f), (f, d))) if shared else None
+    out, inter = oracle.forward(x, lg, k, lambda e: Ws[e], 7.0, cf, shared=sh)
+    cap = oracle.capacity(T, k, E, cf)
+    want = _layer_loops(x, lg, k, Ws, 7.0, cap, sh)
+    np.testing.assert_allclose(out, want, rtol=1e-12, atol=1e-12)
+    if cf > 0:
+        assert (inter["pair_row"] < 0).any()
+
+
+def test_token_permutation_equivariance():
+    cfg = synth.CONFIGS["tiny"]
+    x = synth.bf16_bits_to_f32(synth.x_bits(cfg)).astype(np.float64)
+    lg = synth.logits(cfg)
+    Ws = {e: [synth.bf16_bits_to_f32(synth.expert_weight_bits(cfg, e, w)) for w in ("gate", "up", "down")]
+          for e in range(cfg.E)}
+    out, _ = oracle.forward(x, lg, cfg.k, Ws.__getitem__, 7.0)
+    perm = np.random.default_rng(4).permutation(cfg.T)
+    out_p, _ = oracle.forward(x[perm], lg[perm], cfg.k, Ws.__getitem__, 7.0)
+    np.testing.assert_allclose(out_p, out[perm], rtol=1e-12, atol=1e-15)
+    # linear in W_down
+    Ws2 = {e: [w[0], w[1], 2 * w[2]] for e, w in Ws.items()}
+    out2, _ = oracle.forward(x, lg, cfg.k, Ws2.__getitem__, 7.0)
+    np.testing.assert_allclose(out2, 2 * out, rtol=1e-12, atol=1e-15)
+
+
+def test_all_dropped_token_is_zero_or_shared():
+    # every token picks expert 0 (bias), cap 1: only token 0 is served
+    T, E, k, d, f = 4, 2, 1, 3, 5
+    rng = np.random.default_rng(1)
+    lg = np.array([[5.0, 0.0]] * T, np.float32)
+    x = rng.standard_normal((T, d))
+    W = tuple(rng.standard_normal(s) for s in ((d, f), (d, f), (f, d)))
+    out, inter = oracle.forward(x, lg, k, lambda e: W, 7.0, capacity_factor=0.5)
+    assert inter["cap"] == 1
+    assert np.abs(out[1:]).max() == 0.0 and np.abs(out[0]).max() > 0
+    out_s, _ = oracle.forward(x, lg, k, lambda e: W, 7.0, capacity_factor=0.5, shared=W)
+    np.testing.assert_allclose(out_s[1:], oracle.expert_ffn(x[1:], *W, 7.0), rtol=1e-13)
+
+
+def test_token_outputs_match_forward():
+    cfg = synth.CONFIGS["tiny"].replace(capacity_factor=1.0)
+    x = synth.bf16_bits_to_f32(synth.x_bits(cfg)).astype(np.float64)
+    lg = synth.logits(cfg)
+    Ws = {e: [synth.bf16_bits_to_f32(synth.expert_weight_bits(cfg, e, w)) for w in ("gate", "up", "down")]
+          for e in range(cfg.E)}
+    out, it = oracle.forward(x, lg, cfg.k, Ws.__getitem__, 7.0, cfg.capacity_factor)
+    toks = [0, 5, 17, 63]
+    got = oracle.token_outputs(toks, x, it["idx"], it["w"], it["pair_row"], Ws.__getitem__, 7.0)
+    np.testing.assert_allclose(got, out[toks], rtol=1e-12, atol=1e-15)
+
+
+# --------------------------------------------------------------------------- Q4G32
+
+def test_q4g32_golden_bytes():
+    packed = np.full((2, 16), 0x88, np.uint8)
+    packed[0, 0], packed[0, 1], packed[1, 0] = 0x9F, 0x18, 0x2E
+    scales = np.array([[0.5], [0.25]], np.float16)
+    w = oracle.dequant_q4g32(packed, scales)  # [K=32, N=2]
+    want = np.zeros((32, 2))
+    for ln in _lines("q4g32_bytes.txt"):
+        n, k, v = ln.split()
+        want[int(k), int(n)] = float(v)
+    assert (w == want).all()
+
+
+def test_q4g32_round_trip_and_error_bound():
+    rng = np.random.default_rng(0)
+    # exactly representable: every group holds +-7 so the scale is exactly 0.25
+    q = rng.integers(-7, 8, size=(64, 6))
+    q[0::32, :] = 7
+    w = q * 0.25
+    packed, s = synth.quantize_q4g32(w.astype(np.float32))
+    assert (s == np.float16(0.25)).all()
+    assert (oracle.dequant_q4g32(packed, s) == w).all()
+    # general case: error at most half a step (plus the fp16 rounding of the scale)
+    w = rng.standard_normal((128, 40)).astype(np.float32) * 0.02
+    packed, s = synth.quantize_q4g32(w)
+    err = np.abs(oracle.dequant_q4g32(packed, s) - w)
+    step = np.repeat(s.astype(np.float64), 32, axis=1).T
+    assert (err <= step * (0.5 + 7 * 2.0 ** -10) + 1e-12).all()
