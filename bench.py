@@ -1,0 +1,414 @@
+#!/usr/bin/env python
+"""Benchmark of the routed MoE expert-FFN layer (moe_forward) on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--config prompt] [--impl own|reference]
+
+One step = one moe_forward over one batch: route → permute → expert FFN →
+combine, every kernel of the library, inputs resident in HBM. W warm-up steps,
+then K timed steps, each bracketed by CUDA events on the launching stream, with
+L2 flushed (a 256 MiB write) between steps outside the events. For N > 1 each
+rank (one per GPU, launched by torch.distributed.run) runs its own replica of
+the workload — the layer shards by tokens with no exchange — and the time is
+the max over ranks (NCCL all-reduce of the measured times only).
+
+One JSON line on rank 0: value = tokens/s of the whole job; plus TFLOP/s (or
+GB/s for the decode configs), the roofline of the dominant kernel measured live
+(per-kernel CUDA events inside the library, moe_profile_*), the end-to-end
+number through moe_forward_host (host buffers, copies inside the timed region),
+SM clocks sampled through NVML during the timed region, and the fp64 CPU
+oracle's throughput on this host as a baseline.
+
+--impl reference times that oracle alone (on the host cores, rank 0 only) on
+this arm's config, a bounded sample of the workload per step.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+
+import synth  # noqa: E402
+
+METRIC = "MoE layer tokens/sec and TFLOP/s (% BF16 tensor peak); decode GB/s (% HBM)"
+FLUSH_BYTES = 256 << 20
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--config", default="prompt", choices=sorted(synth.CONFIGS))
+    ap.add_argument("--impl", default="own", choices=["own", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    return ap.parse_args()
+
+
+# --------------------------------------------------------------------------- workload numbers
+
+def workload_numbers(cfg, P, touched):
+    """Algorithmic FLOPs and bytes of one layer call (no padding, no intermediates)."""
+    T, d, f = cfg.T, cfg.d, cfg.f
+    fl_gateup = 2.0 * P * 2 * d * f
+    fl_down = 2.0 * P * f * d
+    wbytes = 2.0 if cfg.weight_format == "bf16" else 0.5 + 2.0 / 32  # q4g32: nibble + fp16 scale / 32
+    n_exp = touched + (1 if cfg.has_shared else 0)
+    if cfg.has_shared:
+        fl_gateup += 2.0 * T * 2 * d * cfg.f_shared
+        fl_down += 2.0 * T * cfg.f_shared * d
+    w_gateup = n_exp * 2 * d * f * wbytes
+    w_down = n_exp * f * d * wbytes
+    io = T * d * 2 + T * d * 4 + T * cfg.E * 4  # x bf16 in, out fp32, logits
+    return {"flops": fl_gateup + fl_down, "flops_gateup": fl_gateup, "flops_down": fl_down,
+            "bytes": w_gateup + w_down + io, "bytes_gateup": w_gateup + T * d * 2,
+            "bytes_down": w_down + T * d * 2}
+
+
+def workload_name(cfg):
+    s = f"{cfg.name}: T={cfg.T} d_model={cfg.d} d_ff={cfg.f} E={cfg.E} top-{cfg.k}"
+    if cfg.capacity_factor:
+        s += f" cf={cfg.capacity_factor}"
+    if cfg.has_shared:
+        s += f" +shared(d_ff={cfg.f_shared})"
+    if cfg.bias != "none":
+        s += f" bias={cfg.bias}"
+    return s + f" weights={cfg.weight_format}"
+
+
+def peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as fh:
+            return json.load(fh), "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+def kernel_source_hash(files):
+    h = hashlib.sha256()
+    for fn in files:
+        with open(os.path.join(ROOT, "mixture_experts_routed_04_b200", "csrc", fn), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def committed_traffic(kernel, files, cfg_name):
+    """dram bytes per launch from a committed ncu summary, if it matches the current source."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(path):
+        return None
+    with open(path) as fh:
+        tab = json.load(fh)
+    ent = tab.get(kernel, {}).get(cfg_name)
+    if not ent or ent.get("source_hash") != kernel_source_hash(files):
+        return None
+    return ent.get("dram_bytes_per_launch")
+
+
+# --------------------------------------------------------------------------- clocks
+
+class ClockSampler:
+    """Polls SM clock and throttle reasons through NVML in a thread (read only)."""
+
+    REASONS = {"hw_slowdown": 0x8, "sw_thermal_slowdown": 0x20, "hw_thermal_slowdown": 0x40,
+               "sw_power_cap": 0x4, "hw_power_brake_slowdown": 0x80}
+
+    def __init__(self, index):
+        self.samples, self.reasons, self.max_mhz = [], set(), None
+        self._stop = threading.Event()
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self._nv = pynvml
+            self._h = pynvml.nvmlDeviceGetHandleByIndex(index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self._h, pynvml.NVML_CLOCK_SM)
+        except Exception:  # NVML missing: report no samples
+            self._nv = None
+
+    def _run(self):
+        nv = self._nv
+        while not self._stop.is_set():
+            try:
+                self.samples.append(nv.nvmlDeviceGetClockInfo(self._h, nv.NVML_CLOCK_SM))
+                r = nv.nvmlDeviceGetCurrentClocksEventReasons(self._h)
+                for name, bit in self.REASONS.items():
+                    if r & bit:
+                        self.reasons.add(name)
+            except Exception:
+                pass
+            time.sleep(0.001)
+
+    def __enter__(self):
+        if self._nv:
+            self._t = threading.Thread(target=self._run, daemon=True)
+            self._t.start()
+        return self
+
+    def __exit__(self, *exc):
+        self._stop.set()
+        if self._nv:
+            self._t.join()
+
+    def summary(self):
+        return {"sm_mhz": statistics.median(self.samples) if self.samples else None,
+                "sm_max_mhz": self.max_mhz, "reasons": sorted(self.reasons), "samples": len(self.samples)}
+
+
+# --------------------------------------------------------------------------- CPU oracle
+
+def cpu_oracle_runner(cfg):
+    """Prepare the oracle's inputs (fp64 weights of every expert) once; return run(tokens)->seconds."""
+    import oracle
+    from synth.device import expert_f64, shared_f64
+    x = synth.bf16_bits_to_f32(synth.x_bits(cfg)).astype(np.float64)
+    lg = synth.logits(cfg)
+    if cfg.weight_format == "q4g32":
+        def load(e):
+            return tuple(oracle.dequant_q4g32(*synth.expert_q4_weights(cfg, e, w)) for w in ("gate", "up", "down"))
+    else:
+        def load(e):
+            return expert_f64(cfg, e)
+    from concurrent.futures import ThreadPoolExecutor
+    with ThreadPoolExecutor(8) as ex:
+        Ws = dict(zip(range(cfg.E), ex.map(load, range(cfg.E))))
+    sh = shared_f64(cfg) if cfg.has_shared else None
+
+    def run(tokens):
+        xs, ls = x[tokens], lg[tokens]
+        t0 = time.perf_counter()
+        oracle.forward(xs, ls, cfg.k, Ws.__getitem__, cfg.swiglu_limit, cfg.capacity_factor, shared=sh)
+        return time.perf_counter() - t0
+
+    return run
+
+
+def blas_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        n = [i["num_threads"] for i in threadpool_info() if i.get("user_api") == "blas"]
+        return max(n) if n else 1
+    except Exception:
+        return os.cpu_count() or 1
+
+
+def cpu_baseline(cfg, budget_s=15.0):
+    """The oracle timed on the host cores on whole-layer calls of the workload, until ~budget_s."""
+    run = cpu_oracle_runner(cfg)
+    toks = np.arange(cfg.T)
+    run(toks[: min(cfg.T, 64)])  # warm BLAS
+    times = []
+    t_end = time.perf_counter() + budget_s
+    while not times or (time.perf_counter() < t_end and len(times) < 50):
+        times.append(run(toks))
+    tps = cfg.T * len(times) / sum(times)
+    return {"value": tps, "unit": "tokens/s", "cores": blas_threads(), "kind": "oracle",
+            "sample": f"{len(times)} whole-layer call(s) of the {cfg.name} workload (T={cfg.T}), fp64 NumPy, "
+                      f"weights pre-converted to fp64 outside the timing"}
+
+
+# --------------------------------------------------------------------------- reference arm
+
+def reference_arm(args, cfg):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    run = cpu_oracle_runner(cfg)
+    est = run(np.arange(min(cfg.T, 256)))  # seconds for 256 tokens
+    per_tok = est / min(cfg.T, 256)
+    budget = 120.0  # seconds of timed CPU work in total
+    n = int(max(1, min(cfg.T, budget / max(args.steps, 1) / max(per_tok, 1e-9))))
+    rng = np.random.default_rng(0)
+    for _ in range(args.warmup):
+        run(np.sort(rng.choice(cfg.T, n, replace=False)))
+    times = [run(np.sort(rng.choice(cfg.T, n, replace=False))) for _ in range(args.steps)]
+    sec = sum(times)
+    tps = n * args.steps / sec
+    line = {"metric": METRIC, "value": tps, "unit": "tokens/s", "n_gpus": args.gpus, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": 1e3 * sec / args.steps, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "impl": "reference",
+            "config": {"workload": workload_name(cfg), "tokens_per_step": n, "l2": "n/a (CPU)"},
+            "cpu_baseline": {"value": tps, "unit": "tokens/s", "cores": blas_threads(), "kind": "oracle",
+                             "sample": f"{n} random tokens of the {cfg.name} workload per step (all experts' "
+                                       f"weights resident as fp64)"},
+            "e2e": {"value": tps, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# --------------------------------------------------------------------------- own arm
+
+def own_arm(args, cfg):
+    import torch
+    from mixture_experts_routed_04_b200 import binding as b
+    from synth.device import upload
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dist = None
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+
+    d = upload(cfg, "cuda")
+    p = b.params_for(cfg)
+    sh = (d["shared_gate"], d["shared_up"], d["shared_down"]) if cfg.has_shared else None
+    W = b.weights(d["w_gate"], d["w_up"], d["w_down"], d.get("s_gate"), d.get("s_up"), d.get("s_down"), shared=sh)
+    ws = b.workspace(p, b.WS_FORWARD)
+    out = torch.empty(cfg.T, cfg.d, dtype=torch.float32, device="cuda")
+    flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device="cuda")
+    stream = torch.cuda.current_stream()
+
+    def step():
+        b.forward(p, d["x"], d["logits"], W, out, ws)
+
+    # routed rows P and touched experts, from the layer's own per-expert counts
+    counts = torch.empty(cfg.E + int(cfg.has_shared), dtype=torch.int32, device="cuda")
+    b.forward(p, d["x"], d["logits"], W, out, ws, counts_out=counts)
+    cap = b.capacity(p)
+    kept = counts[: cfg.E].cpu().numpy()
+    kept = np.minimum(kept, cap) if cap is not None else kept
+    P, touched = int(kept.sum()), int((kept > 0).sum())
+    wl = workload_numbers(cfg, P, touched)
+
+    for _ in range(max(args.warmup, 3)):
+        flush.zero_()
+        step()
+    torch.cuda.synchronize()
+    if b.get_error(ws):
+        raise RuntimeError("device error word set during warm-up")
+
+    K = args.steps
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
+    ends = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
+    if dist:
+        dist.barrier()
+    torch.cuda.synchronize()
+    with ClockSampler(local) as clocks:
+        for i in range(K):
+            flush.zero_()
+            starts[i].record(stream)
+            step()
+            ends[i].record(stream)
+        torch.cuda.synchronize()
+    if dist:
+        dist.barrier()
+    total_ms = sum(s.elapsed_time(e) for s, e in zip(starts, ends))
+    if dist:
+        t = torch.tensor([total_ms], dtype=torch.float64, device="cuda")
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        total_ms = float(t.item())
+    if b.get_error(ws):
+        raise RuntimeError("device error word set during the timed steps")
+    ms = total_ms / K
+
+    # per-kernel times, CUDA events inside the library around each launch (same steps, same flushes)
+    b.profile_collect()
+    b.profile_enable(True)
+    for i in range(K):
+        flush.zero_()
+        step()
+    torch.cuda.synchronize()
+    prof = b.profile_collect()
+    b.profile_enable(False)
+
+    # end to end through moe_forward_host: pinned host x/logits in, out back, per step
+    e2e = None
+    if not args.no_e2e:
+        pe = b.workspace(p, b.WS_FORWARD_HOST)
+        x_h = d["x"].cpu().pin_memory()
+        l_h = d["logits"].cpu().pin_memory()
+        o_h = torch.empty(cfg.T, cfg.d, dtype=torch.float32).pin_memory()
+        for _ in range(3):
+            b.forward_host(p, x_h, l_h, W, o_h, pe)
+        ek = max(3, min(K, 50))
+        e_ms = 0.0
+        for _ in range(ek):
+            flush.zero_()
+            s0, s1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            s0.record(stream)
+            b.forward_host(p, x_h, l_h, W, o_h, pe)
+            s1.record(stream)
+            s1.synchronize()
+            e_ms += s0.elapsed_time(s1)
+        if dist:
+            t = torch.tensor([e_ms], dtype=torch.float64, device="cuda")
+            dist.all_reduce(t, op=dist.ReduceOp.MAX)
+            e_ms = float(t.item())
+        e2e = {"value": cfg.T * world / (e_ms / ek / 1e3), "unit": "tokens/s",
+               "h2d_bytes_per_step": cfg.T * cfg.d * 2 + cfg.T * cfg.E * 4, "d2h_bytes_per_step": cfg.T * cfg.d * 4,
+               "ms_per_step": e_ms / ek}
+
+    pk, pk_src = peaks()
+    tensor_bound = cfg.name not in ("decode1", "decode8", "decode32")
+    kern = "tc_gateup" if tensor_bound else "stream_gateup"
+    kms, kn = prof.get(kern, (0.0, 0))
+    k_avg = kms / kn if kn else float("nan")
+    if tensor_bound:
+        achieved = wl["flops_gateup"] / (k_avg / 1e3) / 1e12
+        peak = pk["bf16_tflops"]
+        roof = {"kernel": "grouped_gemm_kernel<0> (tcgen05 gate/up + SwiGLU)", "bound": "tensor",
+                "achieved": achieved, "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak,
+                "peak_source": f"{pk_src} bf16_tflops (burst)", "avg_launch_ms": k_avg,
+                "algorithmic_per_launch": wl["flops_gateup"],
+                "traffic": committed_traffic("tc_gateup", ["gemm_tc.cu", "common.cuh"], cfg.name)}
+    else:
+        achieved = wl["bytes_gateup"] / (k_avg / 1e3) / 1e9
+        peak = pk["hbm_gbs"]
+        roof = {"kernel": "stream_kernel<0> (few-rows gate/up)", "bound": "hbm", "achieved": achieved,
+                "peak": peak, "unit": "GB/s", "frac": achieved / peak, "peak_source": f"{pk_src} hbm_gbs",
+                "avg_launch_ms": k_avg, "algorithmic_per_launch": wl["bytes_gateup"],
+                "traffic": committed_traffic("stream_gateup", ["stream.cu", "common.cuh"], cfg.name)}
+
+    line = None
+    if rank == 0:
+        tflops = wl["flops"] / (ms / 1e3) / 1e12
+        gbs = wl["bytes"] / (ms / 1e3) / 1e9
+        line = {"metric": METRIC, "value": cfg.T * world / (ms / 1e3), "unit": "tokens/s", "n_gpus": world,
+                "steps": K, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
+                "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+                "config": {"workload": workload_name(cfg), "tokens_per_gpu": cfg.T, "routed_rows": P,
+                           "touched_experts": touched, "parallelism": f"replicas x{world} (no exchange)",
+                           "l2": "flushed between steps (256 MiB write), inputs also larger than L2"},
+                "tflops": tflops, "tensor_frac_of_peak": tflops / pk["bf16_tflops"],
+                "gbs": gbs, "hbm_frac_of_peak": gbs / pk["hbm_gbs"], "peaks": pk_src,
+                "roofline": roof,
+                "kernels_ms_per_step": {k: v[0] / K for k, v in prof.items() if v[1]},
+                "gpu_launches": b.launch_count(p, b.WS_FORWARD) * K,
+                "clocks": clocks.summary(), "e2e": e2e}
+    if dist:
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank == 0:
+        if not args.no_cpu_baseline and world == 1:
+            line["cpu_baseline"] = cpu_baseline(cfg)
+        print(json.dumps(line), flush=True)
+    return 0
+
+
+def main():
+    args = parse()
+    cfg = synth.CONFIGS[args.config]
+    if args.impl == "reference":
+        return reference_arm(args, cfg)
+    return own_arm(args, cfg)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

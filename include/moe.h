@@ -1,0 +1,303 @@
+/*
+ * moe.h — C ABI of the routed mixture-of-experts expert FFN for NVIDIA B200 (sm_100a).
+ *
+ * The layer: top-k routing from router logits with an optional capacity drop,
+ * the token→expert permutation, per-expert gate/up GEMMs with a clamped SwiGLU,
+ * the down GEMM, and the gate-weighted combine back to token order. Sources
+ * (web pages, cited by title and part):
+ *   - "mini-AGI PR #3" minagi/pool.py, requested(): router softmax, top-k,
+ *     renormalised weights; flatten / argsort by expert / bincount; the
+ *     capacity drop (keep mask, counts.clamp(max=limit)).
+ *   - "mini-AGI PR #3/#4" configs/strix_halo_large.yaml, capacity_factor:
+ *     the most of a batch one expert may take as a multiple of its fair
+ *     share; the rest is dropped; 0 removes the cap.
+ *   - "mini-AGI PR #4" minagi/pool.py, experts()/run(): silu(x W1) * (x W3),
+ *     then W2; outputs read back in pair order.
+ *   - "Strata PR #4366" (DS4_FAT_ROWS), Approach: clamped SwiGLU; an
+ *     expert's weights decoded once, its rows gathered, one GEMM.
+ *   - "TensorFold PR #1607", What this changes: served plans with an always-on
+ *     shared expert ("256 + shared").
+ *
+ * Conventions for every call
+ *   - Pointers are DEVICE pointers owned by the caller unless a parameter says
+ *     "host". The library allocates no device memory: scratch comes from the
+ *     caller's workspace `ws` of at least moe_workspace_size() bytes, 256-byte
+ *     aligned. bf16 tensors are passed as uint16_t bit patterns.
+ *   - Calls are asynchronous on `stream` (a cudaStream_t; NULL = legacy
+ *     default stream). They make no host synchronisation, except
+ *     moe_get_error() and moe_forward_host(), which say so.
+ *   - Return value: MOE_OK, or an error detected on the host before any launch
+ *     (nothing was launched), or MOE_ERR_CUDA if a launch failed.
+ *   - Errors found on the device (a bound-checked index out of range, a
+ *     bounded wait that gave up) set bits in a sticky error word at the start
+ *     of the workspace; read it with moe_get_error(), reset with
+ *     moe_clear_error(). A kernel that sets it stops early and returns; its
+ *     outputs are then undefined.
+ *   - Limits: 1 <= k <= min(E, 8); 1 <= E <= 256; d_model and d_ff multiples
+ *     of 64; 1 <= T; shared expert only with bf16 weights and d_ff_shared ==
+ *     d_ff. Pointers to bf16/Q4G32 tensors 16-byte aligned.
+ *   - Calls that share one workspace must not overlap on the GPU.
+ */
+#ifndef MOE_B200_H
+#define MOE_B200_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct CUstream_st* moe_stream_t; /* same object as cudaStream_t */
+
+#if defined(__GNUC__)
+#define MOE_API __attribute__((visibility("default")))
+#else
+#define MOE_API
+#endif
+
+/* return codes */
+#define MOE_OK                      0
+#define MOE_ERR_INVALID_ARG         1 /* a size or flag outside the limits above */
+#define MOE_ERR_WORKSPACE_TOO_SMALL 2
+#define MOE_ERR_UNSUPPORTED         3 /* valid, but not implemented (see limits) */
+#define MOE_ERR_CUDA                4 /* a CUDA call or launch failed */
+#define MOE_ERR_MISALIGNED          5 /* a pointer without the 16-byte alignment */
+#define MOE_ERR_DEVICE              6 /* moe_get_error: the device error word is set */
+
+/* device error word bits (moe_get_error) */
+#define MOE_DEVERR_TIMEOUT 0x1u /* a bounded wait in a pipelined kernel gave up */
+#define MOE_DEVERR_BOUNDS  0x2u /* an expert id or row index outside its range */
+#define MOE_DEVERR_RANGE   0x4u /* an fp16 intermediate (h or y) beyond +-65504 or NaN */
+
+/* weight formats */
+#define MOE_WEIGHTS_BF16  0
+#define MOE_WEIGHTS_Q4G32 1
+
+/* expert kernel variants */
+#define MOE_VARIANT_AUTO   0 /* per expert, from its kept rows (stream_max_rows) */
+#define MOE_VARIANT_TENSOR 1 /* every expert on the tcgen05 tile kernels */
+#define MOE_VARIANT_STREAM 2 /* every expert on the few-rows weight-streaming kernels */
+
+/* layer output dtype */
+#define MOE_OUT_F32  0 /* fp32 (default): the residual stream's dtype */
+#define MOE_OUT_BF16 1
+
+/* workspace kinds for moe_workspace_size() */
+#define MOE_WS_ROUTE        0
+#define MOE_WS_PERMUTE      1
+#define MOE_WS_EXPERT_FFN   2
+#define MOE_WS_COMBINE      3
+#define MOE_WS_FORWARD      4
+#define MOE_WS_FORWARD_HOST 5
+
+typedef struct moe_params {
+    int32_t T;               /* tokens in this call */
+    int32_t d_model;         /* d */
+    int32_t d_ff;            /* f, per routed expert */
+    int32_t E;               /* routed experts */
+    int32_t k;               /* experts per token */
+    float capacity_factor;   /* 0 = no cap; else cap = ceil(cf * T * k / E) rows per expert,
+                                computed in double from this float */
+    float swiglu_limit;      /* L: gate and up pre-activations are clamped to [-L, L]; <= 0: no clamp */
+    int32_t weight_format;   /* MOE_WEIGHTS_* for the routed experts */
+    int32_t has_shared;      /* 1: add an always-on, un-gated shared expert */
+    int32_t d_ff_shared;     /* its f (must equal d_ff) */
+    int32_t variant;         /* MOE_VARIANT_* */
+    int32_t stream_max_rows; /* AUTO: experts with 1..this many kept rows use the streaming
+                                kernels, the rest the tcgen05 tiles; < 0 = library default */
+    int32_t out_dtype;       /* MOE_OUT_F32 | MOE_OUT_BF16 */
+} moe_params;
+
+/*
+ * Expert weights (device pointers).
+ *   BF16:  w_gate, w_up [E, d, f]; w_down [E, f, d]; row-major bf16; s_* NULL.
+ *   Q4G32 (self-defined): a matrix of reduction length K and output width N
+ *          is stored K-major as packed bytes [N, K/2] (byte j of row n holds
+ *          k = 2j in its low nibble, k = 2j+1 in its high nibble; nibble
+ *          u = q + 8, q in [-7, 7]) and fp16 scales [N, K/32], one per group of
+ *          32 consecutive k; the weight is q * s.
+ *          w_gate, w_up: [E, f, d/2] bytes, s_gate, s_up: [E, f, d/32] fp16;
+ *          w_down: [E, d, f/2] bytes, s_down: [E, d, f/32] fp16.
+ *   shared_*: bf16 [d, f], [d, f], [f, d] of the shared expert; NULL if has_shared = 0.
+ */
+typedef struct moe_weights {
+    const void* w_gate;
+    const void* w_up;
+    const void* w_down;
+    const void* s_gate;
+    const void* s_up;
+    const void* s_down;
+    const void* shared_gate;
+    const void* shared_up;
+    const void* shared_down;
+} moe_weights;
+
+/* Library version (major*10000 + minor*100 + patch). */
+MOE_API int moe_version(void);
+
+/* Human-readable name of a return code. */
+MOE_API const char* moe_status_string(int status);
+
+/*
+ * Per-expert capacity: *cap = ceil(cf * T * k / E), or -1 when cf <= 0.
+ * ("mini-AGI" capacity_factor; see the file comment.)
+ */
+MOE_API int moe_capacity(const moe_params* p, int32_t* cap);
+
+/*
+ * Rows of the permuted buffers (sorted_token, sorted_pair, y_rows):
+ * min(T*k, E*cap) (T*k with no cap) plus T when has_shared.
+ */
+MOE_API int moe_max_rows(const moe_params* p, int64_t* rows);
+
+/* Bytes of workspace each call needs (which = MOE_WS_*); 0 on invalid params. */
+MOE_API size_t moe_workspace_size(const moe_params* p, int which);
+
+/*
+ * moe_route — S1 of the path: per token, the top-k experts and their weights.
+ *   "mini-AGI PR #3" requested(): softmax of the logits, top-k, renormalised
+ *   (= a softmax over the k selected logits).
+ * logits   fp32 [T, E] row-major (finite; NaN is outside the contract).
+ * topk_idx int32 [T, k]: expert ids in descending logit order; equal logits
+ *          go to the lower index (-0.0 equals +0.0). Compared exactly in fp32.
+ * topk_w   fp32 [T, k]: exp(l_j - l_max) / sum over the k selected.
+ */
+MOE_API int moe_route(const moe_params* p, const float* logits, int32_t* topk_idx, float* topk_w,
+              void* ws, size_t ws_bytes, moe_stream_t stream);
+
+/*
+ * moe_permute — S2/S3: histogram, prefix offsets, scatter, capacity drop.
+ *   "mini-AGI PR #3" requested(): pairs sorted by expert, bincount, the keep
+ *   mask over each expert's pairs, counts clamped to the limit.
+ * Pair p = t*k + j. Let E' = E + has_shared.
+ * topk_idx     int32 [T, k] (ids in [0, E); out-of-range ids set MOE_DEVERR_BOUNDS)
+ * counts       int32 [E']   pairs requested per expert (shared: T)
+ * kept_counts  int32 [E']   min(counts, cap)
+ * offsets      int32 [E'+1] exclusive prefix of kept_counts; offsets[E'] = rows used
+ * sorted_token int32 [moe_max_rows] token of each row; within an expert ascending
+ * sorted_pair  int32 [moe_max_rows] pair of each row (-1 for shared rows)
+ * pair_row     int32 [T*k]  row of each pair, -1 if dropped
+ * The drop keeps, per expert, its first cap pairs in token order. Bit-exact:
+ * the result is unique (no atomics decide an order).
+ */
+MOE_API int moe_permute(const moe_params* p, const int32_t* topk_idx, int32_t* counts,
+                int32_t* kept_counts, int32_t* offsets, int32_t* sorted_token,
+                int32_t* sorted_pair, int32_t* pair_row, void* ws, size_t ws_bytes,
+                moe_stream_t stream);
+
+/*
+ * moe_expert_ffn — S4..S6 (+ S8, S9): per expert e, rows r in
+ * [offsets[e], offsets[e+1]):
+ *   g = x[sorted_token[r]] W_gate[e],  u = x[sorted_token[r]] W_up[e]
+ *   h = silu(clamp(g, -L, L)) * clamp(u, -L, L)        (fp32, then fp16)
+ *   y_rows[r] = w_r * (h W_down[e])                     (fp32, then fp16)
+ * with w_r = topk_w[sorted_pair[r]] (1 for shared rows).
+ *   "mini-AGI PR #4" experts(); "Strata PR #4366" Approach (clamped SwiGLU,
+ *   an expert's weights decoded once and its rows gathered).
+ * x       bf16 [T, d]; offsets / sorted_token / sorted_pair as moe_permute writes them
+ * topk_w  fp32 [T, k]
+ * y_rows  fp16 [moe_max_rows, d]; rows past offsets[E'] are not written.
+ * Precision: x and the gate/up weights enter the tensor cores as given (bf16),
+ * fp32 accumulate; h is kept in fp16 and the down GEMM runs in fp16 (each
+ * W_down tile is converted bf16 -> fp16 in shared memory, exact for values in
+ * fp16's normal range), fp32 accumulate; y in fp16. A value of h or y past
+ * +-65504 sets MOE_DEVERR_RANGE. (Strata PR #4366 runs its expert GEMM and
+ * SwiGLU in FP16 for the same reason: more significand than bf16.)
+ * Each expert runs either the tcgen05 tile kernels or the few-rows streaming
+ * kernels (params.variant / stream_max_rows). Weights of experts without rows
+ * are never read.
+ */
+MOE_API int moe_expert_ffn(const moe_params* p, const uint16_t* x, const int32_t* offsets,
+                   const int32_t* sorted_token, const int32_t* sorted_pair,
+                   const float* topk_w, const moe_weights* w, uint16_t* y_rows,
+                   void* ws, size_t ws_bytes, moe_stream_t stream);
+
+/*
+ * moe_combine — S7: out[t] = sum over j in 0..k-1 with pair_row[t*k+j] >= 0 of
+ * y_rows[pair_row[t*k+j]] (fp16, already gate-weighted), plus y_rows[offsets[E] + t]
+ * when has_shared; fp32 in fixed j order, written as out_dtype (fp32 by
+ * default, or bf16). Deterministic.
+ *   "mini-AGI PR #4" run(): outputs gathered back in pair order and summed.
+ * A dropped pair adds nothing; the other weights are not renormalised.
+ * offsets may be NULL when has_shared = 0.
+ */
+MOE_API int moe_combine(const moe_params* p, const uint16_t* y_rows, const int32_t* pair_row,
+                const int32_t* offsets, void* out, void* ws, size_t ws_bytes,
+                moe_stream_t stream);
+
+/*
+ * moe_forward — the whole layer (route → permute → expert FFN → combine) on
+ * one stream with no host synchronisation; intermediates live in ws.
+ * x bf16 [T, d], logits fp32 [T, E], out [T, d] of out_dtype (fp32 default).
+ * counts_out: NULL, or int32 [E'] receiving the per-expert requested counts.
+ */
+MOE_API int moe_forward(const moe_params* p, const uint16_t* x, const float* logits,
+                const moe_weights* w, void* out, int32_t* counts_out,
+                void* ws, size_t ws_bytes, moe_stream_t stream);
+
+/*
+ * moe_forward_host — moe_forward with HOST x, logits and out (weights stay on
+ * the device): copies x and logits in, runs the layer, copies out back, then
+ * synchronises the stream. Host buffers may be pageable; pinned is faster.
+ * ws: MOE_WS_FORWARD_HOST bytes (holds device copies of x, logits, out).
+ */
+MOE_API int moe_forward_host(const moe_params* p, const uint16_t* x_host, const float* logits_host,
+                     const moe_weights* w, void* out_host, void* ws, size_t ws_bytes,
+                     moe_stream_t stream);
+
+/*
+ * Synchronises `stream`, then reads the sticky device error word at the start
+ * of ws into *err (host). Returns MOE_OK if it is 0, MOE_ERR_DEVICE if not.
+ */
+MOE_API int moe_get_error(const void* ws, uint32_t* err, moe_stream_t stream);
+
+/* Resets the device error word (asynchronous). */
+MOE_API int moe_clear_error(void* ws, moe_stream_t stream);
+
+/*
+ * Test hook: the time limit, in nanoseconds, of every bounded wait in the
+ * pipelined kernels launched after this call by this process (default 1 s).
+ * 0 restores the default.
+ */
+MOE_API int moe_set_wait_limit_ns(uint64_t ns);
+
+/*
+ * Kernel ids for the profiler and moe_launch_count(). Each is one kernel of
+ * the library; a call launches a fixed sequence of them (no host sync).
+ */
+#define MOE_K_ROUTE          0  /* S1 top-k softmax router */
+#define MOE_K_PERM_COUNT     1  /* S2 per-block histograms */
+#define MOE_K_PERM_SCAN      2  /* S2 block bases, counts, kept, offsets */
+#define MOE_K_PERM_SCATTER   3  /* S3 ranks, drop, row lists */
+#define MOE_K_SCHEDULE       4  /* per-expert variant choice and M-tile prefix */
+#define MOE_K_GATHER         5  /* S4 row gather for the tile kernels */
+#define MOE_K_TC_GATEUP      6  /* S5 tcgen05 gate/up GEMM + clamped SwiGLU */
+#define MOE_K_TC_DOWN        7  /* S6 tcgen05 down GEMM + gate scale */
+#define MOE_K_STREAM_GATEUP  8  /* S8 few-rows gate/up (weight streaming) */
+#define MOE_K_STREAM_REDUCE  9  /* S8 K-split partial sums + SwiGLU */
+#define MOE_K_STREAM_DOWN   10  /* S8 few-rows down */
+#define MOE_K_COMBINE       11  /* S7 gate-weighted combine */
+#define MOE_K_COUNT         12
+
+/*
+ * Number of kernel launches one call of `which` (MOE_WS_ROUTE .. MOE_WS_FORWARD_HOST,
+ * naming moe_route .. moe_forward_host) makes with these params, into *n (host).
+ */
+MOE_API int moe_launch_count(const moe_params* p, int which, int* n);
+
+/*
+ * Per-kernel timing. moe_profile_enable(1): from then on every launch is
+ * bracketed by two CUDA events recorded on its stream (cheap; off by default).
+ * moe_profile_collect(): waits for the recorded events, writes the summed
+ * milliseconds and launch counts per kernel id (host arrays of MOE_K_COUNT)
+ * and forgets them.
+ */
+MOE_API int moe_profile_enable(int on);
+MOE_API int moe_profile_collect(double* total_ms, int64_t* launches);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MOE_B200_H */

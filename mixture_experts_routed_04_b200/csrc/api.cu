@@ -1,0 +1,391 @@
+// api.cu — the C ABI declared in include/moe.h: parameter checks, workspace
+// layout, and the order of launches. Every step of the layer runs in the
+// kernels of this library; nothing here computes on the host beyond sizes.
+#include <atomic>
+#include <cmath>
+#include <cstring>
+
+#include "internal.h"
+
+namespace moe {
+
+cudaError_t launch_schedule(const Dims& D, const int32_t* offsets, int32_t* tile_base, int32_t* stream_list,
+                            int32_t* n_stream, uint32_t* err, cudaStream_t s);
+cudaError_t launch_gather(const Dims& D, const uint16_t* x, const int32_t* sorted_token, const int32_t* offsets,
+                          uint16_t* xg, uint32_t* err, cudaStream_t s);
+cudaError_t launch_tensor_ffn(const Dims& D, const uint16_t* xg, uint16_t* h, const int32_t* tile_base,
+                              const int32_t* offsets, const int32_t* sorted_pair, const float* topk_w,
+                              const moe_weights* w, uint16_t* y_rows, uint32_t* err, uint64_t wait_ns,
+                              cudaStream_t s);
+cudaError_t launch_stream_ffn(const Dims& D, const uint16_t* x, uint16_t* h, float* part, const int32_t* offsets,
+                              const int32_t* stream_list, const int32_t* n_stream, const int32_t* sorted_token,
+                              const int32_t* sorted_pair, const float* topk_w, const moe_weights* w,
+                              uint16_t* y_rows, uint32_t* err, uint64_t wait_ns, cudaStream_t s);
+
+static std::atomic<uint64_t> g_wait_ns{1000000000ull};
+
+int num_sms() {
+    static int cached[64] = {0};
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (dev < 0 || dev >= 64) dev = 0;
+    if (!cached[dev]) {
+        int n = 0;
+        cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+        cached[dev] = n > 0 ? n : 148;
+    }
+    return cached[dev];
+}
+
+static size_t align256(size_t v) { return (v + 255) & ~size_t(255); }
+
+// Host-side checks of moe_params; fills D. Returns MOE_OK or an error code.
+static int make_dims(const moe_params* p, Dims* D) {
+    if (!p || !D) return MOE_ERR_INVALID_ARG;
+    if (p->T < 1 || p->E < 1 || p->E > kMaxE || p->k < 1 || p->k > kMaxK || p->k > p->E) return MOE_ERR_INVALID_ARG;
+    if (p->d_model < 64 || p->d_model % 64 || p->d_ff < 64 || p->d_ff % 64) return MOE_ERR_INVALID_ARG;
+    if (!(p->capacity_factor >= 0.f) || !std::isfinite(p->capacity_factor)) return MOE_ERR_INVALID_ARG;
+    if (!std::isfinite(p->swiglu_limit)) return MOE_ERR_INVALID_ARG;
+    if (p->weight_format != MOE_WEIGHTS_BF16 && p->weight_format != MOE_WEIGHTS_Q4G32) return MOE_ERR_INVALID_ARG;
+    if (p->variant < MOE_VARIANT_AUTO || p->variant > MOE_VARIANT_STREAM) return MOE_ERR_INVALID_ARG;
+    if (p->has_shared != 0 && p->has_shared != 1) return MOE_ERR_INVALID_ARG;
+    if (p->out_dtype != MOE_OUT_F32 && p->out_dtype != MOE_OUT_BF16) return MOE_ERR_INVALID_ARG;
+    const int64_t pairs = int64_t(p->T) * p->k;
+    if (pairs + p->T >= (int64_t(1) << 31)) return MOE_ERR_INVALID_ARG;
+    if (int64_t(p->d_model) * p->d_ff * p->E >= (int64_t(1) << 40)) return MOE_ERR_INVALID_ARG;
+    if (p->has_shared && (p->d_ff_shared != p->d_ff)) return MOE_ERR_UNSUPPORTED;
+    if (p->weight_format == MOE_WEIGHTS_Q4G32) return MOE_ERR_UNSUPPORTED;  // not built yet
+    D->T = p->T;
+    D->d = p->d_model;
+    D->f = p->d_ff;
+    D->E = p->E;
+    D->k = p->k;
+    D->has_shared = p->has_shared;
+    D->Etot = p->E + p->has_shared;
+    D->pairs = pairs;
+    D->cap = -1;
+    int64_t routed_rows = pairs;
+    if (p->capacity_factor > 0.f) {
+        const double c = std::ceil(double(p->capacity_factor) * double(p->T) * double(p->k) / double(p->E));
+        if (c < 0 || c > double(1 << 30)) return MOE_ERR_INVALID_ARG;
+        D->cap = int(c);
+        const int64_t lim = int64_t(D->cap) * p->E;
+        if (lim < routed_rows) routed_rows = lim;
+    }
+    D->rows = routed_rows + (p->has_shared ? p->T : 0);
+    if (D->rows < 1) D->rows = 1;
+    D->perm_blocks = int((pairs + kPermPairsPerBlock - 1) / kPermPairsPerBlock);
+    D->fmt = p->weight_format;
+    D->variant = p->variant;
+    D->stream_max_rows = p->stream_max_rows < 0 ? kDefaultStreamMaxRows : p->stream_max_rows;
+    D->limit = p->swiglu_limit;
+    D->out_bf16 = p->out_dtype == MOE_OUT_BF16;
+    // The streaming kernels hold one K slice of <= 2048 rows in shared memory:
+    // gate/up split d into slices; down needs f <= 2048.
+    const bool stream_ok = p->d_ff <= 2048;
+    if (!stream_ok) {
+        if (D->variant == MOE_VARIANT_STREAM) return MOE_ERR_UNSUPPORTED;
+        D->stream_max_rows = 0;
+    }
+    // K split of the streaming gate/up: enough units to cover the SMs when few
+    // experts are touched (decode), and slices of at most 2048.
+    int ks = 1;
+    while (p->d_model / ks > 2048) ks *= 2;
+    const int64_t touched = std::min<int64_t>(D->Etot, pairs + p->has_shared);
+    const int64_t units = touched * (p->d_ff / 64);
+    while (ks < 8 && units * ks < 4 * 148 && (p->d_model % (ks * 2 * 64)) == 0) ks *= 2;
+    if (p->d_model % (ks * 64)) return MOE_ERR_UNSUPPORTED;
+    D->ks = ks;
+    return MOE_OK;
+}
+
+WsLayout ws_layout(const Dims& D, int which) {
+    WsLayout L;
+    std::memset(&L, 0, sizeof(L));
+    size_t off = 256;  // [0, 256): error word
+    auto take = [&](size_t bytes) {
+        const size_t o = off;
+        off = align256(off + bytes);
+        return o;
+    };
+    const bool perm = which == MOE_WS_PERMUTE || which >= MOE_WS_FORWARD;
+    const bool ffn = which == MOE_WS_EXPERT_FFN || which >= MOE_WS_FORWARD;
+    const bool fwd = which >= MOE_WS_FORWARD;
+    if (perm) {
+        L.blockcounts = take(size_t(D.perm_blocks) * D.E * 4);
+        L.blockbase = take(size_t(D.perm_blocks) * D.E * 4);
+    }
+    if (ffn) {
+        L.tile_base = take(size_t(D.Etot + 1) * 4);
+        L.stream_list = take(size_t(D.Etot) * 4);
+        L.n_stream = take(4);
+        L.xg = take(size_t(D.rows) * D.d * 2);
+        L.h = take(size_t(D.rows) * D.f * 2);
+        if (D.ks > 1) L.part = take(size_t(D.ks) * 2 * D.rows * D.f * 4);
+    }
+    if (fwd) {
+        L.topk_idx = take(size_t(D.pairs) * 4);
+        L.topk_w = take(size_t(D.pairs) * 4);
+        L.counts = take(size_t(D.Etot) * 4);
+        L.kept = take(size_t(D.Etot) * 4);
+        L.offsets = take(size_t(D.Etot + 1) * 4);
+        L.sorted_token = take(size_t(D.rows) * 4);
+        L.sorted_pair = take(size_t(D.rows) * 4);
+        L.pair_row = take(size_t(D.pairs) * 4);
+        L.y_rows = take(size_t(D.rows) * D.d * 2);
+    }
+    if (which == MOE_WS_FORWARD_HOST) {
+        L.x_dev = take(size_t(D.T) * D.d * 2);
+        L.logits_dev = take(size_t(D.T) * D.E * 4);
+        L.out_dev = take(size_t(D.T) * D.d * (D.out_bf16 ? 2 : 4));
+    }
+    L.total = off;
+    return L;
+}
+
+cudaError_t launch_expert_ffn(const Dims& D, const WsLayout& L, const FfnArgs& a, cudaStream_t s) {
+    uint8_t* ws = a.ws;
+    int32_t* tile_base = reinterpret_cast<int32_t*>(ws + L.tile_base);
+    int32_t* stream_list = reinterpret_cast<int32_t*>(ws + L.stream_list);
+    int32_t* n_stream = reinterpret_cast<int32_t*>(ws + L.n_stream);
+    uint16_t* xg = reinterpret_cast<uint16_t*>(ws + L.xg);
+    uint16_t* h = reinterpret_cast<uint16_t*>(ws + L.h);
+    float* part = L.part ? reinterpret_cast<float*>(ws + L.part) : nullptr;
+    cudaError_t e = launch_schedule(D, a.offsets, tile_base, stream_list, n_stream, a.err, s);
+    if (e != cudaSuccess) return e;
+    if (D.variant != MOE_VARIANT_STREAM) {
+        if ((e = launch_gather(D, a.x, a.sorted_token, a.offsets, xg, a.err, s)) != cudaSuccess) return e;
+        if ((e = launch_tensor_ffn(D, xg, h, tile_base, a.offsets, a.sorted_pair, a.topk_w, a.w, a.y_rows, a.err,
+                                   a.wait_ns, s)) != cudaSuccess)
+            return e;
+    }
+    if (D.variant != MOE_VARIANT_TENSOR && D.stream_max_rows > 0) {
+        if ((e = launch_stream_ffn(D, a.x, h, part, a.offsets, stream_list, n_stream, a.sorted_token, a.sorted_pair,
+                                   a.topk_w, a.w, a.y_rows, a.err, a.wait_ns, s)) != cudaSuccess)
+            return e;
+    }
+    return cudaSuccess;
+}
+
+}  // namespace moe
+
+using namespace moe;
+
+static bool al16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+static int check_ws(const Dims& D, int which, const void* ws, size_t ws_bytes) {
+    if (!ws) return MOE_ERR_INVALID_ARG;
+    if (reinterpret_cast<uintptr_t>(ws) & 255u) return MOE_ERR_MISALIGNED;
+    if (ws_bytes < ws_layout(D, which).total) return MOE_ERR_WORKSPACE_TOO_SMALL;
+    return MOE_OK;
+}
+
+static int check_weights(const Dims& D, const moe_weights* w) {
+    if (!w || !w->w_gate || !w->w_up || !w->w_down) return MOE_ERR_INVALID_ARG;
+    if (!al16(w->w_gate) || !al16(w->w_up) || !al16(w->w_down)) return MOE_ERR_MISALIGNED;
+    if (D.has_shared) {
+        if (!w->shared_gate || !w->shared_up || !w->shared_down) return MOE_ERR_INVALID_ARG;
+        if (!al16(w->shared_gate) || !al16(w->shared_up) || !al16(w->shared_down)) return MOE_ERR_MISALIGNED;
+    }
+    return MOE_OK;
+}
+
+static int status_of(cudaError_t e) { return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA; }
+
+extern "C" {
+
+int moe_version(void) { return 100; }
+
+const char* moe_status_string(int s) {
+    switch (s) {
+        case MOE_OK: return "ok";
+        case MOE_ERR_INVALID_ARG: return "invalid argument";
+        case MOE_ERR_WORKSPACE_TOO_SMALL: return "workspace too small";
+        case MOE_ERR_UNSUPPORTED: return "unsupported configuration";
+        case MOE_ERR_CUDA: return "CUDA error";
+        case MOE_ERR_MISALIGNED: return "misaligned pointer";
+        case MOE_ERR_DEVICE: return "device error word set";
+        default: return "unknown status";
+    }
+}
+
+int moe_capacity(const moe_params* p, int32_t* cap) {
+    Dims D;
+    const int st = make_dims(p, &D);
+    if (st != MOE_OK) return st;
+    if (!cap) return MOE_ERR_INVALID_ARG;
+    *cap = D.cap;
+    return MOE_OK;
+}
+
+int moe_max_rows(const moe_params* p, int64_t* rows) {
+    Dims D;
+    const int st = make_dims(p, &D);
+    if (st != MOE_OK) return st;
+    if (!rows) return MOE_ERR_INVALID_ARG;
+    *rows = D.rows;
+    return MOE_OK;
+}
+
+size_t moe_workspace_size(const moe_params* p, int which) {
+    Dims D;
+    if (make_dims(p, &D) != MOE_OK || which < MOE_WS_ROUTE || which > MOE_WS_FORWARD_HOST) return 0;
+    return ws_layout(D, which).total;
+}
+
+int moe_route(const moe_params* p, const float* logits, int32_t* topk_idx, float* topk_w, void* ws,
+              size_t ws_bytes, moe_stream_t stream) {
+    Dims D;
+    int st = make_dims(p, &D);
+    if (st != MOE_OK) return st;
+    if ((st = check_ws(D, MOE_WS_ROUTE, ws, ws_bytes)) != MOE_OK) return st;
+    if (!logits || !topk_idx || !topk_w) return MOE_ERR_INVALID_ARG;
+    return status_of(launch_route(logits, D.T, D.E, D.k, topk_idx, topk_w, stream));
+}
+
+int moe_permute(const moe_params* p, const int32_t* topk_idx, int32_t* counts, int32_t* kept_counts,
+                int32_t* offsets, int32_t* sorted_token, int32_t* sorted_pair, int32_t* pair_row, void* ws,
+                size_t ws_bytes, moe_stream_t stream) {
+    Dims D;
+    int st = make_dims(p, &D);
+    if (st != MOE_OK) return st;
+    if ((st = check_ws(D, MOE_WS_PERMUTE, ws, ws_bytes)) != MOE_OK) return st;
+    if (!topk_idx || !counts || !kept_counts || !offsets || !sorted_token || !sorted_pair || !pair_row)
+        return MOE_ERR_INVALID_ARG;
+    const WsLayout L = ws_layout(D, MOE_WS_PERMUTE);
+    uint8_t* w = static_cast<uint8_t*>(ws);
+    return status_of(launch_permute(D, topk_idx, reinterpret_cast<int32_t*>(w + L.blockcounts),
+                                    reinterpret_cast<int32_t*>(w + L.blockbase), counts, kept_counts, offsets,
+                                    sorted_token, sorted_pair, pair_row, reinterpret_cast<uint32_t*>(w), stream));
+}
+
+int moe_expert_ffn(const moe_params* p, const uint16_t* x, const int32_t* offsets, const int32_t* sorted_token,
+                   const int32_t* sorted_pair, const float* topk_w, const moe_weights* w, uint16_t* y_rows,
+                   void* ws, size_t ws_bytes, moe_stream_t stream) {
+    Dims D;
+    int st = make_dims(p, &D);
+    if (st != MOE_OK) return st;
+    if ((st = check_ws(D, MOE_WS_EXPERT_FFN, ws, ws_bytes)) != MOE_OK) return st;
+    if ((st = check_weights(D, w)) != MOE_OK) return st;
+    if (!x || !offsets || !sorted_token || !sorted_pair || !topk_w || !y_rows) return MOE_ERR_INVALID_ARG;
+    if (!al16(x) || !al16(y_rows)) return MOE_ERR_MISALIGNED;
+    const WsLayout L = ws_layout(D, MOE_WS_EXPERT_FFN);
+    FfnArgs a{x, offsets, sorted_token, sorted_pair, topk_w, w, y_rows, static_cast<uint8_t*>(ws),
+              static_cast<uint32_t*>(ws), g_wait_ns.load()};
+    return status_of(launch_expert_ffn(D, L, a, stream));
+}
+
+int moe_combine(const moe_params* p, const uint16_t* y_rows, const int32_t* pair_row, const int32_t* offsets,
+                void* out, void* ws, size_t ws_bytes, moe_stream_t stream) {
+    Dims D;
+    int st = make_dims(p, &D);
+    if (st != MOE_OK) return st;
+    if ((st = check_ws(D, MOE_WS_COMBINE, ws, ws_bytes)) != MOE_OK) return st;
+    if (!y_rows || !pair_row || !out || (D.has_shared && !offsets)) return MOE_ERR_INVALID_ARG;
+    if (!al16(y_rows) || !al16(out)) return MOE_ERR_MISALIGNED;
+    return status_of(launch_combine(D, y_rows, pair_row, offsets, out, stream));
+}
+
+static int forward_impl(const Dims& D, const WsLayout& L, const uint16_t* x, const float* logits,
+                        const moe_weights* w, void* out, int32_t* counts_out, uint8_t* ws,
+                        cudaStream_t stream) {
+    int32_t* topk_idx = reinterpret_cast<int32_t*>(ws + L.topk_idx);
+    float* topk_w = reinterpret_cast<float*>(ws + L.topk_w);
+    int32_t* counts = reinterpret_cast<int32_t*>(ws + L.counts);
+    int32_t* kept = reinterpret_cast<int32_t*>(ws + L.kept);
+    int32_t* offsets = reinterpret_cast<int32_t*>(ws + L.offsets);
+    int32_t* sorted_token = reinterpret_cast<int32_t*>(ws + L.sorted_token);
+    int32_t* sorted_pair = reinterpret_cast<int32_t*>(ws + L.sorted_pair);
+    int32_t* pair_row = reinterpret_cast<int32_t*>(ws + L.pair_row);
+    uint16_t* y_rows = reinterpret_cast<uint16_t*>(ws + L.y_rows);
+    uint32_t* err = reinterpret_cast<uint32_t*>(ws);
+    cudaError_t e = launch_route(logits, D.T, D.E, D.k, topk_idx, topk_w, stream);
+    if (e != cudaSuccess) return MOE_ERR_CUDA;
+    e = launch_permute(D, topk_idx, reinterpret_cast<int32_t*>(ws + L.blockcounts),
+                       reinterpret_cast<int32_t*>(ws + L.blockbase), counts, kept, offsets, sorted_token,
+                       sorted_pair, pair_row, err, stream);
+    if (e != cudaSuccess) return MOE_ERR_CUDA;
+    FfnArgs a{x, offsets, sorted_token, sorted_pair, topk_w, w, y_rows, ws, err, g_wait_ns.load()};
+    if ((e = launch_expert_ffn(D, L, a, stream)) != cudaSuccess) return MOE_ERR_CUDA;
+    if ((e = launch_combine(D, y_rows, pair_row, offsets, out, stream)) != cudaSuccess) return MOE_ERR_CUDA;
+    if (counts_out &&
+        cudaMemcpyAsync(counts_out, counts, size_t(D.Etot) * 4, cudaMemcpyDeviceToDevice, stream) != cudaSuccess)
+        return MOE_ERR_CUDA;
+    return MOE_OK;
+}
+
+int moe_forward(const moe_params* p, const uint16_t* x, const float* logits, const moe_weights* w, void* out,
+                int32_t* counts_out, void* ws, size_t ws_bytes, moe_stream_t stream) {
+    Dims D;
+    int st = make_dims(p, &D);
+    if (st != MOE_OK) return st;
+    if ((st = check_ws(D, MOE_WS_FORWARD, ws, ws_bytes)) != MOE_OK) return st;
+    if ((st = check_weights(D, w)) != MOE_OK) return st;
+    if (!x || !logits || !out) return MOE_ERR_INVALID_ARG;
+    if (!al16(x) || !al16(out)) return MOE_ERR_MISALIGNED;
+    return forward_impl(D, ws_layout(D, MOE_WS_FORWARD), x, logits, w, out, counts_out, static_cast<uint8_t*>(ws),
+                        stream);
+}
+
+int moe_forward_host(const moe_params* p, const uint16_t* x_host, const float* logits_host, const moe_weights* w,
+                     void* out_host, void* ws, size_t ws_bytes, moe_stream_t stream) {
+    Dims D;
+    int st = make_dims(p, &D);
+    if (st != MOE_OK) return st;
+    if ((st = check_ws(D, MOE_WS_FORWARD_HOST, ws, ws_bytes)) != MOE_OK) return st;
+    if ((st = check_weights(D, w)) != MOE_OK) return st;
+    if (!x_host || !logits_host || !out_host) return MOE_ERR_INVALID_ARG;
+    const WsLayout L = ws_layout(D, MOE_WS_FORWARD_HOST);
+    uint8_t* wsb = static_cast<uint8_t*>(ws);
+    uint16_t* xd = reinterpret_cast<uint16_t*>(wsb + L.x_dev);
+    float* ld = reinterpret_cast<float*>(wsb + L.logits_dev);
+    void* od = wsb + L.out_dev;
+    if (cudaMemcpyAsync(xd, x_host, size_t(D.T) * D.d * 2, cudaMemcpyHostToDevice, stream) != cudaSuccess ||
+        cudaMemcpyAsync(ld, logits_host, size_t(D.T) * D.E * 4, cudaMemcpyHostToDevice, stream) != cudaSuccess)
+        return MOE_ERR_CUDA;
+    st = forward_impl(D, L, xd, ld, w, od, nullptr, wsb, stream);
+    if (st != MOE_OK) return st;
+    if (cudaMemcpyAsync(out_host, od, size_t(D.T) * D.d * (D.out_bf16 ? 2 : 4), cudaMemcpyDeviceToHost, stream) !=
+        cudaSuccess)
+        return MOE_ERR_CUDA;
+    return cudaStreamSynchronize(stream) == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+}
+
+int moe_get_error(const void* ws, uint32_t* err, moe_stream_t stream) {
+    if (!ws || !err) return MOE_ERR_INVALID_ARG;
+    uint32_t v = 0;
+    if (cudaMemcpyAsync(&v, ws, 4, cudaMemcpyDeviceToHost, stream) != cudaSuccess) return MOE_ERR_CUDA;
+    if (cudaStreamSynchronize(stream) != cudaSuccess) return MOE_ERR_CUDA;
+    *err = v;
+    return v ? MOE_ERR_DEVICE : MOE_OK;
+}
+
+int moe_clear_error(void* ws, moe_stream_t stream) {
+    if (!ws) return MOE_ERR_INVALID_ARG;
+    return cudaMemsetAsync(ws, 0, 4, stream) == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+}
+
+int moe_launch_count(const moe_params* p, int which, int* n) {
+    Dims D;
+    const int st = make_dims(p, &D);
+    if (st != MOE_OK) return st;
+    if (!n || which < MOE_WS_ROUTE || which > MOE_WS_FORWARD_HOST) return MOE_ERR_INVALID_ARG;
+    int ffn = 1;  // schedule
+    if (D.variant != MOE_VARIANT_STREAM) ffn += 3;  // gather + two tcgen05 GEMMs
+    if (D.variant != MOE_VARIANT_TENSOR && D.stream_max_rows > 0) ffn += 2 + (D.ks > 1 ? 1 : 0);
+    switch (which) {
+        case MOE_WS_ROUTE: *n = 1; break;
+        case MOE_WS_PERMUTE: *n = 3; break;
+        case MOE_WS_EXPERT_FFN: *n = ffn; break;
+        case MOE_WS_COMBINE: *n = 1; break;
+        default: *n = 1 + 3 + ffn + 1; break;
+    }
+    return MOE_OK;
+}
+
+int moe_set_wait_limit_ns(uint64_t ns) {
+    g_wait_ns.store(ns ? ns : 1000000000ull);
+    return MOE_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,81 @@
+// combine.cu — S7: gate-weighted outputs summed back to token order.
+//
+// "mini-AGI PR #4", minagi/pool.py run(): the expert outputs are read back in
+// pair order (y[e_sorted, slot]) and each token's k outputs are summed with
+// their gate weights. The weights were applied in the down-projection
+// epilogue, so here out[t] = sum over kept j of y_rows[pair_row[t*k+j]]
+// (+ the shared expert's row), accumulated in fp32 in fixed j order, then
+// rounded to bf16 once. A dropped pair (row -1) adds nothing.
+//
+// HBM-bound: one 16-byte vector (8 bf16) per thread per row read; blocks walk
+// tokens with a grid stride; no atomics, so the result is deterministic.
+#include "internal.h"
+
+namespace moe {
+
+namespace {
+
+template <bool OUT_BF16>
+__global__ void __launch_bounds__(256) combine_kernel(const uint16_t* __restrict__ y_rows,
+                                                      const int32_t* __restrict__ pair_row,
+                                                      const int32_t* __restrict__ offsets, int T, int d, int k,
+                                                      int E, int has_shared, void* __restrict__ out) {
+    const int vec_per_row = d / 8;  // d % 64 == 0
+    const int64_t total = int64_t(T) * vec_per_row;
+    const int shared_base = has_shared ? offsets[E] : 0;
+    for (int64_t i = int64_t(blockIdx.x) * blockDim.x + threadIdx.x; i < total; i += int64_t(gridDim.x) * blockDim.x) {
+        const int64_t t = i / vec_per_row;
+        const int c = int(i - t * vec_per_row);
+        float acc[8];
+#pragma unroll
+        for (int q = 0; q < 8; ++q) acc[q] = 0.f;
+        auto add = [&](int64_t r) {
+            const uint4 v = __ldg(reinterpret_cast<const uint4*>(y_rows + r * d) + c);
+            acc[0] += f16_lo(v.x); acc[1] += f16_hi(v.x);
+            acc[2] += f16_lo(v.y); acc[3] += f16_hi(v.y);
+            acc[4] += f16_lo(v.z); acc[5] += f16_hi(v.z);
+            acc[6] += f16_lo(v.w); acc[7] += f16_hi(v.w);
+        };
+        for (int j = 0; j < k; ++j) {
+            const int r = pair_row[t * k + j];
+            if (r >= 0) add(r);
+        }
+        if (has_shared) add(shared_base + t);
+        if (OUT_BF16) {
+            uint4 o;
+            o.x = pack_bf16x2(acc[0], acc[1]);
+            o.y = pack_bf16x2(acc[2], acc[3]);
+            o.z = pack_bf16x2(acc[4], acc[5]);
+            o.w = pack_bf16x2(acc[6], acc[7]);
+            reinterpret_cast<uint4*>(static_cast<uint16_t*>(out) + t * d)[c] = o;
+        } else {
+            float4* dst = reinterpret_cast<float4*>(static_cast<float*>(out) + t * d + c * 8);
+            dst[0] = make_float4(acc[0], acc[1], acc[2], acc[3]);
+            dst[1] = make_float4(acc[4], acc[5], acc[6], acc[7]);
+        }
+    }
+}
+
+}  // namespace
+
+cudaError_t launch_combine(const Dims& D, const uint16_t* y_rows, const int32_t* pair_row, const int32_t* offsets,
+                           void* out, cudaStream_t s) {
+    const int64_t total = int64_t(D.T) * (D.d / 8);
+    const int threads = 256;
+    int64_t blocks = (total + threads - 1) / threads;
+    const int64_t cap = int64_t(num_sms()) * 8;
+    if (blocks > cap) blocks = cap;
+    if (blocks < 1) blocks = 1;
+    {
+        ProfScope prof_(MOE_K_COMBINE, s);
+        if (D.out_bf16)
+            combine_kernel<true><<<int(blocks), threads, 0, s>>>(y_rows, pair_row, offsets, D.T, D.d, D.k, D.E,
+                                                                 D.has_shared, out);
+        else
+            combine_kernel<false><<<int(blocks), threads, 0, s>>>(y_rows, pair_row, offsets, D.T, D.d, D.k, D.E,
+                                                                  D.has_shared, out);
+    }
+    return cudaGetLastError();
+}
+
+}  // namespace moe

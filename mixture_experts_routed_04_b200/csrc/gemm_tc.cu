@@ -1,0 +1,589 @@
+// gemm_tc.cu — S4..S6 on the 5th-generation tensor cores: the tile schedule
+// (K3), the row gather (S4), and one persistent grouped GEMM kernel used twice:
+//   MODE 0: h = silu(clamp(x W_gate[e])) * clamp(x W_up[e])   (S5, SwiGLU fused)
+//   MODE 1: y = w_pair * (h W_down[e])                          (S6, gate scale fused)
+//
+// Prior art: "Strata PR #4366" (DS4_FAT_ROWS), Approach — a popular expert's
+// weights decoded once, its rows gathered, one FP16 cuBLAS GEMM, then a clamped
+// SwiGLU; "mini-AGI PR #4" run() — experts grouped by load, each group at its
+// own size. Here every expert with rows becomes ceil(rows/128) M-tiles of one
+// grouped launch; rows past an expert's end are computed and masked.
+//
+// Kernel shape (one CTA per SM, persistent over work units):
+//   warp 0   TMA producer: A = 128 rows x 64 K of the gathered rows (2-D map,
+//            128-byte swizzle, K-major), B = 64 K x 256 N of the expert's
+//            weights (3-D map [E, K, N], four 64-wide boxes, N-major). Four
+//            48 KB stages in shared memory, mbarrier full/empty pairs.
+//   warp 1   TMEM allocator + single-thread tcgen05.mma issuer: M=128, N=256,
+//            K=16 per instruction, fp32 accumulators in TMEM, two 256-column
+//            buffers so the epilogue of a unit overlaps the next unit's MMAs.
+//   warps 2-5 epilogue: tcgen05.ld 32 lanes x 32 columns, fused SwiGLU or gate
+//            scaling, bf16 stores. Warp w reads TMEM lanes 32*(w%4)..+31.
+// A work unit is (expert, n-tile, m-tile); units of one expert and n-tile are
+// adjacent so its weight tile is read from HBM once and served from L2 to its
+// other M-tiles. Every mbarrier wait is bounded in time; a wait that gives up
+// raises MOE_DEVERR_TIMEOUT, the CTA drains its copies and MMAs, frees TMEM and
+// returns. No TMA multicast is used.
+#include "internal.h"
+
+namespace moe {
+
+namespace tc {
+
+constexpr int BM = 128, BK = 64, BN = 256, STAGES = 4;
+constexpr int A_BYTES = BM * BK * 2;  // 16 KB
+constexpr int B_CHUNK = 64 * BK * 2;  // one 64(N) x 64(K) box, 8 KB
+constexpr int B_BYTES = 4 * B_CHUNK;  // 32 KB
+constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
+constexpr int TMEM_COLS = 512;
+constexpr int SMEM_BYTES = 1024 + STAGES * STAGE_BYTES + 256;  // + barriers
+
+struct GemmParams {
+    int K;        // reduction length (multiple of 64)
+    int n_out;    // output width
+    int n_tiles;  // output tiles per M-tile
+    int E;        // routed experts; index E is the shared expert
+    int Etot;
+    const int32_t* tile_base;  // [Etot+1] exclusive prefix of M-tiles
+    const int32_t* offsets;    // [Etot+1] row offsets
+    uint16_t* out;             // [rows, n_out] fp16 (h or y)
+    const int32_t* sorted_pair;
+    const float* topk_w;
+    float limit;
+    uint32_t* err;
+    uint64_t wait_ns;
+};
+
+struct Unit {
+    int e, m, n, row0, rows;
+};
+
+MOE_DEV Unit decode_unit(int u, const GemmParams& p) {
+    const int g = u / p.n_tiles;  // global M-tile index
+    int lo = 0, hi = p.Etot;      // tile_base[lo] <= g < tile_base[hi]
+    while (hi - lo > 1) {
+        const int mid = (lo + hi) >> 1;
+        if (__ldg(p.tile_base + mid) <= g) lo = mid;
+        else hi = mid;
+    }
+    Unit U;
+    U.e = lo;
+    const int tb = __ldg(p.tile_base + lo);
+    const int mt = __ldg(p.tile_base + lo + 1) - tb;
+    const int local = u - tb * p.n_tiles;
+    U.n = local / mt;
+    U.m = local - U.n * mt;
+    const int off = __ldg(p.offsets + lo);
+    const int kept = __ldg(p.offsets + lo + 1) - off;
+    U.row0 = off + U.m * BM;
+    U.rows = min(BM, kept - U.m * BM);
+    return U;
+}
+
+MOE_DEV float swiglu(float g, float u, float L) {
+    if (L > 0.f) {
+        g = fminf(fmaxf(g, -L), L);
+        u = fminf(fmaxf(u, -L), L);
+    }
+    return g / (1.0f + expf(-g)) * u;
+}
+
+// Threads: MODE 0 has 6 warps (producer, MMA, 4 epilogue); MODE 1 adds 4
+// converter warps (6..9) that turn each landed W_down tile from bf16 into fp16
+// in place, so the down GEMM runs fp16 x fp16 (h is fp16).
+template <int MODE>
+struct Roles {
+    static constexpr int kThreads = MODE == 0 ? 192 : 320;
+    static constexpr uint32_t kIdesc = idesc_f16_f32(BM, BN, /*ab_bf16=*/MODE == 0 ? 1 : 0, /*a_mn=*/0, /*b_mn=*/1);
+};
+
+template <int MODE>
+__global__ void __launch_bounds__(Roles<MODE>::kThreads, 1)
+    grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB0,
+                        const __grid_constant__ CUtensorMap tmB1, const __grid_constant__ CUtensorMap tmS0,
+                        const __grid_constant__ CUtensorMap tmS1, const GemmParams p) {
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint64_t* full = reinterpret_cast<uint64_t*>(smem + STAGES * STAGE_BYTES);
+    uint64_t* conv = full + STAGES;  // MODE 1: B tile converted to fp16
+    uint64_t* empty = conv + STAGES;
+    uint64_t* tfull = empty + STAGES;
+    uint64_t* tempty = tfull + 2;
+    uint64_t* drain = tempty + 2;
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < STAGES; ++s) {
+            mbar_init(full + s, 1);
+            mbar_init(conv + s, 128);
+            mbar_init(empty + s, 1);
+        }
+        for (int a = 0; a < 2; ++a) {
+            mbar_init(tfull + a, 1);
+            mbar_init(tempty + a, 4);
+        }
+        mbar_init(drain, 1);
+        *abort_flag = 0;
+        fence_mbar_init();
+    }
+    if (warp == 0 && lane == 0) {
+        tma_prefetch_desc(&tmA);
+        tma_prefetch_desc(&tmB0);
+        if (MODE == 0) tma_prefetch_desc(&tmB1);
+    }
+    if (warp == 1) {
+        tmem_alloc(tmem_slot, TMEM_COLS);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem_base = *tmem_slot;
+
+    const int total_units = __ldg(p.tile_base + p.Etot) * p.n_tiles;
+    const int KB = p.K / BK;
+
+    if (warp == 0) {
+        // ------------------------------------------------ TMA producer
+        int stage = 0;
+        uint32_t phase = 0, issued = 0, issued_par = 0;
+        bool ok = true;
+        for (int u = blockIdx.x; ok && u < total_units; u += gridDim.x) {
+            const Unit U = decode_unit(u, p);
+            const bool sh = U.e >= p.E;
+            const int z = sh ? 0 : U.e;
+            for (int kb = 0; kb < KB; ++kb) {
+                int okl = 1;
+                if (lane == 0) okl = mbar_wait_bounded(empty + stage, phase ^ 1u, abort_flag, p.err, p.wait_ns);
+                okl = __shfl_sync(0xFFFFFFFFu, okl, 0);
+                if (!okl) {
+                    ok = false;
+                    break;
+                }
+                if (lane == 0) {
+                    uint8_t* sa = smem + stage * STAGE_BYTES;
+                    uint8_t* sb = sa + A_BYTES;
+                    mbar_arrive_expect_tx(full + stage, STAGE_BYTES);
+                    tma_load_2d(sa, &tmA, full + stage, kb * BK, U.row0);
+                    if (MODE == 0) {
+                        const CUtensorMap* mg = sh ? &tmS0 : &tmB0;
+                        const CUtensorMap* mu = sh ? &tmS1 : &tmB1;
+                        const int n0 = U.n * 128;
+                        tma_load_3d(sb, mg, full + stage, n0, kb * BK, z);
+                        tma_load_3d(sb + B_CHUNK, mg, full + stage, n0 + 64, kb * BK, z);
+                        tma_load_3d(sb + 2 * B_CHUNK, mu, full + stage, n0, kb * BK, z);
+                        tma_load_3d(sb + 3 * B_CHUNK, mu, full + stage, n0 + 64, kb * BK, z);
+                    } else {
+                        const CUtensorMap* md = sh ? &tmS0 : &tmB0;
+                        const int n0 = U.n * BN;
+#pragma unroll
+                        for (int c = 0; c < 4; ++c) tma_load_3d(sb + c * B_CHUNK, md, full + stage, n0 + 64 * c, kb * BK, z);
+                    }
+                    issued |= 1u << stage;
+                    issued_par = (issued_par & ~(1u << stage)) | (phase << stage);
+                }
+                if (++stage == STAGES) {
+                    stage = 0;
+                    phase ^= 1u;
+                }
+            }
+        }
+        // On abort, let every copy already issued land before the CTA can exit.
+        if (!ok && lane == 0) {
+            for (int s = 0; s < STAGES; ++s)
+                if (issued >> s & 1u) mbar_wait_bounded(full + s, (issued_par >> s) & 1u, nullptr, p.err, kDrainLimitNs);
+        }
+        __syncwarp();
+    } else if (warp == 1) {
+        // ------------------------------------------------ MMA issuer
+        constexpr uint32_t IDESC = Roles<MODE>::kIdesc;
+        uint64_t* ready = MODE == 0 ? full : conv;
+        int stage = 0, acc = 0;
+        uint32_t phase = 0, acc_phase = 0;
+        bool ok = true;
+        for (int u = blockIdx.x; ok && u < total_units; u += gridDim.x) {
+            int okl = 1;
+            if (lane == 0) okl = mbar_wait_bounded(tempty + acc, acc_phase ^ 1u, abort_flag, p.err, p.wait_ns);
+            okl = __shfl_sync(0xFFFFFFFFu, okl, 0);
+            if (!okl) break;
+            tc_fence_after();
+            const uint32_t d_tmem = tmem_base + uint32_t(acc * BN);
+            for (int kb = 0; kb < KB; ++kb) {
+                if (lane == 0) okl = mbar_wait_bounded(ready + stage, phase, abort_flag, p.err, p.wait_ns);
+                okl = __shfl_sync(0xFFFFFFFFu, okl, 0);
+                if (!okl) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+                if (lane == 0) {
+                    const uint32_t a0 = smem_u32(smem + stage * STAGE_BYTES);
+                    const uint32_t b0 = a0 + A_BYTES;
+#pragma unroll
+                    for (int j = 0; j < BK / 16; ++j) {
+                        // A: K-major, advance 16 elements = 32 bytes inside the swizzle row.
+                        // B: N-major, advance 16 K-rows = 2 KB (two 8-row groups).
+                        const uint64_t ad = sdesc_sw128(a0 + j * 32, 16, 1024);
+                        const uint64_t bd = sdesc_sw128(b0 + j * 2048, B_CHUNK, 1024);
+                        umma_bf16(d_tmem, ad, bd, IDESC, (kb | j) != 0);
+                    }
+                    umma_commit(empty + stage);
+                }
+                __syncwarp();
+                if (++stage == STAGES) {
+                    stage = 0;
+                    phase ^= 1u;
+                }
+            }
+            if (!ok) break;
+            if (lane == 0) umma_commit(tfull + acc);
+            __syncwarp();
+            if (++acc == 2) {
+                acc = 0;
+                acc_phase ^= 1u;
+            }
+        }
+        // every MMA this thread issued has completed before TMEM is freed
+        if (lane == 0) {
+            umma_commit(drain);
+            mbar_wait_bounded(drain, 0, nullptr, p.err, kDrainLimitNs);
+        }
+        __syncwarp();
+    } else if (warp < 6) {
+        // ------------------------------------------------ epilogue (warps 2..5)
+        const int q = warp & 3;
+        int acc = 0;
+        uint32_t acc_phase = 0;
+        bool range_bad = false;
+        for (int u = blockIdx.x; u < total_units; u += gridDim.x) {
+            const Unit U = decode_unit(u, p);
+            int okl = 1;
+            if (lane == 0) okl = mbar_wait_bounded(tfull + acc, acc_phase, abort_flag, p.err, p.wait_ns);
+            okl = __shfl_sync(0xFFFFFFFFu, okl, 0);
+            if (!okl) break;
+            tc_fence_after();
+            const int rit = q * 32 + lane;
+            const bool valid = rit < U.rows;
+            const int64_t row = int64_t(U.row0) + rit;
+            const uint32_t tb = tmem_base + (uint32_t(q * 32) << 16) + uint32_t(acc * BN);
+            if (MODE == 0) {
+#pragma unroll 1
+                for (int c = 0; c < 4; ++c) {
+                    uint32_t g[32], v[32];
+                    tmem_ld_32x32b_x32(tb + c * 32, g);
+                    tmem_ld_32x32b_x32(tb + 128 + c * 32, v);
+                    tmem_ld_wait();
+                    const int col = U.n * 128 + c * 32;
+                    if (valid && col < p.n_out) {
+                        uint32_t pk[16];
+#pragma unroll
+                        for (int i = 0; i < 16; ++i) {
+                            const float h0 = swiglu(__uint_as_float(g[2 * i]), __uint_as_float(v[2 * i]), p.limit);
+                            const float h1 =
+                                swiglu(__uint_as_float(g[2 * i + 1]), __uint_as_float(v[2 * i + 1]), p.limit);
+                            range_bad |= !(f16_range_ok(h0) && f16_range_ok(h1));
+                            pk[i] = pack_f16x2(h0, h1);
+                        }
+                        uint4* dst = reinterpret_cast<uint4*>(p.out + row * p.n_out + col);
+#pragma unroll
+                        for (int i = 0; i < 4; ++i) dst[i] = make_uint4(pk[4 * i], pk[4 * i + 1], pk[4 * i + 2], pk[4 * i + 3]);
+                    }
+                }
+            } else {
+                float w = 0.f;
+                if (valid) {
+                    const int sp = __ldg(p.sorted_pair + row);
+                    w = sp >= 0 ? __ldg(p.topk_w + sp) : 1.0f;
+                }
+#pragma unroll 1
+                for (int c = 0; c < BN / 32; ++c) {
+                    uint32_t v[32];
+                    tmem_ld_32x32b_x32(tb + c * 32, v);
+                    tmem_ld_wait();
+                    const int col = U.n * BN + c * 32;
+                    if (valid && col < p.n_out) {
+                        uint32_t pk[16];
+#pragma unroll
+                        for (int i = 0; i < 16; ++i) {
+                            const float y0 = w * __uint_as_float(v[2 * i]), y1 = w * __uint_as_float(v[2 * i + 1]);
+                            range_bad |= !(f16_range_ok(y0) && f16_range_ok(y1));
+                            pk[i] = pack_f16x2(y0, y1);
+                        }
+                        uint4* dst = reinterpret_cast<uint4*>(p.out + row * p.n_out + col);
+#pragma unroll
+                        for (int i = 0; i < 4; ++i) dst[i] = make_uint4(pk[4 * i], pk[4 * i + 1], pk[4 * i + 2], pk[4 * i + 3]);
+                    }
+                }
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(tempty + acc);
+            if (++acc == 2) {
+                acc = 0;
+                acc_phase ^= 1u;
+            }
+        }
+        if (range_bad) set_error(p.err, MOE_DEVERR_RANGE);
+    } else if (MODE == 1) {
+        // ------------------------------------------------ converters (warps 6..9): W_down bf16 -> fp16
+        const int ct = threadIdx.x - 192;
+        int stage = 0;
+        uint32_t phase = 0;
+        bool ok = true;
+        for (int u = blockIdx.x; ok && u < total_units; u += gridDim.x) {
+            for (int kb = 0; kb < KB; ++kb) {
+                int okl = 1;
+                if (lane == 0) okl = mbar_wait_bounded(full + stage, phase, abort_flag, p.err, p.wait_ns);
+                okl = __shfl_sync(0xFFFFFFFFu, okl, 0);
+                if (!okl) {
+                    ok = false;
+                    break;
+                }
+                uint4* b = reinterpret_cast<uint4*>(smem + stage * STAGE_BYTES + A_BYTES);
+#pragma unroll 4
+                for (int i = ct; i < B_BYTES / 16; i += 128) {
+                    uint4 v = b[i];
+                    v.x = bf16x2_to_f16x2(v.x);
+                    v.y = bf16x2_to_f16x2(v.y);
+                    v.z = bf16x2_to_f16x2(v.z);
+                    v.w = bf16x2_to_f16x2(v.w);
+                    b[i] = v;
+                }
+                fence_proxy_async_smem();  // generic-proxy writes -> visible to the tensor core
+                mbar_arrive(conv + stage);
+                if (++stage == STAGES) {
+                    stage = 0;
+                    phase ^= 1u;
+                }
+            }
+        }
+    }
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc(tmem_base, TMEM_COLS);
+    }
+}
+
+}  // namespace tc
+
+// ---------------------------------------------------------------------------- K3 schedule
+
+// One block of 512 threads; thread e owns expert e (Etot <= 257).
+__global__ void __launch_bounds__(512) schedule_kernel(const int32_t* __restrict__ offsets, int Etot, int variant,
+                                                       int stream_max, int32_t* __restrict__ tile_base,
+                                                       int32_t* __restrict__ stream_list,
+                                                       int32_t* __restrict__ n_stream, uint32_t* err) {
+    __shared__ int sums[2][16];
+    const int e = threadIdx.x, lane = e & 31, w = e >> 5;
+    int kept = 0;
+    if (e < Etot) {
+        kept = offsets[e + 1] - offsets[e];
+        if (kept < 0) {
+            set_error(err, MOE_DEVERR_BOUNDS);
+            kept = 0;
+        }
+    }
+    const int is_stream =
+        (kept > 0 && (variant == MOE_VARIANT_STREAM || (variant == MOE_VARIANT_AUTO && kept <= stream_max))) ? 1 : 0;
+    const int tiles = (kept > 0 && !is_stream) ? (kept + kTileM - 1) / kTileM : 0;
+    int it = tiles, is = is_stream;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+        const int a = __shfl_up_sync(0xFFFFFFFFu, it, off);
+        const int b = __shfl_up_sync(0xFFFFFFFFu, is, off);
+        if (lane >= off) {
+            it += a;
+            is += b;
+        }
+    }
+    if (lane == 31) {
+        sums[0][w] = it;
+        sums[1][w] = is;
+    }
+    __syncthreads();
+    int bt = 0, bs = 0, tt = 0, ts = 0;
+    for (int i = 0; i < 16; ++i) {
+        if (i < w) {
+            bt += sums[0][i];
+            bs += sums[1][i];
+        }
+        tt += sums[0][i];
+        ts += sums[1][i];
+    }
+    if (e < Etot) tile_base[e] = bt + it - tiles;
+    if (is_stream) stream_list[bs + is - 1] = e;
+    if (e == 0) {
+        tile_base[Etot] = tt;
+        n_stream[0] = ts;
+    }
+}
+
+// ---------------------------------------------------------------------------- S4 row gather
+
+// xg[r] = x[sorted_token[r]] for r < offsets[Etot]; 16-byte vectors.
+__global__ void __launch_bounds__(256) gather_rows_kernel(const uint16_t* __restrict__ x,
+                                                          const int32_t* __restrict__ sorted_token,
+                                                          const int32_t* __restrict__ offsets, int Etot, int d,
+                                                          int T, uint16_t* __restrict__ xg, uint32_t* err) {
+    const int vec = d / 8;
+    const int64_t total = int64_t(offsets[Etot]) * vec;
+    for (int64_t i = int64_t(blockIdx.x) * blockDim.x + threadIdx.x; i < total; i += int64_t(gridDim.x) * blockDim.x) {
+        const int64_t r = i / vec;
+        const int c = int(i - r * vec);
+        const int t = __ldg(sorted_token + r);
+        if (t < 0 || t >= T) {
+            set_error(err, MOE_DEVERR_BOUNDS);
+            continue;
+        }
+        reinterpret_cast<uint4*>(xg + r * d)[c] = __ldg(reinterpret_cast<const uint4*>(x + int64_t(t) * d) + c);
+    }
+}
+
+// ---------------------------------------------------------------------------- host side
+
+namespace tc {
+
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+static EncodeTiledFn get_encode() {
+    static EncodeTiledFn fn = nullptr;
+    if (!fn) {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &p, 12000, cudaEnableDefault, &q) ==
+                cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(p);
+    }
+    return fn;
+}
+
+// bf16 tensor map; dims/strides innermost first; box {64, box1, 1...}; 128-byte swizzle.
+static bool make_map(CUtensorMap* m, const void* base, int rank, const uint64_t* dims, const uint64_t* strides_bytes,
+                     const uint32_t* box) {
+    EncodeTiledFn enc = get_encode();
+    if (!enc) return false;
+    cuuint64_t gd[3], gs[2];
+    cuuint32_t bx[3], es[3] = {1, 1, 1};
+    for (int i = 0; i < rank; ++i) {
+        gd[i] = dims[i];
+        bx[i] = box[i];
+    }
+    for (int i = 0; i < rank - 1; ++i) gs[i] = strides_bytes[i];
+    const CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, rank, const_cast<void*>(base), gd, gs, bx, es,
+                           CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                           CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
+// A operand: rows x K bf16 row-major; box 64 (K) x 128 (rows).
+bool map_rows(CUtensorMap* m, const void* base, int64_t rows, int K) {
+    const uint64_t dims[2] = {uint64_t(K), uint64_t(rows)};
+    const uint64_t str[1] = {uint64_t(K) * 2};
+    const uint32_t box[2] = {64, 128};
+    return make_map(m, base, 2, dims, str, box);
+}
+// B operand: [nexp, K, N] bf16 row-major; box 64 (N) x 64 (K) x 1.
+bool map_weights(CUtensorMap* m, const void* base, int nexp, int K, int N) {
+    const uint64_t dims[3] = {uint64_t(N), uint64_t(K), uint64_t(nexp)};
+    const uint64_t str[2] = {uint64_t(N) * 2, uint64_t(N) * uint64_t(K) * 2};
+    const uint32_t box[3] = {64, 64, 1};
+    return make_map(m, base, 3, dims, str, box);
+}
+
+template <int MODE>
+cudaError_t launch_gemm(const CUtensorMap& A, const CUtensorMap& B0, const CUtensorMap& B1, const CUtensorMap& S0,
+                        const CUtensorMap& S1, const GemmParams& p, cudaStream_t s) {
+    static int configured_dev = -1;
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (configured_dev != dev) {
+        cudaError_t e = cudaFuncSetAttribute(grouped_gemm_kernel<MODE>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             SMEM_BYTES);
+        if (e != cudaSuccess) return e;
+        configured_dev = dev;
+    }
+    {
+        ProfScope prof_(MODE == 0 ? MOE_K_TC_GATEUP : MOE_K_TC_DOWN, s);
+        grouped_gemm_kernel<MODE><<<num_sms(), Roles<MODE>::kThreads, SMEM_BYTES, s>>>(A, B0, B1, S0, S1, p);
+    }
+    return cudaGetLastError();
+}
+
+}  // namespace tc
+
+cudaError_t launch_schedule(const Dims& D, const int32_t* offsets, int32_t* tile_base, int32_t* stream_list,
+                            int32_t* n_stream, uint32_t* err, cudaStream_t s) {
+    int smax = D.stream_max_rows;
+    {
+        ProfScope prof_(MOE_K_SCHEDULE, s);
+        schedule_kernel<<<1, 512, 0, s>>>(offsets, D.Etot, D.variant, smax, tile_base, stream_list, n_stream, err);
+    }
+    return cudaGetLastError();
+}
+
+cudaError_t launch_gather(const Dims& D, const uint16_t* x, const int32_t* sorted_token, const int32_t* offsets,
+                          uint16_t* xg, uint32_t* err, cudaStream_t s) {
+    const int64_t total = D.rows * (D.d / 8);
+    int64_t blocks = (total + 255) / 256;
+    const int64_t cap = int64_t(num_sms()) * 8;
+    if (blocks > cap) blocks = cap;
+    if (blocks < 1) blocks = 1;
+    {
+        ProfScope prof_(MOE_K_GATHER, s);
+        gather_rows_kernel<<<int(blocks), 256, 0, s>>>(x, sorted_token, offsets, D.Etot, D.d, D.T, xg, err);
+    }
+    return cudaGetLastError();
+}
+
+// Both tcgen05 GEMMs of the tile variant. h: [rows, f] bf16 scratch.
+cudaError_t launch_tensor_ffn(const Dims& D, const uint16_t* xg, uint16_t* h, const int32_t* tile_base,
+                              const int32_t* offsets, const int32_t* sorted_pair, const float* topk_w,
+                              const moe_weights* w, uint16_t* y_rows, uint32_t* err, uint64_t wait_ns,
+                              cudaStream_t s) {
+    using namespace tc;
+    CUtensorMap mA, mG, mU, mSG, mSU, mH, mD, mSD;
+    if (!map_rows(&mA, xg, D.rows, D.d) || !map_weights(&mG, w->w_gate, D.E, D.d, D.f) ||
+        !map_weights(&mU, w->w_up, D.E, D.d, D.f) || !map_rows(&mH, h, D.rows, D.f) ||
+        !map_weights(&mD, w->w_down, D.E, D.f, D.d))
+        return cudaErrorInvalidValue;
+    if (D.has_shared) {
+        if (!map_weights(&mSG, w->shared_gate, 1, D.d, D.f) || !map_weights(&mSU, w->shared_up, 1, D.d, D.f) ||
+            !map_weights(&mSD, w->shared_down, 1, D.f, D.d))
+            return cudaErrorInvalidValue;
+    } else {
+        mSG = mG;
+        mSU = mU;
+        mSD = mD;
+    }
+    GemmParams p{};
+    p.E = D.E;
+    p.Etot = D.Etot;
+    p.tile_base = tile_base;
+    p.offsets = offsets;
+    p.sorted_pair = sorted_pair;
+    p.topk_w = topk_w;
+    p.limit = D.limit;
+    p.err = err;
+    p.wait_ns = wait_ns;
+    // S5: gate/up + SwiGLU -> h
+    p.K = D.d;
+    p.n_out = D.f;
+    p.n_tiles = (D.f + 127) / 128;
+    p.out = h;
+    cudaError_t e = launch_gemm<0>(mA, mG, mU, mSG, mSU, p, s);
+    if (e != cudaSuccess) return e;
+    // S6: down + gate scale -> y_rows
+    p.K = D.f;
+    p.n_out = D.d;
+    p.n_tiles = (D.d + BN - 1) / BN;
+    p.out = y_rows;
+    return launch_gemm<1>(mH, mD, mD, mSD, mSD, p, s);
+}
+
+}  // namespace moe

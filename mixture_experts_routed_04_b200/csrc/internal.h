@@ -1,0 +1,85 @@
+// internal.h — launchers and workspace layout shared by the kernel files and the C ABI.
+#pragma once
+
+#include "common.cuh"
+
+namespace moe {
+
+constexpr int kMaxE = 256;
+constexpr int kMaxK = 8;
+constexpr int kPermWarps = 8;                         // warps per permutation block
+constexpr int kPermPairsPerWarp = 256;                // 8 rounds of 32 pairs
+constexpr int kPermPairsPerBlock = kPermWarps * kPermPairsPerWarp;
+constexpr int kTileM = 128;                           // rows per tcgen05 tile
+constexpr int kDefaultStreamMaxRows = 16;             // AUTO threshold (rows per expert)
+
+// Everything a call derives from moe_params on the host.
+struct Dims {
+    int T, d, f, E, k, Etot;  // Etot = E + has_shared
+    int has_shared;
+    int cap;                  // -1: no cap
+    int64_t rows;             // rows of the permuted buffers
+    int64_t pairs;            // T * k
+    int perm_blocks;          // blocks of the permutation kernels
+    int fmt, variant, stream_max_rows;
+    float limit;
+    int ks;                   // K-split of the streaming gate/up kernel
+    int out_bf16;             // layer output in bf16 (else fp32)
+};
+
+// Byte offsets of every scratch array inside a workspace (0 = absent).
+struct WsLayout {
+    size_t err;                                    // uint32 error word (always at 0)
+    size_t blockcounts, blockbase;                 // permute: int32 [perm_blocks, E]
+    size_t tile_base, stream_list, n_stream;       // expert_ffn schedule
+    size_t xg, h, part;                            // expert_ffn: gathered x, h, split-K partials
+    size_t topk_idx, topk_w, counts, kept, offsets, sorted_token, sorted_pair, pair_row, y_rows;  // forward
+    size_t x_dev, logits_dev, out_dev;             // forward_host
+    size_t total;
+};
+
+WsLayout ws_layout(const Dims& D, int which);
+
+// ---- launchers (all asynchronous on `s`)
+cudaError_t launch_route(const float* logits, int T, int E, int k, int32_t* topk_idx, float* topk_w,
+                         cudaStream_t s);
+
+cudaError_t launch_permute(const Dims& D, const int32_t* topk_idx, int32_t* blockcounts, int32_t* blockbase,
+                           int32_t* counts, int32_t* kept, int32_t* offsets, int32_t* sorted_token,
+                           int32_t* sorted_pair, int32_t* pair_row, uint32_t* err, cudaStream_t s);
+
+struct FfnArgs {
+    const uint16_t* x;
+    const int32_t* offsets;
+    const int32_t* sorted_token;
+    const int32_t* sorted_pair;
+    const float* topk_w;
+    const moe_weights* w;
+    uint16_t* y_rows;
+    uint8_t* ws;
+    uint32_t* err;
+    uint64_t wait_ns;
+};
+cudaError_t launch_expert_ffn(const Dims& D, const WsLayout& L, const FfnArgs& a, cudaStream_t s);
+
+cudaError_t launch_combine(const Dims& D, const uint16_t* y_rows, const int32_t* pair_row, const int32_t* offsets,
+                           void* out, cudaStream_t s);
+
+// ---- device properties, cached per device
+int num_sms();
+
+// ---- optional per-kernel event timing (moe_profile_enable); no-op when off
+class ProfScope {
+  public:
+    ProfScope(int kernel_id, cudaStream_t s);
+    ~ProfScope();
+    ProfScope(const ProfScope&) = delete;
+    ProfScope& operator=(const ProfScope&) = delete;
+
+  private:
+    int id_;
+    cudaStream_t s_;
+    void* a_;
+};
+
+}  // namespace moe

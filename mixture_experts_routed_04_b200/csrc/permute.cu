@@ -1,0 +1,201 @@
+// permute.cu — S2/S3: per-expert histogram, prefix offsets, scatter and the
+// capacity drop, with no atomics.
+//
+// "mini-AGI PR #3", minagi/pool.py requested(): the (token, expert) pairs are
+// flattened, sorted by expert and counted (bincount); with a capacity, a keep
+// mask over each expert's sorted pairs drops the overflow and the counts are
+// clamped. Here the pairs keep token order inside each expert (pair p = t*k+j
+// ranks before p' > p), and the first `cap` of an expert are kept.
+//
+// Three launches over the T*k pairs, which are cut into blocks of 2048 pairs,
+// 256 per warp in 8 rounds of 32:
+//   count   — each warp counts its pairs per expert (__match_any_sync groups
+//             equal ids in a round; the group's lowest lane adds the popcount
+//             to the warp's own smem row, so no two lanes write one counter),
+//             and the block writes its per-expert totals.
+//   scan    — one block: per expert an exclusive scan over blocks gives each
+//             block its base; counts, kept = min(count, cap), and an exclusive
+//             scan over experts gives offsets.
+//   scatter — each block rebuilds its warp totals, turns them into warp bases,
+//             and ranks every pair: base + earlier peers in its round. Rank <
+//             cap → row offsets[e] + rank.
+// The rank of a pair is the number of earlier pairs with the same expert, so
+// the result is unique and bit-exact. The shared expert, when present, is
+// appended as expert E holding tokens 0..T-1.
+#include "internal.h"
+
+namespace moe {
+
+namespace {
+
+MOE_DEV uint32_t lanemask_lt() {
+    uint32_t m;
+    asm("mov.u32 %0, %%lanemask_lt;" : "=r"(m));
+    return m;
+}
+
+// Fill hist[w][e] with warp w's pair count per expert for block `b`.
+MOE_DEV void warp_histograms(const int32_t* __restrict__ topk_idx, int64_t pairs, int E, int (*hist)[kMaxE],
+                             uint32_t* err) {
+    const int w = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    for (int i = threadIdx.x; i < kPermWarps * kMaxE; i += blockDim.x) (&hist[0][0])[i] = 0;
+    __syncthreads();
+    const int64_t base = int64_t(blockIdx.x) * kPermPairsPerBlock + int64_t(w) * kPermPairsPerWarp;
+    for (int it = 0; it < kPermPairsPerWarp / 32; ++it) {
+        const int64_t p = base + it * 32 + lane;
+        int e = -1;
+        if (p < pairs) {
+            e = topk_idx[p];
+            if (e < 0 || e >= E) {
+                set_error(err, MOE_DEVERR_BOUNDS);
+                e = -1;
+            }
+        }
+        const uint32_t peers = __match_any_sync(0xFFFFFFFFu, e);
+        if (e >= 0 && (__ffs(peers) - 1) == lane) hist[w][e] += __popc(peers);
+        __syncwarp();
+    }
+    __syncthreads();
+}
+
+__global__ void __launch_bounds__(kPermWarps * 32) perm_count_kernel(const int32_t* __restrict__ topk_idx,
+                                                                     int64_t pairs, int E,
+                                                                     int32_t* __restrict__ blockcounts,
+                                                                     uint32_t* err) {
+    __shared__ int hist[kPermWarps][kMaxE];
+    warp_histograms(topk_idx, pairs, E, hist, err);
+    for (int e = threadIdx.x; e < E; e += blockDim.x) {
+        int s = 0;
+#pragma unroll
+        for (int w = 0; w < kPermWarps; ++w) s += hist[w][e];
+        blockcounts[int64_t(blockIdx.x) * E + e] = s;
+    }
+}
+
+// One block of 256 threads: thread e owns expert e.
+__global__ void __launch_bounds__(kMaxE) perm_scan_kernel(const int32_t* __restrict__ blockcounts, int nblocks,
+                                                         int E, int cap, int shared_T,
+                                                         int32_t* __restrict__ blockbase,
+                                                         int32_t* __restrict__ counts, int32_t* __restrict__ kept,
+                                                         int32_t* __restrict__ offsets) {
+    __shared__ int warp_sums[kMaxE / 32];
+    const int e = threadIdx.x, lane = e & 31, w = e >> 5;
+    int kv = 0;
+    if (e < E) {
+        int run = 0;
+        for (int b = 0; b < nblocks; ++b) {
+            const int c = blockcounts[int64_t(b) * E + e];
+            blockbase[int64_t(b) * E + e] = run;
+            run += c;
+        }
+        counts[e] = run;
+        kv = (cap >= 0 && run > cap) ? cap : run;
+        kept[e] = kv;
+    }
+    // exclusive scan of kv over the block
+    int incl = kv;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+        const int v = __shfl_up_sync(0xFFFFFFFFu, incl, off);
+        if (lane >= off) incl += v;
+    }
+    if (lane == 31) warp_sums[w] = incl;
+    __syncthreads();
+    int wbase = 0, total = 0;
+#pragma unroll
+    for (int i = 0; i < kMaxE / 32; ++i) {
+        if (i < w) wbase += warp_sums[i];
+        total += warp_sums[i];
+    }
+    if (e < E) offsets[e] = wbase + incl - kv;
+    if (e == 0) {
+        if (shared_T > 0) {
+            counts[E] = shared_T;
+            kept[E] = shared_T;
+            offsets[E] = total;
+            offsets[E + 1] = total + shared_T;
+        } else {
+            offsets[E] = total;
+        }
+    }
+}
+
+__global__ void __launch_bounds__(kPermWarps * 32) perm_scatter_kernel(
+    const int32_t* __restrict__ topk_idx, int64_t pairs, int k, int E, int cap,
+    const int32_t* __restrict__ blockbase, const int32_t* __restrict__ offsets,
+    int32_t* __restrict__ sorted_token, int32_t* __restrict__ sorted_pair, int32_t* __restrict__ pair_row,
+    int shared_T, uint32_t* err) {
+    __shared__ int hist[kPermWarps][kMaxE];
+    warp_histograms(topk_idx, pairs, E, hist, nullptr);  // errors were reported by the count pass
+    // warp totals -> warp bases (block base + earlier warps), per expert
+    for (int e = threadIdx.x; e < E; e += blockDim.x) {
+        int run = blockbase[int64_t(blockIdx.x) * E + e];
+#pragma unroll
+        for (int w = 0; w < kPermWarps; ++w) {
+            const int c = hist[w][e];
+            hist[w][e] = run;
+            run += c;
+        }
+    }
+    __syncthreads();
+    const int w = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int64_t base = int64_t(blockIdx.x) * kPermPairsPerBlock + int64_t(w) * kPermPairsPerWarp;
+    for (int it = 0; it < kPermPairsPerWarp / 32; ++it) {
+        const int64_t p = base + it * 32 + lane;
+        int e = -1;
+        if (p < pairs) {
+            e = topk_idx[p];
+            if (e < 0 || e >= E) e = -1;
+        }
+        const uint32_t peers = __match_any_sync(0xFFFFFFFFu, e);
+        int rank = 0;
+        if (e >= 0) rank = hist[w][e] + __popc(peers & lanemask_lt());
+        __syncwarp();
+        if (e >= 0 && (__ffs(peers) - 1) == lane) hist[w][e] += __popc(peers);
+        __syncwarp();
+        if (p < pairs) {
+            if (e >= 0 && (cap < 0 || rank < cap)) {
+                const int row = offsets[e] + rank;
+                sorted_token[row] = int32_t(p / k);
+                sorted_pair[row] = int32_t(p);
+                pair_row[p] = row;
+            } else {
+                pair_row[p] = -1;
+            }
+        }
+    }
+    // shared-expert rows: tokens 0..T-1 after the routed rows
+    if (shared_T > 0) {
+        const int base_row = offsets[E];
+        for (int64_t t = int64_t(blockIdx.x) * blockDim.x + threadIdx.x; t < shared_T;
+             t += int64_t(gridDim.x) * blockDim.x) {
+            sorted_token[base_row + t] = int32_t(t);
+            sorted_pair[base_row + t] = -1;
+        }
+    }
+}
+
+}  // namespace
+
+cudaError_t launch_permute(const Dims& D, const int32_t* topk_idx, int32_t* blockcounts, int32_t* blockbase,
+                           int32_t* counts, int32_t* kept, int32_t* offsets, int32_t* sorted_token,
+                           int32_t* sorted_pair, int32_t* pair_row, uint32_t* err, cudaStream_t s) {
+    const int nb = D.perm_blocks;
+    const int shared_T = D.has_shared ? D.T : 0;
+    {
+        ProfScope prof_(MOE_K_PERM_COUNT, s);
+        perm_count_kernel<<<nb, kPermWarps * 32, 0, s>>>(topk_idx, D.pairs, D.E, blockcounts, err);
+    }
+    {
+        ProfScope prof_(MOE_K_PERM_SCAN, s);
+        perm_scan_kernel<<<1, kMaxE, 0, s>>>(blockcounts, nb, D.E, D.cap, shared_T, blockbase, counts, kept, offsets);
+    }
+    {
+        ProfScope prof_(MOE_K_PERM_SCATTER, s);
+        perm_scatter_kernel<<<nb, kPermWarps * 32, 0, s>>>(topk_idx, D.pairs, D.k, D.E, D.cap, blockbase, offsets,
+                                                       sorted_token, sorted_pair, pair_row, shared_T, err);
+    }
+    return cudaGetLastError();
+}
+
+}  // namespace moe

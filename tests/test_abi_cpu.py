@@ -1,0 +1,93 @@
+"""The C-ABI library without a GPU: it builds for sm_100a, loads, exports every
+declared entry point, and its host-side logic (parameter checks, capacity,
+buffer sizes) behaves as documented. No compute call is made here."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import oracle
+from mixture_experts_routed_04_b200 import binding as b
+from mixture_experts_routed_04_b200.build import build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    build()
+    return b.lib()
+
+
+def _declared():
+    with open(os.path.join(ROOT, "include", "moe.h")) as fh:
+        return set(re.findall(r"MOE_API\s+[\w\s\*]+?\b(moe_\w+)\s*\(", fh.read()))
+
+
+def test_exports_every_declared_symbol(lib):
+    declared = _declared()
+    assert len(declared) >= 14
+    assert declared == set(b.EXPORTS)
+    for name in declared:
+        assert hasattr(lib, name), name
+    assert lib.moe_version() >= 100
+
+
+def test_status_strings(lib):
+    for code, text in b.STATUS.items():
+        assert lib.moe_status_string(code).decode() == text
+
+
+def test_capacity_matches_oracle_rule(lib):
+    with open(os.path.join(ROOT, "tests", "golden", "capacity_cases.txt")) as fh:
+        rows = [ln.split() for ln in fh if ln.strip() and not ln.startswith("#")]
+    for T, k, E, cf, _ in rows:
+        T, k, E, cf = int(T), int(k), int(E), float(cf)
+        p = b.params(T, 64, 64, E, k, capacity_factor=cf)
+        assert b.capacity(p) == oracle.capacity(T, k, E, cf)
+
+
+def test_max_rows_and_workspace(lib):
+    p = b.params(4096, 2048, 768, 128, 8)
+    assert b.max_rows(p) == 4096 * 8
+    capped = b.params(8192, 1024, 2048, 128, 2, capacity_factor=1.5)
+    assert b.max_rows(capped) == min(8192 * 2, 128 * 192)
+    shared = b.params(32, 4096, 1536, 256, 8, has_shared=1, d_ff_shared=1536)
+    assert b.max_rows(shared) == 32 * 8 + 32
+    for which in range(6):
+        assert b.workspace_size(p, which) >= 256
+    assert b.workspace_size(p, b.WS_FORWARD) > b.workspace_size(p, b.WS_EXPERT_FFN)
+
+
+@pytest.mark.parametrize("bad", [
+    dict(k=9), dict(k=3, E=2), dict(E=257), dict(d_model=100), dict(d_ff=32), dict(T=0),
+    dict(capacity_factor=-1.0), dict(capacity_factor=float("nan")), dict(variant=7), dict(weight_format=5)])
+def test_invalid_params_rejected_on_host(lib, bad):
+    kw = dict(T=16, d_model=128, d_ff=256, E=8, k=2)
+    kw.update(bad)
+    p = b.params(**kw)
+    assert b.workspace_size(p, b.WS_FORWARD) == 0
+    st = lib.moe_route(ctypes.byref(p), None, None, None, None, 0, None)
+    assert st == 1  # MOE_ERR_INVALID_ARG, before any launch
+
+
+def test_unsupported_and_missing_buffers(lib):
+    p = b.params(8, 128, 256, 8, 2, has_shared=1, d_ff_shared=128)
+    assert lib.moe_route(ctypes.byref(p), None, None, None, None, 0, None) == 3  # UNSUPPORTED
+    ok = b.params(8, 128, 256, 8, 2)
+    # null workspace / buffers: rejected before any CUDA call
+    assert lib.moe_route(ctypes.byref(ok), None, None, None, None, 0, None) == 1
+    assert lib.moe_forward(ctypes.byref(ok), None, None, None, None, None, None, 0, None) == 1
+
+
+def test_product_path_never_touches_the_oracle():
+    pkg = os.path.join(ROOT, "mixture_experts_routed_04_b200")
+    for dirpath, _, files in os.walk(pkg):
+        for fn in files:
+            if fn.endswith((".py", ".cu", ".cuh", ".h", ".cpp")):
+                with open(os.path.join(dirpath, fn)) as fh:
+                    src = fh.read()
+                assert not re.search(r"\boracle\b", src), fn
+    with open(os.path.join(ROOT, "oracle", "__init__.py")) as fh:
+        assert "mixture_experts_routed_04_b200" not in fh.read()
