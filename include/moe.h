@@ -113,12 +113,14 @@ typedef struct moe_params {
  * Expert weights (device pointers).
  *   BF16:  w_gate, w_up [E, d, f]; w_down [E, f, d]; row-major bf16; s_* NULL.
  *   Q4G32 (self-defined): a matrix of reduction length K and output width N
- *          is stored K-major as packed bytes [N, K/2] (byte j of row n holds
- *          k = 2j in its low nibble, k = 2j+1 in its high nibble; nibble
- *          u = q + 8, q in [-7, 7]) and fp16 scales [N, K/32], one per group of
- *          32 consecutive k; the weight is q * s.
- *          w_gate, w_up: [E, f, d/2] bytes, s_gate, s_up: [E, f, d/32] fp16;
- *          w_down: [E, d, f/2] bytes, s_down: [E, d, f/32] fp16.
+ *          is stored K-major as packed bytes [N, K/2]: each row is K/8
+ *          little-endian 32-bit words; word i holds k = 8i..8i+7, nibble
+ *          position p (bits 4p..4p+3) holding k = 8i + {0,2,4,6,1,3,5,7}[p];
+ *          each nibble u = q + 8, q in [-7, 7]. Scales are fp16, group-major
+ *          [K/32, N]: one per group of 32 consecutive k of a column. The
+ *          weight is q * s.
+ *          w_gate, w_up: [E, f, d/2] bytes, s_gate, s_up: [E, d/32, f] fp16;
+ *          w_down: [E, d, f/2] bytes, s_down: [E, f/32, d] fp16.
  *   shared_*: bf16 [d, f], [d, f], [f, d] of the shared expert; NULL if has_shared = 0.
  */
 typedef struct moe_weights {

@@ -175,18 +175,22 @@ def expert_ffn(x_rows, w_gate, w_up, w_down, limit: float):
 def dequant_q4g32(packed: np.ndarray, scales: np.ndarray) -> np.ndarray:
     """Q4G32 (self-defined) → float64 [K, N]: w[k, n] = q * s exactly.
 
-    packed uint8 [N, K/2]: byte j of row n holds k=2j (low nibble) and k=2j+1
-    (high nibble), each nibble u = q + 8. scales fp16 [N, K/32]: one scale per
-    group of 32 consecutive k.
+    packed uint8 [N, K/2]: each row is K/8 little-endian 32-bit words; word i
+    holds k = 8i..8i+7, nibble position p (bits 4p..4p+3) holding
+    k = 8i + (0, 2, 4, 6, 1, 3, 5, 7)[p]; each nibble u = q + 8.
+    scales fp16 [K/32, N]: one scale per group of 32 consecutive k of a column.
     """
     packed = np.asarray(packed, dtype=np.uint8)
     N, K2 = packed.shape
     K = 2 * K2
-    q = np.empty((N, K), np.float64)
-    q[:, 0::2] = (packed & 0x0F).astype(np.float64) - 8.0
-    q[:, 1::2] = (packed >> 4).astype(np.float64) - 8.0
-    s = np.repeat(np.asarray(scales, dtype=np.float16).astype(np.float64), 32, axis=1)
-    return (q * s).T.copy()
+    words = packed.reshape(N, K // 8, 4).astype(np.uint32)
+    words = words[:, :, 0] | (words[:, :, 1] << 8) | (words[:, :, 2] << 16) | (words[:, :, 3] << 24)
+    q = np.empty((N, K // 8, 8), np.float64)
+    for p, kk in enumerate((0, 2, 4, 6, 1, 3, 5, 7)):
+        q[:, :, kk] = ((words >> (4 * p)) & 0xF).astype(np.float64) - 8.0
+    q = q.reshape(N, K)
+    s = np.repeat(np.asarray(scales, dtype=np.float16).astype(np.float64), 32, axis=0)  # [K, N]
+    return q.T * s
 
 
 # --------------------------------------------------------------------------- combine

@@ -180,15 +180,29 @@ def all_expert_weight_bits(cfg: LayerConfig, which: str, threads: int = 8) -> np
 # --------------------------------------------------------------------------- Q4G32 weights
 #
 # Self-defined format. A matrix with reduction dim K and output dim N is stored
-# K-major: packed bytes [N, K/2] where byte j of row n holds k=2j in its low
-# nibble and k=2j+1 in its high nibble, each nibble u = q + 8 with q in [-7, 7];
-# scales [N, K/32] fp16, one per group of 32 consecutive k. The weight is q * s.
+# K-major: packed bytes [N, K/2]. Each row is K/8 little-endian 32-bit words;
+# word i holds k = 8i..8i+7, nibble position p (bits 4p..4p+3) holding
+# k = 8i + (0, 2, 4, 6, 1, 3, 5, 7)[p]: the pair (k, k+1) sits 16 bits apart,
+# which lets a kernel turn one masked word into two fp16 values at once. Each
+# nibble u = q + 8 with q in [-7, 7]. Scales are fp16, group-major [K/32, N]:
+# one per group of 32 consecutive k of each column. The weight is q * s.
 
 Q4_GROUP = 32
+Q4_NIBBLE_K = (0, 2, 4, 6, 1, 3, 5, 7)  # k offset (within a word) of nibble position p
+
+
+def pack_q4_rows(u: np.ndarray) -> np.ndarray:
+    """Pack nibbles u [N, K] (values 0..15) into bytes [N, K/2] in the word order above."""
+    N, K = u.shape
+    u = u.astype(np.uint32).reshape(N, K // 8, 8)
+    words = np.zeros((N, K // 8), np.uint32)
+    for p, kk in enumerate(Q4_NIBBLE_K):
+        words |= u[:, :, kk] << np.uint32(4 * p)
+    return words.astype("<u4").view(np.uint8).reshape(N, K // 2)
 
 
 def quantize_q4g32(w_kn: np.ndarray):
-    """Quantise an fp32 [K, N] matrix to (packed uint8 [N, K/2], scales fp16 [N, K/32]).
+    """Quantise an fp32 [K, N] matrix to (packed uint8 [N, K/2], scales fp16 [K/32, N]).
 
     Per group: s = fp16(max|w| / 7) (1.0 if the group is all zero);
     q = clip(rint(w / s), -7, 7) with the fp16-rounded s.
@@ -202,9 +216,8 @@ def quantize_q4g32(w_kn: np.ndarray):
     s16[s16 == 0] = np.float16(1.0)
     q = np.rint(g / s16.astype(np.float32)[:, :, None])
     q = np.clip(q, -7, 7).astype(np.int8).reshape(N, K)
-    u = (q + 8).astype(np.uint8)
-    packed = (u[:, 0::2] | (u[:, 1::2] << 4)).astype(np.uint8)
-    return packed, s16
+    packed = pack_q4_rows((q + 8).astype(np.uint8))
+    return packed, np.ascontiguousarray(s16.T)
 
 
 def expert_q4_weights(cfg: LayerConfig, e: int, which: str):
@@ -218,7 +231,7 @@ def expert_q4_weights(cfg: LayerConfig, e: int, which: str):
 def all_expert_q4_weights(cfg: LayerConfig, which: str, threads: int = 8):
     K, N = (cfg.d, cfg.f) if which in ("gate", "up") else (cfg.f, cfg.d)
     packed = np.empty((cfg.E, N, K // 2), np.uint8)
-    scales = np.empty((cfg.E, N, K // Q4_GROUP), np.float16)
+    scales = np.empty((cfg.E, K // Q4_GROUP, N), np.float16)
 
     def one(e):
         packed[e], scales[e] = expert_q4_weights(cfg, e, which)

@@ -303,11 +303,11 @@ def test_token_outputs_match_forward():
 # --------------------------------------------------------------------------- Q4G32
 
 def test_q4g32_golden_bytes():
-    packed = np.full((2, 16), 0x88, np.uint8)
-    packed[0, 0], packed[0, 1], packed[1, 0] = 0x9F, 0x18, 0x2E
-    scales = np.array([[0.5], [0.25]], np.float16)
-    w = oracle.dequant_q4g32(packed, scales)  # [K=32, N=2]
-    want = np.zeros((32, 2))
+    packed = np.full((2, 32), 0x88, np.uint8)  # N=2 rows, K=64
+    packed[0, 0], packed[0, 2], packed[0, 6], packed[0, 16], packed[1, 0] = 0x9F, 0x18, 0x8C, 0xB7, 0x2E
+    scales = np.array([[0.5, 0.25], [2.0, 1.0]], np.float16)  # [K/32, N]
+    w = oracle.dequant_q4g32(packed, scales)  # [K=64, N=2]
+    want = np.zeros((64, 2))
     for ln in _lines("q4g32_bytes.txt"):
         n, k, v = ln.split()
         want[int(k), int(n)] = float(v)
@@ -321,11 +321,11 @@ def test_q4g32_round_trip_and_error_bound():
     q[0::32, :] = 7
     w = q * 0.25
     packed, s = synth.quantize_q4g32(w.astype(np.float32))
-    assert (s == np.float16(0.25)).all()
+    assert s.shape == (2, 6) and (s == np.float16(0.25)).all()
     assert (oracle.dequant_q4g32(packed, s) == w).all()
     # general case: error at most half a step (plus the fp16 rounding of the scale)
     w = rng.standard_normal((128, 40)).astype(np.float32) * 0.02
     packed, s = synth.quantize_q4g32(w)
     err = np.abs(oracle.dequant_q4g32(packed, s) - w)
-    step = np.repeat(s.astype(np.float64), 32, axis=1).T
+    step = np.repeat(s.astype(np.float64), 32, axis=0)
     assert (err <= step * (0.5 + 7 * 2.0 ** -10) + 1e-12).all()

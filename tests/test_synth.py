@@ -34,6 +34,6 @@ def test_workload_shapes_and_stats():
     hot = synth.expert_bias(c["capped"])
     assert (hot == 4.0).sum() == 8 and (hot == 0.0).sum() == 120
     packed, s = synth.expert_q4_weights(c["tiny"], 0, "gate")
-    assert packed.shape == (256, 64) and s.shape == (256, 4) and s.dtype == np.float16
+    assert packed.shape == (256, 64) and s.shape == (4, 256) and s.dtype == np.float16
     lo, hi = packed & 15, packed >> 4
     assert lo.min() >= 1 and hi.max() <= 15  # nibbles are q+8 with q in [-7, 7]
