@@ -54,6 +54,11 @@ def parse():
     ap.add_argument("--impl", default="own", choices=["own", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--tokens", type=int, default=0, help="override T of the workload (profiling small cases)")
+    ap.add_argument("--profile-calls", type=int, default=0,
+                    help="only run this many moe_forward calls and exit (for ncu: no timing, no other kernels)")
+    ap.add_argument("--sweep-threshold", action="store_true",
+                    help="time moe_forward for each stream_max_rows and print one JSON line")
     return ap.parse_args()
 
 
@@ -105,16 +110,36 @@ def kernel_source_hash(files):
 
 
 def committed_traffic(kernel, files, cfg_name):
-    """dram bytes per launch from a committed ncu summary, if it matches the current source."""
-    path = os.path.join(ROOT, "profiles", "traffic.json")
+    """DRAM bytes per launch (read + write) from the committed ncu summary table, if its row was
+    taken on the current kernel source; None otherwise."""
+    path = os.path.join(ROOT, "profiles", "dram_traffic.md")
     if not os.path.exists(path):
         return None
+    want = kernel_source_hash(files)
     with open(path) as fh:
-        tab = json.load(fh)
-    ent = tab.get(kernel, {}).get(cfg_name)
-    if not ent or ent.get("source_hash") != kernel_source_hash(files):
-        return None
-    return ent.get("dram_bytes_per_launch")
+        for line in fh:
+            cells = [c.strip().strip("`") for c in line.strip().strip("|").split("|")]
+            if len(cells) >= 5 and cells[0] == kernel and cells[1] == cfg_name and cells[2] == want:
+                return int(cells[3]) + int(cells[4])
+    return None
+
+
+def max_over_ranks(value, dist=None, device="cpu"):
+    """The largest of every rank's value (all ranks call it in the same order); the value itself
+    without a process group. Multi-GPU runs are replicas, so this timing reduction is the only
+    collective on the path."""
+    if dist is None:
+        return value
+    import torch
+    t = torch.tensor([float(value)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def aggregate_tokens_per_s(tokens_per_rank, world, max_ms_per_step):
+    """Whole-job throughput: every rank processes tokens_per_rank per step; the step takes the
+    slowest rank's time."""
+    return tokens_per_rank * world / (max_ms_per_step / 1e3)
 
 
 # --------------------------------------------------------------------------- clocks
@@ -267,9 +292,25 @@ def own_arm(args, cfg):
                                 device_id=torch.device("cuda", local))
 
     d = upload(cfg, "cuda")
-    p = b.params_for(cfg)
-    sh = (d["shared_gate"], d["shared_up"], d["shared_down"]) if cfg.has_shared else None
-    W = b.weights(d["w_gate"], d["w_up"], d["w_down"], d.get("s_gate"), d.get("s_up"), d.get("s_down"), shared=sh)
+    # load-time preparation (outside every step): an fp16 copy of W_down, so the
+    # down GEMM reads fp16 directly (the layer keeps h in fp16)
+    prep_ms = None
+    down_f16 = cfg.weight_format == "bf16"
+    if down_f16:
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        d["w_down_f16"] = b.prepare_down_f16(d["w_down"])
+        if cfg.has_shared:
+            d["shared_down_f16"] = b.prepare_down_f16(d["shared_down"])
+        e1.record()
+        e1.synchronize()
+        prep_ms = e0.elapsed_time(e1)
+    p = b.params_for(cfg, down_dtype=b.DOWN_F16 if down_f16 else b.DOWN_BF16)
+    sh = None
+    if cfg.has_shared:
+        sh = (d["shared_gate"], d["shared_up"], d["shared_down_f16" if down_f16 else "shared_down"])
+    W = b.weights(d["w_gate"], d["w_up"], d["w_down_f16" if down_f16 else "w_down"], d.get("s_gate"),
+                  d.get("s_up"), d.get("s_down"), shared=sh)
     ws = b.workspace(p, b.WS_FORWARD)
     out = torch.empty(cfg.T, cfg.d, dtype=torch.float32, device="cuda")
     flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device="cuda")
@@ -294,26 +335,37 @@ def own_arm(args, cfg):
     if b.get_error(ws):
         raise RuntimeError("device error word set during warm-up")
 
+    # The layer makes no host synchronisation, so one call captures into a CUDA
+    # graph; every timed step replays it (all kernels run, on the real buffers).
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        step()
+    torch.cuda.synchronize()
+
+    def timed_steps(fn, n):
+        s_ev = [torch.cuda.Event(enable_timing=True) for _ in range(n)]
+        e_ev = [torch.cuda.Event(enable_timing=True) for _ in range(n)]
+        for i in range(n):
+            flush.zero_()
+            s_ev[i].record(stream)
+            fn()
+            e_ev[i].record(stream)
+        torch.cuda.synchronize()
+        return sum(a.elapsed_time(z) for a, z in zip(s_ev, e_ev))
+
     K = args.steps
-    starts = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
-    ends = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
+    for _ in range(3):
+        flush.zero_()
+        graph.replay()
     if dist:
         dist.barrier()
     torch.cuda.synchronize()
     with ClockSampler(local) as clocks:
-        for i in range(K):
-            flush.zero_()
-            starts[i].record(stream)
-            step()
-            ends[i].record(stream)
-        torch.cuda.synchronize()
+        total_ms = timed_steps(graph.replay, K)
+    eager_ms = timed_steps(step, max(3, min(K, 50))) / max(3, min(K, 50))
     if dist:
         dist.barrier()
-    total_ms = sum(s.elapsed_time(e) for s, e in zip(starts, ends))
-    if dist:
-        t = torch.tensor([total_ms], dtype=torch.float64, device="cuda")
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        total_ms = float(t.item())
+    total_ms = max_over_ranks(total_ms, dist, "cuda")
     if b.get_error(ws):
         raise RuntimeError("device error word set during the timed steps")
     ms = total_ms / K
@@ -327,6 +379,25 @@ def own_arm(args, cfg):
     torch.cuda.synchronize()
     prof = b.profile_collect()
     b.profile_enable(False)
+
+    # the same steps with W_down given as bf16 (converted to fp16 per tile inside the down GEMM)
+    ms_down_bf16 = None
+    if down_f16:
+        p_bf = b.params_for(cfg, down_dtype=b.DOWN_BF16)
+        W_bf = b.weights(d["w_gate"], d["w_up"], d["w_down"],
+                         shared=(d["shared_gate"], d["shared_up"], d["shared_down"]) if cfg.has_shared else None)
+        kb = max(3, min(K, 50))
+        tot = 0.0
+        for i in range(kb + 3):
+            flush.zero_()
+            s0, s1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            s0.record(stream)
+            b.forward(p_bf, d["x"], d["logits"], W_bf, out, ws)
+            s1.record(stream)
+            s1.synchronize()
+            if i >= 3:
+                tot += s0.elapsed_time(s1)
+        ms_down_bf16 = tot / kb
 
     # end to end through moe_forward_host: pinned host x/logits in, out back, per step
     e2e = None
@@ -347,40 +418,45 @@ def own_arm(args, cfg):
             s1.record(stream)
             s1.synchronize()
             e_ms += s0.elapsed_time(s1)
-        if dist:
-            t = torch.tensor([e_ms], dtype=torch.float64, device="cuda")
-            dist.all_reduce(t, op=dist.ReduceOp.MAX)
-            e_ms = float(t.item())
-        e2e = {"value": cfg.T * world / (e_ms / ek / 1e3), "unit": "tokens/s",
+        e_ms = max_over_ranks(e_ms, dist, "cuda")
+        e2e = {"value": aggregate_tokens_per_s(cfg.T, world, e_ms / ek), "unit": "tokens/s",
                "h2d_bytes_per_step": cfg.T * cfg.d * 2 + cfg.T * cfg.E * 4, "d2h_bytes_per_step": cfg.T * cfg.d * 4,
                "ms_per_step": e_ms / ek}
 
     pk, pk_src = peaks()
-    tensor_bound = cfg.name not in ("decode1", "decode8", "decode32")
-    kern = "tc_gateup" if tensor_bound else "stream_gateup"
+    # Bound: the workload's arithmetic intensity against the measured ridge point.
+    ridge = pk["bf16_tflops"] * 1e12 / (pk["hbm_gbs"] * 1e9)
+    tensor_bound = wl["flops"] / wl["bytes"] >= ridge
+    # Dominant kernel: the largest measured share of the step among the expert GEMMs.
+    names = {"tc_gateup": ("grouped_gemm_kernel<0> (tcgen05 gate/up + clamped SwiGLU)", "gateup", "gemm_tc.cu"),
+             "tc_down": ("grouped_gemm_kernel<1> (tcgen05 down + gate scale)", "down", "gemm_tc.cu"),
+             "stream_gateup": ("stream_kernel<0> (few-rows gate/up)", "gateup", "stream.cu"),
+             "stream_down": ("stream_kernel<1> (few-rows down)", "down", "stream.cu")}
+    kern = max(names, key=lambda k: prof.get(k, (0.0, 0))[0])
     kms, kn = prof.get(kern, (0.0, 0))
     k_avg = kms / kn if kn else float("nan")
+    label, part, src = names[kern]
     if tensor_bound:
-        achieved = wl["flops_gateup"] / (k_avg / 1e3) / 1e12
+        work = wl["flops_" + part]
+        achieved = work / (k_avg / 1e3) / 1e12
         peak = pk["bf16_tflops"]
-        roof = {"kernel": "grouped_gemm_kernel<0> (tcgen05 gate/up + SwiGLU)", "bound": "tensor",
-                "achieved": achieved, "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak,
-                "peak_source": f"{pk_src} bf16_tflops (burst)", "avg_launch_ms": k_avg,
-                "algorithmic_per_launch": wl["flops_gateup"],
-                "traffic": committed_traffic("tc_gateup", ["gemm_tc.cu", "common.cuh"], cfg.name)}
+        roof = {"kernel": label, "bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+                "frac": achieved / peak, "peak_source": f"{pk_src} bf16_tflops (burst)"}
     else:
-        achieved = wl["bytes_gateup"] / (k_avg / 1e3) / 1e9
+        work = wl["bytes_" + part]
+        achieved = work / (k_avg / 1e3) / 1e9
         peak = pk["hbm_gbs"]
-        roof = {"kernel": "stream_kernel<0> (few-rows gate/up)", "bound": "hbm", "achieved": achieved,
-                "peak": peak, "unit": "GB/s", "frac": achieved / peak, "peak_source": f"{pk_src} hbm_gbs",
-                "avg_launch_ms": k_avg, "algorithmic_per_launch": wl["bytes_gateup"],
-                "traffic": committed_traffic("stream_gateup", ["stream.cu", "common.cuh"], cfg.name)}
+        roof = {"kernel": label, "bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
+                "frac": achieved / peak, "peak_source": f"{pk_src} hbm_gbs"}
+    roof.update({"avg_launch_ms": k_avg, "algorithmic_per_launch": work, "share_of_step": kms / K / ms,
+                 "traffic": committed_traffic(kern, [src, "common.cuh"], cfg.name)})
 
     line = None
     if rank == 0:
         tflops = wl["flops"] / (ms / 1e3) / 1e12
         gbs = wl["bytes"] / (ms / 1e3) / 1e9
-        line = {"metric": METRIC, "value": cfg.T * world / (ms / 1e3), "unit": "tokens/s", "n_gpus": world,
+        line = {"metric": METRIC, "value": aggregate_tokens_per_s(cfg.T, world, ms), "unit": "tokens/s",
+                "n_gpus": world,
                 "steps": K, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
                 "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
                 "config": {"workload": workload_name(cfg), "tokens_per_gpu": cfg.T, "routed_rows": P,
@@ -391,6 +467,10 @@ def own_arm(args, cfg):
                 "roofline": roof,
                 "kernels_ms_per_step": {k: v[0] / K for k, v in prof.items() if v[1]},
                 "gpu_launches": b.launch_count(p, b.WS_FORWARD) * K,
+                "step_launch": "CUDA graph replay of one moe_forward call",
+                "ms_per_step_eager": eager_ms,
+                "w_down": "fp16 copy prepared once at load time" if down_f16 else "n/a",
+                "w_down_prep_ms": prep_ms, "ms_per_step_w_down_bf16": ms_down_bf16,
                 "clocks": clocks.summary(), "e2e": e2e}
     if dist:
         dist.barrier()
@@ -402,11 +482,82 @@ def own_arm(args, cfg):
     return 0
 
 
+def prepared_layer(cfg, b, torch, stream_max_rows=-1):
+    """Device inputs, load-time fp16 W_down, params, weights struct, workspace, output."""
+    from synth.device import upload
+    d = upload(cfg, "cuda")
+    f16 = cfg.weight_format == "bf16"
+    wd = b.prepare_down_f16(d["w_down"]) if f16 else d["w_down"]
+    sh = None
+    if cfg.has_shared:
+        sh = (d["shared_gate"], d["shared_up"], b.prepare_down_f16(d["shared_down"]))
+    p = b.params_for(cfg, down_dtype=b.DOWN_F16 if f16 else b.DOWN_BF16, stream_max_rows=stream_max_rows)
+    W = b.weights(d["w_gate"], d["w_up"], wd, d.get("s_gate"), d.get("s_up"), d.get("s_down"), shared=sh)
+    out = torch.empty(cfg.T, cfg.d, dtype=torch.float32, device="cuda")
+    return d, p, W, out
+
+
+def profile_calls(args, cfg):
+    """Only `n` moe_forward calls (the first one warms up): a short, fixed launch sequence for ncu."""
+    import torch
+    from mixture_experts_routed_04_b200 import binding as b
+    d, p, W, out = prepared_layer(cfg, b, torch)
+    ws = b.workspace(p, b.WS_FORWARD)
+    torch.cuda.synchronize()
+    for _ in range(args.profile_calls):
+        b.forward(p, d["x"], d["logits"], W, out, ws)
+    torch.cuda.synchronize()
+    if b.get_error(ws):
+        raise RuntimeError("device error word set")
+    print(json.dumps({"profile_calls": args.profile_calls, "workload": workload_name(cfg)}))
+    return 0
+
+
+def sweep_threshold(args, cfg):
+    """moe_forward time (graph replay, L2 flushed) for each streaming threshold."""
+    import torch
+    from mixture_experts_routed_04_b200 import binding as b
+    d, _, W, out = prepared_layer(cfg, b, torch)
+    flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device="cuda")
+    res = {}
+    for smax in (0, 4, 8, 16, 24, 32, 48, 64, 96, 128):
+        p = b.params_for(cfg, down_dtype=b.DOWN_F16 if cfg.weight_format == "bf16" else b.DOWN_BF16,
+                         stream_max_rows=smax)
+        ws = b.workspace(p, b.WS_FORWARD)
+        for _ in range(3):
+            b.forward(p, d["x"], d["logits"], W, out, ws)
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            b.forward(p, d["x"], d["logits"], W, out, ws)
+        tot, n = 0.0, max(args.steps, 5)
+        for i in range(n + 3):
+            flush.zero_()
+            s0, s1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            s0.record()
+            g.replay()
+            s1.record()
+            s1.synchronize()
+            if i >= 3:
+                tot += s0.elapsed_time(s1)
+        if b.get_error(ws):
+            raise RuntimeError("device error word set")
+        res[smax] = tot / n
+        del g, ws
+    print(json.dumps({"sweep_stream_max_rows_ms": res, "workload": workload_name(cfg), "steps": max(args.steps, 5)}))
+    return 0
+
+
 def main():
     args = parse()
     cfg = synth.CONFIGS[args.config]
+    if args.tokens:
+        cfg = cfg.replace(T=args.tokens)
     if args.impl == "reference":
         return reference_arm(args, cfg)
+    if args.profile_calls:
+        return profile_calls(args, cfg)
+    if args.sweep_threshold:
+        return sweep_threshold(args, cfg)
     return own_arm(args, cfg)
 
 

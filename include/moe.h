@@ -83,6 +83,10 @@ typedef struct CUstream_st* moe_stream_t; /* same object as cudaStream_t */
 #define MOE_OUT_F32  0 /* fp32 (default): the residual stream's dtype */
 #define MOE_OUT_BF16 1
 
+/* dtype of w_down / shared_down (bf16 weight format only) */
+#define MOE_DOWN_BF16 0 /* as given; each tile is converted to fp16 in shared memory */
+#define MOE_DOWN_F16  1 /* prepared once with moe_convert_bf16_to_f16 (load time) */
+
 /* workspace kinds for moe_workspace_size() */
 #define MOE_WS_ROUTE        0
 #define MOE_WS_PERMUTE      1
@@ -105,8 +109,12 @@ typedef struct moe_params {
     int32_t d_ff_shared;     /* its f (must equal d_ff) */
     int32_t variant;         /* MOE_VARIANT_* */
     int32_t stream_max_rows; /* AUTO: experts with 1..this many kept rows use the streaming
-                                kernels, the rest the tcgen05 tiles; < 0 = library default */
+                                kernels, the rest the tcgen05 tiles; < 0 = library default,
+                                set from a measured sweep: 8 when even every touchable
+                                expert cannot give each of the 148 SMs a gate/up tile
+                                (single-token decode), else 0 (tiles for all) */
     int32_t out_dtype;       /* MOE_OUT_F32 | MOE_OUT_BF16 */
+    int32_t down_dtype;      /* MOE_DOWN_BF16 | MOE_DOWN_F16 */
 } moe_params;
 
 /*
@@ -249,6 +257,18 @@ MOE_API int moe_forward_host(const moe_params* p, const uint16_t* x_host, const 
                      moe_stream_t stream);
 
 /*
+ * Weight preparation, done once at load time, outside the layer's calls:
+ * dst[i] = fp16(src[i]) for n bf16 values (round to nearest even; exact for
+ * |v| in fp16's normal range and for bf16 values down to 2^-17). Used to keep
+ * an fp16 copy of W_down so the down GEMM reads fp16 directly (down_dtype =
+ * MOE_DOWN_F16): the layer keeps h in fp16 for precision, and one tcgen05 MMA
+ * takes a single operand type. Values beyond +-65504 set bit MOE_DEVERR_RANGE
+ * in *err_ws's error word when err_ws is not NULL. Asynchronous.
+ */
+MOE_API int moe_convert_bf16_to_f16(const uint16_t* src, uint16_t* dst, int64_t n, void* err_ws,
+                                    moe_stream_t stream);
+
+/*
  * Synchronises `stream`, then reads the sticky device error word at the start
  * of ws into *err (host). Returns MOE_OK if it is 0, MOE_ERR_DEVICE if not.
  */
@@ -280,7 +300,8 @@ MOE_API int moe_set_wait_limit_ns(uint64_t ns);
 #define MOE_K_STREAM_REDUCE  9  /* S8 K-split partial sums + SwiGLU */
 #define MOE_K_STREAM_DOWN   10  /* S8 few-rows down */
 #define MOE_K_COMBINE       11  /* S7 gate-weighted combine */
-#define MOE_K_COUNT         12
+#define MOE_K_CONVERT       12  /* load-time bf16 -> fp16 weight copy (not a layer step) */
+#define MOE_K_COUNT         13
 
 /*
  * Number of kernel launches one call of `which` (MOE_WS_ROUTE .. MOE_WS_FORWARD_HOST,

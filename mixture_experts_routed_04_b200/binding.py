@@ -23,6 +23,7 @@ STATUS = {0: "ok", 1: "invalid argument", 2: "workspace too small", 3: "unsuppor
           4: "CUDA error", 5: "misaligned pointer", 6: "device error word set"}
 DEVERR_TIMEOUT, DEVERR_BOUNDS, DEVERR_RANGE = 0x1, 0x2, 0x4
 OUT_F32, OUT_BF16 = 0, 1
+DOWN_BF16, DOWN_F16 = 0, 1
 WEIGHTS_BF16, WEIGHTS_Q4G32 = 0, 1
 VARIANT_AUTO, VARIANT_TENSOR, VARIANT_STREAM = 0, 1, 2
 WS_ROUTE, WS_PERMUTE, WS_EXPERT_FFN, WS_COMBINE, WS_FORWARD, WS_FORWARD_HOST = range(6)
@@ -31,11 +32,11 @@ WS_ROUTE, WS_PERMUTE, WS_EXPERT_FFN, WS_COMBINE, WS_FORWARD, WS_FORWARD_HOST = r
 EXPORTS = ("moe_version", "moe_status_string", "moe_capacity", "moe_max_rows", "moe_workspace_size",
            "moe_route", "moe_permute", "moe_expert_ffn", "moe_combine", "moe_forward", "moe_forward_host",
            "moe_get_error", "moe_clear_error", "moe_set_wait_limit_ns", "moe_launch_count",
-           "moe_profile_enable", "moe_profile_collect")
+           "moe_profile_enable", "moe_profile_collect", "moe_convert_bf16_to_f16")
 
 # kernel ids (MOE_K_*), in order
 KERNELS = ("route", "perm_count", "perm_scan", "perm_scatter", "schedule", "gather", "tc_gateup", "tc_down",
-           "stream_gateup", "stream_reduce", "stream_down", "combine")
+           "stream_gateup", "stream_reduce", "stream_down", "combine", "convert")
 
 
 class MoeError(RuntimeError):
@@ -47,7 +48,8 @@ class Params(ctypes.Structure):
                 ("E", ctypes.c_int32), ("k", ctypes.c_int32), ("capacity_factor", ctypes.c_float),
                 ("swiglu_limit", ctypes.c_float), ("weight_format", ctypes.c_int32),
                 ("has_shared", ctypes.c_int32), ("d_ff_shared", ctypes.c_int32),
-                ("variant", ctypes.c_int32), ("stream_max_rows", ctypes.c_int32), ("out_dtype", ctypes.c_int32)]
+                ("variant", ctypes.c_int32), ("stream_max_rows", ctypes.c_int32), ("out_dtype", ctypes.c_int32),
+                ("down_dtype", ctypes.c_int32)]
 
 
 class Weights(ctypes.Structure):
@@ -83,6 +85,7 @@ def lib() -> ctypes.CDLL:
             "moe_launch_count": ([_P, ctypes.c_int, ctypes.POINTER(ctypes.c_int)], ctypes.c_int),
             "moe_profile_enable": ([ctypes.c_int], ctypes.c_int),
             "moe_profile_collect": ([ctypes.POINTER(ctypes.c_double), ctypes.POINTER(ctypes.c_int64)], ctypes.c_int),
+            "moe_convert_bf16_to_f16": ([_V, _V, ctypes.c_int64, _V, _V], ctypes.c_int),
         }
         for name, (args, res) in sig.items():
             fn = getattr(L, name)
@@ -92,9 +95,10 @@ def lib() -> ctypes.CDLL:
 
 
 def params(T, d_model, d_ff, E, k, capacity_factor=0.0, swiglu_limit=7.0, weight_format=WEIGHTS_BF16,
-           has_shared=0, d_ff_shared=0, variant=VARIANT_AUTO, stream_max_rows=-1, out_dtype=OUT_F32) -> Params:
+           has_shared=0, d_ff_shared=0, variant=VARIANT_AUTO, stream_max_rows=-1, out_dtype=OUT_F32,
+           down_dtype=DOWN_BF16) -> Params:
     return Params(T, d_model, d_ff, E, k, capacity_factor, swiglu_limit, weight_format, int(has_shared),
-                  d_ff_shared if has_shared else 0, variant, stream_max_rows, out_dtype)
+                  d_ff_shared if has_shared else 0, variant, stream_max_rows, out_dtype, down_dtype)
 
 
 def params_for(cfg, **over) -> Params:
@@ -220,3 +224,18 @@ def profile_collect() -> dict:
     cnt = (ctypes.c_int64 * n)()
     check(lib().moe_profile_collect(ms, cnt), "moe_profile_collect")
     return {KERNELS[i]: (ms[i], cnt[i]) for i in range(n)}
+
+
+def convert_bf16_to_f16(src, dst, err_ws=None, stream=None) -> None:
+    """Load-time weight preparation: dst (fp16) = src (bf16), elementwise."""
+    assert src.numel() == dst.numel()
+    check(lib().moe_convert_bf16_to_f16(_p(src), _p(dst), src.numel(), _p(err_ws), _stream(stream)),
+          "moe_convert_bf16_to_f16")
+
+
+def prepare_down_f16(w_down, stream=None):
+    """fp16 copy of a bf16 W_down (or shared W_down), for down_dtype=DOWN_F16."""
+    import torch
+    out = torch.empty(w_down.shape, dtype=torch.float16, device=w_down.device)
+    convert_bf16_to_f16(w_down, out, stream=stream)
+    return out

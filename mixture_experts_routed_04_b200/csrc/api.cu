@@ -15,12 +15,14 @@ cudaError_t launch_gather(const Dims& D, const uint16_t* x, const int32_t* sorte
                           uint16_t* xg, uint32_t* err, cudaStream_t s);
 cudaError_t launch_tensor_ffn(const Dims& D, const uint16_t* xg, uint16_t* h, const int32_t* tile_base,
                               const int32_t* offsets, const int32_t* sorted_pair, const float* topk_w,
-                              const moe_weights* w, uint16_t* y_rows, uint32_t* err, uint64_t wait_ns,
+                              const moe_weights* w,
+                              uint16_t* y_rows, int32_t* counters, uint32_t* err, uint64_t wait_ns,
                               cudaStream_t s);
-cudaError_t launch_stream_ffn(const Dims& D, const uint16_t* x, uint16_t* h, float* part, const int32_t* offsets,
-                              const int32_t* stream_list, const int32_t* n_stream, const int32_t* sorted_token,
-                              const int32_t* sorted_pair, const float* topk_w, const moe_weights* w,
-                              uint16_t* y_rows, uint32_t* err, uint64_t wait_ns, cudaStream_t s);
+cudaError_t launch_convert_bf16_f16(const uint16_t* src, uint16_t* dst, int64_t n, uint32_t* err, cudaStream_t s);
+cudaError_t launch_stream_ffn(const Dims& D, const uint16_t* xg, uint16_t* h, float* part, const int32_t* offsets,
+                              const int32_t* stream_list, const int32_t* n_stream, const int32_t* sorted_pair,
+                              const float* topk_w, const moe_weights* w, uint16_t* y_rows, uint32_t* err,
+                              uint64_t wait_ns, cudaStream_t s);
 
 static std::atomic<uint64_t> g_wait_ns{1000000000ull};
 
@@ -50,11 +52,14 @@ static int make_dims(const moe_params* p, Dims* D) {
     if (p->variant < MOE_VARIANT_AUTO || p->variant > MOE_VARIANT_STREAM) return MOE_ERR_INVALID_ARG;
     if (p->has_shared != 0 && p->has_shared != 1) return MOE_ERR_INVALID_ARG;
     if (p->out_dtype != MOE_OUT_F32 && p->out_dtype != MOE_OUT_BF16) return MOE_ERR_INVALID_ARG;
+    if (p->down_dtype != MOE_DOWN_BF16 && p->down_dtype != MOE_DOWN_F16) return MOE_ERR_INVALID_ARG;
+    if (p->down_dtype == MOE_DOWN_F16 && p->weight_format != MOE_WEIGHTS_BF16) return MOE_ERR_INVALID_ARG;
     const int64_t pairs = int64_t(p->T) * p->k;
     if (pairs + p->T >= (int64_t(1) << 31)) return MOE_ERR_INVALID_ARG;
     if (int64_t(p->d_model) * p->d_ff * p->E >= (int64_t(1) << 40)) return MOE_ERR_INVALID_ARG;
     if (p->has_shared && (p->d_ff_shared != p->d_ff)) return MOE_ERR_UNSUPPORTED;
-    if (p->weight_format == MOE_WEIGHTS_Q4G32) return MOE_ERR_UNSUPPORTED;  // not built yet
+    if (p->weight_format == MOE_WEIGHTS_Q4G32 && (p->has_shared || p->variant == MOE_VARIANT_STREAM))
+        return MOE_ERR_UNSUPPORTED;  // Q4G32 runs on the tcgen05 tile kernels only
     D->T = p->T;
     D->d = p->d_model;
     D->f = p->d_ff;
@@ -77,24 +82,30 @@ static int make_dims(const moe_params* p, Dims* D) {
     D->perm_blocks = int((pairs + kPermPairsPerBlock - 1) / kPermPairsPerBlock);
     D->fmt = p->weight_format;
     D->variant = p->variant;
-    D->stream_max_rows = p->stream_max_rows < 0 ? kDefaultStreamMaxRows : p->stream_max_rows;
+    // Default variant choice, from the measured sweep over rows-per-expert
+    // thresholds (prompt, capped and decode layers): the tcgen05 tiles win
+    // whenever the touched experts can give every SM a gate/up tile — even for
+    // experts of one row (T=8, 32: 98% of HBM); below that (T=1) experts of up
+    // to kStreamRowsFewExperts rows take the weight-streaming kernels.
+    if (p->stream_max_rows < 0) {
+        const int64_t touched_max = std::min<int64_t>(p->E + p->has_shared, pairs + p->has_shared);
+        const int64_t tiles_max = touched_max * ((p->d_ff + 127) / 128);
+        D->stream_max_rows = tiles_max < kSmCountB200 ? kStreamRowsFewExperts : 0;
+    } else {
+        D->stream_max_rows = p->stream_max_rows;
+    }
     D->limit = p->swiglu_limit;
     D->out_bf16 = p->out_dtype == MOE_OUT_BF16;
-    // The streaming kernels hold one K slice of <= 2048 rows in shared memory:
-    // gate/up split d into slices; down needs f <= 2048.
-    const bool stream_ok = p->d_ff <= 2048;
-    if (!stream_ok) {
-        if (D->variant == MOE_VARIANT_STREAM) return MOE_ERR_UNSUPPORTED;
-        D->stream_max_rows = 0;
-    }
-    // K split of the streaming gate/up: enough units to cover the SMs when few
-    // experts are touched (decode), and slices of at most 2048.
+    D->down_f16 = p->down_dtype == MOE_DOWN_F16;
+    // The streaming kernels take bf16 weights only (Q4G32 runs on the tiles).
+    if (p->weight_format != MOE_WEIGHTS_BF16) D->stream_max_rows = 0;
+    // K split of the streaming gate/up, for load balance only: when few experts
+    // are touched (decode), split d so that there are a few work items per SM
+    // (the slices stay multiples of 64).
     int ks = 1;
-    while (p->d_model / ks > 2048) ks *= 2;
     const int64_t touched = std::min<int64_t>(D->Etot, pairs + p->has_shared);
     const int64_t units = touched * (p->d_ff / 64);
     while (ks < 8 && units * ks < 4 * 148 && (p->d_model % (ks * 2 * 64)) == 0) ks *= 2;
-    if (p->d_model % (ks * 64)) return MOE_ERR_UNSUPPORTED;
     D->ks = ks;
     return MOE_OK;
 }
@@ -118,7 +129,7 @@ WsLayout ws_layout(const Dims& D, int which) {
     if (ffn) {
         L.tile_base = take(size_t(D.Etot + 1) * 4);
         L.stream_list = take(size_t(D.Etot) * 4);
-        L.n_stream = take(4);
+        L.n_stream = take(16);  // [0] streaming experts, [1], [2] tile-unit counters
         L.xg = take(size_t(D.rows) * D.d * 2);
         L.h = take(size_t(D.rows) * D.f * 2);
         if (D.ks > 1) L.part = take(size_t(D.ks) * 2 * D.rows * D.f * 4);
@@ -153,15 +164,18 @@ cudaError_t launch_expert_ffn(const Dims& D, const WsLayout& L, const FfnArgs& a
     float* part = L.part ? reinterpret_cast<float*>(ws + L.part) : nullptr;
     cudaError_t e = launch_schedule(D, a.offsets, tile_base, stream_list, n_stream, a.err, s);
     if (e != cudaSuccess) return e;
+    // Rows in expert order for both variants (fp16 for Q4G32, whose MMAs run
+    // in fp16). A TMA tile::gather4 of the rows inside the GEMM was measured
+    // slower: 32 TMA instructions per k-block left the producer behind.
+    if ((e = launch_gather(D, a.x, a.sorted_token, a.offsets, xg, a.err, s)) != cudaSuccess) return e;
     if (D.variant != MOE_VARIANT_STREAM) {
-        if ((e = launch_gather(D, a.x, a.sorted_token, a.offsets, xg, a.err, s)) != cudaSuccess) return e;
-        if ((e = launch_tensor_ffn(D, xg, h, tile_base, a.offsets, a.sorted_pair, a.topk_w, a.w, a.y_rows, a.err,
-                                   a.wait_ns, s)) != cudaSuccess)
+        if ((e = launch_tensor_ffn(D, xg, h, tile_base, a.offsets, a.sorted_pair, a.topk_w, a.w, a.y_rows,
+                                   n_stream + 1, a.err, a.wait_ns, s)) != cudaSuccess)
             return e;
     }
     if (D.variant != MOE_VARIANT_TENSOR && D.stream_max_rows > 0) {
-        if ((e = launch_stream_ffn(D, a.x, h, part, a.offsets, stream_list, n_stream, a.sorted_token, a.sorted_pair,
-                                   a.topk_w, a.w, a.y_rows, a.err, a.wait_ns, s)) != cudaSuccess)
+        if ((e = launch_stream_ffn(D, xg, h, part, a.offsets, stream_list, n_stream, a.sorted_pair, a.topk_w, a.w,
+                                   a.y_rows, a.err, a.wait_ns, s)) != cudaSuccess)
             return e;
     }
     return cudaSuccess;
@@ -183,6 +197,10 @@ static int check_ws(const Dims& D, int which, const void* ws, size_t ws_bytes) {
 static int check_weights(const Dims& D, const moe_weights* w) {
     if (!w || !w->w_gate || !w->w_up || !w->w_down) return MOE_ERR_INVALID_ARG;
     if (!al16(w->w_gate) || !al16(w->w_up) || !al16(w->w_down)) return MOE_ERR_MISALIGNED;
+    if (D.fmt == MOE_WEIGHTS_Q4G32) {
+        if (!w->s_gate || !w->s_up || !w->s_down) return MOE_ERR_INVALID_ARG;
+        if (!al16(w->s_gate) || !al16(w->s_up) || !al16(w->s_down)) return MOE_ERR_MISALIGNED;
+    }
     if (D.has_shared) {
         if (!w->shared_gate || !w->shared_up || !w->shared_down) return MOE_ERR_INVALID_ARG;
         if (!al16(w->shared_gate) || !al16(w->shared_up) || !al16(w->shared_down)) return MOE_ERR_MISALIGNED;
@@ -371,7 +389,8 @@ int moe_launch_count(const moe_params* p, int which, int* n) {
     if (st != MOE_OK) return st;
     if (!n || which < MOE_WS_ROUTE || which > MOE_WS_FORWARD_HOST) return MOE_ERR_INVALID_ARG;
     int ffn = 1;  // schedule
-    if (D.variant != MOE_VARIANT_STREAM) ffn += 3;  // gather + two tcgen05 GEMMs
+    ffn += 1;                                       // gather
+    if (D.variant != MOE_VARIANT_STREAM) ffn += 2;  // two tcgen05 GEMMs
     if (D.variant != MOE_VARIANT_TENSOR && D.stream_max_rows > 0) ffn += 2 + (D.ks > 1 ? 1 : 0);
     switch (which) {
         case MOE_WS_ROUTE: *n = 1; break;
@@ -381,6 +400,13 @@ int moe_launch_count(const moe_params* p, int which, int* n) {
         default: *n = 1 + 3 + ffn + 1; break;
     }
     return MOE_OK;
+}
+
+int moe_convert_bf16_to_f16(const uint16_t* src, uint16_t* dst, int64_t n, void* err_ws, moe_stream_t stream) {
+    if (n < 0 || (n > 0 && (!src || !dst))) return MOE_ERR_INVALID_ARG;
+    if (!al16(src) || !al16(dst)) return MOE_ERR_MISALIGNED;
+    if (err_ws && (reinterpret_cast<uintptr_t>(err_ws) & 255u)) return MOE_ERR_MISALIGNED;
+    return status_of(launch_convert_bf16_f16(src, dst, n, static_cast<uint32_t*>(err_ws), stream));
 }
 
 int moe_set_wait_limit_ns(uint64_t ns) {

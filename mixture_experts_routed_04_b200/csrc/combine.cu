@@ -79,3 +79,49 @@ cudaError_t launch_combine(const Dims& D, const uint16_t* y_rows, const int32_t*
 }
 
 }  // namespace moe
+
+namespace moe {
+
+namespace {
+
+// dst = fp16(src), 8 values per thread per step; out-of-range values flagged.
+__global__ void __launch_bounds__(256) convert_bf16_f16_kernel(const uint16_t* __restrict__ src,
+                                                               uint16_t* __restrict__ dst, int64_t n, uint32_t* err) {
+    bool bad = false;
+    const int64_t nv = n / 8;
+    for (int64_t i = int64_t(blockIdx.x) * blockDim.x + threadIdx.x; i < nv; i += int64_t(gridDim.x) * blockDim.x) {
+        uint4 v = __ldg(reinterpret_cast<const uint4*>(src) + i);
+        bad |= !(f16_range_ok(bf16_lo(v.x)) && f16_range_ok(bf16_hi(v.x)) && f16_range_ok(bf16_lo(v.y)) &&
+                 f16_range_ok(bf16_hi(v.y)) && f16_range_ok(bf16_lo(v.z)) && f16_range_ok(bf16_hi(v.z)) &&
+                 f16_range_ok(bf16_lo(v.w)) && f16_range_ok(bf16_hi(v.w)));
+        v.x = bf16x2_to_f16x2(v.x);
+        v.y = bf16x2_to_f16x2(v.y);
+        v.z = bf16x2_to_f16x2(v.z);
+        v.w = bf16x2_to_f16x2(v.w);
+        reinterpret_cast<uint4*>(dst)[i] = v;
+    }
+    for (int64_t i = nv * 8 + int64_t(blockIdx.x) * blockDim.x + threadIdx.x; i < n;
+         i += int64_t(gridDim.x) * blockDim.x) {
+        const float f = bf16_to_f32(src[i]);
+        bad |= !f16_range_ok(f);
+        dst[i] = uint16_t(pack_f16x2(f, 0.f) & 0xFFFFu);
+    }
+    if (bad) set_error(err, MOE_DEVERR_RANGE);
+}
+
+}  // namespace
+
+cudaError_t launch_convert_bf16_f16(const uint16_t* src, uint16_t* dst, int64_t n, uint32_t* err, cudaStream_t s) {
+    if (n <= 0) return cudaSuccess;
+    int64_t blocks = (n / 8 + 255) / 256;
+    const int64_t cap = int64_t(num_sms()) * 8;
+    if (blocks > cap) blocks = cap;
+    if (blocks < 1) blocks = 1;
+    {
+        ProfScope prof_(MOE_K_CONVERT, s);
+        convert_bf16_f16_kernel<<<int(blocks), 256, 0, s>>>(src, dst, n, err);
+    }
+    return cudaGetLastError();
+}
+
+}  // namespace moe

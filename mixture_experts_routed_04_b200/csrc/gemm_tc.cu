@@ -1,24 +1,38 @@
-// gemm_tc.cu — S4..S6 on the 5th-generation tensor cores: the tile schedule
-// (K3), the row gather (S4), and one persistent grouped GEMM kernel used twice:
+// gemm_tc.cu — S4..S6 (+ S9) on the 5th-generation tensor cores: the tile
+// schedule (K3), the row gather (S4), and one persistent grouped GEMM kernel
+// used twice per layer:
 //   MODE 0: h = silu(clamp(x W_gate[e])) * clamp(x W_up[e])   (S5, SwiGLU fused)
 //   MODE 1: y = w_pair * (h W_down[e])                          (S6, gate scale fused)
+// with the weights either bf16 ([E, K, N], N contiguous) or Q4G32 (4-bit,
+// dequantised in the kernel once per weight tile: S9).
 //
 // Prior art: "Strata PR #4366" (DS4_FAT_ROWS), Approach — a popular expert's
-// weights decoded once, its rows gathered, one FP16 cuBLAS GEMM, then a clamped
-// SwiGLU; "mini-AGI PR #4" run() — experts grouped by load, each group at its
-// own size. Here every expert with rows becomes ceil(rows/128) M-tiles of one
-// grouped launch; rows past an expert's end are computed and masked.
+// packed weights decoded once to FP16, its rows gathered, one FP16 GEMM, then a
+// clamped SwiGLU in FP16; "mini-AGI PR #4" run() — experts grouped by load,
+// each group at its own size. Here every expert with rows becomes
+// ceil(rows/128) M-tiles of one grouped launch; rows past an expert's end are
+// computed and masked.
 //
 // Kernel shape (one CTA per SM, persistent over work units):
-//   warp 0   TMA producer: A = 128 rows x 64 K of the gathered rows (2-D map,
-//            128-byte swizzle, K-major), B = 64 K x 256 N of the expert's
-//            weights (3-D map [E, K, N], four 64-wide boxes, N-major). Four
-//            48 KB stages in shared memory, mbarrier full/empty pairs.
-//   warp 1   TMEM allocator + single-thread tcgen05.mma issuer: M=128, N=256,
-//            K=16 per instruction, fp32 accumulators in TMEM, two 256-column
-//            buffers so the epilogue of a unit overlaps the next unit's MMAs.
+//   warp 0    TMA producer. A = 128 rows x 64 K of the gathered rows (2-D map,
+//             128-byte swizzle, K-major). B, bf16: 64 K x 256 N of the expert's
+//             weights (3-D map, four 64-wide boxes, N-major). B, Q4G32: the
+//             packed nibbles of 256 N-rows x 64 K (32 bytes a row) and the
+//             k-block's two scale groups.
+//   warp 1    TMEM allocator + single-thread tcgen05.mma issuer: M=128, N=256,
+//             K=16 per instruction, fp32 accumulators in TMEM, two 256-column
+//             buffers so the epilogue of a unit overlaps the next unit's MMAs.
 //   warps 2-5 epilogue: tcgen05.ld 32 lanes x 32 columns, fused SwiGLU or gate
-//            scaling, bf16 stores. Warp w reads TMEM lanes 32*(w%4)..+31.
+//             scaling, fp16 stores. Warp w reads TMEM lanes 32*(w%4)..+31.
+//   warps 6-9 transform (Q4G32, or MODE 1 with W_down given as bf16): turn the
+//             landed B tile into fp16 — bf16 -> fp16 in place (costly: it
+//             competes with the MMA for shared-memory bandwidth, so W_down is
+//             normally prepared as fp16 once at load time and this is skipped),
+//             or nibbles x scale -> fp16 written in the
+//             K-major 128-byte-swizzled layout the MMA reads — then release it
+//             to the MMA warp (generic-proxy writes fenced for the async proxy).
+// Operand types per MMA: MODE 0 bf16 x bf16 (fp16 x fp16 with Q4G32, x being
+// gathered as fp16); MODE 1 fp16 x fp16 (h is fp16). fp32 accumulate always.
 // A work unit is (expert, n-tile, m-tile); units of one expert and n-tile are
 // adjacent so its weight tile is read from HBM once and served from L2 to its
 // other M-tiles. Every mbarrier wait is bounded in time; a wait that gives up
@@ -30,13 +44,36 @@ namespace moe {
 
 namespace tc {
 
-constexpr int BM = 128, BK = 64, BN = 256, STAGES = 4;
+constexpr int BM = 128, BK = 64, BN = 256;
 constexpr int A_BYTES = BM * BK * 2;  // 16 KB
 constexpr int B_CHUNK = 64 * BK * 2;  // one 64(N) x 64(K) box, 8 KB
-constexpr int B_BYTES = 4 * B_CHUNK;  // 32 KB
-constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
+constexpr int B_BYTES = 4 * B_CHUNK;  // 32 KB (256 N x 64 K, 2-byte elements)
+constexpr int P_BYTES = BN * BK / 2;  // Q4G32 nibbles of 256 rows x 64 K: 8 KB
+constexpr int S_BYTES = 2 * BN * 2;   // two scale groups x 256 rows, fp16: 1 KB
 constexpr int TMEM_COLS = 512;
-constexpr int SMEM_BYTES = 1024 + STAGES * STAGE_BYTES + 256;  // + barriers
+
+// WF: weight form. 0 = bf16 as given, 1 = Q4G32, 2 = fp16 (W_down prepared at load time).
+template <int MODE, int WF>
+struct Cfg {
+    static constexpr bool Q4 = WF == 1;
+    static constexpr bool kTransform = Q4 || (MODE == 1 && WF == 0);
+    static constexpr int kThreads = kTransform ? 320 : 192;
+    static constexpr int kStages = Q4 ? 3 : 4;
+    static constexpr int kStageBytes = Q4 ? A_BYTES + B_BYTES + P_BYTES + S_BYTES : A_BYTES + B_BYTES;
+    static constexpr uint32_t kTxBytes = Q4 ? A_BYTES + P_BYTES + S_BYTES : A_BYTES + B_BYTES;
+    static constexpr int kSmem = 1024 + kStages * kStageBytes + 512;  // + barriers, unit ring
+    // warps that read the unit ring: MMA, 4 epilogue (+ 4 transform)
+    static constexpr int kUnitReaders = 1 + 4 + (kTransform ? 4 : 0);
+    // bf16 operands for the bf16 gate/up; fp16 otherwise. B is N-major (bf16
+    // weights as stored) or K-major (dequantised from the K-major Q4G32 rows).
+    static constexpr uint32_t kIdesc =
+        idesc_f16_f32(BM, BN, /*ab_bf16=*/(MODE == 0 && WF == 0) ? 1 : 0, /*a_mn=*/0, /*b_mn=*/Q4 ? 0 : 1);
+    // An expert's last tile with <= 64 rows runs M=64 (half the MMA work). Its
+    // accumulator sits in lanes 0-15 of each 32-lane TMEM sub-partition: row m
+    // in lane 32*(m/16) + m%16, every column as for M=128.
+    static constexpr uint32_t kIdesc64 =
+        idesc_f16_f32(64, BN, /*ab_bf16=*/(MODE == 0 && WF == 0) ? 1 : 0, /*a_mn=*/0, /*b_mn=*/Q4 ? 0 : 1);
+};
 
 struct GemmParams {
     int K;        // reduction length (multiple of 64)
@@ -44,6 +81,7 @@ struct GemmParams {
     int n_tiles;  // output tiles per M-tile
     int E;        // routed experts; index E is the shared expert
     int Etot;
+    int32_t* unit_counter;     // next unit to claim (zeroed by the schedule kernel)
     const int32_t* tile_base;  // [Etot+1] exclusive prefix of M-tiles
     const int32_t* offsets;    // [Etot+1] row offsets
     uint16_t* out;             // [rows, n_out] fp16 (h or y)
@@ -88,29 +126,110 @@ MOE_DEV float swiglu(float g, float u, float L) {
     return g / (1.0f + expf(-g)) * u;
 }
 
-// Threads: MODE 0 has 6 warps (producer, MMA, 4 epilogue); MODE 1 adds 4
-// converter warps (6..9) that turn each landed W_down tile from bf16 into fp16
-// in place, so the down GEMM runs fp16 x fp16 (h is fp16).
-template <int MODE>
-struct Roles {
-    static constexpr int kThreads = MODE == 0 ? 192 : 320;
-    static constexpr uint32_t kIdesc = idesc_f16_f32(BM, BN, /*ab_bf16=*/MODE == 0 ? 1 : 0, /*a_mn=*/0, /*b_mn=*/1);
-};
+MOE_DEV uint32_t lop3_and_or(uint32_t a, uint32_t mask, uint32_t orv) {
+    uint32_t r;
+    asm("lop3.b32 %0, %1, %2, %3, 0xEA;" : "=r"(r) : "r"(a), "r"(mask), "r"(orv));  // (a & b) | c
+    return r;
+}
+MOE_DEV uint32_t hsub2(uint32_t a, uint32_t b) {
+    uint32_t r;
+    asm("sub.rn.f16x2 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(b));
+    return r;
+}
+MOE_DEV uint32_t hmul2(uint32_t a, uint32_t b) {
+    uint32_t r;
+    asm("mul.rn.f16x2 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(b));
+    return r;
+}
 
-template <int MODE>
-__global__ void __launch_bounds__(Roles<MODE>::kThreads, 1)
+// One Q4G32 word (k = 8i..8i+7, nibble p holding k 8i+{0,2,4,6,1,3,5,7}[p])
+// times its scale pair -> eight fp16 in k order. (w >> 4j) & 0x000F000F keeps
+// nibbles j and j+4, i.e. k = 2j and 2j+1; OR-ing 0x6400 makes each the fp16
+// value 1024 + u exactly, minus 1032 gives q = u - 8 exactly, then one rounding
+// for q * s.
+MOE_DEV uint4 dequant_word(uint32_t w, uint32_t s2) {
+    constexpr uint32_t kMask = 0x000F000Fu, kMagic = 0x64006400u, kBias = 0x64086408u;
+    uint4 o;
+    o.x = hmul2(hsub2(lop3_and_or(w, kMask, kMagic), kBias), s2);
+    o.y = hmul2(hsub2(lop3_and_or(w >> 4, kMask, kMagic), kBias), s2);
+    o.z = hmul2(hsub2(lop3_and_or(w >> 8, kMask, kMagic), kBias), s2);
+    o.w = hmul2(hsub2(lop3_and_or(w >> 12, kMask, kMagic), kBias), s2);
+    return o;
+}
+
+// ---------------------------------------------------------------- unit ring
+// Work is claimed dynamically: the producer warp takes the next unit with an
+// atomic counter and publishes it in a shared-memory ring that the MMA,
+// epilogue and transform warps read in order. A CTA that draws slow
+// (DRAM-bound) units therefore takes fewer of them and every SM finishes
+// together. Which CTA computes a unit does not change its result.
+constexpr int UR = 8;  // ring depth; the producer runs at most ~2 units ahead of the epilogue
+
+// Producer: claim and publish the next unit (-1 when none is left). Returns
+// false if the bounded wait gave up. Warp-uniform.
+MOE_DEV bool ring_publish(int& u, int& slot, uint32_t& phase, int* counter, int total, volatile int* ring,
+                          uint64_t* ufull, uint64_t* uempty, volatile int* abort_flag, uint32_t* err, uint64_t ns) {
+    const int lane = threadIdx.x & 31;
+    int ok = 1;
+    if (lane == 0) ok = mbar_wait_bounded(uempty + slot, phase ^ 1u, abort_flag, err, ns);
+    ok = __shfl_sync(0xFFFFFFFFu, ok, 0);
+    if (!ok) return false;
+    int v = 0;
+    if (lane == 0) {
+        v = atomicAdd(counter, 1);
+        if (v >= total) v = -1;
+        ring[slot] = v;
+        mbar_arrive(ufull + slot);
+    }
+    u = __shfl_sync(0xFFFFFFFFu, v, 0);
+    if (++slot == UR) {
+        slot = 0;
+        phase ^= 1u;
+    }
+    return true;
+}
+
+// Reader: the next published unit (-1: done). Returns false if the wait gave up.
+MOE_DEV bool ring_read(int& u, int& slot, uint32_t& phase, volatile int* ring, uint64_t* ufull, uint64_t* uempty,
+                       volatile int* abort_flag, uint32_t* err, uint64_t ns) {
+    const int lane = threadIdx.x & 31;
+    int ok = 1;
+    if (lane == 0) ok = mbar_wait_bounded(ufull + slot, phase, abort_flag, err, ns);
+    ok = __shfl_sync(0xFFFFFFFFu, ok, 0);
+    if (!ok) return false;
+    int v = 0;
+    if (lane == 0) {
+        v = ring[slot];
+        mbar_arrive(uempty + slot);
+    }
+    u = __shfl_sync(0xFFFFFFFFu, v, 0);
+    if (++slot == UR) {
+        slot = 0;
+        phase ^= 1u;
+    }
+    return true;
+}
+
+template <int MODE, int WF>
+__global__ void __launch_bounds__(Cfg<MODE, WF>::kThreads, 1)
     grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB0,
                         const __grid_constant__ CUtensorMap tmB1, const __grid_constant__ CUtensorMap tmS0,
                         const __grid_constant__ CUtensorMap tmS1, const GemmParams p) {
+    using C = Cfg<MODE, WF>;
+    constexpr bool Q4 = C::Q4;
+    constexpr int STAGES = C::kStages, SB = C::kStageBytes;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    uint64_t* full = reinterpret_cast<uint64_t*>(smem + STAGES * STAGE_BYTES);
-    uint64_t* conv = full + STAGES;  // MODE 1: B tile converted to fp16
+    uint64_t* full = reinterpret_cast<uint64_t*>(smem + STAGES * SB);
+    uint64_t* conv = full + STAGES;  // B tile transformed (fp16) and ready for the MMA
     uint64_t* empty = conv + STAGES;
     uint64_t* tfull = empty + STAGES;
     uint64_t* tempty = tfull + 2;
     uint64_t* drain = tempty + 2;
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+    uint64_t* ufull = drain + 1;  // unit ring: slot holds the next claimed unit
+    uint64_t* uempty = ufull + UR;
+    volatile int* unit_ring = reinterpret_cast<volatile int*>(uempty + UR);
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(const_cast<int*>(unit_ring) + UR);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -124,6 +243,10 @@ __global__ void __launch_bounds__(Roles<MODE>::kThreads, 1)
             mbar_init(tfull + a, 1);
             mbar_init(tempty + a, 4);
         }
+        for (int r = 0; r < UR; ++r) {
+            mbar_init(ufull + r, 1);
+            mbar_init(uempty + r, C::kUnitReaders);
+        }
         mbar_init(drain, 1);
         *abort_flag = 0;
         fence_mbar_init();
@@ -131,7 +254,11 @@ __global__ void __launch_bounds__(Roles<MODE>::kThreads, 1)
     if (warp == 0 && lane == 0) {
         tma_prefetch_desc(&tmA);
         tma_prefetch_desc(&tmB0);
-        if (MODE == 0) tma_prefetch_desc(&tmB1);
+        tma_prefetch_desc(&tmB1);
+        if (Q4) {
+            tma_prefetch_desc(&tmS0);
+            tma_prefetch_desc(&tmS1);
+        }
     }
     if (warp == 1) {
         tmem_alloc(tmem_slot, TMEM_COLS);
@@ -150,7 +277,16 @@ __global__ void __launch_bounds__(Roles<MODE>::kThreads, 1)
         int stage = 0;
         uint32_t phase = 0, issued = 0, issued_par = 0;
         bool ok = true;
-        for (int u = blockIdx.x; ok && u < total_units; u += gridDim.x) {
+        int uslot = 0;
+        uint32_t uphase = 0;
+        while (ok) {
+            int u = -1;
+            if (!ring_publish(u, uslot, uphase, p.unit_counter, total_units, unit_ring, ufull, uempty, abort_flag, p.err,
+                              p.wait_ns)) {
+                ok = false;
+                break;
+            }
+            if (u < 0) break;
             const Unit U = decode_unit(u, p);
             const bool sh = U.e >= p.E;
             const int z = sh ? 0 : U.e;
@@ -163,11 +299,26 @@ __global__ void __launch_bounds__(Roles<MODE>::kThreads, 1)
                     break;
                 }
                 if (lane == 0) {
-                    uint8_t* sa = smem + stage * STAGE_BYTES;
+                    uint8_t* sa = smem + stage * SB;
                     uint8_t* sb = sa + A_BYTES;
-                    mbar_arrive_expect_tx(full + stage, STAGE_BYTES);
+                    mbar_arrive_expect_tx(full + stage, C::kTxBytes);
                     tma_load_2d(sa, &tmA, full + stage, kb * BK, U.row0);
-                    if (MODE == 0) {
+                    if (Q4) {
+                        // packed rows [N][32 B] and scales [2 groups][rows] fp16
+                        uint8_t* sp = sb + B_BYTES;
+                        uint8_t* ss = sp + P_BYTES;
+                        if (MODE == 0) {
+                            const int n0 = U.n * 128;
+                            tma_load_3d(sp, &tmB0, full + stage, kb * (BK / 2), n0, z);
+                            tma_load_3d(sp + P_BYTES / 2, &tmB1, full + stage, kb * (BK / 2), n0, z);
+                            tma_load_3d(ss, &tmS0, full + stage, n0, kb * 2, z);
+                            tma_load_3d(ss + S_BYTES / 2, &tmS1, full + stage, n0, kb * 2, z);
+                        } else {
+                            const int n0 = U.n * BN;
+                            tma_load_3d(sp, &tmB0, full + stage, kb * (BK / 2), n0, z);
+                            tma_load_3d(ss, &tmS0, full + stage, n0, kb * 2, z);
+                        }
+                    } else if (MODE == 0) {
                         const CUtensorMap* mg = sh ? &tmS0 : &tmB0;
                         const CUtensorMap* mu = sh ? &tmS1 : &tmB1;
                         const int n0 = U.n * 128;
@@ -198,18 +349,24 @@ __global__ void __launch_bounds__(Roles<MODE>::kThreads, 1)
         __syncwarp();
     } else if (warp == 1) {
         // ------------------------------------------------ MMA issuer
-        constexpr uint32_t IDESC = Roles<MODE>::kIdesc;
-        uint64_t* ready = MODE == 0 ? full : conv;
+        constexpr uint32_t IDESC = C::kIdesc;
+        uint64_t* ready = C::kTransform ? conv : full;
         int stage = 0, acc = 0;
         uint32_t phase = 0, acc_phase = 0;
         bool ok = true;
-        for (int u = blockIdx.x; ok && u < total_units; u += gridDim.x) {
+        int uslot = 0;
+        uint32_t uphase = 0;
+        while (ok) {
+            int u = -1;
+            if (!ring_read(u, uslot, uphase, unit_ring, ufull, uempty, abort_flag, p.err, p.wait_ns)) break;
+            if (u < 0) break;
             int okl = 1;
             if (lane == 0) okl = mbar_wait_bounded(tempty + acc, acc_phase ^ 1u, abort_flag, p.err, p.wait_ns);
             okl = __shfl_sync(0xFFFFFFFFu, okl, 0);
             if (!okl) break;
             tc_fence_after();
             const uint32_t d_tmem = tmem_base + uint32_t(acc * BN);
+            const uint32_t idesc = decode_unit(u, p).rows <= 64 ? C::kIdesc64 : IDESC;
             for (int kb = 0; kb < KB; ++kb) {
                 if (lane == 0) okl = mbar_wait_bounded(ready + stage, phase, abort_flag, p.err, p.wait_ns);
                 okl = __shfl_sync(0xFFFFFFFFu, okl, 0);
@@ -219,15 +376,17 @@ __global__ void __launch_bounds__(Roles<MODE>::kThreads, 1)
                 }
                 tc_fence_after();
                 if (lane == 0) {
-                    const uint32_t a0 = smem_u32(smem + stage * STAGE_BYTES);
+                    const uint32_t a0 = smem_u32(smem + stage * SB);
                     const uint32_t b0 = a0 + A_BYTES;
 #pragma unroll
                     for (int j = 0; j < BK / 16; ++j) {
                         // A: K-major, advance 16 elements = 32 bytes inside the swizzle row.
-                        // B: N-major, advance 16 K-rows = 2 KB (two 8-row groups).
+                        // B: N-major (bf16 weights): advance 16 K-rows = 2 KB;
+                        //    K-major (dequantised Q4G32): like A.
                         const uint64_t ad = sdesc_sw128(a0 + j * 32, 16, 1024);
-                        const uint64_t bd = sdesc_sw128(b0 + j * 2048, B_CHUNK, 1024);
-                        umma_bf16(d_tmem, ad, bd, IDESC, (kb | j) != 0);
+                        const uint64_t bd = Q4 ? sdesc_sw128(b0 + j * 32, 16, 1024)
+                                               : sdesc_sw128(b0 + j * 2048, B_CHUNK, 1024);
+                        umma_bf16(d_tmem, ad, bd, idesc, (kb | j) != 0);
                     }
                     umma_commit(empty + stage);
                 }
@@ -257,15 +416,23 @@ __global__ void __launch_bounds__(Roles<MODE>::kThreads, 1)
         int acc = 0;
         uint32_t acc_phase = 0;
         bool range_bad = false;
-        for (int u = blockIdx.x; u < total_units; u += gridDim.x) {
+        int uslot = 0;
+        uint32_t uphase = 0;
+        while (true) {
+            int u = -1;
+            if (!ring_read(u, uslot, uphase, unit_ring, ufull, uempty, abort_flag, p.err, p.wait_ns)) break;
+            if (u < 0) break;
             const Unit U = decode_unit(u, p);
             int okl = 1;
             if (lane == 0) okl = mbar_wait_bounded(tfull + acc, acc_phase, abort_flag, p.err, p.wait_ns);
             okl = __shfl_sync(0xFFFFFFFFu, okl, 0);
             if (!okl) break;
             tc_fence_after();
-            const int rit = q * 32 + lane;
-            const bool valid = rit < U.rows;
+            // M=128: lane i of quadrant q is row 32q + i. M=64 (tiles of <= 64
+            // rows): only lanes 0-15 of each quadrant hold rows, 16q + i.
+            const bool m64 = U.rows <= 64;
+            const int rit = m64 ? q * 16 + lane : q * 32 + lane;
+            const bool valid = (!m64 || lane < 16) && rit < U.rows;
             const int64_t row = int64_t(U.row0) + rit;
             const uint32_t tb = tmem_base + (uint32_t(q * 32) << 16) + uint32_t(acc * BN);
             if (MODE == 0) {
@@ -326,13 +493,18 @@ __global__ void __launch_bounds__(Roles<MODE>::kThreads, 1)
             }
         }
         if (range_bad) set_error(p.err, MOE_DEVERR_RANGE);
-    } else if (MODE == 1) {
-        // ------------------------------------------------ converters (warps 6..9): W_down bf16 -> fp16
-        const int ct = threadIdx.x - 192;
+    } else if (C::kTransform) {
+        // ------------------------------------------------ transform (warps 6..9)
+        const int ct = threadIdx.x - 192;  // 0..127
         int stage = 0;
         uint32_t phase = 0;
         bool ok = true;
-        for (int u = blockIdx.x; ok && u < total_units; u += gridDim.x) {
+        int uslot = 0;
+        uint32_t uphase = 0;
+        while (ok) {
+            int u = -1;
+            if (!ring_read(u, uslot, uphase, unit_ring, ufull, uempty, abort_flag, p.err, p.wait_ns)) break;
+            if (u < 0) break;
             for (int kb = 0; kb < KB; ++kb) {
                 int okl = 1;
                 if (lane == 0) okl = mbar_wait_bounded(full + stage, phase, abort_flag, p.err, p.wait_ns);
@@ -341,15 +513,40 @@ __global__ void __launch_bounds__(Roles<MODE>::kThreads, 1)
                     ok = false;
                     break;
                 }
-                uint4* b = reinterpret_cast<uint4*>(smem + stage * STAGE_BYTES + A_BYTES);
+                uint8_t* sb = smem + stage * SB + A_BYTES;
+                if (Q4) {
+                    // rows ct and ct+128 of the 256-row B tile; row r: 8 words
+                    // (k 0..63) -> 8 chunks of 8 fp16 at r*128 + ((c ^ (r%8)) * 16)
+                    const uint8_t* sp = sb + B_BYTES;
+                    const uint16_t* ss = reinterpret_cast<const uint16_t*>(sp + P_BYTES);
+#pragma unroll
+                    for (int h = 0; h < 2; ++h) {
+                        const int r = ct + 128 * h;
+                        // scales [2 groups][rows]: MODE 0 holds gate rows then up rows (128 each)
+                        const uint16_t* sr = MODE == 0 ? ss + h * 256 + (r & 127) : ss + r;
+                        const int gstride = MODE == 0 ? 128 : 256;
+                        const uint32_t s0 = sr[0], s1 = sr[gstride];
+                        const uint32_t s0x2 = s0 | (s0 << 16), s1x2 = s1 | (s1 << 16);
+                        const uint4 w0 = reinterpret_cast<const uint4*>(sp + r * 32)[0];
+                        const uint4 w1 = reinterpret_cast<const uint4*>(sp + r * 32)[1];
+                        const uint32_t words[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
+                        uint8_t* row = sb + r * 128;
+#pragma unroll
+                        for (int c = 0; c < 8; ++c)
+                            *reinterpret_cast<uint4*>(row + ((c ^ (r & 7)) << 4)) = dequant_word(words[c], c < 4 ? s0x2 : s1x2);
+                    }
+                } else {
+                    // bf16 -> fp16 in place (position-independent)
+                    uint4* b = reinterpret_cast<uint4*>(sb);
 #pragma unroll 4
-                for (int i = ct; i < B_BYTES / 16; i += 128) {
-                    uint4 v = b[i];
-                    v.x = bf16x2_to_f16x2(v.x);
-                    v.y = bf16x2_to_f16x2(v.y);
-                    v.z = bf16x2_to_f16x2(v.z);
-                    v.w = bf16x2_to_f16x2(v.w);
-                    b[i] = v;
+                    for (int i = ct; i < B_BYTES / 16; i += 128) {
+                        uint4 v = b[i];
+                        v.x = bf16x2_to_f16x2(v.x);
+                        v.y = bf16x2_to_f16x2(v.y);
+                        v.z = bf16x2_to_f16x2(v.z);
+                        v.w = bf16x2_to_f16x2(v.w);
+                        b[i] = v;
+                    }
                 }
                 fence_proxy_async_smem();  // generic-proxy writes -> visible to the tensor core
                 mbar_arrive(conv + stage);
@@ -418,12 +615,16 @@ __global__ void __launch_bounds__(512) schedule_kernel(const int32_t* __restrict
     if (e == 0) {
         tile_base[Etot] = tt;
         n_stream[0] = ts;
+        n_stream[1] = 0;  // unit counters of the two tcgen05 GEMMs (claimed with atomicAdd)
+        n_stream[2] = 0;
     }
 }
 
 // ---------------------------------------------------------------------------- S4 row gather
 
-// xg[r] = x[sorted_token[r]] for r < offsets[Etot]; 16-byte vectors.
+// xg[r] = x[sorted_token[r]] for r < offsets[Etot]; 16-byte vectors. TO_F16:
+// bf16 -> fp16 on the way (the Q4G32 path runs its MMAs in fp16).
+template <bool TO_F16>
 __global__ void __launch_bounds__(256) gather_rows_kernel(const uint16_t* __restrict__ x,
                                                           const int32_t* __restrict__ sorted_token,
                                                           const int32_t* __restrict__ offsets, int Etot, int d,
@@ -438,7 +639,14 @@ __global__ void __launch_bounds__(256) gather_rows_kernel(const uint16_t* __rest
             set_error(err, MOE_DEVERR_BOUNDS);
             continue;
         }
-        reinterpret_cast<uint4*>(xg + r * d)[c] = __ldg(reinterpret_cast<const uint4*>(x + int64_t(t) * d) + c);
+        uint4 v = __ldg(reinterpret_cast<const uint4*>(x + int64_t(t) * d) + c);
+        if (TO_F16) {
+            v.x = bf16x2_to_f16x2(v.x);
+            v.y = bf16x2_to_f16x2(v.y);
+            v.z = bf16x2_to_f16x2(v.z);
+            v.w = bf16x2_to_f16x2(v.w);
+        }
+        reinterpret_cast<uint4*>(xg + r * d)[c] = v;
     }
 }
 
@@ -463,9 +671,9 @@ static EncodeTiledFn get_encode() {
     return fn;
 }
 
-// bf16 tensor map; dims/strides innermost first; box {64, box1, 1...}; 128-byte swizzle.
-static bool make_map(CUtensorMap* m, const void* base, int rank, const uint64_t* dims, const uint64_t* strides_bytes,
-                     const uint32_t* box) {
+// dims/strides innermost first (strides in bytes, rank-1 of them).
+static bool make_map(CUtensorMap* m, CUtensorMapDataType dt, const void* base, int rank, const uint64_t* dims,
+                     const uint64_t* strides_bytes, const uint32_t* box, CUtensorMapSwizzle swz) {
     EncodeTiledFn enc = get_encode();
     if (!enc) return false;
     cuuint64_t gd[3], gs[2];
@@ -475,42 +683,56 @@ static bool make_map(CUtensorMap* m, const void* base, int rank, const uint64_t*
         bx[i] = box[i];
     }
     for (int i = 0; i < rank - 1; ++i) gs[i] = strides_bytes[i];
-    const CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, rank, const_cast<void*>(base), gd, gs, bx, es,
-                           CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+    const CUresult r = enc(m, dt, rank, const_cast<void*>(base), gd, gs, bx, es, CU_TENSOR_MAP_INTERLEAVE_NONE, swz,
                            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     return r == CUDA_SUCCESS;
 }
 
-// A operand: rows x K bf16 row-major; box 64 (K) x 128 (rows).
+// A operand: rows x K 2-byte elements, row-major; box 64 (K) x 128 (rows), 128-byte swizzle.
 bool map_rows(CUtensorMap* m, const void* base, int64_t rows, int K) {
     const uint64_t dims[2] = {uint64_t(K), uint64_t(rows)};
     const uint64_t str[1] = {uint64_t(K) * 2};
     const uint32_t box[2] = {64, 128};
-    return make_map(m, base, 2, dims, str, box);
+    return make_map(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, base, 2, dims, str, box, CU_TENSOR_MAP_SWIZZLE_128B);
 }
-// B operand: [nexp, K, N] bf16 row-major; box 64 (N) x 64 (K) x 1.
+// bf16 B operand: [nexp, K, N] row-major; box 64 (N) x 64 (K) x 1, 128-byte swizzle.
 bool map_weights(CUtensorMap* m, const void* base, int nexp, int K, int N) {
     const uint64_t dims[3] = {uint64_t(N), uint64_t(K), uint64_t(nexp)};
     const uint64_t str[2] = {uint64_t(N) * 2, uint64_t(N) * uint64_t(K) * 2};
     const uint32_t box[3] = {64, 64, 1};
-    return make_map(m, base, 3, dims, str, box);
+    return make_map(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, base, 3, dims, str, box, CU_TENSOR_MAP_SWIZZLE_128B);
+}
+// Q4G32 nibbles: [nexp, N, K/2] bytes; box 32 bytes (64 k) x rows x 1, no swizzle.
+bool map_q4_packed(CUtensorMap* m, const void* base, int nexp, int K, int N, int rows) {
+    const uint64_t dims[3] = {uint64_t(K / 2), uint64_t(N), uint64_t(nexp)};
+    const uint64_t str[2] = {uint64_t(K / 2), uint64_t(N) * uint64_t(K / 2)};
+    const uint32_t box[3] = {32, uint32_t(rows), 1};
+    return make_map(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, base, 3, dims, str, box, CU_TENSOR_MAP_SWIZZLE_NONE);
+}
+// Q4G32 scales: [nexp, K/32, N] fp16; box rows (N) x 2 groups x 1, no swizzle.
+bool map_q4_scales(CUtensorMap* m, const void* base, int nexp, int K, int N, int rows) {
+    const uint64_t dims[3] = {uint64_t(N), uint64_t(K / 32), uint64_t(nexp)};
+    const uint64_t str[2] = {uint64_t(N) * 2, uint64_t(N) * uint64_t(K / 32) * 2};
+    const uint32_t box[3] = {uint32_t(rows), 2, 1};
+    return make_map(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, base, 3, dims, str, box, CU_TENSOR_MAP_SWIZZLE_NONE);
 }
 
-template <int MODE>
+template <int MODE, int WF>
 cudaError_t launch_gemm(const CUtensorMap& A, const CUtensorMap& B0, const CUtensorMap& B1, const CUtensorMap& S0,
                         const CUtensorMap& S1, const GemmParams& p, cudaStream_t s) {
+    using C = Cfg<MODE, WF>;
     static int configured_dev = -1;
     int dev = 0;
     cudaGetDevice(&dev);
     if (configured_dev != dev) {
-        cudaError_t e = cudaFuncSetAttribute(grouped_gemm_kernel<MODE>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                             SMEM_BYTES);
+        cudaError_t e = cudaFuncSetAttribute(grouped_gemm_kernel<MODE, WF>,
+                                             cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmem);
         if (e != cudaSuccess) return e;
         configured_dev = dev;
     }
     {
         ProfScope prof_(MODE == 0 ? MOE_K_TC_GATEUP : MOE_K_TC_DOWN, s);
-        grouped_gemm_kernel<MODE><<<num_sms(), Roles<MODE>::kThreads, SMEM_BYTES, s>>>(A, B0, B1, S0, S1, p);
+        grouped_gemm_kernel<MODE, WF><<<num_sms(), C::kThreads, C::kSmem, s>>>(A, B0, B1, S0, S1, p);
     }
     return cudaGetLastError();
 }
@@ -536,20 +758,56 @@ cudaError_t launch_gather(const Dims& D, const uint16_t* x, const int32_t* sorte
     if (blocks < 1) blocks = 1;
     {
         ProfScope prof_(MOE_K_GATHER, s);
-        gather_rows_kernel<<<int(blocks), 256, 0, s>>>(x, sorted_token, offsets, D.Etot, D.d, D.T, xg, err);
+        if (D.fmt == MOE_WEIGHTS_Q4G32)
+            gather_rows_kernel<true><<<int(blocks), 256, 0, s>>>(x, sorted_token, offsets, D.Etot, D.d, D.T, xg, err);
+        else
+            gather_rows_kernel<false><<<int(blocks), 256, 0, s>>>(x, sorted_token, offsets, D.Etot, D.d, D.T, xg, err);
     }
     return cudaGetLastError();
 }
 
-// Both tcgen05 GEMMs of the tile variant. h: [rows, f] bf16 scratch.
+// Both tcgen05 GEMMs of the tile variant. xg: the gathered rows (bf16, or
+// fp16 for Q4G32); h: [rows, f] fp16 scratch.
 cudaError_t launch_tensor_ffn(const Dims& D, const uint16_t* xg, uint16_t* h, const int32_t* tile_base,
-                              const int32_t* offsets, const int32_t* sorted_pair, const float* topk_w,
-                              const moe_weights* w, uint16_t* y_rows, uint32_t* err, uint64_t wait_ns,
+                              const int32_t* offsets,
+                              const int32_t* sorted_pair, const float* topk_w, const moe_weights* w,
+                              uint16_t* y_rows, int32_t* counters, uint32_t* err, uint64_t wait_ns,
                               cudaStream_t s) {
     using namespace tc;
-    CUtensorMap mA, mG, mU, mSG, mSU, mH, mD, mSD;
-    if (!map_rows(&mA, xg, D.rows, D.d) || !map_weights(&mG, w->w_gate, D.E, D.d, D.f) ||
-        !map_weights(&mU, w->w_up, D.E, D.d, D.f) || !map_rows(&mH, h, D.rows, D.f) ||
+    GemmParams p{};
+    p.E = D.E;
+    p.Etot = D.Etot;
+    p.tile_base = tile_base;
+    p.offsets = offsets;
+    p.sorted_pair = sorted_pair;
+    p.topk_w = topk_w;
+    p.limit = D.limit;
+    p.err = err;
+    p.wait_ns = wait_ns;
+    CUtensorMap mA, mH;
+    if (!map_rows(&mA, xg, D.rows, D.d) || !map_rows(&mH, h, D.rows, D.f)) return cudaErrorInvalidValue;
+    cudaError_t e;
+    if (D.fmt == MOE_WEIGHTS_Q4G32) {
+        CUtensorMap pg, pu, sg, su, pd, sd;
+        if (!map_q4_packed(&pg, w->w_gate, D.E, D.d, D.f, 128) || !map_q4_packed(&pu, w->w_up, D.E, D.d, D.f, 128) ||
+            !map_q4_scales(&sg, w->s_gate, D.E, D.d, D.f, 128) || !map_q4_scales(&su, w->s_up, D.E, D.d, D.f, 128) ||
+            !map_q4_packed(&pd, w->w_down, D.E, D.f, D.d, BN) || !map_q4_scales(&sd, w->s_down, D.E, D.f, D.d, BN))
+            return cudaErrorInvalidValue;
+        p.K = D.d;
+        p.n_out = D.f;
+        p.n_tiles = (D.f + 127) / 128;
+        p.out = h;
+        p.unit_counter = counters;
+        if ((e = launch_gemm<0, 1>(mA, pg, pu, sg, su, p, s)) != cudaSuccess) return e;
+        p.K = D.f;
+        p.n_out = D.d;
+        p.n_tiles = (D.d + BN - 1) / BN;
+        p.out = y_rows;
+        p.unit_counter = counters + 1;
+        return launch_gemm<1, 1>(mH, pd, pd, sd, sd, p, s);
+    }
+    CUtensorMap mG, mU, mSG, mSU, mD, mSD;
+    if (!map_weights(&mG, w->w_gate, D.E, D.d, D.f) || !map_weights(&mU, w->w_up, D.E, D.d, D.f) ||
         !map_weights(&mD, w->w_down, D.E, D.f, D.d))
         return cudaErrorInvalidValue;
     if (D.has_shared) {
@@ -561,29 +819,20 @@ cudaError_t launch_tensor_ffn(const Dims& D, const uint16_t* xg, uint16_t* h, co
         mSU = mU;
         mSD = mD;
     }
-    GemmParams p{};
-    p.E = D.E;
-    p.Etot = D.Etot;
-    p.tile_base = tile_base;
-    p.offsets = offsets;
-    p.sorted_pair = sorted_pair;
-    p.topk_w = topk_w;
-    p.limit = D.limit;
-    p.err = err;
-    p.wait_ns = wait_ns;
     // S5: gate/up + SwiGLU -> h
     p.K = D.d;
     p.n_out = D.f;
     p.n_tiles = (D.f + 127) / 128;
     p.out = h;
-    cudaError_t e = launch_gemm<0>(mA, mG, mU, mSG, mSU, p, s);
-    if (e != cudaSuccess) return e;
+    p.unit_counter = counters;
+    if ((e = launch_gemm<0, 0>(mA, mG, mU, mSG, mSU, p, s)) != cudaSuccess) return e;
     // S6: down + gate scale -> y_rows
     p.K = D.f;
     p.n_out = D.d;
     p.n_tiles = (D.d + BN - 1) / BN;
     p.out = y_rows;
-    return launch_gemm<1>(mH, mD, mD, mSD, mSD, p, s);
+    p.unit_counter = counters + 1;
+    return D.down_f16 ? launch_gemm<1, 2>(mH, mD, mD, mSD, mSD, p, s) : launch_gemm<1, 0>(mH, mD, mD, mSD, mSD, p, s);
 }
 
 }  // namespace moe

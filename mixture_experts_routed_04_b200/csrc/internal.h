@@ -11,7 +11,8 @@ constexpr int kPermWarps = 8;                         // warps per permutation b
 constexpr int kPermPairsPerWarp = 256;                // 8 rounds of 32 pairs
 constexpr int kPermPairsPerBlock = kPermWarps * kPermPairsPerWarp;
 constexpr int kTileM = 128;                           // rows per tcgen05 tile
-constexpr int kDefaultStreamMaxRows = 16;             // AUTO threshold (rows per expert)
+constexpr int kStreamRowsFewExperts = 8;             // AUTO: streaming threshold when few experts are touched
+constexpr int kSmCountB200 = 148;
 
 // Everything a call derives from moe_params on the host.
 struct Dims {
@@ -25,6 +26,7 @@ struct Dims {
     float limit;
     int ks;                   // K-split of the streaming gate/up kernel
     int out_bf16;             // layer output in bf16 (else fp32)
+    int down_f16;             // W_down given as fp16 (prepared at load time)
 };
 
 // Byte offsets of every scratch array inside a workspace (0 = absent).

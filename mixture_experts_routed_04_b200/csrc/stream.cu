@@ -8,55 +8,53 @@
 // "Strata PR #4366" — the light kernels own experts with at most 16 rows;
 // "TensorFold PR #1607" — K-parallel tiles for plans with few pairs per item.
 //
-// Work unit = (expert, 64 output columns, K slice). One CTA per SM, persistent:
-//   warp 0     TMA producer: 64 K-rows x 64 columns (128-byte swizzle) of the
-//              weight matrix (gate and up, or down) per stage, 128 KB ring.
-//   warps 1-4  consumers, 16 columns each: ldmatrix.trans turns a stored
-//              [k][n] tile into the A operand (16 n x 16 k) of mma.sync
-//              m16n8k16 (bf16 in, fp32 accumulate); the expert's rows (<= 8
-//              per chunk, from shared memory) are the N=8 operand. The tensor
-//              pipe is almost idle: it only keeps the instruction count per
-//              weight byte low so the kernel stays HBM-bound.
+// Work item = (expert, 64 output columns, K slice, chunk of <= 8 rows). One
+// CTA per SM, persistent, everything through one TMA ring (128 KB):
+//   warp 0     TMA producer: per 64-K block, the 64 x 64 weight tile(s) (gate
+//              and up, or down; 128-byte swizzle) and the 8 x 64 tile of the
+//              chunk's rows (gathered x, or h; 128-byte swizzle).
+//   warps 1-4  consumers, 16 columns each: ldmatrix.trans turns the stored
+//              [k][n] weight tile into the A operand (16 n x 16 k) of mma.sync
+//              m16n8k16; the rows tile gives the N=8 operand. fp32 accumulate.
+//              The tensor pipe only keeps the instruction count per weight byte
+//              low so the kernel stays HBM-bound.
 // Gate/up (bf16 x and weights) with one K slice applies the clamped SwiGLU and
 // writes h (fp16); with several, fp32 partials go to the workspace and
-// stream_reduce finishes (fixed order, deterministic). Down runs in fp16: the
-// W_down fragments are converted bf16 -> fp16 in registers after ldmatrix, h
-// is fp16; it writes y = w_pair * (h W_down) (fp16).
-// All waits are bounded; no TMA multicast.
+// stream_reduce finishes (fixed order, deterministic). Down runs in fp16 (h is
+// fp16; W_down prepared as fp16, or converted in registers after ldmatrix) and
+// writes y = w_pair * (h W_down) (fp16). All waits are bounded; no TMA
+// multicast; no named barriers, so an abort never strands a warp.
 #include "internal.h"
 
 namespace moe {
 
 namespace st {
 
-constexpr int NS = 64;               // output columns per unit
+constexpr int NS = 64;               // output columns per work item
 constexpr int BKS = 64;              // K-rows per stage
-constexpr int TILE = BKS * NS * 2;   // 8 KB
-constexpr int RING = 128 * 1024;     // weight ring
+constexpr int TILE = BKS * NS * 2;   // weight tile, 8 KB
+constexpr int XT = 8 * BKS * 2;      // rows tile (8 rows x 64 K), 1 KB
+constexpr int RING = 128 * 1024;
 constexpr int CONSUMERS = 4;
 constexpr int THREADS = 32 * (CONSUMERS + 1);
 constexpr int RC = 8;                // rows per chunk (mma N)
-constexpr int MAX_KSLICE = 2048;
-constexpr int XS_STRIDE = MAX_KSLICE + 8;  // bf16 elements per staged row (16-byte pad)
-constexpr int SMEM_BYTES = 1024 + RING + RC * XS_STRIDE * 2 + 512;
+constexpr int SMEM_BYTES = 1024 + RING + 512;
 
 struct StreamParams {
     int mode;            // 0: gate/up, 1: down
     int K, N;            // full reduction length and output width of the matrix
-    int kslice, ks;      // K per unit and number of K slices
+    int kslice, ks;      // K per item and number of K slices
     int E;
     const int32_t* offsets;
     const int32_t* stream_list;
     const int32_t* n_stream;
-    const int32_t* sorted_token;
     const int32_t* sorted_pair;
     const float* topk_w;
-    const uint16_t* src;  // mode 0: x [T, d]; mode 1: h [rows, f]
-    int T;
     uint16_t* out;        // mode 0: h [rows, f]; mode 1: y_rows [rows, d]
     float* part;          // mode 0 with ks > 1: [ks, 2, rows, f] fp32
     int64_t rows;
     float limit;
+    int down_f16;         // mode 1: W_down already fp16 (no conversion)
     uint32_t* err;
     uint64_t wait_ns;
 };
@@ -114,21 +112,18 @@ MOE_DEV void mma_f16_16816(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2,
 
 MOE_DEV uint16_t to_f16(float v) { return uint16_t(pack_f16x2(v, 0.f) & 0xFFFFu); }
 
-MOE_DEV void consumer_sync() { asm volatile("bar.sync 1, %0;" ::"n"(CONSUMERS * 32) : "memory"); }
-
-// MODE 0: two matrices (gate, up) per stage; MODE 1: one (down).
+// MODE 0: two weight tiles (gate, up) per stage; MODE 1: one (down). Plus the rows tile.
 template <int MODE>
 __global__ void __launch_bounds__(THREADS, 1)
     stream_kernel(const __grid_constant__ CUtensorMap tmW0, const __grid_constant__ CUtensorMap tmW1,
                   const __grid_constant__ CUtensorMap tmS0, const __grid_constant__ CUtensorMap tmS1,
-                  const StreamParams p) {
+                  const __grid_constant__ CUtensorMap tmX, const StreamParams p) {
     constexpr int NMAT = MODE == 0 ? 2 : 1;
-    constexpr int STAGE = NMAT * TILE;
+    constexpr int STAGE = NMAT * TILE + XT;  // 17 KB / 9 KB, 1 KB aligned
     constexpr int STAGES = RING / STAGE;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    uint16_t* xs = reinterpret_cast<uint16_t*>(smem + RING);
-    uint64_t* full = reinterpret_cast<uint64_t*>(smem + RING + RC * XS_STRIDE * 2);
+    uint64_t* full = reinterpret_cast<uint64_t*>(smem + RING);
     uint64_t* empty = full + STAGES;
     volatile int* abort_flag = reinterpret_cast<volatile int*>(empty + STAGES);
 
@@ -154,7 +149,7 @@ __global__ void __launch_bounds__(THREADS, 1)
         for (int u = blockIdx.x; ok && u < total; u += gridDim.x) {
             const SUnit U = decode(u, p);
             const bool sh = U.e >= p.E;
-            const int ybase = (sh ? 0 : U.e * p.K) + U.k0;
+            const int wrow = (sh ? 0 : U.e * p.K) + U.k0;  // weight row of k0 in the stacked [E*K, N] view
             const int nchunks = (U.nrows + RC - 1) / RC;
             for (int c = 0; ok && c < nchunks; ++c) {
                 for (int kb = 0; kb < KB; ++kb) {
@@ -168,8 +163,9 @@ __global__ void __launch_bounds__(THREADS, 1)
                     if (lane == 0) {
                         uint8_t* dst = smem + stage * STAGE;
                         mbar_arrive_expect_tx(full + stage, STAGE);
-                        tma_load_2d(dst, sh ? &tmS0 : &tmW0, full + stage, U.n0, ybase + kb * BKS);
-                        if (MODE == 0) tma_load_2d(dst + TILE, sh ? &tmS1 : &tmW1, full + stage, U.n0, ybase + kb * BKS);
+                        tma_load_2d(dst, sh ? &tmS0 : &tmW0, full + stage, U.n0, wrow + kb * BKS);
+                        if (MODE == 0) tma_load_2d(dst + TILE, sh ? &tmS1 : &tmW1, full + stage, U.n0, wrow + kb * BKS);
+                        tma_load_2d(dst + NMAT * TILE, &tmX, full + stage, U.k0 + kb * BKS, U.row0 + c * RC);
                         issued |= 1u << stage;
                         issued_par = (issued_par & ~(1u << stage)) | (phase << stage);
                     }
@@ -180,50 +176,28 @@ __global__ void __launch_bounds__(THREADS, 1)
                 }
             }
         }
+        // On abort, let every copy already issued land before the CTA can exit.
         if (!ok && lane == 0) {
             for (int s = 0; s < STAGES; ++s)
                 if (issued >> s & 1u) mbar_wait_bounded(full + s, (issued_par >> s) & 1u, nullptr, p.err, kDrainLimitNs);
         }
         __syncwarp();
-        return;  // the producer takes no part in the consumers' named barrier
+        return;
     }
 
     // ---------------------------------------------------- consumers (warps 1..4)
-    const int cw = warp - 1;           // columns cw*16 .. cw*16+15 of the unit
-    const int ctid = threadIdx.x - 32;  // 0..127
+    const int cw = warp - 1;  // columns cw*16 .. cw*16+15 of the item
     const int gid = lane >> 2, tig = lane & 3;
-    // After an abort, `ok` turns false and the warp stops waiting and computing,
-    // but it still walks the same units and chunks, so every consumer warp
-    // passes the same sequence of named barriers and none is left waiting.
     int stage = 0;
     uint32_t phase = 0;
     bool ok = true, range_bad = false;
-    for (int u = blockIdx.x; u < total; u += gridDim.x) {
+    for (int u = blockIdx.x; ok && u < total; u += gridDim.x) {
         const SUnit U = decode(u, p);
         const int nchunks = (U.nrows + RC - 1) / RC;
-        for (int c = 0; c < nchunks; ++c) {
+        for (int c = 0; ok && c < nchunks; ++c) {
             const int rc = min(RC, U.nrows - c * RC);
-            // stage this chunk's rows (K slice) in shared memory
-            consumer_sync();
-            const int vpr = p.kslice / 8;
-            for (int i = ctid; ok && i < rc * vpr; i += CONSUMERS * 32) {
-                const int r = i / vpr, cc = i - r * vpr;
-                const int64_t row = int64_t(U.row0) + c * RC + r;
-                int64_t src_row = row;
-                if (MODE == 0) {
-                    src_row = __ldg(p.sorted_token + row);
-                    if (src_row < 0 || src_row >= p.T) {
-                        set_error(p.err, MOE_DEVERR_BOUNDS);
-                        src_row = 0;
-                    }
-                }
-                const uint4 v = __ldg(reinterpret_cast<const uint4*>(p.src + src_row * p.K + U.k0) + cc);
-                *reinterpret_cast<uint4*>(xs + r * XS_STRIDE + cc * 8) = v;
-            }
-            consumer_sync();
-
             float acc0[4] = {0.f, 0.f, 0.f, 0.f}, acc1[4] = {0.f, 0.f, 0.f, 0.f};
-            for (int kb = 0; ok && kb < KB; ++kb) {
+            for (int kb = 0; kb < KB; ++kb) {
                 int okl = 1;
                 if (lane == 0) okl = mbar_wait_bounded(full + stage, phase, abort_flag, p.err, p.wait_ns);
                 okl = __shfl_sync(0xFFFFFFFFu, okl, 0);
@@ -232,16 +206,20 @@ __global__ void __launch_bounds__(THREADS, 1)
                     break;
                 }
                 const uint32_t base0 = smem_u32(smem + stage * STAGE);
+                const uint8_t* xt = smem + stage * STAGE + NMAT * TILE;  // rows tile: row r, k at swizzled spot
 #pragma unroll
                 for (int k16 = 0; k16 < BKS / 16; ++k16) {
-                    // lane l addresses row (l%8) of 8x8 matrix (l/8): k = k16*16 + 8*(l/16) + l%8,
+                    // weight tile: lane l addresses row (l%8) of 8x8 matrix (l/8): k = k16*16 + 8*(l/16) + l%8,
                     // 16-byte chunk 2*cw + (l/8)%2, stored at chunk ^ (k % 8) (128-byte swizzle)
                     const int kr = k16 * 16 + ((lane >> 4) << 3) + (lane & 7);
                     const int ch = (2 * cw + ((lane >> 3) & 1)) ^ (kr & 7);
                     const uint32_t off = uint32_t(kr * 128 + ch * 16);
-                    const int kx = kb * BKS + k16 * 16 + 2 * tig;
-                    const uint32_t b0 = *reinterpret_cast<const uint32_t*>(xs + gid * XS_STRIDE + kx);
-                    const uint32_t b1 = *reinterpret_cast<const uint32_t*>(xs + gid * XS_STRIDE + kx + 8);
+                    // rows tile: row gid, k = k16*16 + 2*tig (+8): chunk (k/8) ^ gid
+                    const int kx = k16 * 16 + 2 * tig;
+                    const uint32_t b0 =
+                        *reinterpret_cast<const uint32_t*>(xt + gid * 128 + (((kx >> 3) ^ gid) << 4) + (kx & 7) * 2);
+                    const uint32_t b1 = *reinterpret_cast<const uint32_t*>(
+                        xt + gid * 128 + ((((kx + 8) >> 3) ^ gid) << 4) + ((kx + 8) & 7) * 2);
                     uint32_t a0, a1, a2, a3;
                     ldmatrix_x4_trans(base0 + off, a0, a1, a2, a3);
                     if (MODE == 0) {
@@ -249,6 +227,9 @@ __global__ void __launch_bounds__(THREADS, 1)
                         mma_bf16_16816(acc0, a0, a1, a2, a3, b0, b1);
                         ldmatrix_x4_trans(base0 + TILE + off, a0, a1, a2, a3);
                         mma_bf16_16816(acc1, a0, a1, a2, a3, b0, b1);
+                    } else if (p.down_f16) {
+                        // h (fp16) against W_down prepared as fp16
+                        mma_f16_16816(acc0, a0, a1, a2, a3, b0, b1);
                     } else {
                         // h (fp16) against W_down converted bf16 -> fp16 in registers
                         mma_f16_16816(acc0, bf16x2_to_f16x2(a0), bf16x2_to_f16x2(a1), bf16x2_to_f16x2(a2),
@@ -262,7 +243,7 @@ __global__ void __launch_bounds__(THREADS, 1)
                     phase ^= 1u;
                 }
             }
-            if (!ok) continue;
+            if (!ok) break;
             // acc[i]: column n = cw*16 + gid + 8*(i/2), row r = 2*tig + (i%2)
 #pragma unroll
             for (int i = 0; i < 4; ++i) {
@@ -336,13 +317,13 @@ static EncodeTiledFn get_encode() {
     return fn;
 }
 
-// 2-D map over a stack of row-major [K, N] bf16 matrices seen as [nexp*K, N]; box 64 x 64.
-static bool map_stack(CUtensorMap* m, const void* base, int64_t nrows, int N) {
+// 2-D map over a row-major [nrows, ncols] 2-byte matrix; box 64 (cols) x box_rows; 128-byte swizzle.
+static bool map_2d(CUtensorMap* m, const void* base, int64_t nrows, int ncols, int box_rows) {
     EncodeTiledFn enc = get_encode();
     if (!enc) return false;
-    cuuint64_t gd[2] = {cuuint64_t(N), cuuint64_t(nrows)};
-    cuuint64_t gs[1] = {cuuint64_t(N) * 2};
-    cuuint32_t bx[2] = {64, BKS}, es[2] = {1, 1};
+    cuuint64_t gd[2] = {cuuint64_t(ncols), cuuint64_t(nrows)};
+    cuuint64_t gs[1] = {cuuint64_t(ncols) * 2};
+    cuuint32_t bx[2] = {64, cuuint32_t(box_rows)}, es[2] = {1, 1};
     return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), gd, gs, bx, es,
                CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
@@ -350,7 +331,8 @@ static bool map_stack(CUtensorMap* m, const void* base, int64_t nrows, int N) {
 
 template <int MODE>
 static cudaError_t launch_one(const CUtensorMap& W0, const CUtensorMap& W1, const CUtensorMap& S0,
-                              const CUtensorMap& S1, const StreamParams& p, int grid, cudaStream_t s) {
+                              const CUtensorMap& S1, const CUtensorMap& X, const StreamParams& p, int grid,
+                              cudaStream_t s) {
     static int configured_dev = -1;
     int dev = 0;
     cudaGetDevice(&dev);
@@ -362,7 +344,7 @@ static cudaError_t launch_one(const CUtensorMap& W0, const CUtensorMap& W1, cons
     }
     {
         ProfScope prof_(MODE == 0 ? MOE_K_STREAM_GATEUP : MOE_K_STREAM_DOWN, s);
-        stream_kernel<MODE><<<grid, THREADS, SMEM_BYTES, s>>>(W0, W1, S0, S1, p);
+        stream_kernel<MODE><<<grid, THREADS, SMEM_BYTES, s>>>(W0, W1, S0, S1, X, p);
     }
     return cudaGetLastError();
 }
@@ -370,18 +352,20 @@ static cudaError_t launch_one(const CUtensorMap& W0, const CUtensorMap& W1, cons
 }  // namespace st
 
 // Gate/up (+ reduce) then down for the experts on the streaming list.
-cudaError_t launch_stream_ffn(const Dims& D, const uint16_t* x, uint16_t* h, float* part, const int32_t* offsets,
-                              const int32_t* stream_list, const int32_t* n_stream, const int32_t* sorted_token,
-                              const int32_t* sorted_pair, const float* topk_w, const moe_weights* w,
-                              uint16_t* y_rows, uint32_t* err, uint64_t wait_ns, cudaStream_t s) {
+// xg: the gathered rows [rows, d] (bf16); h: [rows, f] fp16.
+cudaError_t launch_stream_ffn(const Dims& D, const uint16_t* xg, uint16_t* h, float* part, const int32_t* offsets,
+                              const int32_t* stream_list, const int32_t* n_stream, const int32_t* sorted_pair,
+                              const float* topk_w, const moe_weights* w, uint16_t* y_rows, uint32_t* err,
+                              uint64_t wait_ns, cudaStream_t s) {
     using namespace st;
-    CUtensorMap mG, mU, mD, mSG, mSU, mSD;
-    if (!map_stack(&mG, w->w_gate, int64_t(D.E) * D.d, D.f) || !map_stack(&mU, w->w_up, int64_t(D.E) * D.d, D.f) ||
-        !map_stack(&mD, w->w_down, int64_t(D.E) * D.f, D.d))
+    CUtensorMap mG, mU, mD, mSG, mSU, mSD, mX, mH;
+    if (!map_2d(&mG, w->w_gate, int64_t(D.E) * D.d, D.f, BKS) || !map_2d(&mU, w->w_up, int64_t(D.E) * D.d, D.f, BKS) ||
+        !map_2d(&mD, w->w_down, int64_t(D.E) * D.f, D.d, BKS) || !map_2d(&mX, xg, D.rows, D.d, RC) ||
+        !map_2d(&mH, h, D.rows, D.f, RC))
         return cudaErrorInvalidValue;
     if (D.has_shared) {
-        if (!map_stack(&mSG, w->shared_gate, D.d, D.f) || !map_stack(&mSU, w->shared_up, D.d, D.f) ||
-            !map_stack(&mSD, w->shared_down, D.f, D.d))
+        if (!map_2d(&mSG, w->shared_gate, D.d, D.f, BKS) || !map_2d(&mSU, w->shared_up, D.d, D.f, BKS) ||
+            !map_2d(&mSD, w->shared_down, D.f, D.d, BKS))
             return cudaErrorInvalidValue;
     } else {
         mSG = mG;
@@ -394,12 +378,11 @@ cudaError_t launch_stream_ffn(const Dims& D, const uint16_t* x, uint16_t* h, flo
     p.offsets = offsets;
     p.stream_list = stream_list;
     p.n_stream = n_stream;
-    p.sorted_token = sorted_token;
     p.sorted_pair = sorted_pair;
     p.topk_w = topk_w;
-    p.T = D.T;
     p.rows = D.rows;
     p.limit = D.limit;
+    p.down_f16 = D.down_f16;
     p.err = err;
     p.wait_ns = wait_ns;
     // gate/up
@@ -408,17 +391,16 @@ cudaError_t launch_stream_ffn(const Dims& D, const uint16_t* x, uint16_t* h, flo
     p.N = D.f;
     p.ks = D.ks;
     p.kslice = D.d / D.ks;
-    p.src = x;
     p.out = h;
     p.part = part;
-    cudaError_t e = launch_one<0>(mG, mU, mSG, mSU, p, grid, s);
+    cudaError_t e = launch_one<0>(mG, mU, mSG, mSU, mX, p, grid, s);
     if (e != cudaSuccess) return e;
     if (D.ks > 1) {
         {
-        ProfScope prof_(MOE_K_STREAM_REDUCE, s);
-        stream_reduce_kernel<<<grid * 2, 256, 0, s>>>(part, D.ks, D.rows, D.f, offsets, stream_list, n_stream, D.limit,
-                                                      h, err);
-    }
+            ProfScope prof_(MOE_K_STREAM_REDUCE, s);
+            stream_reduce_kernel<<<grid * 2, 256, 0, s>>>(part, D.ks, D.rows, D.f, offsets, stream_list, n_stream,
+                                                          D.limit, h, err);
+        }
         if ((e = cudaGetLastError()) != cudaSuccess) return e;
     }
     // down
@@ -427,10 +409,9 @@ cudaError_t launch_stream_ffn(const Dims& D, const uint16_t* x, uint16_t* h, flo
     p.N = D.d;
     p.ks = 1;
     p.kslice = D.f;
-    p.src = h;
     p.out = y_rows;
     p.part = nullptr;
-    return launch_one<1>(mD, mD, mSD, mSD, p, grid, s);
+    return launch_one<1>(mD, mD, mSD, mSD, mH, p, grid, s);
 }
 
 }  // namespace moe

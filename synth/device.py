@@ -31,7 +31,7 @@ def upload(cfg: synth.LayerConfig, device="cuda", experts=None, threads: int = 8
         shapes = {"gate": (f, d), "up": (f, d), "down": (d, f)}  # [N, K]
         for w, (N, K) in shapes.items():
             pk = torch.zeros((E, N, K // 2), dtype=torch.uint8, device=device)
-            sc = torch.full((E, N, K // 32), float("nan"), dtype=torch.float16, device=device)
+            sc = torch.full((E, K // 32, N), float("nan"), dtype=torch.float16, device=device)
 
             def one(e, w=w, pk=pk, sc=sc):
                 p, s = synth.expert_q4_weights(cfg, e, w)

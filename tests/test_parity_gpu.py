@@ -3,14 +3,16 @@
 Bar: routing indices, counts, offsets, sorted lists and drop decisions are
 bit-exact; routing weights within 1e-6; the layer output (fp32) and the
 per-row expert outputs y_rows (fp16) within rel-L2 <= 1e-2 and
-max-abs <= 3e-2 * rms(reference); the bf16 output option within the same
-rel-L2 bound.
+max-abs <= 3e-2 * rms(reference); the bf16 output option is the fp32 output
+rounded once.
 
 Small layers (several M-tiles per expert, ragged tails, partial N-tiles) are
-compared element by element, on every kernel variant. The stated workloads are
-compared at full size in the launch configuration the benchmark times
-(moe_forward, automatic variant choice): routing and permutation in full,
-outputs on sampled tokens, each from its own definition in the oracle.
+compared element by element on every kernel variant and both forms of W_down
+(bf16 as given, fp16 prepared at load time). The stated workloads are compared
+at full size in the launch configuration the benchmark times (moe_forward,
+automatic variant choice, W_down prepared as fp16): routing and permutation in
+full, and every output element (the Q4G32 workload: outputs of sampled tokens,
+each from its own definition).
 """
 import numpy as np
 import pytest
@@ -37,6 +39,13 @@ SMALL = {
                                       f_shared=192),
     "zipf_small": synth.LayerConfig("zipf_small", T=512, d=256, f=256, E=32, k=4, bias="zipf"),
 }
+Q4_SMALL = {
+    "q4_tiny": synth.CONFIGS["tiny"].replace(name="q4_tiny", weight_format="q4g32"),
+    "q4_ragged": synth.LayerConfig("q4_ragged", T=700, d=192, f=320, E=6, k=3, weight_format="q4g32"),
+    "q4_zipf": synth.LayerConfig("q4_zipf", T=512, d=256, f=256, E=32, k=4, bias="zipf", weight_format="q4g32"),
+    "q4_capped": synth.LayerConfig("q4_capped", T=300, d=128, f=192, E=8, k=2, capacity_factor=0.9,
+                                   weight_format="q4g32"),
+}
 FULL = ["prompt", "capped", "decode1", "decode8", "decode32"]
 VARIANTS = {"auto": b.VARIANT_AUTO, "tensor": b.VARIANT_TENSOR, "stream": b.VARIANT_STREAM}
 
@@ -59,6 +68,15 @@ def f64(t):
 
 # --------------------------------------------------------------------------- oracle side
 
+def expert_ref(cfg, e, scale=1.0):
+    """(W_gate, W_up, W_down) float64 of expert e, as the layer's weights define them."""
+    if cfg.weight_format == "q4g32":
+        W = tuple(oracle.dequant_q4g32(*synth.expert_q4_weights(cfg, e, w)) for w in ("gate", "up", "down"))
+    else:
+        W = expert_f64(cfg, e)
+    return (W[0] * scale, W[1] * scale, W[2])
+
+
 _REF = {}
 
 
@@ -66,18 +84,14 @@ def reference(cfg, scale=1.0):
     key = (cfg, scale)
     if key not in _REF:
         x = synth.bf16_bits_to_f32(synth.x_bits(cfg)).astype(np.float64)
-        lg = synth.logits(cfg)
-        Ws = {e: tuple(w * (scale if i < 2 else 1.0) for i, w in enumerate(expert_f64(cfg, e)))
-              for e in range(cfg.E)}
         sh = shared_f64(cfg) if cfg.has_shared else None
-        out, it = oracle.forward(x, lg, cfg.k, Ws.__getitem__, cfg.swiglu_limit, cfg.capacity_factor, shared=sh)
-        _REF[key] = (out, it)
+        _REF[key] = oracle.forward(x, synth.logits(cfg), cfg.k, lambda e: expert_ref(cfg, e, scale),
+                                   cfg.swiglu_limit, cfg.capacity_factor, shared=sh)
     return _REF[key]
 
 
 def routing_reference(cfg):
-    lg = synth.logits(cfg)
-    idx, w = oracle.route(lg, cfg.k)
+    idx, w = oracle.route(synth.logits(cfg), cfg.k)
     cap = oracle.capacity(cfg.T, cfg.k, cfg.E, cfg.capacity_factor)
     perm = oracle.permute(idx, cfg.E, cap, shared_T=cfg.T if cfg.has_shared else 0)
     return idx, w, perm
@@ -97,17 +111,28 @@ def device_inputs(cfg, experts=None, scale=1.0):
         if scale != 1.0:
             d["w_gate"].mul_(scale)
             d["w_up"].mul_(scale)
+        if cfg.weight_format == "bf16":  # load-time fp16 copies of W_down
+            d["w_down_f16"] = b.prepare_down_f16(d["w_down"])
+            if cfg.has_shared:
+                d["shared_down_f16"] = b.prepare_down_f16(d["shared_down"])
         _DEV[key] = d
     return _DEV[key]
 
 
-def W_of(d):
-    sh = (d["shared_gate"], d["shared_up"], d["shared_down"]) if "shared_gate" in d else None
-    return b.weights(d["w_gate"], d["w_up"], d["w_down"], shared=sh)
+def W_of(d, down_f16):
+    dn = "w_down_f16" if down_f16 else "w_down"
+    sh = None
+    if "shared_gate" in d:
+        sh = (d["shared_gate"], d["shared_up"], d["shared_down_f16" if down_f16 else "shared_down"])
+    return b.weights(d["w_gate"], d["w_up"], d[dn], d.get("s_gate"), d.get("s_up"), d.get("s_down"), shared=sh)
 
 
-def run_steps(cfg, d, variant):
-    p = b.params_for(cfg, variant=variant)
+def P_of(cfg, variant, down_f16, **kw):
+    return b.params_for(cfg, variant=variant, down_dtype=b.DOWN_F16 if down_f16 else b.DOWN_BF16, **kw)
+
+
+def run_steps(cfg, d, variant, down_f16):
+    p = P_of(cfg, variant, down_f16)
     T, E, k = cfg.T, cfg.E, cfg.k
     Et = E + int(cfg.has_shared)
     rows = b.max_rows(p)
@@ -122,7 +147,7 @@ def run_steps(cfg, d, variant):
     wss = [b.workspace(p, w) for w in (b.WS_ROUTE, b.WS_PERMUTE, b.WS_EXPERT_FFN, b.WS_COMBINE)]
     b.route(p, d["logits"], topk_idx, topk_w, wss[0])
     b.permute(p, topk_idx, counts, kept, offsets, st, sp, pr, wss[1])
-    b.expert_ffn(p, d["x"], offsets, st, sp, topk_w, W_of(d), y, wss[2])
+    b.expert_ffn(p, d["x"], offsets, st, sp, topk_w, W_of(d, down_f16), y, wss[2])
     b.combine(p, y, pr, offsets, out, wss[3])
     torch.cuda.synchronize()
     for ws in wss:
@@ -134,12 +159,13 @@ def run_steps(cfg, d, variant):
             "out": f64(out)}
 
 
-def run_forward(cfg, d, variant=b.VARIANT_AUTO):
-    p = b.params_for(cfg, variant=variant)
+def run_forward(cfg, d, variant=b.VARIANT_AUTO, down_f16=True):
+    p = P_of(cfg, variant, down_f16 and cfg.weight_format == "bf16")
     ws = b.workspace(p, b.WS_FORWARD)
     out = torch.empty(cfg.T, cfg.d, dtype=torch.float32, device="cuda")
     counts = torch.empty(cfg.E + int(cfg.has_shared), dtype=torch.int32, device="cuda")
-    b.forward(p, d["x"], d["logits"], W_of(d), out, ws, counts_out=counts)
+    b.forward(p, d["x"], d["logits"], W_of(d, down_f16 and cfg.weight_format == "bf16"), out, ws,
+              counts_out=counts)
     torch.cuda.synchronize()
     assert b.get_error(ws) == 0
     return out, counts.cpu().numpy()
@@ -154,6 +180,14 @@ def check_routing(cfg, got):
     return idx, w, perm
 
 
+def check_layer(name, cfg, got, scale=1.0):
+    out, it = reference(cfg, scale)
+    w_row = np.array([it["w"].reshape(-1)[p] if p >= 0 else 1.0 for p in it["sorted_pair"]])
+    check_close(got["y"], it["y"] * w_row[:, None], f"{name} y_rows")
+    check_close(got["out"], out, f"{name} out")
+    return out, it
+
+
 # --------------------------------------------------------------------------- tests
 
 def test_library_is_in_tree():
@@ -162,49 +196,67 @@ def test_library_is_in_tree():
     b.lib()
 
 
+@pytest.mark.parametrize("down", ["bf16", "f16"])
 @pytest.mark.parametrize("variant", list(VARIANTS))
 @pytest.mark.parametrize("name", list(SMALL))
-def test_small_layers_every_variant(name, variant):
+def test_small_layers_every_variant(name, variant, down):
     cfg = SMALL[name]
     d = device_inputs(cfg)
-    got = run_steps(cfg, d, VARIANTS[variant])
+    f16 = down == "f16"
+    got = run_steps(cfg, d, VARIANTS[variant], f16)
     check_routing(cfg, got)
-    out, it = reference(cfg)
-    # per-row expert outputs (gate weight applied), then the combined layer output
-    w_row = np.array([it["w"].reshape(-1)[p] if p >= 0 else 1.0 for p in it["sorted_pair"]])
-    check_close(got["y"], it["y"] * w_row[:, None], f"{name}/{variant} y_rows")
-    check_close(got["out"], out, f"{name}/{variant} out")
+    out, it = check_layer(f"{name}/{variant}/{down}", cfg, got)
     # the fused entry point gives the same bits as the step-by-step calls
-    fout, counts = run_forward(cfg, d, VARIANTS[variant])
+    fout, counts = run_forward(cfg, d, VARIANTS[variant], f16)
     assert (counts == it["counts"]).all()
     assert np.array_equal(f64(fout), got["out"])
 
 
-def test_clamp_fires_and_matches():
+@pytest.mark.parametrize("variant", ["auto", "tensor"])
+@pytest.mark.parametrize("name", list(Q4_SMALL))
+def test_q4g32_layers(name, variant):
+    cfg = Q4_SMALL[name]
+    d = device_inputs(cfg)
+    got = run_steps(cfg, d, VARIANTS[variant], False)
+    check_routing(cfg, got)
+    check_layer(f"{name}/{variant}", cfg, got)
+    fout, _ = run_forward(cfg, d, VARIANTS[variant])
+    assert np.array_equal(f64(fout), got["out"])
+
+
+def test_q4g32_streaming_variant_is_refused():
+    cfg = Q4_SMALL["q4_tiny"]
+    p = b.params_for(cfg, variant=b.VARIANT_STREAM)
+    with pytest.raises(b.MoeError):
+        b.workspace(p, b.WS_FORWARD)
+
+
+@pytest.mark.parametrize("down", ["bf16", "f16"])
+def test_clamp_fires_and_matches(down):
     cfg = SMALL["tiny"]
     scale = 32.0  # exact in bf16; pre-activations reach well past the clamp at 7
     d = device_inputs(cfg, scale=scale)
-    out, it = reference(cfg, scale=scale)
     for v in ("tensor", "stream"):
-        got = run_steps(cfg, d, VARIANTS[v])
-        check_close(got["out"], out, f"clamp/{v}")
+        got = run_steps(cfg, d, VARIANTS[v], down == "f16")
+        check_layer(f"clamp/{v}/{down}", cfg, got, scale=scale)
+    _, it = reference(cfg, scale)
     x = synth.bf16_bits_to_f32(synth.x_bits(cfg)).astype(np.float64)
-    g = x[:1] @ (expert_f64(cfg, int(it["idx"][0, 0]))[0] * scale)
+    g = x[:1] @ expert_ref(cfg, int(it["idx"][0, 0]), scale)[0]
     assert np.abs(g).max() > 7.0
 
 
 @pytest.mark.parametrize("name", FULL)
-def test_full_size_workloads_sampled(name):
+def test_full_size_workloads(name):
     cfg = synth.CONFIGS[name]
     idx, w, perm = routing_reference(cfg)
     touched = np.unique(idx[perm["pair_row"].reshape(idx.shape) >= 0])
     d = device_inputs(cfg, experts=touched)
-    got = run_steps(cfg, d, b.VARIANT_AUTO)
+    got = run_steps(cfg, d, b.VARIANT_AUTO, True)
     check_routing(cfg, got)
     # every output element, the oracle drawing each touched expert's weights as it goes
     x = synth.bf16_bits_to_f32(synth.x_bits(cfg)).astype(np.float64)
     sh = shared_f64(cfg) if cfg.has_shared else None
-    ref, it = oracle.forward(x, synth.logits(cfg), cfg.k, lambda e: expert_f64(cfg, e), cfg.swiglu_limit,
+    ref, it = oracle.forward(x, synth.logits(cfg), cfg.k, lambda e: expert_ref(cfg, e), cfg.swiglu_limit,
                              cfg.capacity_factor, shared=sh)
     check_close(got["out"], ref, f"{name} full output (step calls)")
     w_row = np.array([it["w"].reshape(-1)[p] if p >= 0 else 1.0 for p in it["sorted_pair"]])
@@ -214,9 +266,30 @@ def test_full_size_workloads_sampled(name):
     check_close(f64(fout), ref, f"{name} full output (moe_forward)")
     # and a few tokens from the per-token definition, which never permutes
     toks = [0, cfg.T // 2, cfg.T - 1]
-    one = oracle.token_outputs(toks, x, idx, w, perm["pair_row"], lambda e: expert_f64(cfg, e), cfg.swiglu_limit,
+    one = oracle.token_outputs(toks, x, idx, w, perm["pair_row"], lambda e: expert_ref(cfg, e), cfg.swiglu_limit,
                                shared=sh)
     check_close(f64(fout)[toks], one, f"{name} per-token definition")
+
+
+def test_full_size_quantised_workload():
+    cfg = synth.CONFIGS["quant"]
+    d = device_inputs(cfg)
+    got = run_steps(cfg, d, b.VARIANT_AUTO, False)
+    idx, w, perm = check_routing(cfg, got)
+    x = synth.bf16_bits_to_f32(synth.x_bits(cfg)).astype(np.float64)
+    rng = np.random.default_rng(7)
+    toks = sorted(set([0, cfg.T - 1] + rng.choice(cfg.T, 40, replace=False).tolist()))
+    cache = {}
+
+    def experts(e):
+        if e not in cache:
+            cache[e] = expert_ref(cfg, e)
+        return cache[e]
+
+    ref = oracle.token_outputs(toks, x, idx, w, perm["pair_row"], experts, cfg.swiglu_limit)
+    check_close(got["out"][toks], ref, "quant sampled tokens (step calls)")
+    fout, _ = run_forward(cfg, d)
+    check_close(f64(fout)[toks], ref, "quant sampled tokens (moe_forward)")
 
 
 def test_forward_is_deterministic():
@@ -227,17 +300,61 @@ def test_forward_is_deterministic():
     assert torch.equal(a.view(torch.int32), c.view(torch.int32))
 
 
+def test_down_forms_agree():
+    """W_down as bf16 (converted per tile) and prepared fp16 give the same bits."""
+    cfg = SMALL["ragged"]
+    d = device_inputs(cfg)
+    for v in (b.VARIANT_TENSOR, b.VARIANT_STREAM):
+        a, _ = run_forward(cfg, d, v, down_f16=False)
+        c, _ = run_forward(cfg, d, v, down_f16=True)
+        assert torch.equal(a.view(torch.int32), c.view(torch.int32))
+
+
 def test_forward_host_matches_device():
     cfg = SMALL["ragged"]
     d = device_inputs(cfg)
     ref_out, _ = run_forward(cfg, d)
-    p = b.params_for(cfg)
+    p = P_of(cfg, b.VARIANT_AUTO, True)
     ws = b.workspace(p, b.WS_FORWARD_HOST)
     x_h = d["x"].cpu().pin_memory()
     l_h = d["logits"].cpu().pin_memory()
     o_h = torch.empty(cfg.T, cfg.d, dtype=torch.float32).pin_memory()
-    b.forward_host(p, x_h, l_h, W_of(d), o_h, ws)
+    b.forward_host(p, x_h, l_h, W_of(d, True), o_h, ws)
     assert torch.equal(o_h.view(torch.int32), ref_out.cpu().view(torch.int32))
+
+
+def test_bf16_output_option():
+    cfg = SMALL["ragged"]
+    d = device_inputs(cfg)
+    f32_out, _ = run_forward(cfg, d)
+    p = P_of(cfg, b.VARIANT_AUTO, True, out_dtype=b.OUT_BF16)
+    ws = b.workspace(p, b.WS_FORWARD)
+    out = torch.empty(cfg.T, cfg.d, dtype=torch.bfloat16, device="cuda")
+    b.forward(p, d["x"], d["logits"], W_of(d, True), out, ws)
+    torch.cuda.synchronize()
+    assert b.get_error(ws) == 0
+    # the bf16 output is the fp32 output rounded once (to nearest even)
+    assert torch.equal(out.view(torch.int16), f32_out.to(torch.bfloat16).view(torch.int16))
+    ref, _ = reference(cfg)
+    assert np.linalg.norm(f64(out) - ref) / np.linalg.norm(ref) <= REL_L2
+
+
+def test_weight_conversion_is_exact_rounding():
+    rng = np.random.default_rng(5)
+    vals = np.concatenate([rng.standard_normal(10000).astype(np.float32) * 0.02,
+                           # 65280 is the largest bf16 value inside fp16's range (65504 rounds to 65536 in bf16)
+                           np.array([0.0, -0.0, 1e-7, -3e-6, 6.1e-5, 65280.0, -65280.0, 1.0, 2.0 ** -17], np.float32)])
+    bits = synth.f32_to_bf16_bits(vals)
+    src = torch.from_numpy(bits.view(np.int16)).cuda()
+    dst = torch.empty(src.numel(), dtype=torch.float16, device="cuda")
+    ws = torch.zeros(256, dtype=torch.uint8, device="cuda")
+    b.convert_bf16_to_f16(src, dst, err_ws=ws)
+    want = synth.bf16_bits_to_f32(bits).astype(np.float16)  # round to nearest even
+    assert np.array_equal(dst.cpu().numpy().view(np.uint16), want.view(np.uint16))
+    assert b.get_error(ws) == 0
+    big = torch.from_numpy(synth.f32_to_bf16_bits(np.array([1e6] * 8, np.float32)).view(np.int16)).cuda()
+    b.convert_bf16_to_f16(big, torch.empty(8, dtype=torch.float16, device="cuda"), err_ws=ws)
+    assert b.get_error(ws) & b.DEVERR_RANGE
 
 
 def test_out_of_range_expert_ids_are_flagged():
@@ -259,20 +376,3 @@ def test_out_of_range_expert_ids_are_flagged():
     assert int(bufs[0].sum()) == T * k - 2
     b.clear_error(ws)
     assert b.get_error(ws) == 0
-
-
-def test_bf16_output_option():
-    cfg = SMALL["ragged"]
-    d = device_inputs(cfg)
-    f32_out, _ = run_forward(cfg, d)
-    p = b.params_for(cfg, out_dtype=b.OUT_BF16)
-    ws = b.workspace(p, b.WS_FORWARD)
-    out = torch.empty(cfg.T, cfg.d, dtype=torch.bfloat16, device="cuda")
-    b.forward(p, d["x"], d["logits"], W_of(d), out, ws)
-    torch.cuda.synchronize()
-    assert b.get_error(ws) == 0
-    # the bf16 output is the fp32 output rounded once (to nearest even)
-    assert torch.equal(out.view(torch.int16), f32_out.to(torch.bfloat16).view(torch.int16))
-    ref, _ = reference(cfg)
-    got = f64(out)
-    assert np.linalg.norm(got - ref) / np.linalg.norm(ref) <= REL_L2
