@@ -197,6 +197,34 @@ MOE_API int moe_permute(const moe_params* p, const int32_t* topk_idx, int32_t* c
                 moe_stream_t stream);
 
 /*
+ * moe_permute_noalloc — moe_permute without a workspace argument. The pages
+ * have no counterpart: this is a library convenience, not a step of the method.
+ * It computes exactly what moe_permute computes (same outputs, same layouts,
+ * bit-identical) but keeps its scratch (per-block histograms and bases) in a
+ * fixed array inside the library, so the caller passes only inputs, outputs
+ * and a device error word.
+ * Who needs it: callers that must not allocate device memory when they
+ * permute — an engine that has already handed all free memory to its own
+ * budget, or a plugin without an allocator of its own.
+ * Limit: T*k <= MOE_NOALLOC_MAX_PAIRS; larger calls return
+ * MOE_ERR_WORKSPACE_TOO_SMALL before any launch (use moe_permute). The array
+ * (256 KiB) stays resident on every GPU that loads the library until exit.
+ * err_word  device uint32, OR-ed with MOE_DEVERR_BOUNDS for out-of-range ids
+ *           (the caller zeroes it; it is not cleared here).
+ * Returns MOE_ERR_INVALID_ARG for parameters moe_workspace_size rejects and
+ * for null pointers. The first call on a device looks up the array's device
+ * address (a CUDA runtime query, no allocation): make that first call before
+ * any stream capture. Every call uses the same array, so calls whose work may
+ * overlap on the GPU (other streams, other host threads) race: issue them on
+ * one stream. Nothing here calls an allocator.
+ */
+#define MOE_NOALLOC_MAX_PAIRS 262144
+MOE_API int moe_permute_noalloc(const moe_params* p, const int32_t* topk_idx, int32_t* counts,
+                int32_t* kept_counts, int32_t* offsets, int32_t* sorted_token,
+                int32_t* sorted_pair, int32_t* pair_row, uint32_t* err_word,
+                moe_stream_t stream);
+
+/*
  * moe_expert_ffn — S4..S6 (+ S8, S9): per expert e, rows r in
  * [offsets[e], offsets[e+1]):
  *   g = x[sorted_token[r]] W_gate[e],  u = x[sorted_token[r]] W_up[e]

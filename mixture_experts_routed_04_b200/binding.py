@@ -32,7 +32,9 @@ WS_ROUTE, WS_PERMUTE, WS_EXPERT_FFN, WS_COMBINE, WS_FORWARD, WS_FORWARD_HOST = r
 EXPORTS = ("moe_version", "moe_status_string", "moe_capacity", "moe_max_rows", "moe_workspace_size",
            "moe_route", "moe_permute", "moe_expert_ffn", "moe_combine", "moe_forward", "moe_forward_host",
            "moe_get_error", "moe_clear_error", "moe_set_wait_limit_ns", "moe_launch_count",
-           "moe_profile_enable", "moe_profile_collect", "moe_convert_bf16_to_f16")
+           "moe_profile_enable", "moe_profile_collect", "moe_convert_bf16_to_f16",
+           "moe_permute_noalloc")
+NOALLOC_MAX_PAIRS = 262144  # MOE_NOALLOC_MAX_PAIRS
 
 # kernel ids (MOE_K_*), in order
 KERNELS = ("route", "perm_count", "perm_scan", "perm_scatter", "schedule", "gather", "tc_gateup", "tc_down",
@@ -86,6 +88,7 @@ def lib() -> ctypes.CDLL:
             "moe_profile_enable": ([ctypes.c_int], ctypes.c_int),
             "moe_profile_collect": ([ctypes.POINTER(ctypes.c_double), ctypes.POINTER(ctypes.c_int64)], ctypes.c_int),
             "moe_convert_bf16_to_f16": ([_V, _V, ctypes.c_int64, _V, _V], ctypes.c_int),
+            "moe_permute_noalloc": ([_P, _V, _V, _V, _V, _V, _V, _V, _V, _V], ctypes.c_int),
         }
         for name, (args, res) in sig.items():
             fn = getattr(L, name)
@@ -168,6 +171,14 @@ def route(p, logits, topk_idx, topk_w, ws, stream=None):
 def permute(p, topk_idx, counts, kept, offsets, sorted_token, sorted_pair, pair_row, ws, stream=None):
     check(lib().moe_permute(ctypes.byref(p), _p(topk_idx), _p(counts), _p(kept), _p(offsets), _p(sorted_token),
                             _p(sorted_pair), _p(pair_row), _p(ws), ws.numel(), _stream(stream)), "moe_permute")
+
+
+def permute_noalloc(p, topk_idx, counts, kept, offsets, sorted_token, sorted_pair, pair_row, err_word,
+                    stream=None):
+    """moe_permute with the library's fixed scratch array instead of a workspace (one stream only)."""
+    check(lib().moe_permute_noalloc(ctypes.byref(p), _p(topk_idx), _p(counts), _p(kept), _p(offsets),
+                                    _p(sorted_token), _p(sorted_pair), _p(pair_row), _p(err_word),
+                                    _stream(stream)), "moe_permute_noalloc")
 
 
 def expert_ffn(p, x, offsets, sorted_token, sorted_pair, topk_w, W: Weights, y_rows, ws, stream=None):
