@@ -96,7 +96,9 @@ typedef struct CUstream_st* moe_stream_t; /* same object as cudaStream_t */
 #define MOE_WS_FORWARD_HOST 5
 
 typedef struct moe_params {
-    int32_t T;               /* tokens in this call */
+    int32_t T;               /* tokens in this call; 0 = empty batch: every call returns MOE_OK
+                                without a kernel launch (buffers may then be null); moe_permute
+                                and moe_forward's counts_out get zero counts and offsets */
     int32_t d_model;         /* d */
     int32_t d_ff;            /* f, per routed expert */
     int32_t E;               /* routed experts */
@@ -325,7 +327,7 @@ MOE_API int moe_set_wait_limit_ns(uint64_t ns);
 #define MOE_K_TC_GATEUP      6  /* S5 tcgen05 gate/up GEMM + clamped SwiGLU */
 #define MOE_K_TC_DOWN        7  /* S6 tcgen05 down GEMM + gate scale */
 #define MOE_K_STREAM_GATEUP  8  /* S8 few-rows gate/up (weight streaming) */
-#define MOE_K_STREAM_REDUCE  9  /* S8 K-split partial sums + SwiGLU */
+#define MOE_K_STREAM_REDUCE  9  /* unused: the S8 K-split sums now run inside stream gate/up */
 #define MOE_K_STREAM_DOWN   10  /* S8 few-rows down */
 #define MOE_K_COMBINE       11  /* S7 gate-weighted combine */
 #define MOE_K_CONVERT       12  /* load-time bf16 -> fp16 weight copy (not a layer step) */

@@ -10,7 +10,7 @@
 namespace moe {
 
 cudaError_t launch_schedule(const Dims& D, const int32_t* offsets, int32_t* tile_base, int32_t* stream_list,
-                            int32_t* n_stream, uint32_t* err, cudaStream_t s);
+                            int32_t* n_stream, int32_t* fix, int n_fix, uint32_t* err, cudaStream_t s);
 cudaError_t launch_gather(const Dims& D, const uint16_t* x, const int32_t* sorted_token, const int32_t* offsets,
                           uint16_t* xg, uint32_t* err, cudaStream_t s);
 cudaError_t launch_tensor_ffn(const Dims& D, const uint16_t* xg, uint16_t* h, const int32_t* tile_base,
@@ -19,7 +19,8 @@ cudaError_t launch_tensor_ffn(const Dims& D, const uint16_t* xg, uint16_t* h, co
                               uint16_t* y_rows, int32_t* counters, uint32_t* err, uint64_t wait_ns,
                               cudaStream_t s);
 cudaError_t launch_convert_bf16_f16(const uint16_t* src, uint16_t* dst, int64_t n, uint32_t* err, cudaStream_t s);
-cudaError_t launch_stream_ffn(const Dims& D, const uint16_t* xg, uint16_t* h, float* part, const int32_t* offsets,
+cudaError_t launch_stream_ffn(const Dims& D, const uint16_t* xg, uint16_t* h, float* part, int32_t* fix,
+                              const int32_t* offsets,
                               const int32_t* stream_list, const int32_t* n_stream, const int32_t* sorted_pair,
                               const float* topk_w, const moe_weights* w, uint16_t* y_rows, uint32_t* err,
                               uint64_t wait_ns, cudaStream_t s);
@@ -44,7 +45,8 @@ static size_t align256(size_t v) { return (v + 255) & ~size_t(255); }
 // Host-side checks of moe_params; fills D. Returns MOE_OK or an error code.
 static int make_dims(const moe_params* p, Dims* D) {
     if (!p || !D) return MOE_ERR_INVALID_ARG;
-    if (p->T < 1 || p->E < 1 || p->E > kMaxE || p->k < 1 || p->k > kMaxK || p->k > p->E) return MOE_ERR_INVALID_ARG;
+    // T = 0 (an empty batch) is valid: the calls launch nothing and report empty results
+    if (p->T < 0 || p->E < 1 || p->E > kMaxE || p->k < 1 || p->k > kMaxK || p->k > p->E) return MOE_ERR_INVALID_ARG;
     if (p->d_model < 64 || p->d_model % 64 || p->d_ff < 64 || p->d_ff % 64) return MOE_ERR_INVALID_ARG;
     if (!(p->capacity_factor >= 0.f) || !std::isfinite(p->capacity_factor)) return MOE_ERR_INVALID_ARG;
     if (!std::isfinite(p->swiglu_limit)) return MOE_ERR_INVALID_ARG;
@@ -110,6 +112,10 @@ static int make_dims(const moe_params* p, Dims* D) {
     return MOE_OK;
 }
 
+// K-split arrival counters of the streaming gate/up: one per (streaming list
+// entry, 64-column slice of d_ff, consumer warp).
+static int fix_count(const Dims& D) { return D.Etot * (D.f / 64) * 4; }
+
 WsLayout ws_layout(const Dims& D, int which) {
     WsLayout L;
     std::memset(&L, 0, sizeof(L));
@@ -127,12 +133,15 @@ WsLayout ws_layout(const Dims& D, int which) {
         L.blockbase = take(size_t(D.perm_blocks) * D.E * 4);
     }
     if (ffn) {
-        L.tile_base = take(size_t(D.Etot + 1) * 4);
+        L.tile_base = take(size_t(D.Etot + 1) * 2 * 4);  // 128-row and 256-row tile prefixes
         L.stream_list = take(size_t(D.Etot) * 4);
         L.n_stream = take(16);  // [0] streaming experts, [1], [2] tile-unit counters
         L.xg = take(size_t(D.rows) * D.d * 2);
         L.h = take(size_t(D.rows) * D.f * 2);
-        if (D.ks > 1) L.part = take(size_t(D.ks) * 2 * D.rows * D.f * 4);
+        if (D.ks > 1) {
+            L.part = take(size_t(D.ks) * 2 * D.rows * D.f * 4);
+            L.fix = take(size_t(fix_count(D)) * 4);
+        }
     }
     if (fwd) {
         L.topk_idx = take(size_t(D.pairs) * 4);
@@ -154,6 +163,16 @@ WsLayout ws_layout(const Dims& D, int which) {
     return L;
 }
 
+// Whether any expert can take the tcgen05 tiles. An expert holds at most T rows
+// (a token's k experts are distinct; the shared expert holds exactly T), so
+// with T <= stream_max_rows the automatic choice streams every expert and the
+// two persistent GEMMs would only start and exit: they are not launched.
+static bool tiles_needed(const Dims& D) {
+    if (D.variant == MOE_VARIANT_STREAM) return false;
+    if (D.variant == MOE_VARIANT_AUTO && D.stream_max_rows > 0 && D.T <= D.stream_max_rows) return false;
+    return true;
+}
+
 cudaError_t launch_expert_ffn(const Dims& D, const WsLayout& L, const FfnArgs& a, cudaStream_t s) {
     uint8_t* ws = a.ws;
     int32_t* tile_base = reinterpret_cast<int32_t*>(ws + L.tile_base);
@@ -162,19 +181,21 @@ cudaError_t launch_expert_ffn(const Dims& D, const WsLayout& L, const FfnArgs& a
     uint16_t* xg = reinterpret_cast<uint16_t*>(ws + L.xg);
     uint16_t* h = reinterpret_cast<uint16_t*>(ws + L.h);
     float* part = L.part ? reinterpret_cast<float*>(ws + L.part) : nullptr;
-    cudaError_t e = launch_schedule(D, a.offsets, tile_base, stream_list, n_stream, a.err, s);
+    int32_t* fix = L.fix ? reinterpret_cast<int32_t*>(ws + L.fix) : nullptr;
+    cudaError_t e = launch_schedule(D, a.offsets, tile_base, stream_list, n_stream, fix, fix ? fix_count(D) : 0,
+                                    a.err, s);
     if (e != cudaSuccess) return e;
     // Rows in expert order for both variants (fp16 for Q4G32, whose MMAs run
     // in fp16). A TMA tile::gather4 of the rows inside the GEMM was measured
     // slower: 32 TMA instructions per k-block left the producer behind.
     if ((e = launch_gather(D, a.x, a.sorted_token, a.offsets, xg, a.err, s)) != cudaSuccess) return e;
-    if (D.variant != MOE_VARIANT_STREAM) {
+    if (tiles_needed(D)) {
         if ((e = launch_tensor_ffn(D, xg, h, tile_base, a.offsets, a.sorted_pair, a.topk_w, a.w, a.y_rows,
                                    n_stream + 1, a.err, a.wait_ns, s)) != cudaSuccess)
             return e;
     }
     if (D.variant != MOE_VARIANT_TENSOR && D.stream_max_rows > 0) {
-        if ((e = launch_stream_ffn(D, xg, h, part, a.offsets, stream_list, n_stream, a.sorted_pair, a.topk_w, a.w,
+        if ((e = launch_stream_ffn(D, xg, h, part, fix, a.offsets, stream_list, n_stream, a.sorted_pair, a.topk_w, a.w,
                                    a.y_rows, a.err, a.wait_ns, s)) != cudaSuccess)
             return e;
     }
@@ -257,6 +278,7 @@ int moe_route(const moe_params* p, const float* logits, int32_t* topk_idx, float
     int st = make_dims(p, &D);
     if (st != MOE_OK) return st;
     if ((st = check_ws(D, MOE_WS_ROUTE, ws, ws_bytes)) != MOE_OK) return st;
+    if (D.T == 0) return MOE_OK;  // empty batch: the (empty) buffers may be null
     if (!logits || !topk_idx || !topk_w) return MOE_ERR_INVALID_ARG;
     return status_of(launch_route(logits, D.T, D.E, D.k, topk_idx, topk_w, stream));
 }
@@ -284,6 +306,7 @@ int moe_expert_ffn(const moe_params* p, const uint16_t* x, const int32_t* offset
     int st = make_dims(p, &D);
     if (st != MOE_OK) return st;
     if ((st = check_ws(D, MOE_WS_EXPERT_FFN, ws, ws_bytes)) != MOE_OK) return st;
+    if (D.T == 0) return MOE_OK;
     if ((st = check_weights(D, w)) != MOE_OK) return st;
     if (!x || !offsets || !sorted_token || !sorted_pair || !topk_w || !y_rows) return MOE_ERR_INVALID_ARG;
     if (!al16(x) || !al16(y_rows)) return MOE_ERR_MISALIGNED;
@@ -299,6 +322,7 @@ int moe_combine(const moe_params* p, const uint16_t* y_rows, const int32_t* pair
     int st = make_dims(p, &D);
     if (st != MOE_OK) return st;
     if ((st = check_ws(D, MOE_WS_COMBINE, ws, ws_bytes)) != MOE_OK) return st;
+    if (D.T == 0) return MOE_OK;
     if (!y_rows || !pair_row || !out || (D.has_shared && !offsets)) return MOE_ERR_INVALID_ARG;
     if (!al16(y_rows) || !al16(out)) return MOE_ERR_MISALIGNED;
     return status_of(launch_combine(D, y_rows, pair_row, offsets, out, stream));
@@ -338,6 +362,11 @@ int moe_forward(const moe_params* p, const uint16_t* x, const float* logits, con
     int st = make_dims(p, &D);
     if (st != MOE_OK) return st;
     if ((st = check_ws(D, MOE_WS_FORWARD, ws, ws_bytes)) != MOE_OK) return st;
+    if (D.T == 0) {  // empty batch: nothing to read or write but the (optional) counts
+        if (counts_out && cudaMemsetAsync(counts_out, 0, size_t(D.Etot) * 4, stream) != cudaSuccess)
+            return MOE_ERR_CUDA;
+        return MOE_OK;
+    }
     if ((st = check_weights(D, w)) != MOE_OK) return st;
     if (!x || !logits || !out) return MOE_ERR_INVALID_ARG;
     if (!al16(x) || !al16(out)) return MOE_ERR_MISALIGNED;
@@ -351,6 +380,7 @@ int moe_forward_host(const moe_params* p, const uint16_t* x_host, const float* l
     int st = make_dims(p, &D);
     if (st != MOE_OK) return st;
     if ((st = check_ws(D, MOE_WS_FORWARD_HOST, ws, ws_bytes)) != MOE_OK) return st;
+    if (D.T == 0) return MOE_OK;
     if ((st = check_weights(D, w)) != MOE_OK) return st;
     if (!x_host || !logits_host || !out_host) return MOE_ERR_INVALID_ARG;
     const WsLayout L = ws_layout(D, MOE_WS_FORWARD_HOST);
@@ -388,10 +418,14 @@ int moe_launch_count(const moe_params* p, int which, int* n) {
     const int st = make_dims(p, &D);
     if (st != MOE_OK) return st;
     if (!n || which < MOE_WS_ROUTE || which > MOE_WS_FORWARD_HOST) return MOE_ERR_INVALID_ARG;
+    if (D.T == 0) {
+        *n = 0;
+        return MOE_OK;
+    }
     int ffn = 1;  // schedule
     ffn += 1;                                       // gather
-    if (D.variant != MOE_VARIANT_STREAM) ffn += 2;  // two tcgen05 GEMMs
-    if (D.variant != MOE_VARIANT_TENSOR && D.stream_max_rows > 0) ffn += 2 + (D.ks > 1 ? 1 : 0);
+    if (tiles_needed(D)) ffn += 2;                  // two tcgen05 GEMMs
+    if (D.variant != MOE_VARIANT_TENSOR && D.stream_max_rows > 0) ffn += 2;
     switch (which) {
         case MOE_WS_ROUTE: *n = 1; break;
         case MOE_WS_PERMUTE: *n = 3; break;

@@ -20,6 +20,8 @@ __global__ void __launch_bounds__(256) combine_kernel(const uint16_t* __restrict
                                                       const int32_t* __restrict__ pair_row,
                                                       const int32_t* __restrict__ offsets, int T, int d, int k,
                                                       int E, int has_shared, void* __restrict__ out) {
+    griddep_wait();
+    griddep_launch();
     const int vec_per_row = d / 8;  // d % 64 == 0
     const int64_t total = int64_t(T) * vec_per_row;
     const int shared_base = has_shared ? offsets[E] : 0;
@@ -68,12 +70,12 @@ cudaError_t launch_combine(const Dims& D, const uint16_t* y_rows, const int32_t*
     if (blocks < 1) blocks = 1;
     {
         ProfScope prof_(MOE_K_COMBINE, s);
-        if (D.out_bf16)
-            combine_kernel<true><<<int(blocks), threads, 0, s>>>(y_rows, pair_row, offsets, D.T, D.d, D.k, D.E,
-                                                                 D.has_shared, out);
-        else
-            combine_kernel<false><<<int(blocks), threads, 0, s>>>(y_rows, pair_row, offsets, D.T, D.d, D.k, D.E,
-                                                                  D.has_shared, out);
+        const cudaError_t le =
+            D.out_bf16 ? launch_pdl(combine_kernel<true>, dim3(int(blocks)), dim3(threads), 0, s, y_rows, pair_row,
+                                    offsets, D.T, D.d, D.k, D.E, D.has_shared, out)
+                       : launch_pdl(combine_kernel<false>, dim3(int(blocks)), dim3(threads), 0, s, y_rows, pair_row,
+                                    offsets, D.T, D.d, D.k, D.E, D.has_shared, out);
+        if (le != cudaSuccess) return le;
     }
     return cudaGetLastError();
 }
@@ -87,6 +89,8 @@ namespace {
 // dst = fp16(src), 8 values per thread per step; out-of-range values flagged.
 __global__ void __launch_bounds__(256) convert_bf16_f16_kernel(const uint16_t* __restrict__ src,
                                                                uint16_t* __restrict__ dst, int64_t n, uint32_t* err) {
+    griddep_wait();
+    griddep_launch();
     bool bad = false;
     const int64_t nv = n / 8;
     for (int64_t i = int64_t(blockIdx.x) * blockDim.x + threadIdx.x; i < nv; i += int64_t(gridDim.x) * blockDim.x) {
@@ -119,7 +123,9 @@ cudaError_t launch_convert_bf16_f16(const uint16_t* src, uint16_t* dst, int64_t 
     if (blocks < 1) blocks = 1;
     {
         ProfScope prof_(MOE_K_CONVERT, s);
-        convert_bf16_f16_kernel<<<int(blocks), 256, 0, s>>>(src, dst, n, err);
+        const cudaError_t le = launch_pdl(convert_bf16_f16_kernel, dim3(int(blocks)), dim3(256), 0, s, src, dst,
+                                          n, err);
+        if (le != cudaSuccess) return le;
     }
     return cudaGetLastError();
 }

@@ -67,6 +67,16 @@ MOE_DEV void mbar_init(uint64_t* bar, uint32_t count) {
     asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count) : "memory");
 }
 MOE_DEV void fence_mbar_init() { asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory"); }
+// Programmatic dependent launch. Every kernel of the library is launched with
+// programmatic stream serialization, so it may be scheduled while its
+// predecessor drains. It calls griddep_wait() before it reads anything an
+// earlier kernel wrote (the wait returns once the predecessor grid has
+// completed and its writes are visible), then griddep_launch() so that its own
+// successor may start its prologue early. Both are no-ops for a kernel that was
+// launched without the attribute.
+MOE_DEV void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+MOE_DEV void griddep_launch() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
 MOE_DEV void fence_proxy_async_smem() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
 
 MOE_DEV void mbar_arrive_expect_tx(uint64_t* bar, uint32_t bytes) {

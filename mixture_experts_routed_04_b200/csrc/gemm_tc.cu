@@ -15,13 +15,16 @@
 //
 // Kernel shape (one CTA per SM, persistent over work units):
 //   warp 0    TMA producer. A = 128 rows x 64 K of the gathered rows (2-D map,
-//             128-byte swizzle, K-major). B, bf16: 64 K x 256 N of the expert's
-//             weights (3-D map, four 64-wide boxes, N-major). B, Q4G32: the
-//             packed nibbles of 256 N-rows x 64 K (32 bytes a row) and the
-//             k-block's two scale groups.
+//             128-byte swizzle, K-major), two such sub-tiles for 256-row units.
+//             B, bf16: 64 K x 256 N of the expert's weights (3-D map, four
+//             64-wide boxes, N-major). B, Q4G32: the packed nibbles of 256
+//             N-rows x 64 K (32 bytes a row) and the k-block's two scale groups.
 //   warp 1    TMEM allocator + single-thread tcgen05.mma issuer: M=128, N=256,
-//             K=16 per instruction, fp32 accumulators in TMEM, two 256-column
-//             buffers so the epilogue of a unit overlaps the next unit's MMAs.
+//             K=16 per instruction, fp32 accumulators in TMEM. bf16 units are
+//             128 rows with two 256-column buffers, so the epilogue of a unit
+//             overlaps the next unit's MMAs; Q4G32 units are 256 rows (two
+//             M=128 MMAs per B tile, one buffer of 2 x 256 columns), halving
+//             the dequantisation per FLOP.
 //   warps 2-5 epilogue: tcgen05.ld 32 lanes x 32 columns, fused SwiGLU or gate
 //             scaling, fp16 stores. Warp w reads TMEM lanes 32*(w%4)..+31.
 //   warps 6-9 transform (Q4G32, or MODE 1 with W_down given as bf16): turn the
@@ -53,17 +56,29 @@ constexpr int S_BYTES = 2 * BN * 2;   // two scale groups x 256 rows, fp16: 1 KB
 constexpr int TMEM_COLS = 512;
 
 // WF: weight form. 0 = bf16 as given, 1 = Q4G32, 2 = fp16 (W_down prepared at load time).
-template <int MODE, int WF>
+template <int MODE, int WF, int SUB>
 struct Cfg {
     static constexpr bool Q4 = WF == 1;
     static constexpr bool kTransform = Q4 || (MODE == 1 && WF == 0);
-    static constexpr int kThreads = kTransform ? 320 : 192;
-    static constexpr int kStages = Q4 ? 3 : 4;
-    static constexpr int kStageBytes = Q4 ? A_BYTES + B_BYTES + P_BYTES + S_BYTES : A_BYTES + B_BYTES;
-    static constexpr uint32_t kTxBytes = Q4 ? A_BYTES + P_BYTES + S_BYTES : A_BYTES + B_BYTES;
+    // Rows of a unit, in 128-row sub-tiles (SUB = 1 or 2). With SUB = 2 two
+    // M=128 MMAs share every B tile, so B is loaded (and for Q4G32
+    // dequantised) once per 256 rows; the two accumulators then fill TMEM and
+    // there is one accumulator buffer instead of two, so the epilogue is not
+    // overlapped with the next unit's MMAs. Measured on B200: SUB = 2 pays for
+    // the Q4G32 GEMMs (dequantisation halves per FLOP), SUB = 1 for bf16.
+    static constexpr int kSub = SUB;
+    static constexpr int kAcc = 2 / kSub;  // accumulator buffers of kSub x 256 columns
+    static constexpr int kEpiWarps = 4;
+    static constexpr int kTransWarps = kTransform ? 4 : 0;
+    static constexpr int kThreads = 32 * (2 + kEpiWarps + kTransWarps);
+    static constexpr int kABytes = kSub * A_BYTES;
+    static constexpr int kStages = (Q4 || kSub == 2) ? 3 : 4;
+    static constexpr int kStageBytes = Q4 ? kABytes + B_BYTES + P_BYTES + S_BYTES : kABytes + B_BYTES;
+    // bytes a stage receives besides its A sub-tiles (A_BYTES each)
+    static constexpr uint32_t kTxB = Q4 ? P_BYTES + S_BYTES : B_BYTES;
     static constexpr int kSmem = 1024 + kStages * kStageBytes + 512;  // + barriers, unit ring
-    // warps that read the unit ring: MMA, 4 epilogue (+ 4 transform)
-    static constexpr int kUnitReaders = 1 + 4 + (kTransform ? 4 : 0);
+    // warps that read the unit ring: MMA, epilogue, transform
+    static constexpr int kUnitReaders = 1 + kEpiWarps + kTransWarps;
     // bf16 operands for the bf16 gate/up; fp16 otherwise. B is N-major (bf16
     // weights as stored) or K-major (dequantised from the K-major Q4G32 rows).
     static constexpr uint32_t kIdesc =
@@ -96,8 +111,10 @@ struct Unit {
     int e, m, n, row0, rows;
 };
 
-MOE_DEV Unit decode_unit(int u, const GemmParams& p) {
-    const int g = u / p.n_tiles;  // global M-tile index
+// p.tile_base counts units of SUB x 128 rows.
+template <int SUB>
+MOE_DEV Unit decode_unit(int u, const GemmParams& p, int nt) {
+    const int g = u / nt;  // global M-tile index
     int lo = 0, hi = p.Etot;      // tile_base[lo] <= g < tile_base[hi]
     while (hi - lo > 1) {
         const int mid = (lo + hi) >> 1;
@@ -108,13 +125,13 @@ MOE_DEV Unit decode_unit(int u, const GemmParams& p) {
     U.e = lo;
     const int tb = __ldg(p.tile_base + lo);
     const int mt = __ldg(p.tile_base + lo + 1) - tb;
-    const int local = u - tb * p.n_tiles;
+    const int local = u - tb * nt;
     U.n = local / mt;
     U.m = local - U.n * mt;
     const int off = __ldg(p.offsets + lo);
     const int kept = __ldg(p.offsets + lo + 1) - off;
-    U.row0 = off + U.m * BM;
-    U.rows = min(BM, kept - U.m * BM);
+    U.row0 = off + U.m * (SUB * BM);
+    U.rows = min(SUB * BM, kept - U.m * (SUB * BM));
     return U;
 }
 
@@ -123,7 +140,9 @@ MOE_DEV float swiglu(float g, float u, float L) {
         g = fminf(fmaxf(g, -L), L);
         u = fminf(fmaxf(u, -L), L);
     }
-    return g / (1.0f + expf(-g)) * u;
+    // __expf / __fdividef: relative error ~1e-6, far below the fp16 rounding
+    // of h that follows (the accurate forms cost ~5% of the gate/up GEMM).
+    return __fdividef(g, 1.0f + __expf(-g)) * u;
 }
 
 MOE_DEV uint32_t lop3_and_or(uint32_t a, uint32_t mask, uint32_t orv) {
@@ -210,12 +229,12 @@ MOE_DEV bool ring_read(int& u, int& slot, uint32_t& phase, volatile int* ring, u
     return true;
 }
 
-template <int MODE, int WF>
-__global__ void __launch_bounds__(Cfg<MODE, WF>::kThreads, 1)
+template <int MODE, int WF, int SUB>
+__global__ void __launch_bounds__(Cfg<MODE, WF, SUB>::kThreads, 1)
     grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB0,
                         const __grid_constant__ CUtensorMap tmB1, const __grid_constant__ CUtensorMap tmS0,
                         const __grid_constant__ CUtensorMap tmS1, const GemmParams p) {
-    using C = Cfg<MODE, WF>;
+    using C = Cfg<MODE, WF, SUB>;
     constexpr bool Q4 = C::Q4;
     constexpr int STAGES = C::kStages, SB = C::kStageBytes;
     extern __shared__ uint8_t smem_raw[];
@@ -241,7 +260,7 @@ __global__ void __launch_bounds__(Cfg<MODE, WF>::kThreads, 1)
         }
         for (int a = 0; a < 2; ++a) {
             mbar_init(tfull + a, 1);
-            mbar_init(tempty + a, 4);
+            mbar_init(tempty + a, C::kEpiWarps);
         }
         for (int r = 0; r < UR; ++r) {
             mbar_init(ufull + r, 1);
@@ -268,8 +287,12 @@ __global__ void __launch_bounds__(Cfg<MODE, WF>::kThreads, 1)
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem_base = *tmem_slot;
+    // the prologue above touched no global memory; wait for the predecessor here
+    griddep_wait();
+    griddep_launch();
 
-    const int total_units = __ldg(p.tile_base + p.Etot) * p.n_tiles;
+    const int nt = p.n_tiles;
+    const int total_units = __ldg(p.tile_base + p.Etot) * nt;
     const int KB = p.K / BK;
 
     if (warp == 0) {
@@ -287,7 +310,7 @@ __global__ void __launch_bounds__(Cfg<MODE, WF>::kThreads, 1)
                 break;
             }
             if (u < 0) break;
-            const Unit U = decode_unit(u, p);
+            const Unit U = decode_unit<C::kSub>(u, p, nt);
             const bool sh = U.e >= p.E;
             const int z = sh ? 0 : U.e;
             for (int kb = 0; kb < KB; ++kb) {
@@ -300,9 +323,11 @@ __global__ void __launch_bounds__(Cfg<MODE, WF>::kThreads, 1)
                 }
                 if (lane == 0) {
                     uint8_t* sa = smem + stage * SB;
-                    uint8_t* sb = sa + A_BYTES;
-                    mbar_arrive_expect_tx(full + stage, C::kTxBytes);
+                    uint8_t* sb = sa + C::kABytes;
+                    const bool a1 = C::kSub == 2 && U.rows > BM;  // second 128-row sub-tile present
+                    mbar_arrive_expect_tx(full + stage, C::kTxB + (a1 ? 2u : 1u) * A_BYTES);
                     tma_load_2d(sa, &tmA, full + stage, kb * BK, U.row0);
+                    if (a1) tma_load_2d(sa + A_BYTES, &tmA, full + stage, kb * BK, U.row0 + BM);
                     if (Q4) {
                         // packed rows [N][32 B] and scales [2 groups][rows] fp16
                         uint8_t* sp = sb + B_BYTES;
@@ -365,8 +390,13 @@ __global__ void __launch_bounds__(Cfg<MODE, WF>::kThreads, 1)
             okl = __shfl_sync(0xFFFFFFFFu, okl, 0);
             if (!okl) break;
             tc_fence_after();
-            const uint32_t d_tmem = tmem_base + uint32_t(acc * BN);
-            const uint32_t idesc = decode_unit(u, p).rows <= 64 ? C::kIdesc64 : IDESC;
+            const int rows = decode_unit<C::kSub>(u, p, nt).rows;
+            const uint32_t d_tmem = tmem_base + uint32_t(acc * C::kSub * BN);
+            const bool m64 = min(rows, BM) <= 64;
+            const uint32_t idesc = m64 ? C::kIdesc64 : IDESC;
+            // second sub-tile (rows 128..255 of the unit), its accumulator 256 columns on
+            const bool sub1 = C::kSub == 2 && rows > BM;
+            const uint32_t idesc1 = rows - BM <= 64 ? C::kIdesc64 : IDESC;
             for (int kb = 0; kb < KB; ++kb) {
                 if (lane == 0) okl = mbar_wait_bounded(ready + stage, phase, abort_flag, p.err, p.wait_ns);
                 okl = __shfl_sync(0xFFFFFFFFu, okl, 0);
@@ -377,7 +407,7 @@ __global__ void __launch_bounds__(Cfg<MODE, WF>::kThreads, 1)
                 tc_fence_after();
                 if (lane == 0) {
                     const uint32_t a0 = smem_u32(smem + stage * SB);
-                    const uint32_t b0 = a0 + A_BYTES;
+                    const uint32_t b0 = a0 + C::kABytes;
 #pragma unroll
                     for (int j = 0; j < BK / 16; ++j) {
                         // A: K-major, advance 16 elements = 32 bytes inside the swizzle row.
@@ -387,6 +417,9 @@ __global__ void __launch_bounds__(Cfg<MODE, WF>::kThreads, 1)
                         const uint64_t bd = Q4 ? sdesc_sw128(b0 + j * 32, 16, 1024)
                                                : sdesc_sw128(b0 + j * 2048, B_CHUNK, 1024);
                         umma_bf16(d_tmem, ad, bd, idesc, (kb | j) != 0);
+                        if (sub1)
+                            umma_bf16(d_tmem + BN, sdesc_sw128(a0 + A_BYTES + j * 32, 16, 1024), bd, idesc1,
+                                      (kb | j) != 0);
                     }
                     umma_commit(empty + stage);
                 }
@@ -399,7 +432,7 @@ __global__ void __launch_bounds__(Cfg<MODE, WF>::kThreads, 1)
             if (!ok) break;
             if (lane == 0) umma_commit(tfull + acc);
             __syncwarp();
-            if (++acc == 2) {
+            if (++acc == C::kAcc) {
                 acc = 0;
                 acc_phase ^= 1u;
             }
@@ -410,8 +443,9 @@ __global__ void __launch_bounds__(Cfg<MODE, WF>::kThreads, 1)
             mbar_wait_bounded(drain, 0, nullptr, p.err, kDrainLimitNs);
         }
         __syncwarp();
-    } else if (warp < 6) {
-        // ------------------------------------------------ epilogue (warps 2..5)
+    } else if (warp < 2 + C::kEpiWarps) {
+        // ------------------------------------------------ epilogue (warps 2 .. 2+kEpiWarps-1)
+        // Warp w reads TMEM lanes 32*(w%4) .. +31, for each sub-tile in turn.
         const int q = warp & 3;
         int acc = 0;
         uint32_t acc_phase = 0;
@@ -422,80 +456,91 @@ __global__ void __launch_bounds__(Cfg<MODE, WF>::kThreads, 1)
             int u = -1;
             if (!ring_read(u, uslot, uphase, unit_ring, ufull, uempty, abort_flag, p.err, p.wait_ns)) break;
             if (u < 0) break;
-            const Unit U = decode_unit(u, p);
+            const Unit U = decode_unit<C::kSub>(u, p, nt);
             int okl = 1;
             if (lane == 0) okl = mbar_wait_bounded(tfull + acc, acc_phase, abort_flag, p.err, p.wait_ns);
             okl = __shfl_sync(0xFFFFFFFFu, okl, 0);
             if (!okl) break;
             tc_fence_after();
-            // M=128: lane i of quadrant q is row 32q + i. M=64 (tiles of <= 64
-            // rows): only lanes 0-15 of each quadrant hold rows, 16q + i.
-            const bool m64 = U.rows <= 64;
-            const int rit = m64 ? q * 16 + lane : q * 32 + lane;
-            const bool valid = (!m64 || lane < 16) && rit < U.rows;
-            const int64_t row = int64_t(U.row0) + rit;
-            const uint32_t tb = tmem_base + (uint32_t(q * 32) << 16) + uint32_t(acc * BN);
-            if (MODE == 0) {
 #pragma unroll 1
-                for (int c = 0; c < 4; ++c) {
-                    uint32_t g[32], v[32];
-                    tmem_ld_32x32b_x32(tb + c * 32, g);
-                    tmem_ld_32x32b_x32(tb + 128 + c * 32, v);
-                    tmem_ld_wait();
-                    const int col = U.n * 128 + c * 32;
-                    if (valid && col < p.n_out) {
-                        uint32_t pk[16];
+            for (int sub = 0; sub < C::kSub; ++sub) {
+                const int rows = min(BM, U.rows - sub * BM);
+                if (rows <= 0) break;
+                // M=128: lane i of quadrant q is row 32q + i. M=64 (sub-tiles of
+                // <= 64 rows): only lanes 0-15 of each quadrant hold rows, 16q + i.
+                const bool m64 = rows <= 64;
+                const int rit = m64 ? q * 16 + lane : q * 32 + lane;
+                const bool valid = (!m64 || lane < 16) && rit < rows;
+                const int64_t row = int64_t(U.row0) + sub * BM + rit;
+                const uint32_t tb = tmem_base + (uint32_t(q * 32) << 16) + uint32_t((acc * C::kSub + sub) * BN);
+                if (MODE == 0) {
+                    // gate columns first, then the up columns (128 each)
+                    constexpr int hw = 128;
+#pragma unroll 1
+                    for (int c = 0; c < hw / 32; ++c) {
+                        uint32_t g[32], v[32];
+                        tmem_ld_32x32b_x32(tb + c * 32, g);
+                        tmem_ld_32x32b_x32(tb + hw + c * 32, v);
+                        tmem_ld_wait();
+                        const int col = U.n * hw + c * 32;
+                        if (valid && col < p.n_out) {
+                            uint32_t pk[16];
 #pragma unroll
-                        for (int i = 0; i < 16; ++i) {
-                            const float h0 = swiglu(__uint_as_float(g[2 * i]), __uint_as_float(v[2 * i]), p.limit);
-                            const float h1 =
-                                swiglu(__uint_as_float(g[2 * i + 1]), __uint_as_float(v[2 * i + 1]), p.limit);
-                            range_bad |= !(f16_range_ok(h0) && f16_range_ok(h1));
-                            pk[i] = pack_f16x2(h0, h1);
+                            for (int i = 0; i < 16; ++i) {
+                                const float h0 =
+                                    swiglu(__uint_as_float(g[2 * i]), __uint_as_float(v[2 * i]), p.limit);
+                                const float h1 =
+                                    swiglu(__uint_as_float(g[2 * i + 1]), __uint_as_float(v[2 * i + 1]), p.limit);
+                                range_bad |= !(f16_range_ok(h0) && f16_range_ok(h1));
+                                pk[i] = pack_f16x2(h0, h1);
+                            }
+                            uint4* dst = reinterpret_cast<uint4*>(p.out + row * p.n_out + col);
+#pragma unroll
+                            for (int i = 0; i < 4; ++i)
+                                dst[i] = make_uint4(pk[4 * i], pk[4 * i + 1], pk[4 * i + 2], pk[4 * i + 3]);
                         }
-                        uint4* dst = reinterpret_cast<uint4*>(p.out + row * p.n_out + col);
-#pragma unroll
-                        for (int i = 0; i < 4; ++i) dst[i] = make_uint4(pk[4 * i], pk[4 * i + 1], pk[4 * i + 2], pk[4 * i + 3]);
                     }
-                }
-            } else {
-                float w = 0.f;
-                if (valid) {
-                    const int sp = __ldg(p.sorted_pair + row);
-                    w = sp >= 0 ? __ldg(p.topk_w + sp) : 1.0f;
-                }
+                } else {
+                    float w = 0.f;
+                    if (valid) {
+                        const int sp = __ldg(p.sorted_pair + row);
+                        w = sp >= 0 ? __ldg(p.topk_w + sp) : 1.0f;
+                    }
 #pragma unroll 1
-                for (int c = 0; c < BN / 32; ++c) {
-                    uint32_t v[32];
-                    tmem_ld_32x32b_x32(tb + c * 32, v);
-                    tmem_ld_wait();
-                    const int col = U.n * BN + c * 32;
-                    if (valid && col < p.n_out) {
-                        uint32_t pk[16];
+                    for (int c = 0; c < BN / 32; ++c) {
+                        uint32_t v[32];
+                        tmem_ld_32x32b_x32(tb + c * 32, v);
+                        tmem_ld_wait();
+                        const int col = U.n * BN + c * 32;
+                        if (valid && col < p.n_out) {
+                            uint32_t pk[16];
 #pragma unroll
-                        for (int i = 0; i < 16; ++i) {
-                            const float y0 = w * __uint_as_float(v[2 * i]), y1 = w * __uint_as_float(v[2 * i + 1]);
-                            range_bad |= !(f16_range_ok(y0) && f16_range_ok(y1));
-                            pk[i] = pack_f16x2(y0, y1);
+                            for (int i = 0; i < 16; ++i) {
+                                const float y0 = w * __uint_as_float(v[2 * i]);
+                                const float y1 = w * __uint_as_float(v[2 * i + 1]);
+                                range_bad |= !(f16_range_ok(y0) && f16_range_ok(y1));
+                                pk[i] = pack_f16x2(y0, y1);
+                            }
+                            uint4* dst = reinterpret_cast<uint4*>(p.out + row * p.n_out + col);
+#pragma unroll
+                            for (int i = 0; i < 4; ++i)
+                                dst[i] = make_uint4(pk[4 * i], pk[4 * i + 1], pk[4 * i + 2], pk[4 * i + 3]);
                         }
-                        uint4* dst = reinterpret_cast<uint4*>(p.out + row * p.n_out + col);
-#pragma unroll
-                        for (int i = 0; i < 4; ++i) dst[i] = make_uint4(pk[4 * i], pk[4 * i + 1], pk[4 * i + 2], pk[4 * i + 3]);
                     }
                 }
             }
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(tempty + acc);
-            if (++acc == 2) {
+            if (++acc == C::kAcc) {
                 acc = 0;
                 acc_phase ^= 1u;
             }
         }
         if (range_bad) set_error(p.err, MOE_DEVERR_RANGE);
     } else if (C::kTransform) {
-        // ------------------------------------------------ transform (warps 6..9)
-        const int ct = threadIdx.x - 192;  // 0..127
+        // ------------------------------------------------ transform (the last four warps)
+        const int ct = threadIdx.x - 32 * (2 + C::kEpiWarps);  // 0..127
         int stage = 0;
         uint32_t phase = 0;
         bool ok = true;
@@ -513,7 +558,7 @@ __global__ void __launch_bounds__(Cfg<MODE, WF>::kThreads, 1)
                     ok = false;
                     break;
                 }
-                uint8_t* sb = smem + stage * SB + A_BYTES;
+                uint8_t* sb = smem + stage * SB + C::kABytes;
                 if (Q4) {
                     // rows ct and ct+128 of the 256-row B tile; row r: 8 words
                     // (k 0..63) -> 8 chunks of 8 fp16 at r*128 + ((c ^ (r%8)) * 16)
@@ -569,12 +614,20 @@ __global__ void __launch_bounds__(Cfg<MODE, WF>::kThreads, 1)
 // ---------------------------------------------------------------------------- K3 schedule
 
 // One block of 512 threads; thread e owns expert e (Etot <= 257).
+// tile_base[0 .. Etot] is the exclusive prefix of 128-row tiles per expert,
+// tile_base[Etot+1 .. 2*Etot+1] that of 256-row tiles (the gate/up units).
 __global__ void __launch_bounds__(512) schedule_kernel(const int32_t* __restrict__ offsets, int Etot, int variant,
-                                                       int stream_max, int32_t* __restrict__ tile_base,
+                                                       int stream_max,
+                                                       int32_t* __restrict__ tile_base,
                                                        int32_t* __restrict__ stream_list,
-                                                       int32_t* __restrict__ n_stream, uint32_t* err) {
-    __shared__ int sums[2][16];
+                                                       int32_t* __restrict__ n_stream, int32_t* __restrict__ fix,
+                                                       int n_fix, uint32_t* err) {
+    __shared__ int sums[3][16];
+    griddep_wait();
+    griddep_launch();
+
     const int e = threadIdx.x, lane = e & 31, w = e >> 5;
+    for (int i = e; i < n_fix; i += blockDim.x) fix[i] = 0;  // K-split arrivals of the streaming gate/up
     int kept = 0;
     if (e < Etot) {
         kept = offsets[e + 1] - offsets[e];
@@ -586,34 +639,44 @@ __global__ void __launch_bounds__(512) schedule_kernel(const int32_t* __restrict
     const int is_stream =
         (kept > 0 && (variant == MOE_VARIANT_STREAM || (variant == MOE_VARIANT_AUTO && kept <= stream_max))) ? 1 : 0;
     const int tiles = (kept > 0 && !is_stream) ? (kept + kTileM - 1) / kTileM : 0;
-    int it = tiles, is = is_stream;
+    const int tiles2 = (tiles + 1) >> 1;
+    int it = tiles, is = is_stream, i2 = tiles2;
 #pragma unroll
     for (int off = 1; off < 32; off <<= 1) {
         const int a = __shfl_up_sync(0xFFFFFFFFu, it, off);
         const int b = __shfl_up_sync(0xFFFFFFFFu, is, off);
+        const int c = __shfl_up_sync(0xFFFFFFFFu, i2, off);
         if (lane >= off) {
             it += a;
             is += b;
+            i2 += c;
         }
     }
     if (lane == 31) {
         sums[0][w] = it;
         sums[1][w] = is;
+        sums[2][w] = i2;
     }
     __syncthreads();
-    int bt = 0, bs = 0, tt = 0, ts = 0;
+    int bt = 0, bs = 0, b2 = 0, tt = 0, ts = 0, t2 = 0;
     for (int i = 0; i < 16; ++i) {
         if (i < w) {
             bt += sums[0][i];
             bs += sums[1][i];
+            b2 += sums[2][i];
         }
         tt += sums[0][i];
         ts += sums[1][i];
+        t2 += sums[2][i];
     }
-    if (e < Etot) tile_base[e] = bt + it - tiles;
+    if (e < Etot) {
+        tile_base[e] = bt + it - tiles;
+        tile_base[Etot + 1 + e] = b2 + i2 - tiles2;
+    }
     if (is_stream) stream_list[bs + is - 1] = e;
     if (e == 0) {
         tile_base[Etot] = tt;
+        tile_base[2 * Etot + 1] = t2;
         n_stream[0] = ts;
         n_stream[1] = 0;  // unit counters of the two tcgen05 GEMMs (claimed with atomicAdd)
         n_stream[2] = 0;
@@ -629,6 +692,8 @@ __global__ void __launch_bounds__(256) gather_rows_kernel(const uint16_t* __rest
                                                           const int32_t* __restrict__ sorted_token,
                                                           const int32_t* __restrict__ offsets, int Etot, int d,
                                                           int T, uint16_t* __restrict__ xg, uint32_t* err) {
+    griddep_wait();
+    griddep_launch();
     const int vec = d / 8;
     const int64_t total = int64_t(offsets[Etot]) * vec;
     for (int64_t i = int64_t(blockIdx.x) * blockDim.x + threadIdx.x; i < total; i += int64_t(gridDim.x) * blockDim.x) {
@@ -717,22 +782,26 @@ bool map_q4_scales(CUtensorMap* m, const void* base, int nexp, int K, int N, int
     return make_map(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, base, 3, dims, str, box, CU_TENSOR_MAP_SWIZZLE_NONE);
 }
 
-template <int MODE, int WF>
+template <int MODE, int WF, int SUB>
 cudaError_t launch_gemm(const CUtensorMap& A, const CUtensorMap& B0, const CUtensorMap& B1, const CUtensorMap& S0,
                         const CUtensorMap& S1, const GemmParams& p, cudaStream_t s) {
-    using C = Cfg<MODE, WF>;
+    using C = Cfg<MODE, WF, SUB>;
     static int configured_dev = -1;
     int dev = 0;
     cudaGetDevice(&dev);
     if (configured_dev != dev) {
-        cudaError_t e = cudaFuncSetAttribute(grouped_gemm_kernel<MODE, WF>,
+        cudaError_t e = cudaFuncSetAttribute(grouped_gemm_kernel<MODE, WF, SUB>,
                                              cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmem);
         if (e != cudaSuccess) return e;
         configured_dev = dev;
     }
+    GemmParams q = p;
+    if (C::kSub == 2) q.tile_base = p.tile_base + p.Etot + 1;  // 256-row units
     {
         ProfScope prof_(MODE == 0 ? MOE_K_TC_GATEUP : MOE_K_TC_DOWN, s);
-        grouped_gemm_kernel<MODE, WF><<<num_sms(), C::kThreads, C::kSmem, s>>>(A, B0, B1, S0, S1, p);
+        const cudaError_t le = launch_pdl(grouped_gemm_kernel<MODE, WF, SUB>, dim3(num_sms()), dim3(C::kThreads),
+                                          C::kSmem, s, A, B0, B1, S0, S1, q);
+        if (le != cudaSuccess) return le;
     }
     return cudaGetLastError();
 }
@@ -740,11 +809,13 @@ cudaError_t launch_gemm(const CUtensorMap& A, const CUtensorMap& B0, const CUten
 }  // namespace tc
 
 cudaError_t launch_schedule(const Dims& D, const int32_t* offsets, int32_t* tile_base, int32_t* stream_list,
-                            int32_t* n_stream, uint32_t* err, cudaStream_t s) {
+                            int32_t* n_stream, int32_t* fix, int n_fix, uint32_t* err, cudaStream_t s) {
     int smax = D.stream_max_rows;
     {
         ProfScope prof_(MOE_K_SCHEDULE, s);
-        schedule_kernel<<<1, 512, 0, s>>>(offsets, D.Etot, D.variant, smax, tile_base, stream_list, n_stream, err);
+        const cudaError_t le = launch_pdl(schedule_kernel, dim3(1), dim3(512), 0, s, offsets, D.Etot, D.variant,
+                                          smax, tile_base, stream_list, n_stream, fix, n_fix, err);
+        if (le != cudaSuccess) return le;
     }
     return cudaGetLastError();
 }
@@ -758,10 +829,13 @@ cudaError_t launch_gather(const Dims& D, const uint16_t* x, const int32_t* sorte
     if (blocks < 1) blocks = 1;
     {
         ProfScope prof_(MOE_K_GATHER, s);
-        if (D.fmt == MOE_WEIGHTS_Q4G32)
-            gather_rows_kernel<true><<<int(blocks), 256, 0, s>>>(x, sorted_token, offsets, D.Etot, D.d, D.T, xg, err);
-        else
-            gather_rows_kernel<false><<<int(blocks), 256, 0, s>>>(x, sorted_token, offsets, D.Etot, D.d, D.T, xg, err);
+        const cudaError_t le =
+            D.fmt == MOE_WEIGHTS_Q4G32
+                ? launch_pdl(gather_rows_kernel<true>, dim3(int(blocks)), dim3(256), 0, s, x, sorted_token, offsets,
+                             D.Etot, D.d, D.T, xg, err)
+                : launch_pdl(gather_rows_kernel<false>, dim3(int(blocks)), dim3(256), 0, s, x, sorted_token, offsets,
+                             D.Etot, D.d, D.T, xg, err);
+        if (le != cudaSuccess) return le;
     }
     return cudaGetLastError();
 }
@@ -798,13 +872,13 @@ cudaError_t launch_tensor_ffn(const Dims& D, const uint16_t* xg, uint16_t* h, co
         p.n_tiles = (D.f + 127) / 128;
         p.out = h;
         p.unit_counter = counters;
-        if ((e = launch_gemm<0, 1>(mA, pg, pu, sg, su, p, s)) != cudaSuccess) return e;
+        if ((e = launch_gemm<0, 1, 2>(mA, pg, pu, sg, su, p, s)) != cudaSuccess) return e;
         p.K = D.f;
         p.n_out = D.d;
         p.n_tiles = (D.d + BN - 1) / BN;
         p.out = y_rows;
         p.unit_counter = counters + 1;
-        return launch_gemm<1, 1>(mH, pd, pd, sd, sd, p, s);
+        return launch_gemm<1, 1, 2>(mH, pd, pd, sd, sd, p, s);
     }
     CUtensorMap mG, mU, mSG, mSU, mD, mSD;
     if (!map_weights(&mG, w->w_gate, D.E, D.d, D.f) || !map_weights(&mU, w->w_up, D.E, D.d, D.f) ||
@@ -825,14 +899,14 @@ cudaError_t launch_tensor_ffn(const Dims& D, const uint16_t* xg, uint16_t* h, co
     p.n_tiles = (D.f + 127) / 128;
     p.out = h;
     p.unit_counter = counters;
-    if ((e = launch_gemm<0, 0>(mA, mG, mU, mSG, mSU, p, s)) != cudaSuccess) return e;
+    if ((e = launch_gemm<0, 0, 1>(mA, mG, mU, mSG, mSU, p, s)) != cudaSuccess) return e;
     // S6: down + gate scale -> y_rows
     p.K = D.f;
     p.n_out = D.d;
     p.n_tiles = (D.d + BN - 1) / BN;
     p.out = y_rows;
     p.unit_counter = counters + 1;
-    return D.down_f16 ? launch_gemm<1, 2>(mH, mD, mD, mSD, mSD, p, s) : launch_gemm<1, 0>(mH, mD, mD, mSD, mSD, p, s);
+    return D.down_f16 ? launch_gemm<1, 2, 1>(mH, mD, mD, mSD, mSD, p, s) : launch_gemm<1, 0, 1>(mH, mD, mD, mSD, mSD, p, s);
 }
 
 }  // namespace moe

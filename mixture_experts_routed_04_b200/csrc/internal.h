@@ -34,7 +34,7 @@ struct WsLayout {
     size_t err;                                    // uint32 error word (always at 0)
     size_t blockcounts, blockbase;                 // permute: int32 [perm_blocks, E]
     size_t tile_base, stream_list, n_stream;       // expert_ffn schedule
-    size_t xg, h, part;                            // expert_ffn: gathered x, h, split-K partials
+    size_t xg, h, part, fix;                       // expert_ffn: gathered x, h, split-K partials + arrivals
     size_t topk_idx, topk_w, counts, kept, offsets, sorted_token, sorted_pair, pair_row, y_rows;  // forward
     size_t x_dev, logits_dev, out_dev;             // forward_host
     size_t total;
@@ -69,6 +69,24 @@ cudaError_t launch_combine(const Dims& D, const uint16_t* y_rows, const int32_t*
 
 // ---- device properties, cached per device
 int num_sms();
+
+// Launch with programmatic stream serialization (see griddep_wait): the
+// kernel may be scheduled before its predecessor on the stream completes.
+template <typename... KArgs, typename... Args>
+inline cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t s,
+                              Args... args) {
+    cudaLaunchConfig_t cfg{};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = s;
+    cudaLaunchAttribute at[1];
+    at[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    at[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = at;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kernel, static_cast<KArgs>(args)...);
+}
 
 // ---- optional per-kernel event timing (moe_profile_enable); no-op when off
 class ProfScope {

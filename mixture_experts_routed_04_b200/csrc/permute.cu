@@ -63,6 +63,8 @@ __global__ void __launch_bounds__(kPermWarps * 32) perm_count_kernel(const int32
                                                                      int32_t* __restrict__ blockcounts,
                                                                      uint32_t* err) {
     __shared__ int hist[kPermWarps][kMaxE];
+    griddep_wait();
+    griddep_launch();
     warp_histograms(topk_idx, pairs, E, hist, err);
     for (int e = threadIdx.x; e < E; e += blockDim.x) {
         int s = 0;
@@ -79,6 +81,9 @@ __global__ void __launch_bounds__(kMaxE) perm_scan_kernel(const int32_t* __restr
                                                          int32_t* __restrict__ counts, int32_t* __restrict__ kept,
                                                          int32_t* __restrict__ offsets) {
     __shared__ int warp_sums[kMaxE / 32];
+    griddep_wait();
+    griddep_launch();
+
     const int e = threadIdx.x, lane = e & 31, w = e >> 5;
     int kv = 0;
     if (e < E) {
@@ -126,6 +131,8 @@ __global__ void __launch_bounds__(kPermWarps * 32) perm_scatter_kernel(
     int32_t* __restrict__ sorted_token, int32_t* __restrict__ sorted_pair, int32_t* __restrict__ pair_row,
     int shared_T, uint32_t* err) {
     __shared__ int hist[kPermWarps][kMaxE];
+    griddep_wait();
+    griddep_launch();
     warp_histograms(topk_idx, pairs, E, hist, nullptr);  // errors were reported by the count pass
     // warp totals -> warp bases (block base + earlier warps), per expert
     for (int e = threadIdx.x; e < E; e += blockDim.x) {
@@ -180,20 +187,33 @@ __global__ void __launch_bounds__(kPermWarps * 32) perm_scatter_kernel(
 cudaError_t launch_permute(const Dims& D, const int32_t* topk_idx, int32_t* blockcounts, int32_t* blockbase,
                            int32_t* counts, int32_t* kept, int32_t* offsets, int32_t* sorted_token,
                            int32_t* sorted_pair, int32_t* pair_row, uint32_t* err, cudaStream_t s) {
+    if (D.pairs == 0) {  // empty batch: zero counts and offsets, nothing to scatter
+        if (cudaMemsetAsync(counts, 0, size_t(D.Etot) * 4, s) != cudaSuccess ||
+            cudaMemsetAsync(kept, 0, size_t(D.Etot) * 4, s) != cudaSuccess ||
+            cudaMemsetAsync(offsets, 0, size_t(D.Etot + 1) * 4, s) != cudaSuccess)
+            return cudaGetLastError();
+        return cudaSuccess;
+    }
     const int nb = D.perm_blocks;
     const int shared_T = D.has_shared ? D.T : 0;
     {
         ProfScope prof_(MOE_K_PERM_COUNT, s);
-        perm_count_kernel<<<nb, kPermWarps * 32, 0, s>>>(topk_idx, D.pairs, D.E, blockcounts, err);
+        const cudaError_t le = launch_pdl(perm_count_kernel, dim3(nb), dim3(kPermWarps * 32), 0, s, topk_idx,
+                                          D.pairs, D.E, blockcounts, err);
+        if (le != cudaSuccess) return le;
     }
     {
         ProfScope prof_(MOE_K_PERM_SCAN, s);
-        perm_scan_kernel<<<1, kMaxE, 0, s>>>(blockcounts, nb, D.E, D.cap, shared_T, blockbase, counts, kept, offsets);
+        const cudaError_t le = launch_pdl(perm_scan_kernel, dim3(1), dim3(kMaxE), 0, s, blockcounts, nb, D.E,
+                                          D.cap, shared_T, blockbase, counts, kept, offsets);
+        if (le != cudaSuccess) return le;
     }
     {
         ProfScope prof_(MOE_K_PERM_SCATTER, s);
-        perm_scatter_kernel<<<nb, kPermWarps * 32, 0, s>>>(topk_idx, D.pairs, D.k, D.E, D.cap, blockbase, offsets,
-                                                       sorted_token, sorted_pair, pair_row, shared_T, err);
+        const cudaError_t le = launch_pdl(perm_scatter_kernel, dim3(nb), dim3(kPermWarps * 32), 0, s, topk_idx,
+                                          D.pairs, D.k, D.E, D.cap, blockbase, offsets, sorted_token, sorted_pair,
+                                          pair_row, shared_T, err);
+        if (le != cudaSuccess) return le;
     }
     return cudaGetLastError();
 }

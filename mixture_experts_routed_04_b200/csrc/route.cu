@@ -23,6 +23,8 @@ MOE_DEV bool beats(float va, int ia, float vb, int ib) { return va > vb || (va =
 __global__ void __launch_bounds__(256) route_topk_softmax_kernel(const float* __restrict__ logits, int T, int E,
                                                                  int k, int32_t* __restrict__ topk_idx,
                                                                  float* __restrict__ topk_w) {
+    griddep_wait();
+    griddep_launch();
     const int lane = threadIdx.x & 31;
     const int warps_per_block = blockDim.x >> 5;
     const int64_t t = int64_t(blockIdx.x) * warps_per_block + (threadIdx.x >> 5);
@@ -88,7 +90,9 @@ cudaError_t launch_route(const float* logits, int T, int E, int k, int32_t* topk
     const int blocks = (T + wpb - 1) / wpb;
     {
         ProfScope prof_(MOE_K_ROUTE, stream);
-        route_topk_softmax_kernel<<<blocks, threads, 0, stream>>>(logits, T, E, k, topk_idx, topk_w);
+        const cudaError_t le = launch_pdl(route_topk_softmax_kernel, dim3(blocks), dim3(threads), 0, stream,
+                                          logits, T, E, k, topk_idx, topk_w);
+        if (le != cudaSuccess) return le;
     }
     return cudaGetLastError();
 }

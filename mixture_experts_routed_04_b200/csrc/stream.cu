@@ -19,8 +19,10 @@
 //              The tensor pipe only keeps the instruction count per weight byte
 //              low so the kernel stays HBM-bound.
 // Gate/up (bf16 x and weights) with one K slice applies the clamped SwiGLU and
-// writes h (fp16); with several, fp32 partials go to the workspace and
-// stream_reduce finishes (fixed order, deterministic). Down runs in fp16 (h is
+// writes h (fp16); with several, fp32 partials go to the workspace and the
+// warp that completes the last slice of a 16-column strip sums them in slice
+// order and applies the SwiGLU (deterministic: the order never depends on
+// which CTA finishes last). Down runs in fp16 (h is
 // fp16; W_down prepared as fp16, or converted in registers after ldmatrix) and
 // writes y = w_pair * (h W_down) (fp16). All waits are bounded; no TMA
 // multicast; no named barriers, so an abort never strands a warp.
@@ -52,6 +54,8 @@ struct StreamParams {
     const float* topk_w;
     uint16_t* out;        // mode 0: h [rows, f]; mode 1: y_rows [rows, d]
     float* part;          // mode 0 with ks > 1: [ks, 2, rows, f] fp32
+    int32_t* fix;         // mode 0 with ks > 1: arrivals per (list entry, 64-column slice, warp), zeroed
+                          // by the schedule kernel
     int64_t rows;
     float limit;
     int down_f16;         // mode 1: W_down already fp16 (no conversion)
@@ -60,7 +64,7 @@ struct StreamParams {
 };
 
 struct SUnit {
-    int e, n0, k0, ks, row0, nrows;
+    int i, e, n0, k0, ks, row0, nrows;  // i: position in the streaming list
 };
 
 MOE_DEV SUnit decode(int u, const StreamParams& p) {
@@ -69,6 +73,7 @@ MOE_DEV SUnit decode(int u, const StreamParams& p) {
     const int i = u / per;
     const int rem = u - i * per;
     SUnit U;
+    U.i = i;
     U.e = __ldg(p.stream_list + i);
     U.n0 = (rem / p.ks) * NS;
     U.ks = rem % p.ks;
@@ -137,6 +142,9 @@ __global__ void __launch_bounds__(THREADS, 1)
         fence_mbar_init();
     }
     __syncthreads();
+    // the prologue above touched no global memory; wait for the predecessor here
+    griddep_wait();
+    griddep_launch();
 
     const int total = __ldg(p.n_stream) * (p.N / NS) * p.ks;
     const int KB = p.kslice / BKS;
@@ -269,35 +277,35 @@ __global__ void __launch_bounds__(THREADS, 1)
                 }
             }
         }
-    }
-    if (range_bad) set_error(p.err, MOE_DEVERR_RANGE);
-}
-
-// h = swiglu(sum_ks part_g, sum_ks part_u) for the streaming experts' rows (ks > 1).
-__global__ void __launch_bounds__(256) stream_reduce_kernel(const float* __restrict__ part, int ks, int64_t rows,
-                                                            int f, const int32_t* __restrict__ offsets,
-                                                            const int32_t* __restrict__ stream_list,
-                                                            const int32_t* __restrict__ n_stream, float limit,
-                                                            uint16_t* __restrict__ h, uint32_t* err) {
-    const int n = __ldg(n_stream);
-    bool range_bad = false;
-    for (int i = blockIdx.x; i < n; i += gridDim.x) {
-        const int e = __ldg(stream_list + i);
-        const int r0 = __ldg(offsets + e), nr = __ldg(offsets + e + 1) - r0;
-        for (int j = threadIdx.x; j < nr * f; j += blockDim.x) {
-            const int64_t row = r0 + j / f;
-            const int col = j % f;
-            float g = 0.f, u = 0.f;
-            for (int s = 0; s < ks; ++s) {
-                g += part[((int64_t(s) * 2 + 0) * rows + row) * f + col];
-                u += part[((int64_t(s) * 2 + 1) * rows + row) * f + col];
+        if (MODE == 0 && p.ks > 1 && ok) {
+            // K-split fixup: the warp that writes the last of the ks partial
+            // slices of its 16 columns sums them in slice order (the result does
+            // not depend on which CTA arrives last) and applies the SwiGLU.
+            __threadfence();
+            int last = 0;
+            if (lane == 0) {
+                const int64_t slot = (int64_t(U.i) * (p.N / NS) + U.n0 / NS) * CONSUMERS + cw;
+                last = atomicAdd(p.fix + slot, 1) == p.ks - 1;
             }
-            const float hv = swiglu(g, u, limit);
-            range_bad |= !f16_range_ok(hv);
-            h[row * f + col] = to_f16(hv);
+            last = __shfl_sync(0xFFFFFFFFu, last, 0);
+            if (last) {
+                __threadfence();
+                for (int j = lane; j < U.nrows * 16; j += 32) {
+                    const int64_t row = int64_t(U.row0) + j / 16;
+                    const int n = U.n0 + cw * 16 + (j & 15);
+                    float g = 0.f, v = 0.f;
+                    for (int sl = 0; sl < p.ks; ++sl) {
+                        g += __ldcg(p.part + ((int64_t(sl) * 2 + 0) * p.rows + row) * p.N + n);
+                        v += __ldcg(p.part + ((int64_t(sl) * 2 + 1) * p.rows + row) * p.N + n);
+                    }
+                    const float h = swiglu(g, v, p.limit);
+                    range_bad |= !f16_range_ok(h);
+                    p.out[row * p.N + n] = to_f16(h);
+                }
+            }
         }
     }
-    if (range_bad) set_error(err, MOE_DEVERR_RANGE);
+    if (range_bad) set_error(p.err, MOE_DEVERR_RANGE);
 }
 
 using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
@@ -344,7 +352,9 @@ static cudaError_t launch_one(const CUtensorMap& W0, const CUtensorMap& W1, cons
     }
     {
         ProfScope prof_(MODE == 0 ? MOE_K_STREAM_GATEUP : MOE_K_STREAM_DOWN, s);
-        stream_kernel<MODE><<<grid, THREADS, SMEM_BYTES, s>>>(W0, W1, S0, S1, X, p);
+        const cudaError_t le = launch_pdl(stream_kernel<MODE>, dim3(grid), dim3(THREADS), SMEM_BYTES, s, W0, W1,
+                                          S0, S1, X, p);
+        if (le != cudaSuccess) return le;
     }
     return cudaGetLastError();
 }
@@ -353,7 +363,8 @@ static cudaError_t launch_one(const CUtensorMap& W0, const CUtensorMap& W1, cons
 
 // Gate/up (+ reduce) then down for the experts on the streaming list.
 // xg: the gathered rows [rows, d] (bf16); h: [rows, f] fp16.
-cudaError_t launch_stream_ffn(const Dims& D, const uint16_t* xg, uint16_t* h, float* part, const int32_t* offsets,
+cudaError_t launch_stream_ffn(const Dims& D, const uint16_t* xg, uint16_t* h, float* part, int32_t* fix,
+                              const int32_t* offsets,
                               const int32_t* stream_list, const int32_t* n_stream, const int32_t* sorted_pair,
                               const float* topk_w, const moe_weights* w, uint16_t* y_rows, uint32_t* err,
                               uint64_t wait_ns, cudaStream_t s) {
@@ -393,16 +404,9 @@ cudaError_t launch_stream_ffn(const Dims& D, const uint16_t* xg, uint16_t* h, fl
     p.kslice = D.d / D.ks;
     p.out = h;
     p.part = part;
+    p.fix = fix;
     cudaError_t e = launch_one<0>(mG, mU, mSG, mSU, mX, p, grid, s);
     if (e != cudaSuccess) return e;
-    if (D.ks > 1) {
-        {
-            ProfScope prof_(MOE_K_STREAM_REDUCE, s);
-            stream_reduce_kernel<<<grid * 2, 256, 0, s>>>(part, D.ks, D.rows, D.f, offsets, stream_list, n_stream,
-                                                          D.limit, h, err);
-        }
-        if ((e = cudaGetLastError()) != cudaSuccess) return e;
-    }
     // down
     p.mode = 1;
     p.K = D.f;

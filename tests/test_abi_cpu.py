@@ -61,7 +61,7 @@ def test_max_rows_and_workspace(lib):
 
 
 @pytest.mark.parametrize("bad", [
-    dict(k=9), dict(k=3, E=2), dict(E=257), dict(d_model=100), dict(d_ff=32), dict(T=0),
+    dict(k=9), dict(k=3, E=2), dict(E=257), dict(d_model=100), dict(d_ff=32), dict(T=-1),
     dict(capacity_factor=-1.0), dict(capacity_factor=float("nan")), dict(variant=7), dict(weight_format=5)])
 def test_invalid_params_rejected_on_host(lib, bad):
     kw = dict(T=16, d_model=128, d_ff=256, E=8, k=2)
@@ -70,6 +70,17 @@ def test_invalid_params_rejected_on_host(lib, bad):
     assert b.workspace_size(p, b.WS_FORWARD) == 0
     st = lib.moe_route(ctypes.byref(p), None, None, None, None, 0, None)
     assert st == 1  # MOE_ERR_INVALID_ARG, before any launch
+
+
+def test_empty_batch_is_valid_and_launches_nothing(lib):
+    # T = 0: a rank with no tokens. Sizes are defined, the capacity is 0 and no kernel is launched.
+    p = b.params(0, 128, 256, 8, 2, capacity_factor=1.5)
+    assert b.workspace_size(p, b.WS_FORWARD) >= 256
+    assert b.capacity(p) == 0
+    for which in range(6):
+        n = ctypes.c_int(-1)
+        assert lib.moe_launch_count(ctypes.byref(p), which, ctypes.byref(n)) == 0
+        assert n.value == 0
 
 
 def test_unsupported_and_missing_buffers(lib):

@@ -14,6 +14,8 @@ automatic variant choice, W_down prepared as fp16): routing and permutation in
 full, and every output element (the Q4G32 workload: outputs of sampled tokens,
 each from its own definition).
 """
+import ctypes
+
 import numpy as np
 import pytest
 import torch
@@ -376,3 +378,24 @@ def test_out_of_range_expert_ids_are_flagged():
     assert int(bufs[0].sum()) == T * k - 2
     b.clear_error(ws)
     assert b.get_error(ws) == 0
+
+
+def test_empty_batch():
+    """T = 0: every call succeeds without a launch; counts and offsets come back zero."""
+    cfg = synth.LayerConfig("empty", T=0, d=128, f=128, E=8, k=2, has_shared=True, f_shared=128)
+    p = b.params_for(cfg)
+    Et = cfg.E + 1
+    i32 = dict(dtype=torch.int32, device="cuda")
+    counts = torch.full((Et,), -3, **i32)
+    ws = b.workspace(p, b.WS_FORWARD)
+    st = b.lib().moe_forward(ctypes.byref(p), None, None, None, None, ctypes.c_void_p(counts.data_ptr()),
+                             ctypes.c_void_p(ws.data_ptr()), ws.numel(), None)
+    torch.cuda.synchronize()
+    assert st == 0 and int(counts.abs().sum()) == 0
+    bufs = [torch.full((Et,), -3, **i32), torch.full((Et,), -3, **i32), torch.full((Et + 1,), -3, **i32),
+            torch.empty(1, **i32), torch.empty(1, **i32), torch.empty(1, **i32)]
+    wsp = b.workspace(p, b.WS_PERMUTE)
+    b.permute(p, torch.empty(1, 2, **i32), *bufs, wsp)
+    torch.cuda.synchronize()
+    assert all(int(t.abs().sum()) == 0 for t in bufs[:3])
+    assert b.get_error(ws) == 0 and b.get_error(wsp) == 0
