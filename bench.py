@@ -399,16 +399,48 @@ def own_arm(args, cfg):
                 tot += s0.elapsed_time(s1)
         ms_down_bf16 = tot / kb
 
-    # end to end through moe_forward_host: pinned host x/logits in, out back, per step
+    # End to end through the host-buffer entry points: every step copies its x and logits in
+    # from pinned host memory and its output back. "value": a pipelined loop over two streams
+    # (moe_forward_host_async, separate workspaces and host buffers per stream), so one step's
+    # copies overlap another's kernels, as a serving loop runs; "sync": one moe_forward_host
+    # call per step (copies, layer and copy back in sequence, then a host synchronisation).
     e2e = None
     if not args.no_e2e:
-        pe = b.workspace(p, b.WS_FORWARD_HOST)
-        x_h = d["x"].cpu().pin_memory()
-        l_h = d["logits"].cpu().pin_memory()
-        o_h = torch.empty(cfg.T, cfg.d, dtype=torch.float32).pin_memory()
+        h2d = cfg.T * cfg.d * 2 + cfg.T * cfg.E * 4
+        d2h = cfg.T * cfg.d * 4
+        ek = max(3, min(K, 50))
+        slots = [dict(stream=torch.cuda.Stream(), ws=b.workspace(p, b.WS_FORWARD_HOST),
+                      x=d["x"].cpu().pin_memory(), l=d["logits"].cpu().pin_memory(),
+                      o=torch.empty(cfg.T, cfg.d, dtype=torch.float32).pin_memory()) for _ in range(2)]
+
+        def step_async(i):
+            sl = slots[i % len(slots)]
+            b.forward_host_async(p, sl["x"], sl["l"], W, sl["o"], sl["ws"], stream=sl["stream"])
+
+        for i in range(2 * len(slots)):
+            step_async(i)
+        torch.cuda.synchronize()
+        t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        t0.record(stream)
+        for sl in slots:
+            sl["stream"].wait_event(t0)
+        for i in range(ek):
+            step_async(i)
+        for sl in slots:
+            ev = torch.cuda.Event()
+            ev.record(sl["stream"])
+            stream.wait_event(ev)
+        t1.record(stream)
+        t1.synchronize()
+        for sl in slots:
+            if b.get_error(sl["ws"]):
+                raise RuntimeError("device error word set (pipelined end-to-end loop)")
+        pipe_ms = max_over_ranks(t0.elapsed_time(t1) / ek, dist, "cuda")
+
+        pe = slots[0]["ws"]
+        x_h, l_h, o_h = slots[0]["x"], slots[0]["l"], slots[0]["o"]
         for _ in range(3):
             b.forward_host(p, x_h, l_h, W, o_h, pe)
-        ek = max(3, min(K, 50))
         e_ms = 0.0
         for _ in range(ek):
             flush.zero_()
@@ -419,9 +451,12 @@ def own_arm(args, cfg):
             s1.synchronize()
             e_ms += s0.elapsed_time(s1)
         e_ms = max_over_ranks(e_ms, dist, "cuda")
-        e2e = {"value": aggregate_tokens_per_s(cfg.T, world, e_ms / ek), "unit": "tokens/s",
-               "h2d_bytes_per_step": cfg.T * cfg.d * 2 + cfg.T * cfg.E * 4, "d2h_bytes_per_step": cfg.T * cfg.d * 4,
-               "ms_per_step": e_ms / ek}
+        e2e = {"value": aggregate_tokens_per_s(cfg.T, world, pipe_ms), "unit": "tokens/s",
+               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": pipe_ms,
+               "mode": "pipelined: moe_forward_host_async on 2 streams, pinned host buffers; no L2 flush "
+                       "(the touched weights exceed L2)",
+               "sync": {"value": aggregate_tokens_per_s(cfg.T, world, e_ms / ek), "ms_per_step": e_ms / ek,
+                        "mode": "one moe_forward_host call per step (L2 flushed between steps)"}}
 
     pk, pk_src = peaks()
     # Bound: the workload's arithmetic intensity against the measured ridge point.

@@ -34,7 +34,7 @@
  *     moe_clear_error(). A kernel that sets it stops early and returns; its
  *     outputs are then undefined.
  *   - Limits: 1 <= k <= min(E, 8); 1 <= E <= 256; d_model and d_ff multiples
- *     of 64; 1 <= T; shared expert only with bf16 weights and d_ff_shared ==
+ *     of 64; 0 <= T (0: empty batch); shared expert only with bf16 weights and d_ff_shared ==
  *     d_ff. Pointers to bf16/Q4G32 tensors 16-byte aligned.
  *   - Calls that share one workspace must not overlap on the GPU.
  */
@@ -287,6 +287,20 @@ MOE_API int moe_forward_host(const moe_params* p, const uint16_t* x_host, const 
                      moe_stream_t stream);
 
 /*
+ * moe_forward_host_async — moe_forward_host without the final synchronisation:
+ * the copies in, the layer and the copy out are enqueued on `stream` and the
+ * call returns. The caller synchronises the stream (or an event recorded on it)
+ * before it reads out_host or writes x_host / logits_host again. With pinned
+ * host buffers the copies run asynchronously, so calls on two streams with
+ * separate workspaces and buffers overlap one step's copies with another's
+ * kernels (a pipelined serving loop); pageable buffers make the copies
+ * synchronous with the host. Same arguments and errors as moe_forward_host.
+ */
+MOE_API int moe_forward_host_async(const moe_params* p, const uint16_t* x_host, const float* logits_host,
+                     const moe_weights* w, void* out_host, void* ws, size_t ws_bytes,
+                     moe_stream_t stream);
+
+/*
  * Weight preparation, done once at load time, outside the layer's calls:
  * dst[i] = fp16(src[i]) for n bf16 values (round to nearest even; exact for
  * |v| in fp16's normal range and for bf16 values down to 2^-17). Used to keep
@@ -327,7 +341,7 @@ MOE_API int moe_set_wait_limit_ns(uint64_t ns);
 #define MOE_K_TC_GATEUP      6  /* S5 tcgen05 gate/up GEMM + clamped SwiGLU */
 #define MOE_K_TC_DOWN        7  /* S6 tcgen05 down GEMM + gate scale */
 #define MOE_K_STREAM_GATEUP  8  /* S8 few-rows gate/up (weight streaming) */
-#define MOE_K_STREAM_REDUCE  9  /* unused: the S8 K-split sums now run inside stream gate/up */
+#define MOE_K_STREAM_REDUCE  9  /* S8 K-split partial sums + SwiGLU */
 #define MOE_K_STREAM_DOWN   10  /* S8 few-rows down */
 #define MOE_K_COMBINE       11  /* S7 gate-weighted combine */
 #define MOE_K_CONVERT       12  /* load-time bf16 -> fp16 weight copy (not a layer step) */

@@ -33,7 +33,7 @@ EXPORTS = ("moe_version", "moe_status_string", "moe_capacity", "moe_max_rows", "
            "moe_route", "moe_permute", "moe_expert_ffn", "moe_combine", "moe_forward", "moe_forward_host",
            "moe_get_error", "moe_clear_error", "moe_set_wait_limit_ns", "moe_launch_count",
            "moe_profile_enable", "moe_profile_collect", "moe_convert_bf16_to_f16",
-           "moe_permute_noalloc")
+           "moe_permute_noalloc", "moe_forward_host_async")
 NOALLOC_MAX_PAIRS = 262144  # MOE_NOALLOC_MAX_PAIRS
 
 # kernel ids (MOE_K_*), in order
@@ -81,6 +81,7 @@ def lib() -> ctypes.CDLL:
             "moe_combine": ([_P, _V, _V, _V, _V, _V, _S, _V], ctypes.c_int),
             "moe_forward": ([_P, _V, _V, ctypes.POINTER(Weights), _V, _V, _V, _S, _V], ctypes.c_int),
             "moe_forward_host": ([_P, _V, _V, ctypes.POINTER(Weights), _V, _V, _S, _V], ctypes.c_int),
+            "moe_forward_host_async": ([_P, _V, _V, ctypes.POINTER(Weights), _V, _V, _S, _V], ctypes.c_int),
             "moe_get_error": ([_V, ctypes.POINTER(ctypes.c_uint32), _V], ctypes.c_int),
             "moe_clear_error": ([_V, _V], ctypes.c_int),
             "moe_set_wait_limit_ns": ([ctypes.c_uint64], ctypes.c_int),
@@ -200,6 +201,12 @@ def forward_host(p, x_host, logits_host, W: Weights, out_host, ws, stream=None):
     """moe_forward_host: host (CPU, ideally pinned) x/logits/out; synchronises the stream."""
     check(lib().moe_forward_host(ctypes.byref(p), _p(x_host), _p(logits_host), ctypes.byref(W), _p(out_host),
                                  _p(ws), ws.numel(), _stream(stream)), "moe_forward_host")
+
+
+def forward_host_async(p, x_host, logits_host, W: Weights, out_host, ws, stream=None):
+    """moe_forward_host_async: as forward_host, enqueued on the stream without synchronising."""
+    check(lib().moe_forward_host_async(ctypes.byref(p), _p(x_host), _p(logits_host), ctypes.byref(W),
+                                       _p(out_host), _p(ws), ws.numel(), _stream(stream)), "moe_forward_host_async")
 
 
 def get_error(ws, stream=None) -> int:

@@ -10,7 +10,7 @@
 namespace moe {
 
 cudaError_t launch_schedule(const Dims& D, const int32_t* offsets, int32_t* tile_base, int32_t* stream_list,
-                            int32_t* n_stream, int32_t* fix, int n_fix, uint32_t* err, cudaStream_t s);
+                            int32_t* n_stream, uint32_t* err, cudaStream_t s);
 cudaError_t launch_gather(const Dims& D, const uint16_t* x, const int32_t* sorted_token, const int32_t* offsets,
                           uint16_t* xg, uint32_t* err, cudaStream_t s);
 cudaError_t launch_tensor_ffn(const Dims& D, const uint16_t* xg, uint16_t* h, const int32_t* tile_base,
@@ -19,8 +19,7 @@ cudaError_t launch_tensor_ffn(const Dims& D, const uint16_t* xg, uint16_t* h, co
                               uint16_t* y_rows, int32_t* counters, uint32_t* err, uint64_t wait_ns,
                               cudaStream_t s);
 cudaError_t launch_convert_bf16_f16(const uint16_t* src, uint16_t* dst, int64_t n, uint32_t* err, cudaStream_t s);
-cudaError_t launch_stream_ffn(const Dims& D, const uint16_t* xg, uint16_t* h, float* part, int32_t* fix,
-                              const int32_t* offsets,
+cudaError_t launch_stream_ffn(const Dims& D, const uint16_t* xg, uint16_t* h, float* part, const int32_t* offsets,
                               const int32_t* stream_list, const int32_t* n_stream, const int32_t* sorted_pair,
                               const float* topk_w, const moe_weights* w, uint16_t* y_rows, uint32_t* err,
                               uint64_t wait_ns, cudaStream_t s);
@@ -112,10 +111,6 @@ static int make_dims(const moe_params* p, Dims* D) {
     return MOE_OK;
 }
 
-// K-split arrival counters of the streaming gate/up: one per (streaming list
-// entry, 64-column slice of d_ff, consumer warp).
-static int fix_count(const Dims& D) { return D.Etot * (D.f / 64) * 4; }
-
 WsLayout ws_layout(const Dims& D, int which) {
     WsLayout L;
     std::memset(&L, 0, sizeof(L));
@@ -138,10 +133,7 @@ WsLayout ws_layout(const Dims& D, int which) {
         L.n_stream = take(16);  // [0] streaming experts, [1], [2] tile-unit counters
         L.xg = take(size_t(D.rows) * D.d * 2);
         L.h = take(size_t(D.rows) * D.f * 2);
-        if (D.ks > 1) {
-            L.part = take(size_t(D.ks) * 2 * D.rows * D.f * 4);
-            L.fix = take(size_t(fix_count(D)) * 4);
-        }
+        if (D.ks > 1) L.part = take(size_t(D.ks) * 2 * D.rows * D.f * 4);
     }
     if (fwd) {
         L.topk_idx = take(size_t(D.pairs) * 4);
@@ -181,9 +173,7 @@ cudaError_t launch_expert_ffn(const Dims& D, const WsLayout& L, const FfnArgs& a
     uint16_t* xg = reinterpret_cast<uint16_t*>(ws + L.xg);
     uint16_t* h = reinterpret_cast<uint16_t*>(ws + L.h);
     float* part = L.part ? reinterpret_cast<float*>(ws + L.part) : nullptr;
-    int32_t* fix = L.fix ? reinterpret_cast<int32_t*>(ws + L.fix) : nullptr;
-    cudaError_t e = launch_schedule(D, a.offsets, tile_base, stream_list, n_stream, fix, fix ? fix_count(D) : 0,
-                                    a.err, s);
+    cudaError_t e = launch_schedule(D, a.offsets, tile_base, stream_list, n_stream, a.err, s);
     if (e != cudaSuccess) return e;
     // Rows in expert order for both variants (fp16 for Q4G32, whose MMAs run
     // in fp16). A TMA tile::gather4 of the rows inside the GEMM was measured
@@ -195,7 +185,7 @@ cudaError_t launch_expert_ffn(const Dims& D, const WsLayout& L, const FfnArgs& a
             return e;
     }
     if (D.variant != MOE_VARIANT_TENSOR && D.stream_max_rows > 0) {
-        if ((e = launch_stream_ffn(D, xg, h, part, fix, a.offsets, stream_list, n_stream, a.sorted_pair, a.topk_w, a.w,
+        if ((e = launch_stream_ffn(D, xg, h, part, a.offsets, stream_list, n_stream, a.sorted_pair, a.topk_w, a.w,
                                    a.y_rows, a.err, a.wait_ns, s)) != cudaSuccess)
             return e;
     }
@@ -374,8 +364,9 @@ int moe_forward(const moe_params* p, const uint16_t* x, const float* logits, con
                         stream);
 }
 
-int moe_forward_host(const moe_params* p, const uint16_t* x_host, const float* logits_host, const moe_weights* w,
-                     void* out_host, void* ws, size_t ws_bytes, moe_stream_t stream) {
+static int forward_host_impl(const moe_params* p, const uint16_t* x_host, const float* logits_host,
+                             const moe_weights* w, void* out_host, void* ws, size_t ws_bytes, moe_stream_t stream,
+                             bool sync) {
     Dims D;
     int st = make_dims(p, &D);
     if (st != MOE_OK) return st;
@@ -396,7 +387,18 @@ int moe_forward_host(const moe_params* p, const uint16_t* x_host, const float* l
     if (cudaMemcpyAsync(out_host, od, size_t(D.T) * D.d * (D.out_bf16 ? 2 : 4), cudaMemcpyDeviceToHost, stream) !=
         cudaSuccess)
         return MOE_ERR_CUDA;
+    if (!sync) return MOE_OK;
     return cudaStreamSynchronize(stream) == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+}
+
+int moe_forward_host(const moe_params* p, const uint16_t* x_host, const float* logits_host, const moe_weights* w,
+                     void* out_host, void* ws, size_t ws_bytes, moe_stream_t stream) {
+    return forward_host_impl(p, x_host, logits_host, w, out_host, ws, ws_bytes, stream, true);
+}
+
+int moe_forward_host_async(const moe_params* p, const uint16_t* x_host, const float* logits_host,
+                           const moe_weights* w, void* out_host, void* ws, size_t ws_bytes, moe_stream_t stream) {
+    return forward_host_impl(p, x_host, logits_host, w, out_host, ws, ws_bytes, stream, false);
 }
 
 int moe_get_error(const void* ws, uint32_t* err, moe_stream_t stream) {
@@ -425,7 +427,7 @@ int moe_launch_count(const moe_params* p, int which, int* n) {
     int ffn = 1;  // schedule
     ffn += 1;                                       // gather
     if (tiles_needed(D)) ffn += 2;                  // two tcgen05 GEMMs
-    if (D.variant != MOE_VARIANT_TENSOR && D.stream_max_rows > 0) ffn += 2;
+    if (D.variant != MOE_VARIANT_TENSOR && D.stream_max_rows > 0) ffn += 2 + (D.ks > 1 ? 1 : 0);
     switch (which) {
         case MOE_WS_ROUTE: *n = 1; break;
         case MOE_WS_PERMUTE: *n = 3; break;

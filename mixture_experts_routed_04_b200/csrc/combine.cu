@@ -70,11 +70,12 @@ cudaError_t launch_combine(const Dims& D, const uint16_t* y_rows, const int32_t*
     if (blocks < 1) blocks = 1;
     {
         ProfScope prof_(MOE_K_COMBINE, s);
+        const bool pdl = use_pdl(D.T);
         const cudaError_t le =
-            D.out_bf16 ? launch_pdl(combine_kernel<true>, dim3(int(blocks)), dim3(threads), 0, s, y_rows, pair_row,
-                                    offsets, D.T, D.d, D.k, D.E, D.has_shared, out)
-                       : launch_pdl(combine_kernel<false>, dim3(int(blocks)), dim3(threads), 0, s, y_rows, pair_row,
-                                    offsets, D.T, D.d, D.k, D.E, D.has_shared, out);
+            D.out_bf16 ? launch_pdl(pdl, combine_kernel<true>, dim3(int(blocks)), dim3(threads), 0, s, y_rows,
+                                    pair_row, offsets, D.T, D.d, D.k, D.E, D.has_shared, out)
+                       : launch_pdl(pdl, combine_kernel<false>, dim3(int(blocks)), dim3(threads), 0, s, y_rows,
+                                    pair_row, offsets, D.T, D.d, D.k, D.E, D.has_shared, out);
         if (le != cudaSuccess) return le;
     }
     return cudaGetLastError();
@@ -123,8 +124,8 @@ cudaError_t launch_convert_bf16_f16(const uint16_t* src, uint16_t* dst, int64_t 
     if (blocks < 1) blocks = 1;
     {
         ProfScope prof_(MOE_K_CONVERT, s);
-        const cudaError_t le = launch_pdl(convert_bf16_f16_kernel, dim3(int(blocks)), dim3(256), 0, s, src, dst,
-                                          n, err);
+        const cudaError_t le = launch_pdl(false, convert_bf16_f16_kernel, dim3(int(blocks)), dim3(256), 0, s, src,
+                                          dst, n, err);
         if (le != cudaSuccess) return le;
     }
     return cudaGetLastError();

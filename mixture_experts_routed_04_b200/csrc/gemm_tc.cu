@@ -346,16 +346,13 @@ __global__ void __launch_bounds__(Cfg<MODE, WF, SUB>::kThreads, 1)
                     } else if (MODE == 0) {
                         const CUtensorMap* mg = sh ? &tmS0 : &tmB0;
                         const CUtensorMap* mu = sh ? &tmS1 : &tmB1;
-                        const int n0 = U.n * 128;
-                        tma_load_3d(sb, mg, full + stage, n0, kb * BK, z);
-                        tma_load_3d(sb + B_CHUNK, mg, full + stage, n0 + 64, kb * BK, z);
-                        tma_load_3d(sb + 2 * B_CHUNK, mu, full + stage, n0, kb * BK, z);
-                        tma_load_3d(sb + 3 * B_CHUNK, mu, full + stage, n0 + 64, kb * BK, z);
+                        // two 64-column chunks of gate, then two of up: one copy each
+                        tma_load_4d(sb, mg, full + stage, 0, kb * BK, 2 * U.n, z);
+                        tma_load_4d(sb + 2 * B_CHUNK, mu, full + stage, 0, kb * BK, 2 * U.n, z);
                     } else {
                         const CUtensorMap* md = sh ? &tmS0 : &tmB0;
-                        const int n0 = U.n * BN;
-#pragma unroll
-                        for (int c = 0; c < 4; ++c) tma_load_3d(sb + c * B_CHUNK, md, full + stage, n0 + 64 * c, kb * BK, z);
+                        // four 64-column chunks in one copy
+                        tma_load_4d(sb, md, full + stage, 0, kb * BK, 4 * U.n, z);
                     }
                     issued |= 1u << stage;
                     issued_par = (issued_par & ~(1u << stage)) | (phase << stage);
@@ -560,25 +557,25 @@ __global__ void __launch_bounds__(Cfg<MODE, WF, SUB>::kThreads, 1)
                 }
                 uint8_t* sb = smem + stage * SB + C::kABytes;
                 if (Q4) {
-                    // rows ct and ct+128 of the 256-row B tile; row r: 8 words
-                    // (k 0..63) -> 8 chunks of 8 fp16 at r*128 + ((c ^ (r%8)) * 16)
+                    // 512 (row, half) pairs of the 256-row B tile, four per thread;
+                    // half hf of row r is words 4hf..4hf+3 (k 32hf..32hf+31, scale
+                    // group hf) -> chunks 4hf+c of 8 fp16 at r*128 + (((4hf+c) ^ (r%8)) * 16).
+                    // Consecutive lanes read consecutive 16-byte words (no bank conflicts).
                     const uint8_t* sp = sb + B_BYTES;
                     const uint16_t* ss = reinterpret_cast<const uint16_t*>(sp + P_BYTES);
 #pragma unroll
-                    for (int h = 0; h < 2; ++h) {
-                        const int r = ct + 128 * h;
+                    for (int it = 0; it < 4; ++it) {
+                        const int q = ct + 128 * it;
+                        const int r = q >> 1, hf = q & 1;
                         // scales [2 groups][rows]: MODE 0 holds gate rows then up rows (128 each)
-                        const uint16_t* sr = MODE == 0 ? ss + h * 256 + (r & 127) : ss + r;
-                        const int gstride = MODE == 0 ? 128 : 256;
-                        const uint32_t s0 = sr[0], s1 = sr[gstride];
-                        const uint32_t s0x2 = s0 | (s0 << 16), s1x2 = s1 | (s1 << 16);
-                        const uint4 w0 = reinterpret_cast<const uint4*>(sp + r * 32)[0];
-                        const uint4 w1 = reinterpret_cast<const uint4*>(sp + r * 32)[1];
-                        const uint32_t words[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
+                        const uint32_t sc = MODE == 0 ? ss[(r >> 7) * 256 + hf * 128 + (r & 127)] : ss[hf * 256 + r];
+                        const uint32_t s2 = sc | (sc << 16);
+                        const uint4 w = reinterpret_cast<const uint4*>(sp + r * 32)[hf];
+                        const uint32_t words[4] = {w.x, w.y, w.z, w.w};
                         uint8_t* row = sb + r * 128;
 #pragma unroll
-                        for (int c = 0; c < 8; ++c)
-                            *reinterpret_cast<uint4*>(row + ((c ^ (r & 7)) << 4)) = dequant_word(words[c], c < 4 ? s0x2 : s1x2);
+                        for (int c = 0; c < 4; ++c)
+                            *reinterpret_cast<uint4*>(row + (((4 * hf + c) ^ (r & 7)) << 4)) = dequant_word(words[c], s2);
                     }
                 } else {
                     // bf16 -> fp16 in place (position-independent)
@@ -620,14 +617,12 @@ __global__ void __launch_bounds__(512) schedule_kernel(const int32_t* __restrict
                                                        int stream_max,
                                                        int32_t* __restrict__ tile_base,
                                                        int32_t* __restrict__ stream_list,
-                                                       int32_t* __restrict__ n_stream, int32_t* __restrict__ fix,
-                                                       int n_fix, uint32_t* err) {
+                                                       int32_t* __restrict__ n_stream, uint32_t* err) {
     __shared__ int sums[3][16];
     griddep_wait();
     griddep_launch();
 
     const int e = threadIdx.x, lane = e & 31, w = e >> 5;
-    for (int i = e; i < n_fix; i += blockDim.x) fix[i] = 0;  // K-split arrivals of the streaming gate/up
     int kept = 0;
     if (e < Etot) {
         kept = offsets[e + 1] - offsets[e];
@@ -741,8 +736,9 @@ static bool make_map(CUtensorMap* m, CUtensorMapDataType dt, const void* base, i
                      const uint64_t* strides_bytes, const uint32_t* box, CUtensorMapSwizzle swz) {
     EncodeTiledFn enc = get_encode();
     if (!enc) return false;
-    cuuint64_t gd[3], gs[2];
-    cuuint32_t bx[3], es[3] = {1, 1, 1};
+    if (rank < 1 || rank > 5) return false;
+    cuuint64_t gd[5], gs[4];
+    cuuint32_t bx[5], es[5] = {1, 1, 1, 1, 1};
     for (int i = 0; i < rank; ++i) {
         gd[i] = dims[i];
         bx[i] = box[i];
@@ -760,12 +756,14 @@ bool map_rows(CUtensorMap* m, const void* base, int64_t rows, int K) {
     const uint32_t box[2] = {64, 128};
     return make_map(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, base, 2, dims, str, box, CU_TENSOR_MAP_SWIZZLE_128B);
 }
-// bf16 B operand: [nexp, K, N] row-major; box 64 (N) x 64 (K) x 1, 128-byte swizzle.
-bool map_weights(CUtensorMap* m, const void* base, int nexp, int K, int N) {
-    const uint64_t dims[3] = {uint64_t(N), uint64_t(K), uint64_t(nexp)};
-    const uint64_t str[2] = {uint64_t(N) * 2, uint64_t(N) * uint64_t(K) * 2};
-    const uint32_t box[3] = {64, 64, 1};
-    return make_map(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, base, 3, dims, str, box, CU_TENSOR_MAP_SWIZZLE_128B);
+// bf16 B operand: [nexp, K, N] row-major, seen as [nexp, N/64 chunks, K, 64] so that one
+// copy brings `chunks` 64-column boxes of 64 K-rows (128-byte swizzle), stored chunk after
+// chunk (8 KB apart) — fewer copies for the single producer thread to issue.
+bool map_weights(CUtensorMap* m, const void* base, int nexp, int K, int N, int chunks) {
+    const uint64_t dims[4] = {64, uint64_t(K), uint64_t(N / 64), uint64_t(nexp)};
+    const uint64_t str[3] = {uint64_t(N) * 2, 128, uint64_t(N) * uint64_t(K) * 2};
+    const uint32_t box[4] = {64, 64, uint32_t(chunks), 1};
+    return make_map(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, base, 4, dims, str, box, CU_TENSOR_MAP_SWIZZLE_128B);
 }
 // Q4G32 nibbles: [nexp, N, K/2] bytes; box 32 bytes (64 k) x rows x 1, no swizzle.
 bool map_q4_packed(CUtensorMap* m, const void* base, int nexp, int K, int N, int rows) {
@@ -784,7 +782,7 @@ bool map_q4_scales(CUtensorMap* m, const void* base, int nexp, int K, int N, int
 
 template <int MODE, int WF, int SUB>
 cudaError_t launch_gemm(const CUtensorMap& A, const CUtensorMap& B0, const CUtensorMap& B1, const CUtensorMap& S0,
-                        const CUtensorMap& S1, const GemmParams& p, cudaStream_t s) {
+                        const CUtensorMap& S1, const GemmParams& p, bool pdl, cudaStream_t s) {
     using C = Cfg<MODE, WF, SUB>;
     static int configured_dev = -1;
     int dev = 0;
@@ -799,7 +797,7 @@ cudaError_t launch_gemm(const CUtensorMap& A, const CUtensorMap& B0, const CUten
     if (C::kSub == 2) q.tile_base = p.tile_base + p.Etot + 1;  // 256-row units
     {
         ProfScope prof_(MODE == 0 ? MOE_K_TC_GATEUP : MOE_K_TC_DOWN, s);
-        const cudaError_t le = launch_pdl(grouped_gemm_kernel<MODE, WF, SUB>, dim3(num_sms()), dim3(C::kThreads),
+        const cudaError_t le = launch_pdl(pdl, grouped_gemm_kernel<MODE, WF, SUB>, dim3(num_sms()), dim3(C::kThreads),
                                           C::kSmem, s, A, B0, B1, S0, S1, q);
         if (le != cudaSuccess) return le;
     }
@@ -809,12 +807,12 @@ cudaError_t launch_gemm(const CUtensorMap& A, const CUtensorMap& B0, const CUten
 }  // namespace tc
 
 cudaError_t launch_schedule(const Dims& D, const int32_t* offsets, int32_t* tile_base, int32_t* stream_list,
-                            int32_t* n_stream, int32_t* fix, int n_fix, uint32_t* err, cudaStream_t s) {
+                            int32_t* n_stream, uint32_t* err, cudaStream_t s) {
     int smax = D.stream_max_rows;
     {
         ProfScope prof_(MOE_K_SCHEDULE, s);
-        const cudaError_t le = launch_pdl(schedule_kernel, dim3(1), dim3(512), 0, s, offsets, D.Etot, D.variant,
-                                          smax, tile_base, stream_list, n_stream, fix, n_fix, err);
+        const cudaError_t le = launch_pdl(use_pdl(D.T), schedule_kernel, dim3(1), dim3(512), 0, s, offsets, D.Etot,
+                                          D.variant, smax, tile_base, stream_list, n_stream, err);
         if (le != cudaSuccess) return le;
     }
     return cudaGetLastError();
@@ -829,12 +827,13 @@ cudaError_t launch_gather(const Dims& D, const uint16_t* x, const int32_t* sorte
     if (blocks < 1) blocks = 1;
     {
         ProfScope prof_(MOE_K_GATHER, s);
+        const bool pdl = use_pdl(D.T);
         const cudaError_t le =
             D.fmt == MOE_WEIGHTS_Q4G32
-                ? launch_pdl(gather_rows_kernel<true>, dim3(int(blocks)), dim3(256), 0, s, x, sorted_token, offsets,
-                             D.Etot, D.d, D.T, xg, err)
-                : launch_pdl(gather_rows_kernel<false>, dim3(int(blocks)), dim3(256), 0, s, x, sorted_token, offsets,
-                             D.Etot, D.d, D.T, xg, err);
+                ? launch_pdl(pdl, gather_rows_kernel<true>, dim3(int(blocks)), dim3(256), 0, s, x, sorted_token,
+                             offsets, D.Etot, D.d, D.T, xg, err)
+                : launch_pdl(pdl, gather_rows_kernel<false>, dim3(int(blocks)), dim3(256), 0, s, x, sorted_token,
+                             offsets, D.Etot, D.d, D.T, xg, err);
         if (le != cudaSuccess) return le;
     }
     return cudaGetLastError();
@@ -848,6 +847,7 @@ cudaError_t launch_tensor_ffn(const Dims& D, const uint16_t* xg, uint16_t* h, co
                               uint16_t* y_rows, int32_t* counters, uint32_t* err, uint64_t wait_ns,
                               cudaStream_t s) {
     using namespace tc;
+    const bool pdl = use_pdl(D.T);
     GemmParams p{};
     p.E = D.E;
     p.Etot = D.Etot;
@@ -872,21 +872,21 @@ cudaError_t launch_tensor_ffn(const Dims& D, const uint16_t* xg, uint16_t* h, co
         p.n_tiles = (D.f + 127) / 128;
         p.out = h;
         p.unit_counter = counters;
-        if ((e = launch_gemm<0, 1, 2>(mA, pg, pu, sg, su, p, s)) != cudaSuccess) return e;
+        if ((e = launch_gemm<0, 1, 2>(mA, pg, pu, sg, su, p, pdl, s)) != cudaSuccess) return e;
         p.K = D.f;
         p.n_out = D.d;
         p.n_tiles = (D.d + BN - 1) / BN;
         p.out = y_rows;
         p.unit_counter = counters + 1;
-        return launch_gemm<1, 1, 2>(mH, pd, pd, sd, sd, p, s);
+        return launch_gemm<1, 1, 2>(mH, pd, pd, sd, sd, p, pdl, s);
     }
     CUtensorMap mG, mU, mSG, mSU, mD, mSD;
-    if (!map_weights(&mG, w->w_gate, D.E, D.d, D.f) || !map_weights(&mU, w->w_up, D.E, D.d, D.f) ||
-        !map_weights(&mD, w->w_down, D.E, D.f, D.d))
+    if (!map_weights(&mG, w->w_gate, D.E, D.d, D.f, 2) || !map_weights(&mU, w->w_up, D.E, D.d, D.f, 2) ||
+        !map_weights(&mD, w->w_down, D.E, D.f, D.d, 4))
         return cudaErrorInvalidValue;
     if (D.has_shared) {
-        if (!map_weights(&mSG, w->shared_gate, 1, D.d, D.f) || !map_weights(&mSU, w->shared_up, 1, D.d, D.f) ||
-            !map_weights(&mSD, w->shared_down, 1, D.f, D.d))
+        if (!map_weights(&mSG, w->shared_gate, 1, D.d, D.f, 2) || !map_weights(&mSU, w->shared_up, 1, D.d, D.f, 2) ||
+            !map_weights(&mSD, w->shared_down, 1, D.f, D.d, 4))
             return cudaErrorInvalidValue;
     } else {
         mSG = mG;
@@ -899,14 +899,15 @@ cudaError_t launch_tensor_ffn(const Dims& D, const uint16_t* xg, uint16_t* h, co
     p.n_tiles = (D.f + 127) / 128;
     p.out = h;
     p.unit_counter = counters;
-    if ((e = launch_gemm<0, 0, 1>(mA, mG, mU, mSG, mSU, p, s)) != cudaSuccess) return e;
+    if ((e = launch_gemm<0, 0, 1>(mA, mG, mU, mSG, mSU, p, pdl, s)) != cudaSuccess) return e;
     // S6: down + gate scale -> y_rows
     p.K = D.f;
     p.n_out = D.d;
     p.n_tiles = (D.d + BN - 1) / BN;
     p.out = y_rows;
     p.unit_counter = counters + 1;
-    return D.down_f16 ? launch_gemm<1, 2, 1>(mH, mD, mD, mSD, mSD, p, s) : launch_gemm<1, 0, 1>(mH, mD, mD, mSD, mSD, p, s);
+    return D.down_f16 ? launch_gemm<1, 2, 1>(mH, mD, mD, mSD, mSD, p, pdl, s)
+                      : launch_gemm<1, 0, 1>(mH, mD, mD, mSD, mSD, p, pdl, s);
 }
 
 }  // namespace moe

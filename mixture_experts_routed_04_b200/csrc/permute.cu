@@ -198,21 +198,21 @@ cudaError_t launch_permute(const Dims& D, const int32_t* topk_idx, int32_t* bloc
     const int shared_T = D.has_shared ? D.T : 0;
     {
         ProfScope prof_(MOE_K_PERM_COUNT, s);
-        const cudaError_t le = launch_pdl(perm_count_kernel, dim3(nb), dim3(kPermWarps * 32), 0, s, topk_idx,
-                                          D.pairs, D.E, blockcounts, err);
+        const cudaError_t le = launch_pdl(use_pdl(D.T), perm_count_kernel, dim3(nb), dim3(kPermWarps * 32), 0, s,
+                                          topk_idx, D.pairs, D.E, blockcounts, err);
         if (le != cudaSuccess) return le;
     }
     {
         ProfScope prof_(MOE_K_PERM_SCAN, s);
-        const cudaError_t le = launch_pdl(perm_scan_kernel, dim3(1), dim3(kMaxE), 0, s, blockcounts, nb, D.E,
-                                          D.cap, shared_T, blockbase, counts, kept, offsets);
+        const cudaError_t le = launch_pdl(use_pdl(D.T), perm_scan_kernel, dim3(1), dim3(kMaxE), 0, s, blockcounts, nb,
+                                          D.E, D.cap, shared_T, blockbase, counts, kept, offsets);
         if (le != cudaSuccess) return le;
     }
     {
         ProfScope prof_(MOE_K_PERM_SCATTER, s);
-        const cudaError_t le = launch_pdl(perm_scatter_kernel, dim3(nb), dim3(kPermWarps * 32), 0, s, topk_idx,
-                                          D.pairs, D.k, D.E, D.cap, blockbase, offsets, sorted_token, sorted_pair,
-                                          pair_row, shared_T, err);
+        const cudaError_t le = launch_pdl(use_pdl(D.T), perm_scatter_kernel, dim3(nb), dim3(kPermWarps * 32), 0, s,
+                                          topk_idx, D.pairs, D.k, D.E, D.cap, blockbase, offsets, sorted_token,
+                                          sorted_pair, pair_row, shared_T, err);
         if (le != cudaSuccess) return le;
     }
     return cudaGetLastError();

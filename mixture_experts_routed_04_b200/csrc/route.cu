@@ -90,8 +90,8 @@ cudaError_t launch_route(const float* logits, int T, int E, int k, int32_t* topk
     const int blocks = (T + wpb - 1) / wpb;
     {
         ProfScope prof_(MOE_K_ROUTE, stream);
-        const cudaError_t le = launch_pdl(route_topk_softmax_kernel, dim3(blocks), dim3(threads), 0, stream,
-                                          logits, T, E, k, topk_idx, topk_w);
+        const cudaError_t le = launch_pdl(use_pdl(T), route_topk_softmax_kernel, dim3(blocks), dim3(threads), 0,
+                                          stream, logits, T, E, k, topk_idx, topk_w);
         if (le != cudaSuccess) return le;
     }
     return cudaGetLastError();

@@ -8,21 +8,21 @@
 // "Strata PR #4366" — the light kernels own experts with at most 16 rows;
 // "TensorFold PR #1607" — K-parallel tiles for plans with few pairs per item.
 //
-// Work item = (expert, 64 output columns, K slice, chunk of <= 8 rows). One
-// CTA per SM, persistent, everything through one TMA ring (128 KB):
-//   warp 0     TMA producer: per 64-K block, the 64 x 64 weight tile(s) (gate
-//              and up, or down; 128-byte swizzle) and the 8 x 64 tile of the
-//              chunk's rows (gathered x, or h; 128-byte swizzle).
-//   warps 1-4  consumers, 16 columns each: ldmatrix.trans turns the stored
-//              [k][n] weight tile into the A operand (16 n x 16 k) of mma.sync
-//              m16n8k16; the rows tile gives the N=8 operand. fp32 accumulate.
-//              The tensor pipe only keeps the instruction count per weight byte
-//              low so the kernel stays HBM-bound.
+// Work item = (expert, output columns, K slice, chunk of <= 8 rows): 64
+// columns of W_gate and of W_up, or 256 columns of W_down. One CTA per SM,
+// persistent, everything through one TMA ring (119 KB gate/up, 198 KB down):
+//   warp 0     TMA producer: per 64-K block, the 64 x 64 weight boxes (gate
+//              and up, or four of down; 128-byte swizzle) and the 8 x 64 tile
+//              of the chunk's rows (gathered x, or h; 128-byte swizzle).
+//   warps 1-4  consumers, 16 columns of gate and up each, or 64 columns of
+//              down: ldmatrix.trans turns the stored [k][n] weight box into the
+//              A operand (16 n x 16 k) of mma.sync m16n8k16; the rows tile
+//              gives the N=8 operand. fp32 accumulate. The tensor pipe only
+//              keeps the instruction count per weight byte low so the kernel
+//              stays HBM-bound.
 // Gate/up (bf16 x and weights) with one K slice applies the clamped SwiGLU and
-// writes h (fp16); with several, fp32 partials go to the workspace and the
-// warp that completes the last slice of a 16-column strip sums them in slice
-// order and applies the SwiGLU (deterministic: the order never depends on
-// which CTA finishes last). Down runs in fp16 (h is
+// writes h (fp16); with several, fp32 partials go to the workspace and
+// stream_reduce finishes (fixed order, deterministic). Down runs in fp16 (h is
 // fp16; W_down prepared as fp16, or converted in registers after ldmatrix) and
 // writes y = w_pair * (h W_down) (fp16). All waits are bounded; no TMA
 // multicast; no named barriers, so an abort never strands a warp.
@@ -32,15 +32,27 @@ namespace moe {
 
 namespace st {
 
-constexpr int NS = 64;               // output columns per work item
+constexpr int NS = 64;               // columns of one weight box (128 bytes of a row)
 constexpr int BKS = 64;              // K-rows per stage
-constexpr int TILE = BKS * NS * 2;   // weight tile, 8 KB
+constexpr int TILE = BKS * NS * 2;   // weight box, 8 KB
 constexpr int XT = 8 * BKS * 2;      // rows tile (8 rows x 64 K), 1 KB
-constexpr int RING = 128 * 1024;
 constexpr int CONSUMERS = 4;
 constexpr int THREADS = 32 * (CONSUMERS + 1);
 constexpr int RC = 8;                // rows per chunk (mma N)
-constexpr int SMEM_BYTES = 1024 + RING + 512;
+
+// Per matrix: gate/up items are 64 columns of W_gate and of W_up (two boxes a
+// stage, 16 columns of each per consumer warp); down items are 256 columns of
+// W_down (four boxes a stage, 64 columns per warp), so each weight row is read
+// as 512 contiguous bytes — 64-column down items left HBM half idle.
+template <int MODE>
+struct SCfg {
+    static constexpr int NMAT = MODE == 0 ? 2 : 4;                // weight boxes per stage
+    static constexpr int NSU = MODE == 0 ? NS : 4 * NS;           // output columns per item
+    static constexpr int STAGE = NMAT * TILE + XT;                // 17 KB / 33 KB, 1 KB aligned
+    static constexpr int STAGES = MODE == 0 ? 7 : 6;
+    static constexpr int RING = STAGES * STAGE;                   // 119 KB / 198 KB
+    static constexpr int SMEM = 1024 + RING + 512;
+};
 
 struct StreamParams {
     int mode;            // 0: gate/up, 1: down
@@ -54,8 +66,6 @@ struct StreamParams {
     const float* topk_w;
     uint16_t* out;        // mode 0: h [rows, f]; mode 1: y_rows [rows, d]
     float* part;          // mode 0 with ks > 1: [ks, 2, rows, f] fp32
-    int32_t* fix;         // mode 0 with ks > 1: arrivals per (list entry, 64-column slice, warp), zeroed
-                          // by the schedule kernel
     int64_t rows;
     float limit;
     int down_f16;         // mode 1: W_down already fp16 (no conversion)
@@ -64,18 +74,17 @@ struct StreamParams {
 };
 
 struct SUnit {
-    int i, e, n0, k0, ks, row0, nrows;  // i: position in the streaming list
+    int e, n0, k0, ks, row0, nrows;
 };
 
-MOE_DEV SUnit decode(int u, const StreamParams& p) {
-    const int nsl = p.N / NS;
+MOE_DEV SUnit decode(int u, const StreamParams& p, int nsu) {
+    const int nsl = (p.N + nsu - 1) / nsu;
     const int per = nsl * p.ks;
     const int i = u / per;
     const int rem = u - i * per;
     SUnit U;
-    U.i = i;
     U.e = __ldg(p.stream_list + i);
-    U.n0 = (rem / p.ks) * NS;
+    U.n0 = (rem / p.ks) * nsu;
     U.ks = rem % p.ks;
     U.k0 = U.ks * p.kslice;
     U.row0 = __ldg(p.offsets + U.e);
@@ -88,7 +97,7 @@ MOE_DEV float swiglu(float g, float u, float L) {
         g = fminf(fmaxf(g, -L), L);
         u = fminf(fmaxf(u, -L), L);
     }
-    return g / (1.0f + expf(-g)) * u;
+    return __fdividef(g, 1.0f + __expf(-g)) * u;  // as in the tile kernels
 }
 
 MOE_DEV void ldmatrix_x4_trans(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2, uint32_t& r3) {
@@ -123,12 +132,11 @@ __global__ void __launch_bounds__(THREADS, 1)
     stream_kernel(const __grid_constant__ CUtensorMap tmW0, const __grid_constant__ CUtensorMap tmW1,
                   const __grid_constant__ CUtensorMap tmS0, const __grid_constant__ CUtensorMap tmS1,
                   const __grid_constant__ CUtensorMap tmX, const StreamParams p) {
-    constexpr int NMAT = MODE == 0 ? 2 : 1;
-    constexpr int STAGE = NMAT * TILE + XT;  // 17 KB / 9 KB, 1 KB aligned
-    constexpr int STAGES = RING / STAGE;
+    using SC = SCfg<MODE>;
+    constexpr int NMAT = SC::NMAT, NSU = SC::NSU, STAGE = SC::STAGE, STAGES = SC::STAGES;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    uint64_t* full = reinterpret_cast<uint64_t*>(smem + RING);
+    uint64_t* full = reinterpret_cast<uint64_t*>(smem + SC::RING);
     uint64_t* empty = full + STAGES;
     volatile int* abort_flag = reinterpret_cast<volatile int*>(empty + STAGES);
 
@@ -146,7 +154,7 @@ __global__ void __launch_bounds__(THREADS, 1)
     griddep_wait();
     griddep_launch();
 
-    const int total = __ldg(p.n_stream) * (p.N / NS) * p.ks;
+    const int total = __ldg(p.n_stream) * ((p.N + NSU - 1) / NSU) * p.ks;
     const int KB = p.kslice / BKS;
 
     if (warp == 0) {
@@ -155,7 +163,7 @@ __global__ void __launch_bounds__(THREADS, 1)
         uint32_t phase = 0, issued = 0, issued_par = 0;
         bool ok = true;
         for (int u = blockIdx.x; ok && u < total; u += gridDim.x) {
-            const SUnit U = decode(u, p);
+            const SUnit U = decode(u, p, NSU);
             const bool sh = U.e >= p.E;
             const int wrow = (sh ? 0 : U.e * p.K) + U.k0;  // weight row of k0 in the stacked [E*K, N] view
             const int nchunks = (U.nrows + RC - 1) / RC;
@@ -171,8 +179,13 @@ __global__ void __launch_bounds__(THREADS, 1)
                     if (lane == 0) {
                         uint8_t* dst = smem + stage * STAGE;
                         mbar_arrive_expect_tx(full + stage, STAGE);
-                        tma_load_2d(dst, sh ? &tmS0 : &tmW0, full + stage, U.n0, wrow + kb * BKS);
-                        if (MODE == 0) tma_load_2d(dst + TILE, sh ? &tmS1 : &tmW1, full + stage, U.n0, wrow + kb * BKS);
+                        if (MODE == 0) {
+                            tma_load_2d(dst, sh ? &tmS0 : &tmW0, full + stage, U.n0, wrow + kb * BKS);
+                            tma_load_2d(dst + TILE, sh ? &tmS1 : &tmW1, full + stage, U.n0, wrow + kb * BKS);
+                        } else {
+                            // the four boxes in one copy (boxes past N are filled with zeros)
+                            tma_load_3d(dst, sh ? &tmS0 : &tmW0, full + stage, 0, wrow + kb * BKS, U.n0 / NS);
+                        }
                         tma_load_2d(dst + NMAT * TILE, &tmX, full + stage, U.k0 + kb * BKS, U.row0 + c * RC);
                         issued |= 1u << stage;
                         issued_par = (issued_par & ~(1u << stage)) | (phase << stage);
@@ -194,17 +207,24 @@ __global__ void __launch_bounds__(THREADS, 1)
     }
 
     // ---------------------------------------------------- consumers (warps 1..4)
-    const int cw = warp - 1;  // columns cw*16 .. cw*16+15 of the item
+    // gate/up: warp cw takes columns cw*16 .. +15 of both boxes (gate, up);
+    // down: warp cw takes box cw, i.e. columns cw*64 .. +63, as four 16-column groups.
+    constexpr int NG = MODE == 0 ? 1 : 4;  // 16-column groups per warp
+    const int cw = warp - 1;
     const int gid = lane >> 2, tig = lane & 3;
     int stage = 0;
     uint32_t phase = 0;
     bool ok = true, range_bad = false;
     for (int u = blockIdx.x; ok && u < total; u += gridDim.x) {
-        const SUnit U = decode(u, p);
+        const SUnit U = decode(u, p, NSU);
         const int nchunks = (U.nrows + RC - 1) / RC;
         for (int c = 0; ok && c < nchunks; ++c) {
             const int rc = min(RC, U.nrows - c * RC);
-            float acc0[4] = {0.f, 0.f, 0.f, 0.f}, acc1[4] = {0.f, 0.f, 0.f, 0.f};
+            float acc0[NG][4], acc1[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+            for (int g = 0; g < NG; ++g)
+#pragma unroll
+                for (int i = 0; i < 4; ++i) acc0[g][i] = 0.f;
             for (int kb = 0; kb < KB; ++kb) {
                 int okl = 1;
                 if (lane == 0) okl = mbar_wait_bounded(full + stage, phase, abort_flag, p.err, p.wait_ns);
@@ -213,35 +233,40 @@ __global__ void __launch_bounds__(THREADS, 1)
                     ok = false;
                     break;
                 }
-                const uint32_t base0 = smem_u32(smem + stage * STAGE);
+                const uint32_t base0 = smem_u32(smem + stage * STAGE) + (MODE == 0 ? 0 : cw * TILE);
                 const uint8_t* xt = smem + stage * STAGE + NMAT * TILE;  // rows tile: row r, k at swizzled spot
 #pragma unroll
                 for (int k16 = 0; k16 < BKS / 16; ++k16) {
-                    // weight tile: lane l addresses row (l%8) of 8x8 matrix (l/8): k = k16*16 + 8*(l/16) + l%8,
-                    // 16-byte chunk 2*cw + (l/8)%2, stored at chunk ^ (k % 8) (128-byte swizzle)
+                    // weight box: lane l addresses row (l%8) of 8x8 matrix (l/8): k = k16*16 + 8*(l/16) + l%8,
+                    // 16-byte chunk 2*grp + (l/8)%2 of the 128-byte row, stored at chunk ^ (k % 8) (128-byte
+                    // swizzle); grp = cw (gate/up) or the 16-column group g (down)
                     const int kr = k16 * 16 + ((lane >> 4) << 3) + (lane & 7);
-                    const int ch = (2 * cw + ((lane >> 3) & 1)) ^ (kr & 7);
-                    const uint32_t off = uint32_t(kr * 128 + ch * 16);
                     // rows tile: row gid, k = k16*16 + 2*tig (+8): chunk (k/8) ^ gid
                     const int kx = k16 * 16 + 2 * tig;
                     const uint32_t b0 =
                         *reinterpret_cast<const uint32_t*>(xt + gid * 128 + (((kx >> 3) ^ gid) << 4) + (kx & 7) * 2);
                     const uint32_t b1 = *reinterpret_cast<const uint32_t*>(
                         xt + gid * 128 + ((((kx + 8) >> 3) ^ gid) << 4) + ((kx + 8) & 7) * 2);
-                    uint32_t a0, a1, a2, a3;
-                    ldmatrix_x4_trans(base0 + off, a0, a1, a2, a3);
-                    if (MODE == 0) {
-                        // x (bf16) against W_gate / W_up (bf16)
-                        mma_bf16_16816(acc0, a0, a1, a2, a3, b0, b1);
-                        ldmatrix_x4_trans(base0 + TILE + off, a0, a1, a2, a3);
-                        mma_bf16_16816(acc1, a0, a1, a2, a3, b0, b1);
-                    } else if (p.down_f16) {
-                        // h (fp16) against W_down prepared as fp16
-                        mma_f16_16816(acc0, a0, a1, a2, a3, b0, b1);
-                    } else {
-                        // h (fp16) against W_down converted bf16 -> fp16 in registers
-                        mma_f16_16816(acc0, bf16x2_to_f16x2(a0), bf16x2_to_f16x2(a1), bf16x2_to_f16x2(a2),
-                                      bf16x2_to_f16x2(a3), b0, b1);
+#pragma unroll
+                    for (int g = 0; g < NG; ++g) {
+                        const int grp = MODE == 0 ? cw : g;
+                        const int ch = (2 * grp + ((lane >> 3) & 1)) ^ (kr & 7);
+                        const uint32_t off = uint32_t(kr * 128 + ch * 16);
+                        uint32_t a0, a1, a2, a3;
+                        ldmatrix_x4_trans(base0 + off, a0, a1, a2, a3);
+                        if (MODE == 0) {
+                            // x (bf16) against W_gate / W_up (bf16)
+                            mma_bf16_16816(acc0[g], a0, a1, a2, a3, b0, b1);
+                            ldmatrix_x4_trans(base0 + TILE + off, a0, a1, a2, a3);
+                            mma_bf16_16816(acc1, a0, a1, a2, a3, b0, b1);
+                        } else if (p.down_f16) {
+                            // h (fp16) against W_down prepared as fp16
+                            mma_f16_16816(acc0[g], a0, a1, a2, a3, b0, b1);
+                        } else {
+                            // h (fp16) against W_down converted bf16 -> fp16 in registers
+                            mma_f16_16816(acc0[g], bf16x2_to_f16x2(a0), bf16x2_to_f16x2(a1), bf16x2_to_f16x2(a2),
+                                          bf16x2_to_f16x2(a3), b0, b1);
+                        }
                     }
                 }
                 __syncwarp();
@@ -252,60 +277,65 @@ __global__ void __launch_bounds__(THREADS, 1)
                 }
             }
             if (!ok) break;
-            // acc[i]: column n = cw*16 + gid + 8*(i/2), row r = 2*tig + (i%2)
+            // acc[g][i]: column n = (cw*16 | cw*64 + 16g) + gid + 8*(i/2), row r = 2*tig + (i%2)
 #pragma unroll
-            for (int i = 0; i < 4; ++i) {
-                const int r = 2 * tig + (i & 1);
-                if (r >= rc) continue;
-                const int n = U.n0 + cw * 16 + gid + 8 * (i >> 1);
-                const int64_t row = int64_t(U.row0) + c * RC + r;
-                if (MODE == 0) {
-                    if (p.ks == 1) {
-                        const float h = swiglu(acc0[i], acc1[i], p.limit);
-                        range_bad |= !f16_range_ok(h);
-                        p.out[row * p.N + n] = to_f16(h);
+            for (int g = 0; g < NG; ++g) {
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    const int r = 2 * tig + (i & 1);
+                    const int n = U.n0 + (MODE == 0 ? cw * 16 : cw * 64 + g * 16) + gid + 8 * (i >> 1);
+                    if (r >= rc || n >= p.N) continue;
+                    const int64_t row = int64_t(U.row0) + c * RC + r;
+                    if (MODE == 0) {
+                        if (p.ks == 1) {
+                            const float h = swiglu(acc0[g][i], acc1[i], p.limit);
+                            range_bad |= !f16_range_ok(h);
+                            p.out[row * p.N + n] = to_f16(h);
+                        } else {
+                            p.part[((int64_t(U.ks) * 2 + 0) * p.rows + row) * p.N + n] = acc0[g][i];
+                            p.part[((int64_t(U.ks) * 2 + 1) * p.rows + row) * p.N + n] = acc1[i];
+                        }
                     } else {
-                        p.part[((int64_t(U.ks) * 2 + 0) * p.rows + row) * p.N + n] = acc0[i];
-                        p.part[((int64_t(U.ks) * 2 + 1) * p.rows + row) * p.N + n] = acc1[i];
+                        const int sp = __ldg(p.sorted_pair + row);
+                        const float w = sp >= 0 ? __ldg(p.topk_w + sp) : 1.0f;
+                        const float y = w * acc0[g][i];
+                        range_bad |= !f16_range_ok(y);
+                        p.out[row * p.N + n] = to_f16(y);
                     }
-                } else {
-                    const int sp = __ldg(p.sorted_pair + row);
-                    const float w = sp >= 0 ? __ldg(p.topk_w + sp) : 1.0f;
-                    const float y = w * acc0[i];
-                    range_bad |= !f16_range_ok(y);
-                    p.out[row * p.N + n] = to_f16(y);
-                }
-            }
-        }
-        if (MODE == 0 && p.ks > 1 && ok) {
-            // K-split fixup: the warp that writes the last of the ks partial
-            // slices of its 16 columns sums them in slice order (the result does
-            // not depend on which CTA arrives last) and applies the SwiGLU.
-            __threadfence();
-            int last = 0;
-            if (lane == 0) {
-                const int64_t slot = (int64_t(U.i) * (p.N / NS) + U.n0 / NS) * CONSUMERS + cw;
-                last = atomicAdd(p.fix + slot, 1) == p.ks - 1;
-            }
-            last = __shfl_sync(0xFFFFFFFFu, last, 0);
-            if (last) {
-                __threadfence();
-                for (int j = lane; j < U.nrows * 16; j += 32) {
-                    const int64_t row = int64_t(U.row0) + j / 16;
-                    const int n = U.n0 + cw * 16 + (j & 15);
-                    float g = 0.f, v = 0.f;
-                    for (int sl = 0; sl < p.ks; ++sl) {
-                        g += __ldcg(p.part + ((int64_t(sl) * 2 + 0) * p.rows + row) * p.N + n);
-                        v += __ldcg(p.part + ((int64_t(sl) * 2 + 1) * p.rows + row) * p.N + n);
-                    }
-                    const float h = swiglu(g, v, p.limit);
-                    range_bad |= !f16_range_ok(h);
-                    p.out[row * p.N + n] = to_f16(h);
                 }
             }
         }
     }
     if (range_bad) set_error(p.err, MOE_DEVERR_RANGE);
+}
+
+// h = swiglu(sum_ks part_g, sum_ks part_u) for the streaming experts' rows (ks > 1).
+__global__ void __launch_bounds__(256) stream_reduce_kernel(const float* __restrict__ part, int ks, int64_t rows,
+                                                            int f, const int32_t* __restrict__ offsets,
+                                                            const int32_t* __restrict__ stream_list,
+                                                            const int32_t* __restrict__ n_stream, float limit,
+                                                            uint16_t* __restrict__ h, uint32_t* err) {
+    griddep_wait();
+    griddep_launch();
+    const int n = __ldg(n_stream);
+    bool range_bad = false;
+    for (int i = blockIdx.x; i < n; i += gridDim.x) {
+        const int e = __ldg(stream_list + i);
+        const int r0 = __ldg(offsets + e), nr = __ldg(offsets + e + 1) - r0;
+        for (int j = threadIdx.x; j < nr * f; j += blockDim.x) {
+            const int64_t row = r0 + j / f;
+            const int col = j % f;
+            float g = 0.f, u = 0.f;
+            for (int s = 0; s < ks; ++s) {
+                g += part[((int64_t(s) * 2 + 0) * rows + row) * f + col];
+                u += part[((int64_t(s) * 2 + 1) * rows + row) * f + col];
+            }
+            const float hv = swiglu(g, u, limit);
+            range_bad |= !f16_range_ok(hv);
+            h[row * f + col] = to_f16(hv);
+        }
+    }
+    if (range_bad) set_error(err, MOE_DEVERR_RANGE);
 }
 
 using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
@@ -337,23 +367,36 @@ static bool map_2d(CUtensorMap* m, const void* base, int64_t nrows, int ncols, i
                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// The same matrix seen as [ncols/64 chunks, nrows, 64] (3-D, 128-byte swizzle):
+// one copy brings `chunks` 64 x 64 boxes of adjacent columns, 8 KB apart.
+static bool map_chunks(CUtensorMap* m, const void* base, int64_t nrows, int ncols, int chunks) {
+    EncodeTiledFn enc = get_encode();
+    if (!enc) return false;
+    cuuint64_t gd[3] = {64, cuuint64_t(nrows), cuuint64_t(ncols / 64)};
+    cuuint64_t gs[2] = {cuuint64_t(ncols) * 2, 128};
+    cuuint32_t bx[3] = {64, BKS, cuuint32_t(chunks)}, es[3] = {1, 1, 1};
+    return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), gd, gs, bx, es,
+               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 template <int MODE>
 static cudaError_t launch_one(const CUtensorMap& W0, const CUtensorMap& W1, const CUtensorMap& S0,
                               const CUtensorMap& S1, const CUtensorMap& X, const StreamParams& p, int grid,
-                              cudaStream_t s) {
+                              bool pdl, cudaStream_t s) {
     static int configured_dev = -1;
     int dev = 0;
     cudaGetDevice(&dev);
     if (configured_dev != dev) {
         cudaError_t e =
-            cudaFuncSetAttribute(stream_kernel<MODE>, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
+            cudaFuncSetAttribute(stream_kernel<MODE>, cudaFuncAttributeMaxDynamicSharedMemorySize, SCfg<MODE>::SMEM);
         if (e != cudaSuccess) return e;
         configured_dev = dev;
     }
     {
         ProfScope prof_(MODE == 0 ? MOE_K_STREAM_GATEUP : MOE_K_STREAM_DOWN, s);
-        const cudaError_t le = launch_pdl(stream_kernel<MODE>, dim3(grid), dim3(THREADS), SMEM_BYTES, s, W0, W1,
-                                          S0, S1, X, p);
+        const cudaError_t le = launch_pdl(pdl, stream_kernel<MODE>, dim3(grid), dim3(THREADS), SCfg<MODE>::SMEM, s,
+                                          W0, W1, S0, S1, X, p);
         if (le != cudaSuccess) return le;
     }
     return cudaGetLastError();
@@ -363,20 +406,19 @@ static cudaError_t launch_one(const CUtensorMap& W0, const CUtensorMap& W1, cons
 
 // Gate/up (+ reduce) then down for the experts on the streaming list.
 // xg: the gathered rows [rows, d] (bf16); h: [rows, f] fp16.
-cudaError_t launch_stream_ffn(const Dims& D, const uint16_t* xg, uint16_t* h, float* part, int32_t* fix,
-                              const int32_t* offsets,
+cudaError_t launch_stream_ffn(const Dims& D, const uint16_t* xg, uint16_t* h, float* part, const int32_t* offsets,
                               const int32_t* stream_list, const int32_t* n_stream, const int32_t* sorted_pair,
                               const float* topk_w, const moe_weights* w, uint16_t* y_rows, uint32_t* err,
                               uint64_t wait_ns, cudaStream_t s) {
     using namespace st;
     CUtensorMap mG, mU, mD, mSG, mSU, mSD, mX, mH;
     if (!map_2d(&mG, w->w_gate, int64_t(D.E) * D.d, D.f, BKS) || !map_2d(&mU, w->w_up, int64_t(D.E) * D.d, D.f, BKS) ||
-        !map_2d(&mD, w->w_down, int64_t(D.E) * D.f, D.d, BKS) || !map_2d(&mX, xg, D.rows, D.d, RC) ||
+        !map_chunks(&mD, w->w_down, int64_t(D.E) * D.f, D.d, 4) || !map_2d(&mX, xg, D.rows, D.d, RC) ||
         !map_2d(&mH, h, D.rows, D.f, RC))
         return cudaErrorInvalidValue;
     if (D.has_shared) {
         if (!map_2d(&mSG, w->shared_gate, D.d, D.f, BKS) || !map_2d(&mSU, w->shared_up, D.d, D.f, BKS) ||
-            !map_2d(&mSD, w->shared_down, D.f, D.d, BKS))
+            !map_chunks(&mSD, w->shared_down, D.f, D.d, 4))
             return cudaErrorInvalidValue;
     } else {
         mSG = mG;
@@ -404,9 +446,15 @@ cudaError_t launch_stream_ffn(const Dims& D, const uint16_t* xg, uint16_t* h, fl
     p.kslice = D.d / D.ks;
     p.out = h;
     p.part = part;
-    p.fix = fix;
-    cudaError_t e = launch_one<0>(mG, mU, mSG, mSU, mX, p, grid, s);
+    const bool pdl = use_pdl(D.T);
+    cudaError_t e = launch_one<0>(mG, mU, mSG, mSU, mX, p, grid, pdl, s);
     if (e != cudaSuccess) return e;
+    if (D.ks > 1) {
+        ProfScope prof_(MOE_K_STREAM_REDUCE, s);
+        const cudaError_t le = launch_pdl(pdl, stream_reduce_kernel, dim3(grid * 2), dim3(256), 0, s, part, D.ks,
+                                          D.rows, D.f, offsets, stream_list, n_stream, D.limit, h, err);
+        if (le != cudaSuccess) return le;
+    }
     // down
     p.mode = 1;
     p.K = D.f;
@@ -415,7 +463,7 @@ cudaError_t launch_stream_ffn(const Dims& D, const uint16_t* xg, uint16_t* h, fl
     p.kslice = D.f;
     p.out = y_rows;
     p.part = nullptr;
-    return launch_one<1>(mD, mD, mSD, mSD, mH, p, grid, s);
+    return launch_one<1>(mD, mD, mSD, mSD, mH, p, grid, pdl, s);
 }
 
 }  // namespace moe

@@ -325,6 +325,25 @@ def test_forward_host_matches_device():
     assert torch.equal(o_h.view(torch.int32), ref_out.cpu().view(torch.int32))
 
 
+def test_forward_host_async_pipeline_matches_device():
+    """Four steps on two streams (separate workspaces and pinned buffers), copies overlapping kernels."""
+    cfg = SMALL["ragged"]
+    d = device_inputs(cfg)
+    ref_out, _ = run_forward(cfg, d)
+    p = P_of(cfg, b.VARIANT_AUTO, True)
+    W = W_of(d, True)
+    slots = [dict(stream=torch.cuda.Stream(), ws=b.workspace(p, b.WS_FORWARD_HOST),
+                  x=d["x"].cpu().pin_memory(), l=d["logits"].cpu().pin_memory(),
+                  o=torch.full((cfg.T, cfg.d), float("nan"), dtype=torch.float32).pin_memory()) for _ in range(2)]
+    for i in range(4):
+        sl = slots[i % 2]
+        b.forward_host_async(p, sl["x"], sl["l"], W, sl["o"], sl["ws"], stream=sl["stream"])
+    torch.cuda.synchronize()
+    for sl in slots:
+        assert b.get_error(sl["ws"]) == 0
+        assert torch.equal(sl["o"].view(torch.int32), ref_out.cpu().view(torch.int32))
+
+
 def test_bf16_output_option():
     cfg = SMALL["ragged"]
     d = device_inputs(cfg)
