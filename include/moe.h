@@ -329,6 +329,15 @@ MOE_API int moe_clear_error(void* ws, moe_stream_t stream);
 MOE_API int moe_set_wait_limit_ns(uint64_t ns);
 
 /*
+ * Self-test of the failure path (the pages have no counterpart): one tiny
+ * kernel waits, with the same bounded wait as the pipelined kernels, on an
+ * mbarrier that nothing completes. After limit_ns (1 .. 1e10) it gives up,
+ * ORs MOE_DEVERR_TIMEOUT into the error word at err_ws and returns, so the
+ * context stays usable. Asynchronous; read the word with moe_get_error().
+ */
+MOE_API int moe_wait_selftest(void* err_ws, uint64_t limit_ns, moe_stream_t stream);
+
+/*
  * Kernel ids for the profiler and moe_launch_count(). Each is one kernel of
  * the library; a call launches a fixed sequence of them (no host sync).
  */
@@ -345,7 +354,8 @@ MOE_API int moe_set_wait_limit_ns(uint64_t ns);
 #define MOE_K_STREAM_DOWN   10  /* S8 few-rows down */
 #define MOE_K_COMBINE       11  /* S7 gate-weighted combine */
 #define MOE_K_CONVERT       12  /* load-time bf16 -> fp16 weight copy (not a layer step) */
-#define MOE_K_COUNT         13
+#define MOE_K_FRONT         13  /* S1-S3 + schedule fused, moe_forward with T <= 64 */
+#define MOE_K_COUNT         14
 
 /*
  * Number of kernel launches one call of `which` (MOE_WS_ROUTE .. MOE_WS_FORWARD_HOST,

@@ -33,12 +33,12 @@ EXPORTS = ("moe_version", "moe_status_string", "moe_capacity", "moe_max_rows", "
            "moe_route", "moe_permute", "moe_expert_ffn", "moe_combine", "moe_forward", "moe_forward_host",
            "moe_get_error", "moe_clear_error", "moe_set_wait_limit_ns", "moe_launch_count",
            "moe_profile_enable", "moe_profile_collect", "moe_convert_bf16_to_f16",
-           "moe_permute_noalloc", "moe_forward_host_async")
+           "moe_permute_noalloc", "moe_forward_host_async", "moe_wait_selftest")
 NOALLOC_MAX_PAIRS = 262144  # MOE_NOALLOC_MAX_PAIRS
 
 # kernel ids (MOE_K_*), in order
 KERNELS = ("route", "perm_count", "perm_scan", "perm_scatter", "schedule", "gather", "tc_gateup", "tc_down",
-           "stream_gateup", "stream_reduce", "stream_down", "combine", "convert")
+           "stream_gateup", "stream_reduce", "stream_down", "combine", "convert", "front")
 
 
 class MoeError(RuntimeError):
@@ -82,6 +82,7 @@ def lib() -> ctypes.CDLL:
             "moe_forward": ([_P, _V, _V, ctypes.POINTER(Weights), _V, _V, _V, _S, _V], ctypes.c_int),
             "moe_forward_host": ([_P, _V, _V, ctypes.POINTER(Weights), _V, _V, _S, _V], ctypes.c_int),
             "moe_forward_host_async": ([_P, _V, _V, ctypes.POINTER(Weights), _V, _V, _S, _V], ctypes.c_int),
+            "moe_wait_selftest": ([_V, ctypes.c_uint64, _V], ctypes.c_int),
             "moe_get_error": ([_V, ctypes.POINTER(ctypes.c_uint32), _V], ctypes.c_int),
             "moe_clear_error": ([_V, _V], ctypes.c_int),
             "moe_set_wait_limit_ns": ([ctypes.c_uint64], ctypes.c_int),
@@ -207,6 +208,11 @@ def forward_host_async(p, x_host, logits_host, W: Weights, out_host, ws, stream=
     """moe_forward_host_async: as forward_host, enqueued on the stream without synchronising."""
     check(lib().moe_forward_host_async(ctypes.byref(p), _p(x_host), _p(logits_host), ctypes.byref(W),
                                        _p(out_host), _p(ws), ws.numel(), _stream(stream)), "moe_forward_host_async")
+
+
+def wait_selftest(err_ws, limit_ns, stream=None):
+    """moe_wait_selftest: a bounded wait on a barrier nothing completes; sets DEVERR_TIMEOUT."""
+    check(lib().moe_wait_selftest(_p(err_ws), int(limit_ns), _stream(stream)), "moe_wait_selftest")
 
 
 def get_error(ws, stream=None) -> int:

@@ -173,8 +173,9 @@ cudaError_t launch_expert_ffn(const Dims& D, const WsLayout& L, const FfnArgs& a
     uint16_t* xg = reinterpret_cast<uint16_t*>(ws + L.xg);
     uint16_t* h = reinterpret_cast<uint16_t*>(ws + L.h);
     float* part = L.part ? reinterpret_cast<float*>(ws + L.part) : nullptr;
-    cudaError_t e = launch_schedule(D, a.offsets, tile_base, stream_list, n_stream, a.err, s);
-    if (e != cudaSuccess) return e;
+    cudaError_t e = cudaSuccess;
+    if (!a.scheduled && (e = launch_schedule(D, a.offsets, tile_base, stream_list, n_stream, a.err, s)) != cudaSuccess)
+        return e;
     // Rows in expert order for both variants (fp16 for Q4G32, whose MMAs run
     // in fp16). A TMA tile::gather4 of the rows inside the GEMM was measured
     // slower: 32 TMA instructions per k-block left the producer behind.
@@ -302,7 +303,7 @@ int moe_expert_ffn(const moe_params* p, const uint16_t* x, const int32_t* offset
     if (!al16(x) || !al16(y_rows)) return MOE_ERR_MISALIGNED;
     const WsLayout L = ws_layout(D, MOE_WS_EXPERT_FFN);
     FfnArgs a{x, offsets, sorted_token, sorted_pair, topk_w, w, y_rows, static_cast<uint8_t*>(ws),
-              static_cast<uint32_t*>(ws), g_wait_ns.load()};
+              static_cast<uint32_t*>(ws), g_wait_ns.load(), false};
     return status_of(launch_expert_ffn(D, L, a, stream));
 }
 
@@ -331,13 +332,23 @@ static int forward_impl(const Dims& D, const WsLayout& L, const uint16_t* x, con
     int32_t* pair_row = reinterpret_cast<int32_t*>(ws + L.pair_row);
     uint16_t* y_rows = reinterpret_cast<uint16_t*>(ws + L.y_rows);
     uint32_t* err = reinterpret_cast<uint32_t*>(ws);
-    cudaError_t e = launch_route(logits, D.T, D.E, D.k, topk_idx, topk_w, stream);
-    if (e != cudaSuccess) return MOE_ERR_CUDA;
-    e = launch_permute(D, topk_idx, reinterpret_cast<int32_t*>(ws + L.blockcounts),
-                       reinterpret_cast<int32_t*>(ws + L.blockbase), counts, kept, offsets, sorted_token,
-                       sorted_pair, pair_row, err, stream);
-    if (e != cudaSuccess) return MOE_ERR_CUDA;
-    FfnArgs a{x, offsets, sorted_token, sorted_pair, topk_w, w, y_rows, ws, err, g_wait_ns.load()};
+    const bool front = D.T <= kFrontMaxTokens;
+    cudaError_t e;
+    if (front) {  // routing, permutation and schedule in one small kernel
+        e = launch_front_small(D, logits, topk_idx, topk_w, counts, kept, offsets, sorted_token, sorted_pair,
+                               pair_row, reinterpret_cast<int32_t*>(ws + L.tile_base),
+                               reinterpret_cast<int32_t*>(ws + L.stream_list),
+                               reinterpret_cast<int32_t*>(ws + L.n_stream), err, stream);
+        if (e != cudaSuccess) return MOE_ERR_CUDA;
+    } else {
+        e = launch_route(logits, D.T, D.E, D.k, topk_idx, topk_w, stream);
+        if (e != cudaSuccess) return MOE_ERR_CUDA;
+        e = launch_permute(D, topk_idx, reinterpret_cast<int32_t*>(ws + L.blockcounts),
+                           reinterpret_cast<int32_t*>(ws + L.blockbase), counts, kept, offsets, sorted_token,
+                           sorted_pair, pair_row, err, stream);
+        if (e != cudaSuccess) return MOE_ERR_CUDA;
+    }
+    FfnArgs a{x, offsets, sorted_token, sorted_pair, topk_w, w, y_rows, ws, err, g_wait_ns.load(), front};
     if ((e = launch_expert_ffn(D, L, a, stream)) != cudaSuccess) return MOE_ERR_CUDA;
     if ((e = launch_combine(D, y_rows, pair_row, offsets, out, stream)) != cudaSuccess) return MOE_ERR_CUDA;
     if (counts_out &&
@@ -433,7 +444,7 @@ int moe_launch_count(const moe_params* p, int which, int* n) {
         case MOE_WS_PERMUTE: *n = 3; break;
         case MOE_WS_EXPERT_FFN: *n = ffn; break;
         case MOE_WS_COMBINE: *n = 1; break;
-        default: *n = 1 + 3 + ffn + 1; break;
+        default: *n = D.T <= kFrontMaxTokens ? 1 + (ffn - 1) + 1 : 1 + 3 + ffn + 1; break;
     }
     return MOE_OK;
 }

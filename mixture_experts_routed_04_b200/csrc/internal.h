@@ -50,6 +50,14 @@ cudaError_t launch_permute(const Dims& D, const int32_t* topk_idx, int32_t* bloc
                            int32_t* counts, int32_t* kept, int32_t* offsets, int32_t* sorted_token,
                            int32_t* sorted_pair, int32_t* pair_row, uint32_t* err, cudaStream_t s);
 
+// Batches of at most this many tokens run routing, permutation and the tile
+// schedule as one fused single-block kernel (front.cu).
+constexpr int kFrontMaxTokens = 64;
+cudaError_t launch_front_small(const Dims& D, const float* logits, int32_t* topk_idx, float* topk_w,
+                               int32_t* counts, int32_t* kept, int32_t* offsets, int32_t* sorted_token,
+                               int32_t* sorted_pair, int32_t* pair_row, int32_t* tile_base, int32_t* stream_list,
+                               int32_t* n_stream, uint32_t* err, cudaStream_t s);
+
 struct FfnArgs {
     const uint16_t* x;
     const int32_t* offsets;
@@ -61,6 +69,7 @@ struct FfnArgs {
     uint8_t* ws;
     uint32_t* err;
     uint64_t wait_ns;
+    bool scheduled;  // the fused front kernel already wrote the tile schedule
 };
 cudaError_t launch_expert_ffn(const Dims& D, const WsLayout& L, const FfnArgs& a, cudaStream_t s);
 

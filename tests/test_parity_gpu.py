@@ -294,6 +294,19 @@ def test_full_size_quantised_workload():
     check_close(f64(fout)[toks], ref, "quant sampled tokens (moe_forward)")
 
 
+@pytest.mark.parametrize("name", ["tiny", "single_token", "shared_small", "k_equals_E", "small_capped"])
+def test_fused_front_matches_separate_kernels(name):
+    """moe_forward with T <= 64 runs routing, permutation and schedule as one kernel; the layer
+    must equal, bit for bit, the separate route / permute / expert_ffn / combine calls."""
+    cfg = SMALL.get(name) or synth.LayerConfig("small_capped", T=64, d=128, f=128, E=8, k=2, capacity_factor=0.6)
+    assert cfg.T <= 64
+    d = device_inputs(cfg)
+    steps = run_steps(cfg, d, b.VARIANT_AUTO, True)
+    out, counts = run_forward(cfg, d)
+    assert np.array_equal(f64(out), steps["out"])
+    assert np.array_equal(counts, steps["counts"])
+
+
 def test_forward_is_deterministic():
     cfg = synth.CONFIGS["prompt"].replace(T=1024)
     d = device_inputs(cfg)
