@@ -14,7 +14,9 @@ the max over ranks (NCCL all-reduce of the measured times only).
 One JSON line on rank 0: value = tokens/s of the whole job; plus TFLOP/s (or
 GB/s for the decode configs), the roofline of the dominant kernel measured live
 (per-kernel CUDA events inside the library, moe_profile_*), the end-to-end
-number through moe_forward_host (host buffers, copies inside the timed region),
+number through the host-buffer entry points (copies of every step's inputs in
+and output back inside the timed region; a pipelined loop over three streams
+with moe_forward_host_async, and one synchronous moe_forward_host per step),
 SM clocks sampled through NVML during the timed region, and the fp64 CPU
 oracle's throughput on this host as a baseline.
 
@@ -362,10 +364,10 @@ def own_arm(args, cfg):
     torch.cuda.synchronize()
     with ClockSampler(local) as clocks:
         total_ms = timed_steps(graph.replay, K)
-    eager_ms = timed_steps(step, max(3, min(K, 50))) / max(3, min(K, 50))
     if dist:
         dist.barrier()
     total_ms = max_over_ranks(total_ms, dist, "cuda")
+    eager_ms = max_over_ranks(timed_steps(step, max(3, min(K, 50))) / max(3, min(K, 50)), dist, "cuda")
     if b.get_error(ws):
         raise RuntimeError("device error word set during the timed steps")
     ms = total_ms / K
@@ -400,10 +402,11 @@ def own_arm(args, cfg):
         ms_down_bf16 = tot / kb
 
     # End to end through the host-buffer entry points: every step copies its x and logits in
-    # from pinned host memory and its output back. "value": a pipelined loop over two streams
+    # from pinned host memory and its output back. "value": a pipelined loop over three streams
     # (moe_forward_host_async, separate workspaces and host buffers per stream), so one step's
-    # copies overlap another's kernels, as a serving loop runs; "sync": one moe_forward_host
-    # call per step (copies, layer and copy back in sequence, then a host synchronisation).
+    # copies overlap other steps' kernels and copies, as a serving loop runs; "sync": one
+    # moe_forward_host call per step (copies, layer and copy back in sequence, then a host
+    # synchronisation).
     e2e = None
     if not args.no_e2e:
         h2d = cfg.T * cfg.d * 2 + cfg.T * cfg.E * 4
@@ -411,7 +414,7 @@ def own_arm(args, cfg):
         ek = max(3, min(K, 50))
         slots = [dict(stream=torch.cuda.Stream(), ws=b.workspace(p, b.WS_FORWARD_HOST),
                       x=d["x"].cpu().pin_memory(), l=d["logits"].cpu().pin_memory(),
-                      o=torch.empty(cfg.T, cfg.d, dtype=torch.float32).pin_memory()) for _ in range(2)]
+                      o=torch.empty(cfg.T, cfg.d, dtype=torch.float32).pin_memory()) for _ in range(3)]
 
         def step_async(i):
             sl = slots[i % len(slots)]
@@ -453,7 +456,7 @@ def own_arm(args, cfg):
         e_ms = max_over_ranks(e_ms, dist, "cuda")
         e2e = {"value": aggregate_tokens_per_s(cfg.T, world, pipe_ms), "unit": "tokens/s",
                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": pipe_ms,
-               "mode": "pipelined: moe_forward_host_async on 2 streams, pinned host buffers; no L2 flush "
+               "mode": "pipelined: moe_forward_host_async on 3 streams, pinned host buffers; no L2 flush "
                        "(the touched weights exceed L2)",
                "sync": {"value": aggregate_tokens_per_s(cfg.T, world, e_ms / ek), "ms_per_step": e_ms / ek,
                         "mode": "one moe_forward_host call per step (L2 flushed between steps)"}}
