@@ -90,6 +90,14 @@ def test_unsupported_and_missing_buffers(lib):
     # null workspace / buffers: rejected before any CUDA call
     assert lib.moe_route(ctypes.byref(ok), None, None, None, None, 0, None) == 1
     assert lib.moe_forward(ctypes.byref(ok), None, None, None, None, None, None, 0, None) == 1
+    assert lib.moe_forward_host_async(ctypes.byref(ok), None, None, None, None, None, 0, None) == 1
+    assert lib.moe_forward_host_async(ctypes.byref(p), None, None, None, None, None, 0, None) == 3
+    # the wait self-test validates its arguments before any launch
+    assert lib.moe_wait_selftest(None, 1000, None) == 1
+    assert lib.moe_wait_selftest(ctypes.c_void_p(16), 0, None) == 1
+    assert lib.moe_wait_selftest(ctypes.c_void_p(16), 20_000_000_000, None) == 1
+    # the no-allocation permutation checks its parameters and pointers first
+    assert lib.moe_permute_noalloc(ctypes.byref(ok), None, None, None, None, None, None, None, None, None) == 1
 
 
 def test_product_path_never_touches_the_oracle():
