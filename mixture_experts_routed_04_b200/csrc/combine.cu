@@ -31,18 +31,26 @@ __global__ void __launch_bounds__(256) combine_kernel(const uint16_t* __restrict
         float acc[8];
 #pragma unroll
         for (int q = 0; q < 8; ++q) acc[q] = 0.f;
-        auto add = [&](int64_t r) {
-            const uint4 v = __ldg(reinterpret_cast<const uint4*>(y_rows + r * d) + c);
+        auto add = [&](const uint4& v) {
             acc[0] += f16_lo(v.x); acc[1] += f16_hi(v.x);
             acc[2] += f16_lo(v.y); acc[3] += f16_hi(v.y);
             acc[4] += f16_lo(v.z); acc[5] += f16_hi(v.z);
             acc[6] += f16_lo(v.w); acc[7] += f16_hi(v.w);
         };
-        for (int j = 0; j < k; ++j) {
-            const int r = pair_row[t * k + j];
-            if (r >= 0) add(r);
-        }
-        if (has_shared) add(shared_base + t);
+        // all of the token's row loads in flight first, then the sum in the fixed order j = 0..k-1
+        int rr[kMaxK];
+        uint4 yv[kMaxK];
+#pragma unroll
+        for (int j = 0; j < kMaxK; ++j) rr[j] = j < k ? pair_row[t * k + j] : -1;
+#pragma unroll
+        for (int j = 0; j < kMaxK; ++j)
+            if (rr[j] >= 0) yv[j] = __ldg(reinterpret_cast<const uint4*>(y_rows + int64_t(rr[j]) * d) + c);
+        uint4 ys = make_uint4(0, 0, 0, 0);
+        if (has_shared) ys = __ldg(reinterpret_cast<const uint4*>(y_rows + (shared_base + t) * d) + c);
+#pragma unroll
+        for (int j = 0; j < kMaxK; ++j)
+            if (rr[j] >= 0) add(yv[j]);
+        if (has_shared) add(ys);
         if (OUT_BF16) {
             uint4 o;
             o.x = pack_bf16x2(acc[0], acc[1]);
