@@ -104,10 +104,15 @@ def peaks():
 
 
 def kernel_source_hash(files):
+    """SHA-256 (first 16 hex digits) of the kernel sources with their // comments and blank lines
+    removed, so that a comment edit does not invalidate counters taken on the same code."""
     h = hashlib.sha256()
     for fn in files:
-        with open(os.path.join(ROOT, "mixture_experts_routed_04_b200", "csrc", fn), "rb") as fh:
-            h.update(fh.read())
+        with open(os.path.join(ROOT, "mixture_experts_routed_04_b200", "csrc", fn)) as fh:
+            for line in fh:
+                code = line.split("//", 1)[0].rstrip()
+                if code:
+                    h.update(code.encode() + b"\n")
     return h.hexdigest()[:16]
 
 

@@ -127,7 +127,7 @@ MOE_DEV bool mbar_wait_bounded(uint64_t* bar, uint32_t parity, volatile int* abo
 // follow the configurable wait limit, so a short limit can never skip a drain.
 constexpr uint64_t kDrainLimitNs = 2000000000ull;
 
-// ------------------------------------------------------------------ TMA (no multicast anywhere)
+// ------------------------------------------------------------------ TMA (each copy fills only its own CTA)
 
 MOE_DEV void tma_prefetch_desc(const CUtensorMap* m) {
     asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(m)) : "memory");

@@ -39,7 +39,7 @@
 // adjacent so its weight tile is read from HBM once and served from L2 to its
 // other M-tiles. Every mbarrier wait is bounded in time; a wait that gives up
 // raises MOE_DEVERR_TIMEOUT, the CTA drains its copies and MMAs, frees TMEM and
-// returns. No TMA multicast is used.
+// returns. Every TMA copy fills only the issuing CTA's shared memory.
 #include "schedule.cuh"
 
 namespace moe {

@@ -25,7 +25,7 @@
 // stream_reduce finishes (fixed order, deterministic). Down runs in fp16 (h is
 // fp16; W_down prepared as fp16, or converted in registers after ldmatrix) and
 // writes y = w_pair * (h W_down) (fp16). All waits are bounded; no TMA
-// multicast; no named barriers, so an abort never strands a warp.
+// copy into another CTA; no named barriers, so an abort never strands a warp.
 #include "internal.h"
 
 namespace moe {
