@@ -6,7 +6,8 @@
 One step = one moe_forward over one batch: route → permute → expert FFN →
 combine, every kernel of the library, inputs resident in HBM. W warm-up steps,
 then K timed steps, each bracketed by CUDA events on the launching stream, with
-L2 flushed (a 256 MiB write) between steps outside the events. For N > 1 each
+L2 flushed between steps outside the events (a 256 MiB write, then a 256 MiB read
+so the dirty lines are written back before the next step). For N > 1 each
 rank (one per GPU, launched by torch.distributed.run) runs its own replica of
 the workload — the layer shards by tokens with no exchange — and the time is
 the max over ranks (NCCL all-reduce of the measured times only).
@@ -65,6 +66,21 @@ def parse():
 
 
 # --------------------------------------------------------------------------- workload numbers
+
+class L2Flush:
+    """Between timed steps: write a 256 MiB buffer (every L2 line is evicted), then read another
+    256 MiB buffer, so that the lines the write left dirty are written back before the next timed
+    step starts. The step then begins with a cold L2 holding only clean lines of the second buffer,
+    and does not pay for the flush's write-back traffic."""
+
+    def __init__(self, torch):
+        self.w = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device="cuda")
+        self.r = torch.zeros(FLUSH_BYTES // 4, dtype=torch.int32, device="cuda")
+
+    def __call__(self):
+        self.w.zero_()
+        self.r.max()  # a reduction reading the whole buffer; the result stays on the device
+
 
 def workload_numbers(cfg, P, touched):
     """Algorithmic FLOPs and bytes of one layer call (no padding, no intermediates)."""
@@ -320,7 +336,7 @@ def own_arm(args, cfg):
                   d.get("s_up"), d.get("s_down"), shared=sh)
     ws = b.workspace(p, b.WS_FORWARD)
     out = torch.empty(cfg.T, cfg.d, dtype=torch.float32, device="cuda")
-    flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device="cuda")
+    flush = L2Flush(torch)
     stream = torch.cuda.current_stream()
 
     def step():
@@ -336,7 +352,7 @@ def own_arm(args, cfg):
     wl = workload_numbers(cfg, P, touched)
 
     for _ in range(max(args.warmup, 3)):
-        flush.zero_()
+        flush()
         step()
     torch.cuda.synchronize()
     if b.get_error(ws):
@@ -353,7 +369,7 @@ def own_arm(args, cfg):
         s_ev = [torch.cuda.Event(enable_timing=True) for _ in range(n)]
         e_ev = [torch.cuda.Event(enable_timing=True) for _ in range(n)]
         for i in range(n):
-            flush.zero_()
+            flush()
             s_ev[i].record(stream)
             fn()
             e_ev[i].record(stream)
@@ -362,7 +378,7 @@ def own_arm(args, cfg):
 
     K = args.steps
     for _ in range(3):
-        flush.zero_()
+        flush()
         graph.replay()
     if dist:
         dist.barrier()
@@ -381,7 +397,7 @@ def own_arm(args, cfg):
     b.profile_collect()
     b.profile_enable(True)
     for i in range(K):
-        flush.zero_()
+        flush()
         step()
     torch.cuda.synchronize()
     prof = b.profile_collect()
@@ -396,7 +412,7 @@ def own_arm(args, cfg):
         kb = max(3, min(K, 50))
         tot = 0.0
         for i in range(kb + 3):
-            flush.zero_()
+            flush()
             s0, s1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
             s0.record(stream)
             b.forward(p_bf, d["x"], d["logits"], W_bf, out, ws)
@@ -451,7 +467,7 @@ def own_arm(args, cfg):
             b.forward_host(p, x_h, l_h, W, o_h, pe)
         e_ms = 0.0
         for _ in range(ek):
-            flush.zero_()
+            flush()
             s0, s1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
             s0.record(stream)
             b.forward_host(p, x_h, l_h, W, o_h, pe)
@@ -504,7 +520,7 @@ def own_arm(args, cfg):
                 "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
                 "config": {"workload": workload_name(cfg), "tokens_per_gpu": cfg.T, "routed_rows": P,
                            "touched_experts": touched, "parallelism": f"replicas x{world} (no exchange)",
-                           "l2": "flushed between steps (256 MiB write), inputs also larger than L2"},
+                           "l2": "flushed between steps (256 MiB write + 256 MiB read), touched weights also larger than L2"},
                 "tflops": tflops, "tensor_frac_of_peak": tflops / pk["bf16_tflops"],
                 "gbs": gbs, "hbm_frac_of_peak": gbs / pk["hbm_gbs"], "peaks": pk_src,
                 "roofline": roof,
@@ -561,7 +577,7 @@ def sweep_threshold(args, cfg):
     import torch
     from mixture_experts_routed_04_b200 import binding as b
     d, _, W, out = prepared_layer(cfg, b, torch)
-    flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device="cuda")
+    flush = L2Flush(torch)
     res = {}
     for smax in (0, 4, 8, 16, 24, 32, 48, 64, 96, 128):
         p = b.params_for(cfg, down_dtype=b.DOWN_F16 if cfg.weight_format == "bf16" else b.DOWN_BF16,
@@ -574,7 +590,7 @@ def sweep_threshold(args, cfg):
             b.forward(p, d["x"], d["logits"], W, out, ws)
         tot, n = 0.0, max(args.steps, 5)
         for i in range(n + 3):
-            flush.zero_()
+            flush()
             s0, s1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
             s0.record()
             g.replay()

@@ -69,7 +69,8 @@ struct FfnArgs {
     uint8_t* ws;
     uint32_t* err;
     uint64_t wait_ns;
-    bool scheduled;  // the fused front kernel already wrote the tile schedule
+    bool scheduled;            // the fused front kernel already wrote the tile schedule
+    const int32_t* pair_row;   // moe_forward: row of each pair (-1 dropped), for the token-order row copy
 };
 cudaError_t launch_expert_ffn(const Dims& D, const WsLayout& L, const FfnArgs& a, cudaStream_t s);
 

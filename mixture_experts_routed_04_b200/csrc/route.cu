@@ -4,11 +4,14 @@
 // top-k of probs, renormalised. Renormalising the top-k of a full softmax is a
 // softmax over the k selected logits; that is what is computed, in fp32.
 //
-// One warp per token. Each lane keeps up to 8 of the E <= 256 logits in
-// registers (expert lane + 32*i). k rounds of a warp argmax (butterfly
-// shuffles) pick the experts in descending order; equal values go to the lower
-// expert index, and -0.0 equals +0.0 (plain float compares on the given
-// values, never on recomputed probabilities), so the indices are bit-exact.
+// One warp per token (route_one_token in route.cuh). Each lane keeps up to 8 of
+// the E <= 256 logits as order-preserving integer keys (expert lane + 32*i).
+// k rounds pick the experts in descending order: every lane offers its best
+// untaken key, one warp max-reduction gives the winning value and one
+// min-reduction over the lanes holding it the lowest expert index, so equal
+// values go to the lower index and -0.0 equals +0.0 (the keys are built from
+// the given values, never from recomputed probabilities): the indices are
+// bit-exact.
 #include "route.cuh"
 
 namespace moe {

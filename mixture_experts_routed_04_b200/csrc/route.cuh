@@ -5,11 +5,7 @@
 // top-k of probs, renormalised. Renormalising the top-k of a full softmax is a
 // softmax over the k selected logits; that is what is computed, in fp32.
 //
-// One warp per token. Each lane keeps up to 8 of the E <= 256 logits in
-// registers (expert lane + 32*i). k rounds of a warp argmax (butterfly
-// shuffles) pick the experts in descending order; equal values go to the lower
-// expert index, and -0.0 equals +0.0 (plain float compares on the given
-// values, never on recomputed probabilities), so the indices are bit-exact.
+// One warp per token; see route_one_token below for the selection.
 #pragma once
 #include "internal.h"
 
@@ -17,51 +13,55 @@ namespace moe {
 
 constexpr int kRouteMaxPerLane = 8;  // E <= 256
 
-// a beats b: larger value, or equal value and lower index
-MOE_DEV bool route_beats(float va, int ia, float vb, int ib) { return va > vb || (va == vb && ia < ib); }
+// Order-preserving map of a float to an unsigned key (NaN excluded): larger
+// value <-> larger key; -0.0 is mapped like +0.0 so that the two compare equal.
+MOE_DEV uint32_t route_key(float v) {
+    uint32_t u = __float_as_uint(v == 0.f ? 0.f : v);
+    return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+MOE_DEV float route_unkey(uint32_t k) {
+    return __uint_as_float((k & 0x80000000u) ? (k & 0x7FFFFFFFu) : ~k);
+}
 
 // The whole warp routes token `row` (E logits): lane j < k writes selection j
 // to idx_out[j] / w_out[j]. Warp-uniform; every lane must call it.
+// Each round: every lane takes its best untaken logit (larger value, then
+// lower expert index); one warp max-reduction of the keys gives the winning
+// value and one min-reduction over the lanes holding it gives the lowest
+// expert index among equal values.
 MOE_DEV void route_one_token(const float* __restrict__ row, int E, int k, int32_t* __restrict__ idx_out,
                              float* __restrict__ w_out) {
     const int lane = threadIdx.x & 31;
-    float v[kRouteMaxPerLane];
+    uint32_t key[kRouteMaxPerLane];
 #pragma unroll
     for (int i = 0; i < kRouteMaxPerLane; ++i) {
         const int e = lane + 32 * i;
-        v[i] = (e < E) ? __ldg(row + e) : -INFINITY;
+        key[i] = (e < E) ? route_key(__ldg(row + e)) : 0u;  // 0: below every real key (also -inf's)
     }
-    uint32_t taken = 0;  // bit i: v[i] already selected
-    // indices >= E never win: k <= E and a real -inf beats padding by index
+    uint32_t taken = 0;  // bit i: key[i] already selected (or padding)
+#pragma unroll
+    for (int i = 0; i < kRouteMaxPerLane; ++i)
+        if (lane + 32 * i >= E) taken |= 1u << i;
     float sel_v = 0.f;
     int sel_i = 0;
     float top = 0.f;
     for (int j = 0; j < k; ++j) {
-        float bv = -INFINITY;
+        uint32_t bk = 0;
         int bi = 0x7FFFFFFF;
 #pragma unroll
-        for (int i = 0; i < kRouteMaxPerLane; ++i) {
-            const int e = lane + 32 * i;
-            if (!(taken >> i & 1u) && e < E && route_beats(v[i], e, bv, bi)) {
-                bv = v[i];
-                bi = e;
+        for (int i = 0; i < kRouteMaxPerLane; ++i)
+            if (!(taken >> i & 1u) && (key[i] > bk || bi == 0x7FFFFFFF)) {  // first untaken, then strictly larger
+                bk = key[i];
+                bi = lane + 32 * i;
             }
-        }
-#pragma unroll
-        for (int off = 16; off > 0; off >>= 1) {
-            const float ov = __shfl_xor_sync(0xFFFFFFFFu, bv, off);
-            const int oi = __shfl_xor_sync(0xFFFFFFFFu, bi, off);
-            if (route_beats(ov, oi, bv, bi)) {
-                bv = ov;
-                bi = oi;
-            }
-        }
-        // every lane now holds the same winner
-        if ((bi & 31) == lane) taken |= 1u << (bi >> 5);
-        if (j == 0) top = bv;
+        const uint32_t kmax = __reduce_max_sync(0xFFFFFFFFu, bk);
+        const int wi = int(__reduce_min_sync(0xFFFFFFFFu, (bi != 0x7FFFFFFF && bk == kmax) ? uint32_t(bi) : 0xFFFFFFFFu));
+        if ((wi & 31) == lane) taken |= 1u << (wi >> 5);
+        const float wv = route_unkey(kmax);
+        if (j == 0) top = wv;
         if (lane == j) {
-            sel_v = bv;
-            sel_i = bi;
+            sel_v = wv;
+            sel_i = wi;
         }
     }
     // softmax over the k selected (lane j < k holds selection j)
