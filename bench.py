@@ -37,6 +37,7 @@ import threading
 import time
 
 ROOT = os.path.dirname(os.path.abspath(__file__))
+TILE_ARG = {"auto": 0, "one": 1, "pair": 2}  # moe_params.tile_ctas (MOE_TILE_*)
 sys.path.insert(0, ROOT)
 
 import numpy as np  # noqa: E402
@@ -60,6 +61,8 @@ def parse():
     ap.add_argument("--tokens", type=int, default=0, help="override T of the workload (profiling small cases)")
     ap.add_argument("--profile-calls", type=int, default=0,
                     help="only run this many moe_forward calls and exit (for ncu: no timing, no other kernels)")
+    ap.add_argument("--tile", default="auto", choices=["auto", "one", "pair"],
+                    help="SMs per tcgen05 tile (moe_params.tile_ctas); auto = the library's choice")
     ap.add_argument("--sweep-threshold", action="store_true",
                     help="time moe_forward for each stream_max_rows and print one JSON line")
     return ap.parse_args()
@@ -328,7 +331,9 @@ def own_arm(args, cfg):
         e1.record()
         e1.synchronize()
         prep_ms = e0.elapsed_time(e1)
-    p = b.params_for(cfg, down_dtype=b.DOWN_F16 if down_f16 else b.DOWN_BF16)
+    tile = TILE_ARG[args.tile]
+    p = b.params_for(cfg, down_dtype=b.DOWN_F16 if down_f16 else b.DOWN_BF16, tile_ctas=tile)
+    pair = b.tile_ctas(p) == b.TILE_PAIR
     sh = None
     if cfg.has_shared:
         sh = (d["shared_gate"], d["shared_up"], d["shared_down_f16" if down_f16 else "shared_down"])
@@ -406,7 +411,7 @@ def own_arm(args, cfg):
     # the same steps with W_down given as bf16 (converted to fp16 per tile inside the down GEMM)
     ms_down_bf16 = None
     if down_f16:
-        p_bf = b.params_for(cfg, down_dtype=b.DOWN_BF16)
+        p_bf = b.params_for(cfg, down_dtype=b.DOWN_BF16, tile_ctas=tile)
         W_bf = b.weights(d["w_gate"], d["w_up"], d["w_down"],
                          shared=(d["shared_gate"], d["shared_up"], d["shared_down"]) if cfg.has_shared else None)
         kb = max(3, min(K, 50))
@@ -487,10 +492,15 @@ def own_arm(args, cfg):
     ridge = pk["bf16_tflops"] * 1e12 / (pk["hbm_gbs"] * 1e9)
     tensor_bound = wl["flops"] / wl["bytes"] >= ridge
     # Dominant kernel: the largest measured share of the step among the expert GEMMs.
-    names = {"tc_gateup": ("grouped_gemm_kernel<0> (tcgen05 gate/up + clamped SwiGLU)", "gateup", "gemm_tc.cu"),
-             "tc_down": ("grouped_gemm_kernel<1> (tcgen05 down + gate scale)", "down", "gemm_tc.cu"),
-             "stream_gateup": ("stream_kernel<0> (few-rows gate/up)", "gateup", "stream.cu"),
-             "stream_down": ("stream_kernel<1> (few-rows down)", "down", "stream.cu")}
+    one_sm = ["gemm_tc.cu", "gemm_tc.cuh", "common.cuh"]
+    two_sm = ["gemm_pair.cu", "gemm_tc.cuh", "common.cuh"]
+    names = {"tc_gateup": ("grouped_gemm_pair_kernel<0> (tcgen05 SM pairs, gate/up + clamped SwiGLU)", "gateup",
+                           two_sm) if pair else
+             ("grouped_gemm_kernel<0> (tcgen05 gate/up + clamped SwiGLU)", "gateup", one_sm),
+             "tc_down": ("grouped_gemm_pair_kernel<1> (tcgen05 SM pairs, down + gate scale)", "down", two_sm)
+             if pair and down_f16 else ("grouped_gemm_kernel<1> (tcgen05 down + gate scale)", "down", one_sm),
+             "stream_gateup": ("stream_kernel<0> (few-rows gate/up)", "gateup", ["stream.cu", "common.cuh"]),
+             "stream_down": ("stream_kernel<1> (few-rows down)", "down", ["stream.cu", "common.cuh"])}
     kern = max(names, key=lambda k: prof.get(k, (0.0, 0))[0])
     kms, kn = prof.get(kern, (0.0, 0))
     k_avg = kms / kn if kn else float("nan")
@@ -508,7 +518,7 @@ def own_arm(args, cfg):
         roof = {"kernel": label, "bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
                 "frac": achieved / peak, "peak_source": f"{pk_src} hbm_gbs"}
     roof.update({"avg_launch_ms": k_avg, "algorithmic_per_launch": work, "share_of_step": kms / K / ms,
-                 "traffic": committed_traffic(kern, [src, "common.cuh"], cfg.name)})
+                 "traffic": committed_traffic(kern, src, cfg.name)})
 
     line = None
     if rank == 0:
@@ -529,6 +539,7 @@ def own_arm(args, cfg):
                 "step_launch": "CUDA graph replay of one moe_forward call",
                 "ms_per_step_eager": eager_ms,
                 "w_down": "fp16 copy prepared once at load time" if down_f16 else "n/a",
+                "tile_ctas": b.tile_ctas(p),
                 "w_down_prep_ms": prep_ms, "ms_per_step_w_down_bf16": ms_down_bf16,
                 "clocks": clocks.summary(), "e2e": e2e}
     if dist:
@@ -541,7 +552,7 @@ def own_arm(args, cfg):
     return 0
 
 
-def prepared_layer(cfg, b, torch, stream_max_rows=-1):
+def prepared_layer(cfg, b, torch, stream_max_rows=-1, tile_ctas=0):
     """Device inputs, load-time fp16 W_down, params, weights struct, workspace, output."""
     from synth.device import upload
     d = upload(cfg, "cuda")
@@ -550,7 +561,8 @@ def prepared_layer(cfg, b, torch, stream_max_rows=-1):
     sh = None
     if cfg.has_shared:
         sh = (d["shared_gate"], d["shared_up"], b.prepare_down_f16(d["shared_down"]))
-    p = b.params_for(cfg, down_dtype=b.DOWN_F16 if f16 else b.DOWN_BF16, stream_max_rows=stream_max_rows)
+    p = b.params_for(cfg, down_dtype=b.DOWN_F16 if f16 else b.DOWN_BF16, stream_max_rows=stream_max_rows,
+                     tile_ctas=tile_ctas)
     W = b.weights(d["w_gate"], d["w_up"], wd, d.get("s_gate"), d.get("s_up"), d.get("s_down"), shared=sh)
     out = torch.empty(cfg.T, cfg.d, dtype=torch.float32, device="cuda")
     return d, p, W, out
@@ -560,7 +572,7 @@ def profile_calls(args, cfg):
     """Only `n` moe_forward calls (the first one warms up): a short, fixed launch sequence for ncu."""
     import torch
     from mixture_experts_routed_04_b200 import binding as b
-    d, p, W, out = prepared_layer(cfg, b, torch)
+    d, p, W, out = prepared_layer(cfg, b, torch, tile_ctas=TILE_ARG[args.tile])
     ws = b.workspace(p, b.WS_FORWARD)
     torch.cuda.synchronize()
     for _ in range(args.profile_calls):

@@ -87,6 +87,16 @@ typedef struct CUstream_st* moe_stream_t; /* same object as cudaStream_t */
 #define MOE_DOWN_BF16 0 /* as given; each tile is converted to fp16 in shared memory */
 #define MOE_DOWN_F16  1 /* prepared once with moe_convert_bf16_to_f16 (load time) */
 
+/* SMs per tcgen05 tile (moe_params.tile_ctas) */
+#define MOE_TILE_AUTO 0 /* library default: MOE_TILE_ONE (moe_tile_ctas tells which) */
+#define MOE_TILE_ONE  1 /* one SM per 128-row x 256-column tile */
+#define MOE_TILE_PAIR 2 /* two SMs (a cluster, tcgen05 cta_group::2) per 256-row x 256-column
+                           tile, for the bf16 gate/up and the fp16 down GEMMs; a third less
+                           L2-to-SM traffic per FLOP, at the price of rounding each expert's
+                           rows up to 256. Down with W_down given as bf16 and all Q4G32 GEMMs
+                           keep one SM per tile. Measured on B200 slower than MOE_TILE_ONE on
+                           the 4096-token prompt layer, so it is opt-in. */
+
 /* workspace kinds for moe_workspace_size() */
 #define MOE_WS_ROUTE        0
 #define MOE_WS_PERMUTE      1
@@ -117,6 +127,7 @@ typedef struct moe_params {
                                 (single-token decode), else 0 (tiles for all) */
     int32_t out_dtype;       /* MOE_OUT_F32 | MOE_OUT_BF16 */
     int32_t down_dtype;      /* MOE_DOWN_BF16 | MOE_DOWN_F16 */
+    int32_t tile_ctas;       /* SMs per tcgen05 tile: MOE_TILE_* */
 } moe_params;
 
 /*
@@ -162,6 +173,13 @@ MOE_API int moe_capacity(const moe_params* p, int32_t* cap);
  * min(T*k, E*cap) (T*k with no cap) plus T when has_shared.
  */
 MOE_API int moe_max_rows(const moe_params* p, int64_t* rows);
+
+/*
+ * SMs per tcgen05 tile that calls with these params use for the bf16 gate/up
+ * GEMM (MOE_TILE_ONE or MOE_TILE_PAIR), into *ctas. MOE_TILE_AUTO resolves to
+ * MOE_TILE_ONE; MOE_TILE_PAIR with Q4G32 weights resolves to MOE_TILE_ONE.
+ */
+MOE_API int moe_tile_ctas(const moe_params* p, int32_t* ctas);
 
 /* Bytes of workspace each call needs (which = MOE_WS_*); 0 on invalid params. */
 MOE_API size_t moe_workspace_size(const moe_params* p, int which);

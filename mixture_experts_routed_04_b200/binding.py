@@ -26,6 +26,7 @@ OUT_F32, OUT_BF16 = 0, 1
 DOWN_BF16, DOWN_F16 = 0, 1
 WEIGHTS_BF16, WEIGHTS_Q4G32 = 0, 1
 VARIANT_AUTO, VARIANT_TENSOR, VARIANT_STREAM = 0, 1, 2
+TILE_AUTO, TILE_ONE, TILE_PAIR = 0, 1, 2
 WS_ROUTE, WS_PERMUTE, WS_EXPERT_FFN, WS_COMBINE, WS_FORWARD, WS_FORWARD_HOST = range(6)
 
 # every entry point declared in include/moe.h
@@ -33,7 +34,7 @@ EXPORTS = ("moe_version", "moe_status_string", "moe_capacity", "moe_max_rows", "
            "moe_route", "moe_permute", "moe_expert_ffn", "moe_combine", "moe_forward", "moe_forward_host",
            "moe_get_error", "moe_clear_error", "moe_set_wait_limit_ns", "moe_launch_count",
            "moe_profile_enable", "moe_profile_collect", "moe_convert_bf16_to_f16",
-           "moe_permute_noalloc", "moe_forward_host_async", "moe_wait_selftest")
+           "moe_permute_noalloc", "moe_forward_host_async", "moe_wait_selftest", "moe_tile_ctas")
 NOALLOC_MAX_PAIRS = 262144  # MOE_NOALLOC_MAX_PAIRS
 
 # kernel ids (MOE_K_*), in order
@@ -51,7 +52,7 @@ class Params(ctypes.Structure):
                 ("swiglu_limit", ctypes.c_float), ("weight_format", ctypes.c_int32),
                 ("has_shared", ctypes.c_int32), ("d_ff_shared", ctypes.c_int32),
                 ("variant", ctypes.c_int32), ("stream_max_rows", ctypes.c_int32), ("out_dtype", ctypes.c_int32),
-                ("down_dtype", ctypes.c_int32)]
+                ("down_dtype", ctypes.c_int32), ("tile_ctas", ctypes.c_int32)]
 
 
 class Weights(ctypes.Structure):
@@ -74,6 +75,7 @@ def lib() -> ctypes.CDLL:
             "moe_status_string": ([ctypes.c_int], ctypes.c_char_p),
             "moe_capacity": ([_P, ctypes.POINTER(ctypes.c_int32)], ctypes.c_int),
             "moe_max_rows": ([_P, ctypes.POINTER(ctypes.c_int64)], ctypes.c_int),
+            "moe_tile_ctas": ([_P, ctypes.POINTER(ctypes.c_int32)], ctypes.c_int),
             "moe_workspace_size": ([_P, ctypes.c_int], _S),
             "moe_route": ([_P, _V, _V, _V, _V, _S, _V], ctypes.c_int),
             "moe_permute": ([_P, _V, _V, _V, _V, _V, _V, _V, _V, _S, _V], ctypes.c_int),
@@ -101,9 +103,9 @@ def lib() -> ctypes.CDLL:
 
 def params(T, d_model, d_ff, E, k, capacity_factor=0.0, swiglu_limit=7.0, weight_format=WEIGHTS_BF16,
            has_shared=0, d_ff_shared=0, variant=VARIANT_AUTO, stream_max_rows=-1, out_dtype=OUT_F32,
-           down_dtype=DOWN_BF16) -> Params:
+           down_dtype=DOWN_BF16, tile_ctas=TILE_AUTO) -> Params:
     return Params(T, d_model, d_ff, E, k, capacity_factor, swiglu_limit, weight_format, int(has_shared),
-                  d_ff_shared if has_shared else 0, variant, stream_max_rows, out_dtype, down_dtype)
+                  d_ff_shared if has_shared else 0, variant, stream_max_rows, out_dtype, down_dtype, tile_ctas)
 
 
 def params_for(cfg, **over) -> Params:
@@ -135,6 +137,13 @@ def capacity(p: Params):
     v = ctypes.c_int32()
     check(lib().moe_capacity(ctypes.byref(p), ctypes.byref(v)), "moe_capacity")
     return None if v.value < 0 else v.value
+
+
+def tile_ctas(p: Params) -> int:
+    """SMs per tcgen05 tile these params use (TILE_ONE or TILE_PAIR)."""
+    v = ctypes.c_int32()
+    check(lib().moe_tile_ctas(ctypes.byref(p), ctypes.byref(v)), "moe_tile_ctas")
+    return v.value
 
 
 def max_rows(p: Params) -> int:

@@ -98,6 +98,21 @@ MOE_DEV bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
     return ok != 0;
 }
 
+// The same wait with acquire semantics at cluster scope: for a phase completed by
+// arrivals (release, cluster scope) from the other CTA of a pair, so that its
+// earlier writes to this CTA's shared memory are visible after the wait.
+MOE_DEV bool mbar_try_wait_cluster(uint64_t* bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}\n"
+        : "=r"(ok)
+        : "r"(smem_u32(bar)), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+
 MOE_DEV uint64_t globaltimer_ns() {
     uint64_t t;
     asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
@@ -107,12 +122,15 @@ MOE_DEV uint64_t globaltimer_ns() {
 // Wait for the phase of `parity` to complete, for at most limit_ns. Gives up
 // early when another role of the CTA raised *abort. On timeout it raises
 // *abort and sets MOE_DEVERR_TIMEOUT. Returns true when the phase completed.
+// kCluster: acquire at cluster scope (mbar_try_wait_cluster).
+template <bool kCluster = false>
 MOE_DEV bool mbar_wait_bounded(uint64_t* bar, uint32_t parity, volatile int* abort, uint32_t* err,
                                uint64_t limit_ns) {
-    if (mbar_try_wait(bar, parity)) return true;
+    auto try_wait = [&]() { return kCluster ? mbar_try_wait_cluster(bar, parity) : mbar_try_wait(bar, parity); };
+    if (try_wait()) return true;
     const uint64_t t0 = globaltimer_ns();
     for (uint32_t i = 1;; ++i) {
-        if (mbar_try_wait(bar, parity)) return true;
+        if (try_wait()) return true;
         if (abort && *abort) return false;
         if ((i & 63u) == 0 && globaltimer_ns() - t0 > limit_ns) {
             if (abort) *abort = 1;
@@ -155,6 +173,53 @@ MOE_DEV void tma_load_3d(void* dst, const CUtensorMap* m, uint64_t* bar, int32_t
         : "memory");
 }
 
+// ------------------------------------------------------------------ clusters of two CTAs (SM pairs)
+// A pair computes one 256-row tile with tcgen05 ops of cta_group::2: CTA rank 0
+// (the leader) issues the MMAs, which read A and B from the same shared-memory
+// offsets in both CTAs and write both CTAs' TMEM.
+
+MOE_DEV uint32_t cluster_ctarank() {
+    uint32_t r;
+    asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+    return r;
+}
+// The shared::cluster address of the location at CTA-local address `addr` in CTA `rank`.
+MOE_DEV uint32_t mapa_shared(uint32_t addr, uint32_t rank) {
+    uint32_t r;
+    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(addr), "r"(rank));
+    return r;
+}
+// Every thread of both CTAs: writes before are visible to both CTAs after.
+MOE_DEV void cluster_sync_all() {
+    asm volatile("barrier.cluster.arrive.release;\n\tbarrier.cluster.wait.acquire;" ::: "memory");
+}
+MOE_DEV void st_shared_cluster_u32(uint32_t addr, uint32_t v) {
+    asm volatile("st.shared::cluster.u32 [%0], %1;" ::"r"(addr), "r"(v) : "memory");
+}
+// Arrive on an mbarrier of either CTA (shared::cluster address), releasing this
+// thread's earlier writes at cluster scope.
+MOE_DEV void mbar_arrive_cluster(uint32_t addr) {
+    asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(addr) : "memory");
+}
+// TMA tile loads of a pair: the data land in the issuing CTA's shared memory and
+// the byte count is signalled on `bar`, a shared::cluster mbarrier address that
+// may be in the other CTA of the pair (the leader's stage barrier).
+MOE_DEV void tma_load_2d_pair(void* dst, const CUtensorMap* m, uint32_t bar, int32_t x, int32_t y) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%3, "
+        "%4}], [%2];" ::"r"(smem_u32(dst)),
+        "l"(reinterpret_cast<uint64_t>(m)), "r"(bar), "r"(x), "r"(y)
+        : "memory");
+}
+MOE_DEV void tma_load_4d_pair(void* dst, const CUtensorMap* m, uint32_t bar, int32_t x, int32_t y, int32_t z,
+                              int32_t w) {
+    asm volatile(
+        "cp.async.bulk.tensor.4d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%3, "
+        "%4, %5, %6}], [%2];" ::"r"(smem_u32(dst)),
+        "l"(reinterpret_cast<uint64_t>(m)), "r"(bar), "r"(x), "r"(y), "r"(z), "r"(w)
+        : "memory");
+}
+
 // ------------------------------------------------------------------ tcgen05 / TMEM
 
 MOE_DEV void tmem_alloc(uint32_t* dst_smem, uint32_t ncols) {
@@ -182,6 +247,43 @@ MOE_DEV void umma_bf16(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32
 MOE_DEV void umma_commit(uint64_t* bar) {
     asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(smem_u32(bar))
                  : "memory");
+}
+
+// SM-pair forms. Both CTAs' allocating warps (same warp index) allocate,
+// relinquish and free together; the columns are the same in both CTAs.
+MOE_DEV void tmem_alloc_pair(uint32_t* dst_smem, uint32_t ncols) {
+    asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(dst_smem)),
+                 "r"(ncols)
+                 : "memory");
+}
+MOE_DEV void tmem_relinquish_pair() {
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
+}
+MOE_DEV void tmem_dealloc_pair(uint32_t taddr, uint32_t ncols) {
+    asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols) : "memory");
+}
+// D (+)= A * B over the pair, issued by the leader: M rows split 128 + 128 over
+// the two CTAs' A tiles and TMEM, N split N/2 + N/2 over their B tiles.
+MOE_DEV void umma_f16_pair(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc, uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p;\n\t}\n" ::"r"(d_tmem),
+        "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+// Arrive on `bar` (this CTA) once the pair MMAs issued so far have completed.
+MOE_DEV void umma_commit_pair(uint64_t* bar) {
+    asm volatile("tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(smem_u32(bar))
+                 : "memory");
+}
+// The same, arriving on the mbarrier at `bar`'s offset in both CTAs of the pair.
+MOE_DEV void umma_commit_pair_both(uint64_t* bar) {
+    asm volatile(
+        "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 [%0], %1;" ::"r"(
+            smem_u32(bar)),
+        "h"(uint16_t(3))
+        : "memory");
 }
 
 // 32 lanes x 32 consecutive fp32 columns: thread i gets lane (base + i), v[j] = column (col + j).

@@ -40,19 +40,11 @@
 // other M-tiles. Every mbarrier wait is bounded in time; a wait that gives up
 // raises MOE_DEVERR_TIMEOUT, the CTA drains its copies and MMAs, frees TMEM and
 // returns. Every TMA copy fills only the issuing CTA's shared memory.
-#include "schedule.cuh"
+#include "gemm_tc.cuh"
 
 namespace moe {
 
 namespace tc {
-
-constexpr int BM = 128, BK = 64, BN = 256;
-constexpr int A_BYTES = BM * BK * 2;  // 16 KB
-constexpr int B_CHUNK = 64 * BK * 2;  // one 64(N) x 64(K) box, 8 KB
-constexpr int B_BYTES = 4 * B_CHUNK;  // 32 KB (256 N x 64 K, 2-byte elements)
-constexpr int P_BYTES = BN * BK / 2;  // Q4G32 nibbles of 256 rows x 64 K: 8 KB
-constexpr int S_BYTES = 2 * BN * 2;   // two scale groups x 256 rows, fp16: 1 KB
-constexpr int TMEM_COLS = 512;
 
 // WF: weight form. 0 = bf16 as given, 1 = Q4G32, 2 = fp16 (W_down prepared at load time).
 template <int MODE, int WF, int SUB>
@@ -91,61 +83,6 @@ struct Cfg {
         idesc_f16_f32(64, BN, /*ab_bf16=*/(MODE == 0 && WF == 0) ? 1 : 0, /*a_mn=*/0, /*b_mn=*/Q4 ? 0 : 1);
 };
 
-struct GemmParams {
-    int K;        // reduction length (multiple of 64)
-    int n_out;    // output width
-    int n_tiles;  // output tiles per M-tile
-    int E;        // routed experts; index E is the shared expert
-    int Etot;
-    int32_t* unit_counter;     // next unit to claim (zeroed by the schedule kernel)
-    const int32_t* tile_base;  // [Etot+1] exclusive prefix of M-tiles
-    const int32_t* offsets;    // [Etot+1] row offsets
-    uint16_t* out;             // [rows, n_out] fp16 (h or y)
-    const int32_t* sorted_pair;
-    const float* topk_w;
-    float limit;
-    uint32_t* err;
-    uint64_t wait_ns;
-};
-
-struct Unit {
-    int e, m, n, row0, rows;
-};
-
-// p.tile_base counts units of SUB x 128 rows.
-template <int SUB>
-MOE_DEV Unit decode_unit(int u, const GemmParams& p, int nt) {
-    const int g = u / nt;  // global M-tile index
-    int lo = 0, hi = p.Etot;      // tile_base[lo] <= g < tile_base[hi]
-    while (hi - lo > 1) {
-        const int mid = (lo + hi) >> 1;
-        if (__ldg(p.tile_base + mid) <= g) lo = mid;
-        else hi = mid;
-    }
-    Unit U;
-    U.e = lo;
-    const int tb = __ldg(p.tile_base + lo);
-    const int mt = __ldg(p.tile_base + lo + 1) - tb;
-    const int local = u - tb * nt;
-    U.n = local / mt;
-    U.m = local - U.n * mt;
-    const int off = __ldg(p.offsets + lo);
-    const int kept = __ldg(p.offsets + lo + 1) - off;
-    U.row0 = off + U.m * (SUB * BM);
-    U.rows = min(SUB * BM, kept - U.m * (SUB * BM));
-    return U;
-}
-
-MOE_DEV float swiglu(float g, float u, float L) {
-    if (L > 0.f) {
-        g = fminf(fmaxf(g, -L), L);
-        u = fminf(fmaxf(u, -L), L);
-    }
-    // __expf / __fdividef: relative error ~1e-6, far below the fp16 rounding
-    // of h that follows (the accurate forms cost ~5% of the gate/up GEMM).
-    return __fdividef(g, 1.0f + __expf(-g)) * u;
-}
-
 MOE_DEV uint32_t lop3_and_or(uint32_t a, uint32_t mask, uint32_t orv) {
     uint32_t r;
     asm("lop3.b32 %0, %1, %2, %3, 0xEA;" : "=r"(r) : "r"(a), "r"(mask), "r"(orv));  // (a & b) | c
@@ -177,58 +114,6 @@ MOE_DEV uint4 dequant_word(uint32_t w, uint32_t s2) {
     return o;
 }
 
-// ---------------------------------------------------------------- unit ring
-// Work is claimed dynamically: the producer warp takes the next unit with an
-// atomic counter and publishes it in a shared-memory ring that the MMA,
-// epilogue and transform warps read in order. A CTA that draws slow
-// (DRAM-bound) units therefore takes fewer of them and every SM finishes
-// together. Which CTA computes a unit does not change its result.
-constexpr int UR = 8;  // ring depth; the producer runs at most ~2 units ahead of the epilogue
-
-// Producer: claim and publish the next unit (-1 when none is left). Returns
-// false if the bounded wait gave up. Warp-uniform.
-MOE_DEV bool ring_publish(int& u, int& slot, uint32_t& phase, int* counter, int total, volatile int* ring,
-                          uint64_t* ufull, uint64_t* uempty, volatile int* abort_flag, uint32_t* err, uint64_t ns) {
-    const int lane = threadIdx.x & 31;
-    int ok = 1;
-    if (lane == 0) ok = mbar_wait_bounded(uempty + slot, phase ^ 1u, abort_flag, err, ns);
-    ok = __shfl_sync(0xFFFFFFFFu, ok, 0);
-    if (!ok) return false;
-    int v = 0;
-    if (lane == 0) {
-        v = atomicAdd(counter, 1);
-        if (v >= total) v = -1;
-        ring[slot] = v;
-        mbar_arrive(ufull + slot);
-    }
-    u = __shfl_sync(0xFFFFFFFFu, v, 0);
-    if (++slot == UR) {
-        slot = 0;
-        phase ^= 1u;
-    }
-    return true;
-}
-
-// Reader: the next published unit (-1: done). Returns false if the wait gave up.
-MOE_DEV bool ring_read(int& u, int& slot, uint32_t& phase, volatile int* ring, uint64_t* ufull, uint64_t* uempty,
-                       volatile int* abort_flag, uint32_t* err, uint64_t ns) {
-    const int lane = threadIdx.x & 31;
-    int ok = 1;
-    if (lane == 0) ok = mbar_wait_bounded(ufull + slot, phase, abort_flag, err, ns);
-    ok = __shfl_sync(0xFFFFFFFFu, ok, 0);
-    if (!ok) return false;
-    int v = 0;
-    if (lane == 0) {
-        v = ring[slot];
-        mbar_arrive(uempty + slot);
-    }
-    u = __shfl_sync(0xFFFFFFFFu, v, 0);
-    if (++slot == UR) {
-        slot = 0;
-        phase ^= 1u;
-    }
-    return true;
-}
 
 template <int MODE, int WF, int SUB>
 __global__ void __launch_bounds__(Cfg<MODE, WF, SUB>::kThreads, 1)
@@ -464,68 +349,8 @@ __global__ void __launch_bounds__(Cfg<MODE, WF, SUB>::kThreads, 1)
             for (int sub = 0; sub < C::kSub; ++sub) {
                 const int rows = min(BM, U.rows - sub * BM);
                 if (rows <= 0) break;
-                // M=128: lane i of quadrant q is row 32q + i. M=64 (sub-tiles of
-                // <= 64 rows): only lanes 0-15 of each quadrant hold rows, 16q + i.
-                const bool m64 = rows <= 64;
-                const int rit = m64 ? q * 16 + lane : q * 32 + lane;
-                const bool valid = (!m64 || lane < 16) && rit < rows;
-                const int64_t row = int64_t(U.row0) + sub * BM + rit;
                 const uint32_t tb = tmem_base + (uint32_t(q * 32) << 16) + uint32_t((acc * C::kSub + sub) * BN);
-                if (MODE == 0) {
-                    // gate columns first, then the up columns (128 each)
-                    constexpr int hw = 128;
-#pragma unroll 1
-                    for (int c = 0; c < hw / 32; ++c) {
-                        uint32_t g[32], v[32];
-                        tmem_ld_32x32b_x32(tb + c * 32, g);
-                        tmem_ld_32x32b_x32(tb + hw + c * 32, v);
-                        tmem_ld_wait();
-                        const int col = U.n * hw + c * 32;
-                        if (valid && col < p.n_out) {
-                            uint32_t pk[16];
-#pragma unroll
-                            for (int i = 0; i < 16; ++i) {
-                                const float h0 =
-                                    swiglu(__uint_as_float(g[2 * i]), __uint_as_float(v[2 * i]), p.limit);
-                                const float h1 =
-                                    swiglu(__uint_as_float(g[2 * i + 1]), __uint_as_float(v[2 * i + 1]), p.limit);
-                                range_bad |= !(f16_range_ok(h0) && f16_range_ok(h1));
-                                pk[i] = pack_f16x2(h0, h1);
-                            }
-                            uint4* dst = reinterpret_cast<uint4*>(p.out + row * p.n_out + col);
-#pragma unroll
-                            for (int i = 0; i < 4; ++i)
-                                dst[i] = make_uint4(pk[4 * i], pk[4 * i + 1], pk[4 * i + 2], pk[4 * i + 3]);
-                        }
-                    }
-                } else {
-                    float w = 0.f;
-                    if (valid) {
-                        const int sp = __ldg(p.sorted_pair + row);
-                        w = sp >= 0 ? __ldg(p.topk_w + sp) : 1.0f;
-                    }
-#pragma unroll 1
-                    for (int c = 0; c < BN / 32; ++c) {
-                        uint32_t v[32];
-                        tmem_ld_32x32b_x32(tb + c * 32, v);
-                        tmem_ld_wait();
-                        const int col = U.n * BN + c * 32;
-                        if (valid && col < p.n_out) {
-                            uint32_t pk[16];
-#pragma unroll
-                            for (int i = 0; i < 16; ++i) {
-                                const float y0 = w * __uint_as_float(v[2 * i]);
-                                const float y1 = w * __uint_as_float(v[2 * i + 1]);
-                                range_bad |= !(f16_range_ok(y0) && f16_range_ok(y1));
-                                pk[i] = pack_f16x2(y0, y1);
-                            }
-                            uint4* dst = reinterpret_cast<uint4*>(p.out + row * p.n_out + col);
-#pragma unroll
-                            for (int i = 0; i < 4; ++i)
-                                dst[i] = make_uint4(pk[4 * i], pk[4 * i + 1], pk[4 * i + 2], pk[4 * i + 3]);
-                        }
-                    }
-                }
+                epilogue_tile<MODE>(tb, U.n, int64_t(U.row0) + sub * BM, rows, rows <= 64, q, lane, p, range_bad);
             }
             tc_fence_before();
             __syncwarp();
@@ -795,19 +620,33 @@ cudaError_t launch_tensor_ffn(const Dims& D, const uint16_t* xg, uint16_t* h, co
         mSU = mU;
         mSD = mD;
     }
-    // S5: gate/up + SwiGLU -> h
+    // S5: gate/up + SwiGLU -> h (the gate/up maps bring 2 chunks a copy: the
+    // one-SM kernel copies gate and up, each SM of a pair one of them)
     p.K = D.d;
     p.n_out = D.f;
     p.n_tiles = (D.f + 127) / 128;
     p.out = h;
     p.unit_counter = counters;
-    if ((e = launch_gemm<0, 0, 1>(mA, mG, mU, mSG, mSU, p, pdl, s)) != cudaSuccess) return e;
+    e = D.tile_pair ? launch_gemm_pair<0>(mA, mG, mU, mSG, mSU, p, pdl, s)
+                    : launch_gemm<0, 0, 1>(mA, mG, mU, mSG, mSU, p, pdl, s);
+    if (e != cudaSuccess) return e;
     // S6: down + gate scale -> y_rows
     p.K = D.f;
     p.n_out = D.d;
     p.n_tiles = (D.d + BN - 1) / BN;
     p.out = y_rows;
     p.unit_counter = counters + 1;
+    if (D.tile_pair && D.down_f16) {
+        // each SM of a pair copies 128 of the tile's 256 columns: maps of 2 chunks
+        CUtensorMap mD2, mSD2;
+        if (!map_weights(&mD2, w->w_down, D.E, D.f, D.d, 2)) return cudaErrorInvalidValue;
+        if (D.has_shared) {
+            if (!map_weights(&mSD2, w->shared_down, 1, D.f, D.d, 2)) return cudaErrorInvalidValue;
+        } else {
+            mSD2 = mD2;
+        }
+        return launch_gemm_pair<1>(mH, mD2, mD2, mSD2, mSD2, p, pdl, s);
+    }
     return D.down_f16 ? launch_gemm<1, 2, 1>(mH, mD, mD, mSD, mSD, p, pdl, s)
                       : launch_gemm<1, 0, 1>(mH, mD, mD, mSD, mSD, p, pdl, s);
 }

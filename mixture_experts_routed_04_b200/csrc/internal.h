@@ -27,6 +27,7 @@ struct Dims {
     int ks;                   // K-split of the streaming gate/up kernel
     int out_bf16;             // layer output in bf16 (else fp32)
     int down_f16;             // W_down given as fp16 (prepared at load time)
+    int tile_pair;            // bf16 tcgen05 GEMMs on SM pairs (256-row tiles)
 };
 
 // Byte offsets of every scratch array inside a workspace (0 = absent).

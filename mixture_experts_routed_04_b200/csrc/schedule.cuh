@@ -8,7 +8,7 @@ namespace moe {
 // One block of 512 threads; thread e owns expert e (Etot <= 257) and passes its
 // kept row count (0 for e >= Etot). Writes:
 //   tile_base[0 .. Etot]           exclusive prefix of 128-row tiles per expert
-//   tile_base[Etot+1 .. 2*Etot+1]  that of 256-row tiles (Q4G32 units)
+//   tile_base[Etot+1 .. 2*Etot+1]  that of 256-row tiles (Q4G32 and SM-pair units)
 //   stream_list[0 .. n)            experts taken by the streaming kernels
 //   n_stream[0] = n; n_stream[1] = n_stream[2] = 0 (unit counters of the GEMMs)
 // Every thread of the block must call it (it synchronises the block).

@@ -62,7 +62,8 @@ def test_max_rows_and_workspace(lib):
 
 @pytest.mark.parametrize("bad", [
     dict(k=9), dict(k=3, E=2), dict(E=257), dict(d_model=100), dict(d_ff=32), dict(T=-1),
-    dict(capacity_factor=-1.0), dict(capacity_factor=float("nan")), dict(variant=7), dict(weight_format=5)])
+    dict(capacity_factor=-1.0), dict(capacity_factor=float("nan")), dict(variant=7), dict(weight_format=5),
+    dict(tile_ctas=3), dict(tile_ctas=-1)])
 def test_invalid_params_rejected_on_host(lib, bad):
     kw = dict(T=16, d_model=128, d_ff=256, E=8, k=2)
     kw.update(bad)
@@ -70,6 +71,20 @@ def test_invalid_params_rejected_on_host(lib, bad):
     assert b.workspace_size(p, b.WS_FORWARD) == 0
     st = lib.moe_route(ctypes.byref(p), None, None, None, None, 0, None)
     assert st == 1  # MOE_ERR_INVALID_ARG, before any launch
+
+
+def test_tile_shape_choice(lib):
+    """MOE_TILE_AUTO is one SM per tile; SM pairs only on request, and only for bf16 weights."""
+    prompt = dict(T=4096, d_model=2048, d_ff=768, E=128, k=8)
+    assert b.tile_ctas(b.params(**prompt)) == b.TILE_ONE
+    assert b.tile_ctas(b.params(**prompt, tile_ctas=b.TILE_ONE)) == b.TILE_ONE
+    assert b.tile_ctas(b.params(**prompt, tile_ctas=b.TILE_PAIR)) == b.TILE_PAIR
+    assert b.tile_ctas(b.params(8192, 1024, 2048, 128, 2, capacity_factor=1.5)) == b.TILE_ONE
+    assert b.tile_ctas(b.params(1, 4096, 1536, 256, 8, has_shared=1, d_ff_shared=1536)) == b.TILE_ONE
+    assert b.tile_ctas(b.params(64, 128, 256, 8, 2, tile_ctas=b.TILE_PAIR)) == b.TILE_PAIR
+    # the Q4G32 GEMMs keep one SM per tile even when pairs are asked for
+    q4 = b.params(32768, 2048, 768, 128, 8, weight_format=b.WEIGHTS_Q4G32, tile_ctas=b.TILE_PAIR)
+    assert b.tile_ctas(q4) == b.TILE_ONE
 
 
 def test_empty_batch_is_valid_and_launches_nothing(lib):

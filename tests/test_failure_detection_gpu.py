@@ -34,11 +34,12 @@ def test_wait_on_a_barrier_nothing_completes_times_out():
     assert float(x.sum().item()) == 1023 * 1024 / 2
 
 
-@pytest.mark.parametrize("variant", [b.VARIANT_TENSOR, b.VARIANT_STREAM])
-def test_layer_with_tiny_wait_limit_reports_and_recovers(variant):
+@pytest.mark.parametrize("variant,tile", [(b.VARIANT_TENSOR, b.TILE_ONE), (b.VARIANT_TENSOR, b.TILE_PAIR),
+                                          (b.VARIANT_STREAM, b.TILE_AUTO)])
+def test_layer_with_tiny_wait_limit_reports_and_recovers(variant, tile):
     cfg = synth.CONFIGS["tiny"]
     d = device_inputs(cfg)
-    p = P_of(cfg, variant, True)
+    p = P_of(cfg, variant, True, tile_ctas=tile)
     ws = b.workspace(p, b.WS_FORWARD)
     out = torch.empty(cfg.T, cfg.d, dtype=torch.float32, device="cuda")
     b.set_wait_limit_ns(1)
@@ -50,6 +51,6 @@ def test_layer_with_tiny_wait_limit_reports_and_recovers(variant):
         b.set_wait_limit_ns(0)  # back to the default (1 s)
     err = b.get_error(ws)
     assert err & ~(b.DEVERR_TIMEOUT) == 0, f"unexpected error bits {err:#x}"
-    got, _ = run_forward(cfg, d, variant)  # asserts a clean error word itself
+    got, _ = run_forward(cfg, d, variant, tile_ctas=tile)  # asserts a clean error word itself
     ref, _ = reference(cfg)
     check_close(f64(got), ref, "layer after a run with 1 ns waits")

@@ -133,8 +133,8 @@ def P_of(cfg, variant, down_f16, **kw):
     return b.params_for(cfg, variant=variant, down_dtype=b.DOWN_F16 if down_f16 else b.DOWN_BF16, **kw)
 
 
-def run_steps(cfg, d, variant, down_f16):
-    p = P_of(cfg, variant, down_f16)
+def run_steps(cfg, d, variant, down_f16, **kw):
+    p = P_of(cfg, variant, down_f16, **kw)
     T, E, k = cfg.T, cfg.E, cfg.k
     Et = E + int(cfg.has_shared)
     rows = b.max_rows(p)
@@ -161,8 +161,8 @@ def run_steps(cfg, d, variant, down_f16):
             "out": f64(out)}
 
 
-def run_forward(cfg, d, variant=b.VARIANT_AUTO, down_f16=True):
-    p = P_of(cfg, variant, down_f16 and cfg.weight_format == "bf16")
+def run_forward(cfg, d, variant=b.VARIANT_AUTO, down_f16=True, **kw):
+    p = P_of(cfg, variant, down_f16 and cfg.weight_format == "bf16", **kw)
     ws = b.workspace(p, b.WS_FORWARD)
     out = torch.empty(cfg.T, cfg.d, dtype=torch.float32, device="cuda")
     counts = torch.empty(cfg.E + int(cfg.has_shared), dtype=torch.int32, device="cuda")
@@ -212,6 +212,44 @@ def test_small_layers_every_variant(name, variant, down):
     fout, counts = run_forward(cfg, d, VARIANTS[variant], f16)
     assert (counts == it["counts"]).all()
     assert np.array_equal(f64(fout), got["out"])
+
+
+TILES = {"one": b.TILE_ONE, "pair": b.TILE_PAIR}
+
+
+@pytest.mark.parametrize("down", ["bf16", "f16"])
+@pytest.mark.parametrize("tile", list(TILES))
+@pytest.mark.parametrize("name", list(SMALL))
+def test_small_layers_tile_shapes(name, tile, down):
+    """Every expert on the tcgen05 tiles, one SM per 128-row tile or SM pairs on 256-row tiles
+    (the pair kernels cover the bf16 gate/up and the fp16 down; bf16 W_down stays on one SM)."""
+    cfg = SMALL[name]
+    d = device_inputs(cfg)
+    f16 = down == "f16"
+    got = run_steps(cfg, d, b.VARIANT_TENSOR, f16, tile_ctas=TILES[tile])
+    check_routing(cfg, got)
+    check_layer(f"{name}/{tile}/{down}", cfg, got)
+    fout, _ = run_forward(cfg, d, b.VARIANT_TENSOR, f16, tile_ctas=TILES[tile])
+    assert np.array_equal(f64(fout), got["out"])
+
+
+def test_prompt_both_tile_shapes():
+    """The prompt workload at full size with each tile shape, against the per-token definition
+    on sampled tokens, and the two shapes against each other on every element."""
+    cfg = synth.CONFIGS["prompt"]
+    idx, w, perm = routing_reference(cfg)
+    d = device_inputs(cfg)
+    x = synth.bf16_bits_to_f32(synth.x_bits(cfg)).astype(np.float64)
+    rng = np.random.default_rng(11)
+    toks = sorted(set([0, cfg.T - 1] + rng.choice(cfg.T, 48, replace=False).tolist()))
+    ref = oracle.token_outputs(toks, x, idx, w, perm["pair_row"], lambda e: expert_ref(cfg, e), cfg.swiglu_limit)
+    outs = {}
+    for tile, t in TILES.items():
+        out, counts = run_forward(cfg, d, tile_ctas=t)
+        assert (counts == perm["counts"]).all()
+        check_close(f64(out)[toks], ref, f"prompt/{tile} sampled tokens")
+        outs[tile] = f64(out)
+    check_close(outs["pair"], outs["one"], "prompt pair vs one SM per tile")
 
 
 @pytest.mark.parametrize("variant", ["auto", "tensor"])
