@@ -1,5 +1,5 @@
-// gemm_tc.cu — S5, S6 (+ S9) on the 5th-generation tensor cores: the tile
-// schedule (K3) and one persistent grouped GEMM kernel used twice per layer:
+// gemm_tc.cu — S5, S6 (+ S9) on the 5th-generation tensor cores: one
+// persistent grouped GEMM kernel, one SM per tile, used twice per layer:
 //   MODE 0: h = silu(clamp(x W_gate[e])) * clamp(x W_up[e])   (S5, SwiGLU fused)
 //   MODE 1: y = w_pair * (h W_down[e])                          (S6, gate scale fused)
 // with the weights either bf16 ([E, K, N], N contiguous) or Q4G32 (4-bit,
@@ -435,29 +435,6 @@ __global__ void __launch_bounds__(Cfg<MODE, WF, SUB>::kThreads, 1)
 
 }  // namespace tc
 
-// ---------------------------------------------------------------------------- K3 schedule
-
-// One block of 512 threads; thread e owns expert e (Etot <= 257); the
-// schedule itself is schedule_block (shared with the fused front kernel).
-__global__ void __launch_bounds__(512) schedule_kernel(const int32_t* __restrict__ offsets, int Etot, int variant,
-                                                       int stream_max, int32_t* __restrict__ tile_base,
-                                                       int32_t* __restrict__ stream_list,
-                                                       int32_t* __restrict__ n_stream, uint32_t* err) {
-    __shared__ int sums[3][16];
-    griddep_wait();
-    griddep_launch();
-    const int e = threadIdx.x;
-    int kept = 0;
-    if (e < Etot) {
-        kept = offsets[e + 1] - offsets[e];
-        if (kept < 0) {
-            set_error(err, MOE_DEVERR_BOUNDS);
-            kept = 0;
-        }
-    }
-    schedule_block(kept, Etot, variant, stream_max, sums, tile_base, stream_list, n_stream);
-}
-
 // ---------------------------------------------------------------------------- host side
 
 namespace tc {
@@ -553,18 +530,6 @@ cudaError_t launch_gemm(const CUtensorMap& A, const CUtensorMap& B0, const CUten
 }
 
 }  // namespace tc
-
-cudaError_t launch_schedule(const Dims& D, const int32_t* offsets, int32_t* tile_base, int32_t* stream_list,
-                            int32_t* n_stream, uint32_t* err, cudaStream_t s) {
-    int smax = D.stream_max_rows;
-    {
-        ProfScope prof_(MOE_K_SCHEDULE, s);
-        const cudaError_t le = launch_pdl(use_pdl(D.T), schedule_kernel, dim3(1), dim3(512), 0, s, offsets, D.Etot,
-                                          D.variant, smax, tile_base, stream_list, n_stream, err);
-        if (le != cudaSuccess) return le;
-    }
-    return cudaGetLastError();
-}
 
 // Both tcgen05 GEMMs of the tile variant. xg: the gathered rows (bf16, or
 // fp16 for Q4G32); h: [rows, f] fp16 scratch.

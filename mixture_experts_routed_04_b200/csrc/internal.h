@@ -83,8 +83,10 @@ int num_sms();
 
 // Programmatic stream serialization (see griddep_wait) pays off only when the
 // layer's kernels are short: measured on B200, it saved ~2 us of a 106 us
-// single-token decode layer and cost ~10 us of a 490 us 4096-token layer. So
-// it is used for batches of at most kPdlMaxTokens tokens.
+// single-token decode layer and cost ~10 us of a 490 us 4096-token layer —
+// and as much when only the routing, permutation and schedule kernels take it
+// (471 -> 481 us; the 8192-token capped layer 109.7 -> 112.3 us). So it is
+// used for batches of at most kPdlMaxTokens tokens.
 constexpr int kPdlMaxTokens = 64;
 inline bool use_pdl(int64_t T) { return T <= kPdlMaxTokens; }
 
