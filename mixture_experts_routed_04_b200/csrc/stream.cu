@@ -310,6 +310,10 @@ __global__ void __launch_bounds__(THREADS, 1)
 }
 
 // h = swiglu(sum_ks part_g, sum_ks part_u) for the streaming experts' rows (ks > 1).
+// Work item = (streaming expert, 256 columns); each thread owns one column of
+// the expert's rows, so its 2*ks loads are independent and in flight together
+// (single-token decode: one row per expert, 9 experts x 6 items). The partials
+// are summed in slice order, so the result does not depend on the mapping.
 __global__ void __launch_bounds__(256) stream_reduce_kernel(const float* __restrict__ part, int ks, int64_t rows,
                                                             int f, const int32_t* __restrict__ offsets,
                                                             const int32_t* __restrict__ stream_list,
@@ -318,13 +322,16 @@ __global__ void __launch_bounds__(256) stream_reduce_kernel(const float* __restr
     griddep_wait();
     griddep_launch();
     const int n = __ldg(n_stream);
+    const int cpe = (f + 255) / 256;  // 256-column items per expert
     bool range_bad = false;
-    for (int i = blockIdx.x; i < n; i += gridDim.x) {
+    for (int w = blockIdx.x; w < n * cpe; w += gridDim.x) {
+        const int i = w / cpe;
+        const int col = (w - i * cpe) * 256 + int(threadIdx.x);
+        if (col >= f) continue;
         const int e = __ldg(stream_list + i);
         const int r0 = __ldg(offsets + e), nr = __ldg(offsets + e + 1) - r0;
-        for (int j = threadIdx.x; j < nr * f; j += blockDim.x) {
-            const int64_t row = r0 + j / f;
-            const int col = j % f;
+        for (int r = 0; r < nr; ++r) {
+            const int64_t row = int64_t(r0) + r;
             float g = 0.f, u = 0.f;
             for (int s = 0; s < ks; ++s) {
                 g += part[((int64_t(s) * 2 + 0) * rows + row) * f + col];
