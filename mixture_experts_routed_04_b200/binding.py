@@ -19,6 +19,7 @@ PKG = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(PKG, "libmoe_b200.so")
 
 MOE_OK = 0
+MOE_ERR_DEVICE = 6  # moe_get_error: the device error word is set
 STATUS = {0: "ok", 1: "invalid argument", 2: "workspace too small", 3: "unsupported configuration",
           4: "CUDA error", 5: "misaligned pointer", 6: "device error word set"}
 DEVERR_TIMEOUT, DEVERR_BOUNDS, DEVERR_RANGE = 0x1, 0x2, 0x4
@@ -227,7 +228,7 @@ def wait_selftest(err_ws, limit_ns, stream=None):
 def get_error(ws, stream=None) -> int:
     v = ctypes.c_uint32()
     st = lib().moe_get_error(_p(ws), ctypes.byref(v), _stream(stream))
-    if st not in (MOE_OK, 6):
+    if st not in (MOE_OK, MOE_ERR_DEVICE):
         check(st, "moe_get_error")
     return v.value
 
