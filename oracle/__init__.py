@@ -23,7 +23,7 @@ blocking, fusion or reordering beyond what the definition states. Sources:
 * "TensorFold PR #1607", "What this changes": served plans with "256 + shared"
   experts (an always-on shared expert).
 
-Readings taken where the pages are silent (each one is listed in the design doc):
+Readings taken where the pages are silent:
 top-k ties go to the lower expert index; the capacity is
 ``ceil(cf * T * k / E)`` with cf widened from float32; overflow is dropped in
 token order and the kept weights are NOT renormalised; the clamp bounds both
@@ -40,7 +40,7 @@ import math
 import numpy as np
 
 __all__ = [
-    "route", "capacity", "permute", "silu", "swiglu_clamped", "expert_ffn",
+    "route", "router_telemetry", "capacity", "permute", "silu", "swiglu_clamped", "expert_ffn",
     "dequant_q4g32", "combine", "forward", "token_outputs",
 ]
 
@@ -71,6 +71,58 @@ def route(logits: np.ndarray, k: int):
     ex = np.exp(sel - m)
     w = ex / ex.sum(axis=1, keepdims=True)
     return order.astype(np.int32), w
+
+
+# --------------------------------------------------------------------------- router telemetry
+
+WANT_MASS = 0.9  # "the smallest number of experts covering 90% of the probability mass"
+
+
+def router_telemetry(logits: np.ndarray, k: int, z_weight: float = 1e-3):
+    """Router telemetry and auxiliary losses of one batch, float64.
+
+    mini-AGI PR #3, ``requested()`` telemetry hunk, on the full softmax
+    ``probs`` of each token's logits and its top-k ``idx``:
+
+    * ``kept``: the top-k probability mass measured BEFORE the top-k weights
+      are renormalised (afterwards it is 1 by construction), averaged over the
+      tokens: mean_t sum_j probs[t, idx[t, j]].
+    * ``want_k``: per token, the smallest number of experts whose
+      probabilities sum to at least 90% of the mass (the largest ones first);
+      averaged over the tokens like ``kept``.
+    * ``balance``: ``(frac * probs.mean(0)).sum() * n`` with ``frac[e]`` the
+      share of tokens whose first choice ``idx[t, 0]`` is e and n = E.
+    * ``z``: ``logsumexp(logits, -1).pow(2).mean()``.
+    * ``aux`` = balance + z_weight * z (the hunk's default weight is 1e-3).
+
+    The page keeps exponential moving averages of ``1 - kept`` ("pressure")
+    and of ``want`` across calls; those running averages are the caller's
+    state, so the per-batch values are what is returned.
+
+    Returns a dict: per-token ``kept_tok`` [T], ``want_tok`` [T] (int), ``lse``
+    [T]; per-expert ``frac`` [E], ``prob_mean`` [E]; scalars ``kept``,
+    ``want_k``, ``balance``, ``z``, ``aux``.
+    """
+    lg = np.asarray(logits, dtype=np.float32)
+    T, E = lg.shape
+    idx, _ = route(lg, k)
+    x = lg.astype(np.float64)
+    mx = x.max(axis=1, keepdims=True)
+    ex = np.exp(x - mx)
+    lse = mx[:, 0] + np.log(ex.sum(axis=1))
+    probs = ex / ex.sum(axis=1, keepdims=True)
+    kept_tok = np.take_along_axis(probs, idx.astype(np.int64), axis=1).sum(axis=1)
+    srt = -np.sort(-probs, axis=1)  # largest first
+    cum = np.cumsum(srt, axis=1)
+    want_tok = (cum < WANT_MASS).sum(axis=1) + 1  # first m with cum[m-1] >= 0.9
+    want_tok = np.minimum(want_tok, E)
+    frac = np.bincount(idx[:, 0], minlength=E).astype(np.float64) / T
+    prob_mean = probs.mean(axis=0)
+    balance = float((frac * prob_mean).sum() * E)
+    z = float(np.mean(lse ** 2))
+    return {"kept_tok": kept_tok, "want_tok": want_tok.astype(np.int64), "lse": lse, "frac": frac,
+            "prob_mean": prob_mean, "kept": float(kept_tok.mean()), "want_k": float(want_tok.mean()),
+            "balance": balance, "z": z, "aux": balance + z_weight * z}
 
 
 # --------------------------------------------------------------------------- capacity

@@ -21,6 +21,25 @@ with open(oracle.__file__) as _fh:
 
 # name -> (text in the oracle, replacement)
 MUTATIONS = {
+    "telemetry: kept measured after renormalisation": (
+        "kept_tok = np.take_along_axis(probs, idx.astype(np.int64), axis=1).sum(axis=1)",
+        "kept_tok = np.take_along_axis(probs, idx.astype(np.int64), axis=1).sum(axis=1)\n"
+        "    kept_tok = kept_tok / kept_tok"),
+    "telemetry: want off by one": (
+        "want_tok = (cum < WANT_MASS).sum(axis=1) + 1",
+        "want_tok = (cum < WANT_MASS).sum(axis=1)"),
+    "telemetry: want at half the mass": (
+        'WANT_MASS = 0.9  #',
+        'WANT_MASS = 0.5  #'),
+    "telemetry: balance without the factor n": (
+        "balance = float((frac * prob_mean).sum() * E)",
+        "balance = float((frac * prob_mean).sum())"),
+    "telemetry: share of last choices instead of first": (
+        "frac = np.bincount(idx[:, 0], minlength=E)",
+        "frac = np.bincount(idx[:, -1], minlength=E)"),
+    "telemetry: logsumexp without the max": (
+        "lse = mx[:, 0] + np.log(ex.sum(axis=1))",
+        "lse = np.log(ex.sum(axis=1))"),
     "route: top-k of the full softmax, not renormalised": (
         "    m = sel[:, :1]\n    ex = np.exp(sel - m)\n    w = ex / ex.sum(axis=1, keepdims=True)\n",
         "    full = np.exp(lg.astype(np.float64) - lg.max(axis=1, keepdims=True).astype(np.float64))\n"

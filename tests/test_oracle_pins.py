@@ -78,6 +78,80 @@ def test_route_k1_and_k2_closed_forms():
     assert (a >= b).all()
 
 
+# --------------------------------------------------------------------------- router telemetry
+
+def test_router_telemetry_golden_cases():
+    for ln in _lines("router_telemetry_cases.txt"):
+        k, lg, kept, want, lse, bal = [p.split() for p in ln.split("|")]
+        logits = np.array([[float(v) for v in lg]], np.float32)
+        r = oracle.router_telemetry(logits, int(k[0]), z_weight=0.0)
+        np.testing.assert_allclose(r["kept"], float(kept[0]), rtol=0, atol=1e-12)
+        assert r["want_k"] == float(want[0]) and int(r["want_tok"][0]) == int(want[0]), ln
+        np.testing.assert_allclose(r["lse"][0], float(lse[0]), rtol=1e-14)
+        np.testing.assert_allclose(r["z"], float(lse[0]) ** 2, rtol=1e-13)
+        np.testing.assert_allclose(r["balance"], float(bal[0]), rtol=1e-12)
+        np.testing.assert_allclose(r["aux"], r["balance"], rtol=0, atol=0)
+
+
+def test_router_telemetry_want_by_brute_force():
+    """want = the size of the smallest set of experts of mass >= 0.9, over every subset."""
+    rng = np.random.default_rng(21)
+    for E in (2, 3, 5, 7):
+        lg = (rng.standard_normal((25, E)) * 2.5).astype(np.float32)
+        r = oracle.router_telemetry(lg, 1)
+        for t in range(lg.shape[0]):
+            ex = [math.exp(float(v)) for v in lg[t]]
+            p = [v / sum(ex) for v in ex]
+            best = min(len(s) for m in range(1, E + 1) for s in itertools.combinations(range(E), m)
+                       if sum(p[e] for e in s) >= 0.9)
+            assert int(r["want_tok"][t]) == best
+            np.testing.assert_allclose(r["kept_tok"][t], max(p), rtol=1e-13)
+
+
+def test_router_telemetry_loop_definitions():
+    """Every output from Python-float loops over the definitions (first choice, mean probability,
+    logsumexp), against the oracle's array code; kept == 1 when k == E."""
+    rng = np.random.default_rng(8)
+    T, E, k, zw = 40, 6, 2, 0.01
+    lg = (rng.standard_normal((T, E)) * 2).astype(np.float32)
+    r = oracle.router_telemetry(lg, k, z_weight=zw)
+    probs, lses, firsts, kept = [], [], [], []
+    for t in range(T):
+        vals = [float(v) for v in lg[t]]
+        s = sum(math.exp(v) for v in vals)
+        p = [math.exp(v) / s for v in vals]
+        probs.append(p)
+        lses.append(math.log(s))
+        top = sorted(range(E), key=lambda e: (-vals[e], e))
+        firsts.append(top[0])
+        kept.append(sum(p[e] for e in top[:k]))
+    frac = [firsts.count(e) / T for e in range(E)]
+    pm = [sum(probs[t][e] for t in range(T)) / T for e in range(E)]
+    bal = E * sum(frac[e] * pm[e] for e in range(E))
+    z = sum(v * v for v in lses) / T
+    np.testing.assert_allclose(r["frac"], frac, rtol=0, atol=0)
+    np.testing.assert_allclose(r["prob_mean"], pm, rtol=1e-12)
+    np.testing.assert_allclose(r["kept"], sum(kept) / T, rtol=1e-12)
+    np.testing.assert_allclose(r["balance"], bal, rtol=1e-12)
+    np.testing.assert_allclose(r["z"], z, rtol=1e-12)
+    np.testing.assert_allclose(r["aux"], bal + zw * z, rtol=1e-12)
+    np.testing.assert_allclose(oracle.router_telemetry(lg, E)["kept"], 1.0, rtol=1e-14)
+
+
+def test_router_telemetry_balance_extremes():
+    """balance = E when every token sends all its mass to one expert; about 1 when each expert
+    is the sole first choice of an equal share of tokens (the loss's minimum)."""
+    E = 16
+    lg = np.zeros((64, E), np.float32)
+    lg[:, 5] = 60.0
+    r = oracle.router_telemetry(lg, 2)
+    np.testing.assert_allclose(r["balance"], E, rtol=1e-12)
+    assert r["want_k"] == 1.0
+    lg2 = np.zeros((4 * E, E), np.float32)
+    lg2[np.arange(4 * E), np.arange(4 * E) % E] = 60.0
+    np.testing.assert_allclose(oracle.router_telemetry(lg2, 2)["balance"], 1.0, rtol=1e-12)
+
+
 # --------------------------------------------------------------------------- capacity
 
 def test_capacity_golden():
