@@ -42,6 +42,7 @@ import numpy as np
 __all__ = [
     "route", "router_telemetry", "capacity", "permute", "silu", "swiglu_clamped", "expert_ffn",
     "dequant_q4g32", "combine", "forward", "token_outputs",
+    "swiglu_clamped_backward", "expert_ffn_backward", "route_backward", "backward",
 ]
 
 
@@ -320,3 +321,110 @@ def token_outputs(tokens, x, idx, w, pair_row, experts, limit: float, shared=Non
             acc += expert_ffn(xt, *shared, limit)
         res.append(acc[0])
     return np.stack(res) if res else np.zeros((0, x.shape[1]))
+
+
+# --------------------------------------------------------------------------- backward
+
+def swiglu_clamped_backward(g, u, dh, limit: float):
+    """Gradients of h = silu(clamp(g)) * clamp(u) with respect to g and u, float64.
+
+    d silu(z)/dz = s(z) * (1 + z * (1 - s(z))), s the logistic sigmoid. The
+    clamp passes the gradient where -L <= v <= L and stops it outside (its
+    derivative there is 0); ``limit <= 0`` means no clamp.
+    """
+    g = np.asarray(g, dtype=np.float64)
+    u = np.asarray(u, dtype=np.float64)
+    dh = np.asarray(dh, dtype=np.float64)
+    if limit > 0:
+        gc, uc = np.clip(g, -limit, limit), np.clip(u, -limit, limit)
+        pass_g, pass_u = np.abs(g) <= limit, np.abs(u) <= limit
+    else:
+        gc, uc = g, u
+        pass_g = pass_u = np.ones(g.shape, bool)
+    sg = 1.0 / (1.0 + np.exp(-gc))
+    dg = dh * uc * sg * (1.0 + gc * (1.0 - sg)) * pass_g
+    du = dh * gc * sg * pass_u
+    return dg, du
+
+
+def expert_ffn_backward(x_rows, w_gate, w_up, w_down, limit: float, dy):
+    """Backward of ``expert_ffn`` for the rows of one expert, float64.
+
+    Given dy = dL/dy for y = swiglu(x Wg, x Wu) Wd: dh = dy Wd^T,
+    dWd = h^T dy, (dg, du) from ``swiglu_clamped_backward``, dx = dg Wg^T +
+    du Wu^T, dWg = x^T dg, dWu = x^T du. mini-AGI PR #3's tests/test_dispatch.py
+    checks that these expert-weight gradients are the same on every dispatch
+    path; this is their definition.
+
+    Returns (dx [n, d], dWg [d, f], dWu [d, f], dWd [f, d], y [n, d]), y being
+    the forward output (the routing-weight gradient needs it).
+    """
+    x_rows = np.asarray(x_rows, dtype=np.float64)
+    wg, wu, wd = (np.asarray(w, dtype=np.float64) for w in (w_gate, w_up, w_down))
+    dy = np.asarray(dy, dtype=np.float64)
+    g, u = x_rows @ wg, x_rows @ wu
+    h = swiglu_clamped(g, u, limit)
+    dh = dy @ wd.T
+    dg, du = swiglu_clamped_backward(g, u, dh, limit)
+    return dg @ wg.T + du @ wu.T, x_rows.T @ dg, x_rows.T @ du, h.T @ dy, h @ wd
+
+
+def route_backward(logits, k: int, d_w):
+    """Gradient of the routing weights' softmax over the k selected logits.
+
+    w_j = exp(l_j) / sum_i exp(l_i) over the selected; dl_j = w_j (dw_j -
+    sum_i w_i dw_i) for the selected experts, 0 for the others (the top-k
+    choice itself is piecewise constant). Returns dlogits [T, E] float64.
+    """
+    lg = np.asarray(logits, dtype=np.float32)
+    T, E = lg.shape
+    idx, w = route(lg, k)
+    d_w = np.asarray(d_w, dtype=np.float64).reshape(T, k)
+    dsel = w * (d_w - (w * d_w).sum(axis=1, keepdims=True))
+    out = np.zeros((T, E), np.float64)
+    np.put_along_axis(out, idx.astype(np.int64), dsel, axis=1)
+    return out
+
+
+def backward(x, logits, k: int, experts, limit: float, dout, capacity_factor: float = 0.0, shared=None):
+    """Gradients of the layer for an upstream gradient dout = dL/dout, float64.
+
+    out[t] = sum over kept j of w[t, j] * FFN_{idx[t, j]}(x[t]) (+ shared(x[t])).
+    So a kept pair's expert sees dy = w[t, j] * dout[t]; dw[t, j] =
+    <dout[t], FFN_{idx[t, j]}(x[t])> (0 for a dropped pair, whose weight is
+    not renormalised away); dx[t] sums its pairs' input gradients (and the
+    shared expert's, with dy = dout[t]); dlogits from ``route_backward``.
+
+    Returns a dict: dx [T, d], dw_gate/dw_up [E, d, f], dw_down [E, f, d],
+    d_topk_w [T, k], dlogits [T, E], and with a shared expert
+    dshared = (dWg, dWu, dWd).
+    """
+    x = np.asarray(x, dtype=np.float64)
+    dout = np.asarray(dout, dtype=np.float64)
+    T, d = x.shape
+    E = np.asarray(logits).shape[1]
+    idx, w = route(logits, k)
+    cap = capacity(T, k, E, capacity_factor)
+    perm = permute(idx, E, cap)
+    off, tok, sp = perm["offsets"], perm["sorted_token"], perm["sorted_pair"]
+    f = np.asarray(experts(0)[0]).shape[1] if E else 0
+    dx = np.zeros((T, d), np.float64)
+    dwg, dwu, dwd = np.zeros((E, d, f)), np.zeros((E, d, f)), np.zeros((E, f, d))
+    d_w = np.zeros(T * k, np.float64)
+    wf = w.reshape(-1)
+    for e in range(E):
+        a, b = int(off[e]), int(off[e + 1])
+        if b == a:
+            continue
+        rows, pairs = tok[a:b], sp[a:b]
+        dy = wf[pairs][:, None] * dout[rows]
+        dxr, dwg[e], dwu[e], dwd[e], y = expert_ffn_backward(x[rows], *experts(e), limit, dy)
+        np.add.at(dx, rows, dxr)
+        d_w[pairs] = (dout[rows] * y).sum(axis=1)
+    res = {"dx": dx, "dw_gate": dwg, "dw_up": dwu, "dw_down": dwd, "d_topk_w": d_w.reshape(T, k),
+           "dlogits": route_backward(logits, k, d_w), "idx": idx, "w": w, **perm}
+    if shared is not None:
+        dxs, sg, su, sd, _ = expert_ffn_backward(x, *shared, limit, dout)
+        res["dx"] = dx + dxs
+        res["dshared"] = (sg, su, sd)
+    return res

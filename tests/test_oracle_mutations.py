@@ -21,6 +21,27 @@ with open(oracle.__file__) as _fh:
 
 # name -> (text in the oracle, replacement)
 MUTATIONS = {
+    "backward: silu derivative without its second term": (
+        "dg = dh * uc * sg * (1.0 + gc * (1.0 - sg)) * pass_g",
+        "dg = dh * uc * sg * pass_g"),
+    "backward: clamp passes the gradient outside its range": (
+        "pass_g, pass_u = np.abs(g) <= limit, np.abs(u) <= limit",
+        "pass_g = pass_u = np.ones(g.shape, bool)"),
+    "backward: h recomputed without the clamp": (
+        "    h = swiglu_clamped(g, u, limit)\n    dh = dy @ wd.T",
+        "    h = swiglu_clamped(g, u, 0.0)\n    dh = dy @ wd.T"),
+    "backward: down-projection gradient transposed operands": (
+        "x_rows.T @ du, h.T @ dy, h @ wd",
+        "x_rows.T @ du, dy.T @ h, h @ wd"),
+    "backward: input gradient without the up branch": (
+        "return dg @ wg.T + du @ wu.T, x_rows.T @ dg",
+        "return dg @ wg.T, x_rows.T @ dg"),
+    "backward: expert sees dout without the gate weight": (
+        "dy = wf[pairs][:, None] * dout[rows]",
+        "dy = dout[rows]"),
+    "backward: routing gradient without the weighted mean": (
+        "dsel = w * (d_w - (w * d_w).sum(axis=1, keepdims=True))",
+        "dsel = w * d_w"),
     "telemetry: kept measured after renormalisation": (
         "kept_tok = np.take_along_axis(probs, idx.astype(np.int64), axis=1).sum(axis=1)",
         "kept_tok = np.take_along_axis(probs, idx.astype(np.int64), axis=1).sum(axis=1)\n"

@@ -403,3 +403,121 @@ def test_q4g32_round_trip_and_error_bound():
     err = np.abs(oracle.dequant_q4g32(packed, s) - w)
     step = np.repeat(s.astype(np.float64), 32, axis=0)
     assert (err <= step * (0.5 + 7 * 2.0 ** -10) + 1e-12).all()
+
+
+# --------------------------------------------------------------------------- backward
+
+def _tiny_layer(seed, T=7, d=8, f=6, E=4, k=2, wscale=0.5):
+    rng = np.random.default_rng(seed)
+    x = rng.standard_normal((T, d))
+    lg = (rng.standard_normal((T, E)) * 2).astype(np.float32)
+    Ws = [tuple(rng.standard_normal(s) * wscale for s in ((d, f), (d, f), (f, d))) for _ in range(E)]
+    dout = rng.standard_normal((T, d))
+    return x, lg, Ws, dout
+
+
+def _loss(x, lg, Ws, dout, k, limit, cf=0.0, shared=None):
+    out, _ = oracle.forward(x, lg, k, lambda e: Ws[e], limit, cf, shared=shared)
+    return float((out * dout).sum())
+
+
+@pytest.mark.parametrize("limit,cf,shared", [(7.0, 0.0, False), (1.5, 0.0, False), (7.0, 0.6, False),
+                                             (1.5, 0.0, True)])
+def test_backward_against_central_differences(limit, cf, shared):
+    """Every gradient of L = <dout, out> against central differences of the forward oracle
+    (fp64, step 1e-6), with the clamp firing (limit 1.5), a capacity drop and a shared expert."""
+    x, lg, Ws, dout = _tiny_layer(4)
+    k, E = 2, len(Ws)
+    sh = tuple(np.random.default_rng(9).standard_normal(s) * 0.5 for s in ((8, 6), (8, 6), (6, 8))) \
+        if shared else None
+    g = oracle.backward(x, lg, k, lambda e: Ws[e], limit, dout, cf, shared=sh)
+    eps = 1e-6
+
+    def fd(mut):
+        plus, minus = mut(eps), mut(-eps)
+        return (plus - minus) / (2 * eps)
+
+    for t, c in [(0, 0), (3, 5), (6, 7)]:
+        def mx(h, t=t, c=c):
+            xx = x.copy()
+            xx[t, c] += h
+            return _loss(xx, lg, Ws, dout, k, limit, cf, sh)
+        np.testing.assert_allclose(g["dx"][t, c], fd(mx), rtol=1e-6, atol=1e-8)
+    for e in range(E):
+        for wi, key, (i, j) in ((0, "dw_gate", (1, 2)), (1, "dw_up", (7, 0)), (2, "dw_down", (5, 3))):
+            def mw(h, e=e, wi=wi, i=i, j=j):
+                W2 = [list(w) for w in Ws]
+                W2[e][wi] = W2[e][wi].copy()
+                W2[e][wi][i, j] += h
+                return _loss(x, lg, [tuple(w) for w in W2], dout, k, limit, cf, sh)
+            np.testing.assert_allclose(g[key][e, i, j], fd(mw), rtol=1e-6, atol=1e-8)
+    for t in range(0, 7, 2):
+        for ee in range(E):
+            def ml(h, t=t, ee=ee):
+                l2 = lg.astype(np.float64).copy()
+                l2[t, ee] += h
+                # the router reads float32 logits: perturb in float64 through the weights only
+                return _loss_logits64(x, l2, Ws, dout, k, limit, cf, sh)
+            np.testing.assert_allclose(g["dlogits"][t, ee], fd(ml), rtol=1e-5, atol=1e-7)
+    if sh is not None:
+        def msh(h):
+            s2 = (sh[0].copy(), sh[1], sh[2])
+            s2[0][2, 3] += h
+            return _loss(x, lg, Ws, dout, k, limit, cf, s2)
+        np.testing.assert_allclose(g["dshared"][0][2, 3], fd(msh), rtol=1e-6, atol=1e-8)
+
+
+def _loss_logits64(x, lg64, Ws, dout, k, limit, cf, sh):
+    """The layer with the routing weights taken from float64 logits (same top-k choice): the
+    softmax over the selected, as the forward defines it, without the float32 input rounding."""
+    lg32 = lg64.astype(np.float32)
+    idx, _ = oracle.route(lg32, k)
+    sel = np.take_along_axis(lg64, idx.astype(np.int64), axis=1)
+    w = np.exp(sel - sel[:, :1])
+    w /= w.sum(1, keepdims=True)
+    T, E = lg64.shape
+    cap = oracle.capacity(T, k, E, cf)
+    perm = oracle.permute(idx, E, cap)
+    y = np.zeros((int(perm["offsets"][-1]), x.shape[1]))
+    for e in range(E):
+        a, b = int(perm["offsets"][e]), int(perm["offsets"][e + 1])
+        if b > a:
+            y[a:b] = oracle.expert_ffn(x[perm["sorted_token"][a:b]], *Ws[e], limit)
+    out = oracle.combine(y, perm["pair_row"], w, T, k)
+    if sh is not None:
+        out = out + oracle.expert_ffn(x, *sh, limit)
+    return float((out * dout).sum())
+
+
+def test_backward_dense_case_against_autograd():
+    """E = 1, k = 1: the layer is a dense clamped-SwiGLU FFN; torch autograd (float64) of that
+    FFN written out separately gives the same dx and weight gradients."""
+    import torch
+    rng = np.random.default_rng(2)
+    T, d, f, L = 9, 12, 10, 2.0
+    x = rng.standard_normal((T, d))
+    W = tuple(rng.standard_normal(s) for s in ((d, f), (d, f), (f, d)))
+    dout = rng.standard_normal((T, d))
+    g = oracle.backward(x, np.zeros((T, 1), np.float32), 1, lambda e: W, L, dout)
+    xt = torch.tensor(x, requires_grad=True)
+    Wt = [torch.tensor(w, requires_grad=True) for w in W]
+    gg = torch.clamp(xt @ Wt[0], -L, L)
+    uu = torch.clamp(xt @ Wt[1], -L, L)
+    out = (torch.nn.functional.silu(gg) * uu) @ Wt[2]
+    (out * torch.tensor(dout)).sum().backward()
+    np.testing.assert_allclose(g["dx"], xt.grad.numpy(), rtol=1e-12, atol=1e-12)
+    for key, t in zip(("dw_gate", "dw_up", "dw_down"), Wt):
+        np.testing.assert_allclose(g[key][0], t.grad.numpy(), rtol=1e-12, atol=1e-12)
+    assert np.abs(g["dlogits"]).max() == 0.0  # one expert, weight 1: no routing gradient
+
+
+def test_route_backward_closed_form_k2():
+    """k = 2: w0 = sigmoid(l0 - l1), so dl0 = w0 w1 (dw0 - dw1) = -dl1."""
+    lg = np.array([[0.3, 2.0, -1.0, 1.1]], np.float32)
+    dw = np.array([[0.7, -0.4]])
+    dl = oracle.route_backward(lg, 2, dw)
+    a, c = 2.0, float(np.float32(1.1))
+    w0 = 1.0 / (1.0 + math.exp(c - a))
+    np.testing.assert_allclose(dl[0, 1], w0 * (1 - w0) * (0.7 + 0.4), rtol=1e-12)
+    np.testing.assert_allclose(dl[0, 3], -dl[0, 1], rtol=1e-12)
+    assert dl[0, 0] == 0.0 and dl[0, 2] == 0.0
