@@ -19,7 +19,10 @@ number through the host-buffer entry points (copies of every step's inputs in
 and output back inside the timed region; a pipelined loop over three streams
 with moe_forward_host_async, and one synchronous moe_forward_host per step),
 SM clocks sampled through NVML during the timed region, and the fp64 CPU
-oracle's throughput on this host as a baseline.
+oracle's throughput on this host as a baseline. At N = 1 the line also carries
+`per_config`: the other stated workloads (capped, decode T=1/8/32, quantised)
+measured the same way in the same run, each with its dominant kernel's roofline
+and its own clock samples.
 
 --impl reference times that oracle alone (on the host cores, rank 0 only) on
 this arm's config, a bounded sample of the workload per step.
@@ -58,6 +61,8 @@ def parse():
     ap.add_argument("--impl", default="own", choices=["own", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-per-config", action="store_true",
+                    help="skip the other stated workloads (capped, decode1/8/32, quant) in the JSON line")
     ap.add_argument("--tokens", type=int, default=0, help="override T of the workload (profiling small cases)")
     ap.add_argument("--profile-calls", type=int, default=0,
                     help="only run this many moe_forward calls and exit (for ncu: no timing, no other kernels)")
@@ -65,6 +70,8 @@ def parse():
                     help="SMs per tcgen05 tile (moe_params.tile_ctas); auto = the library's choice")
     ap.add_argument("--sweep-threshold", action="store_true",
                     help="time moe_forward for each stream_max_rows and print one JSON line")
+    ap.add_argument("--variant-table", action="store_true",
+                    help="time tiles against streaming on layers of exact rows per expert; one JSON line")
     return ap.parse_args()
 
 
@@ -166,6 +173,54 @@ def aggregate_tokens_per_s(tokens_per_rank, world, max_ms_per_step):
     """Whole-job throughput: every rank processes tokens_per_rank per step; the step takes the
     slowest rank's time."""
     return tokens_per_rank * world / (max_ms_per_step / 1e3)
+
+
+# --------------------------------------------------------------------------- roofline of the dominant kernel
+
+ONE_SM_SRC = ["gemm_tc.cu", "gemm_tc.cuh", "common.cuh"]
+TWO_SM_SRC = ["gemm_pair.cu", "gemm_tc.cuh", "common.cuh"]
+STREAM_SRC = ["stream.cu", "common.cuh"]
+
+
+def dominant_roofline(prof, wl, K, ms, pk, pk_src, pair, down_f16, cfg_name):
+    """Roofline object of the expert GEMM with the largest measured share of the step.
+
+    achieved = the kernel's algorithmic work per launch (FLOPs when the workload's intensity is
+    at or above the measured ridge, else bytes: touched weights + x) / its mean launch time
+    (library CUDA events); traffic = DRAM bytes per launch from the committed ncu table while
+    the kernel source is unchanged; traffic_over_algorithmic = traffic / those algorithmic bytes
+    (weights + x, the scope table's count: the gathered rows, h and y_rows are not in it)."""
+    ridge = pk["bf16_tflops"] * 1e12 / (pk["hbm_gbs"] * 1e9)
+    tensor_bound = wl["flops"] / wl["bytes"] >= ridge
+    names = {"tc_gateup": ("grouped_gemm_pair_kernel<0> (tcgen05 SM pairs, gate/up + clamped SwiGLU)", "gateup",
+                           TWO_SM_SRC) if pair else
+             ("grouped_gemm_kernel<0> (tcgen05 gate/up + clamped SwiGLU)", "gateup", ONE_SM_SRC),
+             "tc_down": ("grouped_gemm_pair_kernel<1> (tcgen05 SM pairs, down + gate scale)", "down", TWO_SM_SRC)
+             if pair and down_f16 else ("grouped_gemm_kernel<1> (tcgen05 down + gate scale)", "down", ONE_SM_SRC),
+             "stream_gateup": ("stream_kernel<0> (few-rows gate/up)", "gateup", STREAM_SRC),
+             "stream_down": ("stream_kernel<1> (few-rows down)", "down", STREAM_SRC)}
+    kern = max(names, key=lambda k: prof.get(k, (0.0, 0))[0])
+    kms, kn = prof.get(kern, (0.0, 0))
+    k_avg = kms / kn if kn else float("nan")
+    label, part, src = names[kern]
+    alg_bytes = wl["bytes_" + part]
+    if tensor_bound:
+        work = wl["flops_" + part]
+        achieved = work / (k_avg / 1e3) / 1e12
+        peak = pk["bf16_tflops"]
+        roof = {"kernel": label, "bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+                "frac": achieved / peak, "peak_source": f"{pk_src} bf16_tflops (burst)"}
+    else:
+        work = alg_bytes
+        achieved = work / (k_avg / 1e3) / 1e9
+        peak = pk["hbm_gbs"]
+        roof = {"kernel": label, "bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
+                "frac": achieved / peak, "peak_source": f"{pk_src} hbm_gbs"}
+    traffic = committed_traffic(kern, src, cfg_name)
+    roof.update({"avg_launch_ms": k_avg, "algorithmic_per_launch": work, "share_of_step": kms / K / ms,
+                 "algorithmic_bytes_per_launch": alg_bytes, "traffic": traffic,
+                 "traffic_over_algorithmic": traffic / alg_bytes if traffic else None})
+    return roof
 
 
 # --------------------------------------------------------------------------- clocks
@@ -297,6 +352,99 @@ def reference_arm(args, cfg):
             "e2e": {"value": tps, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
     return 0
+
+
+# --------------------------------------------------------------------------- the other stated workloads
+
+PER_CONFIG = ("capped", "decode1", "decode8", "decode32", "quant")
+
+
+def upload_routed(cfg, b, torch):
+    """Device inputs with every routed expert's weights (others NaN, never read): the routing
+    is the library's own (moe_route on the device), so only the experts it picks are drawn."""
+    from synth.device import upload
+    lg = torch.from_numpy(synth.logits(cfg)).cuda()
+    p = b.params_for(cfg)
+    idx = torch.empty(cfg.T, cfg.k, dtype=torch.int32, device="cuda")
+    w = torch.empty(cfg.T, cfg.k, dtype=torch.float32, device="cuda")
+    b.route(p, lg, idx, w, b.workspace(p, b.WS_ROUTE))
+    routed = sorted(set(idx.cpu().numpy().reshape(-1).tolist()))
+    del lg, idx, w
+    return upload(cfg, "cuda", experts=routed if len(routed) < cfg.E else None)
+
+
+def measure_workload(cfg, args, b, torch, flush, pk, pk_src, steps):
+    """One stated workload on this GPU: moe_forward as a CUDA-graph replay with L2 flushed
+    between steps (CUDA events on the launching stream), the library's per-kernel events over
+    the same number of steps, the dominant kernel's roofline and the SM clocks sampled while
+    the timed steps ran."""
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    d = upload_routed(cfg, b, torch)
+    f16 = cfg.weight_format == "bf16"
+    wd = b.prepare_down_f16(d["w_down"]) if f16 else d["w_down"]
+    sh = None
+    if cfg.has_shared:
+        sh = (d["shared_gate"], d["shared_up"], b.prepare_down_f16(d["shared_down"]))
+    p = b.params_for(cfg, down_dtype=b.DOWN_F16 if f16 else b.DOWN_BF16, tile_ctas=TILE_ARG[args.tile])
+    W = b.weights(d["w_gate"], d["w_up"], wd, d.get("s_gate"), d.get("s_up"), d.get("s_down"), shared=sh)
+    ws = b.workspace(p, b.WS_FORWARD)
+    out = torch.empty(cfg.T, cfg.d, dtype=torch.float32, device="cuda")
+    counts = torch.empty(cfg.E + int(cfg.has_shared), dtype=torch.int32, device="cuda")
+    stream = torch.cuda.current_stream()
+
+    def step():
+        b.forward(p, d["x"], d["logits"], W, out, ws)
+
+    b.forward(p, d["x"], d["logits"], W, out, ws, counts_out=counts)
+    cap = b.capacity(p)
+    kept = counts[: cfg.E].cpu().numpy()
+    kept = np.minimum(kept, cap) if cap is not None else kept
+    P, touched = int(kept.sum()), int((kept > 0).sum())
+    wl = workload_numbers(cfg, P, touched)
+    for _ in range(3):
+        flush()
+        step()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        step()
+    for _ in range(3):
+        flush()
+        graph.replay()
+    torch.cuda.synchronize()
+    s_ev = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
+    e_ev = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
+    with ClockSampler(local) as clocks:
+        for i in range(steps):
+            flush()
+            s_ev[i].record(stream)
+            graph.replay()
+            e_ev[i].record(stream)
+        torch.cuda.synchronize()
+    ms = sum(a.elapsed_time(z) for a, z in zip(s_ev, e_ev)) / steps
+    b.profile_collect()
+    b.profile_enable(True)
+    for _ in range(steps):
+        flush()
+        step()
+    torch.cuda.synchronize()
+    prof = b.profile_collect()
+    b.profile_enable(False)
+    if b.get_error(ws):
+        raise RuntimeError(f"device error word set ({cfg.name})")
+    roof = dominant_roofline(prof, wl, steps, ms, pk, pk_src, b.tile_ctas(p) == b.TILE_PAIR, f16, cfg.name)
+    tflops = wl["flops"] / (ms / 1e3) / 1e12
+    gbs = wl["bytes"] / (ms / 1e3) / 1e9
+    entry = {"workload": workload_name(cfg), "ms_per_step": ms, "tokens_per_s": cfg.T / (ms / 1e3),
+             "routed_rows": P, "touched_experts": touched,
+             "tflops": tflops, "tensor_frac_of_peak": tflops / pk["bf16_tflops"],
+             "gbs": gbs, "hbm_frac_of_peak": gbs / pk["hbm_gbs"], "bound": roof["bound"],
+             "layer_frac": gbs / pk["hbm_gbs"] if roof["bound"] == "hbm" else tflops / pk["bf16_tflops"],
+             "roofline": roof, "kernels_ms_per_step": {k: v[0] / steps for k, v in prof.items() if v[1]},
+             "steps": steps, "step_launch": "CUDA graph replay of one moe_forward call, L2 flushed between steps",
+             "clocks": clocks.summary()}
+    del graph, d, W, ws, out, wd, sh
+    torch.cuda.empty_cache()
+    return entry
 
 
 # --------------------------------------------------------------------------- own arm
@@ -488,37 +636,7 @@ def own_arm(args, cfg):
                         "mode": "one moe_forward_host call per step (L2 flushed between steps)"}}
 
     pk, pk_src = peaks()
-    # Bound: the workload's arithmetic intensity against the measured ridge point.
-    ridge = pk["bf16_tflops"] * 1e12 / (pk["hbm_gbs"] * 1e9)
-    tensor_bound = wl["flops"] / wl["bytes"] >= ridge
-    # Dominant kernel: the largest measured share of the step among the expert GEMMs.
-    one_sm = ["gemm_tc.cu", "gemm_tc.cuh", "common.cuh"]
-    two_sm = ["gemm_pair.cu", "gemm_tc.cuh", "common.cuh"]
-    names = {"tc_gateup": ("grouped_gemm_pair_kernel<0> (tcgen05 SM pairs, gate/up + clamped SwiGLU)", "gateup",
-                           two_sm) if pair else
-             ("grouped_gemm_kernel<0> (tcgen05 gate/up + clamped SwiGLU)", "gateup", one_sm),
-             "tc_down": ("grouped_gemm_pair_kernel<1> (tcgen05 SM pairs, down + gate scale)", "down", two_sm)
-             if pair and down_f16 else ("grouped_gemm_kernel<1> (tcgen05 down + gate scale)", "down", one_sm),
-             "stream_gateup": ("stream_kernel<0> (few-rows gate/up)", "gateup", ["stream.cu", "common.cuh"]),
-             "stream_down": ("stream_kernel<1> (few-rows down)", "down", ["stream.cu", "common.cuh"])}
-    kern = max(names, key=lambda k: prof.get(k, (0.0, 0))[0])
-    kms, kn = prof.get(kern, (0.0, 0))
-    k_avg = kms / kn if kn else float("nan")
-    label, part, src = names[kern]
-    if tensor_bound:
-        work = wl["flops_" + part]
-        achieved = work / (k_avg / 1e3) / 1e12
-        peak = pk["bf16_tflops"]
-        roof = {"kernel": label, "bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
-                "frac": achieved / peak, "peak_source": f"{pk_src} bf16_tflops (burst)"}
-    else:
-        work = wl["bytes_" + part]
-        achieved = work / (k_avg / 1e3) / 1e9
-        peak = pk["hbm_gbs"]
-        roof = {"kernel": label, "bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
-                "frac": achieved / peak, "peak_source": f"{pk_src} hbm_gbs"}
-    roof.update({"avg_launch_ms": k_avg, "algorithmic_per_launch": work, "share_of_step": kms / K / ms,
-                 "traffic": committed_traffic(kern, src, cfg.name)})
+    roof = dominant_roofline(prof, wl, K, ms, pk, pk_src, pair, down_f16, cfg.name)
 
     line = None
     if rank == 0:
@@ -542,6 +660,17 @@ def own_arm(args, cfg):
                 "tile_ctas": b.tile_ctas(p),
                 "w_down_prep_ms": prep_ms, "ms_per_step_w_down_bf16": ms_down_bf16,
                 "clocks": clocks.summary(), "e2e": e2e}
+    if rank == 0 and world == 1 and not args.no_per_config:
+        # the other stated workloads, measured in the same run (graph replay, L2 flushed);
+        # one GPU only, so that no rank waits at a barrier meanwhile
+        del graph
+        torch.cuda.empty_cache()
+        pc = {}
+        for name in PER_CONFIG:
+            if name != cfg.name:
+                pc[name] = measure_workload(synth.CONFIGS[name], args, b, torch, flush, pk, pk_src,
+                                            max(3, min(args.steps, 20)))
+        line["per_config"] = pc
     if dist:
         dist.barrier()
         dist.destroy_process_group()
@@ -618,6 +747,61 @@ def sweep_threshold(args, cfg):
     return 0
 
 
+def variant_table_sweep(args):
+    """The measured table behind the library's variant choice: moe_forward time (graph replay,
+    L2 flushed) with every expert on the tcgen05 tiles against every routed expert on the
+    weight-streaming kernels, on decode-shaped layers (d=4096, f=1536, E=256, top-8, shared
+    expert) whose routing gives `touched` experts exactly `rows` rows each. One JSON line."""
+    import torch
+    from mixture_experts_routed_04_b200 import binding as b
+    from synth.device import upload
+    touched_list = (8, 12, 16, 20, 24, 32, 48)
+    rows_list = (1, 2, 4, 8, 16)
+    base = synth.LayerConfig("vt", T=48, d=4096, f=1536, E=256, k=8, bias="balanced", touched=48,
+                             has_shared=True, f_shared=1536)
+    d = upload(base, "cuda", experts=range(max(touched_list)))
+    wd = b.prepare_down_f16(d["w_down"])
+    sh = (d["shared_gate"], d["shared_up"], b.prepare_down_f16(d["shared_down"]))
+    W = b.weights(d["w_gate"], d["w_up"], wd, shared=sh)
+    flush = L2Flush(torch)
+    res = []
+    for n in touched_list:
+        for r in rows_list:
+            if (r * n) % base.k:
+                continue
+            cfg = base.replace(T=r * n // base.k, touched=n)
+            x = torch.from_numpy(synth.x_bits(cfg).view(np.int16)).cuda().view(torch.bfloat16)
+            lg = torch.from_numpy(synth.logits(cfg)).cuda()
+            out = torch.empty(cfg.T, cfg.d, dtype=torch.float32, device="cuda")
+            row = {"touched": n, "rows": r, "T": cfg.T, "gateup_tiles": (n + 1) * ((cfg.f + 127) // 128)}
+            for name, v in (("tiles", b.VARIANT_TENSOR), ("stream", b.VARIANT_STREAM)):
+                p = b.params_for(cfg, variant=v, down_dtype=b.DOWN_F16)
+                ws = b.workspace(p, b.WS_FORWARD)
+                for _ in range(3):
+                    b.forward(p, x, lg, W, out, ws)
+                g = torch.cuda.CUDAGraph()
+                with torch.cuda.graph(g):
+                    b.forward(p, x, lg, W, out, ws)
+                tot, k = 0.0, max(args.steps, 5)
+                for i in range(k + 3):
+                    flush()
+                    s0, s1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                    s0.record()
+                    g.replay()
+                    s1.record()
+                    s1.synchronize()
+                    if i >= 3:
+                        tot += s0.elapsed_time(s1)
+                if b.get_error(ws):
+                    raise RuntimeError("device error word set")
+                row[name + "_us"] = 1e3 * tot / k
+                del g, ws
+            res.append(row)
+    print(json.dumps({"variant_table": res, "sms": torch.cuda.get_device_properties(0).multi_processor_count,
+                      "steps": max(args.steps, 5)}))
+    return 0
+
+
 def main():
     args = parse()
     cfg = synth.CONFIGS[args.config]
@@ -629,6 +813,8 @@ def main():
         return profile_calls(args, cfg)
     if args.sweep_threshold:
         return sweep_threshold(args, cfg)
+    if args.variant_table:
+        return variant_table_sweep(args)
     return own_arm(args, cfg)
 
 

@@ -104,6 +104,8 @@ typedef struct CUstream_st* moe_stream_t; /* same object as cudaStream_t */
 #define MOE_WS_COMBINE      3
 #define MOE_WS_FORWARD      4
 #define MOE_WS_FORWARD_HOST 5
+#define MOE_WS_ROUTE_STATS  6
+#define MOE_WS_BACKWARD     7
 
 typedef struct moe_params {
     int32_t T;               /* tokens in this call; 0 = empty batch: every call returns MOE_OK
@@ -197,6 +199,33 @@ MOE_API int moe_route(const moe_params* p, const float* logits, int32_t* topk_id
               void* ws, size_t ws_bytes, moe_stream_t stream);
 
 /*
+ * moe_route_stats — moe_route plus the router's telemetry, in the same kernel.
+ *   "mini-AGI PR #3" requested(), telemetry hunk, on the full softmax p of
+ *   each token's logits (p[t, e] = exp(l - lse)):
+ *   stats[0] kept     mean over tokens of the top-k mass sum_j p[t, idx[t, j]],
+ *                     measured before the weights are renormalised
+ *   stats[1] want_k   mean over tokens of the fewest experts, largest p first
+ *                     (ties to the lower index), whose p sum to at least 0.9
+ *   stats[2] balance  E * sum_e frac[e] * mean_t p[t, e], frac[e] = share of
+ *                     tokens whose first choice idx[t, 0] is e
+ *   stats[3] z        mean over tokens of logsumexp(logits[t])^2
+ *   stats[4] aux      balance + z_weight * z (the page's default weight: 1e-3)
+ *   The page's running averages across calls (pressure = EMA of 1 - kept,
+ *   want_k = EMA of want) are the caller's state; these are per-batch values.
+ * topk_idx, topk_w  as moe_route (bit-identical to it).
+ * stats         device fp32 [5] (required).
+ * kept_tok      device fp32 [T] per-token top-k mass, or NULL.
+ * want_tok      device int32 [T] per-token count, or NULL.
+ * expert_stats  device fp32 [2, E]: frac, then mean p per expert; or NULL.
+ * ws: MOE_WS_ROUTE_STATS bytes (per-block partial sums). Deterministic: fixed
+ * summation orders (fp32 within a block of tokens, fp64 across blocks). With
+ * T = 0 nothing is launched and stats is not written.
+ */
+MOE_API int moe_route_stats(const moe_params* p, const float* logits, int32_t* topk_idx, float* topk_w,
+              float z_weight, float* stats, float* kept_tok, int32_t* want_tok, float* expert_stats,
+              void* ws, size_t ws_bytes, moe_stream_t stream);
+
+/*
  * moe_permute — S2/S3: histogram, prefix offsets, scatter, capacity drop.
  *   "mini-AGI PR #3" requested(): pairs sorted by expert, bincount, the keep
  *   mask over each expert's pairs, counts clamped to the limit.
@@ -231,10 +260,12 @@ MOE_API int moe_permute(const moe_params* p, const int32_t* topk_idx, int32_t* c
  * (256 KiB) stays resident on every GPU that loads the library until exit.
  * err_word  device uint32, OR-ed with MOE_DEVERR_BOUNDS for out-of-range ids
  *           (the caller zeroes it; it is not cleared here).
- * Returns MOE_ERR_INVALID_ARG for parameters moe_workspace_size rejects and
- * for null pointers. The first call on a device looks up the array's device
- * address (a CUDA runtime query, no allocation): make that first call before
- * any stream capture. Every call uses the same array, so calls whose work may
+ * Returns the status moe_permute returns for the same parameters (one shared
+ * check), and MOE_ERR_INVALID_ARG for null pointers. The first call on a
+ * device looks up the array's device address (a CUDA runtime query, no
+ * allocation) and keeps it for the life of the process: make that first call
+ * before any stream capture, and do not use this entry point across a
+ * cudaDeviceReset (the kept address would be stale). Every call uses the same array, so calls whose work may
  * overlap on the GPU (other streams, other host threads) race: issue them on
  * one stream. Nothing here calls an allocator.
  */
@@ -373,11 +404,64 @@ MOE_API int moe_wait_selftest(void* err_ws, uint64_t limit_ns, moe_stream_t stre
 #define MOE_K_COMBINE       11  /* S7 gate-weighted combine */
 #define MOE_K_CONVERT       12  /* load-time bf16 -> fp16 weight copy (not a layer step) */
 #define MOE_K_FRONT         13  /* S1-S3 + schedule fused, moe_forward with T <= 64 */
-#define MOE_K_COUNT         14
+#define MOE_K_ROUTE_STATS   14  /* router telemetry: the final sum over blocks (moe_route_stats) */
+#define MOE_K_BWD_GEMM      15  /* backward tcgen05 GEMMs (moe_expert_ffn_backward) */
+#define MOE_K_BWD_SMALL     16  /* backward schedule, gathers, transpose, reductions */
+#define MOE_K_COUNT         17
 
 /*
- * Number of kernel launches one call of `which` (MOE_WS_ROUTE .. MOE_WS_FORWARD_HOST,
- * naming moe_route .. moe_forward_host) makes with these params, into *n (host).
+ * Gradients written by moe_expert_ffn_backward (device pointers, fp32, row-major).
+ *   dx           [T, d]      required
+ *   dw_gate      [E, d, f]   required (experts without rows get zeros)
+ *   dw_up        [E, d, f]   required
+ *   dw_down      [E, f, d]   required
+ *   d_topk_w     [T, k]      required: dL / d topk_w (0 for a dropped pair)
+ *   dlogits      [T, E]      or NULL: through the softmax over the k selected
+ *                            logits (0 off the selected experts); needs topk_idx
+ *   dshared_*    [d, f], [d, f], [f, d] with has_shared, else NULL
+ */
+typedef struct moe_grads {
+    float* dx;
+    float* dw_gate;
+    float* dw_up;
+    float* dw_down;
+    float* d_topk_w;
+    float* dlogits;
+    float* dshared_gate;
+    float* dshared_up;
+    float* dshared_down;
+} moe_grads;
+
+/*
+ * moe_expert_ffn_backward — gradients of the layer (S5-S7 and the routing
+ * weights) for an upstream gradient dout = dL/d out.
+ *   "mini-AGI PR #3" tests/test_dispatch.py: the layer trains through this
+ *   path and the expert weights (w1, w3, w2 = gate, up, down) get the same
+ *   gradients on every dispatch path. With y = swiglu(x Wg, x Wu) Wd and
+ *   out[t] = sum_j w[t,j] y[t,j] (+ shared): a kept pair's expert sees
+ *   dy = w dout[t]; dh = dy Wd^T; dg, du from the clamped SwiGLU (the clamp
+ *   passes the gradient where -L <= v <= L); dx = sum over the token's pairs
+ *   of dg Wg^T + du Wu^T; dWd = h^T dy, dWg = x^T dg, dWu = x^T du over each
+ *   expert's rows; d w[t,j] = <dout[t], y[t,j]>; dlogits_j = w_j (dw_j -
+ *   sum_i w_i dw_i).
+ * Inputs are the forward's: x bf16 [T, d]; topk_idx, topk_w (moe_route);
+ * offsets, sorted_token, sorted_pair, pair_row (moe_permute); weights bf16 as
+ * for moe_forward (W_down bf16: down_dtype MOE_DOWN_BF16; Q4G32 is not
+ * supported); dout fp32 [T, d]. g: see moe_grads.
+ * Arithmetic: bf16 operands, fp32 accumulation on the tcgen05 tensor cores;
+ * g and u are recomputed (fp32) and h, dg, du rounded to bf16 once.
+ * ws: MOE_WS_BACKWARD bytes. Returns MOE_ERR_UNSUPPORTED for Q4G32 weights or
+ * fp16 W_down. Deterministic (no atomics decide a sum).
+ */
+MOE_API int moe_expert_ffn_backward(const moe_params* p, const uint16_t* x, const int32_t* topk_idx,
+              const float* topk_w, const int32_t* offsets, const int32_t* sorted_token,
+              const int32_t* sorted_pair, const int32_t* pair_row, const moe_weights* w,
+              const float* dout, const moe_grads* g, void* ws, size_t ws_bytes, moe_stream_t stream);
+
+/*
+ * Number of kernel launches one call of `which` (MOE_WS_ROUTE .. MOE_WS_BACKWARD,
+ * naming moe_route .. moe_forward_host, moe_route_stats, moe_expert_ffn_backward)
+ * makes with these params, into *n (host).
  */
 MOE_API int moe_launch_count(const moe_params* p, int which, int* n);
 

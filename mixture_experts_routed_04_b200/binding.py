@@ -28,19 +28,21 @@ DOWN_BF16, DOWN_F16 = 0, 1
 WEIGHTS_BF16, WEIGHTS_Q4G32 = 0, 1
 VARIANT_AUTO, VARIANT_TENSOR, VARIANT_STREAM = 0, 1, 2
 TILE_AUTO, TILE_ONE, TILE_PAIR = 0, 1, 2
-WS_ROUTE, WS_PERMUTE, WS_EXPERT_FFN, WS_COMBINE, WS_FORWARD, WS_FORWARD_HOST = range(6)
+WS_ROUTE, WS_PERMUTE, WS_EXPERT_FFN, WS_COMBINE, WS_FORWARD, WS_FORWARD_HOST, WS_ROUTE_STATS, WS_BACKWARD = range(8)
 
 # every entry point declared in include/moe.h
 EXPORTS = ("moe_version", "moe_status_string", "moe_capacity", "moe_max_rows", "moe_workspace_size",
            "moe_route", "moe_permute", "moe_expert_ffn", "moe_combine", "moe_forward", "moe_forward_host",
            "moe_get_error", "moe_clear_error", "moe_set_wait_limit_ns", "moe_launch_count",
            "moe_profile_enable", "moe_profile_collect", "moe_convert_bf16_to_f16",
-           "moe_permute_noalloc", "moe_forward_host_async", "moe_wait_selftest", "moe_tile_ctas")
+           "moe_permute_noalloc", "moe_forward_host_async", "moe_wait_selftest", "moe_tile_ctas",
+           "moe_route_stats", "moe_expert_ffn_backward")
 NOALLOC_MAX_PAIRS = 262144  # MOE_NOALLOC_MAX_PAIRS
 
 # kernel ids (MOE_K_*), in order
 KERNELS = ("route", "perm_count", "perm_scan", "perm_scatter", "schedule", "gather", "tc_gateup", "tc_down",
-           "stream_gateup", "stream_reduce", "stream_down", "combine", "convert", "front")
+           "stream_gateup", "stream_reduce", "stream_down", "combine", "convert", "front", "route_stats",
+           "bwd_gemm", "bwd_small")
 
 
 class MoeError(RuntimeError):
@@ -61,6 +63,11 @@ class Weights(ctypes.Structure):
                                                "shared_gate", "shared_up", "shared_down")]
 
 
+class Grads(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_void_p) for n in ("dx", "dw_gate", "dw_up", "dw_down", "d_topk_w", "dlogits",
+                                               "dshared_gate", "dshared_up", "dshared_down")]
+
+
 _lib = None
 _P, _V, _S = ctypes.POINTER(Params), ctypes.c_void_p, ctypes.c_size_t
 
@@ -79,6 +86,7 @@ def lib() -> ctypes.CDLL:
             "moe_tile_ctas": ([_P, ctypes.POINTER(ctypes.c_int32)], ctypes.c_int),
             "moe_workspace_size": ([_P, ctypes.c_int], _S),
             "moe_route": ([_P, _V, _V, _V, _V, _S, _V], ctypes.c_int),
+            "moe_route_stats": ([_P, _V, _V, _V, ctypes.c_float, _V, _V, _V, _V, _V, _S, _V], ctypes.c_int),
             "moe_permute": ([_P, _V, _V, _V, _V, _V, _V, _V, _V, _S, _V], ctypes.c_int),
             "moe_expert_ffn": ([_P, _V, _V, _V, _V, _V, ctypes.POINTER(Weights), _V, _V, _S, _V], ctypes.c_int),
             "moe_combine": ([_P, _V, _V, _V, _V, _V, _S, _V], ctypes.c_int),
@@ -94,6 +102,8 @@ def lib() -> ctypes.CDLL:
             "moe_profile_collect": ([ctypes.POINTER(ctypes.c_double), ctypes.POINTER(ctypes.c_int64)], ctypes.c_int),
             "moe_convert_bf16_to_f16": ([_V, _V, ctypes.c_int64, _V, _V], ctypes.c_int),
             "moe_permute_noalloc": ([_P, _V, _V, _V, _V, _V, _V, _V, _V, _V], ctypes.c_int),
+            "moe_expert_ffn_backward": ([_P, _V, _V, _V, _V, _V, _V, _V, ctypes.POINTER(Weights), _V,
+                                         ctypes.POINTER(Grads), _V, _S, _V], ctypes.c_int),
         }
         for name, (args, res) in sig.items():
             fn = getattr(L, name)
@@ -180,6 +190,17 @@ def route(p, logits, topk_idx, topk_w, ws, stream=None):
                           _stream(stream)), "moe_route")
 
 
+STATS = ("kept", "want_k", "balance", "z", "aux")  # moe_route_stats stats[0..4]
+
+
+def route_stats(p, logits, topk_idx, topk_w, stats, ws, z_weight=1e-3, kept_tok=None, want_tok=None,
+                expert_stats=None, stream=None):
+    """moe_route_stats: moe_route plus the router telemetry (stats: device fp32 [5], see STATS)."""
+    check(lib().moe_route_stats(ctypes.byref(p), _p(logits), _p(topk_idx), _p(topk_w), float(z_weight), _p(stats),
+                                _p(kept_tok), _p(want_tok), _p(expert_stats), _p(ws), ws.numel(),
+                                _stream(stream)), "moe_route_stats")
+
+
 def permute(p, topk_idx, counts, kept, offsets, sorted_token, sorted_pair, pair_row, ws, stream=None):
     check(lib().moe_permute(ctypes.byref(p), _p(topk_idx), _p(counts), _p(kept), _p(offsets), _p(sorted_token),
                             _p(sorted_pair), _p(pair_row), _p(ws), ws.numel(), _stream(stream)), "moe_permute")
@@ -201,6 +222,23 @@ def expert_ffn(p, x, offsets, sorted_token, sorted_pair, topk_w, W: Weights, y_r
 def combine(p, y_rows, pair_row, offsets, out, ws, stream=None):
     check(lib().moe_combine(ctypes.byref(p), _p(y_rows), _p(pair_row), _p(offsets), _p(out), _p(ws), ws.numel(),
                             _stream(stream)), "moe_combine")
+
+
+def grads(dx, dw_gate, dw_up, dw_down, d_topk_w, dlogits=None, shared=None) -> Grads:
+    sh = shared or (None, None, None)
+    ts = (dx, dw_gate, dw_up, dw_down, d_topk_w, dlogits, *sh)
+    G = Grads(*(None if t is None else t.data_ptr() for t in ts))
+    G._keep = ts
+    return G
+
+
+def expert_ffn_backward(p, x, topk_idx, topk_w, offsets, sorted_token, sorted_pair, pair_row, W: Weights, dout,
+                        G: Grads, ws, stream=None):
+    """moe_expert_ffn_backward: gradients of the layer for dout (fp32 [T, d]) into G (fp32)."""
+    check(lib().moe_expert_ffn_backward(ctypes.byref(p), _p(x), _p(topk_idx), _p(topk_w), _p(offsets),
+                                        _p(sorted_token), _p(sorted_pair), _p(pair_row), ctypes.byref(W), _p(dout),
+                                        ctypes.byref(G), _p(ws), ws.numel(), _stream(stream)),
+          "moe_expert_ffn_backward")
 
 
 def forward(p, x, logits, W: Weights, out, ws, counts_out=None, stream=None):

@@ -10,7 +10,7 @@
 namespace moe {
 
 cudaError_t launch_schedule(const Dims& D, const int32_t* offsets, int32_t* tile_base, int32_t* stream_list,
-                            int32_t* n_stream, uint32_t* err, cudaStream_t s);
+                            int32_t* n_stream, uint32_t* err, const UnitOrder& order, cudaStream_t s);
 cudaError_t launch_gather(const Dims& D, const uint16_t* x, const int32_t* sorted_token, const int32_t* offsets,
                           uint16_t* xg, uint32_t* err, cudaStream_t s);
 cudaError_t launch_scatter_rows(const Dims& D, const uint16_t* x, const int32_t* pair_row, const int32_t* offsets,
@@ -19,7 +19,7 @@ cudaError_t launch_tensor_ffn(const Dims& D, const uint16_t* xg, uint16_t* h, co
                               const int32_t* offsets, const int32_t* sorted_pair, const float* topk_w,
                               const moe_weights* w,
                               uint16_t* y_rows, int32_t* counters, uint32_t* err, uint64_t wait_ns,
-                              cudaStream_t s);
+                              const long long* units_a, const long long* units_b, cudaStream_t s);
 cudaError_t launch_convert_bf16_f16(const uint16_t* src, uint16_t* dst, int64_t n, uint32_t* err, cudaStream_t s);
 cudaError_t launch_stream_ffn(const Dims& D, const uint16_t* xg, uint16_t* h, float* part, const int32_t* offsets,
                               const int32_t* stream_list, const int32_t* n_stream, const int32_t* sorted_pair,
@@ -44,7 +44,7 @@ int num_sms() {
 static size_t align256(size_t v) { return (v + 255) & ~size_t(255); }
 
 // Host-side checks of moe_params; fills D. Returns MOE_OK or an error code.
-static int make_dims(const moe_params* p, Dims* D) {
+int make_dims(const moe_params* p, Dims* D) {
     if (!p || !D) return MOE_ERR_INVALID_ARG;
     // T = 0 (an empty batch) is valid: the calls launch nothing and report empty results
     if (p->T < 0 || p->E < 1 || p->E > kMaxE || p->k < 1 || p->k > kMaxK || p->k > p->E) return MOE_ERR_INVALID_ARG;
@@ -94,7 +94,7 @@ static int make_dims(const moe_params* p, Dims* D) {
     if (p->stream_max_rows < 0) {
         const int64_t touched_max = std::min<int64_t>(p->E + p->has_shared, pairs + p->has_shared);
         const int64_t tiles_max = touched_max * ((p->d_ff + 127) / 128);
-        D->stream_max_rows = tiles_max < kSmCountB200 ? kStreamRowsFewExperts : 0;
+        D->stream_max_rows = tiles_max < num_sms() ? kStreamRowsFewExperts : 0;
     } else {
         D->stream_max_rows = p->stream_max_rows;
     }
@@ -114,7 +114,8 @@ static int make_dims(const moe_params* p, Dims* D) {
     int ks = 1;
     const int64_t touched = std::min<int64_t>(D->Etot, pairs + p->has_shared);
     const int64_t units = touched * (p->d_ff / 64);
-    while (ks < 8 && units * ks < 4 * 148 && (p->d_model % (ks * 2 * 64)) == 0) ks *= 2;
+    const int64_t sms = num_sms();
+    while (ks < 8 && units * ks < 4 * sms && (p->d_model % (ks * 2 * 64)) == 0) ks *= 2;
     D->ks = ks;
     return MOE_OK;
 }
@@ -128,9 +129,32 @@ WsLayout ws_layout(const Dims& D, int which) {
         off = align256(off + bytes);
         return o;
     };
-    const bool perm = which == MOE_WS_PERMUTE || which >= MOE_WS_FORWARD;
-    const bool ffn = which == MOE_WS_EXPERT_FFN || which >= MOE_WS_FORWARD;
-    const bool fwd = which >= MOE_WS_FORWARD;
+    const bool fwd = which == MOE_WS_FORWARD || which == MOE_WS_FORWARD_HOST;
+    const bool perm = which == MOE_WS_PERMUTE || fwd;
+    const bool ffn = which == MOE_WS_EXPERT_FFN || fwd;
+    if (which == MOE_WS_BACKWARD) {
+        const int64_t rp = bwd_padded_rows(D);
+        const int nt = (D.f + 255) / 256;
+        L.b_poff = take(size_t(D.Etot + 1) * 4);
+        L.b_tile_base = take(size_t(D.Etot + 1) * 4);
+        L.b_wbase = take(size_t(D.Etot + 1) * 4);
+        L.b_counters = take(8 * 4);
+        L.b_xg = take(size_t(rp) * D.d * 2);
+        L.b_xgT = take(size_t(rp) * D.d * 2);
+        L.b_dog = take(size_t(rp) * D.d * 2);
+        L.b_gu = take(size_t(rp) * 2 * D.f * 4);
+        L.b_h = take(size_t(rp) * D.f * 2);
+        L.b_hwT = take(size_t(rp) * D.f * 2);
+        L.b_dgu = take(size_t(rp) * 2 * D.f * 2);
+        L.b_dxr = take(size_t(D.rows) * D.d * 2);
+        L.b_dwp = take(size_t(D.rows) * nt * 4);
+    }
+    if (which == MOE_WS_ROUTE_STATS) {
+        const int nb = route_stats_blocks(D.T > 0 ? D.T : 1);
+        L.stats_p = take(size_t(nb) * D.E * 4);
+        L.stats_c = take(size_t(nb) * D.E * 4);
+        L.stats_s = take(size_t(nb) * 3 * 4);
+    }
     if (perm) {
         L.blockcounts = take(size_t(D.perm_blocks) * D.E * 4);
         L.blockbase = take(size_t(D.perm_blocks) * D.E * 4);
@@ -139,6 +163,10 @@ WsLayout ws_layout(const Dims& D, int which) {
         L.tile_base = take(size_t(D.Etot + 1) * 2 * 4);  // 128-row and 256-row tile prefixes
         L.stream_list = take(size_t(D.Etot) * 4);
         L.n_stream = take(16);  // [0] streaming experts, [1], [2] tile-unit counters
+        // claim orders: at most (ceil(rows / 128) + Etot) M-tiles of 128 rows, times the n-tiles
+        const size_t mtiles = size_t((D.rows + kTileM - 1) / kTileM) + D.Etot;
+        L.units_a = take(mtiles * size_t((D.f + 127) / 128) * 8);
+        L.units_b = take(mtiles * size_t((D.d + 255) / 256) * 8);
         L.xg = take(size_t(D.rows) * D.d * 2);
         L.h = take(size_t(D.rows) * D.f * 2);
         if (D.ks > 1) L.part = take(size_t(D.ks) * 2 * D.rows * D.f * 4);
@@ -182,7 +210,17 @@ cudaError_t launch_expert_ffn(const Dims& D, const WsLayout& L, const FfnArgs& a
     uint16_t* h = reinterpret_cast<uint16_t*>(ws + L.h);
     float* part = L.part ? reinterpret_cast<float*>(ws + L.part) : nullptr;
     cudaError_t e = cudaSuccess;
-    if (!a.scheduled && (e = launch_schedule(D, a.offsets, tile_base, stream_list, n_stream, a.err, s)) != cudaSuccess)
+    // The claim order of the one-SM tile kernels (schedule.cu); the fused small-batch front
+    // kernel and the SM-pair kernels keep the natural order.
+    UnitOrder order{D.fmt == MOE_WEIGHTS_Q4G32 ? 2 : 1, (D.f + 127) / 128, (D.d + 255) / 256, kUnitOrderChunk,
+                    nullptr, nullptr};
+    const bool ordered = !a.scheduled && !D.tile_pair && tiles_needed(D);
+    if (ordered) {
+        order.units_a = reinterpret_cast<long long*>(ws + L.units_a);
+        order.units_b = reinterpret_cast<long long*>(ws + L.units_b);
+    }
+    if (!a.scheduled &&
+        (e = launch_schedule(D, a.offsets, tile_base, stream_list, n_stream, a.err, order, s)) != cudaSuccess)
         return e;
     // Rows in expert order for both variants (fp16 for Q4G32, whose MMAs run
     // in fp16). A TMA tile::gather4 of the rows inside the GEMM was measured
@@ -197,7 +235,8 @@ cudaError_t launch_expert_ffn(const Dims& D, const WsLayout& L, const FfnArgs& a
         return e;
     if (tiles_needed(D)) {
         if ((e = launch_tensor_ffn(D, xg, h, tile_base, a.offsets, a.sorted_pair, a.topk_w, a.w, a.y_rows,
-                                   n_stream + 1, a.err, a.wait_ns, s)) != cudaSuccess)
+                                   n_stream + 1, a.err, a.wait_ns, order.units_a, order.units_b, s)) !=
+            cudaSuccess)
             return e;
     }
     if (D.variant != MOE_VARIANT_TENSOR && D.stream_max_rows > 0) {
@@ -283,7 +322,7 @@ int moe_tile_ctas(const moe_params* p, int32_t* ctas) {
 
 size_t moe_workspace_size(const moe_params* p, int which) {
     Dims D;
-    if (make_dims(p, &D) != MOE_OK || which < MOE_WS_ROUTE || which > MOE_WS_FORWARD_HOST) return 0;
+    if (make_dims(p, &D) != MOE_OK || which < MOE_WS_ROUTE || which > MOE_WS_BACKWARD) return 0;
     return ws_layout(D, which).total;
 }
 
@@ -296,6 +335,23 @@ int moe_route(const moe_params* p, const float* logits, int32_t* topk_idx, float
     if (D.T == 0) return MOE_OK;  // empty batch: the (empty) buffers may be null
     if (!logits || !topk_idx || !topk_w) return MOE_ERR_INVALID_ARG;
     return status_of(launch_route(logits, D.T, D.E, D.k, topk_idx, topk_w, stream));
+}
+
+int moe_route_stats(const moe_params* p, const float* logits, int32_t* topk_idx, float* topk_w, float z_weight,
+                    float* stats, float* kept_tok, int32_t* want_tok, float* expert_stats, void* ws,
+                    size_t ws_bytes, moe_stream_t stream) {
+    Dims D;
+    int st = make_dims(p, &D);
+    if (st != MOE_OK) return st;
+    if ((st = check_ws(D, MOE_WS_ROUTE_STATS, ws, ws_bytes)) != MOE_OK) return st;
+    if (D.T == 0) return MOE_OK;
+    if (!logits || !topk_idx || !topk_w || !stats || !std::isfinite(z_weight)) return MOE_ERR_INVALID_ARG;
+    const WsLayout L = ws_layout(D, MOE_WS_ROUTE_STATS);
+    uint8_t* w = static_cast<uint8_t*>(ws);
+    return status_of(launch_route_stats(logits, D.T, D.E, D.k, topk_idx, topk_w, z_weight, stats, kept_tok,
+                                        want_tok, expert_stats, reinterpret_cast<float*>(w + L.stats_p),
+                                        reinterpret_cast<int32_t*>(w + L.stats_c),
+                                        reinterpret_cast<float*>(w + L.stats_s), stream));
 }
 
 int moe_permute(const moe_params* p, const int32_t* topk_idx, int32_t* counts, int32_t* kept_counts,
@@ -436,6 +492,33 @@ int moe_forward_host_async(const moe_params* p, const uint16_t* x_host, const fl
     return forward_host_impl(p, x_host, logits_host, w, out_host, ws, ws_bytes, stream, false);
 }
 
+int moe_expert_ffn_backward(const moe_params* p, const uint16_t* x, const int32_t* topk_idx, const float* topk_w,
+                            const int32_t* offsets, const int32_t* sorted_token, const int32_t* sorted_pair,
+                            const int32_t* pair_row, const moe_weights* w, const float* dout, const moe_grads* g,
+                            void* ws, size_t ws_bytes, moe_stream_t stream) {
+    Dims D;
+    int st = make_dims(p, &D);
+    if (st != MOE_OK) return st;
+    if (D.fmt != MOE_WEIGHTS_BF16 || D.down_f16) return MOE_ERR_UNSUPPORTED;
+    // the transpose grid holds padded rows / 32 blocks in y (at most 65535)
+    if (bwd_padded_rows(D) / 32 > 65535) return MOE_ERR_UNSUPPORTED;
+    if ((st = check_ws(D, MOE_WS_BACKWARD, ws, ws_bytes)) != MOE_OK) return st;
+    if (D.T == 0) return MOE_OK;
+    if ((st = check_weights(D, w)) != MOE_OK) return st;
+    if (!x || !topk_w || !offsets || !sorted_token || !sorted_pair || !pair_row || !dout || !g) return MOE_ERR_INVALID_ARG;
+    if (!g->dx || !g->dw_gate || !g->dw_up || !g->dw_down || !g->d_topk_w) return MOE_ERR_INVALID_ARG;
+    if (g->dlogits && !topk_idx) return MOE_ERR_INVALID_ARG;
+    if (D.has_shared && (!g->dshared_gate || !g->dshared_up || !g->dshared_down)) return MOE_ERR_INVALID_ARG;
+    if (!al16(x) || !al16(dout) || !al16(g->dx) || !al16(g->dw_gate) || !al16(g->dw_up) || !al16(g->dw_down))
+        return MOE_ERR_MISALIGNED;
+    if (D.has_shared && (!al16(g->dshared_gate) || !al16(g->dshared_up) || !al16(g->dshared_down)))
+        return MOE_ERR_MISALIGNED;
+    BwdArgs a{x, dout, topk_idx, topk_w, offsets, sorted_token, sorted_pair, pair_row, w, g,
+              static_cast<uint8_t*>(ws), ws_layout(D, MOE_WS_BACKWARD), static_cast<uint32_t*>(ws),
+              g_wait_ns.load()};
+    return status_of(launch_backward(D, a, stream));
+}
+
 int moe_get_error(const void* ws, uint32_t* err, moe_stream_t stream) {
     if (!ws || !err) return MOE_ERR_INVALID_ARG;
     uint32_t v = 0;
@@ -454,7 +537,7 @@ int moe_launch_count(const moe_params* p, int which, int* n) {
     Dims D;
     const int st = make_dims(p, &D);
     if (st != MOE_OK) return st;
-    if (!n || which < MOE_WS_ROUTE || which > MOE_WS_FORWARD_HOST) return MOE_ERR_INVALID_ARG;
+    if (!n || which < MOE_WS_ROUTE || which > MOE_WS_BACKWARD) return MOE_ERR_INVALID_ARG;
     if (D.T == 0) {
         *n = 0;
         return MOE_OK;
@@ -468,6 +551,9 @@ int moe_launch_count(const moe_params* p, int which, int* n) {
         case MOE_WS_PERMUTE: *n = 3; break;
         case MOE_WS_EXPERT_FFN: *n = ffn; break;
         case MOE_WS_COMBINE: *n = 1; break;
+        case MOE_WS_ROUTE_STATS: *n = 2; break;
+        // schedule, gather, transpose, 6 GEMMs, zeroing, combine, reduce (+ dlogits: not counted)
+        case MOE_WS_BACKWARD: *n = 12; break;
         default: *n = D.T <= kFrontMaxTokens ? 1 + (ffn - 1) + 1 : 1 + 3 + ffn + 1; break;
     }
     return MOE_OK;

@@ -4,8 +4,9 @@
 // pair order (y[e_sorted, slot]) and each token's k outputs are summed with
 // their gate weights. The weights were applied in the down-projection
 // epilogue, so here out[t] = sum over kept j of y_rows[pair_row[t*k+j]]
-// (+ the shared expert's row), accumulated in fp32 in fixed j order, then
-// rounded to bf16 once. A dropped pair (row -1) adds nothing.
+// (+ the shared expert's row), accumulated in fp32 in fixed j order and
+// stored as fp32 (or, with the bf16 output option, rounded to bf16 once).
+// A dropped pair (row -1) adds nothing.
 //
 // HBM-bound: one 16-byte vector (8 bf16) per thread per row read; blocks walk
 // tokens with a grid stride; no atomics, so the result is deterministic.

@@ -83,6 +83,13 @@ struct Cfg {
         idesc_f16_f32(64, BN, /*ab_bf16=*/(MODE == 0 && WF == 0) ? 1 : 0, /*a_mn=*/0, /*b_mn=*/Q4 ? 0 : 1);
 };
 
+// The first unit of a weight tile to run (m = 0, the leader) streams that tile
+// from HBM while the unit's other M-tiles wait for the same lines; the leader's
+// producer also asks L2 for the weight k-block kPrefetchAhead blocks past the
+// one it loads, so that more of the tile is in flight than the stages hold.
+// 0 = off.
+constexpr int kPrefetchAhead = 0;
+
 MOE_DEV uint32_t lop3_and_or(uint32_t a, uint32_t mask, uint32_t orv) {
     uint32_t r;
     asm("lop3.b32 %0, %1, %2, %3, 0xEA;" : "=r"(r) : "r"(a), "r"(mask), "r"(orv));  // (a & b) | c
@@ -235,10 +242,23 @@ __global__ void __launch_bounds__(Cfg<MODE, WF, SUB>::kThreads, 1)
                         // two 64-column chunks of gate, then two of up: one copy each
                         tma_load_4d(sb, mg, full + stage, 0, kb * BK, 2 * U.n, z);
                         tma_load_4d(sb + 2 * B_CHUNK, mu, full + stage, 0, kb * BK, 2 * U.n, z);
+                        if (kPrefetchAhead > 0 && U.m == 0) {
+                            for (int q = kb == 0 ? 1 : kPrefetchAhead; q <= kPrefetchAhead; ++q) {
+                                if (kb + q >= KB) break;
+                                tma_prefetch_l2_4d(mg, 0, (kb + q) * BK, 2 * U.n, z);
+                                tma_prefetch_l2_4d(mu, 0, (kb + q) * BK, 2 * U.n, z);
+                            }
+                        }
                     } else {
                         const CUtensorMap* md = sh ? &tmS0 : &tmB0;
                         // four 64-column chunks in one copy
                         tma_load_4d(sb, md, full + stage, 0, kb * BK, 4 * U.n, z);
+                        if (kPrefetchAhead > 0 && U.m == 0) {
+                            for (int q = kb == 0 ? 1 : kPrefetchAhead; q <= kPrefetchAhead; ++q) {
+                                if (kb + q >= KB) break;
+                                tma_prefetch_l2_4d(md, 0, (kb + q) * BK, 4 * U.n, z);
+                            }
+                        }
                     }
                     issued |= 1u << stage;
                     issued_par = (issued_par & ~(1u << stage)) | (phase << stage);
@@ -490,6 +510,22 @@ bool map_weights(CUtensorMap* m, const void* base, int nexp, int K, int N, int c
     const uint32_t box[4] = {64, 64, uint32_t(chunks), 1};
     return make_map(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, base, 4, dims, str, box, CU_TENSOR_MAP_SWIZZLE_128B);
 }
+// bf16 weights [nexp, N, K] (K contiguous) read as a K-major B operand: box 64 (K)
+// x 256 (N rows) x 1, 128-byte swizzle — the layout of the A tiles, 256 rows.
+bool map_weights_kmajor(CUtensorMap* m, const void* base, int nexp, int N, int K) {
+    const uint64_t dims[3] = {uint64_t(K), uint64_t(N), uint64_t(nexp)};
+    const uint64_t str[2] = {uint64_t(K) * 2, uint64_t(N) * uint64_t(K) * 2};
+    const uint32_t box[3] = {64, 256, 1};
+    return make_map(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, base, 3, dims, str, box, CU_TENSOR_MAP_SWIZZLE_128B);
+}
+// bf16 activation rows [rows, N] (row stride row_stride elements) read as an N-major B
+// operand (K = rows): seen as [1, N/64 chunks, rows, 64]; one copy brings 4 chunks.
+bool map_act_mn(CUtensorMap* m, const void* base, int64_t rows, int N, int64_t row_stride) {
+    const uint64_t dims[4] = {64, uint64_t(rows), uint64_t(N / 64), 1};
+    const uint64_t str[3] = {uint64_t(row_stride) * 2, 128, uint64_t(row_stride) * uint64_t(rows) * 2};
+    const uint32_t box[4] = {64, 64, 4, 1};
+    return make_map(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, base, 4, dims, str, box, CU_TENSOR_MAP_SWIZZLE_128B);
+}
 // Q4G32 nibbles: [nexp, N, K/2] bytes; box 32 bytes (64 k) x rows x 1, no swizzle.
 bool map_q4_packed(CUtensorMap* m, const void* base, int nexp, int K, int N, int rows) {
     const uint64_t dims[3] = {uint64_t(K / 2), uint64_t(N), uint64_t(nexp)};
@@ -537,7 +573,7 @@ cudaError_t launch_tensor_ffn(const Dims& D, const uint16_t* xg, uint16_t* h, co
                               const int32_t* offsets,
                               const int32_t* sorted_pair, const float* topk_w, const moe_weights* w,
                               uint16_t* y_rows, int32_t* counters, uint32_t* err, uint64_t wait_ns,
-                              cudaStream_t s) {
+                              const long long* units_a, const long long* units_b, cudaStream_t s) {
     using namespace tc;
     const bool pdl = use_pdl(D.T);
     GemmParams p{};
@@ -564,12 +600,14 @@ cudaError_t launch_tensor_ffn(const Dims& D, const uint16_t* xg, uint16_t* h, co
         p.n_tiles = (D.f + 127) / 128;
         p.out = h;
         p.unit_counter = counters;
+        p.units = units_a;
         if ((e = launch_gemm<0, 1, 2>(mA, pg, pu, sg, su, p, pdl, s)) != cudaSuccess) return e;
         p.K = D.f;
         p.n_out = D.d;
         p.n_tiles = (D.d + BN - 1) / BN;
         p.out = y_rows;
         p.unit_counter = counters + 1;
+        p.units = units_b;
         return launch_gemm<1, 1, 2>(mH, pd, pd, sd, sd, p, pdl, s);
     }
     CUtensorMap mG, mU, mSG, mSU, mD, mSD;
@@ -592,6 +630,7 @@ cudaError_t launch_tensor_ffn(const Dims& D, const uint16_t* xg, uint16_t* h, co
     p.n_tiles = (D.f + 127) / 128;
     p.out = h;
     p.unit_counter = counters;
+    p.units = D.tile_pair ? nullptr : units_a;
     e = D.tile_pair ? launch_gemm_pair<0>(mA, mG, mU, mSG, mSU, p, pdl, s)
                     : launch_gemm<0, 0, 1>(mA, mG, mU, mSG, mSU, p, pdl, s);
     if (e != cudaSuccess) return e;
@@ -601,6 +640,7 @@ cudaError_t launch_tensor_ffn(const Dims& D, const uint16_t* xg, uint16_t* h, co
     p.n_tiles = (D.d + BN - 1) / BN;
     p.out = y_rows;
     p.unit_counter = counters + 1;
+    p.units = D.tile_pair ? nullptr : units_b;
     if (D.tile_pair && D.down_f16) {
         // each SM of a pair copies 128 of the tile's 256 columns: maps of 2 chunks
         CUtensorMap mD2, mSD2;

@@ -12,7 +12,6 @@ constexpr int kPermPairsPerWarp = 256;                // 8 rounds of 32 pairs
 constexpr int kPermPairsPerBlock = kPermWarps * kPermPairsPerWarp;
 constexpr int kTileM = 128;                           // rows per tcgen05 tile
 constexpr int kStreamRowsFewExperts = 8;             // AUTO: streaming threshold when few experts are touched
-constexpr int kSmCountB200 = 148;
 
 // Everything a call derives from moe_params on the host.
 struct Dims {
@@ -35,17 +34,31 @@ struct WsLayout {
     size_t err;                                    // uint32 error word (always at 0)
     size_t blockcounts, blockbase;                 // permute: int32 [perm_blocks, E]
     size_t tile_base, stream_list, n_stream;       // expert_ffn schedule
+    size_t units_a, units_b;                       // claim orders of the two tcgen05 GEMMs (int64)
     size_t xg, h, part;                            // expert_ffn: gathered x, h, split-K partials
     size_t topk_idx, topk_w, counts, kept, offsets, sorted_token, sorted_pair, pair_row, y_rows;  // forward
     size_t x_dev, logits_dev, out_dev;             // forward_host
+    size_t stats_p, stats_c, stats_s;              // route_stats: per-block partial sums
+    // backward (padded row space, see backward.cu)
+    size_t b_poff, b_tile_base, b_wbase, b_counters, b_xg, b_xgT, b_dog, b_gu, b_h, b_hwT, b_dgu, b_dxr, b_dwp;
     size_t total;
 };
 
 WsLayout ws_layout(const Dims& D, int which);
 
+// The parameter checks every entry point shares: fills D from moe_params and
+// returns MOE_OK, or the status the entry point returns unchanged.
+int make_dims(const moe_params* p, Dims* D);
+
 // ---- launchers (all asynchronous on `s`)
 cudaError_t launch_route(const float* logits, int T, int E, int k, int32_t* topk_idx, float* topk_w,
                          cudaStream_t s);
+
+int route_stats_blocks(int T);
+cudaError_t launch_route_stats(const float* logits, int T, int E, int k, int32_t* topk_idx, float* topk_w,
+                               float z_weight, float* stats, float* kept_tok, int32_t* want_tok,
+                               float* expert_stats, float* part_p, int32_t* part_c, float* part_s,
+                               cudaStream_t stream);
 
 cudaError_t launch_permute(const Dims& D, const int32_t* topk_idx, int32_t* blockcounts, int32_t* blockbase,
                            int32_t* counts, int32_t* kept, int32_t* offsets, int32_t* sorted_token,
@@ -58,6 +71,17 @@ cudaError_t launch_front_small(const Dims& D, const float* logits, int32_t* topk
                                int32_t* counts, int32_t* kept, int32_t* offsets, int32_t* sorted_token,
                                int32_t* sorted_pair, int32_t* pair_row, int32_t* tile_base, int32_t* stream_list,
                                int32_t* n_stream, uint32_t* err, cudaStream_t s);
+
+// Claim order of the tcgen05 GEMMs' units, written by the schedule kernel
+// (schedule.cu): M-tiles of `sub` x 128 rows; nt_a / nt_b n-tiles per M-tile
+// for gate/up and down; chunk groups per chunk (0: the natural order).
+struct UnitOrder {
+    int sub, nt_a, nt_b, chunk;
+    long long* units_a;
+    long long* units_b;
+};
+// Groups (expert, n-tile) per chunk of the claim order.
+constexpr int kUnitOrderChunk = 32;
 
 struct FfnArgs {
     const uint16_t* x;
@@ -77,6 +101,27 @@ cudaError_t launch_expert_ffn(const Dims& D, const WsLayout& L, const FfnArgs& a
 
 cudaError_t launch_combine(const Dims& D, const uint16_t* y_rows, const int32_t* pair_row, const int32_t* offsets,
                            void* out, cudaStream_t s);
+
+// Backward of the expert FFN (backward.cu).
+struct BwdArgs {
+    const uint16_t* x;
+    const float* dout;
+    const int32_t* topk_idx;
+    const float* topk_w;
+    const int32_t* offsets;
+    const int32_t* sorted_token;
+    const int32_t* sorted_pair;
+    const int32_t* pair_row;
+    const moe_weights* w;
+    const moe_grads* g;
+    uint8_t* ws;
+    WsLayout layout;
+    uint32_t* err;
+    uint64_t wait_ns;
+};
+// Rows of the padded row space the backward allocates.
+int64_t bwd_padded_rows(const Dims& D);
+cudaError_t launch_backward(const Dims& D, const BwdArgs& a, cudaStream_t s);
 
 // ---- device properties, cached per device
 int num_sms();

@@ -33,7 +33,10 @@ static_assert(MOE_NOALLOC_MAX_PAIRS % kPermPairsPerBlock == 0, "pair limit must 
 static __device__ __align__(256) int32_t g_perm_scratch[kNoAllocInts];
 
 // Device address of g_perm_scratch on each device, looked up once per device
-// (with that device current) on the first call made there.
+// (with that device current) on the first call made there. The cached address
+// belongs to that device's primary context: after cudaDeviceReset (or anything
+// else that destroys the context) it is stale, so the entry point must not be
+// used across a reset.
 std::mutex g_mu;
 int32_t* g_scratch_addr[64] = {nullptr};
 
@@ -64,29 +67,17 @@ extern "C" MOE_API int moe_permute_noalloc(const moe_params* p, const int32_t* t
                                            int32_t* sorted_pair, int32_t* pair_row, uint32_t* err_word,
                                            moe_stream_t stream) {
     using namespace moe;
-    if (!p) return MOE_ERR_INVALID_ARG;
-    const size_t need = moe_workspace_size(p, MOE_WS_PERMUTE);  // 0 if the params are invalid
-    if (need == 0) return MOE_ERR_INVALID_ARG;
-    const int64_t pairs = int64_t(p->T) * p->k;
-    if (pairs > MOE_NOALLOC_MAX_PAIRS) return MOE_ERR_WORKSPACE_TOO_SMALL;  // beyond the fixed scratch
+    // the same parameter checks and dimensions as moe_permute, status unchanged
+    Dims D{};
+    const int st = make_dims(p, &D);
+    if (st != MOE_OK) return st;
+    if (D.pairs > MOE_NOALLOC_MAX_PAIRS) return MOE_ERR_WORKSPACE_TOO_SMALL;  // beyond the fixed scratch
     if (!topk_idx || !counts || !kept_counts || !offsets || !sorted_token || !sorted_pair || !pair_row ||
         !err_word)
         return MOE_ERR_INVALID_ARG;
     cudaError_t ce = cudaSuccess;
     int32_t* scratch = scratch_for_current_device(&ce);
     if (!scratch) return MOE_ERR_CUDA;
-    // Same dimensions as moe_permute derives (the parameter checks above passed).
-    Dims D{};
-    D.T = p->T;
-    D.E = p->E;
-    D.k = p->k;
-    D.has_shared = p->has_shared;
-    D.Etot = p->E + p->has_shared;
-    D.pairs = pairs;
-    D.perm_blocks = int((pairs + kPermPairsPerBlock - 1) / kPermPairsPerBlock);
-    int32_t cap = -1;
-    if (moe_capacity(p, &cap) != MOE_OK) return MOE_ERR_INVALID_ARG;
-    D.cap = cap;
     int32_t* blockcounts = scratch;
     int32_t* blockbase = scratch + kNoAllocMaxBlocks * kMaxE;
     const cudaError_t e = launch_permute(D, topk_idx, blockcounts, blockbase, counts, kept_counts, offsets,

@@ -24,13 +24,14 @@ MOE_DEV float route_unkey(uint32_t k) {
 }
 
 // The whole warp routes token `row` (E logits): lane j < k writes selection j
-// to idx_out[j] / w_out[j]. Warp-uniform; every lane must call it.
+// to idx_out[j] / w_out[j]. Warp-uniform; every lane must call it. Returns
+// the first choice (warp-uniform).
 // Each round: every lane takes its best untaken logit (larger value, then
 // lower expert index); one warp max-reduction of the keys gives the winning
 // value and one min-reduction over the lanes holding it gives the lowest
 // expert index among equal values.
-MOE_DEV void route_one_token(const float* __restrict__ row, int E, int k, int32_t* __restrict__ idx_out,
-                             float* __restrict__ w_out) {
+MOE_DEV int route_one_token(const float* __restrict__ row, int E, int k, int32_t* __restrict__ idx_out,
+                            float* __restrict__ w_out) {
     const int lane = threadIdx.x & 31;
     uint32_t key[kRouteMaxPerLane];
 #pragma unroll
@@ -45,6 +46,7 @@ MOE_DEV void route_one_token(const float* __restrict__ row, int E, int k, int32_
     float sel_v = 0.f;
     int sel_i = 0;
     float top = 0.f;
+    int first = 0;
     for (int j = 0; j < k; ++j) {
         uint32_t bk = 0;
         int bi = 0x7FFFFFFF;
@@ -58,7 +60,10 @@ MOE_DEV void route_one_token(const float* __restrict__ row, int E, int k, int32_
         const int wi = int(__reduce_min_sync(0xFFFFFFFFu, (bi != 0x7FFFFFFF && bk == kmax) ? uint32_t(bi) : 0xFFFFFFFFu));
         if ((wi & 31) == lane) taken |= 1u << (wi >> 5);
         const float wv = route_unkey(kmax);
-        if (j == 0) top = wv;
+        if (j == 0) {
+            top = wv;
+            first = wi;
+        }
         if (lane == j) {
             sel_v = wv;
             sel_i = wi;
@@ -73,6 +78,7 @@ MOE_DEV void route_one_token(const float* __restrict__ row, int E, int k, int32_
         idx_out[lane] = sel_i;
         w_out[lane] = ex / s;
     }
+    return first;
 }
 
 }  // namespace moe

@@ -12,12 +12,15 @@ oracle pull only the experts a sampled token touches.
 Value recipe (the workloads of the task's five layer configurations):
 
 * x: N(0, 1) fp32, rounded to bf16 (round-to-nearest-even).
+* upstream gradient (backward): N(0, 1) fp32.
 * router logits: N(0, 1) fp32, plus a per-expert bias:
   - ``zipf``: expert e gets a rank r_e (a seeded permutation of 1..E) and
     bias 3.0 * (1 - ln r_e / ln E), i.e. the log of a Zipf law rescaled to
     [0, 3.0]; the exponent s=1.1 cancels under that rescale. The literal
     reading 3.0 * r^-1.1 is kept as ``zipf_literal``.
   - ``hot``: +4.0 on 8 seeded distinct experts.
+  - ``balanced`` (timing sweeps only): +16 on experts (t*k + j) mod touched,
+    j < k, so every one of ``touched`` experts gets exactly T*k/touched pairs.
 * expert weights W_gate, W_up [d, f] and W_down [f, d]: N(0, 0.02) fp32 → bf16.
 * Q4G32 weights (self-defined 4-bit format): the same N(0, 0.02) draws,
   quantised per group of 32 along K with one fp16 scale per group (see
@@ -36,7 +39,7 @@ from concurrent.futures import ThreadPoolExecutor
 import numpy as np
 
 # stream ids, one per tensor kind
-S_LOGITS, S_X, S_ZIPF_RANK, S_HOT = 1, 2, 3, 4
+S_LOGITS, S_X, S_ZIPF_RANK, S_HOT, S_DOUT = 1, 2, 3, 4, 5
 S_WG, S_WU, S_WD = 10, 11, 12
 S_SWG, S_SWU, S_SWD = 20, 21, 22
 
@@ -52,7 +55,8 @@ class LayerConfig:
     E: int
     k: int
     capacity_factor: float = 0.0
-    bias: str = "none"  # none | zipf | zipf_literal | hot
+    bias: str = "none"  # none | zipf | zipf_literal | hot | balanced
+    touched: int = 0  # balanced: experts 0..touched-1 share the pairs evenly
     has_shared: bool = False
     f_shared: int = 0
     weight_format: str = "bf16"  # bf16 | q4g32
@@ -130,9 +134,23 @@ def expert_bias(cfg: LayerConfig) -> np.ndarray:
 
 
 def logits(cfg: LayerConfig) -> np.ndarray:
-    """Router logits [T, E] fp32: N(0,1) plus the per-expert bias."""
+    """Router logits [T, E] fp32: N(0,1) plus the per-expert bias; with ``balanced``,
+    +16 on experts (t*k + j) mod touched for j < k instead, so those k experts are token t's
+    choice and every touched expert receives T*k/touched pairs (timing sweeps over exact
+    rows per expert)."""
     z = _rng(cfg.seed, S_LOGITS).standard_normal((cfg.T, cfg.E), dtype=np.float32)
+    if cfg.bias == "balanced":
+        n = cfg.touched if cfg.touched else cfg.E
+        t = np.arange(cfg.T)[:, None]
+        cols = (t * cfg.k + np.arange(cfg.k)[None, :]) % n
+        z[np.arange(cfg.T)[:, None], cols] += np.float32(16.0)
+        return z
     return z + expert_bias(cfg)[None, :]
+
+
+def dout(cfg: LayerConfig) -> np.ndarray:
+    """Upstream gradient dL/d out [T, d] fp32 ~ N(0, 1), for the backward."""
+    return _rng(cfg.seed, S_DOUT).standard_normal((cfg.T, cfg.d), dtype=np.float32)
 
 
 def x_bits(cfg: LayerConfig) -> np.ndarray:

@@ -11,8 +11,8 @@ compared element by element on every kernel variant and both forms of W_down
 (bf16 as given, fp16 prepared at load time). The stated workloads are compared
 at full size in the launch configuration the benchmark times (moe_forward,
 automatic variant choice, W_down prepared as fp16): routing and permutation in
-full, and every output element (the Q4G32 workload: outputs of sampled tokens,
-each from its own definition).
+full, and every output element (with sampled tokens from the per-token
+definition beside it), and the bf16 output option on every workload.
 """
 import ctypes
 
@@ -312,13 +312,14 @@ def test_full_size_workloads(name):
 
 
 def test_full_size_quantised_workload():
+    """The T=32768 Q4G32 layer: every output element against the oracle's whole layer (each
+    expert's weights dequantised exactly as q * s), plus sampled tokens from the per-token
+    definition, which never permutes."""
     cfg = synth.CONFIGS["quant"]
     d = device_inputs(cfg)
     got = run_steps(cfg, d, b.VARIANT_AUTO, False)
     idx, w, perm = check_routing(cfg, got)
     x = synth.bf16_bits_to_f32(synth.x_bits(cfg)).astype(np.float64)
-    rng = np.random.default_rng(7)
-    toks = sorted(set([0, cfg.T - 1] + rng.choice(cfg.T, 40, replace=False).tolist()))
     cache = {}
 
     def experts(e):
@@ -326,10 +327,59 @@ def test_full_size_quantised_workload():
             cache[e] = expert_ref(cfg, e)
         return cache[e]
 
-    ref = oracle.token_outputs(toks, x, idx, w, perm["pair_row"], experts, cfg.swiglu_limit)
-    check_close(got["out"][toks], ref, "quant sampled tokens (step calls)")
+    ref, it = oracle.forward(x, synth.logits(cfg), cfg.k, experts, cfg.swiglu_limit, cfg.capacity_factor)
+    check_close(got["out"], ref, "quant full output (step calls)")
+    w_row = np.array([it["w"].reshape(-1)[p] for p in it["sorted_pair"]])
+    check_close(got["y"], it["y"] * w_row[:, None], "quant y_rows")
     fout, _ = run_forward(cfg, d)
-    check_close(f64(fout)[toks], ref, "quant sampled tokens (moe_forward)")
+    check_close(f64(fout), ref, "quant full output (moe_forward)")
+    rng = np.random.default_rng(7)
+    toks = sorted(set([0, cfg.T - 1] + rng.choice(cfg.T, 16, replace=False).tolist()))
+    one = oracle.token_outputs(toks, x, idx, w, perm["pair_row"], experts, cfg.swiglu_limit)
+    check_close(f64(fout)[toks], one, "quant per-token definition")
+
+
+BF16_ULP_REL = 2.0 ** -8  # one rounding to bf16 (8 significant bits) moves a value by at most this, relative
+
+
+@pytest.mark.parametrize("name", ["tiny"] + FULL + ["quant"])
+def test_bf16_output_every_workload(name):
+    """The bf16 output option on every stated workload at full size: it equals the fp32 output
+    rounded once (nearest even); against the oracle, rel-L2 <= 1e-2 and every element within
+    3e-2 * rms(out) plus the one bf16 rounding (2^-8 of the element). On the capped layer most
+    tokens lose every pair, rms(out) is small, and that rounding alone exceeds 3e-2 * rms on a
+    few elements, hence the second term. Prints the measured max-abs / rms."""
+    cfg = synth.CONFIGS[name]
+    idx, w, perm = routing_reference(cfg)
+    touched = np.unique(idx[perm["pair_row"].reshape(idx.shape) >= 0])
+    d = device_inputs(cfg, experts=None if cfg.weight_format == "q4g32" else touched)
+    f32_out, _ = run_forward(cfg, d)
+    p = P_of(cfg, b.VARIANT_AUTO, cfg.weight_format == "bf16", out_dtype=b.OUT_BF16)
+    ws = b.workspace(p, b.WS_FORWARD)
+    out = torch.empty(cfg.T, cfg.d, dtype=torch.bfloat16, device="cuda")
+    b.forward(p, d["x"], d["logits"], W_of(d, cfg.weight_format == "bf16"), out, ws)
+    torch.cuda.synchronize()
+    assert b.get_error(ws) == 0
+    assert torch.equal(out.view(torch.int16), f32_out.to(torch.bfloat16).view(torch.int16))
+    x = synth.bf16_bits_to_f32(synth.x_bits(cfg)).astype(np.float64)
+    sh = shared_f64(cfg) if cfg.has_shared else None
+    cache = {}
+
+    def experts(e):
+        if e not in cache:
+            cache[e] = expert_ref(cfg, e)
+        return cache[e]
+
+    ref, _ = oracle.forward(x, synth.logits(cfg), cfg.k, experts, cfg.swiglu_limit, cfg.capacity_factor,
+                            shared=sh)
+    got = f64(out)
+    diff = np.abs(got - ref)
+    rel = np.linalg.norm(got - ref) / np.linalg.norm(ref)
+    rms = float(np.sqrt(np.mean(ref ** 2)))
+    print(f"bf16 output {name}: rel-L2 {rel:.3e}, max-abs/rms {diff.max() / rms:.3e}")
+    assert rel <= REL_L2, f"{name} bf16 output rel-L2 {rel:.3e}"
+    bound = MAX_ABS_RMS * rms + BF16_ULP_REL * np.abs(ref)
+    assert (diff <= bound).all(), f"{name} bf16 output: max excess {(diff - bound).max():.3e}"
 
 
 @pytest.mark.parametrize("name", ["tiny", "single_token", "shared_small", "k_equals_E", "small_capped"])
@@ -469,3 +519,55 @@ def test_empty_batch():
     torch.cuda.synchronize()
     assert all(int(t.abs().sum()) == 0 for t in bufs[:3])
     assert b.get_error(ws) == 0 and b.get_error(wsp) == 0
+
+
+@pytest.mark.parametrize("name", ["tiny", "prompt", "capped", "decode1", "decode32", "quant"])
+def test_route_stats_against_oracle(name):
+    """moe_route_stats: the routing bit-identical to moe_route; kept, balance, z and aux against
+    the oracle's router telemetry (fp64) within 1e-5 relative; each token's want exact where the
+    fp64 cumulative mass is not within 1e-5 of 90% at the decision, and otherwise one of the two
+    counts on either side of it; two calls bit-identical."""
+    cfg = synth.CONFIGS[name]
+    T, E, k = cfg.T, cfg.E, cfg.k
+    p = b.params_for(cfg)
+    lg_np = synth.logits(cfg)
+    lg = torch.from_numpy(lg_np).cuda()
+    i32 = dict(dtype=torch.int32, device="cuda")
+    f32 = dict(dtype=torch.float32, device="cuda")
+    ref_idx, ref_w = torch.empty(T, k, **i32), torch.empty(T, k, **f32)
+    b.route(p, lg, ref_idx, ref_w, b.workspace(p, b.WS_ROUTE))
+    ws = b.workspace(p, b.WS_ROUTE_STATS)
+    zw = 1e-3
+    runs = []
+    for _ in range(2):
+        idx, w = torch.full((T, k), -1, **i32), torch.full((T, k), float("nan"), **f32)
+        stats, kept = torch.full((5,), float("nan"), **f32), torch.full((T,), float("nan"), **f32)
+        want, est = torch.full((T,), -1, **i32), torch.full((2, E), float("nan"), **f32)
+        b.route_stats(p, lg, idx, w, stats, ws, z_weight=zw, kept_tok=kept, want_tok=want, expert_stats=est)
+        torch.cuda.synchronize()
+        assert b.get_error(ws) == 0
+        runs.append([t.cpu().numpy() for t in (idx, w, stats, kept, want, est)])
+    for a, c in zip(*runs):
+        assert np.array_equal(a.view(np.uint8), c.view(np.uint8)), "two calls differ"
+    idx, w, stats, kept, want, est = runs[0]
+    assert np.array_equal(idx, ref_idx.cpu().numpy())
+    assert np.array_equal(w.view(np.int32), ref_w.cpu().numpy().view(np.int32))
+    r = oracle.router_telemetry(lg_np, k, z_weight=zw)
+    for i, key in enumerate(("kept", "balance", "z", "aux")):
+        got = stats[[0, 2, 3, 4][i]]
+        np.testing.assert_allclose(got, r[key], rtol=1e-5, err_msg=key)
+    np.testing.assert_allclose(kept, r["kept_tok"], rtol=0, atol=1e-5)
+    np.testing.assert_allclose(est[0], r["frac"], rtol=1e-6, atol=0)
+    np.testing.assert_allclose(est[1], r["prob_mean"], rtol=1e-5, atol=1e-8)
+    # want: the fp64 cumulative mass of the sorted probabilities decides it
+    x = lg_np.astype(np.float64)
+    pr = np.exp(x - x.max(1, keepdims=True))
+    pr /= pr.sum(1, keepdims=True)
+    cum = np.cumsum(-np.sort(-pr, axis=1), axis=1)
+    ref_want = r["want_tok"]
+    near = np.abs(cum[np.arange(T), ref_want - 1] - 0.9) < 1e-5
+    near |= (ref_want > 1) & (np.abs(cum[np.arange(T), np.maximum(ref_want - 2, 0)] - 0.9) < 1e-5)
+    exact = ~near
+    assert np.array_equal(want[exact], ref_want[exact])
+    assert (np.abs(want[near] - ref_want[near]) <= 1).all()
+    np.testing.assert_allclose(stats[1], r["want_k"], rtol=0, atol=near.sum() / T + 1e-6)

@@ -63,6 +63,15 @@ def test_noalloc_permute_matches_the_workspace_version_on_two_calls():
     n1 = _compare_with_workspace_version(synth.CONFIGS["capped"])
     n2 = _compare_with_workspace_version(synth.CONFIGS["prompt"])
     assert n1 > 0 and n2 == 4096 * 8
+    # the decode layer: 256 experts plus the shared expert's rows
+    n3 = _compare_with_workspace_version(synth.CONFIGS["decode32"])
+    assert n3 == 32 * 8 + 32
+    # exactly the array's limit, 256 experts and a shared expert: the last block and the
+    # widest expert stride of the fixed array are both in use
+    big = synth.LayerConfig("noalloc_limit", T=b.NOALLOC_MAX_PAIRS // 8, d=64, f=64, E=256, k=8,
+                            has_shared=True, f_shared=64)
+    n4 = _compare_with_workspace_version(big)
+    assert n4 == b.NOALLOC_MAX_PAIRS + big.T
 
 
 def test_noalloc_permute_rejects_sizes_beyond_its_array():
