@@ -19,7 +19,8 @@ cudaError_t launch_tensor_ffn(const Dims& D, const uint16_t* xg, uint16_t* h, co
                               const int32_t* offsets, const int32_t* sorted_pair, const float* topk_w,
                               const moe_weights* w,
                               uint16_t* y_rows, int32_t* counters, uint32_t* err, uint64_t wait_ns,
-                              const long long* units_a, const long long* units_b, cudaStream_t s);
+                              const long long* units_a, const long long* units_b, const uint16_t* x_fused,
+                              const int32_t* sorted_token, cudaStream_t s);
 cudaError_t launch_convert_bf16_f16(const uint16_t* src, uint16_t* dst, int64_t n, uint32_t* err, cudaStream_t s);
 cudaError_t launch_stream_ffn(const Dims& D, const uint16_t* xg, uint16_t* h, float* part, const int32_t* offsets,
                               const int32_t* stream_list, const int32_t* n_stream, const int32_t* sorted_pair,
@@ -201,6 +202,27 @@ static bool tiles_needed(const Dims& D) {
     return true;
 }
 
+// x small enough to stay in L2 while the rows are gathered.
+static bool x_in_l2(const Dims& D) { return int64_t(D.T) * D.d * 2 <= (int64_t(64) << 20); }
+
+// The bf16 gate/up on one SM per tile gathers its rows itself (no gather kernel)
+// when x sits in L2 and no expert streams (the streaming kernels read the
+// gathered copy).
+static bool gather_fused(const Dims& D) {
+    const bool streaming = D.variant != MOE_VARIANT_TENSOR && D.stream_max_rows > 0;
+    return kFusedGather && D.fmt == MOE_WEIGHTS_BF16 && !D.tile_pair && x_in_l2(D) && !streaming && tiles_needed(D);
+}
+
+UnitOrder unit_order_for(const Dims& D, const WsLayout& L, uint8_t* ws) {
+    UnitOrder o{D.fmt == MOE_WEIGHTS_Q4G32 ? 2 : 1, (D.f + 127) / 128, (D.d + 255) / 256, kUnitOrderChunk, nullptr,
+                nullptr};
+    if (!D.tile_pair && tiles_needed(D)) {
+        o.units_a = reinterpret_cast<long long*>(ws + L.units_a);
+        o.units_b = reinterpret_cast<long long*>(ws + L.units_b);
+    }
+    return o;
+}
+
 cudaError_t launch_expert_ffn(const Dims& D, const WsLayout& L, const FfnArgs& a, cudaStream_t s) {
     uint8_t* ws = a.ws;
     int32_t* tile_base = reinterpret_cast<int32_t*>(ws + L.tile_base);
@@ -210,15 +232,10 @@ cudaError_t launch_expert_ffn(const Dims& D, const WsLayout& L, const FfnArgs& a
     uint16_t* h = reinterpret_cast<uint16_t*>(ws + L.h);
     float* part = L.part ? reinterpret_cast<float*>(ws + L.part) : nullptr;
     cudaError_t e = cudaSuccess;
-    // The claim order of the one-SM tile kernels (schedule.cu); the fused small-batch front
-    // kernel and the SM-pair kernels keep the natural order.
-    UnitOrder order{D.fmt == MOE_WEIGHTS_Q4G32 ? 2 : 1, (D.f + 127) / 128, (D.d + 255) / 256, kUnitOrderChunk,
-                    nullptr, nullptr};
-    const bool ordered = !a.scheduled && !D.tile_pair && tiles_needed(D);
-    if (ordered) {
-        order.units_a = reinterpret_cast<long long*>(ws + L.units_a);
-        order.units_b = reinterpret_cast<long long*>(ws + L.units_b);
-    }
+    // The claim order of the one-SM tile kernels (schedule.cu), written by the schedule kernel
+    // or by the permutation's scan; the fused small-batch front kernel keeps the natural order.
+    UnitOrder order = unit_order_for(D, L, ws);
+    if (a.scheduled && !a.units_written) order.units_a = order.units_b = nullptr;
     if (!a.scheduled &&
         (e = launch_schedule(D, a.offsets, tile_base, stream_list, n_stream, a.err, order, s)) != cudaSuccess)
         return e;
@@ -229,14 +246,15 @@ cudaError_t launch_expert_ffn(const Dims& D, const WsLayout& L, const FfnArgs& a
     // token order so that each x row is read from HBM once instead of k times
     // (Q4G32 workload: 234 against 326 us); with x in L2 the row-order gather,
     // which spreads small batches over more threads, is faster.
-    const bool token_order = a.pair_row && int64_t(D.T) * D.d * 2 > (int64_t(64) << 20);
-    if ((e = token_order ? launch_scatter_rows(D, a.x, a.pair_row, a.offsets, xg, a.err, s)
-                         : launch_gather(D, a.x, a.sorted_token, a.offsets, xg, a.err, s)) != cudaSuccess)
+    const bool token_order = a.pair_row && !x_in_l2(D);
+    const bool fused = gather_fused(D);
+    if (!fused && (e = token_order ? launch_scatter_rows(D, a.x, a.pair_row, a.offsets, xg, a.err, s)
+                                   : launch_gather(D, a.x, a.sorted_token, a.offsets, xg, a.err, s)) != cudaSuccess)
         return e;
     if (tiles_needed(D)) {
         if ((e = launch_tensor_ffn(D, xg, h, tile_base, a.offsets, a.sorted_pair, a.topk_w, a.w, a.y_rows,
-                                   n_stream + 1, a.err, a.wait_ns, order.units_a, order.units_b, s)) !=
-            cudaSuccess)
+                                   n_stream + 1, a.err, a.wait_ns, order.units_a, order.units_b,
+                                   fused ? a.x : nullptr, a.sorted_token, s)) != cudaSuccess)
             return e;
     }
     if (D.variant != MOE_VARIANT_TENSOR && D.stream_max_rows > 0) {
@@ -383,7 +401,7 @@ int moe_expert_ffn(const moe_params* p, const uint16_t* x, const int32_t* offset
     if (!al16(x) || !al16(y_rows)) return MOE_ERR_MISALIGNED;
     const WsLayout L = ws_layout(D, MOE_WS_EXPERT_FFN);
     FfnArgs a{x, offsets, sorted_token, sorted_pair, topk_w, w, y_rows, static_cast<uint8_t*>(ws),
-              static_cast<uint32_t*>(ws), g_wait_ns.load(), false, nullptr};
+              static_cast<uint32_t*>(ws), g_wait_ns.load(), false, nullptr, false};
     return status_of(launch_expert_ffn(D, L, a, stream));
 }
 
@@ -423,12 +441,18 @@ static int forward_impl(const Dims& D, const WsLayout& L, const uint16_t* x, con
     } else {
         e = launch_route(logits, D.T, D.E, D.k, topk_idx, topk_w, stream);
         if (e != cudaSuccess) return MOE_ERR_CUDA;
+        // the permutation's scan also writes the tile schedule and the claim orders
+        const UnitOrder o = unit_order_for(D, L, ws);
+        const ScheduleArgs sa{reinterpret_cast<int32_t*>(ws + L.tile_base), reinterpret_cast<int32_t*>(ws + L.stream_list),
+                              reinterpret_cast<int32_t*>(ws + L.n_stream), D.variant, D.stream_max_rows, o.sub, o.nt_a,
+                              o.nt_b, o.chunk, o.units_a, o.units_b};
         e = launch_permute(D, topk_idx, reinterpret_cast<int32_t*>(ws + L.blockcounts),
                            reinterpret_cast<int32_t*>(ws + L.blockbase), counts, kept, offsets, sorted_token,
-                           sorted_pair, pair_row, err, stream);
+                           sorted_pair, pair_row, err, stream, &sa);
         if (e != cudaSuccess) return MOE_ERR_CUDA;
     }
-    FfnArgs a{x, offsets, sorted_token, sorted_pair, topk_w, w, y_rows, ws, err, g_wait_ns.load(), front, pair_row};
+    FfnArgs a{x, offsets, sorted_token, sorted_pair, topk_w, w, y_rows, ws, err, g_wait_ns.load(), true, pair_row,
+              !front};
     if ((e = launch_expert_ffn(D, L, a, stream)) != cudaSuccess) return MOE_ERR_CUDA;
     if ((e = launch_combine(D, y_rows, pair_row, offsets, out, stream)) != cudaSuccess) return MOE_ERR_CUDA;
     if (counts_out &&
@@ -543,7 +567,7 @@ int moe_launch_count(const moe_params* p, int which, int* n) {
         return MOE_OK;
     }
     int ffn = 1;  // schedule
-    ffn += 1;                                       // gather
+    if (!gather_fused(D)) ffn += 1;                 // gather
     if (tiles_needed(D)) ffn += 2;                  // two tcgen05 GEMMs
     if (D.variant != MOE_VARIANT_TENSOR && D.stream_max_rows > 0) ffn += 2 + (D.ks > 1 ? 1 : 0);
     switch (which) {
@@ -554,7 +578,9 @@ int moe_launch_count(const moe_params* p, int which, int* n) {
         case MOE_WS_ROUTE_STATS: *n = 2; break;
         // schedule, gather, transpose, 6 GEMMs, zeroing, combine, reduce (+ dlogits: not counted)
         case MOE_WS_BACKWARD: *n = 12; break;
-        default: *n = D.T <= kFrontMaxTokens ? 1 + (ffn - 1) + 1 : 1 + 3 + ffn + 1; break;
+        // moe_forward: the front kernel(s) write the schedule, so the expert FFN's own
+        // schedule launch is not made
+        default: *n = D.T <= kFrontMaxTokens ? 1 + (ffn - 1) + 1 : 1 + 3 + (ffn - 1) + 1; break;
     }
     return MOE_OK;
 }

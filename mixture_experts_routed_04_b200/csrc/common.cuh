@@ -173,6 +173,18 @@ MOE_DEV void tma_load_3d(void* dst, const CUtensorMap* m, uint64_t* bar, int32_t
         : "memory");
 }
 
+// 16-byte asynchronous copy global -> shared (L2 only); src_bytes < 16 fills the
+// rest with zeros (0: nothing is read).
+MOE_DEV void cp_async_16(uint32_t dst, const void* src, uint32_t src_bytes) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "r"(src_bytes) : "memory");
+}
+MOE_DEV void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+// Wait until at most N of this thread's committed groups are still in flight.
+template <int N>
+MOE_DEV void cp_async_wait() {
+    asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
+}
+
 // Bring a tile into L2 ahead of its load (no shared memory, no completion signal).
 MOE_DEV void tma_prefetch_l2_4d(const CUtensorMap* m, int32_t x, int32_t y, int32_t z, int32_t w) {
     asm volatile("cp.async.bulk.prefetch.tensor.4d.L2.global.tile [%0, {%1, %2, %3, %4}];" ::"l"(

@@ -47,7 +47,10 @@ namespace moe {
 namespace tc {
 
 // WF: weight form. 0 = bf16 as given, 1 = Q4G32, 2 = fp16 (W_down prepared at load time).
-template <int MODE, int WF, int SUB>
+// GATHER (bf16 gate/up, one SM per 128-row tile only): four gather warps copy the
+// A rows straight from x (cp.async, 16 bytes a lane, into the 128-byte-swizzled
+// tile) instead of TMA loads of a gathered copy.
+template <int MODE, int WF, int SUB, bool GATHER = false>
 struct Cfg {
     static constexpr bool Q4 = WF == 1;
     static constexpr bool kTransform = Q4 || (MODE == 1 && WF == 0);
@@ -63,15 +66,17 @@ struct Cfg {
     // transform warps: 8 for Q4G32 (the dequantisation sits between the copy and
     // the MMA of every stage; measured 2% faster than 4), 4 for the bf16 -> fp16 pass
     static constexpr int kTransWarps = kTransform ? (Q4 ? 8 : 4) : 0;
-    static constexpr int kThreads = 32 * (2 + kEpiWarps + kTransWarps);
+    static constexpr int kGatherWarps = GATHER ? 4 : 0;
+    static_assert(!GATHER || (MODE == 0 && WF == 0 && SUB == 1), "gather warps: bf16 gate/up, 128-row units");
+    static constexpr int kThreads = 32 * (2 + kEpiWarps + kTransWarps + kGatherWarps);
     static constexpr int kABytes = kSub * A_BYTES;
     static constexpr int kStages = (Q4 || kSub == 2) ? 3 : 4;
     static constexpr int kStageBytes = Q4 ? kABytes + B_BYTES + P_BYTES + S_BYTES : kABytes + B_BYTES;
     // bytes a stage receives besides its A sub-tiles (A_BYTES each)
     static constexpr uint32_t kTxB = Q4 ? P_BYTES + S_BYTES : B_BYTES;
     static constexpr int kSmem = 1024 + kStages * kStageBytes + 512;  // + barriers, unit ring
-    // warps that read the unit ring: MMA, epilogue, transform
-    static constexpr int kUnitReaders = 1 + kEpiWarps + kTransWarps;
+    // warps that read the unit ring: MMA, epilogue, transform, gather
+    static constexpr int kUnitReaders = 1 + kEpiWarps + kTransWarps + kGatherWarps;
     // bf16 operands for the bf16 gate/up; fp16 otherwise. B is N-major (bf16
     // weights as stored) or K-major (dequantised from the K-major Q4G32 rows).
     static constexpr uint32_t kIdesc =
@@ -122,12 +127,12 @@ MOE_DEV uint4 dequant_word(uint32_t w, uint32_t s2) {
 }
 
 
-template <int MODE, int WF, int SUB>
-__global__ void __launch_bounds__(Cfg<MODE, WF, SUB>::kThreads, 1)
+template <int MODE, int WF, int SUB, bool GATHER = false>
+__global__ void __launch_bounds__(Cfg<MODE, WF, SUB, GATHER>::kThreads, 1)
     grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB0,
                         const __grid_constant__ CUtensorMap tmB1, const __grid_constant__ CUtensorMap tmS0,
                         const __grid_constant__ CUtensorMap tmS1, const GemmParams p) {
-    using C = Cfg<MODE, WF, SUB>;
+    using C = Cfg<MODE, WF, SUB, GATHER>;
     constexpr bool Q4 = C::Q4;
     constexpr int STAGES = C::kStages, SB = C::kStageBytes;
     extern __shared__ uint8_t smem_raw[];
@@ -147,7 +152,7 @@ __global__ void __launch_bounds__(Cfg<MODE, WF, SUB>::kThreads, 1)
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     if (threadIdx.x == 0) {
         for (int s = 0; s < STAGES; ++s) {
-            mbar_init(full + s, 1);
+            mbar_init(full + s, 1 + C::kGatherWarps);  // the producer's byte count (+ one arrival per gather warp)
             mbar_init(conv + s, 32 * C::kTransWarps);
             mbar_init(empty + s, 1);
         }
@@ -218,8 +223,8 @@ __global__ void __launch_bounds__(Cfg<MODE, WF, SUB>::kThreads, 1)
                     uint8_t* sa = smem + stage * SB;
                     uint8_t* sb = sa + C::kABytes;
                     const bool a1 = C::kSub == 2 && U.rows > BM;  // second 128-row sub-tile present
-                    mbar_arrive_expect_tx(full + stage, C::kTxB + (a1 ? 2u : 1u) * A_BYTES);
-                    tma_load_2d(sa, &tmA, full + stage, kb * BK, U.row0);
+                    mbar_arrive_expect_tx(full + stage, C::kTxB + (GATHER ? 0u : (a1 ? 2u : 1u) * A_BYTES));
+                    if (!GATHER) tma_load_2d(sa, &tmA, full + stage, kb * BK, U.row0);
                     if (a1) tma_load_2d(sa + A_BYTES, &tmA, full + stage, kb * BK, U.row0 + BM);
                     if (Q4) {
                         // packed rows [N][32 B] and scales [2 groups][rows] fp16
@@ -381,6 +386,79 @@ __global__ void __launch_bounds__(Cfg<MODE, WF, SUB>::kThreads, 1)
             }
         }
         if (range_bad) set_error(p.err, MOE_DEVERR_RANGE);
+    } else if (GATHER) {
+        // ------------------------------------------------ gather (the last 4 warps)
+        // Warp gw copies tile rows 32gw..32gw+31: lane = (row 4i + lane/8 of the
+        // warp's 32, 16-byte chunk lane%8 of the row's 128 bytes), so one
+        // instruction moves four whole 128-byte rows. A stage is released to
+        // the MMA one stage later: after the next stage's copies are issued,
+        // wait for the older group, make it visible to the tensor core (proxy
+        // fence) and arrive on its full barrier. Rows past the unit's end are
+        // zero-filled.
+        const int gw = warp - (2 + C::kEpiWarps);
+        const int cch = lane & 7;
+        int stage = 0, prev = -1;
+        uint32_t phase = 0;
+        bool ok = true;
+        int uslot = 0;
+        uint32_t uphase = 0;
+        bool bad = false;
+        while (ok) {
+            int u = -1;
+            if (!ring_read(u, uslot, uphase, unit_ring, ufull, uempty, abort_flag, p.err, p.wait_ns)) break;
+            if (u < 0) break;
+            const Unit U = decode_unit<1>(u, p, nt);
+            const uint16_t* src[8];
+            uint32_t nbytes[8];
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+                const int r = 32 * gw + 4 * i + (lane >> 3);
+                src[i] = p.x;
+                nbytes[i] = 0;
+                if (r < U.rows) {
+                    const int t = __ldg(p.sorted_token + U.row0 + r);
+                    if (t >= 0 && t < p.T) {
+                        src[i] = p.x + int64_t(t) * p.K + cch * 8;
+                        nbytes[i] = 16;
+                    } else {
+                        bad = true;
+                    }
+                }
+            }
+            for (int kb = 0; kb < KB; ++kb) {
+                int okl = 1;
+                if (lane == 0) okl = mbar_wait_bounded(empty + stage, phase ^ 1u, abort_flag, p.err, p.wait_ns);
+                okl = __shfl_sync(0xFFFFFFFFu, okl, 0);
+                if (!okl) {
+                    ok = false;
+                    break;
+                }
+                const uint32_t sa = smem_u32(smem + stage * SB);
+#pragma unroll
+                for (int i = 0; i < 8; ++i) {
+                    const int r = 32 * gw + 4 * i + (lane >> 3);
+                    cp_async_16(sa + r * 128 + ((cch ^ (r & 7)) << 4), src[i] + kb * BK, nbytes[i]);
+                }
+                cp_async_commit();
+                if (prev >= 0) {
+                    cp_async_wait<1>();
+                    fence_proxy_async_smem();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(full + prev);
+                }
+                prev = stage;
+                if (++stage == STAGES) {
+                    stage = 0;
+                    phase ^= 1u;
+                }
+            }
+        }
+        // the last stage (or, after an abort, every copy in flight) lands before exit
+        cp_async_wait<0>();
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (ok && prev >= 0 && lane == 0) mbar_arrive(full + prev);
+        if (bad) set_error(p.err, MOE_DEVERR_BOUNDS);
     } else if (C::kTransform) {
         // ------------------------------------------------ transform (the last kTransWarps warps)
         const int ct = threadIdx.x - 32 * (2 + C::kEpiWarps);  // 0 .. 32*kTransWarps-1
@@ -541,15 +619,15 @@ bool map_q4_scales(CUtensorMap* m, const void* base, int nexp, int K, int N, int
     return make_map(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, base, 3, dims, str, box, CU_TENSOR_MAP_SWIZZLE_NONE);
 }
 
-template <int MODE, int WF, int SUB>
+template <int MODE, int WF, int SUB, bool GATHER = false>
 cudaError_t launch_gemm(const CUtensorMap& A, const CUtensorMap& B0, const CUtensorMap& B1, const CUtensorMap& S0,
                         const CUtensorMap& S1, const GemmParams& p, bool pdl, cudaStream_t s) {
-    using C = Cfg<MODE, WF, SUB>;
+    using C = Cfg<MODE, WF, SUB, GATHER>;
     static int configured_dev = -1;
     int dev = 0;
     cudaGetDevice(&dev);
     if (configured_dev != dev) {
-        cudaError_t e = cudaFuncSetAttribute(grouped_gemm_kernel<MODE, WF, SUB>,
+        cudaError_t e = cudaFuncSetAttribute(grouped_gemm_kernel<MODE, WF, SUB, GATHER>,
                                              cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmem);
         if (e != cudaSuccess) return e;
         configured_dev = dev;
@@ -558,7 +636,7 @@ cudaError_t launch_gemm(const CUtensorMap& A, const CUtensorMap& B0, const CUten
     if (C::kSub == 2) q.tile_base = p.tile_base + p.Etot + 1;  // 256-row units
     {
         ProfScope prof_(MODE == 0 ? MOE_K_TC_GATEUP : MOE_K_TC_DOWN, s);
-        const cudaError_t le = launch_pdl(pdl, grouped_gemm_kernel<MODE, WF, SUB>, dim3(num_sms()), dim3(C::kThreads),
+        const cudaError_t le = launch_pdl(pdl, grouped_gemm_kernel<MODE, WF, SUB, GATHER>, dim3(num_sms()), dim3(C::kThreads),
                                           C::kSmem, s, A, B0, B1, S0, S1, q);
         if (le != cudaSuccess) return le;
     }
@@ -573,7 +651,8 @@ cudaError_t launch_tensor_ffn(const Dims& D, const uint16_t* xg, uint16_t* h, co
                               const int32_t* offsets,
                               const int32_t* sorted_pair, const float* topk_w, const moe_weights* w,
                               uint16_t* y_rows, int32_t* counters, uint32_t* err, uint64_t wait_ns,
-                              const long long* units_a, const long long* units_b, cudaStream_t s) {
+                              const long long* units_a, const long long* units_b, const uint16_t* x_fused,
+                              const int32_t* sorted_token, cudaStream_t s) {
     using namespace tc;
     const bool pdl = use_pdl(D.T);
     GemmParams p{};
@@ -631,7 +710,11 @@ cudaError_t launch_tensor_ffn(const Dims& D, const uint16_t* xg, uint16_t* h, co
     p.out = h;
     p.unit_counter = counters;
     p.units = D.tile_pair ? nullptr : units_a;
+    p.x = x_fused;
+    p.sorted_token = sorted_token;
+    p.T = D.T;
     e = D.tile_pair ? launch_gemm_pair<0>(mA, mG, mU, mSG, mSU, p, pdl, s)
+        : x_fused   ? launch_gemm<0, 0, 1, true>(mA, mG, mU, mSG, mSU, p, pdl, s)
                     : launch_gemm<0, 0, 1>(mA, mG, mU, mSG, mSU, p, pdl, s);
     if (e != cudaSuccess) return e;
     // S6: down + gate scale -> y_rows

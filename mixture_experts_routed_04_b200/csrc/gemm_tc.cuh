@@ -37,6 +37,11 @@ struct GemmParams {
     // (expert << 48 | n-tile << 32 | m-tile). Null: the natural order, expert by
     // expert, each n-tile's M-tiles in turn.
     const long long* units;
+    // Rows gathered inside the gate/up GEMM (GATHER kernels): A row r of expert
+    // rows is x[sorted_token[r]], x [T, d] bf16.
+    const uint16_t* x;
+    const int32_t* sorted_token;
+    int T;
 };
 
 struct Unit {

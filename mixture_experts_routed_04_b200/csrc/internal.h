@@ -60,9 +60,21 @@ cudaError_t launch_route_stats(const float* logits, int T, int E, int k, int32_t
                                float* expert_stats, float* part_p, int32_t* part_c, float* part_s,
                                cudaStream_t stream);
 
+// The tile schedule (K3) and the claim orders, when the permutation's scan
+// kernel runs them too (moe_forward with more than kFrontMaxTokens tokens).
+struct ScheduleArgs {
+    int32_t* tile_base;
+    int32_t* stream_list;
+    int32_t* n_stream;
+    int variant, stream_max;
+    int sub, nt_a, nt_b, chunk;
+    long long* units_a;
+    long long* units_b;
+};
 cudaError_t launch_permute(const Dims& D, const int32_t* topk_idx, int32_t* blockcounts, int32_t* blockbase,
                            int32_t* counts, int32_t* kept, int32_t* offsets, int32_t* sorted_token,
-                           int32_t* sorted_pair, int32_t* pair_row, uint32_t* err, cudaStream_t s);
+                           int32_t* sorted_pair, int32_t* pair_row, uint32_t* err, cudaStream_t s,
+                           const ScheduleArgs* sched = nullptr);
 
 // Batches of at most this many tokens run routing, permutation and the tile
 // schedule as one fused single-block kernel (front.cu).
@@ -82,6 +94,8 @@ struct UnitOrder {
 };
 // Groups (expert, n-tile) per chunk of the claim order.
 constexpr int kUnitOrderChunk = 32;
+// The bf16 gate/up GEMM gathers its rows from x itself (no gathered copy).
+constexpr bool kFusedGather = false;
 
 struct FfnArgs {
     const uint16_t* x;
@@ -94,9 +108,13 @@ struct FfnArgs {
     uint8_t* ws;
     uint32_t* err;
     uint64_t wait_ns;
-    bool scheduled;            // the fused front kernel already wrote the tile schedule
+    bool scheduled;            // the front kernels already wrote the tile schedule
     const int32_t* pair_row;   // moe_forward: row of each pair (-1 dropped), for the token-order row copy
+    bool units_written;        // ... and the claim orders (the permutation's scan did)
 };
+// The claim orders a layer's tile GEMMs use, with their workspace arrays (null
+// pointers: the natural order, for the SM-pair kernels or when no tile runs).
+UnitOrder unit_order_for(const Dims& D, const WsLayout& L, uint8_t* ws);
 cudaError_t launch_expert_ffn(const Dims& D, const WsLayout& L, const FfnArgs& a, cudaStream_t s);
 
 cudaError_t launch_combine(const Dims& D, const uint16_t* y_rows, const int32_t* pair_row, const int32_t* offsets,

@@ -22,7 +22,7 @@
 // The rank of a pair is the number of earlier pairs with the same expert, so
 // the result is unique and bit-exact. The shared expert, when present, is
 // appended as expert E holding tokens 0..T-1.
-#include "internal.h"
+#include "schedule.cuh"
 
 namespace moe {
 
@@ -41,16 +41,24 @@ MOE_DEV void warp_histograms(const int32_t* __restrict__ topk_idx, int64_t pairs
     for (int i = threadIdx.x; i < kPermWarps * kMaxE; i += blockDim.x) (&hist[0][0])[i] = 0;
     __syncthreads();
     const int64_t base = int64_t(blockIdx.x) * kPermPairsPerBlock + int64_t(w) * kPermPairsPerWarp;
+    // every round's ids first (one memory latency for the warp's 256 pairs)
+    int ids[kPermPairsPerWarp / 32];
+#pragma unroll
     for (int it = 0; it < kPermPairsPerWarp / 32; ++it) {
         const int64_t p = base + it * 32 + lane;
         int e = -1;
         if (p < pairs) {
-            e = topk_idx[p];
+            e = __ldg(topk_idx + p);
             if (e < 0 || e >= E) {
                 set_error(err, MOE_DEVERR_BOUNDS);
                 e = -1;
             }
         }
+        ids[it] = e;
+    }
+#pragma unroll
+    for (int it = 0; it < kPermPairsPerWarp / 32; ++it) {
+        const int e = ids[it];
         const uint32_t peers = __match_any_sync(0xFFFFFFFFu, e);
         if (e >= 0 && (__ffs(peers) - 1) == lane) hist[w][e] += __popc(peers);
         __syncwarp();
@@ -74,17 +82,23 @@ __global__ void __launch_bounds__(kPermWarps * 32) perm_count_kernel(const int32
     }
 }
 
-// One block of 256 threads: thread e owns expert e.
-__global__ void __launch_bounds__(kMaxE) perm_scan_kernel(const int32_t* __restrict__ blockcounts, int nblocks,
-                                                         int E, int cap, int shared_T,
-                                                         int32_t* __restrict__ blockbase,
-                                                         int32_t* __restrict__ counts, int32_t* __restrict__ kept,
-                                                         int32_t* __restrict__ offsets) {
-    __shared__ int warp_sums[kMaxE / 32];
+// One block: thread e owns expert e (256 threads; 512 with SCHED). With SCHED
+// the block then runs the tile schedule and the claim orders of the tile GEMMs
+// on the kept counts it has just formed (the schedule kernel's work, without
+// a launch of its own).
+template <bool SCHED>
+__global__ void __launch_bounds__(SCHED ? 512 : kMaxE)
+    perm_scan_kernel(const int32_t* __restrict__ blockcounts, int nblocks, int E, int cap, int shared_T,
+                     int32_t* __restrict__ blockbase, int32_t* __restrict__ counts, int32_t* __restrict__ kept,
+                     int32_t* __restrict__ offsets, ScheduleArgs sa) {
+    __shared__ int warp_sums[16];
+    __shared__ int sums[3][16];
+    __shared__ int s_tb[kMaxE + 2], s_ne[kMaxE + 2];
     griddep_wait();
     griddep_launch();
 
     const int e = threadIdx.x, lane = e & 31, w = e >> 5;
+    const int nw = blockDim.x >> 5;
     int kv = 0;
     if (e < E) {
         int run = 0;
@@ -107,8 +121,7 @@ __global__ void __launch_bounds__(kMaxE) perm_scan_kernel(const int32_t* __restr
     if (lane == 31) warp_sums[w] = incl;
     __syncthreads();
     int wbase = 0, total = 0;
-#pragma unroll
-    for (int i = 0; i < kMaxE / 32; ++i) {
+    for (int i = 0; i < nw; ++i) {
         if (i < w) wbase += warp_sums[i];
         total += warp_sums[i];
     }
@@ -122,6 +135,14 @@ __global__ void __launch_bounds__(kMaxE) perm_scan_kernel(const int32_t* __restr
         } else {
             offsets[E] = total;
         }
+    }
+    if (SCHED) {
+        const int Etot = E + (shared_T > 0 ? 1 : 0);
+        const int ke = e < E ? kv : (e == E && shared_T > 0 ? shared_T : 0);
+        schedule_block(ke, Etot, sa.variant, sa.stream_max, sums, sa.tile_base, sa.stream_list, sa.n_stream);
+        if (sa.units_a)
+            unit_orders_block(sa.tile_base, Etot, sa.sub, sa.nt_a, sa.nt_b, sa.chunk, sa.units_a, sa.units_b, s_tb,
+                              s_ne, sums);
     }
 }
 
@@ -147,13 +168,21 @@ __global__ void __launch_bounds__(kPermWarps * 32) perm_scatter_kernel(
     __syncthreads();
     const int w = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int64_t base = int64_t(blockIdx.x) * kPermPairsPerBlock + int64_t(w) * kPermPairsPerWarp;
+    int ids[kPermPairsPerWarp / 32];
+#pragma unroll
     for (int it = 0; it < kPermPairsPerWarp / 32; ++it) {
         const int64_t p = base + it * 32 + lane;
         int e = -1;
         if (p < pairs) {
-            e = topk_idx[p];
+            e = __ldg(topk_idx + p);
             if (e < 0 || e >= E) e = -1;
         }
+        ids[it] = e;
+    }
+#pragma unroll
+    for (int it = 0; it < kPermPairsPerWarp / 32; ++it) {
+        const int64_t p = base + it * 32 + lane;
+        const int e = ids[it];
         const uint32_t peers = __match_any_sync(0xFFFFFFFFu, e);
         int rank = 0;
         if (e >= 0) rank = hist[w][e] + __popc(peers & lanemask_lt());
@@ -186,7 +215,8 @@ __global__ void __launch_bounds__(kPermWarps * 32) perm_scatter_kernel(
 
 cudaError_t launch_permute(const Dims& D, const int32_t* topk_idx, int32_t* blockcounts, int32_t* blockbase,
                            int32_t* counts, int32_t* kept, int32_t* offsets, int32_t* sorted_token,
-                           int32_t* sorted_pair, int32_t* pair_row, uint32_t* err, cudaStream_t s) {
+                           int32_t* sorted_pair, int32_t* pair_row, uint32_t* err, cudaStream_t s,
+                           const ScheduleArgs* sched) {
     if (D.pairs == 0) {  // empty batch: zero counts and offsets, nothing to scatter
         if (cudaMemsetAsync(counts, 0, size_t(D.Etot) * 4, s) != cudaSuccess ||
             cudaMemsetAsync(kept, 0, size_t(D.Etot) * 4, s) != cudaSuccess ||
@@ -204,8 +234,12 @@ cudaError_t launch_permute(const Dims& D, const int32_t* topk_idx, int32_t* bloc
     }
     {
         ProfScope prof_(MOE_K_PERM_SCAN, s);
-        const cudaError_t le = launch_pdl(use_pdl(D.T), perm_scan_kernel, dim3(1), dim3(kMaxE), 0, s, blockcounts, nb,
-                                          D.E, D.cap, shared_T, blockbase, counts, kept, offsets);
+        const ScheduleArgs none{};
+        const cudaError_t le =
+            sched ? launch_pdl(use_pdl(D.T), perm_scan_kernel<true>, dim3(1), dim3(512), 0, s, blockcounts, nb, D.E,
+                               D.cap, shared_T, blockbase, counts, kept, offsets, *sched)
+                  : launch_pdl(use_pdl(D.T), perm_scan_kernel<false>, dim3(1), dim3(kMaxE), 0, s, blockcounts, nb,
+                               D.E, D.cap, shared_T, blockbase, counts, kept, offsets, none);
         if (le != cudaSuccess) return le;
     }
     {
