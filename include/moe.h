@@ -445,13 +445,16 @@ typedef struct moe_grads {
  *   expert's rows; d w[t,j] = <dout[t], y[t,j]>; dlogits_j = w_j (dw_j -
  *   sum_i w_i dw_i).
  * Inputs are the forward's: x bf16 [T, d]; topk_idx, topk_w (moe_route);
- * offsets, sorted_token, sorted_pair, pair_row (moe_permute); weights bf16 as
- * for moe_forward (W_down bf16: down_dtype MOE_DOWN_BF16; Q4G32 is not
- * supported); dout fp32 [T, d]. g: see moe_grads.
- * Arithmetic: bf16 operands, fp32 accumulation on the tcgen05 tensor cores;
- * g and u are recomputed (fp32) and h, dg, du rounded to bf16 once.
+ * offsets, sorted_token, sorted_pair, pair_row (moe_permute); weights as for
+ * moe_forward with down_dtype MOE_DOWN_F16: bf16 W_gate, W_up and the fp16
+ * copy of W_down (and of the shared expert's) that moe_convert_bf16_to_f16
+ * prepares; dout fp32 [T, d]. g: see moe_grads.
+ * Arithmetic on the tcgen05 tensor cores with fp32 accumulation: g and u are
+ * recomputed in fp32; products with the bf16 gate/up weights take bf16
+ * operands (x; dg, du rounded once), the product with W_down and the weight
+ * gradients take fp16 operands (dout rows, h, dg, du rounded once).
  * ws: MOE_WS_BACKWARD bytes. Returns MOE_ERR_UNSUPPORTED for Q4G32 weights or
- * fp16 W_down. Deterministic (no atomics decide a sum).
+ * a bf16 W_down. Deterministic (no atomics decide a sum).
  */
 MOE_API int moe_expert_ffn_backward(const moe_params* p, const uint16_t* x, const int32_t* topk_idx,
               const float* topk_w, const int32_t* offsets, const int32_t* sorted_token,

@@ -10,7 +10,7 @@
 namespace moe {
 
 cudaError_t launch_schedule(const Dims& D, const int32_t* offsets, int32_t* tile_base, int32_t* stream_list,
-                            int32_t* n_stream, uint32_t* err, const UnitOrder& order, cudaStream_t s);
+                            int32_t* n_stream, uint32_t* err, cudaStream_t s);
 cudaError_t launch_gather(const Dims& D, const uint16_t* x, const int32_t* sorted_token, const int32_t* offsets,
                           uint16_t* xg, uint32_t* err, cudaStream_t s);
 cudaError_t launch_scatter_rows(const Dims& D, const uint16_t* x, const int32_t* pair_row, const int32_t* offsets,
@@ -19,8 +19,7 @@ cudaError_t launch_tensor_ffn(const Dims& D, const uint16_t* xg, uint16_t* h, co
                               const int32_t* offsets, const int32_t* sorted_pair, const float* topk_w,
                               const moe_weights* w,
                               uint16_t* y_rows, int32_t* counters, uint32_t* err, uint64_t wait_ns,
-                              const long long* units_a, const long long* units_b, const uint16_t* x_fused,
-                              const int32_t* sorted_token, cudaStream_t s);
+                              const uint16_t* x_fused, const int32_t* sorted_token, cudaStream_t s);
 cudaError_t launch_convert_bf16_f16(const uint16_t* src, uint16_t* dst, int64_t n, uint32_t* err, cudaStream_t s);
 cudaError_t launch_stream_ffn(const Dims& D, const uint16_t* xg, uint16_t* h, float* part, const int32_t* offsets,
                               const int32_t* stream_list, const int32_t* n_stream, const int32_t* sorted_pair,
@@ -147,6 +146,7 @@ WsLayout ws_layout(const Dims& D, int which) {
         L.b_h = take(size_t(rp) * D.f * 2);
         L.b_hwT = take(size_t(rp) * D.f * 2);
         L.b_dgu = take(size_t(rp) * 2 * D.f * 2);
+        L.b_dgu16 = take(size_t(rp) * 2 * D.f * 2);
         L.b_dxr = take(size_t(D.rows) * D.d * 2);
         L.b_dwp = take(size_t(D.rows) * nt * 4);
     }
@@ -164,10 +164,6 @@ WsLayout ws_layout(const Dims& D, int which) {
         L.tile_base = take(size_t(D.Etot + 1) * 2 * 4);  // 128-row and 256-row tile prefixes
         L.stream_list = take(size_t(D.Etot) * 4);
         L.n_stream = take(16);  // [0] streaming experts, [1], [2] tile-unit counters
-        // claim orders: at most (ceil(rows / 128) + Etot) M-tiles of 128 rows, times the n-tiles
-        const size_t mtiles = size_t((D.rows + kTileM - 1) / kTileM) + D.Etot;
-        L.units_a = take(mtiles * size_t((D.f + 127) / 128) * 8);
-        L.units_b = take(mtiles * size_t((D.d + 255) / 256) * 8);
         L.xg = take(size_t(D.rows) * D.d * 2);
         L.h = take(size_t(D.rows) * D.f * 2);
         if (D.ks > 1) L.part = take(size_t(D.ks) * 2 * D.rows * D.f * 4);
@@ -213,16 +209,6 @@ static bool gather_fused(const Dims& D) {
     return kFusedGather && D.fmt == MOE_WEIGHTS_BF16 && !D.tile_pair && x_in_l2(D) && !streaming && tiles_needed(D);
 }
 
-UnitOrder unit_order_for(const Dims& D, const WsLayout& L, uint8_t* ws) {
-    UnitOrder o{D.fmt == MOE_WEIGHTS_Q4G32 ? 2 : 1, (D.f + 127) / 128, (D.d + 255) / 256, kUnitOrderChunk, nullptr,
-                nullptr};
-    if (!D.tile_pair && tiles_needed(D)) {
-        o.units_a = reinterpret_cast<long long*>(ws + L.units_a);
-        o.units_b = reinterpret_cast<long long*>(ws + L.units_b);
-    }
-    return o;
-}
-
 cudaError_t launch_expert_ffn(const Dims& D, const WsLayout& L, const FfnArgs& a, cudaStream_t s) {
     uint8_t* ws = a.ws;
     int32_t* tile_base = reinterpret_cast<int32_t*>(ws + L.tile_base);
@@ -232,12 +218,8 @@ cudaError_t launch_expert_ffn(const Dims& D, const WsLayout& L, const FfnArgs& a
     uint16_t* h = reinterpret_cast<uint16_t*>(ws + L.h);
     float* part = L.part ? reinterpret_cast<float*>(ws + L.part) : nullptr;
     cudaError_t e = cudaSuccess;
-    // The claim order of the one-SM tile kernels (schedule.cu), written by the schedule kernel
-    // or by the permutation's scan; the fused small-batch front kernel keeps the natural order.
-    UnitOrder order = unit_order_for(D, L, ws);
-    if (a.scheduled && !a.units_written) order.units_a = order.units_b = nullptr;
     if (!a.scheduled &&
-        (e = launch_schedule(D, a.offsets, tile_base, stream_list, n_stream, a.err, order, s)) != cudaSuccess)
+        (e = launch_schedule(D, a.offsets, tile_base, stream_list, n_stream, a.err, s)) != cudaSuccess)
         return e;
     // Rows in expert order for both variants (fp16 for Q4G32, whose MMAs run
     // in fp16). A TMA tile::gather4 of the rows inside the GEMM was measured
@@ -253,8 +235,8 @@ cudaError_t launch_expert_ffn(const Dims& D, const WsLayout& L, const FfnArgs& a
         return e;
     if (tiles_needed(D)) {
         if ((e = launch_tensor_ffn(D, xg, h, tile_base, a.offsets, a.sorted_pair, a.topk_w, a.w, a.y_rows,
-                                   n_stream + 1, a.err, a.wait_ns, order.units_a, order.units_b,
-                                   fused ? a.x : nullptr, a.sorted_token, s)) != cudaSuccess)
+                                   n_stream + 1, a.err, a.wait_ns, fused ? a.x : nullptr, a.sorted_token, s)) !=
+            cudaSuccess)
             return e;
     }
     if (D.variant != MOE_VARIANT_TENSOR && D.stream_max_rows > 0) {
@@ -401,7 +383,7 @@ int moe_expert_ffn(const moe_params* p, const uint16_t* x, const int32_t* offset
     if (!al16(x) || !al16(y_rows)) return MOE_ERR_MISALIGNED;
     const WsLayout L = ws_layout(D, MOE_WS_EXPERT_FFN);
     FfnArgs a{x, offsets, sorted_token, sorted_pair, topk_w, w, y_rows, static_cast<uint8_t*>(ws),
-              static_cast<uint32_t*>(ws), g_wait_ns.load(), false, nullptr, false};
+              static_cast<uint32_t*>(ws), g_wait_ns.load(), false, nullptr};
     return status_of(launch_expert_ffn(D, L, a, stream));
 }
 
@@ -441,18 +423,16 @@ static int forward_impl(const Dims& D, const WsLayout& L, const uint16_t* x, con
     } else {
         e = launch_route(logits, D.T, D.E, D.k, topk_idx, topk_w, stream);
         if (e != cudaSuccess) return MOE_ERR_CUDA;
-        // the permutation's scan also writes the tile schedule and the claim orders
-        const UnitOrder o = unit_order_for(D, L, ws);
-        const ScheduleArgs sa{reinterpret_cast<int32_t*>(ws + L.tile_base), reinterpret_cast<int32_t*>(ws + L.stream_list),
-                              reinterpret_cast<int32_t*>(ws + L.n_stream), D.variant, D.stream_max_rows, o.sub, o.nt_a,
-                              o.nt_b, o.chunk, o.units_a, o.units_b};
+        // the permutation's scan also writes the tile schedule
+        const ScheduleArgs sa{reinterpret_cast<int32_t*>(ws + L.tile_base),
+                              reinterpret_cast<int32_t*>(ws + L.stream_list),
+                              reinterpret_cast<int32_t*>(ws + L.n_stream), D.variant, D.stream_max_rows};
         e = launch_permute(D, topk_idx, reinterpret_cast<int32_t*>(ws + L.blockcounts),
                            reinterpret_cast<int32_t*>(ws + L.blockbase), counts, kept, offsets, sorted_token,
                            sorted_pair, pair_row, err, stream, &sa);
         if (e != cudaSuccess) return MOE_ERR_CUDA;
     }
-    FfnArgs a{x, offsets, sorted_token, sorted_pair, topk_w, w, y_rows, ws, err, g_wait_ns.load(), true, pair_row,
-              !front};
+    FfnArgs a{x, offsets, sorted_token, sorted_pair, topk_w, w, y_rows, ws, err, g_wait_ns.load(), true, pair_row};
     if ((e = launch_expert_ffn(D, L, a, stream)) != cudaSuccess) return MOE_ERR_CUDA;
     if ((e = launch_combine(D, y_rows, pair_row, offsets, out, stream)) != cudaSuccess) return MOE_ERR_CUDA;
     if (counts_out &&
@@ -523,7 +503,8 @@ int moe_expert_ffn_backward(const moe_params* p, const uint16_t* x, const int32_
     Dims D;
     int st = make_dims(p, &D);
     if (st != MOE_OK) return st;
-    if (D.fmt != MOE_WEIGHTS_BF16 || D.down_f16) return MOE_ERR_UNSUPPORTED;
+    // bf16 gate/up weights and the fp16 copy of W_down (moe_convert_bf16_to_f16)
+    if (D.fmt != MOE_WEIGHTS_BF16 || !D.down_f16) return MOE_ERR_UNSUPPORTED;
     // the transpose grid holds padded rows / 32 blocks in y (at most 65535)
     if (bwd_padded_rows(D) / 32 > 65535) return MOE_ERR_UNSUPPORTED;
     if ((st = check_ws(D, MOE_WS_BACKWARD, ws, ws_bytes)) != MOE_OK) return st;

@@ -14,17 +14,21 @@
 // rows (poff[e] = padded offset), so the weight gradients, which contract
 // over an expert's rows, run whole 64-row k-blocks. Launches (one stream):
 //   bwd_schedule      padded offsets, tile prefixes, unit counters
-//   bwd_gather        xg = x rows, dog = dout rows (bf16), zero padding rows
-//   transpose         xgT = xg^T  [d, Rp]
-//   GEMM GU           x [Wg|Wu] -> g, u (fp32), h (bf16), (w h)^T (bf16)
-//   GEMM DH           dout_rows Wd^T -> dh = w dhu -> dg, du (bf16); <h, dhu>
+//   bwd_gather        xg = x rows (bf16), dog = dout rows (fp16), zero padding rows
+//   transpose         xgT = xg^T  [d, Rp] (fp16, exact for bf16 x in fp16's range)
+//   GEMM GU           x [Wg|Wu] -> g, u (fp32), h (fp16), (w h)^T (fp16)
+//   GEMM DH           dout_rows Wd^T -> dh = w dhu -> dg, du (bf16 and fp16); <h, dhu>
 //   GEMM DX           [dg|du] [Wg|Wu]^T -> dx rows (fp16, real row order)
 //   GEMM WG x3        dWd = (w h)^T dout_rows; dWg = xg^T dg; dWu = xg^T du
 //   zero_untouched    zero weight gradients of experts without rows
 //   combine           dx[t] = sum of its pairs' dx rows (+ shared)
 //   dw_reduce         d topk_w[p] = sum over n-tiles of <h, dhu>
 //   route_backward    dlogits (optional)
-// Every operand is bf16 with fp32 accumulation (TMEM). The GEMM kernel is the
+// Operands: GU and DX multiply the bf16 gate/up weights, so x and dg, du enter
+// them as bf16; DH multiplies the fp16 copy of W_down (prepared once, as for the
+// forward) by fp16 dout rows; the weight gradients multiply fp16 activations.
+// fp32 accumulation (TMEM) throughout. (All-bf16 operands measured 8x larger
+// weight-gradient errors: rounding dout and dg to 8 significant bits.) The GEMM kernel is the
 // forward kernel's structure (TMA producer warp, one-thread MMA issuer,
 // four epilogue warps, unit ring, bounded waits) with per-mode loads and
 // epilogues; A is always K-major, B K-major (weights read transposed: DH, DX)
@@ -70,9 +74,10 @@ struct Params {
     float limit;
     // outputs
     float* gu;         // [rp, 2f] g then u
-    uint16_t* h;       // [rp, f] bf16
-    uint16_t* hwT;     // [f, rp] bf16, w * h transposed
-    uint16_t* dgu;     // [rp, 2f] bf16, dg then du
+    uint16_t* h;       // [rp, f] fp16
+    uint16_t* hwT;     // [f, rp] fp16, w * h transposed
+    uint16_t* dgu;     // [rp, 2f] bf16, dg then du (operand of DX)
+    uint16_t* dgu16;   // [rp, 2f] fp16, the same (operand of the weight gradients)
     uint16_t* dxr;     // [rows, d] fp16, real row order
     float* dwp;        // [rows, n_tiles of DH] partial <h, dhu>
     float* dw;         // WG: routed experts' gradient [E, M, N]
@@ -193,9 +198,11 @@ MOE_DEV void epilogue(uint32_t tb, const Unit& U, int q, int lane, const Params&
                 for (int i = 0; i < 32; i += 2) {
                     const float h0 = tc::swiglu(__uint_as_float(g[i]), __uint_as_float(v[i]), L);
                     const float h1 = tc::swiglu(__uint_as_float(g[i + 1]), __uint_as_float(v[i + 1]), L);
-                    pk[i / 2] = pack_bf16x2(h0, h1);
-                    p.hwT[int64_t(col + i) * p.rp + prow] = uint16_t(f32_to_bf16_rne(w * h0));
-                    p.hwT[int64_t(col + i + 1) * p.rp + prow] = uint16_t(f32_to_bf16_rne(w * h1));
+                    range_bad |= !(f16_range_ok(h0) && f16_range_ok(h1));
+                    pk[i / 2] = pack_f16x2(h0, h1);
+                    const uint32_t wh = pack_f16x2(w * h0, w * h1);
+                    p.hwT[int64_t(col + i) * p.rp + prow] = uint16_t(wh & 0xFFFFu);
+                    p.hwT[int64_t(col + i + 1) * p.rp + prow] = uint16_t(wh >> 16);
                 }
                 uint4* hd = reinterpret_cast<uint4*>(p.h + prow * f + col);
 #pragma unroll
@@ -214,7 +221,7 @@ MOE_DEV void epilogue(uint32_t tb, const Unit& U, int q, int lane, const Params&
                 const float* gp = p.gu + prow * f2 + col;
                 const float* up = gp + f;
                 const uint32_t* hp = reinterpret_cast<const uint32_t*>(p.h + prow * f + col);
-                uint32_t pg[16], pu[16];
+                uint32_t pg[16], pu[16], qg[16], qu[16];
 #pragma unroll
                 for (int i = 0; i < 32; i += 2) {
                     const uint32_t hh = hp[i / 2];
@@ -222,7 +229,7 @@ MOE_DEV void epilogue(uint32_t tb, const Unit& U, int q, int lane, const Params&
 #pragma unroll
                     for (int s2 = 0; s2 < 2; ++s2) {
                         const float dhu = __uint_as_float(v[i + s2]);
-                        dot += (s2 ? bf16_hi(hh) : bf16_lo(hh)) * dhu;
+                        dot += (s2 ? f16_hi(hh) : f16_lo(hh)) * dhu;
                         const float gv = gp[i + s2], uv = up[i + s2];
                         const float gc = L > 0.f ? fminf(fmaxf(gv, -L), L) : gv;
                         const float uc = L > 0.f ? fminf(fmaxf(uv, -L), L) : uv;
@@ -236,13 +243,21 @@ MOE_DEV void epilogue(uint32_t tb, const Unit& U, int q, int lane, const Params&
                     }
                     pg[i / 2] = pack_bf16x2(dgv[0], dgv[1]);
                     pu[i / 2] = pack_bf16x2(duv[0], duv[1]);
+                    range_bad |= !(f16_range_ok(dgv[0]) && f16_range_ok(dgv[1]) && f16_range_ok(duv[0]) &&
+                                   f16_range_ok(duv[1]));
+                    qg[i / 2] = pack_f16x2(dgv[0], dgv[1]);
+                    qu[i / 2] = pack_f16x2(duv[0], duv[1]);
                 }
                 uint4* gd = reinterpret_cast<uint4*>(p.dgu + prow * f2 + col);
                 uint4* ud = reinterpret_cast<uint4*>(p.dgu + prow * f2 + f + col);
+                uint4* gq = reinterpret_cast<uint4*>(p.dgu16 + prow * f2 + col);
+                uint4* uq = reinterpret_cast<uint4*>(p.dgu16 + prow * f2 + f + col);
 #pragma unroll
                 for (int i = 0; i < 4; ++i) {
                     gd[i] = make_uint4(pg[4 * i], pg[4 * i + 1], pg[4 * i + 2], pg[4 * i + 3]);
                     ud[i] = make_uint4(pu[4 * i], pu[4 * i + 1], pu[4 * i + 2], pu[4 * i + 3]);
+                    gq[i] = make_uint4(qg[4 * i], qg[4 * i + 1], qg[4 * i + 2], qg[4 * i + 3]);
+                    uq[i] = make_uint4(qu[4 * i], qu[4 * i + 1], qu[4 * i + 2], qu[4 * i + 3]);
                 }
             }
         }
@@ -399,7 +414,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     } else if (warp == 1) {
         // ------------------------------------------------ MMA issuer
         constexpr bool kBmn = MODE == GU || MODE == WG;  // B N-major (else K-major)
-        constexpr uint32_t IDESC = idesc_f16_f32(BM, BN, /*ab_bf16=*/1, /*a_mn=*/0, /*b_mn=*/kBmn ? 1 : 0);
+        constexpr int kBf16 = (MODE == GU || MODE == DX) ? 1 : 0;  // else fp16 x fp16
+        constexpr uint32_t IDESC = idesc_f16_f32(BM, BN, kBf16, /*a_mn=*/0, /*b_mn=*/kBmn ? 1 : 0);
         int stage = 0, acc = 0;
         uint32_t phase = 0, acc_phase = 0;
         bool ok = true;
@@ -561,6 +577,7 @@ __global__ void __launch_bounds__(256) bwd_gather_kernel(const uint16_t* __restr
     const int lane = threadIdx.x & 31;
     const int64_t warps = int64_t(gridDim.x) * (blockDim.x >> 5);
     const int total = poff[Etot];
+    bool bad = false;
     for (int64_t pr = int64_t(blockIdx.x) * (blockDim.x >> 5) + (threadIdx.x >> 5); pr < total; pr += warps) {
         int lo = 0, hi = Etot;  // poff[lo] <= pr < poff[hi]
         while (hi - lo > 1) {
@@ -586,16 +603,20 @@ __global__ void __launch_bounds__(256) bwd_gather_kernel(const uint16_t* __restr
                 xv = __ldg(reinterpret_cast<const uint4*>(x + int64_t(t) * d) + c);
                 const float4* s = reinterpret_cast<const float4*>(dout + int64_t(t) * d) + 2 * c;
                 const float4 a = __ldg(s), b = __ldg(s + 1);
-                gv = make_uint4(pack_bf16x2(a.x, a.y), pack_bf16x2(a.z, a.w), pack_bf16x2(b.x, b.y),
-                                pack_bf16x2(b.z, b.w));
+                gv = make_uint4(pack_f16x2(a.x, a.y), pack_f16x2(a.z, a.w), pack_f16x2(b.x, b.y),
+                                pack_f16x2(b.z, b.w));
+                bad |= !(f16_range_ok(a.x) && f16_range_ok(a.y) && f16_range_ok(a.z) && f16_range_ok(a.w) &&
+                         f16_range_ok(b.x) && f16_range_ok(b.y) && f16_range_ok(b.z) && f16_range_ok(b.w));
             }
             xo[c] = xv;
             go[c] = gv;
         }
     }
+    if (bad) set_error(err, MOE_DEVERR_RANGE);
 }
 
-// xgT[c, r] = xg[r, c] for the used padded rows; 32 x 32 tiles through shared memory.
+// xgT[c, r] = fp16(xg[r, c]) for the used padded rows; 32 x 32 tiles through
+// shared memory (bf16 -> fp16 is exact for values in fp16's range).
 __global__ void __launch_bounds__(256) transpose_kernel(const uint16_t* __restrict__ xg, const int32_t* __restrict__ poff,
                                                         int Etot, int d, int64_t rp, uint16_t* __restrict__ xgT) {
     __shared__ uint16_t tile[32][33];
@@ -607,7 +628,8 @@ __global__ void __launch_bounds__(256) transpose_kernel(const uint16_t* __restri
     const int tx = threadIdx.x & 31, ty = threadIdx.x >> 5;  // 32 x 8
     for (int i = ty; i < 32; i += 8) tile[i][tx] = xg[(r0 + i) * d + c0 + tx];
     __syncthreads();
-    for (int i = ty; i < 32; i += 8) xgT[int64_t(c0 + i) * rp + r0 + tx] = tile[tx][i];
+    for (int i = ty; i < 32; i += 8)
+        xgT[int64_t(c0 + i) * rp + r0 + tx] = uint16_t(pack_f16x2(bf16_to_f32(tile[tx][i]), 0.f) & 0xFFFFu);
 }
 
 // d topk_w[p] = sum over the DH n-tiles of <h, dhu> of the pair's row; 0 if dropped.
@@ -693,7 +715,7 @@ cudaError_t launch_mode(const CUtensorMap& A, const CUtensorMap& B0, const CUten
 }  // namespace bwd
 
 namespace tc {
-bool map_weights_kmajor(CUtensorMap* m, const void* base, int nexp, int N, int K);
+bool map_weights_kmajor(CUtensorMap* m, const void* base, int nexp, int N, int K, bool f16 = false);
 bool map_act_mn(CUtensorMap* m, const void* base, int64_t rows, int N, int64_t row_stride);
 }  // namespace tc
 
@@ -716,6 +738,7 @@ cudaError_t launch_backward(const Dims& D, const BwdArgs& a, cudaStream_t s) {
     uint16_t* h = reinterpret_cast<uint16_t*>(ws + L.b_h);
     uint16_t* hwT = reinterpret_cast<uint16_t*>(ws + L.b_hwT);
     uint16_t* dgu = reinterpret_cast<uint16_t*>(ws + L.b_dgu);
+    uint16_t* dgu16 = reinterpret_cast<uint16_t*>(ws + L.b_dgu16);
     uint16_t* dxr = reinterpret_cast<uint16_t*>(ws + L.b_dxr);
     float* dwp = reinterpret_cast<float*>(ws + L.b_dwp);
     cudaError_t e;
@@ -743,14 +766,15 @@ cudaError_t launch_backward(const Dims& D, const BwdArgs& a, cudaStream_t s) {
         !tc::map_rows(&mHwT, hwT, f, int(rp)) || !tc::map_rows(&mXgT, xgT, d, int(rp)) ||
         !tc::map_weights(&mG, w->w_gate, D.E, d, f, 2) || !tc::map_weights(&mU, w->w_up, D.E, d, f, 2) ||
         !tc::map_weights_kmajor(&mGk, w->w_gate, D.E, d, f) || !tc::map_weights_kmajor(&mUk, w->w_up, D.E, d, f) ||
-        !tc::map_weights_kmajor(&mDk, w->w_down, D.E, f, d) || !tc::map_act_mn(&mDogN, dog, rp, d, d) ||
-        !tc::map_act_mn(&mDgN, dgu, rp, f, 2 * int64_t(f)) || !tc::map_act_mn(&mDuN, dgu + f, rp, f, 2 * int64_t(f)))
+        !tc::map_weights_kmajor(&mDk, w->w_down, D.E, f, d, true) || !tc::map_act_mn(&mDogN, dog, rp, d, d) ||
+        !tc::map_act_mn(&mDgN, dgu16, rp, f, 2 * int64_t(f)) ||
+        !tc::map_act_mn(&mDuN, dgu16 + f, rp, f, 2 * int64_t(f)))
         return cudaErrorInvalidValue;
     if (D.has_shared) {
         if (!tc::map_weights(&sG, w->shared_gate, 1, d, f, 2) || !tc::map_weights(&sU, w->shared_up, 1, d, f, 2) ||
             !tc::map_weights_kmajor(&sGk, w->shared_gate, 1, d, f) ||
             !tc::map_weights_kmajor(&sUk, w->shared_up, 1, d, f) ||
-            !tc::map_weights_kmajor(&sDk, w->shared_down, 1, f, d))
+            !tc::map_weights_kmajor(&sDk, w->shared_down, 1, f, d, true))
             return cudaErrorInvalidValue;
     } else {
         sG = mG;
@@ -776,6 +800,7 @@ cudaError_t launch_backward(const Dims& D, const BwdArgs& a, cudaStream_t s) {
     p.h = h;
     p.hwT = hwT;
     p.dgu = dgu;
+    p.dgu16 = dgu16;
     p.dxr = dxr;
     p.dwp = dwp;
     p.err = a.err;

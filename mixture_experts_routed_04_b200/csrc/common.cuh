@@ -185,14 +185,6 @@ MOE_DEV void cp_async_wait() {
     asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
 }
 
-// Bring a tile into L2 ahead of its load (no shared memory, no completion signal).
-MOE_DEV void tma_prefetch_l2_4d(const CUtensorMap* m, int32_t x, int32_t y, int32_t z, int32_t w) {
-    asm volatile("cp.async.bulk.prefetch.tensor.4d.L2.global.tile [%0, {%1, %2, %3, %4}];" ::"l"(
-                     reinterpret_cast<uint64_t>(m)),
-                 "r"(x), "r"(y), "r"(z), "r"(w)
-                 : "memory");
-}
-
 // ------------------------------------------------------------------ clusters of two CTAs (SM pairs)
 // A pair computes one 256-row tile with tcgen05 ops of cta_group::2: CTA rank 0
 // (the leader) issues the MMAs, which read A and B from the same shared-memory

@@ -88,13 +88,6 @@ struct Cfg {
         idesc_f16_f32(64, BN, /*ab_bf16=*/(MODE == 0 && WF == 0) ? 1 : 0, /*a_mn=*/0, /*b_mn=*/Q4 ? 0 : 1);
 };
 
-// The first unit of a weight tile to run (m = 0, the leader) streams that tile
-// from HBM while the unit's other M-tiles wait for the same lines; the leader's
-// producer also asks L2 for the weight k-block kPrefetchAhead blocks past the
-// one it loads, so that more of the tile is in flight than the stages hold.
-// 0 = off.
-constexpr int kPrefetchAhead = 0;
-
 MOE_DEV uint32_t lop3_and_or(uint32_t a, uint32_t mask, uint32_t orv) {
     uint32_t r;
     asm("lop3.b32 %0, %1, %2, %3, 0xEA;" : "=r"(r) : "r"(a), "r"(mask), "r"(orv));  // (a & b) | c
@@ -247,23 +240,10 @@ __global__ void __launch_bounds__(Cfg<MODE, WF, SUB, GATHER>::kThreads, 1)
                         // two 64-column chunks of gate, then two of up: one copy each
                         tma_load_4d(sb, mg, full + stage, 0, kb * BK, 2 * U.n, z);
                         tma_load_4d(sb + 2 * B_CHUNK, mu, full + stage, 0, kb * BK, 2 * U.n, z);
-                        if (kPrefetchAhead > 0 && U.m == 0) {
-                            for (int q = kb == 0 ? 1 : kPrefetchAhead; q <= kPrefetchAhead; ++q) {
-                                if (kb + q >= KB) break;
-                                tma_prefetch_l2_4d(mg, 0, (kb + q) * BK, 2 * U.n, z);
-                                tma_prefetch_l2_4d(mu, 0, (kb + q) * BK, 2 * U.n, z);
-                            }
-                        }
                     } else {
                         const CUtensorMap* md = sh ? &tmS0 : &tmB0;
                         // four 64-column chunks in one copy
                         tma_load_4d(sb, md, full + stage, 0, kb * BK, 4 * U.n, z);
-                        if (kPrefetchAhead > 0 && U.m == 0) {
-                            for (int q = kb == 0 ? 1 : kPrefetchAhead; q <= kPrefetchAhead; ++q) {
-                                if (kb + q >= KB) break;
-                                tma_prefetch_l2_4d(md, 0, (kb + q) * BK, 4 * U.n, z);
-                            }
-                        }
                     }
                     issued |= 1u << stage;
                     issued_par = (issued_par & ~(1u << stage)) | (phase << stage);
@@ -588,15 +568,16 @@ bool map_weights(CUtensorMap* m, const void* base, int nexp, int K, int N, int c
     const uint32_t box[4] = {64, 64, uint32_t(chunks), 1};
     return make_map(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, base, 4, dims, str, box, CU_TENSOR_MAP_SWIZZLE_128B);
 }
-// bf16 weights [nexp, N, K] (K contiguous) read as a K-major B operand: box 64 (K)
+// 2-byte weights [nexp, N, K] (K contiguous) read as a K-major B operand: box 64 (K)
 // x 256 (N rows) x 1, 128-byte swizzle — the layout of the A tiles, 256 rows.
-bool map_weights_kmajor(CUtensorMap* m, const void* base, int nexp, int N, int K) {
+bool map_weights_kmajor(CUtensorMap* m, const void* base, int nexp, int N, int K, bool f16) {
     const uint64_t dims[3] = {uint64_t(K), uint64_t(N), uint64_t(nexp)};
     const uint64_t str[2] = {uint64_t(K) * 2, uint64_t(N) * uint64_t(K) * 2};
     const uint32_t box[3] = {64, 256, 1};
-    return make_map(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, base, 3, dims, str, box, CU_TENSOR_MAP_SWIZZLE_128B);
+    return make_map(m, f16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, base, 3, dims, str,
+                    box, CU_TENSOR_MAP_SWIZZLE_128B);
 }
-// bf16 activation rows [rows, N] (row stride row_stride elements) read as an N-major B
+// 2-byte activation rows [rows, N] (row stride row_stride elements) read as an N-major B
 // operand (K = rows): seen as [1, N/64 chunks, rows, 64]; one copy brings 4 chunks.
 bool map_act_mn(CUtensorMap* m, const void* base, int64_t rows, int N, int64_t row_stride) {
     const uint64_t dims[4] = {64, uint64_t(rows), uint64_t(N / 64), 1};
@@ -651,8 +632,7 @@ cudaError_t launch_tensor_ffn(const Dims& D, const uint16_t* xg, uint16_t* h, co
                               const int32_t* offsets,
                               const int32_t* sorted_pair, const float* topk_w, const moe_weights* w,
                               uint16_t* y_rows, int32_t* counters, uint32_t* err, uint64_t wait_ns,
-                              const long long* units_a, const long long* units_b, const uint16_t* x_fused,
-                              const int32_t* sorted_token, cudaStream_t s) {
+                              const uint16_t* x_fused, const int32_t* sorted_token, cudaStream_t s) {
     using namespace tc;
     const bool pdl = use_pdl(D.T);
     GemmParams p{};
@@ -679,14 +659,12 @@ cudaError_t launch_tensor_ffn(const Dims& D, const uint16_t* xg, uint16_t* h, co
         p.n_tiles = (D.f + 127) / 128;
         p.out = h;
         p.unit_counter = counters;
-        p.units = units_a;
         if ((e = launch_gemm<0, 1, 2>(mA, pg, pu, sg, su, p, pdl, s)) != cudaSuccess) return e;
         p.K = D.f;
         p.n_out = D.d;
         p.n_tiles = (D.d + BN - 1) / BN;
         p.out = y_rows;
         p.unit_counter = counters + 1;
-        p.units = units_b;
         return launch_gemm<1, 1, 2>(mH, pd, pd, sd, sd, p, pdl, s);
     }
     CUtensorMap mG, mU, mSG, mSU, mD, mSD;
@@ -709,7 +687,6 @@ cudaError_t launch_tensor_ffn(const Dims& D, const uint16_t* xg, uint16_t* h, co
     p.n_tiles = (D.f + 127) / 128;
     p.out = h;
     p.unit_counter = counters;
-    p.units = D.tile_pair ? nullptr : units_a;
     p.x = x_fused;
     p.sorted_token = sorted_token;
     p.T = D.T;
@@ -723,7 +700,6 @@ cudaError_t launch_tensor_ffn(const Dims& D, const uint16_t* xg, uint16_t* h, co
     p.n_tiles = (D.d + BN - 1) / BN;
     p.out = y_rows;
     p.unit_counter = counters + 1;
-    p.units = D.tile_pair ? nullptr : units_b;
     if (D.tile_pair && D.down_f16) {
         // each SM of a pair copies 128 of the tile's 256 columns: maps of 2 chunks
         CUtensorMap mD2, mSD2;

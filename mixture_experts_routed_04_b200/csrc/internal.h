@@ -34,13 +34,12 @@ struct WsLayout {
     size_t err;                                    // uint32 error word (always at 0)
     size_t blockcounts, blockbase;                 // permute: int32 [perm_blocks, E]
     size_t tile_base, stream_list, n_stream;       // expert_ffn schedule
-    size_t units_a, units_b;                       // claim orders of the two tcgen05 GEMMs (int64)
     size_t xg, h, part;                            // expert_ffn: gathered x, h, split-K partials
     size_t topk_idx, topk_w, counts, kept, offsets, sorted_token, sorted_pair, pair_row, y_rows;  // forward
     size_t x_dev, logits_dev, out_dev;             // forward_host
     size_t stats_p, stats_c, stats_s;              // route_stats: per-block partial sums
     // backward (padded row space, see backward.cu)
-    size_t b_poff, b_tile_base, b_wbase, b_counters, b_xg, b_xgT, b_dog, b_gu, b_h, b_hwT, b_dgu, b_dxr, b_dwp;
+    size_t b_poff, b_tile_base, b_wbase, b_counters, b_xg, b_xgT, b_dog, b_gu, b_h, b_hwT, b_dgu, b_dgu16, b_dxr, b_dwp;
     size_t total;
 };
 
@@ -60,16 +59,13 @@ cudaError_t launch_route_stats(const float* logits, int T, int E, int k, int32_t
                                float* expert_stats, float* part_p, int32_t* part_c, float* part_s,
                                cudaStream_t stream);
 
-// The tile schedule (K3) and the claim orders, when the permutation's scan
-// kernel runs them too (moe_forward with more than kFrontMaxTokens tokens).
+// The tile schedule (K3), when the permutation's scan kernel runs it too
+// (moe_forward with more than kFrontMaxTokens tokens).
 struct ScheduleArgs {
     int32_t* tile_base;
     int32_t* stream_list;
     int32_t* n_stream;
     int variant, stream_max;
-    int sub, nt_a, nt_b, chunk;
-    long long* units_a;
-    long long* units_b;
 };
 cudaError_t launch_permute(const Dims& D, const int32_t* topk_idx, int32_t* blockcounts, int32_t* blockbase,
                            int32_t* counts, int32_t* kept, int32_t* offsets, int32_t* sorted_token,
@@ -84,16 +80,6 @@ cudaError_t launch_front_small(const Dims& D, const float* logits, int32_t* topk
                                int32_t* sorted_pair, int32_t* pair_row, int32_t* tile_base, int32_t* stream_list,
                                int32_t* n_stream, uint32_t* err, cudaStream_t s);
 
-// Claim order of the tcgen05 GEMMs' units, written by the schedule kernel
-// (schedule.cu): M-tiles of `sub` x 128 rows; nt_a / nt_b n-tiles per M-tile
-// for gate/up and down; chunk groups per chunk (0: the natural order).
-struct UnitOrder {
-    int sub, nt_a, nt_b, chunk;
-    long long* units_a;
-    long long* units_b;
-};
-// Groups (expert, n-tile) per chunk of the claim order.
-constexpr int kUnitOrderChunk = 32;
 // The bf16 gate/up GEMM gathers its rows from x itself (no gathered copy).
 constexpr bool kFusedGather = false;
 
@@ -110,11 +96,7 @@ struct FfnArgs {
     uint64_t wait_ns;
     bool scheduled;            // the front kernels already wrote the tile schedule
     const int32_t* pair_row;   // moe_forward: row of each pair (-1 dropped), for the token-order row copy
-    bool units_written;        // ... and the claim orders (the permutation's scan did)
 };
-// The claim orders a layer's tile GEMMs use, with their workspace arrays (null
-// pointers: the natural order, for the SM-pair kernels or when no tile runs).
-UnitOrder unit_order_for(const Dims& D, const WsLayout& L, uint8_t* ws);
 cudaError_t launch_expert_ffn(const Dims& D, const WsLayout& L, const FfnArgs& a, cudaStream_t s);
 
 cudaError_t launch_combine(const Dims& D, const uint16_t* y_rows, const int32_t* pair_row, const int32_t* offsets,

@@ -83,9 +83,8 @@ __global__ void __launch_bounds__(kPermWarps * 32) perm_count_kernel(const int32
 }
 
 // One block: thread e owns expert e (256 threads; 512 with SCHED). With SCHED
-// the block then runs the tile schedule and the claim orders of the tile GEMMs
-// on the kept counts it has just formed (the schedule kernel's work, without
-// a launch of its own).
+// the block then runs the tile schedule on the kept counts it has just formed
+// (the schedule kernel's work, without a launch of its own).
 template <bool SCHED>
 __global__ void __launch_bounds__(SCHED ? 512 : kMaxE)
     perm_scan_kernel(const int32_t* __restrict__ blockcounts, int nblocks, int E, int cap, int shared_T,
@@ -93,7 +92,6 @@ __global__ void __launch_bounds__(SCHED ? 512 : kMaxE)
                      int32_t* __restrict__ offsets, ScheduleArgs sa) {
     __shared__ int warp_sums[16];
     __shared__ int sums[3][16];
-    __shared__ int s_tb[kMaxE + 2], s_ne[kMaxE + 2];
     griddep_wait();
     griddep_launch();
 
@@ -140,9 +138,6 @@ __global__ void __launch_bounds__(SCHED ? 512 : kMaxE)
         const int Etot = E + (shared_T > 0 ? 1 : 0);
         const int ke = e < E ? kv : (e == E && shared_T > 0 ? shared_T : 0);
         schedule_block(ke, Etot, sa.variant, sa.stream_max, sums, sa.tile_base, sa.stream_list, sa.n_stream);
-        if (sa.units_a)
-            unit_orders_block(sa.tile_base, Etot, sa.sub, sa.nt_a, sa.nt_b, sa.chunk, sa.units_a, sa.units_b, s_tb,
-                              s_ne, sums);
     }
 }
 

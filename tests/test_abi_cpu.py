@@ -128,16 +128,16 @@ def test_product_path_never_touches_the_oracle():
 
 
 def test_backward_host_checks(lib):
-    """moe_expert_ffn_backward refuses Q4G32 weights and an fp16 W_down before touching any
-    pointer; its workspace grows with the padded row space."""
+    """moe_expert_ffn_backward refuses Q4G32 weights and a bf16 W_down (it multiplies the fp16
+    copy) before touching any pointer; its workspace grows with the padded row space."""
     p = b.params(T=64, d_model=128, d_ff=256, E=8, k=2, weight_format=b.WEIGHTS_Q4G32)
     st = lib.moe_expert_ffn_backward(ctypes.byref(p), None, None, None, None, None, None, None, None, None, None,
                                      None, 0, None)
     assert st == 3  # MOE_ERR_UNSUPPORTED
-    p = b.params(T=64, d_model=128, d_ff=256, E=8, k=2, down_dtype=b.DOWN_F16)
+    p = b.params(T=64, d_model=128, d_ff=256, E=8, k=2, down_dtype=b.DOWN_BF16)
     st = lib.moe_expert_ffn_backward(ctypes.byref(p), None, None, None, None, None, None, None, None, None, None,
                                      None, 0, None)
     assert st == 3
-    small = b.workspace_size(b.params(T=64, d_model=128, d_ff=256, E=8, k=2), b.WS_BACKWARD)
-    large = b.workspace_size(b.params(T=640, d_model=128, d_ff=256, E=8, k=2), b.WS_BACKWARD)
+    small = b.workspace_size(b.params(T=64, d_model=128, d_ff=256, E=8, k=2, down_dtype=b.DOWN_F16), b.WS_BACKWARD)
+    large = b.workspace_size(b.params(T=640, d_model=128, d_ff=256, E=8, k=2, down_dtype=b.DOWN_F16), b.WS_BACKWARD)
     assert 0 < small < large

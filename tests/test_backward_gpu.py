@@ -1,14 +1,19 @@
 """Backward of the expert FFN (moe_expert_ffn_backward) against the fp64 oracle.
 
-The upstream gradient dout is seeded N(0, 1); every gradient — dx, the three
-expert weight gradients of every expert (zeros for experts without rows), the
-routing-weight gradient d topk_w, dlogits and the shared expert's weight
-gradients — is compared element by element with oracle.backward within the
-layer's bar: rel-L2 <= 1e-2 and max-abs <= 3e-2 * rms(reference). The GPU
-runs bf16 operands (x, weights, dout rounded once, h, dg, du rounded once)
-with fp32 accumulation. Small layers span several M-tiles per expert with
-ragged tails, capacity drops, a shared expert, skew and k = E; the prompt
-workload runs at full size. Two calls give the same bits.
+The upstream gradient dout is seeded N(0, 1) (synth.dout); every gradient —
+dx, the three expert weight gradients of every expert (zeros for experts
+without rows), the routing-weight gradient d topk_w, dlogits and the shared
+expert's weight gradients — is compared element by element with
+oracle.backward: rel-L2 <= 1e-2, and every element within 3e-2 * rms(ref)
+plus 2^-6 of its own magnitude. The second term is the 16-bit operand
+rounding carried by large elements: with one token a weight gradient is an
+outer product, whose largest element is ~20x its rms, so an error relative to
+each element (fp16: 2^-11 per rounded operand) reaches a few percent of rms.
+The GPU multiplies the bf16 gate/up weights by bf16 operands and the fp16
+W_down copy and the weight gradients by fp16 operands, accumulating in fp32.
+Small layers span several M-tiles per expert with ragged tails, capacity
+drops, a shared expert, skew, k = E and a firing clamp; the prompt workload
+runs at full size. Two calls give the same bits.
 """
 import numpy as np
 import pytest
@@ -21,7 +26,7 @@ from synth.device import expert_f64, shared_f64, upload
 
 pytestmark = pytest.mark.gpu
 
-REL_L2, MAX_ABS_RMS = 1e-2, 3e-2
+REL_L2, MAX_ABS_RMS, ELEM_REL = 1e-2, 3e-2, 2.0 ** -6
 
 LAYERS = {
     "tiny": synth.CONFIGS["tiny"],
@@ -44,9 +49,10 @@ def check_close(got, ref, what):
     diff = got - ref
     rel = np.linalg.norm(diff) / max(np.linalg.norm(ref), 1e-300)
     rms = float(np.sqrt(np.mean(ref ** 2)))
-    mx = float(np.abs(diff).max()) if diff.size else 0.0
-    assert rel <= REL_L2 and mx <= MAX_ABS_RMS * rms, \
-        f"{what}: rel-L2 {rel:.3e} (<= {REL_L2}), max-abs {mx:.3e} (<= {MAX_ABS_RMS * rms:.3e})"
+    excess = np.abs(diff) - (MAX_ABS_RMS * rms + ELEM_REL * np.abs(ref))
+    worst = float(excess.max()) if diff.size else -1.0
+    assert rel <= REL_L2 and worst <= 0.0, \
+        f"{what}: rel-L2 {rel:.3e} (<= {REL_L2}), worst element over its bound by {worst:.3e}"
 
 
 def dout_of(cfg):
@@ -54,7 +60,7 @@ def dout_of(cfg):
 
 
 def run_backward(cfg, d, dout):
-    p = b.params_for(cfg)
+    p = b.params_for(cfg, down_dtype=b.DOWN_F16)
     T, E, k, dm, f = cfg.T, cfg.E, cfg.k, cfg.d, cfg.f
     Et = E + int(cfg.has_shared)
     rows = b.max_rows(p)
@@ -65,8 +71,9 @@ def run_backward(cfg, d, dout):
     st, sp, pr = torch.empty(rows, **i32), torch.empty(rows, **i32), torch.empty(T * k, **i32)
     b.route(p, d["logits"], idx, w, b.workspace(p, b.WS_ROUTE))
     b.permute(p, idx, counts, kept, offsets, st, sp, pr, b.workspace(p, b.WS_PERMUTE))
-    sh = (d["shared_gate"], d["shared_up"], d["shared_down"]) if cfg.has_shared else None
-    W = b.weights(d["w_gate"], d["w_up"], d["w_down"], shared=sh)
+    # the backward multiplies the fp16 copy of W_down, prepared once as for the forward
+    sh = (d["shared_gate"], d["shared_up"], b.prepare_down_f16(d["shared_down"])) if cfg.has_shared else None
+    W = b.weights(d["w_gate"], d["w_up"], b.prepare_down_f16(d["w_down"]), shared=sh)
     nan = float("nan")
     outs = dict(dx=torch.full((T, dm), nan, **f32), dw_gate=torch.full((E, dm, f), nan, **f32),
                 dw_up=torch.full((E, dm, f), nan, **f32), dw_down=torch.full((E, f, dm), nan, **f32),
