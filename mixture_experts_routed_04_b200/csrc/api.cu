@@ -192,6 +192,12 @@ WsLayout ws_layout(const Dims& D, int which) {
 // (a token's k experts are distinct; the shared expert holds exactly T), so
 // with T <= stream_max_rows the automatic choice streams every expert and the
 // two persistent GEMMs would only start and exit: they are not launched.
+// Whether the weight-streaming kernels run: every expert with a forced
+// MOE_VARIANT_STREAM, else the experts of at most stream_max_rows rows.
+static bool streams(const Dims& D) {
+    return D.variant == MOE_VARIANT_STREAM || (D.variant == MOE_VARIANT_AUTO && D.stream_max_rows > 0);
+}
+
 static bool tiles_needed(const Dims& D) {
     if (D.variant == MOE_VARIANT_STREAM) return false;
     if (D.variant == MOE_VARIANT_AUTO && D.stream_max_rows > 0 && D.T <= D.stream_max_rows) return false;
@@ -205,7 +211,7 @@ static bool x_in_l2(const Dims& D) { return int64_t(D.T) * D.d * 2 <= (int64_t(6
 // when x sits in L2 and no expert streams (the streaming kernels read the
 // gathered copy).
 static bool gather_fused(const Dims& D) {
-    const bool streaming = D.variant != MOE_VARIANT_TENSOR && D.stream_max_rows > 0;
+    const bool streaming = streams(D);
     return kFusedGather && D.fmt == MOE_WEIGHTS_BF16 && !D.tile_pair && x_in_l2(D) && !streaming && tiles_needed(D);
 }
 
@@ -239,7 +245,7 @@ cudaError_t launch_expert_ffn(const Dims& D, const WsLayout& L, const FfnArgs& a
             cudaSuccess)
             return e;
     }
-    if (D.variant != MOE_VARIANT_TENSOR && D.stream_max_rows > 0) {
+    if (streams(D)) {
         if ((e = launch_stream_ffn(D, xg, h, part, a.offsets, stream_list, n_stream, a.sorted_pair, a.topk_w, a.w,
                                    a.y_rows, a.err, a.wait_ns, s)) != cudaSuccess)
             return e;
@@ -550,7 +556,7 @@ int moe_launch_count(const moe_params* p, int which, int* n) {
     int ffn = 1;  // schedule
     if (!gather_fused(D)) ffn += 1;                 // gather
     if (tiles_needed(D)) ffn += 2;                  // two tcgen05 GEMMs
-    if (D.variant != MOE_VARIANT_TENSOR && D.stream_max_rows > 0) ffn += 2 + (D.ks > 1 ? 1 : 0);
+    if (streams(D)) ffn += 2 + (D.ks > 1 ? 1 : 0);
     switch (which) {
         case MOE_WS_ROUTE: *n = 1; break;
         case MOE_WS_PERMUTE: *n = 3; break;

@@ -40,6 +40,9 @@ SMALL = {
     "shared_small": synth.LayerConfig("shared_small", T=20, d=256, f=192, E=16, k=4, has_shared=True,
                                       f_shared=192),
     "zipf_small": synth.LayerConfig("zipf_small", T=512, d=256, f=256, E=32, k=4, bias="zipf"),
+    # 32 touched experts x 5 gate/up tiles >= 148 SMs: the automatic choice keeps every expert
+    # on the tiles, so a forced streaming variant must still launch the streaming kernels
+    "many_experts": synth.LayerConfig("many_experts", T=8, d=128, f=640, E=32, k=4),
 }
 Q4_SMALL = {
     "q4_tiny": synth.CONFIGS["tiny"].replace(name="q4_tiny", weight_format="q4g32"),
