@@ -123,10 +123,8 @@ typedef struct moe_params {
     int32_t d_ff_shared;     /* its f (must equal d_ff) */
     int32_t variant;         /* MOE_VARIANT_* */
     int32_t stream_max_rows; /* AUTO: experts with 1..this many kept rows use the streaming
-                                kernels, the rest the tcgen05 tiles; < 0 = library default,
-                                set from a measured sweep: 8 when even every touchable
-                                expert cannot give each of the 148 SMs a gate/up tile
-                                (single-token decode), else 0 (tiles for all) */
+                                kernels, the rest the tcgen05 tiles; < 0 = library default
+                                from the measured table (moe_variant_table) */
     int32_t out_dtype;       /* MOE_OUT_F32 | MOE_OUT_BF16 */
     int32_t down_dtype;      /* MOE_DOWN_BF16 | MOE_DOWN_F16 */
     int32_t tile_ctas;       /* SMs per tcgen05 tile: MOE_TILE_* */
@@ -182,6 +180,19 @@ MOE_API int moe_max_rows(const moe_params* p, int64_t* rows);
  * MOE_TILE_ONE; MOE_TILE_PAIR with Q4G32 weights resolves to MOE_TILE_ONE.
  */
 MOE_API int moe_tile_ctas(const moe_params* p, int32_t* ctas);
+
+/*
+ * The measured table behind the default variant choice (stream_max_rows < 0):
+ * row i says that experts of at most max_rows[i] kept rows take the weight-
+ * streaming kernels while the touched experts' gate/up tiles (min(E', T*k +
+ * has_shared) experts x ceil(d_ff/128)) number fewer than tiles_per_sm[i] x
+ * the GPU's SMs; the first matching row applies, and past the last every
+ * expert takes the tcgen05 tiles. The pages' analogues are Strata PR #4366's
+ * light kernels for experts of <= 16 rows and TensorFold PR #1607's bound on
+ * pairs per item ("What this changes"); these entries were measured on B200.
+ * Copies up to n rows into the host arrays; returns the table's row count.
+ */
+MOE_API int moe_variant_table(float* tiles_per_sm, int32_t* max_rows, int n);
 
 /* Bytes of workspace each call needs (which = MOE_WS_*); 0 on invalid params. */
 MOE_API size_t moe_workspace_size(const moe_params* p, int which);

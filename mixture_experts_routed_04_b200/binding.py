@@ -36,7 +36,7 @@ EXPORTS = ("moe_version", "moe_status_string", "moe_capacity", "moe_max_rows", "
            "moe_get_error", "moe_clear_error", "moe_set_wait_limit_ns", "moe_launch_count",
            "moe_profile_enable", "moe_profile_collect", "moe_convert_bf16_to_f16",
            "moe_permute_noalloc", "moe_forward_host_async", "moe_wait_selftest", "moe_tile_ctas",
-           "moe_route_stats", "moe_expert_ffn_backward")
+           "moe_route_stats", "moe_expert_ffn_backward", "moe_variant_table")
 NOALLOC_MAX_PAIRS = 262144  # MOE_NOALLOC_MAX_PAIRS
 
 # kernel ids (MOE_K_*), in order
@@ -102,6 +102,8 @@ def lib() -> ctypes.CDLL:
             "moe_profile_collect": ([ctypes.POINTER(ctypes.c_double), ctypes.POINTER(ctypes.c_int64)], ctypes.c_int),
             "moe_convert_bf16_to_f16": ([_V, _V, ctypes.c_int64, _V, _V], ctypes.c_int),
             "moe_permute_noalloc": ([_P, _V, _V, _V, _V, _V, _V, _V, _V, _V], ctypes.c_int),
+            "moe_variant_table": ([ctypes.POINTER(ctypes.c_float), ctypes.POINTER(ctypes.c_int32), ctypes.c_int],
+                                  ctypes.c_int),
             "moe_expert_ffn_backward": ([_P, _V, _V, _V, _V, _V, _V, _V, ctypes.POINTER(Weights), _V,
                                          ctypes.POINTER(Grads), _V, _S, _V], ctypes.c_int),
         }
@@ -277,6 +279,14 @@ def clear_error(ws, stream=None) -> None:
 
 def set_wait_limit_ns(ns: int) -> None:
     check(lib().moe_set_wait_limit_ns(ns), "moe_set_wait_limit_ns")
+
+
+def variant_table():
+    """[(tiles_per_sm, max_rows), ...]: the measured rows of the default variant choice."""
+    n = lib().moe_variant_table(None, None, 0)
+    a, r = (ctypes.c_float * n)(), (ctypes.c_int32 * n)()
+    lib().moe_variant_table(a, r, n)
+    return [(float(a[i]), int(r[i])) for i in range(n)]
 
 
 def launch_count(p: Params, which: int) -> int:

@@ -86,15 +86,18 @@ int make_dims(const moe_params* p, Dims* D) {
     D->perm_blocks = int((pairs + kPermPairsPerBlock - 1) / kPermPairsPerBlock);
     D->fmt = p->weight_format;
     D->variant = p->variant;
-    // Default variant choice, from the measured sweep over rows-per-expert
-    // thresholds (prompt, capped and decode layers): the tcgen05 tiles win
-    // whenever the touched experts can give every SM a gate/up tile — even for
-    // experts of one row (T=8, 32: 98% of HBM); below that (T=1) experts of up
-    // to kStreamRowsFewExperts rows take the weight-streaming kernels.
+    // Default variant choice from the measured table (kStreamTable): the
+    // touched experts' gate/up tiles (at most min(E', pairs') experts) against
+    // the SM count picks the largest expert that still streams.
     if (p->stream_max_rows < 0) {
         const int64_t touched_max = std::min<int64_t>(p->E + p->has_shared, pairs + p->has_shared);
-        const int64_t tiles_max = touched_max * ((p->d_ff + 127) / 128);
-        D->stream_max_rows = tiles_max < num_sms() ? kStreamRowsFewExperts : 0;
+        const double ratio = double(touched_max * ((p->d_ff + 127) / 128)) / double(num_sms());
+        D->stream_max_rows = 0;
+        for (int i = 0; i < kStreamTableRows; ++i)
+            if (ratio < double(kStreamTable[i].tiles_per_sm)) {
+                D->stream_max_rows = kStreamTable[i].max_rows;
+                break;
+            }
     } else {
         D->stream_max_rows = p->stream_max_rows;
     }
@@ -528,6 +531,15 @@ int moe_expert_ffn_backward(const moe_params* p, const uint16_t* x, const int32_
               static_cast<uint8_t*>(ws), ws_layout(D, MOE_WS_BACKWARD), static_cast<uint32_t*>(ws),
               g_wait_ns.load()};
     return status_of(launch_backward(D, a, stream));
+}
+
+int moe_variant_table(float* tiles_per_sm, int32_t* max_rows, int n) {
+    if (n < 0 || (n > 0 && (!tiles_per_sm || !max_rows))) return -1;
+    for (int i = 0; i < kStreamTableRows && i < n; ++i) {
+        tiles_per_sm[i] = kStreamTable[i].tiles_per_sm;
+        max_rows[i] = kStreamTable[i].max_rows;
+    }
+    return kStreamTableRows;
 }
 
 int moe_get_error(const void* ws, uint32_t* err, moe_stream_t stream) {

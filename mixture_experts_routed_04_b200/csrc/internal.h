@@ -11,7 +11,18 @@ constexpr int kPermWarps = 8;                         // warps per permutation b
 constexpr int kPermPairsPerWarp = 256;                // 8 rounds of 32 pairs
 constexpr int kPermPairsPerBlock = kPermWarps * kPermPairsPerWarp;
 constexpr int kTileM = 128;                           // rows per tcgen05 tile
-constexpr int kStreamRowsFewExperts = 8;             // AUTO: streaming threshold when few experts are touched
+// AUTO variant choice, measured on B200 (decode-shaped layers, d=4096, f=1536,
+// E=256 + shared, whose routing gives `touched` experts the same rows each;
+// every expert on the tcgen05 tiles against every routed expert streaming):
+// experts of at most max_rows kept rows take the weight-streaming kernels while
+// the touched experts' gate/up tiles number fewer than tiles_per_sm x SMs; the
+// first matching row applies; past the last row every expert takes the tiles.
+struct StreamRule {
+    float tiles_per_sm;
+    int max_rows;
+};
+constexpr StreamRule kStreamTable[] = {{1.5f, 4}, {2.5f, 1}};
+constexpr int kStreamTableRows = int(sizeof(kStreamTable) / sizeof(kStreamTable[0]));
 
 // Everything a call derives from moe_params on the host.
 struct Dims {

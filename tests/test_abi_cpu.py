@@ -141,3 +141,33 @@ def test_backward_host_checks(lib):
     small = b.workspace_size(b.params(T=64, d_model=128, d_ff=256, E=8, k=2, down_dtype=b.DOWN_F16), b.WS_BACKWARD)
     large = b.workspace_size(b.params(T=640, d_model=128, d_ff=256, E=8, k=2, down_dtype=b.DOWN_F16), b.WS_BACKWARD)
     assert 0 < small < large
+
+
+def test_variant_table_is_finite_and_monotone(lib):
+    """The measured table of the default variant choice: finite, tile bounds increasing,
+    streamed expert sizes shrinking as more tiles are available, and every entry sensible."""
+    import math
+    table = b.variant_table()
+    assert 1 <= len(table) <= 16
+    bounds = [t for t, _ in table]
+    rows = [r for _, r in table]
+    assert all(math.isfinite(t) and 0.0 < t < 64.0 for t in bounds)
+    assert all(1 <= r <= 64 for r in rows)
+    assert all(a < c for a, c in zip(bounds, bounds[1:]))
+    assert all(a >= c for a, c in zip(rows, rows[1:]))
+
+
+def test_default_variant_follows_the_table(lib):
+    """Single-token decode (8 routed experts + the shared one: 108 gate/up tiles on 148 SMs, or
+    whatever the host's default count) streams; eight tokens (up to 65 experts) take the tiles.
+    The streaming kernels add launches to moe_forward's count."""
+    def launches(T):
+        p = b.params(T=T, d_model=4096, d_ff=1536, E=256, k=8, has_shared=1, d_ff_shared=1536)
+        return b.launch_count(p, b.WS_FORWARD), b.launch_count(b.params(
+            T=T, d_model=4096, d_ff=1536, E=256, k=8, has_shared=1, d_ff_shared=1536,
+            variant=b.VARIANT_TENSOR), b.WS_FORWARD)
+    auto1, tiles1 = launches(1)
+    auto8, tiles8 = launches(8)
+    # T=1: the two tile GEMMs give way to the streaming gate/up, its K-split reduce and down
+    assert auto1 == tiles1 - 2 + 3
+    assert auto8 == tiles8  # T=8: every expert on the tiles
