@@ -447,6 +447,81 @@ def measure_workload(cfg, args, b, torch, flush, pk, pk_src, steps):
     return entry
 
 
+def measure_extra_rows(cfg, b, torch, flush, pk, pk_src, steps):
+    """The layer's backward (moe_expert_ffn_backward) and the router with its telemetry
+    (moe_route_stats) on the workload, each timed with CUDA events around a graph replay of one
+    call, L2 flushed between calls. Backward work: 16 d f FLOPs per routed row (recomputed gate/up
+    4df, dh 2df, dx 4df, weight gradients 6df) plus the shared expert's rows; telemetry: the
+    logits read once (4 E bytes per token)."""
+    from synth.device import upload
+    d = upload(cfg, "cuda")
+    p = b.params_for(cfg, down_dtype=b.DOWN_F16)
+    T, E, k, dm, f = cfg.T, cfg.E, cfg.k, cfg.d, cfg.f
+    Et = E + int(cfg.has_shared)
+    rows = b.max_rows(p)
+    i32 = dict(dtype=torch.int32, device="cuda")
+    f32 = dict(dtype=torch.float32, device="cuda")
+    idx, w = torch.empty(T, k, **i32), torch.empty(T, k, **f32)
+    counts, kept, offsets = torch.empty(Et, **i32), torch.empty(Et, **i32), torch.empty(Et + 1, **i32)
+    st, sp, pr = torch.empty(rows, **i32), torch.empty(rows, **i32), torch.empty(T * k, **i32)
+    b.route(p, d["logits"], idx, w, b.workspace(p, b.WS_ROUTE))
+    b.permute(p, idx, counts, kept, offsets, st, sp, pr, b.workspace(p, b.WS_PERMUTE))
+    sh = (d["shared_gate"], d["shared_up"], b.prepare_down_f16(d["shared_down"])) if cfg.has_shared else None
+    W = b.weights(d["w_gate"], d["w_up"], b.prepare_down_f16(d["w_down"]), shared=sh)
+    dout = torch.from_numpy(synth.dout(cfg)).cuda()
+    g = dict(dx=torch.empty(T, dm, **f32), dwg=torch.empty(E, dm, f, **f32), dwu=torch.empty(E, dm, f, **f32),
+             dwd=torch.empty(E, f, dm, **f32), dtw=torch.empty(T, k, **f32), dl=torch.empty(T, E, **f32))
+    shg = tuple(torch.empty(s_, **f32) for s_ in ((dm, f), (dm, f), (f, dm))) if cfg.has_shared else None
+    G = b.grads(g["dx"], g["dwg"], g["dwu"], g["dwd"], g["dtw"], g["dl"], shared=shg)
+    wsb = b.workspace(p, b.WS_BACKWARD)
+    stats = torch.empty(5, **f32)
+    wss = b.workspace(p, b.WS_ROUTE_STATS)
+    idx2, w2 = torch.empty(T, k, **i32), torch.empty(T, k, **f32)
+
+    def bwd():
+        b.expert_ffn_backward(p, d["x"], idx, w, offsets, st, sp, pr, W, dout, G, wsb)
+
+    def rstats():
+        b.route_stats(p, d["logits"], idx2, w2, stats, wss)
+
+    out = {}
+    for name, fn in (("backward", bwd), ("route_stats", rstats)):
+        for _ in range(3):
+            fn()
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph):
+            fn()
+        tot = 0.0
+        for i in range(steps + 3):
+            flush()
+            s0, s1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            s0.record()
+            graph.replay()
+            s1.record()
+            s1.synchronize()
+            if i >= 3:
+                tot += s0.elapsed_time(s1)
+        out[name] = tot / steps
+        del graph
+    if b.get_error(wsb) or b.get_error(wss):
+        raise RuntimeError("device error word set (backward / route_stats)")
+    P = int(offsets[E].item())
+    fl = 16.0 * P * dm * f + (16.0 * T * dm * f if cfg.has_shared else 0.0)
+    tfl = fl / (out["backward"] / 1e3) / 1e12
+    gbs = T * E * 4 / (out["route_stats"] / 1e3) / 1e9
+    res = {"backward": {"call": "moe_expert_ffn_backward", "ms": out["backward"], "flops": fl, "tflops": tfl,
+                        "frac_of_peak": tfl / pk["bf16_tflops"], "peak_source": f"{pk_src} bf16_tflops (burst)",
+                        "work": "16 d f FLOPs per routed row: recomputed gate/up, dh, dx, three weight gradients"},
+           "route_stats": {"call": "moe_route_stats", "ms": out["route_stats"], "gbs": gbs,
+                           "frac_of_peak": gbs / pk["hbm_gbs"], "peak_source": f"{pk_src} hbm_gbs",
+                           "work": "the logits read once (4 E bytes per token); latency-bound at this size"},
+           "workload": workload_name(cfg), "steps": steps,
+           "step_launch": "CUDA graph replay of one call, L2 flushed between calls"}
+    del d, W, G, g, wsb, wss
+    torch.cuda.empty_cache()
+    return res
+
+
 # --------------------------------------------------------------------------- own arm
 
 def own_arm(args, cfg):
@@ -671,6 +746,8 @@ def own_arm(args, cfg):
                 pc[name] = measure_workload(synth.CONFIGS[name], args, b, torch, flush, pk, pk_src,
                                             max(3, min(args.steps, 20)))
         line["per_config"] = pc
+        # the scope table's next rows on this workload: the backward and the router telemetry
+        line["next_rows"] = measure_extra_rows(cfg, b, torch, flush, pk, pk_src, max(3, min(args.steps, 20)))
     if dist:
         dist.barrier()
         dist.destroy_process_group()

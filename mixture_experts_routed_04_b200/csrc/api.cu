@@ -143,15 +143,14 @@ WsLayout ws_layout(const Dims& D, int which) {
         L.b_wbase = take(size_t(D.Etot + 1) * 4);
         L.b_counters = take(8 * 4);
         L.b_xg = take(size_t(rp) * D.d * 2);
-        L.b_xgT = take(size_t(rp) * D.d * 2);
+        L.b_xg16 = take(size_t(rp) * D.d * 2);
         L.b_dog = take(size_t(rp) * D.d * 2);
-        L.b_gu = take(size_t(rp) * 2 * D.f * 4);
-        L.b_h = take(size_t(rp) * D.f * 2);
-        L.b_hwT = take(size_t(rp) * D.f * 2);
+        L.b_gu = take(size_t(rp) * 2 * D.f * 2);
+        L.b_hw = take(size_t(rp) * D.f * 2);
         L.b_dgu = take(size_t(rp) * 2 * D.f * 2);
         L.b_dgu16 = take(size_t(rp) * 2 * D.f * 2);
         L.b_dxr = take(size_t(D.rows) * D.d * 2);
-        L.b_dwp = take(size_t(D.rows) * nt * 4);
+        L.b_dwp = take(size_t(D.rows) * nt * 2 * 4);
     }
     if (which == MOE_WS_ROUTE_STATS) {
         const int nb = route_stats_blocks(D.T > 0 ? D.T : 1);
@@ -514,8 +513,6 @@ int moe_expert_ffn_backward(const moe_params* p, const uint16_t* x, const int32_
     if (st != MOE_OK) return st;
     // bf16 gate/up weights and the fp16 copy of W_down (moe_convert_bf16_to_f16)
     if (D.fmt != MOE_WEIGHTS_BF16 || !D.down_f16) return MOE_ERR_UNSUPPORTED;
-    // the transpose grid holds padded rows / 32 blocks in y (at most 65535)
-    if (bwd_padded_rows(D) / 32 > 65535) return MOE_ERR_UNSUPPORTED;
     if ((st = check_ws(D, MOE_WS_BACKWARD, ws, ws_bytes)) != MOE_OK) return st;
     if (D.T == 0) return MOE_OK;
     if ((st = check_weights(D, w)) != MOE_OK) return st;

@@ -14,12 +14,13 @@
 // rows (poff[e] = padded offset), so the weight gradients, which contract
 // over an expert's rows, run whole 64-row k-blocks. Launches (one stream):
 //   bwd_schedule      padded offsets, tile prefixes, unit counters
-//   bwd_gather        xg = x rows (bf16), dog = dout rows (fp16), zero padding rows
-//   transpose         xgT = xg^T  [d, Rp] (fp16, exact for bf16 x in fp16's range)
-//   GEMM GU           x [Wg|Wu] -> g, u (fp32), h (fp16), (w h)^T (fp16)
-//   GEMM DH           dout_rows Wd^T -> dh = w dhu -> dg, du (bf16 and fp16); <h, dhu>
+//   bwd_gather        xg = x rows (bf16 and fp16), dog = dout rows (fp16), zero padding rows
+//   GEMM GU           x [Wg|Wu] -> g, u, w h (fp16)
+//   GEMM DH           dout_rows Wd^T -> dh = w dhu -> dg, du (bf16 and fp16); <h, dhu> with
+//                     h = silu(clamp g) clamp u recomputed from the stored g, u
 //   GEMM DX           [dg|du] [Wg|Wu]^T -> dx rows (fp16, real row order)
-//   GEMM WG x3        dWd = (w h)^T dout_rows; dWg = xg^T dg; dWu = xg^T du
+//   GEMM WG x3        dWd = (w h)^T dout_rows; dWg = xg^T dg; dWu = xg^T du (A read
+//                     N-major straight from the row buffers: no transposed copy)
 //   zero_untouched    zero weight gradients of experts without rows
 //   combine           dx[t] = sum of its pairs' dx rows (+ shared)
 //   dw_reduce         d topk_w[p] = sum over n-tiles of <h, dhu>
@@ -31,8 +32,10 @@
 // weight-gradient errors: rounding dout and dg to 8 significant bits.) The GEMM kernel is the
 // forward kernel's structure (TMA producer warp, one-thread MMA issuer,
 // four epilogue warps, unit ring, bounded waits) with per-mode loads and
-// epilogues; A is always K-major, B K-major (weights read transposed: DH, DX)
-// or N-major (weights as stored: GU; activations: WG).
+// epilogues; A is K-major (rows) or, for the weight gradients, N-major (the
+// row buffers read as [K = rows, M]); B K-major (weights read transposed: DH,
+// DX) or N-major (weights as stored: GU; activations: WG). The weight-gradient
+// tiles (fp32) go out through shared memory as whole 128-byte row segments.
 #include "gemm_tc.cuh"
 
 namespace moe {
@@ -52,9 +55,13 @@ enum { GU = 0, DH = 1, DX = 2, WG = 3 };
 
 constexpr int kStages = 4;
 constexpr int kStageBytes = A_BYTES + B_BYTES;
-constexpr int kEpiWarps = 4;
+// Eight epilogue warps, two per 32-lane TMEM quadrant, each taking every other
+// 32-column chunk: the epilogues load and store per row (g, u, dg, du, dx, the
+// gradient tiles), and four warps left the MMAs waiting on them.
+constexpr int kEpiWarps = 8;
 constexpr int kThreads = 32 * (2 + kEpiWarps);
-constexpr int kSmem = 1024 + kStages * kStageBytes + 512;
+constexpr int kStageOut = kEpiWarps * 32 * 32 * 4;  // WG: one 32 x 32 fp32 block per epilogue warp
+constexpr int kSmem = 1024 + kStages * kStageBytes + 512 + kStageOut;
 constexpr int kUnitReaders = 1 + kEpiWarps;
 constexpr int kPad = 64;  // rows of an expert are padded to a multiple of this
 
@@ -63,7 +70,7 @@ struct Params {
     int n_tiles;  // output tiles per M-tile
     int E, Etot;
     int d, f;
-    int64_t rp;                // padded rows allocated (row stride of the transposed buffers)
+    int64_t rp;                // padded rows allocated
     int32_t* unit_counter;
     const int32_t* tile_base;  // [Etot+1] prefix of 128-row M-tiles over padded rows
     const int32_t* poff;       // [Etot+1] padded row offsets
@@ -73,13 +80,12 @@ struct Params {
     const float* topk_w;
     float limit;
     // outputs
-    float* gu;         // [rp, 2f] g then u
-    uint16_t* h;       // [rp, f] fp16
-    uint16_t* hwT;     // [f, rp] fp16, w * h transposed
+    uint16_t* gu;      // [rp, 2f] fp16 g then u (outside the clamp: +-next fp16 above L)
+    uint16_t* hw;      // [rp, f] fp16, w * h
     uint16_t* dgu;     // [rp, 2f] bf16, dg then du (operand of DX)
     uint16_t* dgu16;   // [rp, 2f] fp16, the same (operand of the weight gradients)
     uint16_t* dxr;     // [rows, d] fp16, real row order
-    float* dwp;        // [rows, n_tiles of DH] partial <h, dhu>
+    float* dwp;        // [rows, 2 x n_tiles of DH] partial <h, dhu> (per DH n-tile, per epilogue half)
     float* dw;         // WG: routed experts' gradient [E, M, N]
     float* sdw;        // WG: the shared expert's [M, N]
     int M, N;          // WG output dims
@@ -143,98 +149,147 @@ MOE_DEV float silu_f(float z, float& s) {
 }
 
 // Epilogue of one unit: warp quadrant q holds tile rows 32q..32q+31 (lane = row).
+// The fp16 store of a pre-activation for the SwiGLU backward: v itself inside
+// [-L, L] (rounding never leaves it: L is an fp16 value and rounding is
+// monotone), else the next fp16 beyond +-L, so the backward clamps it back to
+// +-L and sees it outside the range exactly when v was.
+MOE_DEV float clamp_code(float v, float L) {
+    if (!(L > 0.f) || fabsf(v) <= L) return v;
+    const float beyond = f16_lo((pack_f16x2(L, 0.f) & 0xFFFFu) + 1u);  // L > 0: one fp16 step above
+    return v > 0.f ? beyond : -beyond;
+}
+
+// Row modes: the padded row this thread writes, its real row (-1 for padding
+// or past the tile) and the pair's gate weight (1 for the shared expert, 0 for
+// padding). Loaded before the accumulator is waited for, so the dependent
+// loads overlap the unit's MMAs.
+struct RowInfo {
+    int real;
+    float w;
+};
+MOE_DEV RowInfo row_info(const Unit& U, int q, int lane, const Params& p) {
+    RowInfo r{-1, 0.f};
+    const int rit = q * 32 + lane;
+    if (rit >= U.rows) return r;
+    const int j = U.row0 + rit - __ldg(p.poff + U.e);
+    const int off = __ldg(p.offsets + U.e);
+    if (j < __ldg(p.offsets + U.e + 1) - off) {
+        r.real = off + j;
+        const int sp = __ldg(p.sorted_pair + r.real);
+        r.w = sp >= 0 ? __ldg(p.topk_w + sp) : 1.0f;
+    }
+    return r;
+}
+
 template <int MODE>
-MOE_DEV void epilogue(uint32_t tb, const Unit& U, int q, int lane, const Params& p, bool& range_bad) {
+MOE_DEV void epilogue(uint32_t tb, const Unit& U, int q, int half, int lane, const Params& p, bool& range_bad,
+                      float* stage_out, RowInfo ri) {
     const int rit = q * 32 + lane;
     const bool valid = rit < U.rows;
     if (MODE == WG) {
-        const int mrow = U.row0 + rit;
-        float* out = (U.e < p.E ? p.dw + int64_t(U.e) * p.M * p.N : p.sdw) + int64_t(mrow) * p.N;
+        // each 32 x 32 fp32 block: lane = row into shared memory (16-byte groups XOR-swizzled by
+        // row, conflict-free), then 4 rows x 128 bytes per warp store instruction
+        float* base = U.e < p.E ? p.dw + int64_t(U.e) * p.M * p.N : p.sdw;
+        const int g8 = lane & 7;
 #pragma unroll 1
-        for (int c = 0; c < BN / 32; ++c) {
+        for (int c = half; c < BN / 32; c += 2) {
             uint32_t v[32];
             tmem_ld_32x32b_x32(tb + c * 32, v);
             tmem_ld_wait();
             const int col = U.n * BN + c * 32;
-            if (valid && col < p.N) {
-                uint4* dst = reinterpret_cast<uint4*>(out + col);
+            if (col >= p.N) break;
 #pragma unroll
-                for (int i = 0; i < 8; ++i) dst[i] = make_uint4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
+            for (int g = 0; g < 8; ++g)
+                *reinterpret_cast<uint4*>(stage_out + lane * 32 + ((g ^ (lane & 7)) << 2)) =
+                    make_uint4(v[4 * g], v[4 * g + 1], v[4 * g + 2], v[4 * g + 3]);
+            __syncwarp();
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+                const int r = 4 * i + (lane >> 3);  // row of this warp's 32
+                const int mrow = U.row0 + q * 32 + r;
+                const uint4 val = *reinterpret_cast<const uint4*>(stage_out + r * 32 + ((g8 ^ (r & 7)) << 2));
+                if (q * 32 + r < U.rows)
+                    *reinterpret_cast<uint4*>(base + int64_t(mrow) * p.N + col + 4 * g8) = val;
             }
+            __syncwarp();
         }
         return;
     }
-    // row modes: padded row -> real row (or padding) and the pair's gate weight
+    // row modes: padded row, its real row (or padding) and the pair's gate weight
     const int64_t prow = int64_t(U.row0) + rit;
-    const int po = __ldg(p.poff + U.e);
-    const int off = __ldg(p.offsets + U.e);
-    const int j = int(prow) - po;
-    const int real = (valid && j < __ldg(p.offsets + U.e + 1) - off) ? off + j : -1;
-    float w = 0.f;
-    if (real >= 0) {
-        const int sp = __ldg(p.sorted_pair + real);
-        w = sp >= 0 ? __ldg(p.topk_w + sp) : 1.0f;
-    }
+    const int real = ri.real;
+    const float w = ri.w;
     const int f = p.f, f2 = 2 * p.f;
     const float L = p.limit;
     if (MODE == GU) {
 #pragma unroll 1
-        for (int c = 0; c < 4; ++c) {
+        for (int c = half; c < 4; c += 2) {
             uint32_t g[32], v[32];
             tmem_ld_32x32b_x32(tb + c * 32, g);
             tmem_ld_32x32b_x32(tb + 128 + c * 32, v);
             tmem_ld_wait();
             const int col = U.n * 128 + c * 32;
             if (valid && col < f) {
+                uint32_t pg[16], pu[16], pw[16];
+#pragma unroll
+                for (int i = 0; i < 16; ++i) {
+                    const float g0 = __uint_as_float(g[2 * i]), g1 = __uint_as_float(g[2 * i + 1]);
+                    const float u0 = __uint_as_float(v[2 * i]), u1 = __uint_as_float(v[2 * i + 1]);
+                    const float h0 = tc::swiglu(g0, u0, L), h1 = tc::swiglu(g1, u1, L);
+                    const float cg0 = clamp_code(g0, L), cg1 = clamp_code(g1, L);
+                    const float cu0 = clamp_code(u0, L), cu1 = clamp_code(u1, L);
+                    range_bad |= !(f16_range_ok(h0) && f16_range_ok(h1) && f16_range_ok(cg0) && f16_range_ok(cg1) &&
+                                   f16_range_ok(cu0) && f16_range_ok(cu1));
+                    pg[i] = pack_f16x2(cg0, cg1);
+                    pu[i] = pack_f16x2(cu0, cu1);
+                    pw[i] = pack_f16x2(w * h0, w * h1);
+                }
                 uint4* gd = reinterpret_cast<uint4*>(p.gu + prow * f2 + col);
                 uint4* ud = reinterpret_cast<uint4*>(p.gu + prow * f2 + f + col);
+                uint4* wd = reinterpret_cast<uint4*>(p.hw + prow * f + col);
 #pragma unroll
-                for (int i = 0; i < 8; ++i) {
-                    gd[i] = make_uint4(g[4 * i], g[4 * i + 1], g[4 * i + 2], g[4 * i + 3]);
-                    ud[i] = make_uint4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
+                for (int i = 0; i < 4; ++i) {
+                    gd[i] = make_uint4(pg[4 * i], pg[4 * i + 1], pg[4 * i + 2], pg[4 * i + 3]);
+                    ud[i] = make_uint4(pu[4 * i], pu[4 * i + 1], pu[4 * i + 2], pu[4 * i + 3]);
+                    wd[i] = make_uint4(pw[4 * i], pw[4 * i + 1], pw[4 * i + 2], pw[4 * i + 3]);
                 }
-                uint32_t pk[16];
-#pragma unroll
-                for (int i = 0; i < 32; i += 2) {
-                    const float h0 = tc::swiglu(__uint_as_float(g[i]), __uint_as_float(v[i]), L);
-                    const float h1 = tc::swiglu(__uint_as_float(g[i + 1]), __uint_as_float(v[i + 1]), L);
-                    range_bad |= !(f16_range_ok(h0) && f16_range_ok(h1));
-                    pk[i / 2] = pack_f16x2(h0, h1);
-                    const uint32_t wh = pack_f16x2(w * h0, w * h1);
-                    p.hwT[int64_t(col + i) * p.rp + prow] = uint16_t(wh & 0xFFFFu);
-                    p.hwT[int64_t(col + i + 1) * p.rp + prow] = uint16_t(wh >> 16);
-                }
-                uint4* hd = reinterpret_cast<uint4*>(p.h + prow * f + col);
-#pragma unroll
-                for (int i = 0; i < 4; ++i) hd[i] = make_uint4(pk[4 * i], pk[4 * i + 1], pk[4 * i + 2], pk[4 * i + 3]);
             }
         }
     } else if (MODE == DH) {
         float dot = 0.f;
 #pragma unroll 1
-        for (int c = 0; c < BN / 32; ++c) {
+        for (int c = half; c < BN / 32; c += 2) {
             uint32_t v[32];
             tmem_ld_32x32b_x32(tb + c * 32, v);
             tmem_ld_wait();
             const int col = U.n * BN + c * 32;
             if (valid && col < f) {
-                const float* gp = p.gu + prow * f2 + col;
-                const float* up = gp + f;
-                const uint32_t* hp = reinterpret_cast<const uint32_t*>(p.h + prow * f + col);
+                // the chunk's g and u (fp16) in 8 vector loads issued together; h = silu(gc) uc
+                // is recomputed from them for the routing-weight dot
+                uint4 gq4[4], uq4[4];
+                const uint4* gsrc = reinterpret_cast<const uint4*>(p.gu + prow * f2 + col);
+                const uint4* usrc = reinterpret_cast<const uint4*>(p.gu + prow * f2 + f + col);
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    gq4[i] = gsrc[i];
+                    uq4[i] = usrc[i];
+                }
+                const uint32_t* gw = reinterpret_cast<const uint32_t*>(gq4);
+                const uint32_t* uw = reinterpret_cast<const uint32_t*>(uq4);
                 uint32_t pg[16], pu[16], qg[16], qu[16];
 #pragma unroll
                 for (int i = 0; i < 32; i += 2) {
-                    const uint32_t hh = hp[i / 2];
+                    const uint32_t gg = gw[i / 2], uu = uw[i / 2];
                     float dgv[2], duv[2];
 #pragma unroll
                     for (int s2 = 0; s2 < 2; ++s2) {
                         const float dhu = __uint_as_float(v[i + s2]);
-                        dot += (s2 ? f16_hi(hh) : f16_lo(hh)) * dhu;
-                        const float gv = gp[i + s2], uv = up[i + s2];
+                        const float gv = s2 ? f16_hi(gg) : f16_lo(gg), uv = s2 ? f16_hi(uu) : f16_lo(uu);
                         const float gc = L > 0.f ? fminf(fmaxf(gv, -L), L) : gv;
                         const float uc = L > 0.f ? fminf(fmaxf(uv, -L), L) : uv;
                         float sg;
                         const float sl = silu_f(gc, sg);
+                        dot += sl * uc * dhu;  // h = silu(gc) uc
                         const float dh = w * dhu;
                         const bool pg_ = !(L > 0.f) || fabsf(gv) <= L;
                         const bool pu_ = !(L > 0.f) || fabsf(uv) <= L;
@@ -261,10 +316,10 @@ MOE_DEV void epilogue(uint32_t tb, const Unit& U, int q, int lane, const Params&
                 }
             }
         }
-        if (real >= 0) p.dwp[int64_t(real) * p.n_tiles + U.n] = dot;
+        if (real >= 0) p.dwp[(int64_t(real) * p.n_tiles + U.n) * 2 + half] = dot;
     } else {  // DX
 #pragma unroll 1
-        for (int c = 0; c < BN / 32; ++c) {
+        for (int c = half; c < BN / 32; c += 2) {
             uint32_t v[32];
             tmem_ld_32x32b_x32(tb + c * 32, v);
             tmem_ld_wait();
@@ -307,6 +362,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     volatile int* unit_ring = reinterpret_cast<volatile int*>(uempty + UR);
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(const_cast<int*>(unit_ring) + UR);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+    float* stage_out = reinterpret_cast<float*>(smem + kStages * kStageBytes + 512);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     if (threadIdx.x == 0) {
@@ -381,7 +437,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                     uint8_t* sb = sa + A_BYTES;
                     mbar_arrive_expect_tx(full + stage, A_BYTES + B_BYTES);
                     if (MODE == WG) {
-                        tma_load_2d(sa, &tmA, full + stage, po + kb * BK, U.row0);
+                        // A: 128 M-columns of the row buffer (two 64-wide chunks) x 64 K-rows, N-major
+                        tma_load_4d(sa, &tmA, full + stage, 0, po + kb * BK, 2 * U.m, 0);
                         tma_load_4d(sb, &tmB0, full + stage, 0, po + kb * BK, 4 * U.n, 0);
                     } else {
                         tma_load_2d(sa, &tmA, full + stage, kb * BK, U.row0);
@@ -414,8 +471,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     } else if (warp == 1) {
         // ------------------------------------------------ MMA issuer
         constexpr bool kBmn = MODE == GU || MODE == WG;  // B N-major (else K-major)
+        constexpr bool kAmn = MODE == WG;                // A N-major (else K-major)
         constexpr int kBf16 = (MODE == GU || MODE == DX) ? 1 : 0;  // else fp16 x fp16
-        constexpr uint32_t IDESC = idesc_f16_f32(BM, BN, kBf16, /*a_mn=*/0, /*b_mn=*/kBmn ? 1 : 0);
+        constexpr uint32_t IDESC = idesc_f16_f32(BM, BN, kBf16, kAmn ? 1 : 0, kBmn ? 1 : 0);
         int stage = 0, acc = 0;
         uint32_t phase = 0, acc_phase = 0;
         bool ok = true;
@@ -445,7 +503,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                     const uint32_t b0 = a0 + A_BYTES;
 #pragma unroll
                     for (int jj = 0; jj < BK / 16; ++jj) {
-                        const uint64_t ad = sdesc_sw128(a0 + jj * 32, 16, 1024);
+                        const uint64_t ad =
+                            kAmn ? sdesc_sw128(a0 + jj * 2048, B_CHUNK, 1024) : sdesc_sw128(a0 + jj * 32, 16, 1024);
                         const uint64_t bd =
                             kBmn ? sdesc_sw128(b0 + jj * 2048, B_CHUNK, 1024) : sdesc_sw128(b0 + jj * 32, 16, 1024);
                         umma_bf16(d_tmem, ad, bd, IDESC, (kb | jj) != 0);
@@ -472,8 +531,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         __syncwarp();
     } else {
-        // ------------------------------------------------ epilogue (warps 2..5)
-        const int q = warp & 3;
+        // ------------------------------------------------ epilogue (warps 2 .. 2+kEpiWarps-1)
+        const int q = warp & 3;                // TMEM lanes 32q .. 32q+31
+        const int half = (warp - 2) / 4;       // every other 32-column chunk
         int acc = 0;
         uint32_t acc_phase = 0;
         bool range_bad = false;
@@ -484,13 +544,14 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (!tc::ring_read(u, uslot, uphase, unit_ring, ufull, uempty, abort_flag, p.err, p.wait_ns)) break;
             if (u < 0) break;
             const Unit U = decode<MODE>(u, p);
+            const RowInfo ri = MODE == WG ? RowInfo{-1, 0.f} : row_info(U, q, lane, p);
             int okl = 1;
             if (lane == 0) okl = mbar_wait_bounded(tfull + acc, acc_phase, abort_flag, p.err, p.wait_ns);
             okl = __shfl_sync(0xFFFFFFFFu, okl, 0);
             if (!okl) break;
             tc_fence_after();
             const uint32_t tb = tmem_base + (uint32_t(q * 32) << 16) + uint32_t(acc * BN);
-            epilogue<MODE>(tb, U, q, lane, p, range_bad);
+            epilogue<MODE>(tb, U, q, half, lane, p, range_bad, stage_out + (warp - 2) * 32 * 32, ri);
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(tempty + acc);
@@ -564,14 +625,16 @@ __global__ void __launch_bounds__(512) bwd_schedule_kernel(const int32_t* __rest
     if (e < 8) counters[e] = 0;
 }
 
-// One warp per padded row (grid-stride): xg = x[token], dog = bf16(dout[token]),
-// zero for padding rows. Rows past poff[Etot] are not touched.
+// One warp per padded row (grid-stride): xg = x[token] (bf16, for the products
+// with the bf16 gate/up weights) and its fp16 copy xg16 (exact for x in fp16's
+// range; for the weight gradients), dog = fp16(dout[token]); zero for padding
+// rows. Rows past poff[Etot] are not touched.
 __global__ void __launch_bounds__(256) bwd_gather_kernel(const uint16_t* __restrict__ x, const float* __restrict__ dout,
                                                          const int32_t* __restrict__ sorted_token,
                                                          const int32_t* __restrict__ offsets,
                                                          const int32_t* __restrict__ poff, int Etot, int T, int d,
-                                                         uint16_t* __restrict__ xg, uint16_t* __restrict__ dog,
-                                                         uint32_t* err) {
+                                                         uint16_t* __restrict__ xg, uint16_t* __restrict__ xg16,
+                                                         uint16_t* __restrict__ dog, uint32_t* err) {
     griddep_wait();
     griddep_launch();
     const int lane = threadIdx.x & 31;
@@ -596,6 +659,7 @@ __global__ void __launch_bounds__(256) bwd_gather_kernel(const uint16_t* __restr
             }
         }
         uint4* xo = reinterpret_cast<uint4*>(xg + pr * d);
+        uint4* xh = reinterpret_cast<uint4*>(xg16 + pr * d);
         uint4* go = reinterpret_cast<uint4*>(dog + pr * d);
         for (int c = lane; c < d / 8; c += 32) {
             uint4 xv = make_uint4(0, 0, 0, 0), gv = make_uint4(0, 0, 0, 0);
@@ -609,30 +673,16 @@ __global__ void __launch_bounds__(256) bwd_gather_kernel(const uint16_t* __restr
                          f16_range_ok(b.x) && f16_range_ok(b.y) && f16_range_ok(b.z) && f16_range_ok(b.w));
             }
             xo[c] = xv;
+            xh[c] = make_uint4(bf16x2_to_f16x2(xv.x), bf16x2_to_f16x2(xv.y), bf16x2_to_f16x2(xv.z),
+                               bf16x2_to_f16x2(xv.w));
             go[c] = gv;
         }
     }
     if (bad) set_error(err, MOE_DEVERR_RANGE);
 }
 
-// xgT[c, r] = fp16(xg[r, c]) for the used padded rows; 32 x 32 tiles through
-// shared memory (bf16 -> fp16 is exact for values in fp16's range).
-__global__ void __launch_bounds__(256) transpose_kernel(const uint16_t* __restrict__ xg, const int32_t* __restrict__ poff,
-                                                        int Etot, int d, int64_t rp, uint16_t* __restrict__ xgT) {
-    __shared__ uint16_t tile[32][33];
-    griddep_wait();
-    griddep_launch();
-    const int64_t r0 = int64_t(blockIdx.y) * 32;
-    if (r0 >= poff[Etot]) return;
-    const int c0 = blockIdx.x * 32;
-    const int tx = threadIdx.x & 31, ty = threadIdx.x >> 5;  // 32 x 8
-    for (int i = ty; i < 32; i += 8) tile[i][tx] = xg[(r0 + i) * d + c0 + tx];
-    __syncthreads();
-    for (int i = ty; i < 32; i += 8)
-        xgT[int64_t(c0 + i) * rp + r0 + tx] = uint16_t(pack_f16x2(bf16_to_f32(tile[tx][i]), 0.f) & 0xFFFFu);
-}
-
-// d topk_w[p] = sum over the DH n-tiles of <h, dhu> of the pair's row; 0 if dropped.
+// d topk_w[p] = sum over the DH n-tiles (and both epilogue halves, in order) of
+// <h, dhu> of the pair's row; 0 if dropped.
 __global__ void __launch_bounds__(256) dw_reduce_kernel(const int32_t* __restrict__ pair_row,
                                                         const float* __restrict__ dwp, int64_t pairs, int nt,
                                                         int64_t rows, float* __restrict__ d_topk_w, uint32_t* err) {
@@ -646,7 +696,7 @@ __global__ void __launch_bounds__(256) dw_reduce_kernel(const int32_t* __restric
         }
         float s = 0.f;
         if (r >= 0)
-            for (int n = 0; n < nt; ++n) s += dwp[int64_t(r) * nt + n];
+            for (int n = 0; n < 2 * nt; ++n) s += dwp[int64_t(r) * 2 * nt + n];
         d_topk_w[q] = s;
     }
 }
@@ -716,7 +766,7 @@ cudaError_t launch_mode(const CUtensorMap& A, const CUtensorMap& B0, const CUten
 
 namespace tc {
 bool map_weights_kmajor(CUtensorMap* m, const void* base, int nexp, int N, int K, bool f16 = false);
-bool map_act_mn(CUtensorMap* m, const void* base, int64_t rows, int N, int64_t row_stride);
+bool map_act_mn(CUtensorMap* m, const void* base, int64_t rows, int N, int64_t row_stride, int chunks);
 }  // namespace tc
 
 int64_t bwd_padded_rows(const Dims& D) { return (D.rows + bwd::kPad - 1) / bwd::kPad * bwd::kPad + int64_t(bwd::kPad) * D.Etot; }
@@ -732,11 +782,10 @@ cudaError_t launch_backward(const Dims& D, const BwdArgs& a, cudaStream_t s) {
     int32_t* wbase = reinterpret_cast<int32_t*>(ws + L.b_wbase);
     int32_t* counters = reinterpret_cast<int32_t*>(ws + L.b_counters);
     uint16_t* xg = reinterpret_cast<uint16_t*>(ws + L.b_xg);
-    uint16_t* xgT = reinterpret_cast<uint16_t*>(ws + L.b_xgT);
+    uint16_t* xg16 = reinterpret_cast<uint16_t*>(ws + L.b_xg16);
     uint16_t* dog = reinterpret_cast<uint16_t*>(ws + L.b_dog);
-    float* gu = reinterpret_cast<float*>(ws + L.b_gu);
-    uint16_t* h = reinterpret_cast<uint16_t*>(ws + L.b_h);
-    uint16_t* hwT = reinterpret_cast<uint16_t*>(ws + L.b_hwT);
+    uint16_t* gu = reinterpret_cast<uint16_t*>(ws + L.b_gu);
+    uint16_t* hw = reinterpret_cast<uint16_t*>(ws + L.b_hw);
     uint16_t* dgu = reinterpret_cast<uint16_t*>(ws + L.b_dgu);
     uint16_t* dgu16 = reinterpret_cast<uint16_t*>(ws + L.b_dgu16);
     uint16_t* dxr = reinterpret_cast<uint16_t*>(ws + L.b_dxr);
@@ -753,22 +802,19 @@ cudaError_t launch_backward(const Dims& D, const BwdArgs& a, cudaStream_t s) {
         int64_t blocks = (rp + 7) / 8;
         if (blocks > int64_t(num_sms()) * 8) blocks = int64_t(num_sms()) * 8;
         if ((e = launch_pdl(false, bwd_gather_kernel, dim3(int(blocks)), dim3(256), 0, s, a.x, a.dout, a.sorted_token,
-                            a.offsets, poff, Etot, D.T, d, xg, dog, a.err)) != cudaSuccess)
-            return e;
-        if ((e = launch_pdl(false, transpose_kernel, dim3(d / 32, unsigned(rp / 32)), dim3(256), 0, s, xg, poff, Etot,
-                            d, rp, xgT)) != cudaSuccess)
+                            a.offsets, poff, Etot, D.T, d, xg, xg16, dog, a.err)) != cudaSuccess)
             return e;
     }
     const moe_weights* w = a.w;
-    CUtensorMap mX, mDog, mDgu, mHwT, mXgT;
+    CUtensorMap mX, mDog, mDgu, mHwN, mXgN;
     CUtensorMap mG, mU, mGk, mUk, mDk, sG, sU, sGk, sUk, sDk, mDogN, mDgN, mDuN;
     if (!tc::map_rows(&mX, xg, rp, d) || !tc::map_rows(&mDog, dog, rp, d) || !tc::map_rows(&mDgu, dgu, rp, 2 * f) ||
-        !tc::map_rows(&mHwT, hwT, f, int(rp)) || !tc::map_rows(&mXgT, xgT, d, int(rp)) ||
+        !tc::map_act_mn(&mHwN, hw, rp, f, f, 2) || !tc::map_act_mn(&mXgN, xg16, rp, d, d, 2) ||
         !tc::map_weights(&mG, w->w_gate, D.E, d, f, 2) || !tc::map_weights(&mU, w->w_up, D.E, d, f, 2) ||
         !tc::map_weights_kmajor(&mGk, w->w_gate, D.E, d, f) || !tc::map_weights_kmajor(&mUk, w->w_up, D.E, d, f) ||
-        !tc::map_weights_kmajor(&mDk, w->w_down, D.E, f, d, true) || !tc::map_act_mn(&mDogN, dog, rp, d, d) ||
-        !tc::map_act_mn(&mDgN, dgu16, rp, f, 2 * int64_t(f)) ||
-        !tc::map_act_mn(&mDuN, dgu16 + f, rp, f, 2 * int64_t(f)))
+        !tc::map_weights_kmajor(&mDk, w->w_down, D.E, f, d, true) || !tc::map_act_mn(&mDogN, dog, rp, d, d, 4) ||
+        !tc::map_act_mn(&mDgN, dgu16, rp, f, 2 * int64_t(f), 4) ||
+        !tc::map_act_mn(&mDuN, dgu16 + f, rp, f, 2 * int64_t(f), 4))
         return cudaErrorInvalidValue;
     if (D.has_shared) {
         if (!tc::map_weights(&sG, w->shared_gate, 1, d, f, 2) || !tc::map_weights(&sU, w->shared_up, 1, d, f, 2) ||
@@ -797,8 +843,7 @@ cudaError_t launch_backward(const Dims& D, const BwdArgs& a, cudaStream_t s) {
     p.topk_w = a.topk_w;
     p.limit = D.limit;
     p.gu = gu;
-    p.h = h;
-    p.hwT = hwT;
+    p.hw = hw;
     p.dgu = dgu;
     p.dgu16 = dgu16;
     p.dxr = dxr;
@@ -827,17 +872,17 @@ cudaError_t launch_backward(const Dims& D, const BwdArgs& a, cudaStream_t s) {
     p.dw = a.g->dw_down;
     p.sdw = a.g->dshared_down;
     p.unit_counter = counters + 3;
-    if ((e = launch_mode<WG>(mHwT, mDogN, mDogN, mDogN, mDogN, p, s)) != cudaSuccess) return e;
+    if ((e = launch_mode<WG>(mHwN, mDogN, mDogN, mDogN, mDogN, p, s)) != cudaSuccess) return e;
     p.M = d;
     p.N = f;
     p.dw = a.g->dw_gate;
     p.sdw = a.g->dshared_gate;
     p.unit_counter = counters + 4;
-    if ((e = launch_mode<WG>(mXgT, mDgN, mDgN, mDgN, mDgN, p, s)) != cudaSuccess) return e;
+    if ((e = launch_mode<WG>(mXgN, mDgN, mDgN, mDgN, mDgN, p, s)) != cudaSuccess) return e;
     p.dw = a.g->dw_up;
     p.sdw = a.g->dshared_up;
     p.unit_counter = counters + 5;
-    if ((e = launch_mode<WG>(mXgT, mDuN, mDuN, mDuN, mDuN, p, s)) != cudaSuccess) return e;
+    if ((e = launch_mode<WG>(mXgN, mDuN, mDuN, mDuN, mDuN, p, s)) != cudaSuccess) return e;
     {
         ProfScope prof_(MOE_K_BWD_SMALL, s);
         const int64_t per = int64_t(d) * f;

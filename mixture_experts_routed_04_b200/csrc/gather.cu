@@ -1,14 +1,16 @@
 // gather.cu — S4: the row gather. xg[r] = x[sorted_token[r]] for every row
 // of every expert, in expert order, so the GEMMs' A operand (and the streaming
 // kernels' rows tile) is a plain TMA box. A gather inside the GEMM (TMA
-// tile::gather4 or cp.async warps) was measured slower on B200, and so was a
-// 4-way unrolled version of this loop.
+// tile::gather4, or cp.async warps: gemm_tc.cu's GATHER kernels) was measured
+// slower on B200.
 #include "internal.h"
 
 namespace moe {
 
-// xg[r] = x[sorted_token[r]] for r < offsets[Etot]; 16-byte vectors. TO_F16:
-// bf16 -> fp16 on the way (the Q4G32 path runs its MMAs in fp16).
+// xg[r] = x[sorted_token[r]] for r < offsets[Etot]. One warp per row (grid
+// stride): the row's token is read once, then each lane moves up to eight
+// 16-byte vectors of the row with all its loads in flight before its stores.
+// TO_F16: bf16 -> fp16 on the way (the Q4G32 path runs its MMAs in fp16).
 template <bool TO_F16>
 __global__ void __launch_bounds__(256) gather_rows_kernel(const uint16_t* __restrict__ x,
                                                           const int32_t* __restrict__ sorted_token,
@@ -16,24 +18,39 @@ __global__ void __launch_bounds__(256) gather_rows_kernel(const uint16_t* __rest
                                                           int T, uint16_t* __restrict__ xg, uint32_t* err) {
     griddep_wait();
     griddep_launch();
+    const int lane = threadIdx.x & 31;
     const int vec = d / 8;
-    const int64_t total = int64_t(offsets[Etot]) * vec;
-    for (int64_t i = int64_t(blockIdx.x) * blockDim.x + threadIdx.x; i < total; i += int64_t(gridDim.x) * blockDim.x) {
-        const int64_t r = i / vec;
-        const int c = int(i - r * vec);
+    const int64_t rows = offsets[Etot];
+    const int64_t warps = int64_t(gridDim.x) * (blockDim.x >> 5);
+    for (int64_t r = int64_t(blockIdx.x) * (blockDim.x >> 5) + (threadIdx.x >> 5); r < rows; r += warps) {
         const int t = __ldg(sorted_token + r);
         if (t < 0 || t >= T) {
-            set_error(err, MOE_DEVERR_BOUNDS);
+            if (lane == 0) set_error(err, MOE_DEVERR_BOUNDS);
             continue;
         }
-        uint4 v = __ldg(reinterpret_cast<const uint4*>(x + int64_t(t) * d) + c);
-        if (TO_F16) {
-            v.x = bf16x2_to_f16x2(v.x);
-            v.y = bf16x2_to_f16x2(v.y);
-            v.z = bf16x2_to_f16x2(v.z);
-            v.w = bf16x2_to_f16x2(v.w);
+        const uint4* src = reinterpret_cast<const uint4*>(x + int64_t(t) * d);
+        uint4* dst = reinterpret_cast<uint4*>(xg + r * d);
+        for (int c0 = 0; c0 < vec; c0 += 8 * 32) {
+            uint4 v[8];
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+                const int c = c0 + i * 32 + lane;
+                if (c < vec) v[i] = __ldg(src + c);
+            }
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+                const int c = c0 + i * 32 + lane;
+                if (c < vec) {
+                    if (TO_F16) {
+                        v[i].x = bf16x2_to_f16x2(v[i].x);
+                        v[i].y = bf16x2_to_f16x2(v[i].y);
+                        v[i].z = bf16x2_to_f16x2(v[i].z);
+                        v[i].w = bf16x2_to_f16x2(v[i].w);
+                    }
+                    dst[c] = v[i];
+                }
+            }
         }
-        reinterpret_cast<uint4*>(xg + r * d)[c] = v;
     }
 }
 
@@ -101,8 +118,7 @@ cudaError_t launch_scatter_rows(const Dims& D, const uint16_t* x, const int32_t*
 
 cudaError_t launch_gather(const Dims& D, const uint16_t* x, const int32_t* sorted_token, const int32_t* offsets,
                           uint16_t* xg, uint32_t* err, cudaStream_t s) {
-    const int64_t total = D.rows * (D.d / 8);
-    int64_t blocks = (total + 255) / 256;
+    int64_t blocks = (D.rows + 7) / 8;  // 8 warps (rows) per block
     const int64_t cap = int64_t(num_sms()) * 8;
     if (blocks > cap) blocks = cap;
     if (blocks < 1) blocks = 1;

@@ -577,12 +577,13 @@ bool map_weights_kmajor(CUtensorMap* m, const void* base, int nexp, int N, int K
     return make_map(m, f16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, base, 3, dims, str,
                     box, CU_TENSOR_MAP_SWIZZLE_128B);
 }
-// 2-byte activation rows [rows, N] (row stride row_stride elements) read as an N-major B
-// operand (K = rows): seen as [1, N/64 chunks, rows, 64]; one copy brings 4 chunks.
-bool map_act_mn(CUtensorMap* m, const void* base, int64_t rows, int N, int64_t row_stride) {
+// 2-byte activation rows [rows, N] (row stride row_stride elements) read as an N-major
+// operand with K = rows: seen as [1, N/64 chunks, rows, 64]; one copy brings `chunks`
+// 64-column chunks of 64 K-rows (4 for a 256-wide B, 2 for a 128-wide A).
+bool map_act_mn(CUtensorMap* m, const void* base, int64_t rows, int N, int64_t row_stride, int chunks) {
     const uint64_t dims[4] = {64, uint64_t(rows), uint64_t(N / 64), 1};
     const uint64_t str[3] = {uint64_t(row_stride) * 2, 128, uint64_t(row_stride) * uint64_t(rows) * 2};
-    const uint32_t box[4] = {64, 64, 4, 1};
+    const uint32_t box[4] = {64, 64, uint32_t(chunks), 1};
     return make_map(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, base, 4, dims, str, box, CU_TENSOR_MAP_SWIZZLE_128B);
 }
 // Q4G32 nibbles: [nexp, N, K/2] bytes; box 32 bytes (64 k) x rows x 1, no swizzle.

@@ -50,7 +50,7 @@ struct WsLayout {
     size_t x_dev, logits_dev, out_dev;             // forward_host
     size_t stats_p, stats_c, stats_s;              // route_stats: per-block partial sums
     // backward (padded row space, see backward.cu)
-    size_t b_poff, b_tile_base, b_wbase, b_counters, b_xg, b_xgT, b_dog, b_gu, b_h, b_hwT, b_dgu, b_dgu16, b_dxr, b_dwp;
+    size_t b_poff, b_tile_base, b_wbase, b_counters, b_xg, b_xg16, b_dog, b_gu, b_hw, b_dgu, b_dgu16, b_dxr, b_dwp;
     size_t total;
 };
 

@@ -41,14 +41,21 @@ __global__ void __launch_bounds__(256) route_topk_softmax_kernel(const float* __
 //
 // route_stats_kernel: one warp per token as in the router (the same
 // route_one_token, so idx and w are those of moe_route), then over the same
-// token: max and sum of exp over all E (warp reductions), and selection
-// rounds in descending order (ties to the lower index) summing exp in that
-// order until the top-k mass and the 90% count are both known. Each block
+// token: max and sum of exp over all E (warp reductions); the top-k mass from
+// the k-th selected key (every value above it plus enough of its ties); the
+// 90% count by bisection over the 32-bit order-preserving keys for the
+// largest threshold whose values hold >= 90% of the mass (32 rounds of a masked
+// warp sum, whatever E), then as many of that value's ties as the remaining
+// mass needs — the count of the largest-first definition. Each block
 // keeps per-expert sums of p and first-choice counts, reduced over its warps
-// in warp order into one row of partials; route_stats_final sums the rows in
-// block order (fp64). Fixed orders throughout: the results are deterministic.
+// in warp order into one row of partials; route_stats_final sums the rows
+// (fp64, lanes over block rows, then a fixed shuffle tree). Fixed orders
+// throughout: the results are deterministic.
 
 constexpr int kStatsWarps = 8;
+// Partial rows a lane of the final sum reads: the telemetry kernel runs at most
+// 32 x this many blocks (route_stats_blocks).
+constexpr int kStatsMaxRowsPerLane = 16;
 constexpr float kWantMass = 0.9f;
 
 template <bool PER_TOKEN>
@@ -72,7 +79,8 @@ __global__ void __launch_bounds__(kStatsWarps * 32)
     float a_kept = 0.f, a_want = 0.f, a_z = 0.f;
     for (int64_t t = int64_t(blockIdx.x) * kStatsWarps + w; t < T; t += int64_t(gridDim.x) * kStatsWarps) {
         const float* row = logits + t * E;
-        const int first = route_one_token(row, E, k, topk_idx + t * k, topk_w + t * k);
+        uint32_t kth = 0;
+        const int first = route_one_token(row, E, k, topk_idx + t * k, topk_w + t * k, &kth);
         float v[kRouteMaxPerLane];
         uint32_t key[kRouteMaxPerLane];
         float mx = -INFINITY;
@@ -99,33 +107,59 @@ __global__ void __launch_bounds__(kStatsWarps * 32)
             accp[i] += ex[i] * inv;
             accc[i] += (lane + 32 * i == first) ? 1 : 0;
         }
-        // selection rounds, largest first, ties to the lower index (as the router)
-        uint32_t taken = 0;
-#pragma unroll
-        for (int i = 0; i < kRouteMaxPerLane; ++i)
-            if (lane + 32 * i >= E) taken |= 1u << i;
-        const float thr = kWantMass * S;
-        float cum = 0.f, kept_t = 0.f;
-        int want = 0;
-        for (int r = 0; r < E; ++r) {
-            uint32_t bk = 0;
-            int bi = 0x7FFFFFFF;
+        // mass and count of the values whose key is > tau (over the valid experts)
+        auto above = [&](uint32_t tau, float& mass, int& cnt) {
+            float m = 0.f;
+            int c = 0;
 #pragma unroll
             for (int i = 0; i < kRouteMaxPerLane; ++i)
-                if (!(taken >> i & 1u) && (key[i] > bk || bi == 0x7FFFFFFF)) {
-                    bk = key[i];
-                    bi = lane + 32 * i;
+                if (lane + 32 * i < E && key[i] > tau) {
+                    m += ex[i];
+                    ++c;
                 }
-            const uint32_t kmax = __reduce_max_sync(0xFFFFFFFFu, bk);
-            const int wi =
-                int(__reduce_min_sync(0xFFFFFFFFu, (bi != 0x7FFFFFFF && bk == kmax) ? uint32_t(bi) : 0xFFFFFFFFu));
-            if ((wi & 31) == lane) taken |= 1u << (wi >> 5);
-            cum += expf(route_unkey(kmax) - mx);
-            if (r == k - 1) kept_t = cum * inv;
-            if (want == 0 && cum >= thr) want = r + 1;
-            if (want != 0 && r >= k - 1) break;
+#pragma unroll
+            for (int off = 16; off > 0; off >>= 1) {
+                m += __shfl_xor_sync(0xFFFFFFFFu, m, off);
+                c += __shfl_xor_sync(0xFFFFFFFFu, c, off);
+            }
+            mass = m;
+            cnt = c;
+        };
+        // kept: the k selected = every value above the k-th key plus enough of its ties
+        float m_above;
+        int c_above;
+        above(kth, m_above, c_above);
+        const float e_kth = expf(route_unkey(kth) - mx);
+        const float kept_t = (m_above + float(k - c_above) * e_kth) * inv;
+        // want: tau* = the largest key whose values at or above it hold >= 90% of the mass
+        // (bisection over the 32-bit keys; mass(key >= tau) = mass(key > tau - 1)); then
+        // the values above tau* plus as many of its ties as the remaining mass needs, in
+        // the largest-first order of the definition
+        const float thr = kWantMass * S;
+        // the rounds need only the mass (one warp sum; the count is taken once at the end)
+        auto mass_above = [&](uint32_t tau) {
+            float m = 0.f;
+#pragma unroll
+            for (int i = 0; i < kRouteMaxPerLane; ++i)
+                if (lane + 32 * i < E && key[i] > tau) m += ex[i];
+#pragma unroll
+            for (int off = 16; off > 0; off >>= 1) m += __shfl_xor_sync(0xFFFFFFFFu, m, off);
+            return m;
+        };
+        uint32_t lo = 0u, hi = 0xFFFFFFFFu;
+        while (lo < hi) {
+            const uint32_t mid = lo + ((hi - lo) >> 1) + 1u;
+            if (mass_above(mid - 1u) >= thr) lo = mid;
+            else hi = mid - 1u;
         }
-        if (want == 0) want = E;  // the whole mass, up to rounding
+        above(lo, m_above, c_above);
+        const float e_tau = expf(route_unkey(lo) - mx);
+        int want = c_above;
+        float cum = m_above;
+        do {
+            cum += e_tau;
+            ++want;
+        } while (cum < thr && want < E);
         a_kept += kept_t;
         a_want += float(want);
         const float lse = mx + logf(S);
@@ -156,8 +190,9 @@ __global__ void __launch_bounds__(kStatsWarps * 32)
             a += sp[j][e];
             c += sc[j][e];
         }
-        part_p[int64_t(blockIdx.x) * E + e] = a;
-        part_c[int64_t(blockIdx.x) * E + e] = c;
+        // expert-major [E, blocks]: the final sum reads each expert's rows contiguously
+        part_p[int64_t(e) * gridDim.x + blockIdx.x] = a;
+        part_c[int64_t(e) * gridDim.x + blockIdx.x] = c;
     }
     if (threadIdx.x < 3) {
         float a = 0.f;
@@ -166,10 +201,19 @@ __global__ void __launch_bounds__(kStatsWarps * 32)
     }
 }
 
-// One block: thread e sums expert e's partial rows in block order; then the
-// scalars. stats = {kept, want_k, balance, z, aux}; expert_stats (nullable) =
-// {frac [E], prob_mean [E]}.
-__global__ void __launch_bounds__(kMaxE) route_stats_final(const float* __restrict__ part_p,
+// One block of 1024 threads: warp w takes experts w, w + 32, ...; lane l sums
+// block rows l, l + 32, ... (fp64; the partials are expert-major, so a warp's
+// loads are coalesced) and a fixed shuffle tree adds the lanes, so
+// the order of every sum is fixed. Then warp 0 sums the balance terms and the
+// scalars the same way. stats = {kept, want_k, balance, z, aux}; expert_stats
+// (nullable) = {frac [E], prob_mean [E]}.
+MOE_DEV double warp_sum_fixed(double v) {
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) v += __shfl_xor_sync(0xFFFFFFFFu, v, off);
+    return v;
+}
+
+__global__ void __launch_bounds__(1024) route_stats_final(const float* __restrict__ part_p,
                                                           const int32_t* __restrict__ part_c,
                                                           const float* __restrict__ part_s, int nblk, int T, int E,
                                                           float z_weight, float* __restrict__ stats,
@@ -177,45 +221,69 @@ __global__ void __launch_bounds__(kMaxE) route_stats_final(const float* __restri
     __shared__ double term[kMaxE];
     griddep_wait();
     griddep_launch();
-    const int e = threadIdx.x;
-    double pm = 0.0;
-    long long cnt = 0;
-    if (e < E) {
-        for (int b = 0; b < nblk; ++b) {
-            pm += double(part_p[int64_t(b) * E + e]);
-            cnt += part_c[int64_t(b) * E + e];
+    const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
+    for (int e = w; e < E; e += 32) {
+        // this lane's block rows b = lane + 32 j, loaded into registers first (all in
+        // flight together), then summed in j order
+        float vp[kStatsMaxRowsPerLane];
+        int vc[kStatsMaxRowsPerLane];
+#pragma unroll
+        for (int j = 0; j < kStatsMaxRowsPerLane; ++j) {
+            const int b = lane + 32 * j;
+            vp[j] = b < nblk ? part_p[int64_t(e) * nblk + b] : 0.f;
+            vc[j] = b < nblk ? part_c[int64_t(e) * nblk + b] : 0;
         }
-        pm /= double(T);
-        const double frac = double(cnt) / double(T);
-        term[e] = frac * pm;
-        if (expert_stats) {
-            expert_stats[e] = float(frac);
-            expert_stats[E + e] = float(pm);
+        double pm = 0.0, cnt = 0.0;
+#pragma unroll
+        for (int j = 0; j < kStatsMaxRowsPerLane; ++j) {
+            pm += double(vp[j]);
+            cnt += double(vc[j]);
+        }
+        pm = warp_sum_fixed(pm) / double(T);
+        const double frac = warp_sum_fixed(cnt) / double(T);
+        if (lane == 0) {
+            term[e] = frac * pm;
+            if (expert_stats) {
+                expert_stats[e] = float(frac);
+                expert_stats[E + e] = float(pm);
+            }
         }
     }
     __syncthreads();
-    if (e == 0) {
-        double bal = 0.0, s[3] = {0.0, 0.0, 0.0};
-        for (int j = 0; j < E; ++j) bal += term[j];
-        bal *= double(E);
-        for (int b = 0; b < nblk; ++b)
-            for (int j = 0; j < 3; ++j) s[j] += double(part_s[b * 3 + j]);
-        const double z = s[2] / double(T);
-        stats[0] = float(s[0] / double(T));
-        stats[1] = float(s[1] / double(T));
-        stats[2] = float(bal);
-        stats[3] = float(z);
-        stats[4] = float(bal + double(z_weight) * z);
+    if (w == 0) {
+        double bal = 0.0, sc[3] = {0.0, 0.0, 0.0};
+        for (int e = lane; e < E; e += 32) bal += term[e];
+        float vs[kStatsMaxRowsPerLane][3];
+#pragma unroll
+        for (int jb = 0; jb < kStatsMaxRowsPerLane; ++jb) {
+            const int b = lane + 32 * jb;
+#pragma unroll
+            for (int j = 0; j < 3; ++j) vs[jb][j] = b < nblk ? part_s[b * 3 + j] : 0.f;
+        }
+#pragma unroll
+        for (int jb = 0; jb < kStatsMaxRowsPerLane; ++jb)
+#pragma unroll
+            for (int j = 0; j < 3; ++j) sc[j] += double(vs[jb][j]);
+        bal = warp_sum_fixed(bal) * double(E);
+        for (int j = 0; j < 3; ++j) sc[j] = warp_sum_fixed(sc[j]);
+        if (lane == 0) {
+            const double z = sc[2] / double(T);
+            stats[0] = float(sc[0] / double(T));
+            stats[1] = float(sc[1] / double(T));
+            stats[2] = float(bal);
+            stats[3] = float(z);
+            stats[4] = float(bal + double(z_weight) * z);
+        }
     }
 }
-
 }  // namespace
 
-// Blocks of the telemetry kernel: enough tokens per block to keep its partial
-// rows few (the final sum is one block), enough blocks to fill the GPU.
+// Blocks of the telemetry kernel: a warp per token up to the most partial rows
+// the final sum reads (32 x kStatsMaxRowsPerLane); larger batches loop.
 int route_stats_blocks(int T) {
     const int need = (T + kStatsWarps - 1) / kStatsWarps;
-    return need < 2 * num_sms() ? need : 2 * num_sms();
+    const int cap = 32 * kStatsMaxRowsPerLane;
+    return need < cap ? need : cap;
 }
 
 cudaError_t launch_route_stats(const float* logits, int T, int E, int k, int32_t* topk_idx, float* topk_w,
@@ -237,7 +305,7 @@ cudaError_t launch_route_stats(const float* logits, int T, int E, int k, int32_t
     }
     {
         ProfScope prof_(MOE_K_ROUTE_STATS, stream);
-        const cudaError_t le = launch_pdl(pdl, route_stats_final, dim3(1), dim3(kMaxE), 0, stream, part_p, part_c,
+        const cudaError_t le = launch_pdl(pdl, route_stats_final, dim3(1), dim3(1024), 0, stream, part_p, part_c,
                                           part_s, nb, T, E, z_weight, stats, expert_stats);
         if (le != cudaSuccess) return le;
     }

@@ -25,13 +25,14 @@ MOE_DEV float route_unkey(uint32_t k) {
 
 // The whole warp routes token `row` (E logits): lane j < k writes selection j
 // to idx_out[j] / w_out[j]. Warp-uniform; every lane must call it. Returns
-// the first choice (warp-uniform).
+// the first choice (warp-uniform); *kth_key (if given) gets the k-th selected
+// value's key.
 // Each round: every lane takes its best untaken logit (larger value, then
 // lower expert index); one warp max-reduction of the keys gives the winning
 // value and one min-reduction over the lanes holding it gives the lowest
 // expert index among equal values.
 MOE_DEV int route_one_token(const float* __restrict__ row, int E, int k, int32_t* __restrict__ idx_out,
-                            float* __restrict__ w_out) {
+                            float* __restrict__ w_out, uint32_t* kth_key = nullptr) {
     const int lane = threadIdx.x & 31;
     uint32_t key[kRouteMaxPerLane];
 #pragma unroll
@@ -60,6 +61,7 @@ MOE_DEV int route_one_token(const float* __restrict__ row, int E, int k, int32_t
         const int wi = int(__reduce_min_sync(0xFFFFFFFFu, (bi != 0x7FFFFFFF && bk == kmax) ? uint32_t(bi) : 0xFFFFFFFFu));
         if ((wi & 31) == lane) taken |= 1u << (wi >> 5);
         const float wv = route_unkey(kmax);
+        if (kth_key && j == k - 1) *kth_key = kmax;
         if (j == 0) {
             top = wv;
             first = wi;
