@@ -38,6 +38,7 @@ import statistics
 import sys
 import threading
 import time
+import types
 
 ROOT = os.path.dirname(os.path.abspath(__file__))
 TILE_ARG = {"auto": 0, "one": 1, "pair": 2}  # moe_params.tile_ctas (MOE_TILE_*)
@@ -66,6 +67,8 @@ def parse():
     ap.add_argument("--tokens", type=int, default=0, help="override T of the workload (profiling small cases)")
     ap.add_argument("--profile-calls", type=int, default=0,
                     help="only run this many moe_forward calls and exit (for ncu: no timing, no other kernels)")
+    ap.add_argument("--profile-op", default="forward", choices=["forward", "backward", "route_stats"],
+                    help="entry point the --profile-calls calls make")
     ap.add_argument("--tile", default="auto", choices=["auto", "one", "pair"],
                     help="SMs per tcgen05 tile (moe_params.tile_ctas); auto = the library's choice")
     ap.add_argument("--sweep-threshold", action="store_true",
@@ -447,12 +450,9 @@ def measure_workload(cfg, args, b, torch, flush, pk, pk_src, steps):
     return entry
 
 
-def measure_extra_rows(cfg, b, torch, flush, pk, pk_src, steps):
-    """The layer's backward (moe_expert_ffn_backward) and the router with its telemetry
-    (moe_route_stats) on the workload, each timed with CUDA events around a graph replay of one
-    call, L2 flushed between calls. Backward work: 16 d f FLOPs per routed row (recomputed gate/up
-    4df, dh 2df, dx 4df, weight gradients 6df) plus the shared expert's rows; telemetry: the
-    logits read once (4 E bytes per token)."""
+def extra_ops(cfg, b, torch):
+    """Closures running one moe_expert_ffn_backward and one moe_route_stats call on the workload
+    (routing and permutation done once beforehand), and the workspaces whose error words they set."""
     from synth.device import upload
     d = upload(cfg, "cuda")
     p = b.params_for(cfg, down_dtype=b.DOWN_F16)
@@ -484,6 +484,18 @@ def measure_extra_rows(cfg, b, torch, flush, pk, pk_src, steps):
     def rstats():
         b.route_stats(p, d["logits"], idx2, w2, stats, wss)
 
+    return types.SimpleNamespace(bwd=bwd, rstats=rstats, ws=(wsb, wss), offsets=offsets, tensors=(d, W, G, g))
+
+
+def measure_extra_rows(cfg, b, torch, flush, pk, pk_src, steps):
+    """The layer's backward (moe_expert_ffn_backward) and the router with its telemetry
+    (moe_route_stats) on the workload, each timed with CUDA events around a graph replay of one
+    call, L2 flushed between calls. Backward work: 16 d f FLOPs per routed row (recomputed gate/up
+    4df, dh 2df, dx 4df, weight gradients 6df) plus the shared expert's rows; telemetry: the
+    logits read once (4 E bytes per token)."""
+    T, E, dm, f = cfg.T, cfg.E, cfg.d, cfg.f
+    ops = extra_ops(cfg, b, torch)
+    bwd, rstats, (wsb, wss) = ops.bwd, ops.rstats, ops.ws
     out = {}
     for name, fn in (("backward", bwd), ("route_stats", rstats)):
         for _ in range(3):
@@ -505,7 +517,7 @@ def measure_extra_rows(cfg, b, torch, flush, pk, pk_src, steps):
         del graph
     if b.get_error(wsb) or b.get_error(wss):
         raise RuntimeError("device error word set (backward / route_stats)")
-    P = int(offsets[E].item())
+    P = int(ops.offsets[E].item())
     fl = 16.0 * P * dm * f + (16.0 * T * dm * f if cfg.has_shared else 0.0)
     tfl = fl / (out["backward"] / 1e3) / 1e12
     gbs = T * E * 4 / (out["route_stats"] / 1e3) / 1e9
@@ -517,7 +529,7 @@ def measure_extra_rows(cfg, b, torch, flush, pk, pk_src, steps):
                            "work": "the logits read once (4 E bytes per token); latency-bound at this size"},
            "workload": workload_name(cfg), "steps": steps,
            "step_launch": "CUDA graph replay of one call, L2 flushed between calls"}
-    del d, W, G, g, wsb, wss
+    del ops, bwd, rstats, wsb, wss
     torch.cuda.empty_cache()
     return res
 
@@ -775,18 +787,28 @@ def prepared_layer(cfg, b, torch, stream_max_rows=-1, tile_ctas=0):
 
 
 def profile_calls(args, cfg):
-    """Only `n` moe_forward calls (the first one warms up): a short, fixed launch sequence for ncu."""
+    """Only `n` calls of one entry point (the first one warms up): a short, fixed launch sequence
+    for ncu. --profile-op: moe_forward (default), moe_expert_ffn_backward or moe_route_stats."""
     import torch
     from mixture_experts_routed_04_b200 import binding as b
-    d, p, W, out = prepared_layer(cfg, b, torch, tile_ctas=TILE_ARG[args.tile])
-    ws = b.workspace(p, b.WS_FORWARD)
+    if args.profile_op == "forward":
+        d, p, W, out = prepared_layer(cfg, b, torch, tile_ctas=TILE_ARG[args.tile])
+        ws = b.workspace(p, b.WS_FORWARD)
+        wss = (ws,)
+
+        def fn():
+            b.forward(p, d["x"], d["logits"], W, out, ws)
+    else:
+        ops = extra_ops(cfg, b, torch)
+        wss = ops.ws
+        fn = ops.bwd if args.profile_op == "backward" else ops.rstats
     torch.cuda.synchronize()
     for _ in range(args.profile_calls):
-        b.forward(p, d["x"], d["logits"], W, out, ws)
+        fn()
     torch.cuda.synchronize()
-    if b.get_error(ws):
+    if any(b.get_error(w) for w in wss):
         raise RuntimeError("device error word set")
-    print(json.dumps({"profile_calls": args.profile_calls, "workload": workload_name(cfg)}))
+    print(json.dumps({"profile_calls": args.profile_calls, "op": args.profile_op, "workload": workload_name(cfg)}))
     return 0
 
 

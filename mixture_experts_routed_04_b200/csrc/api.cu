@@ -565,14 +565,14 @@ int moe_launch_count(const moe_params* p, int which, int* n) {
     int ffn = 1;  // schedule
     if (!gather_fused(D)) ffn += 1;                 // gather
     if (tiles_needed(D)) ffn += 2;                  // two tcgen05 GEMMs
-    if (streams(D)) ffn += 2 + (D.ks > 1 ? 1 : 0);
+    if (streams(D)) ffn += 2 + (D.ks > 1 && !stream_fold(D) ? 1 : 0);  // + the K-split reduce
     switch (which) {
         case MOE_WS_ROUTE: *n = 1; break;
         case MOE_WS_PERMUTE: *n = 3; break;
         case MOE_WS_EXPERT_FFN: *n = ffn; break;
         case MOE_WS_COMBINE: *n = 1; break;
         case MOE_WS_ROUTE_STATS: *n = 2; break;
-        // schedule, gather, transpose, 6 GEMMs, zeroing, combine, reduce (+ dlogits: not counted)
+        // schedule, gather, 6 GEMMs, zeroing, combine, routing-weight reduce, route backward
         case MOE_WS_BACKWARD: *n = 12; break;
         // moe_forward: the front kernel(s) write the schedule, so the expert FFN's own
         // schedule launch is not made

@@ -65,6 +65,8 @@ cudaError_t launch_route(const float* logits, int T, int E, int k, int32_t* topk
                          cudaStream_t s);
 
 int route_stats_blocks(int T);
+// The streaming down kernel sums the K-split gate/up partials itself (stream.cu).
+bool stream_fold(const Dims& D);
 cudaError_t launch_route_stats(const float* logits, int T, int E, int k, int32_t* topk_idx, float* topk_w,
                                float z_weight, float* stats, float* kept_tok, int32_t* want_tok,
                                float* expert_stats, float* part_p, int32_t* part_c, float* part_s,

@@ -44,15 +44,26 @@ constexpr int RC = 8;                // rows per chunk (mma N)
 // stage, 16 columns of each per consumer warp); down items are 256 columns of
 // W_down (four boxes a stage, 64 columns per warp), so each weight row is read
 // as 512 contiguous bytes — 64-column down items left HBM half idle.
-template <int MODE>
+// FOLD (down only): the gate/up ran K-split and its fp32 partials are summed
+// here, into an [RC rows, f] fp16 buffer of h per chunk (no reduce kernel, no
+// rows tile in the stages).
+template <int MODE, bool FOLD = false>
 struct SCfg {
     static constexpr int NMAT = MODE == 0 ? 2 : 4;                // weight boxes per stage
     static constexpr int NSU = MODE == 0 ? NS : 4 * NS;           // output columns per item
-    static constexpr int STAGE = NMAT * TILE + XT;                // 17 KB / 33 KB, 1 KB aligned
+    static constexpr int STAGE = NMAT * TILE + (FOLD ? 0 : XT);   // 17 KB / 33 KB (32 KB folded), 1 KB aligned
     static constexpr int STAGES = MODE == 0 ? 7 : 6;
     static constexpr int RING = STAGES * STAGE;                   // 119 KB / 198 KB
-    static constexpr int SMEM = 1024 + RING + 512;
+    static constexpr int SMEM = 1024 + RING + 512;                // + barriers, abort flag
 };
+// Row stride of the folded h buffer: 16 bytes past the row, so that the 8 rows a
+// consumer warp reads at one k fall in distinct banks.
+__host__ __device__ inline int fold_row_bytes(int f) { return 2 * f + 16; }
+constexpr int kFoldMaxSmem = 232448;  // dynamic shared memory a block may opt into
+inline bool fold_fits(int f) { return SCfg<1, true>::SMEM + RC * fold_row_bytes(f) <= kFoldMaxSmem; }
+constexpr int kFoldMaxSlices = 4;  // K-split counts the fold takes (its loads are held in registers)
+constexpr int kFoldQ = 3;          // column pairs a consumer thread sums at a time
+static_assert((2 * 7 + 3) * 8 <= 512, "stage barriers, abort flag and the fold's barriers fit the reserved bytes");
 
 struct StreamParams {
     int mode;            // 0: gate/up, 1: down
@@ -65,6 +76,8 @@ struct StreamParams {
     const int32_t* sorted_pair;
     const float* topk_w;
     uint16_t* out;        // mode 0: h [rows, f]; mode 1: y_rows [rows, d]
+    const float* hpart;   // mode 1 folded: the gate/up partials [ksg, 2, rows, f]
+    int ksg;              // mode 1 folded: their K-split count
     float* part;          // mode 0 with ks > 1: [ks, 2, rows, f] fp32
     int64_t rows;
     float limit;
@@ -127,18 +140,23 @@ MOE_DEV void mma_f16_16816(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2,
 MOE_DEV uint16_t to_f16(float v) { return uint16_t(pack_f16x2(v, 0.f) & 0xFFFFu); }
 
 // MODE 0: two weight tiles (gate, up) per stage; MODE 1: one (down). Plus the rows tile.
-template <int MODE>
+template <int MODE, bool FOLD = false>
 __global__ void __launch_bounds__(THREADS, 1)
     stream_kernel(const __grid_constant__ CUtensorMap tmW0, const __grid_constant__ CUtensorMap tmW1,
                   const __grid_constant__ CUtensorMap tmS0, const __grid_constant__ CUtensorMap tmS1,
                   const __grid_constant__ CUtensorMap tmX, const StreamParams p) {
-    using SC = SCfg<MODE>;
+    using SC = SCfg<MODE, FOLD>;
+    static_assert(!FOLD || MODE == 1, "the fold is the down kernel's");
     constexpr int NMAT = SC::NMAT, NSU = SC::NSU, STAGE = SC::STAGE, STAGES = SC::STAGES;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint64_t* full = reinterpret_cast<uint64_t*>(smem + SC::RING);
     uint64_t* empty = full + STAGES;
     volatile int* abort_flag = reinterpret_cast<volatile int*>(empty + STAGES);
+    // FOLD: h of the current chunk written (every consumer thread) / read (every consumer thread)
+    uint64_t* hready = empty + STAGES + 1;
+    uint64_t* hfree = hready + 1;
+    uint8_t* hbuf = smem + SC::RING + 512;  // FOLD: [RC][fold_row_bytes(f)] fp16
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     if (threadIdx.x == 0) {
@@ -146,6 +164,8 @@ __global__ void __launch_bounds__(THREADS, 1)
             mbar_init(full + s, 1);
             mbar_init(empty + s, CONSUMERS);
         }
+        mbar_init(hready, 32 * CONSUMERS);
+        mbar_init(hfree, 32 * CONSUMERS);
         *abort_flag = 0;
         fence_mbar_init();
     }
@@ -186,7 +206,8 @@ __global__ void __launch_bounds__(THREADS, 1)
                             // the four boxes in one copy (boxes past N are filled with zeros)
                             tma_load_3d(dst, sh ? &tmS0 : &tmW0, full + stage, 0, wrow + kb * BKS, U.n0 / NS);
                         }
-                        tma_load_2d(dst + NMAT * TILE, &tmX, full + stage, U.k0 + kb * BKS, U.row0 + c * RC);
+                        if (!FOLD)
+                            tma_load_2d(dst + NMAT * TILE, &tmX, full + stage, U.k0 + kb * BKS, U.row0 + c * RC);
                         issued |= 1u << stage;
                         issued_par = (issued_par & ~(1u << stage)) | (phase << stage);
                     }
@@ -213,8 +234,9 @@ __global__ void __launch_bounds__(THREADS, 1)
     const int cw = warp - 1;
     const int gid = lane >> 2, tig = lane & 3;
     int stage = 0;
-    uint32_t phase = 0;
+    uint32_t phase = 0, hph = 0;
     bool ok = true, range_bad = false;
+    const int HS = FOLD ? fold_row_bytes(p.K) : 0;
     for (int u = blockIdx.x; ok && u < total; u += gridDim.x) {
         const SUnit U = decode(u, p, NSU);
         const int nchunks = (U.nrows + RC - 1) / RC;
@@ -225,6 +247,57 @@ __global__ void __launch_bounds__(THREADS, 1)
             for (int g = 0; g < NG; ++g)
 #pragma unroll
                 for (int i = 0; i < 4; ++i) acc0[g][i] = 0.f;
+            if (FOLD) {
+                // h of the chunk's rows from the gate/up partials, slices summed in order (as
+                // stream_reduce_kernel does), once every consumer is done with the previous
+                // chunk's; the weight stages keep streaming in meanwhile
+                int okl = mbar_wait_bounded(hfree, hph ^ 1u, abort_flag, p.err, p.wait_ns);
+                if (!__all_sync(0xFFFFFFFFu, okl)) {
+                    ok = false;
+                    break;
+                }
+                const int64_t slice = int64_t(p.rows) * p.K;  // g of slice s at 2s, u at 2s + 1
+                for (int r = 0; r < rc; ++r) {
+                    const float* hrow = p.hpart + (int64_t(U.row0) + c * RC + r) * p.K;
+                    // kFoldQ column pairs a thread at a time, every slice's loads issued together
+                    for (int q0 = cw * 32 + lane; q0 < p.K / 2; q0 += kFoldQ * 32 * CONSUMERS) {
+                        float2 gs[kFoldQ][kFoldMaxSlices], us[kFoldQ][kFoldMaxSlices];
+#pragma unroll
+                        for (int j = 0; j < kFoldQ; ++j) {
+                            const int q = q0 + j * 32 * CONSUMERS;
+#pragma unroll
+                            for (int sl = 0; sl < kFoldMaxSlices; ++sl)
+                                if (sl < p.ksg && q < p.K / 2) {
+                                    gs[j][sl] = __ldg(reinterpret_cast<const float2*>(hrow + 2 * sl * slice) + q);
+                                    us[j][sl] = __ldg(reinterpret_cast<const float2*>(hrow + (2 * sl + 1) * slice) + q);
+                                }
+                        }
+#pragma unroll
+                        for (int j = 0; j < kFoldQ; ++j) {
+                            const int q = q0 + j * 32 * CONSUMERS;
+                            if (q >= p.K / 2) break;
+                            float g0 = 0.f, g1 = 0.f, u0 = 0.f, u1 = 0.f;
+#pragma unroll
+                            for (int sl = 0; sl < kFoldMaxSlices; ++sl)
+                                if (sl < p.ksg) {
+                                    g0 += gs[j][sl].x;
+                                    g1 += gs[j][sl].y;
+                                    u0 += us[j][sl].x;
+                                    u1 += us[j][sl].y;
+                                }
+                            const float h0 = swiglu(g0, u0, p.limit), h1 = swiglu(g1, u1, p.limit);
+                            range_bad |= !(f16_range_ok(h0) && f16_range_ok(h1));
+                            *reinterpret_cast<uint32_t*>(hbuf + r * HS + 4 * q) = pack_f16x2(h0, h1);
+                        }
+                    }
+                }
+                mbar_arrive(hready);
+                okl = mbar_wait_bounded(hready, hph, abort_flag, p.err, p.wait_ns);
+                if (!__all_sync(0xFFFFFFFFu, okl)) {
+                    ok = false;
+                    break;
+                }
+            }
             for (int kb = 0; kb < KB; ++kb) {
                 int okl = 1;
                 if (lane == 0) okl = mbar_wait_bounded(full + stage, phase, abort_flag, p.err, p.wait_ns);
@@ -242,11 +315,19 @@ __global__ void __launch_bounds__(THREADS, 1)
                     // swizzle); grp = cw (gate/up) or the 16-column group g (down)
                     const int kr = k16 * 16 + ((lane >> 4) << 3) + (lane & 7);
                     // rows tile: row gid, k = k16*16 + 2*tig (+8): chunk (k/8) ^ gid
+                    // (FOLD: row gid of the chunk's h buffer, k from the item's start)
                     const int kx = k16 * 16 + 2 * tig;
-                    const uint32_t b0 =
-                        *reinterpret_cast<const uint32_t*>(xt + gid * 128 + (((kx >> 3) ^ gid) << 4) + (kx & 7) * 2);
-                    const uint32_t b1 = *reinterpret_cast<const uint32_t*>(
-                        xt + gid * 128 + ((((kx + 8) >> 3) ^ gid) << 4) + ((kx + 8) & 7) * 2);
+                    uint32_t b0, b1;
+                    if (FOLD) {
+                        const uint8_t* hb = hbuf + gid * HS + (kb * BKS + kx) * 2;
+                        b0 = *reinterpret_cast<const uint32_t*>(hb);
+                        b1 = *reinterpret_cast<const uint32_t*>(hb + 16);
+                    } else {
+                        b0 = *reinterpret_cast<const uint32_t*>(xt + gid * 128 + (((kx >> 3) ^ gid) << 4) +
+                                                                 (kx & 7) * 2);
+                        b1 = *reinterpret_cast<const uint32_t*>(xt + gid * 128 + ((((kx + 8) >> 3) ^ gid) << 4) +
+                                                                 ((kx + 8) & 7) * 2);
+                    }
 #pragma unroll
                     for (int g = 0; g < NG; ++g) {
                         const int grp = MODE == 0 ? cw : g;
@@ -277,6 +358,10 @@ __global__ void __launch_bounds__(THREADS, 1)
                 }
             }
             if (!ok) break;
+            if (FOLD) {
+                mbar_arrive(hfree);  // this thread's reads of the chunk's h are done
+                hph ^= 1u;
+            }
             // acc[g][i]: column n = (cw*16 | cw*64 + 16g) + gid + 8*(i/2), row r = 2*tig + (i%2)
 #pragma unroll
             for (int g = 0; g < NG; ++g) {
@@ -387,23 +472,24 @@ static bool map_chunks(CUtensorMap* m, const void* base, int64_t nrows, int ncol
                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-template <int MODE>
+// smem: the dynamic shared memory of this launch (SCfg::SMEM, plus the h buffer when folded).
+template <int MODE, bool FOLD = false>
 static cudaError_t launch_one(const CUtensorMap& W0, const CUtensorMap& W1, const CUtensorMap& S0,
                               const CUtensorMap& S1, const CUtensorMap& X, const StreamParams& p, int grid,
-                              bool pdl, cudaStream_t s) {
+                              int smem, bool pdl, cudaStream_t s) {
     static int configured_dev = -1;
     int dev = 0;
     cudaGetDevice(&dev);
     if (configured_dev != dev) {
-        cudaError_t e =
-            cudaFuncSetAttribute(stream_kernel<MODE>, cudaFuncAttributeMaxDynamicSharedMemorySize, SCfg<MODE>::SMEM);
+        cudaError_t e = cudaFuncSetAttribute(stream_kernel<MODE, FOLD>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             FOLD ? kFoldMaxSmem : SCfg<MODE, FOLD>::SMEM);
         if (e != cudaSuccess) return e;
         configured_dev = dev;
     }
     {
         ProfScope prof_(MODE == 0 ? MOE_K_STREAM_GATEUP : MOE_K_STREAM_DOWN, s);
-        const cudaError_t le = launch_pdl(pdl, stream_kernel<MODE>, dim3(grid), dim3(THREADS), SCfg<MODE>::SMEM, s,
-                                          W0, W1, S0, S1, X, p);
+        const cudaError_t le = launch_pdl(pdl, stream_kernel<MODE, FOLD>, dim3(grid), dim3(THREADS), smem, s, W0,
+                                          W1, S0, S1, X, p);
         if (le != cudaSuccess) return le;
     }
     return cudaGetLastError();
@@ -454,9 +540,10 @@ cudaError_t launch_stream_ffn(const Dims& D, const uint16_t* xg, uint16_t* h, fl
     p.out = h;
     p.part = part;
     const bool pdl = use_pdl(D.T);
-    cudaError_t e = launch_one<0>(mG, mU, mSG, mSU, mX, p, grid, pdl, s);
+    cudaError_t e = launch_one<0>(mG, mU, mSG, mSU, mX, p, grid, SCfg<0>::SMEM, pdl, s);
     if (e != cudaSuccess) return e;
-    if (D.ks > 1) {
+    const bool fold = stream_fold(D);
+    if (D.ks > 1 && !fold) {
         ProfScope prof_(MOE_K_STREAM_REDUCE, s);
         const cudaError_t le = launch_pdl(pdl, stream_reduce_kernel, dim3(grid * 2), dim3(256), 0, s, part, D.ks,
                                           D.rows, D.f, offsets, stream_list, n_stream, D.limit, h, err);
@@ -470,7 +557,17 @@ cudaError_t launch_stream_ffn(const Dims& D, const uint16_t* xg, uint16_t* h, fl
     p.kslice = D.f;
     p.out = y_rows;
     p.part = nullptr;
-    return launch_one<1>(mD, mD, mSD, mSD, mH, p, grid, pdl, s);
+    if (fold) {
+        p.hpart = part;
+        p.ksg = D.ks;
+        return launch_one<1, true>(mD, mD, mSD, mSD, mH, p, grid, SCfg<1, true>::SMEM + RC * fold_row_bytes(D.f),
+                                   pdl, s);
+    }
+    return launch_one<1>(mD, mD, mSD, mSD, mH, p, grid, SCfg<1>::SMEM, pdl, s);
 }
+
+// The streaming down kernel sums the K-split gate/up partials itself (no reduce
+// kernel) when its h buffer of RC rows fits beside its stages.
+bool stream_fold(const Dims& D) { return D.ks > 1 && D.ks <= st::kFoldMaxSlices && st::fold_fits(D.f); }
 
 }  // namespace moe

@@ -160,7 +160,7 @@ def test_variant_table_is_finite_and_monotone(lib):
 def test_default_variant_follows_the_table(lib):
     """Single-token decode (8 routed experts + the shared one: 108 gate/up tiles on 148 SMs, or
     whatever the host's default count) streams; eight tokens (up to 65 experts) take the tiles.
-    The streaming kernels add launches to moe_forward's count."""
+    The streaming kernels replace the two tile GEMMs in moe_forward's count."""
     def launches(T):
         p = b.params(T=T, d_model=4096, d_ff=1536, E=256, k=8, has_shared=1, d_ff_shared=1536)
         return b.launch_count(p, b.WS_FORWARD), b.launch_count(b.params(
@@ -168,6 +168,18 @@ def test_default_variant_follows_the_table(lib):
             variant=b.VARIANT_TENSOR), b.WS_FORWARD)
     auto1, tiles1 = launches(1)
     auto8, tiles8 = launches(8)
-    # T=1: the two tile GEMMs give way to the streaming gate/up, its K-split reduce and down
-    assert auto1 == tiles1 - 2 + 3
+    # T=1: the two tile GEMMs give way to the streaming gate/up and down (the down kernel
+    # sums the gate/up's K-split partials itself)
+    assert auto1 == tiles1 - 2 + 2
     assert auto8 == tiles8  # T=8: every expert on the tiles
+
+
+def test_streaming_reduce_folds_into_down_when_h_fits(lib):
+    """The K-split gate/up partials are summed by the streaming down kernel while its h buffer
+    (8 rows of d_ff fp16) fits beside its stages, else by a separate reduce launch."""
+    def launches(f):
+        p = b.params(T=3, d_model=256, d_ff=f, E=4, k=2, variant=b.VARIANT_STREAM)
+        return b.launch_count(p, b.WS_EXPERT_FFN)
+    # schedule + gather + streaming gate/up + down, (+ reduce)
+    assert launches(2112) == 4
+    assert launches(2176) == 5

@@ -43,6 +43,9 @@ SMALL = {
     # 32 touched experts x 5 gate/up tiles >= 148 SMs: the automatic choice keeps every expert
     # on the tiles, so a forced streaming variant must still launch the streaming kernels
     "many_experts": synth.LayerConfig("many_experts", T=8, d=128, f=640, E=32, k=4),
+    # d_ff too wide for the streaming down kernel's h buffer: the K-split gate/up partials go
+    # through the separate reduce kernel (at d_ff <= 2136 the down kernel sums them itself)
+    "wide_ff": synth.LayerConfig("wide_ff", T=3, d=256, f=2176, E=4, k=2),
 }
 Q4_SMALL = {
     "q4_tiny": synth.CONFIGS["tiny"].replace(name="q4_tiny", weight_format="q4g32"),
