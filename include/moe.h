@@ -417,7 +417,7 @@ MOE_API int moe_wait_selftest(void* err_ws, uint64_t limit_ns, moe_stream_t stre
 #define MOE_K_FRONT         13  /* S1-S3 + schedule fused, moe_forward with T <= 64 */
 #define MOE_K_ROUTE_STATS   14  /* router telemetry: the final sum over blocks (moe_route_stats) */
 #define MOE_K_BWD_GEMM      15  /* backward tcgen05 GEMMs (moe_expert_ffn_backward) */
-#define MOE_K_BWD_SMALL     16  /* backward schedule, gathers, transpose, reductions */
+#define MOE_K_BWD_SMALL     16  /* backward schedule, gathers, zeroing, reductions */
 #define MOE_K_COUNT         17
 
 /*

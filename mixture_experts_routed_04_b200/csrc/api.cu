@@ -238,8 +238,9 @@ cudaError_t launch_expert_ffn(const Dims& D, const WsLayout& L, const FfnArgs& a
     // which spreads small batches over more threads, is faster.
     const bool token_order = a.pair_row && !x_in_l2(D);
     const bool fused = gather_fused(D);
-    if (!fused && (e = token_order ? launch_scatter_rows(D, a.x, a.pair_row, a.offsets, xg, a.err, s)
-                                   : launch_gather(D, a.x, a.sorted_token, a.offsets, xg, a.err, s)) != cudaSuccess)
+    if (!fused && !a.gathered &&
+        (e = token_order ? launch_scatter_rows(D, a.x, a.pair_row, a.offsets, xg, a.err, s)
+                         : launch_gather(D, a.x, a.sorted_token, a.offsets, xg, a.err, s)) != cudaSuccess)
         return e;
     if (tiles_needed(D)) {
         if ((e = launch_tensor_ffn(D, xg, h, tile_base, a.offsets, a.sorted_pair, a.topk_w, a.w, a.y_rows,
@@ -426,7 +427,8 @@ static int forward_impl(const Dims& D, const WsLayout& L, const uint16_t* x, con
         e = launch_front_small(D, logits, topk_idx, topk_w, counts, kept, offsets, sorted_token, sorted_pair,
                                pair_row, reinterpret_cast<int32_t*>(ws + L.tile_base),
                                reinterpret_cast<int32_t*>(ws + L.stream_list),
-                               reinterpret_cast<int32_t*>(ws + L.n_stream), err, stream);
+                               reinterpret_cast<int32_t*>(ws + L.n_stream), x,
+                               front_gathers(D) ? reinterpret_cast<uint16_t*>(ws + L.xg) : nullptr, err, stream);
         if (e != cudaSuccess) return MOE_ERR_CUDA;
     } else {
         e = launch_route(logits, D.T, D.E, D.k, topk_idx, topk_w, stream);
@@ -440,7 +442,8 @@ static int forward_impl(const Dims& D, const WsLayout& L, const uint16_t* x, con
                            sorted_pair, pair_row, err, stream, &sa);
         if (e != cudaSuccess) return MOE_ERR_CUDA;
     }
-    FfnArgs a{x, offsets, sorted_token, sorted_pair, topk_w, w, y_rows, ws, err, g_wait_ns.load(), true, pair_row};
+    FfnArgs a{x, offsets, sorted_token, sorted_pair, topk_w, w, y_rows, ws, err, g_wait_ns.load(), true, pair_row,
+              front && front_gathers(D)};
     if ((e = launch_expert_ffn(D, L, a, stream)) != cudaSuccess) return MOE_ERR_CUDA;
     if ((e = launch_combine(D, y_rows, pair_row, offsets, out, stream)) != cudaSuccess) return MOE_ERR_CUDA;
     if (counts_out &&
@@ -575,8 +578,11 @@ int moe_launch_count(const moe_params* p, int which, int* n) {
         // schedule, gather, 6 GEMMs, zeroing, combine, routing-weight reduce, route backward
         case MOE_WS_BACKWARD: *n = 12; break;
         // moe_forward: the front kernel(s) write the schedule, so the expert FFN's own
-        // schedule launch is not made
-        default: *n = D.T <= kFrontMaxTokens ? 1 + (ffn - 1) + 1 : 1 + 3 + (ffn - 1) + 1; break;
+        // schedule launch is not made (nor, for the smallest batches, the gather)
+        default:
+            *n = D.T <= kFrontMaxTokens ? 1 + (ffn - 1) - (front_gathers(D) && !gather_fused(D) ? 1 : 0) + 1
+                                        : 1 + 3 + (ffn - 1) + 1;
+            break;
     }
     return MOE_OK;
 }

@@ -88,10 +88,15 @@ cudaError_t launch_permute(const Dims& D, const int32_t* topk_idx, int32_t* bloc
 // Batches of at most this many tokens run routing, permutation and the tile
 // schedule as one fused single-block kernel (front.cu).
 constexpr int kFrontMaxTokens = 64;
+// The fused front kernel also gathers the rows (bf16) when at most this many bytes of
+// rows can result: one block copies them faster than a separate launch starts.
+constexpr int64_t kFrontGatherBytes = 96 << 10;
+bool front_gathers(const Dims& D);
+// x / xg: the rows to gather and their destination when front_gathers(D), else null.
 cudaError_t launch_front_small(const Dims& D, const float* logits, int32_t* topk_idx, float* topk_w,
                                int32_t* counts, int32_t* kept, int32_t* offsets, int32_t* sorted_token,
                                int32_t* sorted_pair, int32_t* pair_row, int32_t* tile_base, int32_t* stream_list,
-                               int32_t* n_stream, uint32_t* err, cudaStream_t s);
+                               int32_t* n_stream, const uint16_t* x, uint16_t* xg, uint32_t* err, cudaStream_t s);
 
 // The bf16 gate/up GEMM gathers its rows from x itself (no gathered copy).
 constexpr bool kFusedGather = false;
@@ -109,6 +114,7 @@ struct FfnArgs {
     uint64_t wait_ns;
     bool scheduled;            // the front kernels already wrote the tile schedule
     const int32_t* pair_row;   // moe_forward: row of each pair (-1 dropped), for the token-order row copy
+    bool gathered = false;     // the front kernel already wrote the gathered rows
 };
 cudaError_t launch_expert_ffn(const Dims& D, const WsLayout& L, const FfnArgs& a, cudaStream_t s);
 

@@ -52,10 +52,10 @@ __global__ void __launch_bounds__(256) route_topk_softmax_kernel(const float* __
 // (fp64, lanes over block rows, then a fixed shuffle tree). Fixed orders
 // throughout: the results are deterministic.
 
-constexpr int kStatsWarps = 8;
+constexpr int kStatsWarps = 16;
 // Partial rows a lane of the final sum reads: the telemetry kernel runs at most
 // 32 x this many blocks (route_stats_blocks).
-constexpr int kStatsMaxRowsPerLane = 16;
+constexpr int kStatsMaxRowsPerLane = 8;
 constexpr float kWantMass = 0.9f;
 
 template <bool PER_TOKEN>

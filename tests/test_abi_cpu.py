@@ -172,6 +172,10 @@ def test_default_variant_follows_the_table(lib):
     # sums the gate/up's K-split partials itself)
     assert auto1 == tiles1 - 2 + 2
     assert auto8 == tiles8  # T=8: every expert on the tiles
+    # the single-token layer: the front kernel (routing, permutation, schedule and, for at most
+    # 96 KB of rows, the gather), the two streaming kernels, the combine
+    assert auto1 == 4
+    assert auto8 == 5  # front, gather, two tile GEMMs, combine
 
 
 def test_streaming_reduce_folds_into_down_when_h_fits(lib):
