@@ -59,7 +59,7 @@ constexpr int kStatsMaxRowsPerLane = 8;
 constexpr float kWantMass = 0.9f;
 
 template <bool PER_TOKEN>
-__global__ void __launch_bounds__(kStatsWarps * 32)
+__global__ void __launch_bounds__(kStatsWarps * 32, 2)
     route_stats_kernel(const float* __restrict__ logits, int T, int E, int k, int32_t* __restrict__ topk_idx,
                        float* __restrict__ topk_w, float* __restrict__ kept_tok, int32_t* __restrict__ want_tok,
                        float* __restrict__ part_p, int32_t* __restrict__ part_c, float* __restrict__ part_s) {
