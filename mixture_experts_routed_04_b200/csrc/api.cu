@@ -24,7 +24,7 @@ cudaError_t launch_convert_bf16_f16(const uint16_t* src, uint16_t* dst, int64_t 
 cudaError_t launch_stream_ffn(const Dims& D, const uint16_t* xg, uint16_t* h, float* part, const int32_t* offsets,
                               const int32_t* stream_list, const int32_t* n_stream, const int32_t* sorted_pair,
                               const float* topk_w, const moe_weights* w, uint16_t* y_rows, uint32_t* err,
-                              uint64_t wait_ns, cudaStream_t s);
+                              uint64_t wait_ns, const CombineArgs* comb, cudaStream_t s);
 
 static std::atomic<uint64_t> g_wait_ns{1000000000ull};
 
@@ -180,6 +180,7 @@ WsLayout ws_layout(const Dims& D, int which) {
         L.sorted_pair = take(size_t(D.rows) * 4);
         L.pair_row = take(size_t(D.pairs) * 4);
         L.y_rows = take(size_t(D.rows) * D.d * 2);
+        L.comb = take(size_t(combine_blocks(D)) * 4);
     }
     if (which == MOE_WS_FORWARD_HOST) {
         L.x_dev = take(size_t(D.T) * D.d * 2);
@@ -204,6 +205,13 @@ static bool tiles_needed(const Dims& D) {
     if (D.variant == MOE_VARIANT_STREAM) return false;
     if (D.variant == MOE_VARIANT_AUTO && D.stream_max_rows > 0 && D.T <= D.stream_max_rows) return false;
     return true;
+}
+
+// moe_forward of at most kCombFuseMaxTokens tokens whose experts all stream: the
+// streaming down kernel does the combine (its last arrival on each 256-column
+// block sums that block), so the combine launch is not made.
+static bool combine_fused(const Dims& D) {
+    return D.T <= kFrontMaxTokens && D.T <= kCombFuseMaxTokens && streams(D) && !tiles_needed(D);
 }
 
 // x small enough to stay in L2 while the rows are gathered.
@@ -250,7 +258,7 @@ cudaError_t launch_expert_ffn(const Dims& D, const WsLayout& L, const FfnArgs& a
     }
     if (streams(D)) {
         if ((e = launch_stream_ffn(D, xg, h, part, a.offsets, stream_list, n_stream, a.sorted_pair, a.topk_w, a.w,
-                                   a.y_rows, a.err, a.wait_ns, s)) != cudaSuccess)
+                                   a.y_rows, a.err, a.wait_ns, a.comb, s)) != cudaSuccess)
             return e;
     }
     return cudaSuccess;
@@ -422,13 +430,16 @@ static int forward_impl(const Dims& D, const WsLayout& L, const uint16_t* x, con
     uint16_t* y_rows = reinterpret_cast<uint16_t*>(ws + L.y_rows);
     uint32_t* err = reinterpret_cast<uint32_t*>(ws);
     const bool front = D.T <= kFrontMaxTokens;
+    const bool fuse_comb = combine_fused(D);
+    const CombineArgs comb{reinterpret_cast<int32_t*>(ws + L.comb), pair_row, out};
     cudaError_t e;
     if (front) {  // routing, permutation and schedule in one small kernel
         e = launch_front_small(D, logits, topk_idx, topk_w, counts, kept, offsets, sorted_token, sorted_pair,
                                pair_row, reinterpret_cast<int32_t*>(ws + L.tile_base),
                                reinterpret_cast<int32_t*>(ws + L.stream_list),
                                reinterpret_cast<int32_t*>(ws + L.n_stream), x,
-                               front_gathers(D) ? reinterpret_cast<uint16_t*>(ws + L.xg) : nullptr, err, stream);
+                               front_gathers(D) ? reinterpret_cast<uint16_t*>(ws + L.xg) : nullptr,
+                               fuse_comb ? comb.count : nullptr, err, stream);
         if (e != cudaSuccess) return MOE_ERR_CUDA;
     } else {
         e = launch_route(logits, D.T, D.E, D.k, topk_idx, topk_w, stream);
@@ -443,9 +454,10 @@ static int forward_impl(const Dims& D, const WsLayout& L, const uint16_t* x, con
         if (e != cudaSuccess) return MOE_ERR_CUDA;
     }
     FfnArgs a{x, offsets, sorted_token, sorted_pair, topk_w, w, y_rows, ws, err, g_wait_ns.load(), true, pair_row,
-              front && front_gathers(D)};
+              front && front_gathers(D), fuse_comb ? &comb : nullptr};
     if ((e = launch_expert_ffn(D, L, a, stream)) != cudaSuccess) return MOE_ERR_CUDA;
-    if ((e = launch_combine(D, y_rows, pair_row, offsets, out, stream)) != cudaSuccess) return MOE_ERR_CUDA;
+    if (!fuse_comb && (e = launch_combine(D, y_rows, pair_row, offsets, out, stream)) != cudaSuccess)
+        return MOE_ERR_CUDA;
     if (counts_out &&
         cudaMemcpyAsync(counts_out, counts, size_t(D.Etot) * 4, cudaMemcpyDeviceToDevice, stream) != cudaSuccess)
         return MOE_ERR_CUDA;
@@ -578,10 +590,12 @@ int moe_launch_count(const moe_params* p, int which, int* n) {
         // schedule, gather, 6 GEMMs, zeroing, combine, routing-weight reduce, route backward
         case MOE_WS_BACKWARD: *n = 12; break;
         // moe_forward: the front kernel(s) write the schedule, so the expert FFN's own
-        // schedule launch is not made (nor, for the smallest batches, the gather)
+        // schedule launch is not made (nor, for the smallest batches, the gather, and
+        // when the streaming down kernel combines, the combine)
         default:
-            *n = D.T <= kFrontMaxTokens ? 1 + (ffn - 1) - (front_gathers(D) && !gather_fused(D) ? 1 : 0) + 1
-                                        : 1 + 3 + (ffn - 1) + 1;
+            *n = D.T <= kFrontMaxTokens
+                     ? 1 + (ffn - 1) - (front_gathers(D) && !gather_fused(D) ? 1 : 0) + (combine_fused(D) ? 0 : 1)
+                     : 1 + 3 + (ffn - 1) + 1;
             break;
     }
     return MOE_OK;

@@ -29,7 +29,8 @@ __global__ void __launch_bounds__(kFrontThreads)
                        int32_t* __restrict__ sorted_token, int32_t* __restrict__ sorted_pair,
                        int32_t* __restrict__ pair_row, int32_t* __restrict__ tile_base,
                        int32_t* __restrict__ stream_list, int32_t* __restrict__ n_stream,
-                       const uint16_t* __restrict__ x, int d, uint16_t* __restrict__ xg, uint32_t* err) {
+                       const uint16_t* __restrict__ x, int d, uint16_t* __restrict__ xg,
+                       int32_t* __restrict__ comb_count, int ncomb, uint32_t* err) {
     __shared__ int hist[kFrontWarps][kMaxE];  // per-warp counts per expert, then warp bases
     __shared__ int s_off[kMaxE + 2];
     __shared__ int s_tok[kFrontThreads + kFrontMaxTokens];  // token of each row (S4, when gathering)
@@ -39,6 +40,8 @@ __global__ void __launch_bounds__(kFrontThreads)
     griddep_launch();
     const int tid = threadIdx.x, lane = tid & 31, w = tid >> 5;
     const int pairs = T * k;
+    if (comb_count)
+        for (int i = tid; i < ncomb; i += kFrontThreads) comb_count[i] = 0;
 
     // S1: warp w routes tokens w, w + 16, ...
     for (int t = w; t < T; t += kFrontWarps)
@@ -158,7 +161,8 @@ bool front_gathers(const Dims& D) {
 cudaError_t launch_front_small(const Dims& D, const float* logits, int32_t* topk_idx, float* topk_w,
                                int32_t* counts, int32_t* kept, int32_t* offsets, int32_t* sorted_token,
                                int32_t* sorted_pair, int32_t* pair_row, int32_t* tile_base, int32_t* stream_list,
-                               int32_t* n_stream, const uint16_t* x, uint16_t* xg, uint32_t* err, cudaStream_t s) {
+                               int32_t* n_stream, const uint16_t* x, uint16_t* xg, int32_t* comb_count,
+                               uint32_t* err, cudaStream_t s) {
     if (D.T > kFrontMaxTokens || int64_t(D.T) * D.k > kFrontThreads || D.E > kMaxE) return cudaErrorInvalidValue;
     if (xg && (!x || !front_gathers(D))) return cudaErrorInvalidValue;
     {
@@ -166,7 +170,8 @@ cudaError_t launch_front_small(const Dims& D, const float* logits, int32_t* topk
         const cudaError_t le = launch_pdl(use_pdl(D.T), front_small_kernel, dim3(1), dim3(kFrontThreads), 0, s,
                                           logits, D.T, D.E, D.k, D.cap, D.has_shared, D.variant, D.stream_max_rows,
                                           topk_idx, topk_w, counts, kept, offsets, sorted_token, sorted_pair,
-                                          pair_row, tile_base, stream_list, n_stream, x, D.d, xg, err);
+                                          pair_row, tile_base, stream_list, n_stream, x, D.d, xg, comb_count,
+                                          combine_blocks(D), err);
         if (le != cudaSuccess) return le;
     }
     return cudaGetLastError();

@@ -47,6 +47,7 @@ struct WsLayout {
     size_t tile_base, stream_list, n_stream;       // expert_ffn schedule
     size_t xg, h, part;                            // expert_ffn: gathered x, h, split-K partials
     size_t topk_idx, topk_w, counts, kept, offsets, sorted_token, sorted_pair, pair_row, y_rows;  // forward
+    size_t comb;                                   // forward: fused-combine arrival counters
     size_t x_dev, logits_dev, out_dev;             // forward_host
     size_t stats_p, stats_c, stats_s;              // route_stats: per-block partial sums
     // backward (padded row space, see backward.cu)
@@ -93,13 +94,26 @@ constexpr int kFrontMaxTokens = 64;
 constexpr int64_t kFrontGatherBytes = 96 << 10;
 bool front_gathers(const Dims& D);
 // x / xg: the rows to gather and their destination when front_gathers(D), else null.
+// comb_count: the fused combine's counters to zero (combine_blocks(D) of them), or null.
 cudaError_t launch_front_small(const Dims& D, const float* logits, int32_t* topk_idx, float* topk_w,
                                int32_t* counts, int32_t* kept, int32_t* offsets, int32_t* sorted_token,
                                int32_t* sorted_pair, int32_t* pair_row, int32_t* tile_base, int32_t* stream_list,
-                               int32_t* n_stream, const uint16_t* x, uint16_t* xg, uint32_t* err, cudaStream_t s);
+                               int32_t* n_stream, const uint16_t* x, uint16_t* xg, int32_t* comb_count,
+                               uint32_t* err, cudaStream_t s);
 
 // The bf16 gate/up GEMM gathers its rows from x itself (no gathered copy).
 constexpr bool kFusedGather = false;
+
+// moe_forward of a few tokens whose experts all stream: the streaming down kernel
+// also does the combine (stream.cu); count: [combine_blocks(D)] int32, zeroed by the
+// front kernel.
+struct CombineArgs {
+    int32_t* count;
+    const int32_t* pair_row;
+    void* out;
+};
+constexpr int kCombFuseMaxTokens = 2;
+inline int combine_blocks(const Dims& D) { return (D.d + 255) / 256; }
 
 struct FfnArgs {
     const uint16_t* x;
@@ -115,6 +129,7 @@ struct FfnArgs {
     bool scheduled;            // the front kernels already wrote the tile schedule
     const int32_t* pair_row;   // moe_forward: row of each pair (-1 dropped), for the token-order row copy
     bool gathered = false;     // the front kernel already wrote the gathered rows
+    const CombineArgs* comb = nullptr;  // the streaming down kernel also combines
 };
 cudaError_t launch_expert_ffn(const Dims& D, const WsLayout& L, const FfnArgs& a, cudaStream_t s);
 

@@ -84,7 +84,59 @@ struct StreamParams {
     int down_f16;         // mode 1: W_down already fp16 (no conversion)
     uint32_t* err;
     uint64_t wait_ns;
+    // mode 1, every expert streaming (moe_forward of a few tokens): the combine fused in.
+    // comb_count: [ceil(N/256)] arrivals per column block, zeroed by the front kernel.
+    int32_t* comb_count;
+    const int32_t* pair_row;  // [T*k] row of each pair, -1 dropped
+    void* comb_out;           // [T, N] fp32, or bf16 with comb_bf16
+    int comb_bf16, T, k, has_shared;
 };
+
+// The combine of output columns [n0, n0 + 256) for every token, by one warp (8
+// columns a lane): the kept pairs' y rows in the fixed order j = 0..k-1, then the
+// shared expert's row, summed in fp32 as combine_kernel does. y rows are read
+// from L2 (other SMs wrote them).
+MOE_DEV void combine_columns(const StreamParams& p, int n0, int lane) {
+    const int c = n0 + lane * 8;
+    if (c >= p.N) return;
+    const int shared_base = p.has_shared ? __ldg(p.offsets + p.E) : 0;
+    for (int t = 0; t < p.T; ++t) {
+        float acc[8];
+#pragma unroll
+        for (int q = 0; q < 8; ++q) acc[q] = 0.f;
+        auto add = [&](const uint4& v) {
+            acc[0] += f16_lo(v.x); acc[1] += f16_hi(v.x);
+            acc[2] += f16_lo(v.y); acc[3] += f16_hi(v.y);
+            acc[4] += f16_lo(v.z); acc[5] += f16_hi(v.z);
+            acc[6] += f16_lo(v.w); acc[7] += f16_hi(v.w);
+        };
+        int rr[kMaxK];
+        uint4 yv[kMaxK];
+#pragma unroll
+        for (int j = 0; j < kMaxK; ++j) rr[j] = j < p.k ? __ldg(p.pair_row + int64_t(t) * p.k + j) : -1;
+#pragma unroll
+        for (int j = 0; j < kMaxK; ++j)
+            if (rr[j] >= 0) yv[j] = __ldcg(reinterpret_cast<const uint4*>(p.out + int64_t(rr[j]) * p.N + c));
+        uint4 ys = make_uint4(0, 0, 0, 0);
+        if (p.has_shared) ys = __ldcg(reinterpret_cast<const uint4*>(p.out + int64_t(shared_base + t) * p.N + c));
+#pragma unroll
+        for (int j = 0; j < kMaxK; ++j)
+            if (rr[j] >= 0) add(yv[j]);
+        if (p.has_shared) add(ys);
+        if (p.comb_bf16) {
+            uint4 o;
+            o.x = pack_bf16x2(acc[0], acc[1]);
+            o.y = pack_bf16x2(acc[2], acc[3]);
+            o.z = pack_bf16x2(acc[4], acc[5]);
+            o.w = pack_bf16x2(acc[6], acc[7]);
+            *reinterpret_cast<uint4*>(static_cast<uint16_t*>(p.comb_out) + int64_t(t) * p.N + c) = o;
+        } else {
+            float4* dst = reinterpret_cast<float4*>(static_cast<float*>(p.comb_out) + int64_t(t) * p.N + c);
+            dst[0] = make_float4(acc[0], acc[1], acc[2], acc[3]);
+            dst[1] = make_float4(acc[4], acc[5], acc[6], acc[7]);
+        }
+    }
+}
 
 struct SUnit {
     int e, n0, k0, ks, row0, nrows;
@@ -390,6 +442,22 @@ __global__ void __launch_bounds__(THREADS, 1)
                 }
             }
         }
+        // Fused combine: once its y stores for the item are made, each consumer warp
+        // arrives on the item's column block (fence, then a counter); the warp making the
+        // block's last arrival (every streaming expert's item, every consumer warp) sums
+        // the block's columns of every token. Which warp that is does not change the sum.
+        if (MODE == 1 && p.comb_count && ok) {
+            __threadfence();
+            __syncwarp();
+            int last = 0;
+            if (lane == 0)
+                last = atomicAdd(p.comb_count + U.n0 / NSU, 1) == __ldg(p.n_stream) * CONSUMERS - 1 ? 1 : 0;
+            last = __shfl_sync(0xFFFFFFFFu, last, 0);
+            if (last) {
+                __threadfence();
+                combine_columns(p, U.n0, lane);
+            }
+        }
     }
     if (range_bad) set_error(p.err, MOE_DEVERR_RANGE);
 }
@@ -502,7 +570,7 @@ static cudaError_t launch_one(const CUtensorMap& W0, const CUtensorMap& W1, cons
 cudaError_t launch_stream_ffn(const Dims& D, const uint16_t* xg, uint16_t* h, float* part, const int32_t* offsets,
                               const int32_t* stream_list, const int32_t* n_stream, const int32_t* sorted_pair,
                               const float* topk_w, const moe_weights* w, uint16_t* y_rows, uint32_t* err,
-                              uint64_t wait_ns, cudaStream_t s) {
+                              uint64_t wait_ns, const CombineArgs* comb, cudaStream_t s) {
     using namespace st;
     CUtensorMap mG, mU, mD, mSG, mSU, mSD, mX, mH;
     if (!map_2d(&mG, w->w_gate, int64_t(D.E) * D.d, D.f, BKS) || !map_2d(&mU, w->w_up, int64_t(D.E) * D.d, D.f, BKS) ||
@@ -557,6 +625,15 @@ cudaError_t launch_stream_ffn(const Dims& D, const uint16_t* xg, uint16_t* h, fl
     p.kslice = D.f;
     p.out = y_rows;
     p.part = nullptr;
+    if (comb) {
+        p.comb_count = comb->count;
+        p.pair_row = comb->pair_row;
+        p.comb_out = comb->out;
+        p.comb_bf16 = D.out_bf16;
+        p.T = D.T;
+        p.k = D.k;
+        p.has_shared = D.has_shared;
+    }
     if (fold) {
         p.hpart = part;
         p.ksg = D.ks;

@@ -46,6 +46,9 @@ SMALL = {
     # d_ff too wide for the streaming down kernel's h buffer: the K-split gate/up partials go
     # through the separate reduce kernel (at d_ff <= 2136 the down kernel sums them itself)
     "wide_ff": synth.LayerConfig("wide_ff", T=3, d=256, f=2176, E=4, k=2),
+    # two tokens with a shared expert: every expert streams and the streaming down kernel
+    # also does the combine (a 256-column block of d=320 is partial)
+    "two_tokens": synth.LayerConfig("two_tokens", T=2, d=320, f=256, E=8, k=3, has_shared=True, f_shared=256),
 }
 Q4_SMALL = {
     "q4_tiny": synth.CONFIGS["tiny"].replace(name="q4_tiny", weight_format="q4g32"),
