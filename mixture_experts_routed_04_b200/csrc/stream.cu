@@ -69,7 +69,7 @@ struct StreamParams {
     int mode;            // 0: gate/up, 1: down
     int K, N;            // full reduction length and output width of the matrix
     int kslice, ks;      // K per item and number of K slices
-    int E;
+    int E, etot;          // routed experts; with the shared one
     const int32_t* offsets;
     const int32_t* stream_list;
     const int32_t* n_stream;
@@ -149,6 +149,10 @@ MOE_DEV SUnit decode(int u, const StreamParams& p, int nsu) {
     const int rem = u - i * per;
     SUnit U;
     U.e = __ldg(p.stream_list + i);
+    if (U.e < 0 || U.e >= p.etot) {  // never for a list the schedule wrote
+        set_error(p.err, MOE_DEVERR_BOUNDS);
+        U.e = 0;
+    }
     U.n0 = (rem / p.ks) * nsu;
     U.ks = rem % p.ks;
     U.k0 = U.ks * p.kslice;
@@ -223,6 +227,9 @@ __global__ void __launch_bounds__(THREADS, 1)
     }
     __syncthreads();
     // the prologue above touched no global memory; wait for the predecessor here
+    // (letting the folded down kernel's producer stream its first weight stages before
+    // the wait, as the weights and the item list allow, measured 76.3 -> 76.0 us on
+    // single-token decode: its blocks only become resident as the gate/up blocks exit)
     griddep_wait();
     griddep_launch();
 
@@ -589,6 +596,7 @@ cudaError_t launch_stream_ffn(const Dims& D, const uint16_t* xg, uint16_t* h, fl
     const int grid = num_sms();
     StreamParams p{};
     p.E = D.E;
+    p.etot = D.Etot;
     p.offsets = offsets;
     p.stream_list = stream_list;
     p.n_stream = n_stream;
