@@ -518,12 +518,27 @@ def measure_extra_rows(cfg, b, torch, flush, pk, pk_src, steps):
     if b.get_error(wsb) or b.get_error(wss):
         raise RuntimeError("device error word set (backward / route_stats)")
     P = int(ops.offsets[E].item())
+    counts = ops.offsets[1:E + 1] - ops.offsets[:E]
+    touched = int((counts > 0).sum().item())
     fl = 16.0 * P * dm * f + (16.0 * T * dm * f if cfg.has_shared else 0.0)
     tfl = fl / (out["backward"] / 1e3) / 1e12
+    # algorithmic bytes: each touched expert's weights read once (bf16 gate/up, fp16 W_down), every
+    # expert's three fp32 weight gradients written (zeros for the untouched), x and dout read, dx
+    # written, the routing weights and logits' gradients (small)
+    nsh = 1 if cfg.has_shared else 0
+    bb = ((touched + nsh) * 3.0 * dm * f * 2 + (E + nsh) * 3.0 * dm * f * 4 + T * dm * (2 + 4 + 4)
+          + T * cfg.k * 4 * 3 + T * E * 4 * 2)
+    bgbs = bb / (out["backward"] / 1e3) / 1e9
+    t_tensor = fl / (pk["bf16_tflops"] * 1e12)
+    t_hbm = bb / (pk["hbm_gbs"] * 1e9)
     gbs = T * E * 4 / (out["route_stats"] / 1e3) / 1e9
     res = {"backward": {"call": "moe_expert_ffn_backward", "ms": out["backward"], "flops": fl, "tflops": tfl,
                         "frac_of_peak": tfl / pk["bf16_tflops"], "peak_source": f"{pk_src} bf16_tflops (burst)",
-                        "work": "16 d f FLOPs per routed row: recomputed gate/up, dh, dx, three weight gradients"},
+                        "bytes": bb, "gbs": bgbs, "hbm_frac_of_peak": bgbs / pk["hbm_gbs"],
+                        "bound": "hbm" if t_hbm > t_tensor else "tensor",
+                        "frac_of_bound": max(t_hbm, t_tensor) / (out["backward"] / 1e3),
+                        "work": "16 d f FLOPs per routed row: recomputed gate/up, dh, dx, three weight gradients; "
+                                "bytes: touched weights read once, all fp32 weight gradients written, x, dout, dx"},
            "route_stats": {"call": "moe_route_stats", "ms": out["route_stats"], "gbs": gbs,
                            "frac_of_peak": gbs / pk["hbm_gbs"], "peak_source": f"{pk_src} hbm_gbs",
                            "work": "the logits read once (4 E bytes per token); latency-bound at this size"},

@@ -61,7 +61,9 @@ constexpr int kStageBytes = A_BYTES + B_BYTES;
 constexpr int kEpiWarps = 8;
 constexpr int kThreads = 32 * (2 + kEpiWarps);
 constexpr int kStageOut = kEpiWarps * 32 * 32 * 4;  // WG: one 32 x 32 fp32 block per epilogue warp
-constexpr int kSmem = 1024 + kStages * kStageBytes + 512 + kStageOut;
+// + barriers and unit ring (512), padding so the staging blocks are 1024-byte aligned
+// (the 128-byte-swizzled boxes of the TMA stores)
+constexpr int kSmem = 1024 + kStages * kStageBytes + 1024 + kStageOut;
 constexpr int kUnitReaders = 1 + kEpiWarps;
 constexpr int kPad = 64;  // rows of an expert are padded to a multiple of this
 
@@ -183,14 +185,16 @@ MOE_DEV RowInfo row_info(const Unit& U, int q, int lane, const Params& p) {
 
 template <int MODE>
 MOE_DEV void epilogue(uint32_t tb, const Unit& U, int q, int half, int lane, const Params& p, bool& range_bad,
-                      float* stage_out, RowInfo ri) {
+                      float* stage_out, RowInfo ri, const CUtensorMap* st_dw, const CUtensorMap* st_sdw) {
     const int rit = q * 32 + lane;
     const bool valid = rit < U.rows;
     if (MODE == WG) {
-        // each 32 x 32 fp32 block: lane = row into shared memory (16-byte groups XOR-swizzled by
-        // row, conflict-free), then 4 rows x 128 bytes per warp store instruction
-        float* base = U.e < p.E ? p.dw + int64_t(U.e) * p.M * p.N : p.sdw;
-        const int g8 = lane & 7;
+        // each 32 x 32 fp32 block: lane = row into shared memory in the 128-byte swizzle
+        // (16-byte group g of row r at g ^ (r % 8): conflict-free), then one TMA store of the
+        // box by lane 0 (rows past M are not written); the block's buffer is reused once the
+        // previous store has read it
+        const CUtensorMap* st = U.e < p.E ? st_dw : st_sdw;
+        const int z = U.e < p.E ? U.e : 0;
 #pragma unroll 1
         for (int c = half; c < BN / 32; c += 2) {
             uint32_t v[32];
@@ -198,20 +202,18 @@ MOE_DEV void epilogue(uint32_t tb, const Unit& U, int q, int half, int lane, con
             tmem_ld_wait();
             const int col = U.n * BN + c * 32;
             if (col >= p.N) break;
+            if (lane == 0) bulk_wait_read0();
+            __syncwarp();
 #pragma unroll
             for (int g = 0; g < 8; ++g)
                 *reinterpret_cast<uint4*>(stage_out + lane * 32 + ((g ^ (lane & 7)) << 2)) =
                     make_uint4(v[4 * g], v[4 * g + 1], v[4 * g + 2], v[4 * g + 3]);
+            fence_proxy_async_smem();
             __syncwarp();
-#pragma unroll
-            for (int i = 0; i < 8; ++i) {
-                const int r = 4 * i + (lane >> 3);  // row of this warp's 32
-                const int mrow = U.row0 + q * 32 + r;
-                const uint4 val = *reinterpret_cast<const uint4*>(stage_out + r * 32 + ((g8 ^ (r & 7)) << 2));
-                if (q * 32 + r < U.rows)
-                    *reinterpret_cast<uint4*>(base + int64_t(mrow) * p.N + col + 4 * g8) = val;
+            if (lane == 0) {
+                tma_store_3d(st, stage_out, col, U.row0 + q * 32, z);
+                bulk_commit();
             }
-            __syncwarp();
         }
         return;
     }
@@ -362,7 +364,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     volatile int* unit_ring = reinterpret_cast<volatile int*>(uempty + UR);
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(const_cast<int*>(unit_ring) + UR);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
-    float* stage_out = reinterpret_cast<float*>(smem + kStages * kStageBytes + 512);
+    float* stage_out = reinterpret_cast<float*>(smem + kStages * kStageBytes + 1024);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     if (threadIdx.x == 0) {
@@ -551,7 +553,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (!okl) break;
             tc_fence_after();
             const uint32_t tb = tmem_base + (uint32_t(q * 32) << 16) + uint32_t(acc * BN);
-            epilogue<MODE>(tb, U, q, half, lane, p, range_bad, stage_out + (warp - 2) * 32 * 32, ri);
+            epilogue<MODE>(tb, U, q, half, lane, p, range_bad, stage_out + (warp - 2) * 32 * 32, ri, &tmS0, &tmS1);
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(tempty + acc);
@@ -561,6 +563,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
         }
         if (range_bad) set_error(p.err, MOE_DEVERR_RANGE);
+        if (MODE == WG && lane == 0) bulk_wait0();  // this warp's gradient stores are complete
     }
     __syncthreads();
     if (warp == 1) {
@@ -766,6 +769,7 @@ cudaError_t launch_mode(const CUtensorMap& A, const CUtensorMap& B0, const CUten
 
 namespace tc {
 bool map_weights_kmajor(CUtensorMap* m, const void* base, int nexp, int N, int K, bool f16 = false);
+bool map_f32_tiles(CUtensorMap* m, const void* base, int nexp, int M, int N);
 bool map_act_mn(CUtensorMap* m, const void* base, int64_t rows, int N, int64_t row_stride, int chunks);
 }  // namespace tc
 
@@ -866,23 +870,28 @@ cudaError_t launch_backward(const Dims& D, const BwdArgs& a, cudaStream_t s) {
     p.n_tiles = (d + BN - 1) / BN;
     p.unit_counter = counters + 2;
     if ((e = launch_mode<DX>(mDgu, mGk, mUk, sGk, sUk, p, s)) != cudaSuccess) return e;
-    // WG: dW_down = (w h)^T dout_rows [f, d]; dW_gate = xg^T dg, dW_up = xg^T du [d, f]
-    p.M = f;
-    p.N = d;
-    p.dw = a.g->dw_down;
-    p.sdw = a.g->dshared_down;
-    p.unit_counter = counters + 3;
-    if ((e = launch_mode<WG>(mHwN, mDogN, mDogN, mDogN, mDogN, p, s)) != cudaSuccess) return e;
-    p.M = d;
-    p.N = f;
-    p.dw = a.g->dw_gate;
-    p.sdw = a.g->dshared_gate;
-    p.unit_counter = counters + 4;
-    if ((e = launch_mode<WG>(mXgN, mDgN, mDgN, mDgN, mDgN, p, s)) != cudaSuccess) return e;
-    p.dw = a.g->dw_up;
-    p.sdw = a.g->dshared_up;
-    p.unit_counter = counters + 5;
-    if ((e = launch_mode<WG>(mXgN, mDuN, mDuN, mDuN, mDuN, p, s)) != cudaSuccess) return e;
+    // WG: dW_down = (w h)^T dout_rows [f, d]; dW_gate = xg^T dg, dW_up = xg^T du [d, f]. The
+    // S0 / S1 maps of a WG launch are its TMA store maps: the routed experts' gradient and
+    // the shared expert's (the routed map again without one).
+    auto wg = [&](const CUtensorMap& A, const CUtensorMap& B, float* dw, float* sdw, int M, int N,
+                  int32_t* counter) -> cudaError_t {
+        CUtensorMap stD, stS;
+        if (!tc::map_f32_tiles(&stD, dw, D.E, M, N) || (sdw && !tc::map_f32_tiles(&stS, sdw, 1, M, N)))
+            return cudaErrorInvalidValue;
+        if (!sdw) stS = stD;
+        p.M = M;
+        p.N = N;
+        p.dw = dw;
+        p.sdw = sdw;
+        p.unit_counter = counter;
+        return launch_mode<WG>(A, B, B, stD, stS, p, s);
+    };
+    float* sd = D.has_shared ? a.g->dshared_down : nullptr;
+    float* sg = D.has_shared ? a.g->dshared_gate : nullptr;
+    float* su = D.has_shared ? a.g->dshared_up : nullptr;
+    if ((e = wg(mHwN, mDogN, a.g->dw_down, sd, f, d, counters + 3)) != cudaSuccess) return e;
+    if ((e = wg(mXgN, mDgN, a.g->dw_gate, sg, d, f, counters + 4)) != cudaSuccess) return e;
+    if ((e = wg(mXgN, mDuN, a.g->dw_up, su, d, f, counters + 5)) != cudaSuccess) return e;
     {
         ProfScope prof_(MOE_K_BWD_SMALL, s);
         const int64_t per = int64_t(d) * f;

@@ -157,6 +157,20 @@ MOE_DEV void tma_load_2d(void* dst, const CUtensorMap* m, uint64_t* bar, int32_t
         "l"(reinterpret_cast<uint64_t>(m)), "r"(smem_u32(bar)), "r"(x), "r"(y)
         : "memory");
 }
+// Bulk tensor store of a shared-memory box to global (the box at coordinates
+// x, y, z of map m; elements past the tensor's bounds are not written), in this
+// thread's bulk group. Make the box's generic-proxy writes visible first
+// (fence_proxy_async_smem by every writer), and wait for the group's read
+// (bulk_wait_read0) before writing the box again.
+MOE_DEV void tma_store_3d(const CUtensorMap* m, const void* src, int32_t x, int32_t y, int32_t z) {
+    asm volatile("cp.async.bulk.tensor.3d.global.shared::cta.bulk_group [%0, {%2, %3, %4}], [%1];" ::"l"(
+                     reinterpret_cast<uint64_t>(m)),
+                 "r"(smem_u32(src)), "r"(x), "r"(y), "r"(z)
+                 : "memory");
+}
+MOE_DEV void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+MOE_DEV void bulk_wait_read0() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
+MOE_DEV void bulk_wait0() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
 MOE_DEV void tma_load_4d(void* dst, const CUtensorMap* m, uint64_t* bar, int32_t x, int32_t y, int32_t z,
                          int32_t w) {
     asm volatile(

@@ -586,6 +586,13 @@ bool map_act_mn(CUtensorMap* m, const void* base, int64_t rows, int N, int64_t r
     const uint32_t box[4] = {64, 64, uint32_t(chunks), 1};
     return make_map(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, base, 4, dims, str, box, CU_TENSOR_MAP_SWIZZLE_128B);
 }
+// fp32 [nexp, M, N] written by 32 x 32 boxes (128-byte swizzle) from shared memory.
+bool map_f32_tiles(CUtensorMap* m, const void* base, int nexp, int M, int N) {
+    const uint64_t dims[3] = {uint64_t(N), uint64_t(M), uint64_t(nexp)};
+    const uint64_t str[2] = {uint64_t(N) * 4, uint64_t(M) * uint64_t(N) * 4};
+    const uint32_t box[3] = {32, 32, 1};
+    return make_map(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, base, 3, dims, str, box, CU_TENSOR_MAP_SWIZZLE_128B);
+}
 // Q4G32 nibbles: [nexp, N, K/2] bytes; box 32 bytes (64 k) x rows x 1, no swizzle.
 bool map_q4_packed(CUtensorMap* m, const void* base, int nexp, int K, int N, int rows) {
     const uint64_t dims[3] = {uint64_t(K / 2), uint64_t(N), uint64_t(nexp)};
