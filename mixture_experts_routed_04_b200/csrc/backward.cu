@@ -259,23 +259,37 @@ MOE_DEV void epilogue(uint32_t tb, const Unit& U, int q, int half, int lane, con
         }
     } else if (MODE == DH) {
         float dot = 0.f;
+        // the chunk's g and u (fp16), 8 vector loads issued together, one chunk ahead: the
+        // next chunk's are in flight while this one is computed and stored
+        auto load_gu = [&](int c, uint4 (&gq)[4], uint4 (&uq)[4]) {
+            const int col = U.n * BN + c * 32;
+            if (valid && col < f && c < BN / 32) {
+                const uint4* gsrc = reinterpret_cast<const uint4*>(p.gu + prow * f2 + col);
+                const uint4* usrc = reinterpret_cast<const uint4*>(p.gu + prow * f2 + f + col);
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    gq[i] = gsrc[i];
+                    uq[i] = usrc[i];
+                }
+            }
+        };
+        uint4 gn[4], un[4];
+        load_gu(half, gn, un);
 #pragma unroll 1
         for (int c = half; c < BN / 32; c += 2) {
+            uint4 gq4[4], uq4[4];
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                gq4[i] = gn[i];
+                uq4[i] = un[i];
+            }
+            load_gu(c + 2, gn, un);
             uint32_t v[32];
             tmem_ld_32x32b_x32(tb + c * 32, v);
             tmem_ld_wait();
             const int col = U.n * BN + c * 32;
             if (valid && col < f) {
-                // the chunk's g and u (fp16) in 8 vector loads issued together; h = silu(gc) uc
-                // is recomputed from them for the routing-weight dot
-                uint4 gq4[4], uq4[4];
-                const uint4* gsrc = reinterpret_cast<const uint4*>(p.gu + prow * f2 + col);
-                const uint4* usrc = reinterpret_cast<const uint4*>(p.gu + prow * f2 + f + col);
-#pragma unroll
-                for (int i = 0; i < 4; ++i) {
-                    gq4[i] = gsrc[i];
-                    uq4[i] = usrc[i];
-                }
+                // h = silu(gc) uc is recomputed from g and u for the routing-weight dot
                 const uint32_t* gw = reinterpret_cast<const uint32_t*>(gq4);
                 const uint32_t* uw = reinterpret_cast<const uint32_t*>(uq4);
                 uint32_t pg[16], pu[16], qg[16], qu[16];
