@@ -185,7 +185,7 @@ MOE_DEV RowInfo row_info(const Unit& U, int q, int lane, const Params& p) {
 
 template <int MODE>
 MOE_DEV void epilogue(uint32_t tb, const Unit& U, int q, int half, int lane, const Params& p, bool& range_bad,
-                      float* stage_out, RowInfo ri, const CUtensorMap* st_dw, const CUtensorMap* st_sdw) {
+                      float* stage_out, RowInfo ri, const CUtensorMap* st0, const CUtensorMap* st1) {
     const int rit = q * 32 + lane;
     const bool valid = rit < U.rows;
     if (MODE == WG) {
@@ -193,7 +193,7 @@ MOE_DEV void epilogue(uint32_t tb, const Unit& U, int q, int half, int lane, con
         // (16-byte group g of row r at g ^ (r % 8): conflict-free), then one TMA store of the
         // box by lane 0 (rows past M are not written); the block's buffer is reused once the
         // previous store has read it
-        const CUtensorMap* st = U.e < p.E ? st_dw : st_sdw;
+        const CUtensorMap* st = U.e < p.E ? st0 : st1;  // the routed experts' gradient, the shared one's
         const int z = U.e < p.E ? U.e : 0;
 #pragma unroll 1
         for (int c = half; c < BN / 32; c += 2) {
@@ -259,6 +259,9 @@ MOE_DEV void epilogue(uint32_t tb, const Unit& U, int q, int half, int lane, con
         }
     } else if (MODE == DH) {
         float dot = 0.f;
+        // padded row counts are multiples of 64, so a warp's 32 rows are all valid or none
+        const bool wvalid = q * 32 < U.rows && (U.rows & 31) == 0;
+        if (q * 32 < U.rows && (U.rows & 31) != 0 && lane == 0) set_error(p.err, MOE_DEVERR_BOUNDS);
         // the chunk's g and u (fp16), 8 vector loads issued together, one chunk ahead: the
         // next chunk's are in flight while this one is computed and stored
         auto load_gu = [&](int c, uint4 (&gq)[4], uint4 (&uq)[4]) {
@@ -288,7 +291,7 @@ MOE_DEV void epilogue(uint32_t tb, const Unit& U, int q, int half, int lane, con
             tmem_ld_32x32b_x32(tb + c * 32, v);
             tmem_ld_wait();
             const int col = U.n * BN + c * 32;
-            if (valid && col < f) {
+            if (wvalid && col < f) {  // warp-uniform: the TMA stores below need every lane
                 // h = silu(gc) uc is recomputed from g and u for the routing-weight dot
                 const uint32_t* gw = reinterpret_cast<const uint32_t*>(gq4);
                 const uint32_t* uw = reinterpret_cast<const uint32_t*>(uq4);
@@ -319,16 +322,27 @@ MOE_DEV void epilogue(uint32_t tb, const Unit& U, int q, int half, int lane, con
                     qg[i / 2] = pack_f16x2(dgv[0], dgv[1]);
                     qu[i / 2] = pack_f16x2(duv[0], duv[1]);
                 }
-                uint4* gd = reinterpret_cast<uint4*>(p.dgu + prow * f2 + col);
-                uint4* ud = reinterpret_cast<uint4*>(p.dgu + prow * f2 + f + col);
-                uint4* gq = reinterpret_cast<uint4*>(p.dgu16 + prow * f2 + col);
-                uint4* uq = reinterpret_cast<uint4*>(p.dgu16 + prow * f2 + f + col);
+                // the chunk's four 32 x 32 boxes (dg, du in bf16, then in fp16) leave by TMA
+                // stores through this warp's two 2 KB buffers (64-byte swizzle: 16-byte group j
+                // of row r at j ^ ((r / 2) % 4)); a buffer is rewritten once the store that
+                // used it two boxes ago has read it. The warp's 32 rows are all inside the
+                // expert's padded rows (their count is a multiple of 64), so whole boxes go out.
 #pragma unroll
-                for (int i = 0; i < 4; ++i) {
-                    gd[i] = make_uint4(pg[4 * i], pg[4 * i + 1], pg[4 * i + 2], pg[4 * i + 3]);
-                    ud[i] = make_uint4(pu[4 * i], pu[4 * i + 1], pu[4 * i + 2], pu[4 * i + 3]);
-                    gq[i] = make_uint4(qg[4 * i], qg[4 * i + 1], qg[4 * i + 2], qg[4 * i + 3]);
-                    uq[i] = make_uint4(qu[4 * i], qu[4 * i + 1], qu[4 * i + 2], qu[4 * i + 3]);
+                for (int bx = 0; bx < 4; ++bx) {
+                    const uint32_t* src = bx == 0 ? pg : bx == 1 ? pu : bx == 2 ? qg : qu;
+                    uint8_t* buf = reinterpret_cast<uint8_t*>(stage_out) + (bx & 1) * 2048;
+                    if (lane == 0) bulk_wait_read1();
+                    __syncwarp();
+#pragma unroll
+                    for (int j = 0; j < 4; ++j)
+                        *reinterpret_cast<uint4*>(buf + lane * 64 + ((j ^ ((lane >> 1) & 3)) << 4)) =
+                            make_uint4(src[4 * j], src[4 * j + 1], src[4 * j + 2], src[4 * j + 3]);
+                    fence_proxy_async_smem();
+                    __syncwarp();
+                    if (lane == 0) {
+                        tma_store_2d(bx < 2 ? st0 : st1, buf, (bx & 1 ? f : 0) + col, int(prow));  // bf16, fp16
+                        bulk_commit();
+                    }
                 }
             }
         }
@@ -358,9 +372,11 @@ MOE_DEV void epilogue(uint32_t tb, const Unit& U, int q, int half, int lane, con
 
 // Operand maps per mode:
 //   GU: A = xg; B0/B1 = W_gate/W_up (N-major, 2 chunks a copy), S0/S1 the shared expert's.
-//   DH: A = dout rows; B0 = W_down read K-major ([E, f, d] as N = f rows of K = d); S0 shared.
+//   DH: A = dout rows; B0 = W_down read K-major ([E, f, d] as N = f rows of K = d); S0 shared;
+//       B1 / S1 the TMA store maps of dg|du in bf16 and in fp16.
 //   DX: A = [dg|du]; B0/B1 = W_gate/W_up read K-major ([E, d, f] as N = d rows of K = f); S0/S1 shared.
-//   WG: A = (w h)^T or xg^T [M, rp]; B0 = the activation rows, N-major (4 chunks a copy).
+//   WG: A = (w h)^T or xg^T [M, rp]; B0 = the activation rows, N-major (4 chunks a copy);
+//       S0 / S1 the TMA store maps of the routed experts' and the shared expert's gradient.
 template <int MODE>
 __global__ void __launch_bounds__(kThreads, 1)
     bwd_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB0,
@@ -567,7 +583,9 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (!okl) break;
             tc_fence_after();
             const uint32_t tb = tmem_base + (uint32_t(q * 32) << 16) + uint32_t(acc * BN);
-            epilogue<MODE>(tb, U, q, half, lane, p, range_bad, stage_out + (warp - 2) * 32 * 32, ri, &tmS0, &tmS1);
+            // TMA store maps: WG S0 / S1 (routed, shared gradient); DH B1 / S1 (dg|du bf16, fp16)
+            epilogue<MODE>(tb, U, q, half, lane, p, range_bad, stage_out + (warp - 2) * 32 * 32, ri,
+                           MODE == DH ? &tmB1 : &tmS0, &tmS1);
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(tempty + acc);
@@ -577,7 +595,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
         }
         if (range_bad) set_error(p.err, MOE_DEVERR_RANGE);
-        if (MODE == WG && lane == 0) bulk_wait0();  // this warp's gradient stores are complete
+        if ((MODE == WG || MODE == DH) && lane == 0) bulk_wait0();  // this warp's TMA stores are complete
     }
     __syncthreads();
     if (warp == 1) {
@@ -784,6 +802,7 @@ cudaError_t launch_mode(const CUtensorMap& A, const CUtensorMap& B0, const CUten
 namespace tc {
 bool map_weights_kmajor(CUtensorMap* m, const void* base, int nexp, int N, int K, bool f16 = false);
 bool map_f32_tiles(CUtensorMap* m, const void* base, int nexp, int M, int N);
+bool map_rows_store32(CUtensorMap* m, const void* base, int64_t rows, int cols, bool f16);
 bool map_act_mn(CUtensorMap* m, const void* base, int64_t rows, int N, int64_t row_stride, int chunks);
 }  // namespace tc
 
@@ -878,7 +897,13 @@ cudaError_t launch_backward(const Dims& D, const BwdArgs& a, cudaStream_t s) {
     p.K = d;
     p.n_tiles = nt_dh;
     p.unit_counter = counters + 1;
-    if ((e = launch_mode<DH>(mDog, mDk, mDk, sDk, sDk, p, s)) != cudaSuccess) return e;
+    {
+        // B1 / S1 of the DH launch: its TMA store maps for dg|du in bf16 and in fp16
+        CUtensorMap stB, stH;
+        if (!tc::map_rows_store32(&stB, dgu, rp, 2 * f, false) || !tc::map_rows_store32(&stH, dgu16, rp, 2 * f, true))
+            return cudaErrorInvalidValue;
+        if ((e = launch_mode<DH>(mDog, mDk, stB, sDk, stH, p, s)) != cudaSuccess) return e;
+    }
     // DX: dx rows
     p.K = 2 * f;
     p.n_tiles = (d + BN - 1) / BN;

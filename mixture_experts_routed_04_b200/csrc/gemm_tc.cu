@@ -586,6 +586,15 @@ bool map_act_mn(CUtensorMap* m, const void* base, int64_t rows, int N, int64_t r
     const uint32_t box[4] = {64, 64, uint32_t(chunks), 1};
     return make_map(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, base, 4, dims, str, box, CU_TENSOR_MAP_SWIZZLE_128B);
 }
+// 2-byte rows [rows, cols] (bf16 or fp16) written by 32 x 32 boxes (64-byte swizzle)
+// from shared memory.
+bool map_rows_store32(CUtensorMap* m, const void* base, int64_t rows, int cols, bool f16) {
+    const uint64_t dims[2] = {uint64_t(cols), uint64_t(rows)};
+    const uint64_t str[1] = {uint64_t(cols) * 2};
+    const uint32_t box[2] = {32, 32};
+    return make_map(m, f16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, base, 2, dims, str,
+                    box, CU_TENSOR_MAP_SWIZZLE_64B);
+}
 // fp32 [nexp, M, N] written by 32 x 32 boxes (128-byte swizzle) from shared memory.
 bool map_f32_tiles(CUtensorMap* m, const void* base, int nexp, int M, int N) {
     const uint64_t dims[3] = {uint64_t(N), uint64_t(M), uint64_t(nexp)};
