@@ -183,9 +183,31 @@ MOE_DEV RowInfo row_info(const Unit& U, int q, int lane, const Params& p) {
     return r;
 }
 
+// One 32 x 32 box of 2-byte values (this lane's row: src, 16 packed pairs) out by a TMA
+// store through buffer nb % 2 of the warp's two 2 KB buffers, in the 64-byte swizzle
+// (16-byte group j of row r at j ^ ((r / 2) % 4)); a buffer is rewritten once the store
+// that used it two boxes ago has read it. nb counts the warp's boxes across units.
+MOE_DEV void store_box32(uint8_t* stage, int& nb, const uint32_t (&src)[16], const CUtensorMap* m, int x, int y,
+                         int lane) {
+    uint8_t* buf = stage + (nb & 1) * 2048;
+    if (lane == 0) bulk_wait_read1();
+    __syncwarp();
+#pragma unroll
+    for (int j = 0; j < 4; ++j)
+        *reinterpret_cast<uint4*>(buf + lane * 64 + ((j ^ ((lane >> 1) & 3)) << 4)) =
+            make_uint4(src[4 * j], src[4 * j + 1], src[4 * j + 2], src[4 * j + 3]);
+    fence_proxy_async_smem();
+    __syncwarp();
+    if (lane == 0) {
+        tma_store_2d(m, buf, x, y);
+        bulk_commit();
+    }
+    ++nb;
+}
+
 template <int MODE>
 MOE_DEV void epilogue(uint32_t tb, const Unit& U, int q, int half, int lane, const Params& p, bool& range_bad,
-                      float* stage_out, RowInfo ri, const CUtensorMap* st0, const CUtensorMap* st1) {
+                      float* stage_out, RowInfo ri, const CUtensorMap* st0, const CUtensorMap* st1, int& nb) {
     const int rit = q * 32 + lane;
     const bool valid = rit < U.rows;
     if (MODE == WG) {
@@ -223,6 +245,10 @@ MOE_DEV void epilogue(uint32_t tb, const Unit& U, int q, int half, int lane, con
     const float w = ri.w;
     const int f = p.f, f2 = 2 * p.f;
     const float L = p.limit;
+    // padded row counts are multiples of 64, so a warp's 32 rows are all valid or none (the
+    // TMA stores of GU and DH write whole 32-row boxes)
+    const bool wvalid = q * 32 < U.rows && (U.rows & 31) == 0;
+    if (q * 32 < U.rows && (U.rows & 31) != 0 && lane == 0) set_error(p.err, MOE_DEVERR_BOUNDS);
     if (MODE == GU) {
 #pragma unroll 1
         for (int c = half; c < 4; c += 2) {
@@ -231,7 +257,7 @@ MOE_DEV void epilogue(uint32_t tb, const Unit& U, int q, int half, int lane, con
             tmem_ld_32x32b_x32(tb + 128 + c * 32, v);
             tmem_ld_wait();
             const int col = U.n * 128 + c * 32;
-            if (valid && col < f) {
+            if (wvalid && col < f) {  // warp-uniform: the TMA stores below need every lane
                 uint32_t pg[16], pu[16], pw[16];
 #pragma unroll
                 for (int i = 0; i < 16; ++i) {
@@ -246,22 +272,16 @@ MOE_DEV void epilogue(uint32_t tb, const Unit& U, int q, int half, int lane, con
                     pu[i] = pack_f16x2(cu0, cu1);
                     pw[i] = pack_f16x2(w * h0, w * h1);
                 }
-                uint4* gd = reinterpret_cast<uint4*>(p.gu + prow * f2 + col);
-                uint4* ud = reinterpret_cast<uint4*>(p.gu + prow * f2 + f + col);
-                uint4* wd = reinterpret_cast<uint4*>(p.hw + prow * f + col);
-#pragma unroll
-                for (int i = 0; i < 4; ++i) {
-                    gd[i] = make_uint4(pg[4 * i], pg[4 * i + 1], pg[4 * i + 2], pg[4 * i + 3]);
-                    ud[i] = make_uint4(pu[4 * i], pu[4 * i + 1], pu[4 * i + 2], pu[4 * i + 3]);
-                    wd[i] = make_uint4(pw[4 * i], pw[4 * i + 1], pw[4 * i + 2], pw[4 * i + 3]);
-                }
+                // g, u codes (gu) and w h (hw): three boxes by TMA store (lane 0's row is the
+                // warp's first)
+                uint8_t* stage = reinterpret_cast<uint8_t*>(stage_out);
+                store_box32(stage, nb, pg, st0, col, int(prow), lane);
+                store_box32(stage, nb, pu, st0, f + col, int(prow), lane);
+                store_box32(stage, nb, pw, st1, col, int(prow), lane);
             }
         }
     } else if (MODE == DH) {
         float dot = 0.f;
-        // padded row counts are multiples of 64, so a warp's 32 rows are all valid or none
-        const bool wvalid = q * 32 < U.rows && (U.rows & 31) == 0;
-        if (q * 32 < U.rows && (U.rows & 31) != 0 && lane == 0) set_error(p.err, MOE_DEVERR_BOUNDS);
         // the chunk's g and u (fp16), 8 vector loads issued together, one chunk ahead: the
         // next chunk's are in flight while this one is computed and stored
         auto load_gu = [&](int c, uint4 (&gq)[4], uint4 (&uq)[4]) {
@@ -327,23 +347,11 @@ MOE_DEV void epilogue(uint32_t tb, const Unit& U, int q, int half, int lane, con
                 // of row r at j ^ ((r / 2) % 4)); a buffer is rewritten once the store that
                 // used it two boxes ago has read it. The warp's 32 rows are all inside the
                 // expert's padded rows (their count is a multiple of 64), so whole boxes go out.
-#pragma unroll
-                for (int bx = 0; bx < 4; ++bx) {
-                    const uint32_t* src = bx == 0 ? pg : bx == 1 ? pu : bx == 2 ? qg : qu;
-                    uint8_t* buf = reinterpret_cast<uint8_t*>(stage_out) + (bx & 1) * 2048;
-                    if (lane == 0) bulk_wait_read1();
-                    __syncwarp();
-#pragma unroll
-                    for (int j = 0; j < 4; ++j)
-                        *reinterpret_cast<uint4*>(buf + lane * 64 + ((j ^ ((lane >> 1) & 3)) << 4)) =
-                            make_uint4(src[4 * j], src[4 * j + 1], src[4 * j + 2], src[4 * j + 3]);
-                    fence_proxy_async_smem();
-                    __syncwarp();
-                    if (lane == 0) {
-                        tma_store_2d(bx < 2 ? st0 : st1, buf, (bx & 1 ? f : 0) + col, int(prow));  // bf16, fp16
-                        bulk_commit();
-                    }
-                }
+                uint8_t* stage = reinterpret_cast<uint8_t*>(stage_out);
+                store_box32(stage, nb, pg, st0, col, int(prow), lane);  // bf16
+                store_box32(stage, nb, pu, st0, f + col, int(prow), lane);
+                store_box32(stage, nb, qg, st1, col, int(prow), lane);  // fp16
+                store_box32(stage, nb, qu, st1, f + col, int(prow), lane);
             }
         }
         if (real >= 0) p.dwp[(int64_t(real) * p.n_tiles + U.n) * 2 + half] = dot;
@@ -372,16 +380,17 @@ MOE_DEV void epilogue(uint32_t tb, const Unit& U, int q, int half, int lane, con
 
 // Operand maps per mode:
 //   GU: A = xg; B0/B1 = W_gate/W_up (N-major, 2 chunks a copy), S0/S1 the shared expert's.
-//   DH: A = dout rows; B0 = W_down read K-major ([E, f, d] as N = f rows of K = d); S0 shared;
-//       B1 / S1 the TMA store maps of dg|du in bf16 and in fp16.
+//   DH: A = dout rows; B0 = W_down read K-major ([E, f, d] as N = f rows of K = d); S0 shared.
 //   DX: A = [dg|du]; B0/B1 = W_gate/W_up read K-major ([E, d, f] as N = d rows of K = f); S0/S1 shared.
-//   WG: A = (w h)^T or xg^T [M, rp]; B0 = the activation rows, N-major (4 chunks a copy);
-//       S0 / S1 the TMA store maps of the routed experts' and the shared expert's gradient.
+//   WG: A = (w h)^T or xg^T [M, rp]; B0 = the activation rows, N-major (4 chunks a copy).
+// TMA store maps O0 / O1: GU g|u and w h (fp16); DH dg|du in bf16 and in fp16; WG the
+// routed experts' and the shared expert's gradient (fp32); DX none.
 template <int MODE>
 __global__ void __launch_bounds__(kThreads, 1)
     bwd_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB0,
                     const __grid_constant__ CUtensorMap tmB1, const __grid_constant__ CUtensorMap tmS0,
-                    const __grid_constant__ CUtensorMap tmS1, const Params p) {
+                    const __grid_constant__ CUtensorMap tmS1, const __grid_constant__ CUtensorMap tmO0,
+                    const __grid_constant__ CUtensorMap tmO1, const Params p) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint64_t* full = reinterpret_cast<uint64_t*>(smem + kStages * kStageBytes);
@@ -571,6 +580,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         bool range_bad = false;
         int uslot = 0;
         uint32_t uphase = 0;
+        int nb = 0;  // TMA store boxes of this warp (GU, DH)
         while (true) {
             int u = -1;
             if (!tc::ring_read(u, uslot, uphase, unit_ring, ufull, uempty, abort_flag, p.err, p.wait_ns)) break;
@@ -583,9 +593,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (!okl) break;
             tc_fence_after();
             const uint32_t tb = tmem_base + (uint32_t(q * 32) << 16) + uint32_t(acc * BN);
-            // TMA store maps: WG S0 / S1 (routed, shared gradient); DH B1 / S1 (dg|du bf16, fp16)
-            epilogue<MODE>(tb, U, q, half, lane, p, range_bad, stage_out + (warp - 2) * 32 * 32, ri,
-                           MODE == DH ? &tmB1 : &tmS0, &tmS1);
+            epilogue<MODE>(tb, U, q, half, lane, p, range_bad, stage_out + (warp - 2) * 32 * 32, ri, &tmO0, &tmO1,
+                           nb);
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(tempty + acc);
@@ -595,7 +604,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
         }
         if (range_bad) set_error(p.err, MOE_DEVERR_RANGE);
-        if ((MODE == WG || MODE == DH) && lane == 0) bulk_wait0();  // this warp's TMA stores are complete
+        if (MODE != DX && lane == 0) bulk_wait0();  // this warp's TMA stores are complete
     }
     __syncthreads();
     if (warp == 1) {
@@ -778,7 +787,8 @@ __global__ void __launch_bounds__(256) zero_untouched_kernel(const int32_t* __re
 
 template <int MODE>
 cudaError_t launch_mode(const CUtensorMap& A, const CUtensorMap& B0, const CUtensorMap& B1, const CUtensorMap& S0,
-                        const CUtensorMap& S1, const Params& p, cudaStream_t s) {
+                        const CUtensorMap& S1, const CUtensorMap& O0, const CUtensorMap& O1, const Params& p,
+                        cudaStream_t s) {
     static int configured_dev = -1;
     int dev = 0;
     cudaGetDevice(&dev);
@@ -791,7 +801,8 @@ cudaError_t launch_mode(const CUtensorMap& A, const CUtensorMap& B0, const CUten
     {
         ProfScope prof_(MOE_K_BWD_GEMM, s);
         const cudaError_t le =
-            launch_pdl(false, bwd_gemm_kernel<MODE>, dim3(num_sms()), dim3(kThreads), kSmem, s, A, B0, B1, S0, S1, p);
+            launch_pdl(false, bwd_gemm_kernel<MODE>, dim3(num_sms()), dim3(kThreads), kSmem, s, A, B0, B1, S0, S1, O0,
+                       O1, p);
         if (le != cudaSuccess) return le;
     }
     return cudaGetLastError();
@@ -892,26 +903,32 @@ cudaError_t launch_backward(const Dims& D, const BwdArgs& a, cudaStream_t s) {
     p.K = d;
     p.n_tiles = (f + 127) / 128;
     p.unit_counter = counters + 0;
-    if ((e = launch_mode<GU>(mX, mG, mU, sG, sU, p, s)) != cudaSuccess) return e;
+    {
+        // GU's TMA store maps: the g|u codes and w h (fp16)
+        CUtensorMap stGU, stHW;
+        if (!tc::map_rows_store32(&stGU, gu, rp, 2 * f, true) || !tc::map_rows_store32(&stHW, hw, rp, f, true))
+            return cudaErrorInvalidValue;
+        if ((e = launch_mode<GU>(mX, mG, mU, sG, sU, stGU, stHW, p, s)) != cudaSuccess) return e;
+    }
     // DH: dg, du; <h, dhu> partials
     p.K = d;
     p.n_tiles = nt_dh;
     p.unit_counter = counters + 1;
     {
-        // B1 / S1 of the DH launch: its TMA store maps for dg|du in bf16 and in fp16
+        // DH's TMA store maps: dg|du in bf16 and in fp16
         CUtensorMap stB, stH;
         if (!tc::map_rows_store32(&stB, dgu, rp, 2 * f, false) || !tc::map_rows_store32(&stH, dgu16, rp, 2 * f, true))
             return cudaErrorInvalidValue;
-        if ((e = launch_mode<DH>(mDog, mDk, stB, sDk, stH, p, s)) != cudaSuccess) return e;
+        if ((e = launch_mode<DH>(mDog, mDk, mDk, sDk, sDk, stB, stH, p, s)) != cudaSuccess) return e;
     }
     // DX: dx rows
     p.K = 2 * f;
     p.n_tiles = (d + BN - 1) / BN;
     p.unit_counter = counters + 2;
-    if ((e = launch_mode<DX>(mDgu, mGk, mUk, sGk, sUk, p, s)) != cudaSuccess) return e;
-    // WG: dW_down = (w h)^T dout_rows [f, d]; dW_gate = xg^T dg, dW_up = xg^T du [d, f]. The
-    // S0 / S1 maps of a WG launch are its TMA store maps: the routed experts' gradient and
-    // the shared expert's (the routed map again without one).
+    if ((e = launch_mode<DX>(mDgu, mGk, mUk, sGk, sUk, mDgu, mDgu, p, s)) != cudaSuccess) return e;
+    // WG: dW_down = (w h)^T dout_rows [f, d]; dW_gate = xg^T dg, dW_up = xg^T du [d, f]; its
+    // TMA store maps: the routed experts' gradient and the shared expert's (the routed map
+    // again without one).
     auto wg = [&](const CUtensorMap& A, const CUtensorMap& B, float* dw, float* sdw, int M, int N,
                   int32_t* counter) -> cudaError_t {
         CUtensorMap stD, stS;
@@ -923,7 +940,7 @@ cudaError_t launch_backward(const Dims& D, const BwdArgs& a, cudaStream_t s) {
         p.dw = dw;
         p.sdw = sdw;
         p.unit_counter = counter;
-        return launch_mode<WG>(A, B, B, stD, stS, p, s);
+        return launch_mode<WG>(A, B, B, B, B, stD, stS, p, s);
     };
     float* sd = D.has_shared ? a.g->dshared_down : nullptr;
     float* sg = D.has_shared ? a.g->dshared_gate : nullptr;
