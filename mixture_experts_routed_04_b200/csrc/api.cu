@@ -83,7 +83,8 @@ int make_dims(const moe_params* p, Dims* D) {
     }
     D->rows = routed_rows + (p->has_shared ? p->T : 0);
     if (D->rows < 1) D->rows = 1;
-    D->perm_blocks = int((pairs + kPermPairsPerBlock - 1) / kPermPairsPerBlock);
+    const int64_t ppb = int64_t(kPermWarps) * 32 * perm_rounds(pairs);  // pairs per permutation block
+    D->perm_blocks = int((pairs + ppb - 1) / ppb);
     D->fmt = p->weight_format;
     D->variant = p->variant;
     // Default variant choice from the measured table (kStreamTable): the

@@ -8,8 +8,13 @@ namespace moe {
 constexpr int kMaxE = 256;
 constexpr int kMaxK = 8;
 constexpr int kPermWarps = 8;                         // warps per permutation block
-constexpr int kPermPairsPerWarp = 256;                // 8 rounds of 32 pairs
-constexpr int kPermPairsPerBlock = kPermWarps * kPermPairsPerWarp;
+// Rounds of 32 pairs per permutation warp: 2 (512-pair blocks) spread prompt-sized
+// batches over more SMs; above kPermSmallPairs pairs, 8 (2048-pair blocks) keep the
+// scan over the blocks short.
+constexpr int kPermRoundsSmall = 2, kPermRoundsLarge = 8;
+constexpr int64_t kPermSmallPairs = 65536;
+inline int perm_rounds(int64_t pairs) { return pairs <= kPermSmallPairs ? kPermRoundsSmall : kPermRoundsLarge; }
+constexpr int kPermMaxPairsPerBlock = kPermWarps * 32 * kPermRoundsLarge;
 constexpr int kTileM = 128;                           // rows per tcgen05 tile
 // AUTO variant choice, measured on B200 (decode-shaped layers, d=4096, f=1536,
 // E=256 + shared, whose routing gives `touched` experts the same rows each;

@@ -9,8 +9,8 @@
 // this library's permutation. Such a caller passes only its inputs and
 // outputs; the per-block histograms and bases live in g_perm_scratch below.
 //
-// Costs and limits: the array is MOE_NOALLOC_MAX_PAIRS / 2048 blocks x 256
-// experts x 2 int32 (256 KiB) and stays allocated on every GPU that loads the
+// Costs and limits: the array is 128 permutation blocks x 256 experts x 2 int32
+// (256 KiB) and stays allocated on every GPU that loads the
 // library until the process exits. Every call uses the same array, so calls
 // whose work overlaps on the GPU (different streams, or different host
 // threads) race and must not be issued; calls on one stream are ordered and
@@ -24,10 +24,14 @@ namespace moe {
 
 namespace {
 
-constexpr int kNoAllocMaxBlocks = MOE_NOALLOC_MAX_PAIRS / kPermPairsPerBlock;  // 128
+// the most blocks a call may use: small batches' blocks at kPermSmallPairs, or large ones'
+constexpr int kNoAllocMaxBlocks =
+    (kPermSmallPairs / (kPermWarps * 32 * kPermRoundsSmall)) > (MOE_NOALLOC_MAX_PAIRS / kPermMaxPairsPerBlock)
+        ? int(kPermSmallPairs / (kPermWarps * 32 * kPermRoundsSmall))
+        : int(MOE_NOALLOC_MAX_PAIRS / kPermMaxPairsPerBlock);  // 128
 constexpr int kNoAllocInts = 2 * kNoAllocMaxBlocks * kMaxE;                   // counts + bases
 
-static_assert(MOE_NOALLOC_MAX_PAIRS % kPermPairsPerBlock == 0, "pair limit must be whole blocks");
+static_assert(MOE_NOALLOC_MAX_PAIRS % kPermMaxPairsPerBlock == 0, "pair limit must be whole blocks");
 
 // The fixed scratch: per-block expert counts, then per-block expert bases.
 static __device__ __align__(256) int32_t g_perm_scratch[kNoAllocInts];
@@ -71,7 +75,8 @@ extern "C" MOE_API int moe_permute_noalloc(const moe_params* p, const int32_t* t
     Dims D{};
     const int st = make_dims(p, &D);
     if (st != MOE_OK) return st;
-    if (D.pairs > MOE_NOALLOC_MAX_PAIRS) return MOE_ERR_WORKSPACE_TOO_SMALL;  // beyond the fixed scratch
+    if (D.pairs > MOE_NOALLOC_MAX_PAIRS || D.perm_blocks > kNoAllocMaxBlocks)
+        return MOE_ERR_WORKSPACE_TOO_SMALL;  // beyond the fixed scratch
     if (!topk_idx || !counts || !kept_counts || !offsets || !sorted_token || !sorted_pair || !pair_row ||
         !err_word)
         return MOE_ERR_INVALID_ARG;

@@ -7,8 +7,10 @@
 // clamped. Here the pairs keep token order inside each expert (pair p = t*k+j
 // ranks before p' > p), and the first `cap` of an expert are kept.
 //
-// Three launches over the T*k pairs, which are cut into blocks of 2048 pairs,
-// 256 per warp in 8 rounds of 32:
+// Three launches over the T*k pairs, which are cut into blocks of 8 warps x
+// ROUNDS rounds of 32 pairs (2 rounds up to 64K pairs, so that the counts and the
+// scatter of prompt-sized batches spread over more SMs; 8 rounds above, so that the
+// scan over the blocks stays short):
 //   count   — each warp counts its pairs per expert (__match_any_sync groups
 //             equal ids in a round; the group's lowest lane adds the popcount
 //             to the warp's own smem row, so no two lanes write one counter),
@@ -35,16 +37,17 @@ MOE_DEV uint32_t lanemask_lt() {
 }
 
 // Fill hist[w][e] with warp w's pair count per expert for block `b`.
+template <int ROUNDS>
 MOE_DEV void warp_histograms(const int32_t* __restrict__ topk_idx, int64_t pairs, int E, int (*hist)[kMaxE],
                              uint32_t* err) {
     const int w = threadIdx.x >> 5, lane = threadIdx.x & 31;
     for (int i = threadIdx.x; i < kPermWarps * kMaxE; i += blockDim.x) (&hist[0][0])[i] = 0;
     __syncthreads();
-    const int64_t base = int64_t(blockIdx.x) * kPermPairsPerBlock + int64_t(w) * kPermPairsPerWarp;
+    const int64_t base = (int64_t(blockIdx.x) * kPermWarps + w) * (32 * ROUNDS);
     // every round's ids first (one memory latency for the warp's 256 pairs)
-    int ids[kPermPairsPerWarp / 32];
+    int ids[ROUNDS];
 #pragma unroll
-    for (int it = 0; it < kPermPairsPerWarp / 32; ++it) {
+    for (int it = 0; it < ROUNDS; ++it) {
         const int64_t p = base + it * 32 + lane;
         int e = -1;
         if (p < pairs) {
@@ -57,7 +60,7 @@ MOE_DEV void warp_histograms(const int32_t* __restrict__ topk_idx, int64_t pairs
         ids[it] = e;
     }
 #pragma unroll
-    for (int it = 0; it < kPermPairsPerWarp / 32; ++it) {
+    for (int it = 0; it < ROUNDS; ++it) {
         const int e = ids[it];
         const uint32_t peers = __match_any_sync(0xFFFFFFFFu, e);
         if (e >= 0 && (__ffs(peers) - 1) == lane) hist[w][e] += __popc(peers);
@@ -66,6 +69,7 @@ MOE_DEV void warp_histograms(const int32_t* __restrict__ topk_idx, int64_t pairs
     __syncthreads();
 }
 
+template <int ROUNDS>
 __global__ void __launch_bounds__(kPermWarps * 32) perm_count_kernel(const int32_t* __restrict__ topk_idx,
                                                                      int64_t pairs, int E,
                                                                      int32_t* __restrict__ blockcounts,
@@ -73,7 +77,7 @@ __global__ void __launch_bounds__(kPermWarps * 32) perm_count_kernel(const int32
     __shared__ int hist[kPermWarps][kMaxE];
     griddep_wait();
     griddep_launch();
-    warp_histograms(topk_idx, pairs, E, hist, err);
+    warp_histograms<ROUNDS>(topk_idx, pairs, E, hist, err);
     for (int e = threadIdx.x; e < E; e += blockDim.x) {
         int s = 0;
 #pragma unroll
@@ -100,6 +104,7 @@ __global__ void __launch_bounds__(SCHED ? 512 : kMaxE)
     int kv = 0;
     if (e < E) {
         int run = 0;
+#pragma unroll 8
         for (int b = 0; b < nblocks; ++b) {
             const int c = blockcounts[int64_t(b) * E + e];
             blockbase[int64_t(b) * E + e] = run;
@@ -141,6 +146,7 @@ __global__ void __launch_bounds__(SCHED ? 512 : kMaxE)
     }
 }
 
+template <int ROUNDS>
 __global__ void __launch_bounds__(kPermWarps * 32) perm_scatter_kernel(
     const int32_t* __restrict__ topk_idx, int64_t pairs, int k, int E, int cap,
     const int32_t* __restrict__ blockbase, const int32_t* __restrict__ offsets,
@@ -149,7 +155,7 @@ __global__ void __launch_bounds__(kPermWarps * 32) perm_scatter_kernel(
     __shared__ int hist[kPermWarps][kMaxE];
     griddep_wait();
     griddep_launch();
-    warp_histograms(topk_idx, pairs, E, hist, nullptr);  // errors were reported by the count pass
+    warp_histograms<ROUNDS>(topk_idx, pairs, E, hist, nullptr);  // errors were reported by the count pass
     // warp totals -> warp bases (block base + earlier warps), per expert
     for (int e = threadIdx.x; e < E; e += blockDim.x) {
         int run = blockbase[int64_t(blockIdx.x) * E + e];
@@ -162,10 +168,10 @@ __global__ void __launch_bounds__(kPermWarps * 32) perm_scatter_kernel(
     }
     __syncthreads();
     const int w = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int64_t base = int64_t(blockIdx.x) * kPermPairsPerBlock + int64_t(w) * kPermPairsPerWarp;
-    int ids[kPermPairsPerWarp / 32];
+    const int64_t base = (int64_t(blockIdx.x) * kPermWarps + w) * (32 * ROUNDS);
+    int ids[ROUNDS];
 #pragma unroll
-    for (int it = 0; it < kPermPairsPerWarp / 32; ++it) {
+    for (int it = 0; it < ROUNDS; ++it) {
         const int64_t p = base + it * 32 + lane;
         int e = -1;
         if (p < pairs) {
@@ -175,7 +181,7 @@ __global__ void __launch_bounds__(kPermWarps * 32) perm_scatter_kernel(
         ids[it] = e;
     }
 #pragma unroll
-    for (int it = 0; it < kPermPairsPerWarp / 32; ++it) {
+    for (int it = 0; it < ROUNDS; ++it) {
         const int64_t p = base + it * 32 + lane;
         const int e = ids[it];
         const uint32_t peers = __match_any_sync(0xFFFFFFFFu, e);
@@ -223,8 +229,12 @@ cudaError_t launch_permute(const Dims& D, const int32_t* topk_idx, int32_t* bloc
     const int shared_T = D.has_shared ? D.T : 0;
     {
         ProfScope prof_(MOE_K_PERM_COUNT, s);
-        const cudaError_t le = launch_pdl(use_pdl(D.T), perm_count_kernel, dim3(nb), dim3(kPermWarps * 32), 0, s,
-                                          topk_idx, D.pairs, D.E, blockcounts, err);
+        const bool small = perm_rounds(D.pairs) == kPermRoundsSmall;
+        const cudaError_t le =
+            small ? launch_pdl(use_pdl(D.T), perm_count_kernel<kPermRoundsSmall>, dim3(nb), dim3(kPermWarps * 32), 0,
+                               s, topk_idx, D.pairs, D.E, blockcounts, err)
+                  : launch_pdl(use_pdl(D.T), perm_count_kernel<kPermRoundsLarge>, dim3(nb), dim3(kPermWarps * 32), 0,
+                               s, topk_idx, D.pairs, D.E, blockcounts, err);
         if (le != cudaSuccess) return le;
     }
     {
@@ -239,9 +249,14 @@ cudaError_t launch_permute(const Dims& D, const int32_t* topk_idx, int32_t* bloc
     }
     {
         ProfScope prof_(MOE_K_PERM_SCATTER, s);
-        const cudaError_t le = launch_pdl(use_pdl(D.T), perm_scatter_kernel, dim3(nb), dim3(kPermWarps * 32), 0, s,
-                                          topk_idx, D.pairs, D.k, D.E, D.cap, blockbase, offsets, sorted_token,
-                                          sorted_pair, pair_row, shared_T, err);
+        const bool small = perm_rounds(D.pairs) == kPermRoundsSmall;
+        const cudaError_t le =
+            small ? launch_pdl(use_pdl(D.T), perm_scatter_kernel<kPermRoundsSmall>, dim3(nb), dim3(kPermWarps * 32),
+                               0, s, topk_idx, D.pairs, D.k, D.E, D.cap, blockbase, offsets, sorted_token,
+                               sorted_pair, pair_row, shared_T, err)
+                  : launch_pdl(use_pdl(D.T), perm_scatter_kernel<kPermRoundsLarge>, dim3(nb), dim3(kPermWarps * 32),
+                               0, s, topk_idx, D.pairs, D.k, D.E, D.cap, blockbase, offsets, sorted_token,
+                               sorted_pair, pair_row, shared_T, err);
         if (le != cudaSuccess) return le;
     }
     return cudaGetLastError();
