@@ -682,7 +682,7 @@ cudaError_t launch_tensor_ffn(const Dims& D, const uint16_t* xg, uint16_t* h, co
         p.n_tiles = (D.d + BN - 1) / BN;
         p.out = y_rows;
         p.unit_counter = counters + 1;
-        return launch_gemm<1, 1, 1>(mH, pd, pd, sd, sd, p, pdl, s);
+        return launch_gemm<1, 1, 2>(mH, pd, pd, sd, sd, p, pdl, s);
     }
     CUtensorMap mG, mU, mSG, mSU, mD, mSD;
     if (!map_weights(&mG, w->w_gate, D.E, D.d, D.f, 2) || !map_weights(&mU, w->w_up, D.E, D.d, D.f, 2) ||
