@@ -475,7 +475,9 @@ MOE_API int moe_expert_ffn_backward(const moe_params* p, const uint16_t* x, cons
 /*
  * Number of kernel launches one call of `which` (MOE_WS_ROUTE .. MOE_WS_BACKWARD,
  * naming moe_route .. moe_forward_host, moe_route_stats, moe_expert_ffn_backward)
- * makes with these params, into *n (host).
+ * makes with these params, into *n (host). For moe_expert_ffn_backward the count
+ * includes the routing-logit gradient, launched when dlogits is given (one fewer
+ * without).
  */
 MOE_API int moe_launch_count(const moe_params* p, int which, int* n);
 

@@ -588,7 +588,8 @@ int moe_launch_count(const moe_params* p, int which, int* n) {
         case MOE_WS_EXPERT_FFN: *n = ffn; break;
         case MOE_WS_COMBINE: *n = 1; break;
         case MOE_WS_ROUTE_STATS: *n = 2; break;
-        // schedule, gather, 6 GEMMs, zeroing, combine, routing-weight reduce, route backward
+        // schedule, gather, 6 GEMMs, zeroing, combine, routing-weight reduce, and the routing
+        // backward (when dlogits is asked for; 11 without)
         case MOE_WS_BACKWARD: *n = 12; break;
         // moe_forward: the front kernel(s) write the schedule, so the expert FFN's own
         // schedule launch is not made (nor, for the smallest batches, the gather, and

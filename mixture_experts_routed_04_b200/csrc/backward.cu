@@ -967,11 +967,12 @@ cudaError_t launch_backward(const Dims& D, const BwdArgs& a, cudaStream_t s) {
         if ((e = launch_pdl(false, dw_reduce_kernel, dim3(int(blocks)), dim3(256), 0, s, a.pair_row, dwp, D.pairs,
                             nt_dh, int64_t(D.rows), a.g->d_topk_w, a.err)) != cudaSuccess)
             return e;
-        if (a.g->dlogits && a.topk_idx) {
-            if ((e = launch_pdl(false, route_backward_kernel, dim3((D.T + 7) / 8), dim3(256), 0, s, a.topk_idx,
-                                a.topk_w, a.g->d_topk_w, D.T, D.E, D.k, a.g->dlogits)) != cudaSuccess)
-                return e;
-        }
+    }
+    if (a.g->dlogits && a.topk_idx) {
+        ProfScope prof_(MOE_K_BWD_SMALL, s);
+        if ((e = launch_pdl(false, route_backward_kernel, dim3((D.T + 7) / 8), dim3(256), 0, s, a.topk_idx, a.topk_w,
+                            a.g->d_topk_w, D.T, D.E, D.k, a.g->dlogits)) != cudaSuccess)
+            return e;
     }
     return cudaGetLastError();
 }
