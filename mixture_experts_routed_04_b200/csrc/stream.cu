@@ -10,7 +10,7 @@
 //
 // Work item = (expert, output columns, K slice, chunk of <= 8 rows): 64
 // columns of W_gate and of W_up, or 256 columns of W_down. One CTA per SM,
-// persistent, everything through one TMA ring (119 KB gate/up, 198 KB down):
+// persistent, everything through one TMA ring (204 KB gate/up, 198 KB down):
 //   warp 0     TMA producer: per 64-K block, the 64 x 64 weight boxes (gate
 //              and up, or four of down; 128-byte swizzle) and the 8 x 64 tile
 //              of the chunk's rows (gathered x, or h; 128-byte swizzle).
@@ -52,8 +52,8 @@ struct SCfg {
     static constexpr int NMAT = MODE == 0 ? 2 : 4;                // weight boxes per stage
     static constexpr int NSU = MODE == 0 ? NS : 4 * NS;           // output columns per item
     static constexpr int STAGE = NMAT * TILE + (FOLD ? 0 : XT);   // 17 KB / 33 KB (32 KB folded), 1 KB aligned
-    static constexpr int STAGES = MODE == 0 ? 7 : 6;
-    static constexpr int RING = STAGES * STAGE;                   // 119 KB / 198 KB
+    static constexpr int STAGES = MODE == 0 ? 12 : 6;
+    static constexpr int RING = STAGES * STAGE;                   // 204 KB / 198 KB
     static constexpr int SMEM = 1024 + RING + 512;                // + barriers, abort flag
 };
 // Row stride of the folded h buffer: 16 bytes past the row, so that the 8 rows a
@@ -63,7 +63,8 @@ constexpr int kFoldMaxSmem = 232448;  // dynamic shared memory a block may opt i
 inline bool fold_fits(int f) { return SCfg<1, true>::SMEM + RC * fold_row_bytes(f) <= kFoldMaxSmem; }
 constexpr int kFoldMaxSlices = 4;  // K-split counts the fold takes (its loads are held in registers)
 constexpr int kFoldQ = 3;          // column pairs a consumer thread sums at a time
-static_assert((2 * 7 + 3) * 8 <= 512, "stage barriers, abort flag and the fold's barriers fit the reserved bytes");
+static_assert((2 * SCfg<0>::STAGES + 3) * 8 <= 512 && (2 * SCfg<1>::STAGES + 3) * 8 <= 512,
+              "stage barriers, abort flag and the fold's barriers fit the reserved bytes");
 
 struct StreamParams {
     int mode;            // 0: gate/up, 1: down
