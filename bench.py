@@ -65,6 +65,9 @@ def parse():
     ap.add_argument("--no-per-config", action="store_true",
                     help="skip the other stated workloads (capped, decode1/8/32, quant) in the JSON line")
     ap.add_argument("--tokens", type=int, default=0, help="override T of the workload (profiling small cases)")
+    ap.add_argument("--experts", type=int, default=0,
+                    help="override E of the workload (profiling: a decode layer with fewer untouched experts "
+                         "runs the same kernels on the same touched weights, with less memory held)")
     ap.add_argument("--profile-calls", type=int, default=0,
                     help="only run this many moe_forward calls and exit (for ncu: no timing, no other kernels)")
     ap.add_argument("--profile-op", default="forward", choices=["forward", "backward", "route_stats"],
@@ -921,6 +924,8 @@ def main():
     cfg = synth.CONFIGS[args.config]
     if args.tokens:
         cfg = cfg.replace(T=args.tokens)
+    if args.experts:
+        cfg = cfg.replace(E=args.experts)
     if args.impl == "reference":
         return reference_arm(args, cfg)
     if args.profile_calls:
