@@ -593,11 +593,12 @@ int moe_launch_count(const moe_params* p, int which, int* n) {
         case MOE_WS_BACKWARD: *n = 12; break;
         // moe_forward: the front kernel(s) write the schedule, so the expert FFN's own
         // schedule launch is not made (nor, for the smallest batches, the gather, and
-        // when the streaming down kernel combines, the combine)
+        // when the streaming down kernel combines, the combine); nor, when the scatter
+        // blocks form the scan themselves, the permutation's scan launch
         default:
             *n = D.T <= kFrontMaxTokens
                      ? 1 + (ffn - 1) - (front_gathers(D) && !gather_fused(D) ? 1 : 0) + (combine_fused(D) ? 0 : 1)
-                     : 1 + 3 + (ffn - 1) + 1;
+                     : 1 + (perm_scan_fused(D) ? 2 : 3) + (ffn - 1) + 1;
             break;
     }
     return MOE_OK;

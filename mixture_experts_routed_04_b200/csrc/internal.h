@@ -15,6 +15,11 @@ constexpr int kPermRoundsSmall = 2, kPermRoundsLarge = 8;
 constexpr int64_t kPermSmallPairs = 65536;
 inline int perm_rounds(int64_t pairs) { return pairs <= kPermSmallPairs ? kPermRoundsSmall : kPermRoundsLarge; }
 constexpr int kPermMaxPairsPerBlock = kPermWarps * 32 * kPermRoundsLarge;
+// moe_forward's permutation without its scan launch: each scatter block copies the
+// per-block counts ([blocks][E], at most this many bytes) into shared memory and forms
+// its own bases and the expert offsets; block 0 writes counts, kept, offsets and the
+// tile schedule (one thread per expert: Etot <= the block's 256 threads).
+constexpr int kScanFusedMaxBytes = 96 * 1024;
 constexpr int kTileM = 128;                           // rows per tcgen05 tile
 // AUTO variant choice, measured on B200 (decode-shaped layers, d=4096, f=1536,
 // E=256 + shared, whose routing gives `touched` experts the same rows each;
@@ -44,6 +49,9 @@ struct Dims {
     int down_f16;             // W_down given as fp16 (prepared at load time)
     int tile_pair;            // bf16 tcgen05 GEMMs on SM pairs (256-row tiles)
 };
+inline bool perm_scan_fused(const Dims& D) {
+    return D.Etot <= kPermWarps * 32 && int64_t(D.perm_blocks) * D.E * 4 <= kScanFusedMaxBytes;
+}
 
 // Byte offsets of every scratch array inside a workspace (0 = absent).
 struct WsLayout {

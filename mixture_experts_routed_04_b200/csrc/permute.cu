@@ -146,19 +146,99 @@ __global__ void __launch_bounds__(SCHED ? 512 : kMaxE)
     }
 }
 
-template <int ROUNDS>
+// The scan's outputs a fused scatter block forms itself (FUSED; perm_scan_kernel otherwise).
+struct ScanOut {
+    const int32_t* blockcounts;  // [nblocks][E] from the count pass (16-byte aligned)
+    int nblocks;
+    int32_t* counts;             // block 0 writes counts, kept, offsets and the schedule
+    int32_t* kept;
+    int32_t* offsets;
+    ScheduleArgs sa;
+};
+
+// FUSED: the per-block counts are copied to shared memory (dynamic, nblocks * E
+// ints) and every block forms its base (its earlier blocks' counts, per expert)
+// and the expert offsets itself, in the scan kernel's order, so no scan launch is
+// made; offsets then come from shared memory instead of the scan's output.
+template <int ROUNDS, bool FUSED>
 __global__ void __launch_bounds__(kPermWarps * 32) perm_scatter_kernel(
     const int32_t* __restrict__ topk_idx, int64_t pairs, int k, int E, int cap,
     const int32_t* __restrict__ blockbase, const int32_t* __restrict__ offsets,
     int32_t* __restrict__ sorted_token, int32_t* __restrict__ sorted_pair, int32_t* __restrict__ pair_row,
-    int shared_T, uint32_t* err) {
+    int shared_T, uint32_t* err, ScanOut so) {
     __shared__ int hist[kPermWarps][kMaxE];
+    __shared__ int s_base[FUSED ? kMaxE : 1];
+    __shared__ int s_off[FUSED ? kMaxE + 1 : 1];
+    __shared__ int warp_sums[kPermWarps];
+    __shared__ int sums[3][16];
+    extern __shared__ int4 s_counts4[];
     griddep_wait();
     griddep_launch();
+    if (FUSED) {
+        const int* s_counts = reinterpret_cast<const int*>(s_counts4);
+        const int n = so.nblocks * E;
+        const int n4 = n >> 2;
+        const int4* src4 = reinterpret_cast<const int4*>(so.blockcounts);
+#pragma unroll 4
+        for (int i = threadIdx.x; i < n4; i += blockDim.x) s_counts4[i] = src4[i];
+        for (int i = 4 * n4 + threadIdx.x; i < n; i += blockDim.x)
+            reinterpret_cast<int*>(s_counts4)[i] = so.blockcounts[i];
+        __syncthreads();
+        const int e = threadIdx.x, lane = e & 31, w = e >> 5;
+        int kv = 0;
+        if (e < E) {
+            int before = 0, total = 0;
+#pragma unroll 8
+            for (int b = 0; b < so.nblocks; ++b) {
+                const int c = s_counts[b * E + e];
+                total += c;
+                before += b < int(blockIdx.x) ? c : 0;
+            }
+            s_base[e] = before;
+            kv = (cap >= 0 && total > cap) ? cap : total;
+            if (blockIdx.x == 0) {
+                so.counts[e] = total;
+                so.kept[e] = kv;
+            }
+        }
+        // exclusive scan of kv over the experts
+        int incl = kv;
+#pragma unroll
+        for (int off = 1; off < 32; off <<= 1) {
+            const int v = __shfl_up_sync(0xFFFFFFFFu, incl, off);
+            if (lane >= off) incl += v;
+        }
+        if (lane == 31) warp_sums[w] = incl;
+        __syncthreads();
+        int wbase = 0, routed = 0;
+#pragma unroll
+        for (int i = 0; i < kPermWarps; ++i) {
+            if (i < w) wbase += warp_sums[i];
+            routed += warp_sums[i];
+        }
+        if (e < E) s_off[e] = wbase + incl - kv;
+        if (e == 0) s_off[E] = routed;
+        if (blockIdx.x == 0) {
+            if (e < E) so.offsets[e] = wbase + incl - kv;
+            if (e == 0) {
+                so.offsets[E] = routed;
+                if (shared_T > 0) {
+                    so.counts[E] = shared_T;
+                    so.kept[E] = shared_T;
+                    so.offsets[E + 1] = routed + shared_T;
+                }
+            }
+            const int Etot = E + (shared_T > 0 ? 1 : 0);
+            const int ke = e < E ? kv : (e == E && shared_T > 0 ? shared_T : 0);
+            schedule_block(ke, Etot, so.sa.variant, so.sa.stream_max, sums, so.sa.tile_base, so.sa.stream_list,
+                           so.sa.n_stream);
+        }
+        __syncthreads();
+    }
     warp_histograms<ROUNDS>(topk_idx, pairs, E, hist, nullptr);  // errors were reported by the count pass
     // warp totals -> warp bases (block base + earlier warps), per expert
     for (int e = threadIdx.x; e < E; e += blockDim.x) {
-        int run = blockbase[int64_t(blockIdx.x) * E + e];
+        int run = FUSED ? s_base[e] : blockbase[int64_t(blockIdx.x) * E + e];
 #pragma unroll
         for (int w = 0; w < kPermWarps; ++w) {
             const int c = hist[w][e];
@@ -192,7 +272,7 @@ __global__ void __launch_bounds__(kPermWarps * 32) perm_scatter_kernel(
         __syncwarp();
         if (p < pairs) {
             if (e >= 0 && (cap < 0 || rank < cap)) {
-                const int row = offsets[e] + rank;
+                const int row = (FUSED ? s_off[e] : offsets[e]) + rank;
                 sorted_token[row] = int32_t(p / k);
                 sorted_pair[row] = int32_t(p);
                 pair_row[p] = row;
@@ -203,7 +283,7 @@ __global__ void __launch_bounds__(kPermWarps * 32) perm_scatter_kernel(
     }
     // shared-expert rows: tokens 0..T-1 after the routed rows
     if (shared_T > 0) {
-        const int base_row = offsets[E];
+        const int base_row = FUSED ? s_off[E] : offsets[E];
         for (int64_t t = int64_t(blockIdx.x) * blockDim.x + threadIdx.x; t < shared_T;
              t += int64_t(gridDim.x) * blockDim.x) {
             sorted_token[base_row + t] = int32_t(t);
@@ -237,7 +317,8 @@ cudaError_t launch_permute(const Dims& D, const int32_t* topk_idx, int32_t* bloc
                                s, topk_idx, D.pairs, D.E, blockcounts, err);
         if (le != cudaSuccess) return le;
     }
-    {
+    const bool fused = sched && perm_scan_fused(D);
+    if (!fused) {
         ProfScope prof_(MOE_K_PERM_SCAN, s);
         const ScheduleArgs none{};
         const cudaError_t le =
@@ -250,13 +331,38 @@ cudaError_t launch_permute(const Dims& D, const int32_t* topk_idx, int32_t* bloc
     {
         ProfScope prof_(MOE_K_PERM_SCATTER, s);
         const bool small = perm_rounds(D.pairs) == kPermRoundsSmall;
-        const cudaError_t le =
-            small ? launch_pdl(use_pdl(D.T), perm_scatter_kernel<kPermRoundsSmall>, dim3(nb), dim3(kPermWarps * 32),
-                               0, s, topk_idx, D.pairs, D.k, D.E, D.cap, blockbase, offsets, sorted_token,
-                               sorted_pair, pair_row, shared_T, err)
-                  : launch_pdl(use_pdl(D.T), perm_scatter_kernel<kPermRoundsLarge>, dim3(nb), dim3(kPermWarps * 32),
-                               0, s, topk_idx, D.pairs, D.k, D.E, D.cap, blockbase, offsets, sorted_token,
-                               sorted_pair, pair_row, shared_T, err);
+        cudaError_t le;
+        if (fused) {
+            static int configured_dev = -1;
+            int dev = 0;
+            cudaGetDevice(&dev);
+            if (configured_dev != dev) {
+                if ((le = cudaFuncSetAttribute(perm_scatter_kernel<kPermRoundsSmall, true>,
+                                               cudaFuncAttributeMaxDynamicSharedMemorySize, kScanFusedMaxBytes)) !=
+                        cudaSuccess ||
+                    (le = cudaFuncSetAttribute(perm_scatter_kernel<kPermRoundsLarge, true>,
+                                               cudaFuncAttributeMaxDynamicSharedMemorySize, kScanFusedMaxBytes)) !=
+                        cudaSuccess)
+                    return le;
+                configured_dev = dev;
+            }
+            const ScanOut so{blockcounts, nb, counts, kept, offsets, *sched};
+            const int smem = nb * D.E * 4;
+            le = small ? launch_pdl(use_pdl(D.T), perm_scatter_kernel<kPermRoundsSmall, true>, dim3(nb),
+                                    dim3(kPermWarps * 32), smem, s, topk_idx, D.pairs, D.k, D.E, D.cap, blockbase,
+                                    offsets, sorted_token, sorted_pair, pair_row, shared_T, err, so)
+                       : launch_pdl(use_pdl(D.T), perm_scatter_kernel<kPermRoundsLarge, true>, dim3(nb),
+                                    dim3(kPermWarps * 32), smem, s, topk_idx, D.pairs, D.k, D.E, D.cap, blockbase,
+                                    offsets, sorted_token, sorted_pair, pair_row, shared_T, err, so);
+        } else {
+            const ScanOut none{};
+            le = small ? launch_pdl(use_pdl(D.T), perm_scatter_kernel<kPermRoundsSmall, false>, dim3(nb),
+                                    dim3(kPermWarps * 32), 0, s, topk_idx, D.pairs, D.k, D.E, D.cap, blockbase,
+                                    offsets, sorted_token, sorted_pair, pair_row, shared_T, err, none)
+                       : launch_pdl(use_pdl(D.T), perm_scatter_kernel<kPermRoundsLarge, false>, dim3(nb),
+                                    dim3(kPermWarps * 32), 0, s, topk_idx, D.pairs, D.k, D.E, D.cap, blockbase,
+                                    offsets, sorted_token, sorted_pair, pair_row, shared_T, err, none);
+        }
         if (le != cudaSuccess) return le;
     }
     return cudaGetLastError();

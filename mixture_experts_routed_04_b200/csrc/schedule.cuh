@@ -5,8 +5,8 @@
 
 namespace moe {
 
-// One block of 512 threads; thread e owns expert e (Etot <= 257) and passes its
-// kept row count (0 for e >= Etot). Writes:
+// One block of at least Etot threads (at most 512); thread e owns expert e and
+// passes its kept row count (0 for e >= Etot). Writes:
 //   tile_base[0 .. Etot]           exclusive prefix of 128-row tiles per expert
 //   tile_base[Etot+1 .. 2*Etot+1]  that of 256-row tiles (Q4G32 and SM-pair units)
 //   stream_list[0 .. n)            experts taken by the streaming kernels
@@ -39,7 +39,8 @@ MOE_DEV void schedule_block(int kept, int Etot, int variant, int stream_max, int
     }
     __syncthreads();
     int bt = 0, bs = 0, b2 = 0, tt = 0, ts = 0, t2 = 0;
-    for (int i = 0; i < 16; ++i) {
+    const int nw = int(blockDim.x >> 5);
+    for (int i = 0; i < nw; ++i) {
         if (i < w) {
             bt += sums[0][i];
             bs += sums[1][i];

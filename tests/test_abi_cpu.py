@@ -187,3 +187,18 @@ def test_streaming_reduce_folds_into_down_when_h_fits(lib):
     # schedule + gather + streaming gate/up + down, (+ reduce)
     assert launches(2112) == 4
     assert launches(2176) == 5
+
+
+def test_forward_permutation_forms_its_scan_in_the_scatter(lib):
+    """Above the front kernel's batch size, moe_forward's scatter blocks form the permutation's
+    scan themselves (no scan launch) while the per-block counts fit their shared memory and one
+    thread per expert fits a block; moe_permute keeps its three launches."""
+    def fwd(T, E=128, k=8):
+        return b.launch_count(b.params(T=T, d_model=2048, d_ff=768, E=E, k=k), b.WS_FORWARD)
+    # routing, count, scatter (with the scan and the schedule), gather, gate/up, down, combine
+    assert fwd(4096) == 7
+    assert fwd(32768) == 7  # 128 blocks of 2048 pairs x 128 experts: 64 KB of counts
+    assert fwd(1024, E=256, k=8) == 7  # 256 experts, no shared one: a thread each
+    p = b.params(T=4096, d_model=2048, d_ff=768, E=256, k=8, has_shared=1, d_ff_shared=768)
+    assert b.launch_count(p, b.WS_FORWARD) == 8  # 257 experts: the scan kernel runs
+    assert b.launch_count(b.params(T=4096, d_model=2048, d_ff=768, E=128, k=8), b.WS_PERMUTE) == 3
