@@ -404,7 +404,8 @@ MOE_API int moe_wait_selftest(void* err_ws, uint64_t limit_ns, moe_stream_t stre
 #define MOE_K_ROUTE          0  /* S1 top-k softmax router */
 #define MOE_K_PERM_COUNT     1  /* S2 per-block histograms */
 #define MOE_K_PERM_SCAN      2  /* S2 block bases, counts, kept, offsets */
-#define MOE_K_PERM_SCATTER   3  /* S3 ranks, drop, row lists */
+#define MOE_K_PERM_SCATTER   3  /* S3 ranks, drop, row lists (in moe_forward also the
+                                   scan's outputs and the schedule, when they fit) */
 #define MOE_K_SCHEDULE       4  /* per-expert variant choice and M-tile prefix */
 #define MOE_K_GATHER         5  /* S4 row gather for the tile kernels */
 #define MOE_K_TC_GATEUP      6  /* S5 tcgen05 gate/up GEMM + clamped SwiGLU */
