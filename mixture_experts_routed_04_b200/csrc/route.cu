@@ -27,7 +27,10 @@ __global__ void __launch_bounds__(256) route_topk_softmax_kernel(const float* __
     const int warps_per_block = blockDim.x >> 5;
     const int64_t t = int64_t(blockIdx.x) * warps_per_block + (threadIdx.x >> 5);
     if (t >= T) return;
-    route_one_token(logits + t * E, E, k, topk_idx + t * k, topk_w + t * k);
+    if (E <= 128)  // four keys a lane: half the selection work of the 256-expert form
+        route_one_token<4>(logits + t * E, E, k, topk_idx + t * k, topk_w + t * k);
+    else
+        route_one_token(logits + t * E, E, k, topk_idx + t * k, topk_w + t * k);
 }
 
 

@@ -31,18 +31,21 @@ MOE_DEV float route_unkey(uint32_t k) {
 // lower expert index); one warp max-reduction of the keys gives the winning
 // value and one min-reduction over the lanes holding it gives the lowest
 // expert index among equal values.
+// NK: keys a lane holds (E <= 32 NK); the routing kernel takes NK = 4 for E <= 128.
+template <int NK = kRouteMaxPerLane>
 MOE_DEV int route_one_token(const float* __restrict__ row, int E, int k, int32_t* __restrict__ idx_out,
                             float* __restrict__ w_out, uint32_t* kth_key = nullptr) {
+    static_assert(NK >= 1 && NK <= kRouteMaxPerLane, "keys per lane");
     const int lane = threadIdx.x & 31;
-    uint32_t key[kRouteMaxPerLane];
+    uint32_t key[NK];
 #pragma unroll
-    for (int i = 0; i < kRouteMaxPerLane; ++i) {
+    for (int i = 0; i < NK; ++i) {
         const int e = lane + 32 * i;
         key[i] = (e < E) ? route_key(__ldg(row + e)) : 0u;  // 0: below every real key (also -inf's)
     }
     uint32_t taken = 0;  // bit i: key[i] already selected (or padding)
 #pragma unroll
-    for (int i = 0; i < kRouteMaxPerLane; ++i)
+    for (int i = 0; i < NK; ++i)
         if (lane + 32 * i >= E) taken |= 1u << i;
     float sel_v = 0.f;
     int sel_i = 0;
@@ -52,7 +55,7 @@ MOE_DEV int route_one_token(const float* __restrict__ row, int E, int k, int32_t
         uint32_t bk = 0;
         int bi = 0x7FFFFFFF;
 #pragma unroll
-        for (int i = 0; i < kRouteMaxPerLane; ++i)
+        for (int i = 0; i < NK; ++i)
             if (!(taken >> i & 1u) && (key[i] > bk || bi == 0x7FFFFFFF)) {  // first untaken, then strictly larger
                 bk = key[i];
                 bi = lane + 32 * i;
