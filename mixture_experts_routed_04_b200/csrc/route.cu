@@ -5,7 +5,8 @@
 // softmax over the k selected logits; that is what is computed, in fp32.
 //
 // One warp per token (route_one_token in route.cuh). Each lane keeps up to 8 of
-// the E <= 256 logits as order-preserving integer keys (expert lane + 32*i).
+// the E <= 256 logits (4 in this kernel when E <= 128) as order-preserving integer
+// keys (expert lane + 32*i).
 // k rounds pick the experts in descending order: every lane offers its best
 // untaken key, one warp max-reduction gives the winning value and one
 // min-reduction over the lanes holding it the lowest expert index, so equal
