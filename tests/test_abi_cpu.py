@@ -202,3 +202,5 @@ def test_forward_permutation_forms_its_scan_in_the_scatter(lib):
     p = b.params(T=4096, d_model=2048, d_ff=768, E=256, k=8, has_shared=1, d_ff_shared=768)
     assert b.launch_count(p, b.WS_FORWARD) == 8  # 257 experts: the scan kernel runs
     assert b.launch_count(b.params(T=4096, d_model=2048, d_ff=768, E=128, k=8), b.WS_PERMUTE) == 3
+    # 128 blocks of 2048 pairs x 256 experts: 128 KB of counts, above the 96 KB the blocks copy
+    assert fwd(32768, E=256, k=8) == 8
