@@ -29,6 +29,9 @@ LAYERS = {
     "ragged": synth.LayerConfig("ragged", T=700, d=192, f=320, E=6, k=3),
     # d_ff too wide for the down kernel's h buffer: the separate K-split reduce
     "wide_ff": synth.LayerConfig("wide_ff", T=3, d=256, f=2176, E=4, k=2),
+    # 257 experts: the permutation's scan as its own launch
+    "scan_launch": synth.LayerConfig("scan_launch", T=96, d=128, f=128, E=256, k=2, has_shared=True,
+                                     f_shared=128),
     "q4_capped": synth.LayerConfig("q4_capped", T=300, d=128, f=192, E=8, k=2, capacity_factor=0.9,
                                    weight_format="q4g32"),
 }

@@ -49,6 +49,11 @@ SMALL = {
     # two tokens with a shared expert: every expert streams and the streaming down kernel
     # also does the combine (a 256-column block of d=320 is partial)
     "two_tokens": synth.LayerConfig("two_tokens", T=2, d=320, f=256, E=8, k=3, has_shared=True, f_shared=256),
+    # 257 experts with the shared one, above the front kernel's batch: the permutation's scan
+    # runs as its own launch (one thread per expert no longer fits a scatter block), and the
+    # automatic choice mixes streaming (experts of a few rows) with tiles (the shared expert)
+    "scan_launch": synth.LayerConfig("scan_launch", T=96, d=128, f=128, E=256, k=2, has_shared=True,
+                                     f_shared=128),
 }
 Q4_SMALL = {
     "q4_tiny": synth.CONFIGS["tiny"].replace(name="q4_tiny", weight_format="q4g32"),
